@@ -1,0 +1,292 @@
+"""Pins of the scalar CPU oracle to facts outside itself (no GPU needed).
+
+Each test ties one oracle function to something the pages or mathematics
+fix: hand-worked examples from the bitnet-cpu page's definitions (golden
+files), brute force over tiny inputs, closed forms, library special cases
+(torch / numpy evaluations of the same definition), and invariants.
+"""
+import itertools
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def f32_to_bf16_bits_np(f):
+    """Independent RNE narrowing in numpy (for building inputs only)."""
+    u = np.asarray(f, np.float32).view(np.uint32).astype(np.uint64)
+    lower = u & 0xFFFF
+    upper = u >> 16
+    up = (lower > 0x8000) | ((lower == 0x8000) & ((upper & 1) == 1))
+    return (upper + up.astype(np.uint64)).astype(np.uint16)
+
+
+def bf16_to_f32(bits):
+    return synth.bf16_bits_to_f32(np.asarray(bits, np.uint16))
+
+
+# --------------------------------------------------------------------- pack
+
+def _pack_golden():
+    rows = []
+    with open(os.path.join(GOLDEN, "pack_examples.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if not line:
+                continue
+            *w, b = line.split()
+            rows.append(([int(v) for v in w], int(b, 16)))
+    return rows
+
+
+def test_pack_golden_examples():
+    rows = _pack_golden()
+    assert len(rows) >= 5
+    for w, byte in rows:
+        got = oracle.pack(np.array([w], np.int8))
+        assert got.shape == (1, 1)
+        assert int(got[0, 0]) == byte, (w, hex(int(got[0, 0])), hex(byte))
+
+
+def test_pack_brute_force_all_81_tuples():
+    tuples = list(itertools.product((-1, 0, 1), repeat=4))
+    w = np.array(tuples, np.int8)              # [81, 4] -> one byte per row
+    packed = oracle.pack(w)[:, 0]
+    assert len(set(packed.tolist())) == 81     # injective
+    for t, b in zip(tuples, packed.tolist()):
+        fields = [(b >> (2 * i)) & 3 for i in range(4)]
+        assert all(f in (1, 2, 3) for f in fields)
+        assert [f - 2 for f in fields] == list(t)  # element i in bits 2i..2i+1
+
+
+def test_pack_row_layout_and_roundtrip():
+    k = synth.key(99, 0, synth.T_WEIGHT)
+    w = synth.ternary(k, 37, 96)
+    p = oracle.pack(w)
+    assert p.shape == (37, 24) and p.dtype == np.uint8
+    # byte j of row n covers elements 4j..4j+3 of that row only
+    for n in (0, 5, 36):
+        for j in (0, 7, 23):
+            assert int(p[n, j]) == int(oracle.pack(w[n:n + 1, 4 * j:4 * j + 4])[0, 0])
+    assert np.array_equal(oracle.unpack(p, 96), w)
+
+
+def test_pack_of_unpack_is_identity_on_valid_bytes():
+    rng = np.random.default_rng(3)
+    fields = rng.integers(1, 4, size=(16, 32, 4))
+    bytes_ = (fields[..., 0] | fields[..., 1] << 2 | fields[..., 2] << 4
+              | fields[..., 3] << 6).astype(np.uint8)
+    assert np.array_equal(oracle.pack(oracle.unpack(bytes_, 128)), bytes_)
+
+
+def test_pack_rejects_out_of_range_and_bad_k():
+    with pytest.raises(oracle.OracleError):
+        oracle.pack(np.array([[0, 2, 0, 0]], np.int8))
+    with pytest.raises(oracle.OracleError):
+        oracle.pack(np.array([[0, -2, 0, 0]], np.int8))
+    with pytest.raises(oracle.OracleError):
+        oracle.pack(np.zeros((2, 6), np.int8))
+
+
+def test_unpack_code_zero_decodes_to_minus_two():
+    # 0b00 is never produced by pack; decode is code - 2 for every code.
+    assert oracle.unpack(np.array([[0x00]], np.uint8), 4).tolist() == [[-2] * 4]
+    assert oracle.unpack(np.array([[0xE4]], np.uint8), 4).tolist() == [[-2, -1, 0, 1]]
+
+
+# ----------------------------------------------------------------- quantize
+
+def _quant_golden():
+    rows = []
+    with open(os.path.join(GOLDEN, "quantize_examples.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if not line:
+                continue
+            xs, qs, ss = [p.split(":", 1)[1].strip() for p in line.split("|")]
+            rows.append(([float(v) for v in xs.split()],
+                         [int(v) for v in qs.split()], int(ss, 16)))
+    return rows
+
+
+def test_quantize_golden_examples():
+    rows = _quant_golden()
+    assert len(rows) >= 5
+    for xs, qs, sbits in rows:
+        bits = f32_to_bf16_bits_np(np.array([xs], np.float32))
+        q, s = oracle.quantize(bits)
+        assert q[0].tolist() == qs, (xs, q[0].tolist(), qs)
+        assert int(s[0]) == sbits, (xs, hex(int(s[0])), hex(sbits))
+
+
+def test_quantize_invariants_random_rows():
+    k = synth.key(98, 0, synth.T_ACT)
+    x = synth.act_bf16(k, 64, 1000)
+    q, s = oracle.quantize(x)
+    xf = bf16_to_f32(x).astype(np.float64)
+    absmax = np.maximum(np.abs(xf).max(axis=1), 1e-5)
+    s32 = (np.float32(1) * absmax.astype(np.float32)) / np.float32(127)
+    assert np.all(np.abs(q.astype(np.int32)) <= 127)
+    assert np.all(np.abs(q).max(axis=1) == 127)           # the absmax maps to 127
+    err = np.abs(xf / s32.astype(np.float64)[:, None] - q)
+    assert err.max() <= 0.5 + 1e-5                          # round to nearest
+    # stored scale is the bf16 rounding of absmax / 127 (within half a bf16 ulp)
+    sf = bf16_to_f32(s).astype(np.float64)
+    rel = np.abs(sf - absmax / 127.0) / (absmax / 127.0)
+    assert rel.max() <= 2.0 ** -8 + 1e-7
+
+
+def test_quantize_matches_torch_fp32_evaluation():
+    """Library special case: the page's torch expression evaluated in fp32."""
+    torch = pytest.importorskip("torch")
+    k = synth.key(97, 0, synth.T_ACT)
+    x = synth.act_bf16(k, 257, 2048)
+    # add exact ties: entries equal to (j + 0.5) * scale for a power-of-two scale
+    x[0, :8] = f32_to_bf16_bits_np(np.array([127, 0.5, 1.5, 2.5, -0.5, -1.5, 3.5, -2.5], np.float32))
+    q, s = oracle.quantize(x)
+    xt = torch.from_numpy(x.view(np.int16).copy()).view(torch.bfloat16).float()
+    absmax = xt.abs().amax(dim=-1, keepdim=True).clamp(min=1e-5)
+    scale = absmax / 127.0
+    qt = (xt / scale).round().clamp(-127, 127).to(torch.int8)
+    st = scale.squeeze(-1).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(qt.numpy(), q)
+    assert np.array_equal(st, s)
+
+
+def test_f32_to_bf16_matches_torch_rounding():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(5)
+    u = rng.integers(0, 2 ** 32, size=20000, dtype=np.uint64).astype(np.uint32)
+    u[:4000] = (u[:4000] & 0xFFFF0000) | 0x8000      # exact ties
+    f = u.view(np.float32)
+    f = f[np.isfinite(f)]
+    ours = np.array([oracle.f32_to_bf16(float(v)) for v in f[:6000]], np.uint16)
+    ref = torch.from_numpy(f[:6000].copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+# ---------------------------------------------------------------------- acc
+
+def _brute_acc(q, w):
+    M, K = q.shape
+    N = w.shape[0]
+    out = np.zeros((M, N), np.int64)
+    for m in range(M):
+        for n in range(N):
+            s = 0
+            for k in range(K):
+                s += int(q[m, k]) * int(w[n, k])
+            out[m, n] = s
+    return out
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 4), (3, 5, 8), (7, 2, 64), (8, 8, 32)])
+def test_acc_brute_force_tiny(M, N, K):
+    rng = np.random.default_rng(M * 100 + N * 10 + K)
+    q = rng.integers(-127, 128, size=(M, K)).astype(np.int8)
+    w = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    got = oracle.acc(q, oracle.pack(w))
+    assert np.array_equal(got, _brute_acc(q, w))
+
+
+def test_acc_exhaustive_k4():
+    # every ternary 4-vector against a fixed set of activation rows
+    w = np.array(list(itertools.product((-1, 0, 1), repeat=4)), np.int8)
+    q = np.array([[1, 2, 3, 4], [-127, 127, -127, 127], [5, -7, 0, 9]], np.int8)
+    assert np.array_equal(oracle.acc(q, oracle.pack(w)), _brute_acc(q, w))
+
+
+def test_acc_matches_float64_matmul():
+    """Library special case: integer-valued float64 matmul is exact here."""
+    k = synth.key(96, 0, synth.T_WEIGHT)
+    w = synth.ternary(k, 96, 512)
+    rng = np.random.default_rng(9)
+    q = rng.integers(-127, 128, size=(13, 512)).astype(np.int8)
+    ref = q.astype(np.float64) @ w.astype(np.float64).T
+    assert np.array_equal(oracle.acc(q, oracle.pack(w)), ref.astype(np.int64))
+
+
+def test_acc_special_cases():
+    rng = np.random.default_rng(11)
+    K = 64
+    q = rng.integers(-127, 128, size=(5, K)).astype(np.int8)
+    zero = np.zeros((K, K), np.int8)
+    eye = np.eye(K, dtype=np.int8)
+    ones = np.ones((3, K), np.int8)
+    assert np.all(oracle.acc(q, oracle.pack(zero)) == 0)
+    assert np.array_equal(oracle.acc(q, oracle.pack(eye)), q.astype(np.int32))
+    assert np.array_equal(oracle.acc(q, oracle.pack(-eye)), -q.astype(np.int32))
+    rs = q.astype(np.int32).sum(axis=1)
+    assert np.array_equal(oracle.acc(q, oracle.pack(ones)), np.repeat(rs[:, None], 3, 1))
+
+
+def test_acc_extreme_magnitude():
+    K = 11008
+    q = np.full((1, K), -127, np.int8)
+    w = np.full((2, K), 1, np.int8)
+    w[1] = -1
+    got = oracle.acc(q, oracle.pack(w))
+    assert got.tolist() == [[-127 * K, 127 * K]]
+
+
+# ----------------------------------------------------------------- epilogue
+
+def test_epilogue_power_of_two_scales_closed_form():
+    # acc * 2^a * 2^b is exact in fp32, so out = bf16_rne(acc * 2^(a+b)).
+    rng = np.random.default_rng(12)
+    acc = rng.integers(-2 ** 20, 2 ** 20, size=(4, 64)).astype(np.int32)
+    sa = f32_to_bf16_bits_np(np.array([2.0 ** -7, 2.0 ** -3, 1.0, 2.0 ** 4], np.float32))
+    sw = np.array([2.0 ** -5], np.float32)
+    out = oracle.epilogue(acc, sa, sw)
+    exact = acc.astype(np.float64) * np.array([2.0 ** -12, 2.0 ** -8, 2.0 ** -5, 2.0 ** -1])[:, None]
+    assert np.array_equal(out, f32_to_bf16_bits_np(exact.astype(np.float32)))
+
+
+def test_epilogue_within_one_ulp_of_exact_product():
+    rng = np.random.default_rng(13)
+    acc = rng.integers(-200000, 200000, size=(16, 256)).astype(np.int32)
+    sa = f32_to_bf16_bits_np(rng.uniform(0.001, 0.2, 16).astype(np.float32))
+    sw = rng.uniform(0.01, 0.1, 256).astype(np.float32)
+    out = oracle.epilogue(acc, sa, sw)
+    exact = acc.astype(np.float64) * bf16_to_f32(sa).astype(np.float64)[:, None] * sw.astype(np.float64)[None, :]
+    got = bf16_to_f32(out).astype(np.float64)
+    ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(exact), 1e-30))) - 7)
+    assert np.all(np.abs(got - exact) <= ulp + 1e-30)
+    # per-column scale is honoured (len N) and a scalar is broadcast (len 1)
+    out1 = oracle.epilogue(acc, sa, sw[:1])
+    outN = oracle.epilogue(acc, sa, np.full(256, sw[0], np.float32))
+    assert np.array_equal(out1, outN)
+
+
+# --------------------------------------------------------------- composition
+
+def test_linear_is_quantize_then_gemm():
+    kw = synth.key(95, 0, synth.T_WEIGHT)
+    kx = synth.key(95, 0, synth.T_ACT)
+    w = synth.ternary(kw, 200, 256)
+    x = synth.act_bf16(kx, 9, 256)
+    sw = synth.scale_wt(synth.key(95, 0, synth.T_SCALE_WT))
+    p = oracle.pack(w)
+    q, sa = oracle.quantize(x)
+    assert np.array_equal(oracle.linear(x, p, sw), oracle.gemm(q, p, sa, sw))
+    assert np.array_equal(oracle.linear(x, p, sw, threads=4), oracle.linear(x, p, sw))
+    assert np.array_equal(oracle.gemm_threads(q, p, sa, sw, 3), oracle.gemm(q, p, sa, sw))
+
+
+def test_linear_close_to_float64_dequantised_product():
+    """The whole layer tracks the real-valued product of its quantised parts."""
+    kw = synth.key(94, 0, synth.T_WEIGHT)
+    kx = synth.key(94, 0, synth.T_ACT)
+    w = synth.ternary(kw, 64, 512)
+    x = synth.act_bf16(kx, 4, 512)
+    sw = np.array([0.05], np.float32)
+    p = oracle.pack(w)
+    q, sa = oracle.quantize(x)
+    y = bf16_to_f32(oracle.linear(x, p, sw)).astype(np.float64)
+    ref = (q.astype(np.float64) @ w.astype(np.float64).T) * bf16_to_f32(sa)[:, None] * 0.05
+    assert np.allclose(y, ref, rtol=2 ** -7, atol=1e-6)
