@@ -1,0 +1,470 @@
+#!/usr/bin/env python
+"""Benchmark of the BitNet b1.58 W1.58A8 linear layer on B200.
+
+Default workload (one "step"): the BitNet-b1.58-2B decode sweep at M = 1 --
+30 layers x 7 BitLinears (Q, K, V, O, gate, up, down) plus the LM head, 211
+calls of the fused quantise + GEMV with fresh seeded weights per layer and a
+fresh activation row per call. The step is issued as the 211 C-ABI calls in
+order on one stream and replayed as a CUDA graph (programmatic dependent
+launch edges between the kernels). Metric: GB/s of algorithmic bytes
+(packed weights + bf16 activations + bf16 outputs + weight scales).
+
+Also reported: the prefill GEMM (M = 8192, K = 4096 -> N = 11008) in INT8
+TOPS against the dense INT8 tensor peak, and the LM-head GEMV alone.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (launched with torch.distributed.run): every rank runs its own
+decode sweep (independent decode streams over replicated weights, no
+collective on the data path); value = all ranks' bytes / max-over-ranks time.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+from synth import workloads as W  # noqa: E402
+
+METRIC = "W1.58A8 linear: GB/s at M=1 decode, INT8 TOPS at M≥2048, vs B200 roofline"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ env
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in getattr(self, "lines", []):
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_gemm_bitnet_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if
+    the kernel sources are unchanged since it was taken; else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("source_hash") != source_hash():
+        return None
+    k = rec.get("kernels", {}).get(kernel)
+    return None if k is None else k.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------- decode sweep
+
+def sweep_calls():
+    names = [n for n, _, _ in W.DECODE_2B_LAYER]
+    out = []
+    for layer, name, K, N in W.decode_2b_sweep():
+        variant = names.index(name) if name in names else len(names)
+        out.append((layer, variant, K, N))
+    return out
+
+
+def call_bytes(M, K, N, sw_len=1):
+    return N * K // 4 + 2 * M * K + 2 * M * N + 4 * sw_len
+
+
+def build_decode(bn, dev, rank):
+    calls = sweep_calls()
+    packed, scales = [], []
+    for layer, variant, K, N in calls:
+        w = synth.ternary(synth.key(W.W_DECODE_2B, layer, synth.T_WEIGHT, variant), N, K)
+        wd = torch.from_numpy(w).to(dev)
+        packed.append(bn.bitnet_pack_weights(wd))
+        del wd
+        sw = synth.scale_wt(synth.key(W.W_DECODE_2B, layer, synth.T_SCALE_WT, variant))
+        scales.append(torch.from_numpy(sw).to(dev))
+    xs_total = sum(K for _, _, K, _ in calls)
+    outs_total = sum(N for _, _, _, N in calls)
+    x_host = torch.empty((xs_total,), dtype=torch.bfloat16).pin_memory()
+    xv = x_host.view(torch.int16).numpy().view(np.uint16)
+    off = 0
+    for layer, variant, K, N in calls:
+        xv[off:off + K] = synth.act_bf16(
+            synth.key(W.W_DECODE_2B, layer, synth.T_ACT, variant + 16 * rank), 1, K)[0]
+        off += K
+    x_dev = x_host.to(dev)
+    out_dev = torch.empty((outs_total,), dtype=torch.bfloat16, device=dev)
+    out_host = torch.empty((outs_total,), dtype=torch.bfloat16).pin_memory()
+    xs, outs = [], []
+    xo = oo = 0
+    for _, _, K, N in calls:
+        xs.append(x_dev[xo:xo + K].view(1, K))
+        outs.append(out_dev[oo:oo + N].view(1, N))
+        xo += K
+        oo += N
+    nbytes = sum(call_bytes(1, K, N) for _, _, K, N in calls)
+    return dict(calls=calls, packed=packed, scales=scales, xs=xs, outs=outs, x_host=x_host,
+                x_dev=x_dev, out_dev=out_dev, out_host=out_host, bytes=nbytes)
+
+
+def make_sweep(bn, d):
+    """The step as raw C-ABI calls (pointers prepared once)."""
+    import ctypes
+    L = bn.lib()
+    args = []
+    for (layer, variant, K, N), p, s, x, o in zip(d["calls"], d["packed"], d["scales"],
+                                                  d["xs"], d["outs"]):
+        args.append((ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(x.data_ptr()),
+                     ctypes.c_void_p(p.data_ptr()), ctypes.c_void_p(s.data_ptr()), K, N))
+
+    def sweep():
+        st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        for o, x, p, s, K, N in args:
+            r = L.bitnet_gemv_fused(o, x, 0, p, s, 1, 1, N, K, st)
+            if r != 0:
+                raise RuntimeError(f"bitnet_gemv_fused: {bn.status_string(r)}")
+    return sweep
+
+
+def time_graph(g, steps, warmup, barrier):
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record()
+    for i in range(steps):
+        g.replay()
+        ev[i + 1].record()
+    torch.cuda.synchronize()
+    barrier()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    return ev[0].elapsed_time(ev[-1]), per
+
+
+def time_e2e(g, d, steps, warmup, barrier):
+    def step():
+        d["x_dev"].copy_(d["x_host"], non_blocking=True)
+        g.replay()
+        d["out_host"].copy_(d["out_dev"], non_blocking=True)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    return e0.elapsed_time(e1)
+
+
+def lm_head_alone(bn, d, dev, reps=20):
+    """The LM-head GEMV (82 MB of packed weights) timed alone, L2 flushed."""
+    i = len(d["calls"]) - 1
+    _, _, K, N = d["calls"][i]
+    flush = torch.empty((2 * L2_BYTES,), dtype=torch.uint8, device=dev)
+    times = []
+    for r in range(reps + 3):
+        flush.fill_(r & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        bn.bitnet_gemv_fused(d["xs"][i], d["packed"][i], d["scales"][i], out=d["outs"][i])
+        e1.record()
+        torch.cuda.synchronize()
+        if r >= 3:
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    return {"K": K, "N": N, "ms": ms, "gbs": call_bytes(1, K, N) / ms / 1e6}
+
+
+# ---------------------------------------------------------------- prefill
+
+def prefill(bn, dev, pk, reps=10):
+    M, K, N = 8192, 4096, 11008
+    x = synth.act_bf16(synth.key(W.W_PREFILL, 0, synth.T_ACT, 0), M, K)
+    w = synth.ternary(synth.key(W.W_PREFILL, 0, synth.T_WEIGHT, 0), N, K)
+    sw = synth.scale_wt(synth.key(W.W_PREFILL, 0, synth.T_SCALE_WT, 0))
+    xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+    wp = bn.bitnet_pack_weights(torch.from_numpy(w).to(dev))
+    swd = torch.from_numpy(sw).to(dev)
+    xq, sa = bn.bitnet_quantize_act(xd)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty((bn.bitnet_linear_workspace_bytes(M, K),), dtype=torch.uint8, device=dev)
+    flush = torch.empty((2 * L2_BYTES,), dtype=torch.uint8, device=dev)
+    tg, tl = [], []
+    for r in range(reps + 3):
+        flush.fill_(r & 0xFF)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record()
+        bn.bitnet_gemm(xq, wp, sa, swd, out=out)
+        e[1].record()
+        torch.cuda.synchronize()
+        flush.fill_((r + 1) & 0xFF)
+        f = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        f[0].record()
+        bn.bitnet_linear(xd, wp, swd, out=out, workspace=ws)
+        f[1].record()
+        torch.cuda.synchronize()
+        if r >= 3:
+            tg.append(e[0].elapsed_time(e[1]))
+            tl.append(f[0].elapsed_time(f[1]))
+    bn.bitnet_device_status()
+    ops = 2.0 * M * N * K
+    g_ms, l_ms = statistics.median(tg), statistics.median(tl)
+    tops = ops / g_ms / 1e9
+    peak = pk["bf16_tflops"] * INT8_OVER_BF16
+    return {"M": M, "K": K, "N": N, "gemm_ms": g_ms, "gemm_tops": tops,
+            "linear_ms": l_ms, "linear_tops": ops / l_ms / 1e9,
+            "roofline": {"bound": "tensor", "achieved": tops, "peak": peak, "unit": "TOPS",
+                         "frac": tops / peak,
+                         "peak_source": f"{pk['source']} bf16 burst x {INT8_OVER_BF16:g} (int8/bf16 nominal)",
+                         "traffic": recorded_traffic("gemm_i8_tcgen05_kernel")}}
+
+
+# ----------------------------------------------------------- CPU oracle
+
+def cpu_baseline(seconds):
+    """The scalar oracle on the host cores: layer 0's seven decode calls,
+    repeated for about `seconds` s, in GB/s of the same algorithmic bytes."""
+    import oracle
+    threads = os.cpu_count() or 1
+    calls = [c for c in sweep_calls() if c[0] == 0]
+    prepared = []
+    for layer, variant, K, N in calls:
+        w = synth.ternary(synth.key(W.W_DECODE_2B, layer, synth.T_WEIGHT, variant), N, K)
+        p = oracle.pack(w)
+        sw = synth.scale_wt(synth.key(W.W_DECODE_2B, layer, synth.T_SCALE_WT, variant))
+        x = synth.act_bf16(synth.key(W.W_DECODE_2B, layer, synth.T_ACT, variant), 1, K)
+        prepared.append((x, p, sw, call_bytes(1, K, N)))
+    t0 = time.perf_counter()
+    nbytes = 0
+    reps = 0
+    while True:
+        for x, p, sw, b in prepared:
+            oracle.linear_cols_threads(x, p, sw, threads)
+            nbytes += b
+        reps += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"decode layer 0 (7 BitLinears, {nbytes // reps / 1e6:.1f} MB packed) x {reps}, "
+                      f"M=1, columns split over {threads} threads, {dt:.1f} s"}
+
+
+# ----------------------------------------------------------------- main
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if world != args.gpus and args.gpus > 1:
+        pass
+    config = {"workload": "bitnet-b1.58-2B decode sweep, M=1: 30 layers x 7 BitLinears "
+                          "(2560->2560, 2560->640 x2, 2560->2560, 2560->6912 x2, 6912->2560) "
+                          "+ LM head 2560->128256",
+              "calls_per_step": len(W.decode_2b_sweep()),
+              "packed_weight_bytes_per_step": W.decode_2b_packed_bytes(),
+              "l2": "inputs larger than L2 (603 MB of packed weights streamed per step)",
+              "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        cb = cpu_baseline(max(1.0, args.cpu_seconds / 2))
+        per_step_s = W.decode_2b_packed_bytes() / (cb["value"] * 1e9)
+        line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT,
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": per_step_s * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+                "data": "synthetic (seeded, shaped like the pages' workloads)",
+                "config": config, "cpu_baseline": cb,
+                "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    import bit_gemm_bitnet_b200 as bn
+    bn.lib()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    pk = peaks()
+    d = build_decode(bn, dev, rank)
+    sweep = make_sweep(bn, d)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        sweep()
+        torch.cuda.synchronize()
+        bn.bitnet_device_status()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            sweep()
+        torch.cuda.synchronize()
+        with ClockSampler(local) as clk:
+            total_ms, per = time_graph(g, args.steps, args.warmup, barrier)
+        e2e_ms = time_e2e(g, d, args.steps, args.warmup, barrier)
+    bn.bitnet_device_status()
+
+    if pg is not None:
+        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+
+    ms_step = total_ms / args.steps
+    value = d["bytes"] * world * args.steps / (total_ms / 1e3) / 1e9
+    e2e_val = d["bytes"] * world * args.steps / (e2e_ms / 1e3) / 1e9
+    per_rank_gbs = d["bytes"] / (ms_step / 1e3) / 1e9
+    clocks = clk.summary()
+    lm = lm_head_alone(bn, d, dev)
+    pre = None if args.no_prefill else prefill(bn, dev, pk)
+
+    if rank != 0:
+        if pg is not None:
+            pg.destroy_process_group()
+        return 0
+    cb = None if args.no_cpu_baseline or world > 1 else cpu_baseline(args.cpu_seconds)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8", "data": "synthetic (seeded; shapes and distributions of the pages' workloads)",
+        "config": config,
+        "roofline": {"bound": "hbm", "achieved": per_rank_gbs, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": per_rank_gbs / pk["hbm_gbs"],
+                     "peak_source": f"{pk['source']} hbm_gbs",
+                     "kernel": "gemv_kernel (all 211 launches of the step)",
+                     "traffic": recorded_traffic("gemv_kernel")},
+        "cpu_baseline": cb,
+        "e2e": {"value": e2e_val, "unit": UNIT,
+                "h2d_bytes_per_step": int(d["x_host"].numel() * 2),
+                "d2h_bytes_per_step": int(d["out_host"].numel() * 2)},
+        "gpu_launches": len(d["calls"]) * args.steps,
+        "clocks": clocks,
+        "step_ms_min_median": [min(per), statistics.median(per)],
+        "lm_head_alone": {**lm, "frac": lm["gbs"] / pk["hbm_gbs"]},
+        "prefill_gemm": pre,
+    }
+    print(json.dumps(line))
+    if pg is not None:
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

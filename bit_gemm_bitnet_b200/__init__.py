@@ -1,0 +1,253 @@
+"""BitNet b1.58 W1.58A8 linear layer on B200: Python binding of libbitnet_b200.
+
+A thin ctypes layer over the C ABI declared in ``include/bitnet.h``. It only
+marshals arguments: it checks tensor dtypes, devices and contiguity, allocates
+outputs with torch, passes raw device pointers and the current CUDA stream,
+and turns status codes into exceptions. Every step of the computation runs in
+the library's CUDA kernels; there is no fallback of any kind. If the library
+is missing, every call raises.
+
+Function names follow the C entry points (and the bitnet-cpu page's API:
+pack_weights, quantize_activation, bitnet_gemm, bitnet_gemv_fused,
+bitnet_linear).
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbitnet_b200.so")
+
+OK, ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_VALUE, ERR_WORKSPACE, \
+    ERR_CUDA, ERR_TIMEOUT = range(9)
+BF16 = 0
+
+# every symbol include/bitnet.h declares
+EXPORTS = (
+    "bitnet_pack_weights", "bitnet_quantize_act", "bitnet_gemm",
+    "bitnet_gemv_fused", "bitnet_linear_workspace_bytes", "bitnet_linear",
+    "bitnet_device_status", "bitnet_status_string", "bitnet_gemm_acc_i32",
+    "bitnet_gemv_fused_debug",
+)
+
+_lib = None
+
+
+class BitnetError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+class BitnetValueError(BitnetError, ValueError):
+    pass
+
+
+def lib():
+    """Load libbitnet_b200.so (built in-tree); raise if it is absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"libbitnet_b200.so not found at {LIB_PATH}; build it with "
+                "`python -m bit_gemm_bitnet_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, SZ, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+        sig = {
+            "bitnet_pack_weights": [P, P, I64, I64, P],
+            "bitnet_quantize_act": [P, P, P, I, I64, I64, P],
+            "bitnet_gemm": [P, P, P, P, P, I64, I64, I64, I64, P],
+            "bitnet_gemv_fused": [P, P, I, P, P, I64, I64, I64, I64, P],
+            "bitnet_linear": [P, P, I, P, P, I64, I64, I64, I64, P, SZ, P],
+            "bitnet_device_status": [P],
+            "bitnet_gemm_acc_i32": [P, P, P, I64, I64, I64, P],
+            "bitnet_gemv_fused_debug": [P, P, P, P, I, P, I64, I64, I64, P],
+        }
+        for name, args in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_int
+        L.bitnet_linear_workspace_bytes.argtypes = [I64, I64]
+        L.bitnet_linear_workspace_bytes.restype = SZ
+        L.bitnet_status_string.argtypes = [ctypes.c_int]
+        L.bitnet_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_string(status):
+    return lib().bitnet_status_string(int(status)).decode()
+
+
+def _check(status, what):
+    if status == OK:
+        return
+    if status in (ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_VALUE, ERR_WORKSPACE):
+        raise BitnetValueError(status, what)
+    raise BitnetError(status, what)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t, dtype, name, ndim=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must be {ndim}-D, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _scale_wt(scale_wt, N, device):
+    """fp32 weight scale of length 1 or N (bf16 [N] is widened exactly)."""
+    if not isinstance(scale_wt, torch.Tensor):
+        scale_wt = torch.tensor([float(scale_wt)], dtype=torch.float32, device=device)
+    if scale_wt.dtype == torch.bfloat16:
+        scale_wt = scale_wt.float()
+    sw = scale_wt.reshape(-1).contiguous()
+    _need(sw, torch.float32, "scale_wt")
+    if sw.numel() not in (1, N):
+        raise ValueError(f"scale_wt must have 1 or N={N} elements, got {sw.numel()}")
+    return sw
+
+
+# ---------------------------------------------------------------- entries
+
+def bitnet_pack_weights(w, out=None):
+    """int8 [N, K] in {-1, 0, +1} -> uint8 [N, K/4] (synchronises)."""
+    _need(w, torch.int8, "w", 2)
+    N, K = w.shape
+    if out is None:
+        out = torch.empty((N, K // 4), dtype=torch.uint8, device=w.device)
+    _check(lib().bitnet_pack_weights(_ptr(out), _ptr(w), N, K, _stream(w.device)),
+           "bitnet_pack_weights")
+    return out
+
+
+def bitnet_quantize_act(x, x_q=None, scale_act=None):
+    """bf16 [..., K] -> (int8 [M, K], bf16 [M])."""
+    x2 = x.reshape(-1, x.shape[-1])
+    _need(x2, torch.bfloat16, "x", 2)
+    M, K = x2.shape
+    if x_q is None:
+        x_q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if scale_act is None:
+        scale_act = torch.empty((M,), dtype=torch.bfloat16, device=x.device)
+    _check(lib().bitnet_quantize_act(_ptr(x_q), _ptr(scale_act), _ptr(x2), BF16, M, K,
+                                     _stream(x.device)), "bitnet_quantize_act")
+    return x_q, scale_act
+
+
+def bitnet_gemm(x_q, w_packed, scale_act, scale_wt, out=None):
+    """int8 [M, K] x packed [N, K/4] -> bf16 [M, N]."""
+    _need(x_q, torch.int8, "x_q", 2)
+    _need(w_packed, torch.uint8, "w_packed", 2)
+    _need(scale_act, torch.bfloat16, "scale_act", 1)
+    M, K = x_q.shape
+    N = w_packed.shape[0]
+    if w_packed.shape[1] * 4 != K:
+        raise ValueError(f"w_packed {tuple(w_packed.shape)} does not match K={K}")
+    sw = _scale_wt(scale_wt, N, x_q.device)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x_q.device)
+    _check(lib().bitnet_gemm(_ptr(out), _ptr(x_q), _ptr(w_packed), _ptr(scale_act),
+                             _ptr(sw), sw.numel(), M, N, K, _stream(x_q.device)),
+           "bitnet_gemm")
+    return out
+
+
+def bitnet_gemv_fused(x, w_packed, scale_wt, out=None):
+    """bf16 [M, K] (M < 16) -> bf16 [M, N], quantisation fused."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(w_packed, torch.uint8, "w_packed", 2)
+    M, K = x.shape
+    N = w_packed.shape[0]
+    if w_packed.shape[1] * 4 != K:
+        raise ValueError(f"w_packed {tuple(w_packed.shape)} does not match K={K}")
+    sw = _scale_wt(scale_wt, N, x.device)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _check(lib().bitnet_gemv_fused(_ptr(out), _ptr(x), BF16, _ptr(w_packed), _ptr(sw),
+                                   sw.numel(), M, N, K, _stream(x.device)),
+           "bitnet_gemv_fused")
+    return out
+
+
+def bitnet_linear_workspace_bytes(M, K):
+    return int(lib().bitnet_linear_workspace_bytes(M, K))
+
+
+def bitnet_linear(x, w_packed, scale_wt, out=None, workspace=None):
+    """bf16 [..., K] -> bf16 [..., N]; dispatches by M like the page's
+    bitnet_linear (fused GEMV for M < 16, else quantise + GEMM)."""
+    orig = x.shape
+    K = orig[-1]
+    x2 = x.reshape(-1, K)
+    _need(x2, torch.bfloat16, "x", 2)
+    _need(w_packed, torch.uint8, "w_packed", 2)
+    M = x2.shape[0]
+    N = w_packed.shape[0]
+    if w_packed.shape[1] * 4 != K:
+        raise ValueError(f"w_packed {tuple(w_packed.shape)} does not match K={K}")
+    sw = _scale_wt(scale_wt, N, x.device)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    need = bitnet_linear_workspace_bytes(M, K)
+    if need and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
+    wsp = _ptr(workspace) if need else None
+    _check(lib().bitnet_linear(_ptr(out), _ptr(x2), BF16, _ptr(w_packed), _ptr(sw),
+                               sw.numel(), M, N, K, wsp, need, _stream(x.device)),
+           "bitnet_linear")
+    return out.view(*orig[:-1], N)
+
+
+def bitnet_device_status(device=None):
+    """Synchronise the current stream; raise if a kernel gave up a wait."""
+    dev = device if device is not None else torch.cuda.current_device()
+    _check(lib().bitnet_device_status(_stream(dev)), "bitnet_device_status")
+
+
+# ------------------------------------------------------------- test hooks
+
+def bitnet_gemm_acc_i32(x_q, w_packed, out=None):
+    _need(x_q, torch.int8, "x_q", 2)
+    _need(w_packed, torch.uint8, "w_packed", 2)
+    M, K = x_q.shape
+    N = w_packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.int32, device=x_q.device)
+    _check(lib().bitnet_gemm_acc_i32(_ptr(out), _ptr(x_q), _ptr(w_packed), M, N, K,
+                                     _stream(x_q.device)), "bitnet_gemm_acc_i32")
+    return out
+
+
+def bitnet_gemv_fused_debug(x, w_packed):
+    """-> (int32 acc [M, N], int8 codes [M, K], bf16 scales [M])."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(w_packed, torch.uint8, "w_packed", 2)
+    M, K = x.shape
+    N = w_packed.shape[0]
+    acc = torch.empty((M, N), dtype=torch.int32, device=x.device)
+    xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    sa = torch.empty((M,), dtype=torch.bfloat16, device=x.device)
+    _check(lib().bitnet_gemv_fused_debug(_ptr(acc), _ptr(xq), _ptr(sa), _ptr(x), BF16,
+                                         _ptr(w_packed), M, N, K, _stream(x.device)),
+           "bitnet_gemv_fused_debug")
+    return acc, xq, sa
+
+
+# the page's Python names
+pack_weights = bitnet_pack_weights
+quantize_activation = bitnet_quantize_act

@@ -1,0 +1,453 @@
+// libbitnet_b200: C ABI entry points (declared in include/bitnet.h).
+//
+// Host code only validates arguments, picks a kernel variant and launches it
+// on the caller's stream; all arithmetic runs in the kernels included below.
+#include <mutex>
+
+#include "../../include/bitnet.h"
+#include "common.cuh"
+#include "gemm_tcgen05.cuh"
+#include "gemv.cuh"
+#include "pack_quant.cuh"
+
+namespace bitnet {
+namespace {
+
+constexpr int64_t kMaxGemvElems = 196608;  // M * K limit of the fused GEMV
+constexpr int kGemvMaxM = 15;
+constexpr int kLinearGemvMaxM = 15;
+
+inline bool aligned(const void* p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+// Launch with programmatic stream serialisation (PDL) enabled.
+template <typename Kernel, typename... Args>
+bitnet_status launch_pdl(Kernel k, dim3 grid, dim3 block, size_t smem,
+                         cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, args...);
+  return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  bool ready = false;
+};
+
+DeviceInfo g_dev[64];
+std::mutex g_mu;
+
+bitnet_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BITNET_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return BITNET_ERR_CUDA;
+    d.ready = true;
+  }
+  *out = &d;
+  return BITNET_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library does not link libcuda directly.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
+                                   void*, const cuuint64_t*, const cuuint64_t*,
+                                   const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D uint8 tensor map: rows x cols bytes, row pitch `pitch` bytes,
+// box of box_rows x box_cols bytes.
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                 uint64_t pitch, uint32_t box_rows, uint32_t box_cols,
+                 CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {pitch};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bitnet_status check_compute_shape(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K <= 0 || K % 32 != 0) return BITNET_ERR_SHAPE;
+  // index arithmetic inside the kernels is 32-bit per dimension
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return BITNET_ERR_SHAPE;
+  return BITNET_OK;
+}
+
+bitnet_status check_scale_wt(const float* sw, int64_t len, int64_t N) {
+  if (sw == nullptr) return BITNET_ERR_NULL;
+  if (len != 1 && len != N) return BITNET_ERR_SHAPE;
+  if (!aligned(sw, 4)) return BITNET_ERR_ALIGN;
+  return BITNET_OK;
+}
+
+// ---------------------------------------------------------------- GEMV
+template <int MB, int RB, int WPC, bool PREQ>
+bitnet_status launch_gemv_t(const GemvParams& p, int grid_x, int grid_y,
+                            size_t smem, cudaStream_t st) {
+  auto k = gemv_kernel<MB, RB, WPC, PREQ>;
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return BITNET_ERR_CUDA;
+  }
+  return launch_pdl(k, dim3(grid_x, grid_y), dim3(kGemvThreads), smem, st, p);
+}
+
+template <int RB, int WPC, bool PREQ>
+bitnet_status launch_gemv_mb(int mb, const GemvParams& p, int gx, int gy,
+                             size_t smem, cudaStream_t st) {
+  switch (mb) {
+    case 1: return launch_gemv_t<1, RB, WPC, PREQ>(p, gx, gy, smem, st);
+    case 2: return launch_gemv_t<2, RB, WPC, PREQ>(p, gx, gy, smem, st);
+    case 4: return launch_gemv_t<4, RB, WPC, PREQ>(p, gx, gy, smem, st);
+    case 8: return launch_gemv_t<8, RB, WPC, PREQ>(p, gx, gy, smem, st);
+    default: return launch_gemv_t<16, RB, WPC, PREQ>(p, gx, gy, smem, st);
+  }
+}
+
+int bucket_of(int m) { return m <= 1 ? 1 : m <= 2 ? 2 : m <= 4 ? 4 : m <= 8 ? 8 : 16; }
+
+// Shared by the fused GEMV (PREQ = false, M <= 15) and the pre-quantised
+// SIMT fallback of bitnet_gemm (PREQ = true, any M, row chunks of MB).
+bitnet_status run_gemv(const GemvParams& p, bool preq, cudaStream_t st) {
+  DeviceInfo* dev = nullptr;
+  bitnet_status s = device_info(&dev);
+  if (s != BITNET_OK) return s;
+  const int K = p.K, N = p.N, M = p.M;
+  int mb, gy;
+  size_t smem;
+  if (!preq) {
+    mb = bucket_of(M);
+    gy = 1;
+    smem = kGemvSmallBytes + static_cast<size_t>(M) * K;
+  } else {
+    mb = K <= 12288 ? 16 : K <= 24576 ? 8 : K <= 49152 ? 4 : K <= 98304 ? 2 : 1;
+    if (static_cast<int64_t>(mb) * K > kMaxGemvElems) return BITNET_ERR_SHAPE;
+    gy = (M + mb - 1) / mb;
+    smem = kGemvSmallBytes + static_cast<size_t>(mb) * K;
+    if (gy > 65535) return BITNET_ERR_SHAPE;
+  }
+  const int rb = N >= 16 * 4 * 2 * dev->sms ? 4 : 1;
+  const int rows_per_cta = kGemvGroups * rb;
+  int gx = (N + rows_per_cta - 1) / rows_per_cta;
+  // at most what can be resident at once (the kernel strides over rows)
+  const int per_sm_smem = static_cast<int>(228 * 1024 / (smem + 1024));
+  const int per_sm = per_sm_smem < 16 ? (per_sm_smem < 1 ? 1 : per_sm_smem) : 16;
+  const int cap = dev->sms * per_sm;
+  if (gx > cap) gx = cap;
+  if (gx < 1) gx = 1;
+  const bool wide = (K % 64) == 0;
+  if (rb == 4) {
+    if (wide)
+      return preq ? launch_gemv_mb<4, 4, true>(mb, p, gx, gy, smem, st)
+                  : launch_gemv_mb<4, 4, false>(mb, p, gx, gy, smem, st);
+    return preq ? launch_gemv_mb<4, 2, true>(mb, p, gx, gy, smem, st)
+                : launch_gemv_mb<4, 2, false>(mb, p, gx, gy, smem, st);
+  }
+  if (wide)
+    return preq ? launch_gemv_mb<1, 4, true>(mb, p, gx, gy, smem, st)
+                : launch_gemv_mb<1, 4, false>(mb, p, gx, gy, smem, st);
+  return preq ? launch_gemv_mb<1, 2, true>(mb, p, gx, gy, smem, st)
+              : launch_gemv_mb<1, 2, false>(mb, p, gx, gy, smem, st);
+}
+
+// ---------------------------------------------------------------- GEMM
+bool gemm_tcgen05_ok(const int8_t* xq, const uint8_t* wp, int64_t K) {
+  // TMA: row pitches must be multiples of 16 bytes (K/4 for the packed
+  // weights) and base addresses 16-byte aligned.
+  return (K % 64) == 0 && aligned(xq, 16) && aligned(wp, 16);
+}
+
+bitnet_status run_gemm(void* out, bool acc_out, const int8_t* xq,
+                       const uint8_t* wp, const uint16_t* sa, const float* sw,
+                       int64_t sw_len, int64_t M, int64_t N, int64_t K,
+                       cudaStream_t st) {
+  if (M == 0 || N == 0) return BITNET_OK;
+  if (!gemm_tcgen05_ok(xq, wp, K)) {
+    GemvParams p = {};
+    if (acc_out) p.acc_out = static_cast<int32_t*>(out);
+    else p.out = static_cast<uint16_t*>(out);
+    p.xq = xq;
+    p.sa_in = sa;
+    p.wp = wp;
+    p.sw = sw;
+    p.sw_len = static_cast<int>(sw_len);
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    return run_gemv(p, true, st);
+  }
+  DeviceInfo* dev = nullptr;
+  bitnet_status s = device_info(&dev);
+  if (s != BITNET_OK) return s;
+  CUtensorMap mx, mw;
+  if (!make_map_u8(&mx, xq, M, K, K, gemm::BM, gemm::BK, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_u8(&mw, wp, N, K / 4, K / 4, gemm::BN, gemm::BK / 4,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+    return BITNET_ERR_CUDA;
+  const int64_t tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + gemm::BN - 1) / gemm::BN);
+  if (tiles > INT32_MAX) return BITNET_ERR_SHAPE;
+  const int grid = static_cast<int>(tiles < dev->sms ? tiles : dev->sms);
+  if (acc_out) {
+    auto k = gemm::gemm_i8_tcgen05_kernel<true>;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gemm::SMEM_BYTES) != cudaSuccess)
+      return BITNET_ERR_CUDA;
+    return launch_pdl(k, dim3(grid), dim3(gemm::NUM_THREADS), gemm::SMEM_BYTES, st,
+                      mx, mw, out, sa, sw, static_cast<int>(sw_len), static_cast<int>(M),
+                      static_cast<int>(N), static_cast<int>(K));
+  }
+  auto k = gemm::gemm_i8_tcgen05_kernel<false>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           gemm::SMEM_BYTES) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  return launch_pdl(k, dim3(grid), dim3(gemm::NUM_THREADS), gemm::SMEM_BYTES, st, mx,
+                    mw, out, sa, sw, static_cast<int>(sw_len), static_cast<int>(M),
+                    static_cast<int>(N), static_cast<int>(K));
+}
+
+bitnet_status run_quantize(int8_t* xq, uint16_t* sa, const uint16_t* x, int64_t M,
+                           int64_t K, cudaStream_t st) {
+  if (M == 0) return BITNET_OK;
+  if (M > INT32_MAX) return BITNET_ERR_SHAPE;
+  const int64_t nvec = K / 8;
+  const dim3 grid(static_cast<unsigned>(M)), block(kQuantThreads);
+  if (nvec <= 1 * kQuantThreads)
+    return launch_pdl(quantize_rows_kernel<1>, grid, block, 0, st, xq, sa, x, static_cast<int>(K));
+  if (nvec <= 2 * kQuantThreads)
+    return launch_pdl(quantize_rows_kernel<2>, grid, block, 0, st, xq, sa, x, static_cast<int>(K));
+  if (nvec <= 4 * kQuantThreads)
+    return launch_pdl(quantize_rows_kernel<4>, grid, block, 0, st, xq, sa, x, static_cast<int>(K));
+  if (nvec <= 8 * kQuantThreads)
+    return launch_pdl(quantize_rows_kernel<8>, grid, block, 0, st, xq, sa, x, static_cast<int>(K));
+  return launch_pdl(quantize_rows_kernel<0>, grid, block, 0, st, xq, sa, x, static_cast<int>(K));
+}
+
+size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+bool linear_uses_gemv(int64_t M, int64_t K) {
+  return M >= 1 && M <= kLinearGemvMaxM && M * K <= kMaxGemvElems;
+}
+
+}  // namespace
+}  // namespace bitnet
+
+using namespace bitnet;
+
+extern "C" {
+
+const char* bitnet_status_string(bitnet_status s) {
+  switch (s) {
+    case BITNET_OK: return "BITNET_OK";
+    case BITNET_ERR_NULL: return "BITNET_ERR_NULL: a required pointer is NULL";
+    case BITNET_ERR_SHAPE: return "BITNET_ERR_SHAPE: M, N, K or a length is out of range";
+    case BITNET_ERR_DTYPE: return "BITNET_ERR_DTYPE: activation dtype not supported";
+    case BITNET_ERR_ALIGN: return "BITNET_ERR_ALIGN: pointer not aligned as required";
+    case BITNET_ERR_VALUE: return "BITNET_ERR_VALUE: weight outside {-1, 0, +1}";
+    case BITNET_ERR_WORKSPACE: return "BITNET_ERR_WORKSPACE: workspace missing or too small";
+    case BITNET_ERR_CUDA: return "BITNET_ERR_CUDA: CUDA call or launch failed";
+    case BITNET_ERR_TIMEOUT: return "BITNET_ERR_TIMEOUT: a kernel gave up a bounded wait";
+  }
+  return "BITNET_ERR_UNKNOWN";
+}
+
+bitnet_status bitnet_pack_weights(uint8_t* w_packed, const int8_t* w, int64_t N,
+                                  int64_t K, void* stream) {
+  if (N < 0 || K < 0 || K % 4 != 0) return BITNET_ERR_SHAPE;
+  if (N == 0 || K == 0) return BITNET_OK;
+  if (w_packed == nullptr || w == nullptr) return BITNET_ERR_NULL;
+  if (!aligned(w, 4)) return BITNET_ERR_ALIGN;
+  cudaStream_t st = as_stream(stream);
+  const unsigned zero = 0;
+  if (cudaMemcpyToSymbolAsync(g_pack_bad_value, &zero, sizeof zero, 0,
+                              cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  const int64_t total = N * (K / 4);
+  DeviceInfo* dev = nullptr;
+  bitnet_status s = device_info(&dev);
+  if (s != BITNET_OK) return s;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 8 * dev->sms) blocks = 8 * dev->sms;
+  pack_weights_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(w_packed, w, total);
+  if (cudaGetLastError() != cudaSuccess) return BITNET_ERR_CUDA;
+  unsigned bad = 0;
+  if (cudaMemcpyFromSymbolAsync(&bad, g_pack_bad_value, sizeof bad, 0,
+                                cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return BITNET_ERR_CUDA;
+  return bad ? BITNET_ERR_VALUE : BITNET_OK;
+}
+
+bitnet_status bitnet_quantize_act(int8_t* x_q, uint16_t* scale_act, const void* x,
+                                  bitnet_dtype dt, int64_t M, int64_t K, void* stream) {
+  if (dt != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (M < 0 || K <= 0 || K % 32 != 0 || K > INT32_MAX) return BITNET_ERR_SHAPE;
+  if (M == 0) return BITNET_OK;
+  if (x_q == nullptr || scale_act == nullptr || x == nullptr) return BITNET_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(x_q, 16) || !aligned(scale_act, 2)) return BITNET_ERR_ALIGN;
+  return run_quantize(x_q, scale_act, static_cast<const uint16_t*>(x), M, K,
+                      as_stream(stream));
+}
+
+bitnet_status bitnet_gemm(uint16_t* out, const int8_t* x_q, const uint8_t* w_packed,
+                          const uint16_t* scale_act, const float* scale_wt,
+                          int64_t scale_wt_len, int64_t M, int64_t N, int64_t K,
+                          void* stream) {
+  bitnet_status s = check_compute_shape(M, N, K);
+  if (s != BITNET_OK) return s;
+  if (M == 0 || N == 0) return BITNET_OK;
+  if (out == nullptr || x_q == nullptr || w_packed == nullptr || scale_act == nullptr)
+    return BITNET_ERR_NULL;
+  s = check_scale_wt(scale_wt, scale_wt_len, N);
+  if (s != BITNET_OK) return s;
+  if (!aligned(out, 16) || !aligned(x_q, 16) || !aligned(w_packed, 16) ||
+      !aligned(scale_act, 2))
+    return BITNET_ERR_ALIGN;
+  return run_gemm(out, false, x_q, w_packed, scale_act, scale_wt, scale_wt_len, M, N, K,
+                  as_stream(stream));
+}
+
+bitnet_status bitnet_gemm_acc_i32(int32_t* acc, const int8_t* x_q, const uint8_t* w_packed,
+                                  int64_t M, int64_t N, int64_t K, void* stream) {
+  bitnet_status s = check_compute_shape(M, N, K);
+  if (s != BITNET_OK) return s;
+  if (M == 0 || N == 0) return BITNET_OK;
+  if (acc == nullptr || x_q == nullptr || w_packed == nullptr) return BITNET_ERR_NULL;
+  if (!aligned(acc, 16) || !aligned(x_q, 16) || !aligned(w_packed, 16)) return BITNET_ERR_ALIGN;
+  return run_gemm(acc, true, x_q, w_packed, nullptr, nullptr, 1, M, N, K, as_stream(stream));
+}
+
+static bitnet_status gemv_common(GemvParams& p, const void* x, bitnet_dtype dt,
+                                 const uint8_t* w_packed, int64_t M, int64_t N, int64_t K) {
+  if (dt != BITNET_BF16) return BITNET_ERR_DTYPE;
+  bitnet_status s = check_compute_shape(M, N, K);
+  if (s != BITNET_OK) return s;
+  if (M < 1 || M > kGemvMaxM || M * K > kMaxGemvElems) return BITNET_ERR_SHAPE;
+  if (x == nullptr || w_packed == nullptr) return BITNET_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(w_packed, 16)) return BITNET_ERR_ALIGN;
+  p.x = static_cast<const uint16_t*>(x);
+  p.wp = w_packed;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  return BITNET_OK;
+}
+
+bitnet_status bitnet_gemv_fused(uint16_t* out, const void* x, bitnet_dtype dt,
+                                const uint8_t* w_packed, const float* scale_wt,
+                                int64_t scale_wt_len, int64_t M, int64_t N, int64_t K,
+                                void* stream) {
+  GemvParams p = {};
+  bitnet_status s = gemv_common(p, x, dt, w_packed, M, N, K);
+  if (s != BITNET_OK) return s;
+  if (N == 0) return BITNET_OK;
+  if (out == nullptr) return BITNET_ERR_NULL;
+  if (!aligned(out, 16)) return BITNET_ERR_ALIGN;
+  s = check_scale_wt(scale_wt, scale_wt_len, N);
+  if (s != BITNET_OK) return s;
+  p.out = out;
+  p.sw = scale_wt;
+  p.sw_len = static_cast<int>(scale_wt_len);
+  return run_gemv(p, false, as_stream(stream));
+}
+
+bitnet_status bitnet_gemv_fused_debug(int32_t* acc, int8_t* x_q, uint16_t* scale_act,
+                                      const void* x, bitnet_dtype dt,
+                                      const uint8_t* w_packed, int64_t M, int64_t N,
+                                      int64_t K, void* stream) {
+  GemvParams p = {};
+  bitnet_status s = gemv_common(p, x, dt, w_packed, M, N, K);
+  if (s != BITNET_OK) return s;
+  if (acc == nullptr || x_q == nullptr || scale_act == nullptr) return BITNET_ERR_NULL;
+  if (!aligned(acc, 16) || !aligned(x_q, 16) || !aligned(scale_act, 2)) return BITNET_ERR_ALIGN;
+  p.acc_out = acc;
+  p.dbg_q = x_q;
+  p.dbg_sa = scale_act;
+  p.sw_len = 1;
+  if (N == 0) p.N = 0;  // still quantises (block 0) with no weight rows
+  return run_gemv(p, false, as_stream(stream));
+}
+
+size_t bitnet_linear_workspace_bytes(int64_t M, int64_t K) {
+  if (M <= 0 || K <= 0) return 0;
+  if (linear_uses_gemv(M, K)) return 0;
+  return align256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
+         align256(static_cast<size_t>(M) * 2);
+}
+
+bitnet_status bitnet_linear(uint16_t* out, const void* x, bitnet_dtype dt,
+                            const uint8_t* w_packed, const float* scale_wt,
+                            int64_t scale_wt_len, int64_t M, int64_t N, int64_t K,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  if (dt != BITNET_BF16) return BITNET_ERR_DTYPE;
+  bitnet_status s = check_compute_shape(M, N, K);
+  if (s != BITNET_OK) return s;
+  if (M == 0 || N == 0) return BITNET_OK;
+  if (linear_uses_gemv(M, K))
+    return bitnet_gemv_fused(out, x, dt, w_packed, scale_wt, scale_wt_len, M, N, K, stream);
+  const size_t need = bitnet_linear_workspace_bytes(M, K);
+  if (workspace == nullptr || workspace_bytes < need) return BITNET_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return BITNET_ERR_ALIGN;
+  if (out == nullptr || x == nullptr || w_packed == nullptr) return BITNET_ERR_NULL;
+  s = check_scale_wt(scale_wt, scale_wt_len, N);
+  if (s != BITNET_OK) return s;
+  if (!aligned(out, 16) || !aligned(x, 16) || !aligned(w_packed, 16)) return BITNET_ERR_ALIGN;
+  int8_t* xq = static_cast<int8_t*>(workspace);
+  uint16_t* sa = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) +
+                                             align256(static_cast<size_t>(M) * K));
+  cudaStream_t st = as_stream(stream);
+  s = run_quantize(xq, sa, static_cast<const uint16_t*>(x), M, K, st);
+  if (s != BITNET_OK) return s;
+  return run_gemm(out, false, xq, w_packed, sa, scale_wt, scale_wt_len, M, N, K, st);
+}
+
+bitnet_status bitnet_device_status(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return BITNET_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof v) != cudaSuccess) return BITNET_ERR_CUDA;
+  if (v != 0) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero) != cudaSuccess)
+      return BITNET_ERR_CUDA;
+    return BITNET_ERR_TIMEOUT;
+  }
+  return BITNET_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,303 @@
+// Decode GEMV with fused per-token quantisation (M < 16), and the same kernel
+// reading pre-quantised rows (a SIMT fallback for shapes the tensor-core GEMM
+// does not take).
+//
+// The work is bound by streaming the packed weights from HBM once. Layout:
+//   * 8 lanes share one weight row ("group"), 4 groups per warp, 4 warps per
+//     CTA; a group handles RB consecutive rows at a time.
+//   * a lane reads 16-byte chunks (64 weights) of its rows with streaming
+//     128-bit loads; the next batch is loaded while the current one is used,
+//     and the first batch is loaded before waiting on the previous kernel in
+//     the stream (programmatic dependent launch).
+//   * the quantised activations live in shared memory with every 16-element
+//     group transposed 4x4, so that the four 2-bit planes of a packed word,
+//     (w >> 2i) & 0x03030303, line up with one activation word each and feed
+//     dp4a without any byte shuffling. The codes are used as unsigned values
+//     c = w + 2, and sum_k q*w = sum_k q*c - 2 * sum_k q is corrected per row.
+//   * partial sums are reduced over the 8 lanes with warp shuffles, and the
+//     fp32 scale epilogue writes bf16.
+#pragma once
+#include "common.cuh"
+#include "pack_quant.cuh"
+
+namespace bitnet {
+
+constexpr int kGemvThreads = 128;
+constexpr int kGemvLanesPerRow = 8;
+constexpr int kGemvGroups = kGemvThreads / kGemvLanesPerRow;  // 16 per CTA
+constexpr int kGemvU = 2;           // chunks per lane per batch
+constexpr int kGemvSmallBytes = 512;  // per-row scalars before the q rows
+
+struct GemvParams {
+  uint16_t* out;          // bf16 [M, N], or
+  int32_t* acc_out;       // int32 [M, N] (test hook)
+  const uint16_t* x;      // bf16 [M, K] (fused quantisation)
+  const int8_t* xq;       // int8 [M, K] (pre-quantised path)
+  const uint16_t* sa_in;  // bf16 [M]    (pre-quantised path)
+  const uint8_t* wp;      // uint8 [N, K/4]
+  const float* sw;
+  int sw_len;
+  int M, N, K;
+  int8_t* dbg_q;          // optional: codes quantised on chip (block 0)
+  uint16_t* dbg_sa;       // optional: their scales (block 0)
+};
+
+// 4x4 byte transpose of a 16-byte group: out word i byte b = in word b byte i.
+__device__ __forceinline__ uint4 transpose16(const uint4& a) {
+  const uint32_t t0 = prmt(a.x, a.y, 0x5140u);
+  const uint32_t t1 = prmt(a.x, a.y, 0x7362u);
+  const uint32_t t2 = prmt(a.z, a.w, 0x5140u);
+  const uint32_t t3 = prmt(a.z, a.w, 0x7362u);
+  return make_uint4(prmt(t0, t2, 0x5410u), prmt(t0, t2, 0x7632u),
+                    prmt(t1, t3, 0x5410u), prmt(t1, t3, 0x7632u));
+}
+
+__device__ __forceinline__ int bytesum_s8(uint32_t w) {
+  return __dp4a(static_cast<int>(w), 0x01010101, 0);
+}
+
+template <int RB, int WPC>
+__device__ __forceinline__ void gemv_load_batch(
+    uint32_t (&wb)[kGemvU][RB][WPC], const uint8_t* __restrict__ wp, int nb,
+    int c, int N, int R, int KB) {
+#pragma unroll
+  for (int u = 0; u < kGemvU; ++u) {
+    const int cc = c + kGemvLanesPerRow * u;
+#pragma unroll
+    for (int r = 0; r < RB; ++r) {
+      const int n = nb + r;
+      if (n < N && cc < R) {
+        const uint8_t* p = wp + static_cast<int64_t>(n) * KB + cc * (4 * WPC);
+        if constexpr (WPC == 4) {
+          const uint4 v = ldg_stream_v4(p);
+          wb[u][r][0] = v.x; wb[u][r][1] = v.y;
+          wb[u][r][2] = v.z; wb[u][r][3] = v.w;
+        } else {
+          const uint2 v = ldg_stream_v2(p);
+          wb[u][r][0] = v.x; wb[u][r][1] = v.y;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < WPC; ++j) wb[u][r][j] = 0u;
+      }
+    }
+  }
+}
+
+template <int MB, int RB, int WPC, bool PREQ>
+__global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  int* qsum = reinterpret_cast<int*>(smem);                  // [MB]
+  float* saf = reinterpret_cast<float*>(smem + 64);          // [MB]
+  uint32_t* red = reinterpret_cast<uint32_t*>(smem + 128);   // [4][MB]
+  uint8_t* qs = smem + kGemvSmallBytes;                      // [Mc][K]
+
+  pdl_launch_dependents();
+
+  const int K = p.K, N = p.N;
+  const int m_base = PREQ ? static_cast<int>(blockIdx.y) * MB : 0;
+  const int Mc = PREQ ? min(MB, p.M - m_base) : p.M;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int sub = lane & (kGemvLanesPerRow - 1);
+  const int group = warp * (32 / kGemvLanesPerRow) + (lane / kGemvLanesPerRow);
+  const int KB = K / 4;
+  const int R = K / (16 * WPC);
+  const int row_stride = gridDim.x * kGemvGroups * RB;
+  // n0: this group's first row; wfirst: the warp's first group's row, which
+  // drives the loop so that all 32 lanes take the same trip count; cb: the
+  // warp-uniform chunk base of the current batch (lane chunks cb + sub + 8u).
+  int n0 = (static_cast<int>(blockIdx.x) * kGemvGroups + group) * RB;
+  int wfirst = (static_cast<int>(blockIdx.x) * kGemvGroups + warp * (32 / kGemvLanesPerRow)) * RB;
+  int cb = 0;
+
+  // First weight batch before waiting for the producer of the activations.
+  uint32_t wc[kGemvU][RB][WPC];
+  gemv_load_batch<RB, WPC>(wc, p.wp, n0, cb + sub, N, R, KB);
+
+  pdl_wait();
+
+  // ---- stage the quantised activations (transposed groups) in smem -------
+  const int groups16 = K / 16;
+  if constexpr (!PREQ) {
+    uint32_t mb[MB];
+#pragma unroll
+    for (int m = 0; m < MB; ++m) {
+      mb[m] = 0;
+      if (m < Mc) {
+        const uint4* row = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m) * K);
+        for (int v = tid; v < K / 8; v += kGemvThreads)
+          mb[m] = max(mb[m], absmax_bits8(__ldg(row + v)));
+      }
+      mb[m] = __reduce_max_sync(0xFFFFFFFFu, mb[m]);
+      if (lane == 0) red[warp * MB + m] = mb[m];
+    }
+    __syncthreads();
+    RowQuant rq[MB];
+#pragma unroll
+    for (int m = 0; m < MB; ++m) {
+      uint32_t t = 0;
+#pragma unroll
+      for (int w = 0; w < kGemvThreads / 32; ++w) t = max(t, red[w * MB + m]);
+      rq[m] = row_quant(bf16_bits_to_f32(t));
+    }
+    int qs_part[MB];
+#pragma unroll
+    for (int m = 0; m < MB; ++m) {
+      qs_part[m] = 0;
+      if (m < Mc) {
+        const uint4* row = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m) * K);
+        for (int g = tid; g < groups16; g += kGemvThreads) {
+          const uint2 lo = quant8(__ldg(row + 2 * g), rq[m]);
+          const uint2 hi = quant8(__ldg(row + 2 * g + 1), rq[m]);
+          const uint4 nat = make_uint4(lo.x, lo.y, hi.x, hi.y);
+          qs_part[m] += bytesum_s8(nat.x) + bytesum_s8(nat.y) +
+                        bytesum_s8(nat.z) + bytesum_s8(nat.w);
+          *reinterpret_cast<uint4*>(qs + static_cast<int64_t>(m) * K + 16 * g) =
+              transpose16(nat);
+          if (p.dbg_q != nullptr && blockIdx.x == 0)
+            *reinterpret_cast<uint4*>(p.dbg_q + static_cast<int64_t>(m) * K + 16 * g) = nat;
+        }
+      }
+    }
+    __syncthreads();  // red[] reuse
+#pragma unroll
+    for (int m = 0; m < MB; ++m) {
+      const int s = __reduce_add_sync(0xFFFFFFFFu, qs_part[m]);
+      if (lane == 0) red[warp * MB + m] = static_cast<uint32_t>(s);
+    }
+    __syncthreads();
+    if (tid < MB) {
+      int s = 0;
+      for (int w = 0; w < kGemvThreads / 32; ++w) s += static_cast<int>(red[w * MB + tid]);
+      qsum[tid] = s;
+    }
+    // every thread holds the same rq[]; thread 0 publishes the scales
+    if (tid == 0) {
+#pragma unroll
+      for (int m = 0; m < MB; ++m) {
+        const uint16_t sb = f32_to_bf16_bits(rq[m].s);
+        saf[m] = bf16_bits_to_f32(sb);
+        if (p.dbg_sa != nullptr && blockIdx.x == 0 && m < Mc) p.dbg_sa[m] = sb;
+      }
+    }
+  } else {
+    int qs_part[MB];
+#pragma unroll
+    for (int m = 0; m < MB; ++m) {
+      qs_part[m] = 0;
+      if (m < Mc) {
+        const uint4* row = reinterpret_cast<const uint4*>(
+            p.xq + static_cast<int64_t>(m_base + m) * K);
+        for (int g = tid; g < groups16; g += kGemvThreads) {
+          const uint4 nat = __ldg(row + g);
+          qs_part[m] += bytesum_s8(nat.x) + bytesum_s8(nat.y) +
+                        bytesum_s8(nat.z) + bytesum_s8(nat.w);
+          *reinterpret_cast<uint4*>(qs + static_cast<int64_t>(m) * K + 16 * g) =
+              transpose16(nat);
+        }
+      }
+      const int s = __reduce_add_sync(0xFFFFFFFFu, qs_part[m]);
+      if (lane == 0) red[warp * MB + m] = static_cast<uint32_t>(s);
+    }
+    __syncthreads();
+    if (tid < MB) {
+      int s = 0;
+      for (int w = 0; w < kGemvThreads / 32; ++w) s += static_cast<int>(red[w * MB + tid]);
+      qsum[tid] = s;
+      saf[tid] = tid < Mc ? bf16_bits_to_f32(p.sa_in[m_base + tid]) : 0.0f;
+    }
+  }
+  __syncthreads();
+
+  // ---- stream the weights ------------------------------------------------
+  int acc[RB][MB];
+#pragma unroll
+  for (int r = 0; r < RB; ++r)
+#pragma unroll
+    for (int m = 0; m < MB; ++m) acc[r][m] = 0;
+
+  while (wfirst < N) {
+    int cbn = cb + kGemvLanesPerRow * kGemvU;
+    int nn = n0, wn_first = wfirst;
+    const bool row_done = cbn >= R;  // warp-uniform
+    if (row_done) {
+      cbn = 0;
+      nn = n0 + row_stride;
+      wn_first = wfirst + row_stride;
+    }
+    uint32_t wn[kGemvU][RB][WPC];
+    gemv_load_batch<RB, WPC>(wn, p.wp, nn, cbn + sub, N, R, KB);
+
+#pragma unroll
+    for (int u = 0; u < kGemvU; ++u) {
+      const int cc = cb + sub + kGemvLanesPerRow * u;
+      if (cc < R) {
+#pragma unroll
+        for (int j = 0; j < WPC; ++j) {
+          const int g = cc * WPC + j;
+          uint4 Q[MB];
+#pragma unroll
+          for (int m = 0; m < MB; ++m)
+            if (m < Mc) Q[m] = *reinterpret_cast<const uint4*>(qs + static_cast<int64_t>(m) * K + 16 * g);
+#pragma unroll
+          for (int r = 0; r < RB; ++r) {
+            const uint32_t w = wc[u][r][j];
+            const uint32_t e0 = w & 0x03030303u;
+            const uint32_t e1 = (w >> 2) & 0x03030303u;
+            const uint32_t e2 = (w >> 4) & 0x03030303u;
+            const uint32_t e3 = (w >> 6) & 0x03030303u;
+#pragma unroll
+            for (int m = 0; m < MB; ++m) {
+              if (m < Mc) {
+                int a = acc[r][m];
+                a = dp4a_s32(e0, Q[m].x, a);
+                a = dp4a_s32(e1, Q[m].y, a);
+                a = dp4a_s32(e2, Q[m].z, a);
+                a = dp4a_s32(e3, Q[m].w, a);
+                acc[r][m] = a;
+              }
+            }
+          }
+        }
+      }
+    }
+
+    if (row_done) {
+#pragma unroll
+      for (int r = 0; r < RB; ++r) {
+#pragma unroll
+        for (int m = 0; m < MB; ++m) {
+          int v = acc[r][m];
+          v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
+          v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
+          v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
+          acc[r][m] = 0;
+          const int idx = r * MB + m;
+          const int n = n0 + r;
+          if ((idx & (kGemvLanesPerRow - 1)) == sub && m < Mc && n < N) {
+            const int a = v - 2 * qsum[m];
+            const int64_t o = static_cast<int64_t>(m_base + m) * N + n;
+            if (p.acc_out != nullptr) {
+              p.acc_out[o] = a;
+            } else {
+              const float s_w = p.sw[p.sw_len == 1 ? 0 : n];
+              const float y = __fmul_rn(__fmul_rn(__int2float_rn(a), saf[m]), s_w);
+              p.out[o] = f32_to_bf16_bits(y);
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kGemvU; ++u)
+#pragma unroll
+      for (int r = 0; r < RB; ++r)
+#pragma unroll
+        for (int j = 0; j < WPC; ++j) wc[u][r][j] = wn[u][r][j];
+    n0 = nn;
+    wfirst = wn_first;
+    cb = cbn;
+  }
+}
+
+}  // namespace bitnet

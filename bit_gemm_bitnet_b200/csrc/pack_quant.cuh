@@ -1,0 +1,117 @@
+// Weight packing and per-token activation quantisation kernels.
+#pragma once
+#include "common.cuh"
+
+namespace bitnet {
+
+// pack_weights (bitnet-cpu page): code = w + 2, four codes per byte, element
+// 4j+i of a row in bits 2i..2i+1 of byte j. One thread per output byte;
+// values outside {-1, 0, +1} raise g_pack_bad_value.
+__global__ void pack_weights_kernel(uint8_t* __restrict__ out,
+                                    const int8_t* __restrict__ w,
+                                    int64_t total_bytes) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  unsigned bad = 0;
+  for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+       j < total_bytes; j += stride) {
+    // w is 4-byte aligned and K % 4 == 0, so byte j's four weights are the
+    // int32 at element 4j.
+    const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(w) + j);
+    uint32_t byte = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int s = static_cast<int8_t>((v >> (8 * i)) & 0xFFu);
+      bad |= static_cast<unsigned>(s < -1 || s > 1);
+      byte |= (static_cast<uint32_t>(s + 2) & 3u) << (2 * i);
+    }
+    out[j] = static_cast<uint8_t>(byte);
+  }
+  if (bad) atomicOr(&g_pack_bad_value, 1u);
+}
+
+// |bf16| ordering equals the ordering of the magnitude bits for finite
+// values, so the row absmax is a max over (bits & 0x7FFF).
+__device__ __forceinline__ uint32_t absmax_bits8(const uint4& v) {
+  uint32_t m = 0;
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m = max(m, w[i] & 0x7FFFu);
+    m = max(m, (w[i] >> 16) & 0x7FFFu);
+  }
+  return m;
+}
+
+// Quantise the 8 bf16 values of v; returns them packed as 8 int8 (uint2),
+// natural order.
+__device__ __forceinline__ uint2 quant8(const uint4& v, const RowQuant& rq) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[2] = {0, 0};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int lo = quant_one(bf16_bits_to_f32(w[i] & 0xFFFFu), rq);
+    const int hi = quant_one(bf16_bits_to_f32(w[i] >> 16), rq);
+    const uint32_t pair = (static_cast<uint32_t>(lo) & 0xFFu) |
+                          ((static_cast<uint32_t>(hi) & 0xFFu) << 8);
+    o[i >> 1] |= pair << (16 * (i & 1));
+  }
+  return make_uint2(o[0], o[1]);
+}
+
+constexpr int kQuantThreads = 256;
+
+// quantize_activation (bitnet-cpu page), one CTA per row. VPT > 0: the row is
+// held in registers (VPT 16-byte vectors per thread, K <= 8 * 256 * VPT);
+// VPT == 0: two passes over global memory for longer rows.
+template <int VPT>
+__global__ void __launch_bounds__(kQuantThreads)
+    quantize_rows_kernel(int8_t* __restrict__ xq, uint16_t* __restrict__ sa,
+                         const uint16_t* __restrict__ x, int K) {
+  __shared__ uint32_t red[kQuantThreads / 32];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int64_t m = blockIdx.x;
+  const uint4* row = reinterpret_cast<const uint4*>(x + m * K);
+  uint2* qrow = reinterpret_cast<uint2*>(xq + m * K);
+  const int nvec = K / 8;
+  const int tid = threadIdx.x;
+
+  uint4 v[VPT > 0 ? VPT : 1];
+  uint32_t mb = 0;
+  if constexpr (VPT > 0) {
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int idx = tid + i * kQuantThreads;
+      if (idx < nvec) {
+        v[i] = ldg_stream_v4(row + idx);
+        mb = max(mb, absmax_bits8(v[i]));
+      }
+    }
+  } else {
+    for (int idx = tid; idx < nvec; idx += kQuantThreads)
+      mb = max(mb, absmax_bits8(__ldg(row + idx)));
+  }
+  mb = __reduce_max_sync(0xFFFFFFFFu, mb);
+  if ((tid & 31) == 0) red[tid >> 5] = mb;
+  __syncthreads();
+  if (tid < 32) {
+    uint32_t t = tid < kQuantThreads / 32 ? red[tid] : 0u;
+    t = __reduce_max_sync(0xFFFFFFFFu, t);
+    if (tid == 0) red[0] = t;
+  }
+  __syncthreads();
+  const RowQuant rq = row_quant(bf16_bits_to_f32(red[0]));
+  if constexpr (VPT > 0) {
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int idx = tid + i * kQuantThreads;
+      if (idx < nvec) qrow[idx] = quant8(v[i], rq);
+    }
+  } else {
+    for (int idx = tid; idx < nvec; idx += kQuantThreads)
+      qrow[idx] = quant8(__ldg(row + idx), rq);
+  }
+  if (tid == 0) sa[m] = f32_to_bf16_bits(rq.s);
+}
+
+}  // namespace bitnet

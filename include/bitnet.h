@@ -1,0 +1,160 @@
+/* bitnet.h — C ABI of libbitnet_b200: the BitNet b1.58 W1.58A8 linear layer
+ * (ternary weights x per-token INT8 activations) on NVIDIA B200 (sm_100a).
+ *
+ * The operations are the ones the bitnet-cpu page (torch-ext/bitnet_cpu/
+ * __init__.py) defines for the bitnet-tc kernel family:
+ *   pack_weights, quantize_activation, bitnet_gemm, bitnet_gemv_fused and
+ *   bitnet_linear (dispatch by M).
+ *
+ * Conventions for every entry point
+ *   - Outputs come first, as in the native ops that page calls.
+ *   - All array pointers are caller-owned DEVICE pointers on the current CUDA
+ *     device; the library keeps no reference to them after the call returns.
+ *     Matrices are dense and row-major (last index contiguous).
+ *   - bf16 values are passed as their raw 16-bit patterns (uint16_t).
+ *   - `stream` is a cudaStream_t (NULL means the legacy default stream). All
+ *     work is enqueued asynchronously on it; only bitnet_pack_weights and
+ *     bitnet_device_status synchronise it.
+ *   - Arguments are validated before anything is launched; on any error the
+ *     call returns a status other than BITNET_OK and enqueues nothing.
+ *   - Shapes: M (tokens), N (output features), K (input features).
+ *     Compute entry points need K > 0 and K % 32 == 0 (the page's BitLinear
+ *     asserts in_features % 32 == 0); M == 0 or N == 0 is a valid no-op.
+ *   - Alignment: x, x_q, w_packed and out must be 16-byte aligned; scale
+ *     arrays need their natural alignment.
+ *   - Kernels are launched with programmatic stream serialisation: a kernel
+ *     of this library may begin while the preceding kernel on the stream is
+ *     still running, and reads `w_packed` / `scale_wt` before waiting for it.
+ *     Weights and weight scales are therefore load-time constants: they must
+ *     not be written by a kernel that is still running on the same stream
+ *     when the call is enqueued (bitnet_pack_weights synchronises, so its
+ *     output is always safe). Activations and outputs are ordered normally.
+ */
+#ifndef BITNET_B200_H
+#define BITNET_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BITNET_OK = 0,
+  BITNET_ERR_NULL = 1,      /* a required pointer is NULL */
+  BITNET_ERR_SHAPE = 2,     /* M, N, K or a length is out of range */
+  BITNET_ERR_DTYPE = 3,     /* activation dtype not supported */
+  BITNET_ERR_ALIGN = 4,     /* a pointer is not aligned as required */
+  BITNET_ERR_VALUE = 5,     /* pack: a weight is outside {-1, 0, +1} */
+  BITNET_ERR_WORKSPACE = 6, /* workspace NULL or smaller than required */
+  BITNET_ERR_CUDA = 7,      /* a CUDA runtime call or launch failed */
+  BITNET_ERR_TIMEOUT = 8    /* a kernel gave up a bounded wait (device) */
+} bitnet_status;
+
+typedef enum {
+  BITNET_BF16 = 0 /* activations in bf16; other values are rejected */
+} bitnet_dtype;
+
+/* Pack ternary weights into 2-bit codes, four per byte.
+ * Defined by pack_weights() on the bitnet-cpu page: code = w + 2
+ * (-1 -> 1, 0 -> 2, +1 -> 3); byte j of row n holds elements 4j..4j+3 of
+ * that row, element 4j+i in bits 2i..2i+1 (element 0 in the low bits).
+ *   w_packed  out, uint8 [N, K/4]
+ *   w         in,  int8  [N, K], values in {-1, 0, +1}
+ * Needs K % 4 == 0 (the page's assert). Synchronises `stream` to report
+ * BITNET_ERR_VALUE when any input value is outside {-1, 0, +1}; in that case
+ * the contents of w_packed are unspecified. */
+bitnet_status bitnet_pack_weights(uint8_t* w_packed, const int8_t* w,
+                                  int64_t N, int64_t K, void* stream);
+
+/* Per-token absmax INT8 activation quantisation.
+ * Defined by quantize_activation() on the bitnet-cpu page: for each row m,
+ * absmax = max_k |x[m,k]| clamped below at 1e-5, s = absmax / 127 (fp32,
+ * IEEE division), x_q[m,k] = clamp(round_half_even(x[m,k] / s), -127, 127),
+ * scale_act[m] = bf16(s) (round to nearest even). bf16 inputs are widened to
+ * fp32 before any arithmetic.
+ *   x_q        out, int8 [M, K]
+ *   scale_act  out, bf16 [M]
+ *   x          in,  [M, K] of dtype `dt` (only BITNET_BF16) */
+bitnet_status bitnet_quantize_act(int8_t* x_q, uint16_t* scale_act,
+                                  const void* x, bitnet_dtype dt, int64_t M,
+                                  int64_t K, void* stream);
+
+/* Ternary x INT8 GEMM with the scale epilogue (bitnet_gemm() on the bitnet-cpu
+ * page; batched tensor-core path of the bitnet-tc announcement):
+ *   acc[m,n] = sum_k x_q[m,k] * (code(w_packed[n], k) - 2)   (exact int32)
+ *   out[m,n] = bf16( (fp32(acc) * fp32(scale_act[m])) * scale_wt[n or 0] )
+ *   out        out, bf16 [M, N]
+ *   x_q        in,  int8 [M, K]
+ *   w_packed   in,  uint8 [N, K/4]
+ *   scale_act  in,  bf16 [M]
+ *   scale_wt   in,  fp32, scale_wt_len elements: 1 (per tensor) or N
+ * Any M >= 0. */
+bitnet_status bitnet_gemm(uint16_t* out, const int8_t* x_q,
+                          const uint8_t* w_packed, const uint16_t* scale_act,
+                          const float* scale_wt, int64_t scale_wt_len,
+                          int64_t M, int64_t N, int64_t K, void* stream);
+
+/* Fused quantise + ternary GEMV for decode (bitnet_gemv_fused() on the
+ * bitnet-cpu page; the fused dp4a GEMV of the bitnet-tc announcement).
+ * Same result, bit for bit, as bitnet_quantize_act followed by bitnet_gemm.
+ *   out       out, bf16 [M, N]
+ *   x         in,  [M, K] of dtype `dt` (only BITNET_BF16)
+ *   w_packed, scale_wt, scale_wt_len as for bitnet_gemm.
+ * Needs 1 <= M <= 15 (the page dispatches M < 16 here) and M * K <= 196608
+ * (the quantised rows are kept on chip); otherwise BITNET_ERR_SHAPE. */
+bitnet_status bitnet_gemv_fused(uint16_t* out, const void* x, bitnet_dtype dt,
+                                const uint8_t* w_packed, const float* scale_wt,
+                                int64_t scale_wt_len, int64_t M, int64_t N,
+                                int64_t K, void* stream);
+
+/* Workspace bitnet_linear needs for (M, K): 0 when it takes the fused GEMV
+ * path, otherwise room for the int8 [M, K] activations and the bf16 [M]
+ * scales, each 256-byte aligned. */
+size_t bitnet_linear_workspace_bytes(int64_t M, int64_t K);
+
+/* One-shot BitLinear forward (bitnet_linear() on the bitnet-cpu page):
+ * M < 16 (and the fused GEMV's size limit met) -> bitnet_gemv_fused;
+ * otherwise bitnet_quantize_act into `workspace`, then bitnet_gemm.
+ * The page's version allocates its intermediates; a C ABI takes them from
+ * the caller instead: `workspace` (device memory, 256-byte aligned) of at
+ * least bitnet_linear_workspace_bytes(M, K) bytes, or NULL when that is 0. */
+bitnet_status bitnet_linear(uint16_t* out, const void* x, bitnet_dtype dt,
+                            const uint8_t* w_packed, const float* scale_wt,
+                            int64_t scale_wt_len, int64_t M, int64_t N,
+                            int64_t K, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* Synchronise `stream`, then read and clear the device-side error word the
+ * kernels set when a bounded wait gives up. BITNET_ERR_TIMEOUT if it was
+ * set (the outputs of the affected call are then unspecified), BITNET_OK
+ * otherwise, BITNET_ERR_CUDA if the synchronisation itself failed. */
+bitnet_status bitnet_device_status(void* stream);
+
+/* Human-readable name of a status. Never NULL. */
+const char* bitnet_status_string(bitnet_status s);
+
+/* ---- test hooks: the same kernels with the epilogue replaced ------------
+ * Exist so that the exact int32 accumulators (and the fused path's int8
+ * codes and scales) can be compared bit for bit with a reference, as the
+ * bitnet-tc announcement's "bit-exact across every dispatch path" needs. */
+
+/* The batched GEMM kernel storing acc[m, n] (int32 [M, N]) instead of bf16. */
+bitnet_status bitnet_gemm_acc_i32(int32_t* acc, const int8_t* x_q,
+                                  const uint8_t* w_packed, int64_t M,
+                                  int64_t N, int64_t K, void* stream);
+
+/* The fused GEMV kernel storing acc[m, n] (int32 [M, N]) instead of bf16, and
+ * the int8 codes [M, K] and bf16 scales [M] it quantised on chip. */
+bitnet_status bitnet_gemv_fused_debug(int32_t* acc, int8_t* x_q,
+                                      uint16_t* scale_act, const void* x,
+                                      bitnet_dtype dt, const uint8_t* w_packed,
+                                      int64_t M, int64_t N, int64_t K,
+                                      void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITNET_B200_H */

@@ -38,12 +38,14 @@ def lib():
                                             _I64, _P, ctypes.c_int]
         L.oracle_gemm_threads.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64,
                                           _I64, _P, ctypes.c_int]
+        L.oracle_linear_threads_cols.argtypes = [_P, _P, _P, _I64, _I64, _I64,
+                                                 _I64, _P, ctypes.c_int]
         L.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
         L.oracle_f32_to_bf16.restype = ctypes.c_uint16
         for name in ("oracle_pack", "oracle_unpack", "oracle_quantize",
                      "oracle_acc", "oracle_epilogue", "oracle_gemm",
                      "oracle_linear", "oracle_linear_threads",
-                     "oracle_gemm_threads"):
+                     "oracle_gemm_threads", "oracle_linear_threads_cols"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -145,6 +147,20 @@ def linear(x_bf16_bits, packed, scale_wt, threads=1):
         st = lib().oracle_linear_threads(_ptr(x), _ptr(packed), _ptr(sw),
                                          sw.size, M, N, K, _ptr(out), threads)
     _check(st, "linear")
+    return out
+
+
+def linear_cols_threads(x_bf16_bits, packed, scale_wt, threads):
+    """linear with the output columns split across host threads."""
+    x = _c(x_bf16_bits, np.uint16)
+    packed = _c(packed, np.uint8)
+    sw = _c(scale_wt, np.float32).reshape(-1)
+    M, K = x.shape
+    N = packed.shape[0]
+    out = np.empty((M, N), np.uint16)
+    _check(lib().oracle_linear_threads_cols(_ptr(x), _ptr(packed), _ptr(sw), sw.size,
+                                            M, N, K, _ptr(out), threads),
+           "linear_cols_threads")
     return out
 
 

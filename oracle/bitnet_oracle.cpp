@@ -251,6 +251,52 @@ int oracle_gemm_threads(const int8_t* q, const uint8_t* packed,
   return OK;
 }
 
+// The same linear with the output columns split across host threads: the
+// rows are quantised once, then each thread runs the scalar contraction and
+// epilogue above for its slice of weight rows. Used only to time the oracle
+// at small M (decode), where a row split would leave threads idle.
+int oracle_linear_threads_cols(const uint16_t* x, const uint8_t* packed,
+                               const float* scale_wt, int64_t scale_wt_len,
+                               int64_t M, int64_t N, int64_t K, uint16_t* out,
+                               int nthreads) {
+  if (M < 0 || N < 0 || K <= 0 || K % 4 != 0) return ERR_SHAPE;
+  if (scale_wt_len != 1 && scale_wt_len != N) return ERR_SHAPE;
+  std::vector<int8_t> q(static_cast<size_t>(M) * static_cast<size_t>(K));
+  std::vector<uint16_t> sa(static_cast<size_t>(M));
+  int st = oracle_quantize(x, M, K, q.data(), sa.data());
+  if (st != OK) return st;
+  if (nthreads < 1) nthreads = 1;
+  if (N < nthreads) nthreads = static_cast<int>(N > 0 ? N : 1);
+  std::vector<int> status(static_cast<size_t>(nthreads), OK);
+  std::vector<std::thread> pool;
+  const int64_t per = (N + nthreads - 1) / nthreads;
+  const int64_t KB = K / 4;
+  for (int t = 0; t < nthreads; ++t) {
+    const int64_t n0 = t * per;
+    const int64_t n1 = (n0 + per < N) ? n0 + per : N;
+    if (n0 >= n1) continue;
+    pool.emplace_back([=, &q, &sa, &status] {
+      const int64_t nn = n1 - n0;
+      std::vector<int32_t> acc(static_cast<size_t>(M) * static_cast<size_t>(nn));
+      std::vector<uint16_t> part(static_cast<size_t>(M) * static_cast<size_t>(nn));
+      int s = oracle_acc(q.data(), packed + n0 * KB, M, nn, K, acc.data());
+      if (s == OK)
+        s = oracle_epilogue(acc.data(), sa.data(),
+                            scale_wt + (scale_wt_len == 1 ? 0 : n0),
+                            scale_wt_len == 1 ? 1 : nn, M, nn, part.data());
+      if (s == OK)
+        for (int64_t m = 0; m < M; ++m)
+          for (int64_t n = 0; n < nn; ++n)
+            out[m * N + n0 + n] = part[static_cast<size_t>(m * nn + n)];
+      status[static_cast<size_t>(t)] = s;
+    });
+  }
+  for (auto& th : pool) th.join();
+  for (int s : status)
+    if (s != OK) return s;
+  return OK;
+}
+
 // Narrowing used by the oracle, exposed so a test can pin it against a
 // library conversion on its own.
 uint16_t oracle_f32_to_bf16(float f) { return float_to_bf16_bits_rne(f); }

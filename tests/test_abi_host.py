@@ -1,0 +1,95 @@
+"""The C ABI library loads, exports what include/bitnet.h declares, and its
+argument validation rejects bad calls before touching the GPU (no device
+needed: every call here returns before any CUDA work)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bit_gemm_bitnet_b200 as bn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitnet.h")
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bitnet_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = header_functions()
+    for n in ("bitnet_pack_weights", "bitnet_quantize_act", "bitnet_gemm",
+              "bitnet_gemv_fused", "bitnet_linear"):
+        assert n in names
+    assert set(names) == set(bn.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = bn.lib()
+    for n in header_functions():
+        assert hasattr(L, n), n
+
+
+def test_status_strings():
+    for s in range(9):
+        assert bn.status_string(s).startswith("BITNET_")
+    assert "UNKNOWN" in bn.status_string(99)
+
+
+def test_workspace_bytes():
+    assert bn.bitnet_linear_workspace_bytes(1, 4096) == 0
+    assert bn.bitnet_linear_workspace_bytes(15, 4096) == 0
+    assert bn.bitnet_linear_workspace_bytes(16, 4096) == 16 * 4096 + 256
+    assert bn.bitnet_linear_workspace_bytes(8192, 11008) == 8192 * 11008 + 16384
+    # M * K over the fused GEMV's on-chip limit takes the split path
+    assert bn.bitnet_linear_workspace_bytes(15, 16384) > 0
+    assert bn.bitnet_linear_workspace_bytes(0, 4096) == 0
+
+
+P = ctypes.c_void_p
+FAKE = P(0x10000)        # 16-byte aligned, never dereferenced: calls fail first
+ODD = P(0x10008)
+
+
+@pytest.mark.parametrize("call,expect", [
+    (lambda L: L.bitnet_gemm(None, FAKE, FAKE, FAKE, FAKE, 1, 4, 4, 64, None), bn.ERR_NULL),
+    (lambda L: L.bitnet_gemm(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, 4, 48, None), bn.ERR_SHAPE),
+    (lambda L: L.bitnet_gemm(FAKE, FAKE, FAKE, FAKE, FAKE, 1, -1, 4, 64, None), bn.ERR_SHAPE),
+    (lambda L: L.bitnet_gemm(FAKE, FAKE, FAKE, FAKE, FAKE, 3, 4, 4, 64, None), bn.ERR_SHAPE),
+    (lambda L: L.bitnet_gemm(FAKE, FAKE, FAKE, FAKE, None, 1, 4, 4, 64, None), bn.ERR_NULL),
+    (lambda L: L.bitnet_gemm(ODD, FAKE, FAKE, FAKE, FAKE, 1, 4, 4, 64, None), bn.ERR_ALIGN),
+    (lambda L: L.bitnet_gemm(FAKE, FAKE, ODD, FAKE, FAKE, 1, 4, 4, 64, None), bn.ERR_ALIGN),
+    (lambda L: L.bitnet_gemv_fused(FAKE, FAKE, 0, FAKE, FAKE, 1, 16, 4, 64, None), bn.ERR_SHAPE),
+    (lambda L: L.bitnet_gemv_fused(FAKE, FAKE, 0, FAKE, FAKE, 1, 0, 4, 64, None), bn.ERR_SHAPE),
+    (lambda L: L.bitnet_gemv_fused(FAKE, FAKE, 1, FAKE, FAKE, 1, 1, 4, 64, None), bn.ERR_DTYPE),
+    (lambda L: L.bitnet_gemv_fused(FAKE, ODD, 0, FAKE, FAKE, 1, 1, 4, 64, None), bn.ERR_ALIGN),
+    (lambda L: L.bitnet_gemv_fused(FAKE, FAKE, 0, FAKE, FAKE, 1, 15, 4, 16384, None), bn.ERR_SHAPE),
+    (lambda L: L.bitnet_quantize_act(FAKE, FAKE, FAKE, 0, 2, 40, None), bn.ERR_SHAPE),
+    (lambda L: L.bitnet_quantize_act(FAKE, FAKE, None, 0, 2, 64, None), bn.ERR_NULL),
+    (lambda L: L.bitnet_quantize_act(FAKE, FAKE, FAKE, 2, 2, 64, None), bn.ERR_DTYPE),
+    (lambda L: L.bitnet_pack_weights(FAKE, FAKE, 4, 6, None), bn.ERR_SHAPE),
+    (lambda L: L.bitnet_pack_weights(None, FAKE, 4, 8, None), bn.ERR_NULL),
+    (lambda L: L.bitnet_linear(FAKE, FAKE, 0, FAKE, FAKE, 1, 32, 4, 64, None, 0, None),
+     bn.ERR_WORKSPACE),
+    (lambda L: L.bitnet_linear(FAKE, FAKE, 0, FAKE, FAKE, 1, 32, 4, 64, P(0x10010), 1 << 20,
+                               None), bn.ERR_ALIGN),
+    (lambda L: L.bitnet_linear(FAKE, FAKE, 0, FAKE, FAKE, 1, 32, 4, 65, FAKE, 1 << 20, None),
+     bn.ERR_SHAPE),
+    (lambda L: L.bitnet_gemm_acc_i32(FAKE, None, FAKE, 4, 4, 64, None), bn.ERR_NULL),
+    (lambda L: L.bitnet_gemv_fused_debug(FAKE, FAKE, None, FAKE, 0, FAKE, 1, 4, 64, None),
+     bn.ERR_NULL),
+])
+def test_validation_rejects_before_launch(call, expect):
+    assert call(bn.lib()) == expect
+
+
+def test_noop_sizes_return_ok_without_work():
+    L = bn.lib()
+    assert L.bitnet_gemm(None, None, None, None, None, 1, 0, 4, 64, None) == bn.OK
+    assert L.bitnet_gemm(None, None, None, None, None, 1, 4, 0, 64, None) == bn.OK
+    assert L.bitnet_pack_weights(None, None, 0, 8, None) == bn.OK
+    assert L.bitnet_quantize_act(None, None, None, 0, 0, 64, None) == bn.OK
+    assert L.bitnet_linear(None, None, 0, None, None, 1, 0, 4, 64, None, 0, None) == bn.OK

@@ -276,6 +276,9 @@ def test_linear_is_quantize_then_gemm():
     assert np.array_equal(oracle.linear(x, p, sw), oracle.gemm(q, p, sa, sw))
     assert np.array_equal(oracle.linear(x, p, sw, threads=4), oracle.linear(x, p, sw))
     assert np.array_equal(oracle.gemm_threads(q, p, sa, sw, 3), oracle.gemm(q, p, sa, sw))
+    assert np.array_equal(oracle.linear_cols_threads(x, p, sw, 7), oracle.linear(x, p, sw))
+    swn = synth.uniform_f32(synth.key(95, 1, 3), 200, 0.01, 0.1)
+    assert np.array_equal(oracle.linear_cols_threads(x, p, swn, 5), oracle.linear(x, p, swn))
 
 
 def test_linear_close_to_float64_dequantised_product():

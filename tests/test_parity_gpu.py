@@ -1,0 +1,254 @@
+"""Parity of the CUDA path (through the C ABI) with the scalar CPU oracle.
+
+Integer stages (packed bytes, int8 codes, bf16 scale bits, int32
+accumulators) must match bit for bit; bf16 outputs within 1 bf16 ulp
+(relative error <= 2^-8), the tolerance the method's description states.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth import workloads as W
+import bit_gemm_bitnet_b200 as bn
+from helpers import bf16_bits, bf16_ulp_diff, f32_to_bf16_bits, to_dev
+
+pytestmark = pytest.mark.gpu
+
+BF16_ULP_TOL = 1
+
+
+@pytest.fixture(autouse=True)
+def _gpu(cuda_ok):
+    yield
+    bn.bitnet_device_status()
+
+
+def weights(wl, layer, N, K, tensor=synth.T_WEIGHT, variant=0):
+    return synth.ternary(synth.key(wl, layer, tensor, variant), N, K)
+
+
+def acts(wl, layer, M, K, outliers=True, variant=0):
+    return synth.act_bf16(synth.key(wl, layer, synth.T_ACT, variant), M, K,
+                          outliers=outliers)
+
+
+def sw_of(wl, layer, variant=0):
+    return synth.scale_wt(synth.key(wl, layer, synth.T_SCALE_WT, variant))
+
+
+def assert_bf16_close(got_bits, ref_bits):
+    d = bf16_ulp_diff(got_bits, ref_bits)
+    assert d.max() <= BF16_ULP_TOL, f"max ulp {d.max()} at {np.unravel_index(d.argmax(), d.shape)}"
+
+
+# ------------------------------------------------------------------- pack
+
+@pytest.mark.parametrize("N,K", [(1, 4), (7, 12), (512, 512), (640, 2560), (33, 6912)])
+def test_pack_bitexact(N, K):
+    w = weights(90, 0, N, K)
+    got = bn.bitnet_pack_weights(to_dev(w)).cpu().numpy()
+    assert np.array_equal(got, oracle.pack(w))
+
+
+def test_pack_rejects_bad_values():
+    w = weights(90, 1, 16, 64)
+    w[3, 5] = 2
+    with pytest.raises(bn.BitnetValueError):
+        bn.bitnet_pack_weights(to_dev(w))
+
+
+def test_pack_empty():
+    out = bn.bitnet_pack_weights(torch.zeros((0, 8), dtype=torch.int8, device="cuda"))
+    assert out.shape == (0, 2)
+
+
+# --------------------------------------------------------------- quantise
+
+@pytest.mark.parametrize("M,K", [(1, 32), (3, 96), (17, 512), (300, 2560), (64, 4096),
+                                 (5, 11008), (2, 16416), (3, 20000)])
+def test_quantize_bitexact(M, K):
+    x = acts(91, K, M, K)
+    q_ref, s_ref = oracle.quantize(x)
+    q, s = bn.bitnet_quantize_act(to_dev(x, torch.bfloat16))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(bf16_bits(s), s_ref)
+
+
+def test_quantize_ties_and_edge_rows():
+    K = 256
+    rows = []
+    # exact ties: absmax 127 * 2^e makes the scale exactly 2^e
+    for e in (-3, 0, 2):
+        r = np.zeros(K, np.float32)
+        r[0] = 127 * 2.0 ** e
+        r[1:129] = (np.arange(128) - 64 + 0.5) * 2.0 ** e   # (j + 0.5) * s
+        rows.append(r)
+    rows.append(np.zeros(K, np.float32))                    # all-zero row
+    r = np.zeros(K, np.float32); r[7] = 1e-6; rows.append(r)  # absmax < eps
+    r = np.full(K, -3.0, np.float32); rows.append(r)         # constant negative
+    # near-ties: values within a few ulp of (j + 0.5) * s for an inexact s
+    rng = np.random.default_rng(0)
+    r = rng.standard_normal(K).astype(np.float32)
+    r[0] = 10.0
+    s = np.float32(10.0) / np.float32(127.0)
+    j = rng.integers(-126, 126, K // 2)
+    r[1:K // 2 + 1] = ((j + 0.5) * s).astype(np.float32)
+    rows.append(r)
+    x = f32_to_bf16_bits(np.stack(rows))
+    q_ref, s_ref = oracle.quantize(x)
+    q, sc = bn.bitnet_quantize_act(to_dev(x, torch.bfloat16))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(bf16_bits(sc), s_ref)
+
+
+def test_quantize_rejects_bad_shape():
+    with pytest.raises(bn.BitnetValueError):
+        bn.bitnet_quantize_act(torch.zeros((2, 48), dtype=torch.bfloat16, device="cuda"))
+
+
+# ------------------------------------------------------------ fused GEMV
+
+GEMV_CASES = [(1, 512, 512), (4, 512, 512), (1, 2560, 640), (2, 96, 40), (3, 160, 33),
+              (15, 4096, 300), (8, 11008, 130), (1, 2560, 128256 // 16), (5, 6912, 2560),
+              (1, 32, 1), (9, 1024, 4099)]
+
+
+@pytest.mark.parametrize("M,K,N", GEMV_CASES)
+def test_gemv_fused_debug_bitexact(M, K, N):
+    x = acts(92, K, M, K)
+    w = weights(92, N, N, K)
+    p = oracle.pack(w)
+    q_ref, s_ref = oracle.quantize(x)
+    acc_ref = oracle.acc(q_ref, p)
+    acc, q, s = bn.bitnet_gemv_fused_debug(to_dev(x, torch.bfloat16), to_dev(p))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(bf16_bits(s), s_ref)
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+
+
+@pytest.mark.parametrize("M,K,N", GEMV_CASES)
+@pytest.mark.parametrize("per_row_scale", [False, True])
+def test_gemv_fused_matches_oracle(M, K, N, per_row_scale):
+    x = acts(93, K, M, K)
+    w = weights(93, N, N, K)
+    p = oracle.pack(w)
+    sw = (synth.uniform_f32(synth.key(93, N, 3), N, 0.01, 0.1) if per_row_scale
+          else sw_of(93, N))
+    ref = oracle.linear(x, p, sw)
+    got = bn.bitnet_gemv_fused(to_dev(x, torch.bfloat16), to_dev(p), to_dev(sw))
+    assert_bf16_close(bf16_bits(got), ref)
+
+
+def test_gemv_fused_rejects_m16_and_big_mk():
+    x = torch.zeros((16, 512), dtype=torch.bfloat16, device="cuda")
+    p = torch.zeros((8, 128), dtype=torch.uint8, device="cuda")
+    with pytest.raises(bn.BitnetValueError):
+        bn.bitnet_gemv_fused(x, p, 1.0)
+    x = torch.zeros((15, 16384), dtype=torch.bfloat16, device="cuda")
+    p = torch.zeros((8, 4096), dtype=torch.uint8, device="cuda")
+    with pytest.raises(bn.BitnetValueError):
+        bn.bitnet_gemv_fused(x, p, 1.0)
+
+
+# ------------------------------------------------------------------ GEMM
+
+GEMM_CASES = [(4, 512, 512), (1, 128, 256), (130, 384, 300), (128, 4096, 256),
+              (257, 2560, 520), (64, 11008, 384), (300, 256, 1000), (37, 96, 77),
+              (200, 160, 64), (16, 6912, 2560)]
+
+
+@pytest.mark.parametrize("M,K,N", GEMM_CASES)
+def test_gemm_acc_bitexact(M, K, N):
+    rng = np.random.default_rng(M * 7 + K + N)
+    q = rng.integers(-127, 128, size=(M, K)).astype(np.int8)
+    w = weights(94, N, N, K)
+    p = oracle.pack(w)
+    acc = bn.bitnet_gemm_acc_i32(to_dev(q), to_dev(p))
+    assert np.array_equal(acc.cpu().numpy(), oracle.acc(q, p))
+
+
+@pytest.mark.parametrize("M,K,N", GEMM_CASES)
+def test_gemm_matches_oracle(M, K, N):
+    x = acts(95, K, M, K, outliers=False)
+    q, sa = oracle.quantize(x)
+    w = weights(95, N, N, K)
+    p = oracle.pack(w)
+    sw = synth.uniform_f32(synth.key(95, N, 3), N, 0.01, 0.1)
+    ref = oracle.gemm(q, p, sa, sw)
+    got = bn.bitnet_gemm(to_dev(q), to_dev(p), to_dev(sa, torch.bfloat16), to_dev(sw))
+    assert_bf16_close(bf16_bits(got), ref)
+
+
+def test_gemm_extreme_accumulators():
+    # |acc| = 127 * K at the largest K of the workloads
+    K, M, N = 11008, 3, 256
+    q = np.full((M, K), 127, np.int8)
+    q[1] = -127
+    w = np.ones((N, K), np.int8)
+    w[1::2] = -1
+    p = oracle.pack(w)
+    acc = bn.bitnet_gemm_acc_i32(to_dev(q), to_dev(p)).cpu().numpy()
+    assert np.array_equal(acc, oracle.acc(q, p))
+
+
+def test_gemm_empty_and_sentinel():
+    # M = 0 is a no-op; outputs outside [M, N] are never written
+    p = torch.zeros((64, 128), dtype=torch.uint8, device="cuda")
+    q = torch.zeros((0, 512), dtype=torch.int8, device="cuda")
+    sa = torch.zeros((0,), dtype=torch.bfloat16, device="cuda")
+    out = bn.bitnet_gemm(q, p, sa, 1.0)
+    assert out.shape == (0, 64)
+    M, K, N = 5, 256, 40
+    buf = torch.full((M * N + 64,), 0x7F7F, dtype=torch.int16, device="cuda")
+    out = buf[:M * N].view(torch.bfloat16).view(M, N)
+    x = acts(96, 0, M, K)
+    q, sa = oracle.quantize(x)
+    w = weights(96, 0, N, K)
+    pk = oracle.pack(w)
+    bn.bitnet_gemm(to_dev(q), to_dev(pk), to_dev(sa, torch.bfloat16), 0.05, out=out)
+    assert torch.all(buf[M * N:] == 0x7F7F)
+    assert_bf16_close(bf16_bits(out), oracle.gemm(q, pk, sa, np.array([0.05], np.float32)))
+
+
+# ---------------------------------------------------------------- linear
+
+@pytest.mark.parametrize("M", [1, 4, 15, 16, 17, 129])
+def test_linear_dispatch_matches_oracle(M):
+    K, N = 1024, 384
+    x = acts(97, M, M, K)
+    w = weights(97, M, N, K)
+    p = oracle.pack(w)
+    sw = sw_of(97, M)
+    got = bn.bitnet_linear(to_dev(x, torch.bfloat16), to_dev(p), to_dev(sw))
+    assert_bf16_close(bf16_bits(got), oracle.linear(x, p, sw))
+
+
+def test_gemv_and_gemm_paths_agree_tiny_config():
+    """Tiny workload through both the fused GEMV and the GEMM (bit-exact)."""
+    M, K, N = W.TINY["M"], W.TINY["K"], W.TINY["N"]
+    x = acts(W.W_TINY, 0, M, K)
+    w = weights(W.W_TINY, 0, N, K)
+    sw = sw_of(W.W_TINY, 0)
+    p = bn.bitnet_pack_weights(to_dev(w))
+    xd = to_dev(x, torch.bfloat16)
+    y1 = bn.bitnet_gemv_fused(xd, p, to_dev(sw))
+    q, sa = bn.bitnet_quantize_act(xd)
+    y2 = bn.bitnet_gemm(q, p, sa, to_dev(sw))
+    ref = oracle.linear(x, oracle.pack(w), sw)
+    assert np.array_equal(bf16_bits(y1), bf16_bits(y2))
+    assert_bf16_close(bf16_bits(y1), ref)
+
+
+def test_linear_workspace_errors():
+    x = torch.zeros((32, 512), dtype=torch.bfloat16, device="cuda")
+    p = torch.zeros((64, 128), dtype=torch.uint8, device="cuda")
+    sw = torch.ones(1, dtype=torch.float32, device="cuda")
+    out = torch.empty((32, 64), dtype=torch.bfloat16, device="cuda")
+    L = bn.lib()
+    import ctypes
+    st = L.bitnet_linear(ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(x.data_ptr()), 0,
+                         ctypes.c_void_p(p.data_ptr()), ctypes.c_void_p(sw.data_ptr()), 1,
+                         32, 64, 512, None, 0, None)
+    assert st == bn.ERR_WORKSPACE
