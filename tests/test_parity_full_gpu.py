@@ -1,0 +1,111 @@
+"""Parity at the workloads' full sizes, in the launch configuration the bench
+times. Outputs the oracle can afford are compared in full; at prefill sizes
+a seeded sample of rows (quantisation and the contraction are row-local, so
+the oracle computes those rows alone) plus the last, ragged row."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth import workloads as W
+import bit_gemm_bitnet_b200 as bn
+from helpers import bf16_bits, bf16_ulp_diff, to_dev
+
+pytestmark = pytest.mark.gpu
+THREADS = max(1, min(32, os.cpu_count() or 1))
+
+
+@pytest.fixture(autouse=True)
+def _gpu(cuda_ok):
+    yield
+    bn.bitnet_device_status()
+
+
+def close(got, ref):
+    d = bf16_ulp_diff(got, ref)
+    assert d.max() <= 1, f"max ulp {d.max()}"
+
+
+def test_decode_sweep_graph_matches_oracle():
+    """Two layers of the 2B decode sweep plus the LM head, issued as the
+    bench issues them (C-ABI calls captured in one CUDA graph)."""
+    names = [n for n, _, _ in W.DECODE_2B_LAYER]
+    calls = [(layer, names.index(n), K, N) for layer in (0, 29) for n, K, N in W.DECODE_2B_LAYER]
+    calls.append((30, len(names), W.DECODE_2B_LM_HEAD[1], W.DECODE_2B_LM_HEAD[2]))
+    host, dev = [], []
+    for layer, v, K, N in calls:
+        w = synth.ternary(synth.key(W.W_DECODE_2B, layer, synth.T_WEIGHT, v), N, K)
+        sw = synth.scale_wt(synth.key(W.W_DECODE_2B, layer, synth.T_SCALE_WT, v))
+        x = synth.act_bf16(synth.key(W.W_DECODE_2B, layer, synth.T_ACT, v), 1, K)
+        p = oracle.pack(w)
+        host.append((x, p, sw))
+        dev.append((to_dev(x, torch.bfloat16), bn.bitnet_pack_weights(to_dev(w)), to_dev(sw),
+                    torch.empty((1, N), dtype=torch.bfloat16, device="cuda")))
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for x, p, sw, o in dev:
+                bn.bitnet_gemv_fused(x, p, sw, out=o)
+        for o in (d[3] for d in dev):
+            o.fill_(0)
+        g.replay()
+        g.replay()
+    torch.cuda.synchronize()
+    for (x, p, sw), d in zip(host, dev):
+        close(bf16_bits(d[3]), oracle.linear_cols_threads(x, p, sw, THREADS))
+
+
+@pytest.mark.parametrize("M", W.LLAMA_GEMV_M)
+@pytest.mark.parametrize("shape", W.LLAMA_GEMV_SHAPES)
+def test_llama_gemv_full(M, shape):
+    name, K, N = shape
+    v = [s[0] for s in W.LLAMA_GEMV_SHAPES].index(name)
+    w = synth.ternary(synth.key(W.W_LLAMA_GEMV, M, synth.T_WEIGHT, v), N, K)
+    x = synth.act_bf16(synth.key(W.W_LLAMA_GEMV, M, synth.T_ACT, v), M, K)
+    sw = synth.scale_wt(synth.key(W.W_LLAMA_GEMV, M, synth.T_SCALE_WT, v))
+    p = oracle.pack(w)
+    got = bn.bitnet_gemv_fused(to_dev(x, torch.bfloat16), bn.bitnet_pack_weights(to_dev(w)),
+                               to_dev(sw))
+    close(bf16_bits(got), oracle.linear_cols_threads(x, p, sw, THREADS))
+
+
+@pytest.mark.parametrize("M", W.MIDBATCH_M)
+@pytest.mark.parametrize("KN", W.MIDBATCH_SHAPES)
+def test_midbatch_gemm(M, KN):
+    K, N = KN
+    x = synth.act_bf16(synth.key(W.W_MIDBATCH, M, synth.T_ACT, N), M, K, outliers=False)
+    q, sa = oracle.quantize(x)
+    w = synth.ternary(synth.key(W.W_MIDBATCH, M, synth.T_WEIGHT, N), N, K)
+    sw = synth.scale_wt(synth.key(W.W_MIDBATCH, M, synth.T_SCALE_WT, N))
+    p = oracle.pack(w)
+    pd = bn.bitnet_pack_weights(to_dev(w))
+    got = bn.bitnet_gemm(to_dev(q), pd, to_dev(sa, torch.bfloat16), to_dev(sw))
+    rows = np.arange(M) if M <= 64 else np.unique(np.r_[np.random.default_rng(M).choice(M, 24, replace=False), M - 1])
+    ref = oracle.gemm_threads(q[rows], p, sa[rows], sw, THREADS)
+    close(bf16_bits(got)[rows], ref)
+    acc = bn.bitnet_gemm_acc_i32(to_dev(q), pd).cpu().numpy()
+    assert np.array_equal(acc[rows[:8]], oracle.acc(q[rows[:8]], p))
+
+
+@pytest.mark.parametrize("M", W.PREFILL_M)
+@pytest.mark.parametrize("KN", W.PREFILL_SHAPES)
+def test_prefill_linear_sampled_rows(M, KN):
+    K, N = KN
+    x = synth.act_bf16(synth.key(W.W_PREFILL, M, synth.T_ACT, K), M, K)
+    w = synth.ternary(synth.key(W.W_PREFILL, M, synth.T_WEIGHT, K), N, K)
+    sw = synth.scale_wt(synth.key(W.W_PREFILL, M, synth.T_SCALE_WT, K))
+    p = oracle.pack(w)
+    xd = to_dev(x, torch.bfloat16)
+    pd = bn.bitnet_pack_weights(to_dev(w))
+    y = bn.bitnet_linear(xd, pd, to_dev(sw))
+    xq, sa = bn.bitnet_quantize_act(xd)
+    rows = np.unique(np.r_[np.random.default_rng(M + K).choice(M, 40, replace=False), 0, M - 1])
+    q_ref, s_ref = oracle.quantize(x[rows])
+    assert np.array_equal(xq.cpu().numpy()[rows], q_ref)
+    assert np.array_equal(bf16_bits(sa)[rows], s_ref)
+    ref = oracle.linear(x[rows], p, sw, threads=THREADS)
+    close(bf16_bits(y)[rows], ref)
