@@ -204,22 +204,64 @@ def build_decode(bn, dev, rank):
                 x_dev=x_dev, out_dev=out_dev, out_host=out_host, bytes=nbytes)
 
 
-def make_sweep(bn, d):
-    """The step as raw C-ABI calls (pointers prepared once)."""
+def make_sweep(bn, d, order="independent", branches=8):
+    """The step as raw C-ABI calls (pointers prepared once), issued in one of
+    three orders:
+      independent  the 211 calls are independent problems (each has its own
+                   activation row), issued round-robin on `branches` streams
+                   forked from and joined back into the capturing stream;
+      layer        the dependency order of a transformer layer: Q, K, V
+                   concurrently, then O, then gate and up concurrently, then
+                   down; layers one after another, the LM head last;
+      stream       every call after the previous one on one stream.
+    Within a stream, consecutive kernels overlap through programmatic
+    dependent launch; across streams they are ordered by events only."""
     import ctypes
     L = bn.lib()
     args = []
     for (layer, variant, K, N), p, s, x, o in zip(d["calls"], d["packed"], d["scales"],
                                                   d["xs"], d["outs"]):
-        args.append((ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(x.data_ptr()),
-                     ctypes.c_void_p(p.data_ptr()), ctypes.c_void_p(s.data_ptr()), K, N))
+        args.append((layer, variant, ctypes.c_void_p(o.data_ptr()),
+                     ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(p.data_ptr()),
+                     ctypes.c_void_p(s.data_ptr()), K, N))
+    side = [torch.cuda.Stream() for _ in range(max(branches, 3))]
+
+    def issue(a):
+        _, _, o, x, p, s, K, N = a
+        st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        r = L.bitnet_gemv_fused(o, x, 0, p, s, 1, 1, N, K, st)
+        if r != 0:
+            raise RuntimeError(f"bitnet_gemv_fused: {bn.status_string(r)}")
+
+    def fan(groups):
+        main = torch.cuda.current_stream()
+        for i, grp in enumerate(groups):
+            side[i].wait_stream(main)
+            with torch.cuda.stream(side[i]):
+                for a in grp:
+                    issue(a)
+        for i in range(len(groups)):
+            main.wait_stream(side[i])
 
     def sweep():
-        st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-        for o, x, p, s, K, N in args:
-            r = L.bitnet_gemv_fused(o, x, 0, p, s, 1, 1, N, K, st)
-            if r != 0:
-                raise RuntimeError(f"bitnet_gemv_fused: {bn.status_string(r)}")
+        if order == "stream":
+            for a in args:
+                issue(a)
+        elif order == "independent":
+            fan([args[i::branches] for i in range(branches)])
+        else:
+            by_layer = {}
+            for a in args:
+                by_layer.setdefault(a[0], []).append(a)
+            for layer in sorted(by_layer):
+                calls = {a[1]: a for a in by_layer[layer]}
+                if len(calls) == 1:
+                    issue(next(iter(calls.values())))
+                    continue
+                fan([[calls[0]], [calls[1]], [calls[2]]])   # Q, K, V
+                issue(calls[3])                             # O
+                fan([[calls[4]], [calls[5]]])               # gate, up
+                issue(calls[6])                             # down
     return sweep
 
 
@@ -367,6 +409,9 @@ def main():
               "calls_per_step": len(W.decode_2b_sweep()),
               "packed_weight_bytes_per_step": W.decode_2b_packed_bytes(),
               "l2": "inputs larger than L2 (603 MB of packed weights streamed per step)",
+              "issue_order": "independent calls (each has its own activation row) on 8 "
+                             "graph branches; 'issue_orders' reports the transformer-layer "
+                             "dependency order and a single stream",
               "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
     if args.impl == "reference":
@@ -406,25 +451,34 @@ def main():
 
     pk = peaks()
     d = build_decode(bn, dev, rank)
-    sweep = make_sweep(bn, d)
     stream = torch.cuda.Stream(device=dev)
+    graphs = {}
     with torch.cuda.stream(stream):
-        sweep()
-        torch.cuda.synchronize()
-        bn.bitnet_device_status()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
+        for order in ("independent", "layer", "stream"):
+            sweep = make_sweep(bn, d, order)
             sweep()
-        torch.cuda.synchronize()
+            torch.cuda.synchronize()
+            bn.bitnet_device_status()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                sweep()
+            torch.cuda.synchronize()
+            graphs[order] = g
         with ClockSampler(local) as clk:
-            total_ms, per = time_graph(g, args.steps, args.warmup, barrier)
-        e2e_ms = time_e2e(g, d, args.steps, args.warmup, barrier)
+            total_ms, per = time_graph(graphs["independent"], args.steps, args.warmup, barrier)
+        e2e_ms = time_e2e(graphs["independent"], d, args.steps, args.warmup, barrier)
+        other = {}
+        for order in ("layer", "stream"):
+            t_ms, _ = time_graph(graphs[order], args.steps, args.warmup, barrier)
+            other[order] = t_ms
     bn.bitnet_device_status()
 
     if pg is not None:
-        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+        t = torch.tensor([total_ms, e2e_ms, other["layer"], other["stream"]],
+                         dtype=torch.float64, device=dev)
         pg.all_reduce(t, op=pg.ReduceOp.MAX)
         total_ms, e2e_ms = float(t[0]), float(t[1])
+        other = {"layer": float(t[2]), "stream": float(t[3])}
 
     ms_step = total_ms / args.steps
     value = d["bytes"] * world * args.steps / (total_ms / 1e3) / 1e9
@@ -457,6 +511,10 @@ def main():
         "gpu_launches": len(d["calls"]) * args.steps,
         "clocks": clocks,
         "step_ms_min_median": [min(per), statistics.median(per)],
+        "issue_orders": {
+            o: {"ms_per_step": other[o] / args.steps,
+                "gbs": d["bytes"] * world * args.steps / (other[o] / 1e3) / 1e9}
+            for o in ("layer", "stream")},
         "lm_head_alone": {**lm, "frac": lm["gbs"] / pk["hbm_gbs"]},
         "prefill_gemm": pre,
     }

@@ -117,27 +117,49 @@ bitnet_status check_scale_wt(const float* sw, int64_t len, int64_t N) {
 }
 
 // ---------------------------------------------------------------- GEMV
-template <int MB, int RB, int WPC, bool PREQ>
-bitnet_status launch_gemv_t(const GemvParams& p, int grid_x, int grid_y,
-                            size_t smem, cudaStream_t st) {
-  auto k = gemv_kernel<MB, RB, WPC, PREQ>;
+template <int MB, int L, int WPC, bool PREQ>
+bitnet_status launch_gemv_t(const GemvParams& p, int needed_x, int grid_y, size_t smem,
+                            int sms, cudaStream_t st) {
+  auto k = gemv_kernel<MB, L, WPC, PREQ>;
   if (smem > 48 * 1024) {
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return BITNET_ERR_CUDA;
   }
-  return launch_pdl(k, dim3(grid_x, grid_y), dim3(kGemvThreads), smem, st, p);
+  // persistent: no more CTAs than can be resident at once
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kGemvThreads, smem) !=
+      cudaSuccess)
+    return BITNET_ERR_CUDA;
+  if (occ < 1) occ = 1;
+  int gx = needed_x;
+  const int cap = occ * sms;
+  if (gx > cap) gx = cap;
+  if (gx < 1) gx = 1;
+  return launch_pdl(k, dim3(gx, grid_y), dim3(kGemvThreads), smem, st, p);
 }
 
-template <int RB, int WPC, bool PREQ>
-bitnet_status launch_gemv_mb(int mb, const GemvParams& p, int gx, int gy,
-                             size_t smem, cudaStream_t st) {
+template <int L, int WPC, bool PREQ>
+bitnet_status launch_gemv_mb(int mb, const GemvParams& p, int gx, int gy, size_t smem,
+                             int sms, cudaStream_t st) {
   switch (mb) {
-    case 1: return launch_gemv_t<1, RB, WPC, PREQ>(p, gx, gy, smem, st);
-    case 2: return launch_gemv_t<2, RB, WPC, PREQ>(p, gx, gy, smem, st);
-    case 4: return launch_gemv_t<4, RB, WPC, PREQ>(p, gx, gy, smem, st);
-    case 8: return launch_gemv_t<8, RB, WPC, PREQ>(p, gx, gy, smem, st);
-    default: return launch_gemv_t<16, RB, WPC, PREQ>(p, gx, gy, smem, st);
+    case 1: return launch_gemv_t<1, L, WPC, PREQ>(p, gx, gy, smem, sms, st);
+    case 2: return launch_gemv_t<2, L, WPC, PREQ>(p, gx, gy, smem, sms, st);
+    case 4: return launch_gemv_t<4, L, WPC, PREQ>(p, gx, gy, smem, sms, st);
+    case 8: return launch_gemv_t<8, L, WPC, PREQ>(p, gx, gy, smem, sms, st);
+    default: return launch_gemv_t<16, L, WPC, PREQ>(p, gx, gy, smem, sms, st);
+  }
+}
+
+template <int WPC, bool PREQ>
+bitnet_status launch_gemv_l(int lanes, int mb, const GemvParams& p, int gy, size_t smem,
+                            int sms, cudaStream_t st) {
+  const int rows_per_cta = (kGemvThreads / 32) * (32 / lanes);
+  const int gx = (p.N + rows_per_cta - 1) / rows_per_cta;
+  switch (lanes) {
+    case 8: return launch_gemv_mb<8, WPC, PREQ>(mb, p, gx, gy, smem, sms, st);
+    case 16: return launch_gemv_mb<16, WPC, PREQ>(mb, p, gx, gy, smem, sms, st);
+    default: return launch_gemv_mb<32, WPC, PREQ>(mb, p, gx, gy, smem, sms, st);
   }
 }
 
@@ -149,7 +171,7 @@ bitnet_status run_gemv(const GemvParams& p, bool preq, cudaStream_t st) {
   DeviceInfo* dev = nullptr;
   bitnet_status s = device_info(&dev);
   if (s != BITNET_OK) return s;
-  const int K = p.K, N = p.N, M = p.M;
+  const int K = p.K, M = p.M;
   int mb, gy;
   size_t smem;
   if (!preq) {
@@ -163,28 +185,15 @@ bitnet_status run_gemv(const GemvParams& p, bool preq, cudaStream_t st) {
     smem = kGemvSmallBytes + static_cast<size_t>(mb) * K;
     if (gy > 65535) return BITNET_ERR_SHAPE;
   }
-  const int rb = N >= 16 * 4 * 2 * dev->sms ? 4 : 1;
-  const int rows_per_cta = kGemvGroups * rb;
-  int gx = (N + rows_per_cta - 1) / rows_per_cta;
-  // at most what can be resident at once (the kernel strides over rows)
-  const int per_sm_smem = static_cast<int>(228 * 1024 / (smem + 1024));
-  const int per_sm = per_sm_smem < 16 ? (per_sm_smem < 1 ? 1 : per_sm_smem) : 16;
-  const int cap = dev->sms * per_sm;
-  if (gx > cap) gx = cap;
-  if (gx < 1) gx = 1;
   const bool wide = (K % 64) == 0;
-  if (rb == 4) {
-    if (wide)
-      return preq ? launch_gemv_mb<4, 4, true>(mb, p, gx, gy, smem, st)
-                  : launch_gemv_mb<4, 4, false>(mb, p, gx, gy, smem, st);
-    return preq ? launch_gemv_mb<4, 2, true>(mb, p, gx, gy, smem, st)
-                : launch_gemv_mb<4, 2, false>(mb, p, gx, gy, smem, st);
-  }
+  const int chunks = wide ? K / 64 : K / 32;  // chunks per weight row
+  // lanes per row: the fewest that keep a lane at <= 8 chunks of a row
+  const int lanes = chunks <= 8 * 8 ? 8 : chunks <= 8 * 16 ? 16 : 32;
   if (wide)
-    return preq ? launch_gemv_mb<1, 4, true>(mb, p, gx, gy, smem, st)
-                : launch_gemv_mb<1, 4, false>(mb, p, gx, gy, smem, st);
-  return preq ? launch_gemv_mb<1, 2, true>(mb, p, gx, gy, smem, st)
-              : launch_gemv_mb<1, 2, false>(mb, p, gx, gy, smem, st);
+    return preq ? launch_gemv_l<4, true>(lanes, mb, p, gy, smem, dev->sms, st)
+                : launch_gemv_l<4, false>(lanes, mb, p, gy, smem, dev->sms, st);
+  return preq ? launch_gemv_l<2, true>(lanes, mb, p, gy, smem, dev->sms, st)
+              : launch_gemv_l<2, false>(lanes, mb, p, gy, smem, dev->sms, st);
 }
 
 // ---------------------------------------------------------------- GEMM

@@ -3,12 +3,14 @@
 // does not take).
 //
 // The work is bound by streaming the packed weights from HBM once. Layout:
-//   * 8 lanes share one weight row ("group"), 4 groups per warp, 4 warps per
-//     CTA; a group handles RB consecutive rows at a time.
-//   * a lane reads 16-byte chunks (64 weights) of its rows with streaming
-//     128-bit loads; the next batch is loaded while the current one is used,
-//     and the first batch is loaded before waiting on the previous kernel in
-//     the stream (programmatic dependent launch).
+//   * L lanes (8, 16 or 32, chosen so that a lane holds at most 8 chunks of a
+//     row) share one weight row; 8 warps per CTA; CTAs are persistent (as
+//     many as fit at once) and stride over the rows.
+//   * a lane issues all loads of its part of a row at once (16-byte streaming
+//     loads, 64 weights each), and the next row's loads before using the
+//     current one; the first row is requested before waiting on the previous
+//     kernel in the stream (programmatic dependent launch), so small layers
+//     have their weights in flight while the activations are quantised.
 //   * the quantised activations live in shared memory with every 16-element
 //     group transposed 4x4, so that the four 2-bit planes of a packed word,
 //     (w >> 2i) & 0x03030303, line up with one activation word each and feed
@@ -22,11 +24,10 @@
 
 namespace bitnet {
 
-constexpr int kGemvThreads = 128;
-constexpr int kGemvLanesPerRow = 8;
-constexpr int kGemvGroups = kGemvThreads / kGemvLanesPerRow;  // 16 per CTA
-constexpr int kGemvU = 2;           // chunks per lane per batch
-constexpr int kGemvSmallBytes = 512;  // per-row scalars before the q rows
+constexpr int kGemvThreads = 256;
+constexpr int kGemvWarps = kGemvThreads / 32;
+constexpr int kGemvCPL = 8;           // chunks per lane loaded at once
+constexpr int kGemvSmallBytes = 1024;  // per-row scalars before the q rows
 
 struct GemvParams {
   uint16_t* out;          // bf16 [M, N], or
@@ -56,63 +57,67 @@ __device__ __forceinline__ int bytesum_s8(uint32_t w) {
   return __dp4a(static_cast<int>(w), 0x01010101, 0);
 }
 
-template <int RB, int WPC>
-__device__ __forceinline__ void gemv_load_batch(
-    uint32_t (&wb)[kGemvU][RB][WPC], const uint8_t* __restrict__ wp, int nb,
-    int c, int N, int R, int KB) {
+// Load the chunks lane `sub` owns in piece `pc` of weight row `n`:
+// chunk c = pc * L * CPL + sub + L * i (i < CPL), zero past the row or N.
+template <int L, int WPC>
+__device__ __forceinline__ void gemv_load_row(uint32_t (&wb)[kGemvCPL][WPC],
+                                              const uint8_t* __restrict__ wp, int n,
+                                              int pc, int sub, int N, int R, int KB) {
+  const int c0 = pc * L * kGemvCPL + sub;
 #pragma unroll
-  for (int u = 0; u < kGemvU; ++u) {
-    const int cc = c + kGemvLanesPerRow * u;
-#pragma unroll
-    for (int r = 0; r < RB; ++r) {
-      const int n = nb + r;
-      if (n < N && cc < R) {
-        const uint8_t* p = wp + static_cast<int64_t>(n) * KB + cc * (4 * WPC);
-        if constexpr (WPC == 4) {
-          const uint4 v = ldg_stream_v4(p);
-          wb[u][r][0] = v.x; wb[u][r][1] = v.y;
-          wb[u][r][2] = v.z; wb[u][r][3] = v.w;
-        } else {
-          const uint2 v = ldg_stream_v2(p);
-          wb[u][r][0] = v.x; wb[u][r][1] = v.y;
-        }
+  for (int i = 0; i < kGemvCPL; ++i) {
+    const int c = c0 + L * i;
+    if (n < N && c < R) {
+      const uint8_t* ptr = wp + static_cast<int64_t>(n) * KB + c * (4 * WPC);
+      if constexpr (WPC == 4) {
+        const uint4 v = ldg_stream_v4(ptr);
+        wb[i][0] = v.x; wb[i][1] = v.y; wb[i][2] = v.z; wb[i][3] = v.w;
       } else {
-#pragma unroll
-        for (int j = 0; j < WPC; ++j) wb[u][r][j] = 0u;
+        const uint2 v = ldg_stream_v2(ptr);
+        wb[i][0] = v.x; wb[i][1] = v.y;
       }
+    } else {
+#pragma unroll
+      for (int j = 0; j < WPC; ++j) wb[i][j] = 0u;
     }
   }
 }
 
-template <int MB, int RB, int WPC, bool PREQ>
+// MB: rows of x per CTA (bucket); L: lanes per weight row (8, 16 or 32);
+// WPC: 32-bit words per chunk (4: 16-byte chunks, needs K % 64 == 0; 2: 8-byte
+// chunks); PREQ: activations come pre-quantised (x_q + scale_act).
+template <int MB, int L, int WPC, bool PREQ>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
   int* qsum = reinterpret_cast<int*>(smem);                  // [MB]
   float* saf = reinterpret_cast<float*>(smem + 64);          // [MB]
-  uint32_t* red = reinterpret_cast<uint32_t*>(smem + 128);   // [4][MB]
+  uint32_t* red = reinterpret_cast<uint32_t*>(smem + 128);   // [warps][MB]
   uint8_t* qs = smem + kGemvSmallBytes;                      // [Mc][K]
+  static_assert(kGemvWarps * MB * 4 <= kGemvSmallBytes - 128, "reduction scratch");
 
   pdl_launch_dependents();
 
+  constexpr int G = 32 / L;                  // weight rows per warp at a time
+  constexpr int GPC = kGemvWarps * G;        // weight rows per CTA at a time
   const int K = p.K, N = p.N;
   const int m_base = PREQ ? static_cast<int>(blockIdx.y) * MB : 0;
   const int Mc = PREQ ? min(MB, p.M - m_base) : p.M;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int sub = lane & (kGemvLanesPerRow - 1);
-  const int group = warp * (32 / kGemvLanesPerRow) + (lane / kGemvLanesPerRow);
+  const int sub = lane % L;
   const int KB = K / 4;
-  const int R = K / (16 * WPC);
-  const int row_stride = gridDim.x * kGemvGroups * RB;
-  // n0: this group's first row; wfirst: the warp's first group's row, which
-  // drives the loop so that all 32 lanes take the same trip count; cb: the
-  // warp-uniform chunk base of the current batch (lane chunks cb + sub + 8u).
-  int n0 = (static_cast<int>(blockIdx.x) * kGemvGroups + group) * RB;
-  int wfirst = (static_cast<int>(blockIdx.x) * kGemvGroups + warp * (32 / kGemvLanesPerRow)) * RB;
-  int cb = 0;
+  const int R = K / (16 * WPC);                            // chunks per row
+  const int pieces = (R + L * kGemvCPL - 1) / (L * kGemvCPL);
+  const int stride = gridDim.x * GPC;
+  // n: this group's row; wrow: the warp's first row, which drives the loop so
+  // that all 32 lanes take the same trip count.
+  int n = static_cast<int>(blockIdx.x) * GPC + warp * G + lane / L;
+  int wrow = static_cast<int>(blockIdx.x) * GPC + warp * G;
+  int pc = 0;
 
-  // First weight batch before waiting for the producer of the activations.
-  uint32_t wc[kGemvU][RB][WPC];
-  gemv_load_batch<RB, WPC>(wc, p.wp, n0, cb + sub, N, R, KB);
+  // The first row's weights are requested before waiting for the kernel
+  // that produces the activations.
+  uint32_t cur[kGemvCPL][WPC];
+  gemv_load_row<L, WPC>(cur, p.wp, n, 0, sub, N, R, KB);
 
   pdl_wait();
 
@@ -137,7 +142,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
     for (int m = 0; m < MB; ++m) {
       uint32_t t = 0;
 #pragma unroll
-      for (int w = 0; w < kGemvThreads / 32; ++w) t = max(t, red[w * MB + m]);
+      for (int w = 0; w < kGemvWarps; ++w) t = max(t, red[w * MB + m]);
       rq[m] = row_quant(bf16_bits_to_f32(t));
     }
     int qs_part[MB];
@@ -168,7 +173,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
     __syncthreads();
     if (tid < MB) {
       int s = 0;
-      for (int w = 0; w < kGemvThreads / 32; ++w) s += static_cast<int>(red[w * MB + tid]);
+      for (int w = 0; w < kGemvWarps; ++w) s += static_cast<int>(red[w * MB + tid]);
       qsum[tid] = s;
     }
     // every thread holds the same rq[]; thread 0 publishes the scales
@@ -202,7 +207,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
     __syncthreads();
     if (tid < MB) {
       int s = 0;
-      for (int w = 0; w < kGemvThreads / 32; ++w) s += static_cast<int>(red[w * MB + tid]);
+      for (int w = 0; w < kGemvWarps; ++w) s += static_cast<int>(red[w * MB + tid]);
       qsum[tid] = s;
       // the int32 test hook passes no scales
       saf[tid] = (tid < Mc && p.sa_in != nullptr) ? bf16_bits_to_f32(p.sa_in[m_base + tid]) : 0.0f;
@@ -211,52 +216,45 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
   __syncthreads();
 
   // ---- stream the weights ------------------------------------------------
-  int acc[RB][MB];
+  int acc[MB];
 #pragma unroll
-  for (int r = 0; r < RB; ++r)
-#pragma unroll
-    for (int m = 0; m < MB; ++m) acc[r][m] = 0;
+  for (int m = 0; m < MB; ++m) acc[m] = 0;
 
-  while (wfirst < N) {
-    int cbn = cb + kGemvLanesPerRow * kGemvU;
-    int nn = n0, wn_first = wfirst;
-    const bool row_done = cbn >= R;  // warp-uniform
+  while (wrow < N) {
+    // next unit: the next piece of this row, or the next row's first piece
+    int pn = pc + 1, nn = n, wn = wrow;
+    const bool row_done = pn == pieces;  // warp-uniform
     if (row_done) {
-      cbn = 0;
-      nn = n0 + row_stride;
-      wn_first = wfirst + row_stride;
+      pn = 0;
+      nn = n + stride;
+      wn = wrow + stride;
     }
-    uint32_t wn[kGemvU][RB][WPC];
-    gemv_load_batch<RB, WPC>(wn, p.wp, nn, cbn + sub, N, R, KB);
+    uint32_t nxt[kGemvCPL][WPC];
+    gemv_load_row<L, WPC>(nxt, p.wp, nn, pn, sub, N, R, KB);
 
+    const int c0 = pc * L * kGemvCPL + sub;
 #pragma unroll
-    for (int u = 0; u < kGemvU; ++u) {
-      const int cc = cb + sub + kGemvLanesPerRow * u;
-      if (cc < R) {
+    for (int i = 0; i < kGemvCPL; ++i) {
+      const int c = c0 + L * i;
+      if (c < R) {
 #pragma unroll
         for (int j = 0; j < WPC; ++j) {
-          const int g = cc * WPC + j;
-          uint4 Q[MB];
+          const int g = c * WPC + j;
+          const uint32_t w = cur[i][j];
+          const uint32_t e0 = w & 0x03030303u;
+          const uint32_t e1 = (w >> 2) & 0x03030303u;
+          const uint32_t e2 = (w >> 4) & 0x03030303u;
+          const uint32_t e3 = (w >> 6) & 0x03030303u;
 #pragma unroll
-          for (int m = 0; m < MB; ++m)
-            if (m < Mc) Q[m] = *reinterpret_cast<const uint4*>(qs + static_cast<int64_t>(m) * K + 16 * g);
-#pragma unroll
-          for (int r = 0; r < RB; ++r) {
-            const uint32_t w = wc[u][r][j];
-            const uint32_t e0 = w & 0x03030303u;
-            const uint32_t e1 = (w >> 2) & 0x03030303u;
-            const uint32_t e2 = (w >> 4) & 0x03030303u;
-            const uint32_t e3 = (w >> 6) & 0x03030303u;
-#pragma unroll
-            for (int m = 0; m < MB; ++m) {
-              if (m < Mc) {
-                int a = acc[r][m];
-                a = dp4a_s32(e0, Q[m].x, a);
-                a = dp4a_s32(e1, Q[m].y, a);
-                a = dp4a_s32(e2, Q[m].z, a);
-                a = dp4a_s32(e3, Q[m].w, a);
-                acc[r][m] = a;
-              }
+          for (int m = 0; m < MB; ++m) {
+            if (m < Mc) {
+              const uint4 Q = *reinterpret_cast<const uint4*>(qs + static_cast<int64_t>(m) * K + 16 * g);
+              int a = acc[m];
+              a = dp4a_s32(e0, Q.x, a);
+              a = dp4a_s32(e1, Q.y, a);
+              a = dp4a_s32(e2, Q.z, a);
+              a = dp4a_s32(e3, Q.w, a);
+              acc[m] = a;
             }
           }
         }
@@ -265,39 +263,31 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
 
     if (row_done) {
 #pragma unroll
-      for (int r = 0; r < RB; ++r) {
+      for (int m = 0; m < MB; ++m) {
+        int v = acc[m];
 #pragma unroll
-        for (int m = 0; m < MB; ++m) {
-          int v = acc[r][m];
-          v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
-          v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
-          v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
-          acc[r][m] = 0;
-          const int idx = r * MB + m;
-          const int n = n0 + r;
-          if ((idx & (kGemvLanesPerRow - 1)) == sub && m < Mc && n < N) {
-            const int a = v - 2 * qsum[m];
-            const int64_t o = static_cast<int64_t>(m_base + m) * N + n;
-            if (p.acc_out != nullptr) {
-              p.acc_out[o] = a;
-            } else {
-              const float s_w = p.sw[p.sw_len == 1 ? 0 : n];
-              const float y = __fmul_rn(__fmul_rn(__int2float_rn(a), saf[m]), s_w);
-              p.out[o] = f32_to_bf16_bits(y);
-            }
+        for (int o = 1; o < L; o <<= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        acc[m] = 0;
+        if ((m % L) == sub && m < Mc && n < N) {
+          const int a = v - 2 * qsum[m];
+          const int64_t o = static_cast<int64_t>(m_base + m) * N + n;
+          if (p.acc_out != nullptr) {
+            p.acc_out[o] = a;
+          } else {
+            const float s_w = p.sw[p.sw_len == 1 ? 0 : n];
+            const float y = __fmul_rn(__fmul_rn(__int2float_rn(a), saf[m]), s_w);
+            p.out[o] = f32_to_bf16_bits(y);
           }
         }
       }
     }
 #pragma unroll
-    for (int u = 0; u < kGemvU; ++u)
+    for (int i = 0; i < kGemvCPL; ++i)
 #pragma unroll
-      for (int r = 0; r < RB; ++r)
-#pragma unroll
-        for (int j = 0; j < WPC; ++j) wc[u][r][j] = wn[u][r][j];
-    n0 = nn;
-    wfirst = wn_first;
-    cb = cbn;
+      for (int j = 0; j < WPC; ++j) cur[i][j] = nxt[i][j];
+    n = nn;
+    wrow = wn;
+    pc = pn;
   }
 }
 
