@@ -220,8 +220,11 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
 #pragma unroll
   for (int m = 0; m < MB; ++m) acc[m] = 0;
 
-  while (wrow < N) {
-    // next unit: the next piece of this row, or the next row's first piece
+  // One unit = one piece of one row. `use` holds the current unit; the next
+  // unit's loads go into `fill` before `use` is consumed. The two buffers
+  // alternate (no register copies, which would wait on the loads in flight).
+  uint32_t other[kGemvCPL][WPC];
+  auto step = [&](uint32_t (&use)[kGemvCPL][WPC], uint32_t (&fill)[kGemvCPL][WPC]) -> bool {
     int pn = pc + 1, nn = n, wn = wrow;
     const bool row_done = pn == pieces;  // warp-uniform
     if (row_done) {
@@ -229,8 +232,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
       nn = n + stride;
       wn = wrow + stride;
     }
-    uint32_t nxt[kGemvCPL][WPC];
-    gemv_load_row<L, WPC>(nxt, p.wp, nn, pn, sub, N, R, KB);
+    if (wn < N) gemv_load_row<L, WPC>(fill, p.wp, nn, pn, sub, N, R, KB);
 
     const int c0 = pc * L * kGemvCPL + sub;
 #pragma unroll
@@ -240,7 +242,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
 #pragma unroll
         for (int j = 0; j < WPC; ++j) {
           const int g = c * WPC + j;
-          const uint32_t w = cur[i][j];
+          const uint32_t w = use[i][j];
           const uint32_t e0 = w & 0x03030303u;
           const uint32_t e1 = (w >> 2) & 0x03030303u;
           const uint32_t e2 = (w >> 4) & 0x03030303u;
@@ -281,13 +283,15 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
         }
       }
     }
-#pragma unroll
-    for (int i = 0; i < kGemvCPL; ++i)
-#pragma unroll
-      for (int j = 0; j < WPC; ++j) cur[i][j] = nxt[i][j];
     n = nn;
     wrow = wn;
     pc = pn;
+    return wrow < N;
+  };
+
+  if (wrow < N) {
+    while (step(cur, other) && step(other, cur)) {
+    }
   }
 }
 
