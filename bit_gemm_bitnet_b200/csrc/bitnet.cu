@@ -13,7 +13,6 @@
 namespace bitnet {
 namespace {
 
-constexpr int64_t kMaxGemvElems = 196608;  // M * K limit of the fused GEMV
 constexpr int kGemvMaxM = 15;
 constexpr int kLinearGemvMaxM = 15;
 
@@ -117,83 +116,122 @@ bitnet_status check_scale_wt(const float* sw, int64_t len, int64_t N) {
 }
 
 // ---------------------------------------------------------------- GEMV
-template <int MB, int L, int WPC, bool PREQ>
-bitnet_status launch_gemv_t(const GemvParams& p, int needed_x, int grid_y, size_t smem,
-                            int sms, cudaStream_t st) {
-  auto k = gemv_kernel<MB, L, WPC, PREQ>;
+size_t align128(size_t v) { return (v + 127) & ~static_cast<size_t>(127); }
+
+constexpr size_t kSmemLimit = 232448;  // per-CTA opt-in maximum on sm_100
+
+// Shared memory of the GEMV for `rows` activation rows of length K and a ring
+// of `stages` stages of `rw` rows per warp.
+size_t gemv_smem(int rows, int64_t K, int rw, int stages) {
+  return kGemvHeaderBytes + align128(static_cast<size_t>(rows) * K) +
+         static_cast<size_t>(stages) * align128(static_cast<size_t>(8 * rw) * (K / 4));
+}
+
+// Does the GEMV fit `rows` activation rows of length K (two stages of one
+// row per warp at least)?
+bool gemv_fits(int rows, int64_t K) { return gemv_smem(rows, K, 1, 2) <= kSmemLimit; }
+
+int pow2_floor(int64_t v) {
+  int r = 1;
+  while (static_cast<int64_t>(r) * 2 <= v) r *= 2;
+  return r;
+}
+
+template <int MB, int RW, bool WIDE, bool PREQ>
+bitnet_status launch_gemv_t(const GemvParams& p, int grid_y, size_t smem, int sms,
+                            cudaStream_t st) {
+  auto k = gemv_kernel<MB, RW, WIDE, PREQ>;
   if (smem > 48 * 1024) {
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return BITNET_ERR_CUDA;
   }
-  // persistent: no more CTAs than can be resident at once
+  // persistent: no more CTAs than row blocks, nor than can be resident
   int occ = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kGemvThreads, smem) !=
-      cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kGemvThreads, smem) != cudaSuccess)
     return BITNET_ERR_CUDA;
   if (occ < 1) occ = 1;
-  int gx = needed_x;
-  const int cap = occ * sms;
-  if (gx > cap) gx = cap;
+  const int nblocks = (p.N + p.rows_per_block - 1) / p.rows_per_block;
+  int gx = nblocks < occ * sms ? nblocks : occ * sms;
   if (gx < 1) gx = 1;
   return launch_pdl(k, dim3(gx, grid_y), dim3(kGemvThreads), smem, st, p);
 }
 
-template <int L, int WPC, bool PREQ>
-bitnet_status launch_gemv_mb(int mb, const GemvParams& p, int gx, int gy, size_t smem,
-                             int sms, cudaStream_t st) {
-  switch (mb) {
-    case 1: return launch_gemv_t<1, L, WPC, PREQ>(p, gx, gy, smem, sms, st);
-    case 2: return launch_gemv_t<2, L, WPC, PREQ>(p, gx, gy, smem, sms, st);
-    case 4: return launch_gemv_t<4, L, WPC, PREQ>(p, gx, gy, smem, sms, st);
-    case 8: return launch_gemv_t<8, L, WPC, PREQ>(p, gx, gy, smem, sms, st);
-    default: return launch_gemv_t<16, L, WPC, PREQ>(p, gx, gy, smem, sms, st);
+template <int MB, bool WIDE, bool PREQ>
+bitnet_status launch_gemv_rw(int rw, const GemvParams& p, int gy, size_t smem, int sms,
+                             cudaStream_t st) {
+  switch (rw) {
+    case 1: return launch_gemv_t<MB, 1, WIDE, PREQ>(p, gy, smem, sms, st);
+    case 2: return launch_gemv_t<MB, 2, WIDE, PREQ>(p, gy, smem, sms, st);
+    case 4:
+      if constexpr (MB <= 8) return launch_gemv_t<MB, 4, WIDE, PREQ>(p, gy, smem, sms, st);
+      return BITNET_ERR_SHAPE;
+    default:
+      if constexpr (MB <= 4) return launch_gemv_t<MB, 8, WIDE, PREQ>(p, gy, smem, sms, st);
+      return BITNET_ERR_SHAPE;
   }
 }
 
-template <int WPC, bool PREQ>
-bitnet_status launch_gemv_l(int lanes, int mb, const GemvParams& p, int gy, size_t smem,
-                            int sms, cudaStream_t st) {
-  const int rows_per_cta = (kGemvThreads / 32) * (32 / lanes);
-  const int gx = (p.N + rows_per_cta - 1) / rows_per_cta;
-  switch (lanes) {
-    case 8: return launch_gemv_mb<8, WPC, PREQ>(mb, p, gx, gy, smem, sms, st);
-    case 16: return launch_gemv_mb<16, WPC, PREQ>(mb, p, gx, gy, smem, sms, st);
-    default: return launch_gemv_mb<32, WPC, PREQ>(mb, p, gx, gy, smem, sms, st);
+template <bool WIDE, bool PREQ>
+bitnet_status launch_gemv_mb(int mb, int rw, const GemvParams& p, int gy, size_t smem, int sms,
+                             cudaStream_t st) {
+  switch (mb) {
+    case 1: return launch_gemv_rw<1, WIDE, PREQ>(rw, p, gy, smem, sms, st);
+    case 2: return launch_gemv_rw<2, WIDE, PREQ>(rw, p, gy, smem, sms, st);
+    case 4: return launch_gemv_rw<4, WIDE, PREQ>(rw, p, gy, smem, sms, st);
+    case 8: return launch_gemv_rw<8, WIDE, PREQ>(rw, p, gy, smem, sms, st);
+    default: return launch_gemv_rw<16, WIDE, PREQ>(rw, p, gy, smem, sms, st);
   }
 }
 
 int bucket_of(int m) { return m <= 1 ? 1 : m <= 2 ? 2 : m <= 4 ? 4 : m <= 8 ? 8 : 16; }
 
 // Shared by the fused GEMV (PREQ = false, M <= 15) and the pre-quantised
-// SIMT fallback of bitnet_gemm (PREQ = true, any M, row chunks of MB).
-bitnet_status run_gemv(const GemvParams& p, bool preq, cudaStream_t st) {
+// SIMT path of bitnet_gemm (PREQ = true, any M, row chunks of MB).
+bitnet_status run_gemv(GemvParams p, bool preq, cudaStream_t st) {
   DeviceInfo* dev = nullptr;
   bitnet_status s = device_info(&dev);
   if (s != BITNET_OK) return s;
-  const int K = p.K, M = p.M;
-  int mb, gy;
-  size_t smem;
+  const int64_t K = p.K;
+  int mb, gy, qrows;
   if (!preq) {
-    mb = bucket_of(M);
+    mb = bucket_of(p.M);
     gy = 1;
-    smem = kGemvSmallBytes + static_cast<size_t>(M) * K;
+    qrows = p.M;
   } else {
-    mb = K <= 12288 ? 16 : K <= 24576 ? 8 : K <= 49152 ? 4 : K <= 98304 ? 2 : 1;
-    if (static_cast<int64_t>(mb) * K > kMaxGemvElems) return BITNET_ERR_SHAPE;
-    gy = (M + mb - 1) / mb;
-    smem = kGemvSmallBytes + static_cast<size_t>(mb) * K;
+    mb = 16;
+    while (mb > 1 && !gemv_fits(mb, K)) mb /= 2;
+    gy = (p.M + mb - 1) / mb;
+    qrows = mb;
     if (gy > 65535) return BITNET_ERR_SHAPE;
   }
+  if (!gemv_fits(qrows, K)) return BITNET_ERR_SHAPE;
+  // rows per warp per stage: a stage near 40 KB, enough row blocks to cover
+  // the SMs, and at most 32 accumulators per lane
+  const int64_t KB = K / 4;
+  int rw = pow2_floor(kGemvStageTarget / (8 * KB));
+  const int by_n = pow2_floor(p.N / (8 * static_cast<int64_t>(dev->sms)));
+  if (rw > by_n) rw = by_n;
+  if (rw > 32 / mb) rw = 32 / mb;
+  if (rw > 8) rw = 8;
+  if (rw < 1) rw = 1;
+  while (rw > 1 && !(gemv_smem(qrows, K, rw, 2) <= kSmemLimit)) rw /= 2;
+  const size_t stage = align128(static_cast<size_t>(8 * rw) * KB);
+  int stages = static_cast<int>(kGemvRingTarget / stage);
+  if (stages > kGemvMaxStages) stages = kGemvMaxStages;
+  if (stages < 2) stages = 2;
+  while (stages > 2 && gemv_smem(qrows, K, rw, stages) > kSmemLimit) --stages;
+  p.rows_per_block = 8 * rw;
+  p.stages = stages;
+  p.q_bytes = static_cast<uint32_t>(align128(static_cast<size_t>(qrows) * K));
+  p.stage_bytes = static_cast<uint32_t>(stage);
+  const size_t smem = gemv_smem(qrows, K, rw, stages);
   const bool wide = (K % 64) == 0;
-  const int chunks = wide ? K / 64 : K / 32;  // chunks per weight row
-  // lanes per row: the fewest that keep a lane at <= 8 chunks of a row
-  const int lanes = chunks <= 8 * 8 ? 8 : chunks <= 8 * 16 ? 16 : 32;
   if (wide)
-    return preq ? launch_gemv_l<4, true>(lanes, mb, p, gy, smem, dev->sms, st)
-                : launch_gemv_l<4, false>(lanes, mb, p, gy, smem, dev->sms, st);
-  return preq ? launch_gemv_l<2, true>(lanes, mb, p, gy, smem, dev->sms, st)
-              : launch_gemv_l<2, false>(lanes, mb, p, gy, smem, dev->sms, st);
+    return preq ? launch_gemv_mb<true, true>(mb, rw, p, gy, smem, dev->sms, st)
+                : launch_gemv_mb<true, false>(mb, rw, p, gy, smem, dev->sms, st);
+  return preq ? launch_gemv_mb<false, true>(mb, rw, p, gy, smem, dev->sms, st)
+              : launch_gemv_mb<false, false>(mb, rw, p, gy, smem, dev->sms, st);
 }
 
 // ---------------------------------------------------------------- GEMM
@@ -271,7 +309,7 @@ bitnet_status run_quantize(int8_t* xq, uint16_t* sa, const uint16_t* x, int64_t 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 bool linear_uses_gemv(int64_t M, int64_t K) {
-  return M >= 1 && M <= kLinearGemvMaxM && M * K <= kMaxGemvElems;
+  return M >= 1 && M <= kLinearGemvMaxM && K <= INT32_MAX && gemv_fits(static_cast<int>(M), K);
 }
 
 }  // namespace
@@ -367,7 +405,7 @@ static bitnet_status gemv_common(GemvParams& p, const void* x, bitnet_dtype dt,
   if (dt != BITNET_BF16) return BITNET_ERR_DTYPE;
   bitnet_status s = check_compute_shape(M, N, K);
   if (s != BITNET_OK) return s;
-  if (M < 1 || M > kGemvMaxM || M * K > kMaxGemvElems) return BITNET_ERR_SHAPE;
+  if (M < 1 || M > kGemvMaxM || !gemv_fits(static_cast<int>(M), K)) return BITNET_ERR_SHAPE;
   if (x == nullptr || w_packed == nullptr) return BITNET_ERR_NULL;
   if (!aligned(x, 16) || !aligned(w_packed, 16)) return BITNET_ERR_ALIGN;
   p.x = static_cast<const uint16_t*>(x);

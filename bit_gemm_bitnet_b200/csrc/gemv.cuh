@@ -1,33 +1,37 @@
 // Decode GEMV with fused per-token quantisation (M < 16), and the same kernel
-// reading pre-quantised rows (a SIMT fallback for shapes the tensor-core GEMM
-// does not take).
+// reading pre-quantised rows (the SIMT path of bitnet_gemm for shapes the
+// tensor-core GEMM does not take).
 //
-// The work is bound by streaming the packed weights from HBM once. Layout:
-//   * L lanes (8, 16 or 32, chosen so that a lane holds at most 8 chunks of a
-//     row) share one weight row; 8 warps per CTA; CTAs are persistent (as
-//     many as fit at once) and stride over the rows.
-//   * a lane issues all loads of its part of a row at once (16-byte streaming
-//     loads, 64 weights each), and the next row's loads before using the
-//     current one; the first row is requested before waiting on the previous
-//     kernel in the stream (programmatic dependent launch), so small layers
-//     have their weights in flight while the activations are quantised.
-//   * the quantised activations live in shared memory with every 16-element
-//     group transposed 4x4, so that the four 2-bit planes of a packed word,
-//     (w >> 2i) & 0x03030303, line up with one activation word each and feed
-//     dp4a without any byte shuffling. The codes are used as unsigned values
-//     c = w + 2, and sum_k q*w = sum_k q*c - 2 * sum_k q is corrected per row.
-//   * partial sums are reduced over the 8 lanes with warp shuffles, and the
-//     fp32 scale epilogue writes bf16.
+// The work is bound by streaming the packed weights from HBM once:
+//   * a producer warp streams blocks of consecutive weight rows (contiguous
+//     in memory) into a ring of shared-memory stages with bulk async copies
+//     (cp.async.bulk, completion counted on an mbarrier per stage). The first
+//     stages are requested before waiting on the previous kernel of the
+//     stream (programmatic dependent launch), so a small layer's weights are
+//     in flight while its activations are being quantised;
+//   * eight consumer warps quantise the activation rows into shared memory
+//     once per CTA, with every 16-element group transposed 4x4 so that the
+//     four 2-bit planes of a packed word, (w >> 2i) & 0x03030303, line up
+//     with one activation word each and feed dp4a directly. The codes are
+//     used as unsigned c = w + 2 and sum q*w = sum q*c - 2 * sum q;
+//   * in a stage, warp w owns RW rows; lane l owns the 32-bit weight words
+//     l, l + 32, ... of every row (16 weights each), so each activation word
+//     it loads serves RW rows. Row sums are reduced with warp shuffles and
+//     the fp32 scale epilogue writes bf16;
+//   * CTAs are persistent (as many as fit) and walk the row blocks; loops
+//     are kept rolled so the code a launch has to fetch stays small.
 #pragma once
 #include "common.cuh"
 #include "pack_quant.cuh"
 
 namespace bitnet {
 
-constexpr int kGemvThreads = 256;
-constexpr int kGemvWarps = kGemvThreads / 32;
-constexpr int kGemvCPL = 8;           // chunks per lane loaded at once
-constexpr int kGemvSmallBytes = 1024;  // per-row scalars before the q rows
+constexpr int kGemvConsumerWarps = 8;
+constexpr int kGemvThreads = (kGemvConsumerWarps + 1) * 32;  // + producer warp
+constexpr int kGemvMaxStages = 8;
+constexpr int kGemvHeaderBytes = 1024;
+constexpr int kGemvStageTarget = 40 * 1024;  // bytes per stage (aim)
+constexpr int kGemvRingTarget = 160 * 1024;  // bytes of stages per CTA (aim)
 
 struct GemvParams {
   uint16_t* out;          // bf16 [M, N], or
@@ -39,6 +43,10 @@ struct GemvParams {
   const float* sw;
   int sw_len;
   int M, N, K;
+  int rows_per_block;     // 8 * RW
+  int stages;             // ring depth (<= kGemvMaxStages)
+  uint32_t q_bytes;       // shared bytes reserved for the quantised rows
+  uint32_t stage_bytes;   // shared bytes per stage (>= rows_per_block * K/4)
   int8_t* dbg_q;          // optional: codes quantised on chip (block 0)
   uint16_t* dbg_sa;       // optional: their scales (block 0)
 };
@@ -57,71 +65,78 @@ __device__ __forceinline__ int bytesum_s8(uint32_t w) {
   return __dp4a(static_cast<int>(w), 0x01010101, 0);
 }
 
-// Load the chunks lane `sub` owns in piece `pc` of weight row `n`:
-// chunk c = pc * L * CPL + sub + L * i (i < CPL), zero past the row or N.
-template <int L, int WPC>
-__device__ __forceinline__ void gemv_load_row(uint32_t (&wb)[kGemvCPL][WPC],
-                                              const uint8_t* __restrict__ wp, int n,
-                                              int pc, int sub, int N, int R, int KB) {
-  const int c0 = pc * L * kGemvCPL + sub;
-#pragma unroll
-  for (int i = 0; i < kGemvCPL; ++i) {
-    const int c = c0 + L * i;
-    if (n < N && c < R) {
-      const uint8_t* ptr = wp + static_cast<int64_t>(n) * KB + c * (4 * WPC);
-      if constexpr (WPC == 4) {
-        const uint4 v = ldg_stream_v4(ptr);
-        wb[i][0] = v.x; wb[i][1] = v.y; wb[i][2] = v.z; wb[i][3] = v.w;
-      } else {
-        const uint2 v = ldg_stream_v2(ptr);
-        wb[i][0] = v.x; wb[i][1] = v.y;
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < WPC; ++j) wb[i][j] = 0u;
-    }
-  }
-}
-
-// MB: rows of x per CTA (bucket); L: lanes per weight row (8, 16 or 32);
-// WPC: 32-bit words per chunk (4: 16-byte chunks, needs K % 64 == 0; 2: 8-byte
-// chunks); PREQ: activations come pre-quantised (x_q + scale_act).
-template <int MB, int L, int WPC, bool PREQ>
+// MB: rows of x per CTA (bucket); RW: weight rows per consumer warp per stage;
+// WIDE: K % 64 == 0 (rows 16-byte aligned: one bulk copy per stage),
+// otherwise the producer lanes copy the stage in 8-byte pieces;
+// PREQ: activations come pre-quantised (x_q + scale_act).
+template <int MB, int RW, bool WIDE, bool PREQ>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
-  extern __shared__ __align__(16) uint8_t smem[];
+  extern __shared__ __align__(128) uint8_t smem[];
   int* qsum = reinterpret_cast<int*>(smem);                  // [MB]
   float* saf = reinterpret_cast<float*>(smem + 64);          // [MB]
-  uint32_t* red = reinterpret_cast<uint32_t*>(smem + 128);   // [warps][MB]
-  uint8_t* qs = smem + kGemvSmallBytes;                      // [Mc][K]
-  static_assert(kGemvWarps * MB * 4 <= kGemvSmallBytes - 128, "reduction scratch");
+  uint32_t* red = reinterpret_cast<uint32_t*>(smem + 128);   // [8][MB]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 768);  // full[8], empty[8]
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + 1016);
+  uint8_t* qs = smem + kGemvHeaderBytes;                     // [Mc][K]
+  uint8_t* ring = qs + p.q_bytes;
+  static_assert(kGemvConsumerWarps * MB * 4 <= 640, "reduction scratch");
 
-  pdl_launch_dependents();
-
-  constexpr int G = 32 / L;                  // weight rows per warp at a time
-  constexpr int GPC = kGemvWarps * G;        // weight rows per CTA at a time
   const int K = p.K, N = p.N;
+  const int KB = K / 4;
+  const int words = K / 16;  // 32-bit packed words per row
+  const int RPB = p.rows_per_block;
+  const int S = p.stages;
+  const int nblocks = (N + RPB - 1) / RPB;
   const int m_base = PREQ ? static_cast<int>(blockIdx.y) * MB : 0;
   const int Mc = PREQ ? min(MB, p.M - m_base) : p.M;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int sub = lane % L;
-  const int KB = K / 4;
-  const int R = K / (16 * WPC);                            // chunks per row
-  const int pieces = (R + L * kGemvCPL - 1) / (L * kGemvCPL);
-  const int stride = gridDim.x * GPC;
-  // n: this group's row; wrow: the warp's first row, which drives the loop so
-  // that all 32 lanes take the same trip count.
-  int n = static_cast<int>(blockIdx.x) * GPC + warp * G + lane / L;
-  int wrow = static_cast<int>(blockIdx.x) * GPC + warp * G;
-  int pc = 0;
+  auto full = [&](int s) { return smem_u32(bars + s); };
+  auto empty = [&](int s) { return smem_u32(bars + kGemvMaxStages + s); };
 
-  // The first row's weights are requested before waiting for the kernel
-  // that produces the activations.
-  uint32_t cur[kGemvCPL][WPC];
-  gemv_load_row<L, WPC>(cur, p.wp, n, 0, sub, N, R, KB);
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full(s), WIDE ? 1u : 32u);
+      mbar_init(empty(s), kGemvConsumerWarps);
+    }
+    *abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_launch_dependents();
 
-  pdl_wait();
+  if (warp == kGemvConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    // Weights do not depend on the previous kernel: no griddepcontrol.wait.
+    uint32_t it = 0;
+    for (int b = blockIdx.x; b < nblocks; b += gridDim.x, ++it) {
+      const int s = it % S;
+      const uint32_t ph = (it / S) & 1u;
+      if (!mbar_wait(empty(s), ph ^ 1u, abort)) break;
+      const int n0 = b * RPB;
+      const int rows = min(RPB, N - n0);
+      const uint8_t* src = p.wp + static_cast<int64_t>(n0) * KB;
+      uint8_t* dst = ring + static_cast<size_t>(s) * p.stage_bytes;
+      if constexpr (WIDE) {
+        if (lane == 0) {
+          const uint32_t bytes = static_cast<uint32_t>(rows) * KB;
+          mbar_arrive_expect_tx(full(s), bytes);
+          bulk_load(smem_u32(dst), src, bytes, full(s));
+        }
+      } else {
+        const int pieces = rows * (KB / 8);
+        for (int i = lane; i < pieces; i += 32) cp_async_8(smem_u32(dst + 8 * i), src + 8 * i);
+        cp_async_arrive_noinc(full(s));
+      }
+    }
+    // drain: every copy issued has landed before the CTA may exit
+    const uint32_t first = it > static_cast<uint32_t>(S) ? it - S : 0u;
+    for (uint32_t j = first; j < it; ++j) mbar_wait_drain(full(j % S), (j / S) & 1u);
+    return;
+  }
 
-  // ---- stage the quantised activations (transposed groups) in smem -------
+  // -------------------------------------------------------------- consumers
+  pdl_wait();  // the activations may come from the previous kernel
+  constexpr uint32_t kConsumers = kGemvConsumerWarps * 32;
   const int groups16 = K / 16;
   if constexpr (!PREQ) {
     uint32_t mb[MB];
@@ -130,19 +145,19 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
       mb[m] = 0;
       if (m < Mc) {
         const uint4* row = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m) * K);
-        for (int v = tid; v < K / 8; v += kGemvThreads)
-          mb[m] = max(mb[m], absmax_bits8(__ldg(row + v)));
+#pragma unroll 1
+        for (int v = tid; v < K / 8; v += kConsumers) mb[m] = max(mb[m], absmax_bits8(__ldg(row + v)));
       }
       mb[m] = __reduce_max_sync(0xFFFFFFFFu, mb[m]);
       if (lane == 0) red[warp * MB + m] = mb[m];
     }
-    __syncthreads();
+    named_barrier_sync(1, kConsumers);
     RowQuant rq[MB];
 #pragma unroll
     for (int m = 0; m < MB; ++m) {
       uint32_t t = 0;
 #pragma unroll
-      for (int w = 0; w < kGemvWarps; ++w) t = max(t, red[w * MB + m]);
+      for (int w = 0; w < kGemvConsumerWarps; ++w) t = max(t, red[w * MB + m]);
       rq[m] = row_quant(bf16_bits_to_f32(t));
     }
     int qs_part[MB];
@@ -151,33 +166,32 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
       qs_part[m] = 0;
       if (m < Mc) {
         const uint4* row = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m) * K);
-        for (int g = tid; g < groups16; g += kGemvThreads) {
+#pragma unroll 1
+        for (int g = tid; g < groups16; g += kConsumers) {
           const uint2 lo = quant8(__ldg(row + 2 * g), rq[m]);
           const uint2 hi = quant8(__ldg(row + 2 * g + 1), rq[m]);
           const uint4 nat = make_uint4(lo.x, lo.y, hi.x, hi.y);
-          qs_part[m] += bytesum_s8(nat.x) + bytesum_s8(nat.y) +
-                        bytesum_s8(nat.z) + bytesum_s8(nat.w);
-          *reinterpret_cast<uint4*>(qs + static_cast<int64_t>(m) * K + 16 * g) =
-              transpose16(nat);
+          qs_part[m] += bytesum_s8(nat.x) + bytesum_s8(nat.y) + bytesum_s8(nat.z) +
+                        bytesum_s8(nat.w);
+          *reinterpret_cast<uint4*>(qs + static_cast<int64_t>(m) * K + 16 * g) = transpose16(nat);
           if (p.dbg_q != nullptr && blockIdx.x == 0)
             *reinterpret_cast<uint4*>(p.dbg_q + static_cast<int64_t>(m) * K + 16 * g) = nat;
         }
       }
     }
-    __syncthreads();  // red[] reuse
+    named_barrier_sync(1, kConsumers);  // red[] reuse
 #pragma unroll
     for (int m = 0; m < MB; ++m) {
       const int s = __reduce_add_sync(0xFFFFFFFFu, qs_part[m]);
       if (lane == 0) red[warp * MB + m] = static_cast<uint32_t>(s);
     }
-    __syncthreads();
+    named_barrier_sync(1, kConsumers);
     if (tid < MB) {
       int s = 0;
-      for (int w = 0; w < kGemvWarps; ++w) s += static_cast<int>(red[w * MB + tid]);
+      for (int w = 0; w < kGemvConsumerWarps; ++w) s += static_cast<int>(red[w * MB + tid]);
       qsum[tid] = s;
     }
-    // every thread holds the same rq[]; thread 0 publishes the scales
-    if (tid == 0) {
+    if (tid == 0) {  // every thread holds the same rq[]
 #pragma unroll
       for (int m = 0; m < MB; ++m) {
         const uint16_t sb = f32_to_bf16_bits(rq[m].s);
@@ -191,86 +205,90 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
     for (int m = 0; m < MB; ++m) {
       qs_part[m] = 0;
       if (m < Mc) {
-        const uint4* row = reinterpret_cast<const uint4*>(
-            p.xq + static_cast<int64_t>(m_base + m) * K);
-        for (int g = tid; g < groups16; g += kGemvThreads) {
+        const uint4* row = reinterpret_cast<const uint4*>(p.xq + static_cast<int64_t>(m_base + m) * K);
+#pragma unroll 1
+        for (int g = tid; g < groups16; g += kConsumers) {
           const uint4 nat = __ldg(row + g);
-          qs_part[m] += bytesum_s8(nat.x) + bytesum_s8(nat.y) +
-                        bytesum_s8(nat.z) + bytesum_s8(nat.w);
-          *reinterpret_cast<uint4*>(qs + static_cast<int64_t>(m) * K + 16 * g) =
-              transpose16(nat);
+          qs_part[m] += bytesum_s8(nat.x) + bytesum_s8(nat.y) + bytesum_s8(nat.z) +
+                        bytesum_s8(nat.w);
+          *reinterpret_cast<uint4*>(qs + static_cast<int64_t>(m) * K + 16 * g) = transpose16(nat);
         }
       }
       const int s = __reduce_add_sync(0xFFFFFFFFu, qs_part[m]);
       if (lane == 0) red[warp * MB + m] = static_cast<uint32_t>(s);
     }
-    __syncthreads();
+    named_barrier_sync(1, kConsumers);
     if (tid < MB) {
       int s = 0;
-      for (int w = 0; w < kGemvWarps; ++w) s += static_cast<int>(red[w * MB + tid]);
+      for (int w = 0; w < kGemvConsumerWarps; ++w) s += static_cast<int>(red[w * MB + tid]);
       qsum[tid] = s;
       // the int32 test hook passes no scales
       saf[tid] = (tid < Mc && p.sa_in != nullptr) ? bf16_bits_to_f32(p.sa_in[m_base + tid]) : 0.0f;
     }
   }
-  __syncthreads();
+  named_barrier_sync(1, kConsumers);
 
-  // ---- stream the weights ------------------------------------------------
-  int acc[MB];
-#pragma unroll
-  for (int m = 0; m < MB; ++m) acc[m] = 0;
+  uint32_t it = 0;
+  for (int b = blockIdx.x; b < nblocks; b += gridDim.x, ++it) {
+    const int s = it % S;
+    const uint32_t ph = (it / S) & 1u;
+    if (!mbar_wait(full(s), ph, abort)) break;
+    const uint8_t* stage = ring + static_cast<size_t>(s) * p.stage_bytes;
+    const int r0 = warp * RW;  // this warp's first row in the block
+    const int n0 = b * RPB + r0;
+    int rows = min(RW, N - n0);
+    if (rows < 0) rows = 0;
 
-  // One unit = one piece of one row. `use` holds the current unit; the next
-  // unit's loads go into `fill` before `use` is consumed. The two buffers
-  // alternate (no register copies, which would wait on the loads in flight).
-  uint32_t other[kGemvCPL][WPC];
-  auto step = [&](uint32_t (&use)[kGemvCPL][WPC], uint32_t (&fill)[kGemvCPL][WPC]) -> bool {
-    int pn = pc + 1, nn = n, wn = wrow;
-    const bool row_done = pn == pieces;  // warp-uniform
-    if (row_done) {
-      pn = 0;
-      nn = n + stride;
-      wn = wrow + stride;
-    }
-    if (wn < N) gemv_load_row<L, WPC>(fill, p.wp, nn, pn, sub, N, R, KB);
+    int acc[RW][MB];
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+#pragma unroll
+      for (int m = 0; m < MB; ++m) acc[r][m] = 0;
 
-    const int c0 = pc * L * kGemvCPL + sub;
+    if (rows > 0) {
+      const uint32_t* wrow = reinterpret_cast<const uint32_t*>(stage + static_cast<size_t>(r0) * KB);
+#pragma unroll 1
+      for (int t = lane; t < words; t += 32) {
+        uint4 Q[MB];
 #pragma unroll
-    for (int i = 0; i < kGemvCPL; ++i) {
-      const int c = c0 + L * i;
-      if (c < R) {
+        for (int m = 0; m < MB; ++m)
+          if (m < Mc) Q[m] = *reinterpret_cast<const uint4*>(qs + static_cast<int64_t>(m) * K + 16 * t);
 #pragma unroll
-        for (int j = 0; j < WPC; ++j) {
-          const int g = c * WPC + j;
-          const uint32_t w = use[i][j];
-          const uint32_t e0 = w & 0x03030303u;
-          const uint32_t e1 = (w >> 2) & 0x03030303u;
-          const uint32_t e2 = (w >> 4) & 0x03030303u;
-          const uint32_t e3 = (w >> 6) & 0x03030303u;
+        for (int r = 0; r < RW; ++r) {
+          if (r < rows) {
+            const uint32_t w = wrow[r * (KB / 4) + t];
+            const uint32_t e0 = w & 0x03030303u;
+            const uint32_t e1 = (w >> 2) & 0x03030303u;
+            const uint32_t e2 = (w >> 4) & 0x03030303u;
+            const uint32_t e3 = (w >> 6) & 0x03030303u;
 #pragma unroll
-          for (int m = 0; m < MB; ++m) {
-            if (m < Mc) {
-              const uint4 Q = *reinterpret_cast<const uint4*>(qs + static_cast<int64_t>(m) * K + 16 * g);
-              int a = acc[m];
-              a = dp4a_s32(e0, Q.x, a);
-              a = dp4a_s32(e1, Q.y, a);
-              a = dp4a_s32(e2, Q.z, a);
-              a = dp4a_s32(e3, Q.w, a);
-              acc[m] = a;
+            for (int m = 0; m < MB; ++m) {
+              if (m < Mc) {
+                int a = acc[r][m];
+                a = dp4a_s32(e0, Q[m].x, a);
+                a = dp4a_s32(e1, Q[m].y, a);
+                a = dp4a_s32(e2, Q[m].z, a);
+                a = dp4a_s32(e3, Q[m].w, a);
+                acc[r][m] = a;
+              }
             }
           }
         }
       }
     }
+    // the stage's shared memory may be refilled once every warp is done
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty(s));
 
-    if (row_done) {
+#pragma unroll
+    for (int r = 0; r < RW; ++r) {
 #pragma unroll
       for (int m = 0; m < MB; ++m) {
-        int v = acc[m];
+        int v = acc[r][m];
 #pragma unroll
-        for (int o = 1; o < L; o <<= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-        acc[m] = 0;
-        if ((m % L) == sub && m < Mc && n < N) {
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        if (((r * MB + m) & 31) == lane && r < rows && m < Mc) {
+          const int n = n0 + r;
           const int a = v - 2 * qsum[m];
           const int64_t o = static_cast<int64_t>(m_base + m) * N + n;
           if (p.acc_out != nullptr) {
@@ -282,15 +300,6 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
           }
         }
       }
-    }
-    n = nn;
-    wrow = wn;
-    pc = pn;
-    return wrow < N;
-  };
-
-  if (wrow < N) {
-    while (step(cur, other) && step(other, cur)) {
     }
   }
 }
