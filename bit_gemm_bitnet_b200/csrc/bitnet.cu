@@ -124,12 +124,13 @@ constexpr size_t kSmemLimit = 232448;  // per-CTA opt-in maximum on sm_100
 // of `stages` stages of `rw` rows per warp.
 size_t gemv_smem(int rows, int64_t K, int rw, int stages) {
   return kGemvHeaderBytes + align128(static_cast<size_t>(rows) * K) +
-         static_cast<size_t>(stages) * align128(static_cast<size_t>(8 * rw) * (K / 4));
+         static_cast<size_t>(stages) *
+             align128(static_cast<size_t>(kGemvConsumerWarps * rw) * (K / 4));
 }
 
-// Does the GEMV fit `rows` activation rows of length K (two stages of one
+// Does the GEMV fit `rows` activation rows of length K (one stage of one
 // row per warp at least)?
-bool gemv_fits(int rows, int64_t K) { return gemv_smem(rows, K, 1, 2) <= kSmemLimit; }
+bool gemv_fits(int rows, int64_t K) { return gemv_smem(rows, K, 1, 1) <= kSmemLimit; }
 
 int pow2_floor(int64_t v) {
   int r = 1;
@@ -164,10 +165,10 @@ bitnet_status launch_gemv_rw(int rw, const GemvParams& p, int gy, size_t smem, i
     case 1: return launch_gemv_t<MB, 1, WIDE, PREQ>(p, gy, smem, sms, st);
     case 2: return launch_gemv_t<MB, 2, WIDE, PREQ>(p, gy, smem, sms, st);
     case 4:
-      if constexpr (MB <= 8) return launch_gemv_t<MB, 4, WIDE, PREQ>(p, gy, smem, sms, st);
+      if constexpr (MB != 2 && MB <= 8) return launch_gemv_t<MB, 4, WIDE, PREQ>(p, gy, smem, sms, st);
       return BITNET_ERR_SHAPE;
     default:
-      if constexpr (MB <= 4) return launch_gemv_t<MB, 8, WIDE, PREQ>(p, gy, smem, sms, st);
+      if constexpr (MB == 1 || MB == 4) return launch_gemv_t<MB, 8, WIDE, PREQ>(p, gy, smem, sms, st);
       return BITNET_ERR_SHAPE;
   }
 }
@@ -207,21 +208,27 @@ bitnet_status run_gemv(GemvParams p, bool preq, cudaStream_t st) {
   }
   if (!gemv_fits(qrows, K)) return BITNET_ERR_SHAPE;
   // rows per warp per stage: a stage near 40 KB, enough row blocks to cover
-  // the SMs, and at most 32 accumulators per lane
+  // the SMs, and at most 32 accumulator registers per lane
   const int64_t KB = K / 4;
-  int rw = pow2_floor(kGemvStageTarget / (8 * KB));
-  const int by_n = pow2_floor(p.N / (8 * static_cast<int64_t>(dev->sms)));
+  const int warps = kGemvConsumerWarps;
+  int rw = pow2_floor(kGemvStageTarget / (warps * KB));
+  const int by_n = pow2_floor(p.N / (static_cast<int64_t>(warps) * dev->sms));
   if (rw > by_n) rw = by_n;
-  if (rw > 32 / mb) rw = 32 / mb;
+  const int acc_per_row = mb * (mb <= 2 ? 4 : 1);
+  while (rw > 1 && rw * acc_per_row > 32) rw /= 2;
   if (rw > 8) rw = 8;
   if (rw < 1) rw = 1;
-  while (rw > 1 && !(gemv_smem(qrows, K, rw, 2) <= kSmemLimit)) rw /= 2;
-  const size_t stage = align128(static_cast<size_t>(8 * rw) * KB);
+  while (rw > 1 && gemv_smem(qrows, K, rw, 1) > kSmemLimit) rw /= 2;
+  const size_t stage = align128(static_cast<size_t>(warps * rw) * KB);
+  // ring depth: no deeper than the row blocks one CTA will see
+  const int64_t nblocks = (p.N + warps * rw - 1) / (warps * rw);
+  const int64_t per_cta = (nblocks + dev->sms - 1) / dev->sms;
   int stages = static_cast<int>(kGemvRingTarget / stage);
+  if (stages > per_cta) stages = static_cast<int>(per_cta);
   if (stages > kGemvMaxStages) stages = kGemvMaxStages;
-  if (stages < 2) stages = 2;
-  while (stages > 2 && gemv_smem(qrows, K, rw, stages) > kSmemLimit) --stages;
-  p.rows_per_block = 8 * rw;
+  if (stages < 1) stages = 1;
+  while (stages > 1 && gemv_smem(qrows, K, rw, stages) > kSmemLimit) --stages;
+  p.rows_per_block = warps * rw;
   p.stages = stages;
   p.q_bytes = static_cast<uint32_t>(align128(static_cast<size_t>(qrows) * K));
   p.stage_bytes = static_cast<uint32_t>(stage);

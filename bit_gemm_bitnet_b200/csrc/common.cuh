@@ -103,6 +103,12 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 __device__ __forceinline__ int dp4a_s32(uint32_t a, uint32_t b, int c) {
   return __dp4a(static_cast<int>(a), static_cast<int>(b), c);
 }
+// dp4a with unsigned bytes in `a` and signed bytes in `b`.
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
 
 // ------------------------------------------------------- shared / mbarrier
 

@@ -9,15 +9,18 @@
 //     stages are requested before waiting on the previous kernel of the
 //     stream (programmatic dependent launch), so a small layer's weights are
 //     in flight while its activations are being quantised;
-//   * eight consumer warps quantise the activation rows into shared memory
+//   * sixteen consumer warps quantise the activation rows into shared memory
 //     once per CTA, with every 16-element group transposed 4x4 so that the
 //     four 2-bit planes of a packed word, (w >> 2i) & 0x03030303, line up
 //     with one activation word each and feed dp4a directly. The codes are
 //     used as unsigned c = w + 2 and sum q*w = sum q*c - 2 * sum q;
 //   * in a stage, warp w owns RW rows; lane l owns the 32-bit weight words
 //     l, l + 32, ... of every row (16 weights each), so each activation word
-//     it loads serves RW rows. Row sums are reduced with warp shuffles and
-//     the fp32 scale epilogue writes bf16;
+//     it loads serves RW rows. For one or two activation rows the planes are
+//     masked in place, c_i * 4^i = w & (3 << 2i), into four accumulators
+//     whose sums are exact multiples of 4^i (recombined with arithmetic
+//     shifts): one AND and one dp4a per plane. Row sums are reduced with warp
+//     shuffles and the fp32 scale epilogue writes bf16;
 //   * CTAs are persistent (as many as fit) and walk the row blocks; loops
 //     are kept rolled so the code a launch has to fetch stays small.
 #pragma once
@@ -26,10 +29,11 @@
 
 namespace bitnet {
 
-constexpr int kGemvConsumerWarps = 8;
-constexpr int kGemvThreads = (kGemvConsumerWarps + 1) * 32;  // + producer warp
+constexpr int kGemvConsumerWarps = 16;
+constexpr int kGemvConsumers = kGemvConsumerWarps * 32;
+constexpr int kGemvThreads = kGemvConsumers + 32;  // + producer warp
 constexpr int kGemvMaxStages = 8;
-constexpr int kGemvHeaderBytes = 1024;
+constexpr int kGemvHeaderBytes = 2048;
 constexpr int kGemvStageTarget = 40 * 1024;  // bytes per stage (aim)
 constexpr int kGemvRingTarget = 160 * 1024;  // bytes of stages per CTA (aim)
 
@@ -43,7 +47,7 @@ struct GemvParams {
   const float* sw;
   int sw_len;
   int M, N, K;
-  int rows_per_block;     // 8 * RW
+  int rows_per_block;     // 16 * RW
   int stages;             // ring depth (<= kGemvMaxStages)
   uint32_t q_bytes;       // shared bytes reserved for the quantised rows
   uint32_t stage_bytes;   // shared bytes per stage (>= rows_per_block * K/4)
@@ -65,6 +69,72 @@ __device__ __forceinline__ int bytesum_s8(uint32_t w) {
   return __dp4a(static_cast<int>(w), 0x01010101, 0);
 }
 
+__device__ __forceinline__ uint32_t absmax_bits16(const uint4& a, const uint4& b) {
+  return max(absmax_bits8(a), absmax_bits8(b));
+}
+
+// Partial dot products of one warp's RW rows of a stage with the quantised
+// activation rows, for lane `lane` (words lane, lane + 32, ...).
+// PLANES: four plane accumulators per (row, activation row); else one.
+template <int MB, int RW, bool PLANES, bool FULL>
+__device__ __forceinline__ void gemv_rows(int (&acc)[RW][MB][PLANES ? 4 : 1],
+                                          const uint32_t* __restrict__ wrow, int words,
+                                          const uint8_t* __restrict__ qs, int K, int Mc,
+                                          int rows, int lane) {
+#pragma unroll 1
+  for (int t = lane; t < words; t += 32) {
+    if constexpr (PLANES) {
+      uint4 Q[MB];
+#pragma unroll
+      for (int m = 0; m < MB; ++m)
+        if (MB == 1 || m < Mc) Q[m] = *reinterpret_cast<const uint4*>(qs + m * K + 16 * t);
+#pragma unroll
+      for (int r = 0; r < RW; ++r) {
+        if (FULL || r < rows) {
+          const uint32_t w = wrow[r * words + t];
+          const uint32_t p0 = w & 0x03030303u, p1 = w & 0x0C0C0C0Cu;
+          const uint32_t p2 = w & 0x30303030u, p3 = w & 0xC0C0C0C0u;
+#pragma unroll
+          for (int m = 0; m < MB; ++m) {
+            if (MB == 1 || m < Mc) {
+              acc[r][m][0] = dp4a_s32(p0, Q[m].x, acc[r][m][0]);
+              acc[r][m][1] = dp4a_s32(p1, Q[m].y, acc[r][m][1]);
+              acc[r][m][2] = dp4a_s32(p2, Q[m].z, acc[r][m][2]);
+              acc[r][m][3] = dp4a_us(p3, Q[m].w, acc[r][m][3]);
+            }
+          }
+        }
+      }
+    } else {
+      // planes of the warp's rows first, then one activation word at a time
+      uint32_t e[RW][4];
+#pragma unroll
+      for (int r = 0; r < RW; ++r) {
+        const uint32_t w = (FULL || r < rows) ? wrow[r * words + t] : 0u;
+        e[r][0] = w & 0x03030303u;
+        e[r][1] = (w >> 2) & 0x03030303u;
+        e[r][2] = (w >> 4) & 0x03030303u;
+        e[r][3] = (w >> 6) & 0x03030303u;
+      }
+#pragma unroll
+      for (int m = 0; m < MB; ++m) {
+        if (m < Mc) {
+          const uint4 Q = *reinterpret_cast<const uint4*>(qs + m * K + 16 * t);
+#pragma unroll
+          for (int r = 0; r < RW; ++r) {
+            int a = acc[r][m][0];
+            a = dp4a_s32(e[r][0], Q.x, a);
+            a = dp4a_s32(e[r][1], Q.y, a);
+            a = dp4a_s32(e[r][2], Q.z, a);
+            a = dp4a_s32(e[r][3], Q.w, a);
+            acc[r][m][0] = a;
+          }
+        }
+      }
+    }
+  }
+}
+
 // MB: rows of x per CTA (bucket); RW: weight rows per consumer warp per stage;
 // WIDE: K % 64 == 0 (rows 16-byte aligned: one bulk copy per stage),
 // otherwise the producer lanes copy the stage in 8-byte pieces;
@@ -74,12 +144,16 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   int* qsum = reinterpret_cast<int*>(smem);                  // [MB]
   float* saf = reinterpret_cast<float*>(smem + 64);          // [MB]
-  uint32_t* red = reinterpret_cast<uint32_t*>(smem + 128);   // [8][MB]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 768);  // full[8], empty[8]
-  volatile int* abort = reinterpret_cast<volatile int*>(smem + 1016);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 128);  // full[8], empty[8]
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + 256);
+  float* rq_s = reinterpret_cast<float*>(smem + 320);        // [MB]
+  float* rq_r = reinterpret_cast<float*>(smem + 384);        // [MB]
+  uint32_t* red = reinterpret_cast<uint32_t*>(smem + 512);   // [16 warps][MB]
   uint8_t* qs = smem + kGemvHeaderBytes;                     // [Mc][K]
   uint8_t* ring = qs + p.q_bytes;
-  static_assert(kGemvConsumerWarps * MB * 4 <= 640, "reduction scratch");
+  static_assert(kGemvConsumerWarps * MB * 4 <= kGemvHeaderBytes - 512, "reduction scratch");
+  constexpr bool PLANES = MB <= 2;
+  constexpr bool HOLD = MB <= 2;  // keep the activation row in registers
 
   const int K = p.K, N = p.N;
   const int KB = K / 4;
@@ -88,7 +162,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
   const int S = p.stages;
   const int nblocks = (N + RPB - 1) / RPB;
   const int m_base = PREQ ? static_cast<int>(blockIdx.y) * MB : 0;
-  const int Mc = PREQ ? min(MB, p.M - m_base) : p.M;
+  const int Mc = PREQ ? min(MB, p.M - m_base) : (MB == 1 ? 1 : p.M);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   auto full = [&](int s) { return smem_u32(bars + s); };
   auto empty = [&](int s) { return smem_u32(bars + kGemvMaxStages + s); };
@@ -136,68 +210,89 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
 
   // -------------------------------------------------------------- consumers
   pdl_wait();  // the activations may come from the previous kernel
-  constexpr uint32_t kConsumers = kGemvConsumerWarps * 32;
   const int groups16 = K / 16;
   if constexpr (!PREQ) {
+    // absmax of every activation row (each thread owns 16-element groups
+    // tid, tid + 512, ...; with HOLD the first two stay in registers)
+    uint4 hv[HOLD ? MB : 1][2][2];
     uint32_t mb[MB];
 #pragma unroll
     for (int m = 0; m < MB; ++m) {
       mb[m] = 0;
-      if (m < Mc) {
+      if (MB == 1 || m < Mc) {
         const uint4* row = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m) * K);
+        if constexpr (HOLD) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int g = tid + j * kGemvConsumers;
+            if (g < groups16) {
+              hv[m][j][0] = __ldg(row + 2 * g);
+              hv[m][j][1] = __ldg(row + 2 * g + 1);
+              mb[m] = max(mb[m], absmax_bits16(hv[m][j][0], hv[m][j][1]));
+            }
+          }
+        }
 #pragma unroll 1
-        for (int v = tid; v < K / 8; v += kConsumers) mb[m] = max(mb[m], absmax_bits8(__ldg(row + v)));
+        for (int g = tid + (HOLD ? 2 : 0) * kGemvConsumers; g < groups16; g += kGemvConsumers)
+          mb[m] = max(mb[m], absmax_bits16(__ldg(row + 2 * g), __ldg(row + 2 * g + 1)));
       }
       mb[m] = __reduce_max_sync(0xFFFFFFFFu, mb[m]);
       if (lane == 0) red[warp * MB + m] = mb[m];
     }
-    named_barrier_sync(1, kConsumers);
-    RowQuant rq[MB];
-#pragma unroll
-    for (int m = 0; m < MB; ++m) {
+    named_barrier_sync(1, kGemvConsumers);
+    if (tid < MB) {  // one thread per activation row: its quantiser and scale
       uint32_t t = 0;
-#pragma unroll
-      for (int w = 0; w < kGemvConsumerWarps; ++w) t = max(t, red[w * MB + m]);
-      rq[m] = row_quant(bf16_bits_to_f32(t));
+      for (int w = 0; w < kGemvConsumerWarps; ++w) t = max(t, red[w * MB + tid]);
+      const RowQuant q = row_quant(bf16_bits_to_f32(t));
+      rq_s[tid] = q.s;
+      rq_r[tid] = q.r;
+      const uint16_t sb = f32_to_bf16_bits(q.s);
+      saf[tid] = bf16_bits_to_f32(sb);
+      if (p.dbg_sa != nullptr && blockIdx.x == 0 && tid < Mc) p.dbg_sa[tid] = sb;
     }
+    named_barrier_sync(1, kGemvConsumers);
     int qs_part[MB];
 #pragma unroll
     for (int m = 0; m < MB; ++m) {
       qs_part[m] = 0;
-      if (m < Mc) {
+      if (MB == 1 || m < Mc) {
+        RowQuant rqm;
+        rqm.s = rq_s[m];
+        rqm.r = rq_r[m];
         const uint4* row = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m) * K);
-#pragma unroll 1
-        for (int g = tid; g < groups16; g += kConsumers) {
-          const uint2 lo = quant8(__ldg(row + 2 * g), rq[m]);
-          const uint2 hi = quant8(__ldg(row + 2 * g + 1), rq[m]);
+        auto quant_group = [&](int g, const uint4& a, const uint4& b) {
+          const uint2 lo = quant8(a, rqm);
+          const uint2 hi = quant8(b, rqm);
           const uint4 nat = make_uint4(lo.x, lo.y, hi.x, hi.y);
           qs_part[m] += bytesum_s8(nat.x) + bytesum_s8(nat.y) + bytesum_s8(nat.z) +
                         bytesum_s8(nat.w);
-          *reinterpret_cast<uint4*>(qs + static_cast<int64_t>(m) * K + 16 * g) = transpose16(nat);
+          *reinterpret_cast<uint4*>(qs + m * K + 16 * g) = transpose16(nat);
           if (p.dbg_q != nullptr && blockIdx.x == 0)
             *reinterpret_cast<uint4*>(p.dbg_q + static_cast<int64_t>(m) * K + 16 * g) = nat;
+        };
+        if constexpr (HOLD) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int g = tid + j * kGemvConsumers;
+            if (g < groups16) quant_group(g, hv[m][j][0], hv[m][j][1]);
+          }
         }
+#pragma unroll 1
+        for (int g = tid + (HOLD ? 2 : 0) * kGemvConsumers; g < groups16; g += kGemvConsumers)
+          quant_group(g, __ldg(row + 2 * g), __ldg(row + 2 * g + 1));
       }
     }
-    named_barrier_sync(1, kConsumers);  // red[] reuse
+    named_barrier_sync(1, kGemvConsumers);  // red[] reuse
 #pragma unroll
     for (int m = 0; m < MB; ++m) {
       const int s = __reduce_add_sync(0xFFFFFFFFu, qs_part[m]);
       if (lane == 0) red[warp * MB + m] = static_cast<uint32_t>(s);
     }
-    named_barrier_sync(1, kConsumers);
+    named_barrier_sync(1, kGemvConsumers);
     if (tid < MB) {
       int s = 0;
       for (int w = 0; w < kGemvConsumerWarps; ++w) s += static_cast<int>(red[w * MB + tid]);
       qsum[tid] = s;
-    }
-    if (tid == 0) {  // every thread holds the same rq[]
-#pragma unroll
-      for (int m = 0; m < MB; ++m) {
-        const uint16_t sb = f32_to_bf16_bits(rq[m].s);
-        saf[m] = bf16_bits_to_f32(sb);
-        if (p.dbg_sa != nullptr && blockIdx.x == 0 && m < Mc) p.dbg_sa[m] = sb;
-      }
     }
   } else {
     int qs_part[MB];
@@ -207,17 +302,17 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
       if (m < Mc) {
         const uint4* row = reinterpret_cast<const uint4*>(p.xq + static_cast<int64_t>(m_base + m) * K);
 #pragma unroll 1
-        for (int g = tid; g < groups16; g += kConsumers) {
+        for (int g = tid; g < groups16; g += kGemvConsumers) {
           const uint4 nat = __ldg(row + g);
           qs_part[m] += bytesum_s8(nat.x) + bytesum_s8(nat.y) + bytesum_s8(nat.z) +
                         bytesum_s8(nat.w);
-          *reinterpret_cast<uint4*>(qs + static_cast<int64_t>(m) * K + 16 * g) = transpose16(nat);
+          *reinterpret_cast<uint4*>(qs + m * K + 16 * g) = transpose16(nat);
         }
       }
       const int s = __reduce_add_sync(0xFFFFFFFFu, qs_part[m]);
       if (lane == 0) red[warp * MB + m] = static_cast<uint32_t>(s);
     }
-    named_barrier_sync(1, kConsumers);
+    named_barrier_sync(1, kGemvConsumers);
     if (tid < MB) {
       int s = 0;
       for (int w = 0; w < kGemvConsumerWarps; ++w) s += static_cast<int>(red[w * MB + tid]);
@@ -226,7 +321,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
       saf[tid] = (tid < Mc && p.sa_in != nullptr) ? bf16_bits_to_f32(p.sa_in[m_base + tid]) : 0.0f;
     }
   }
-  named_barrier_sync(1, kConsumers);
+  named_barrier_sync(1, kGemvConsumers);
 
   uint32_t it = 0;
   for (int b = blockIdx.x; b < nblocks; b += gridDim.x, ++it) {
@@ -239,43 +334,19 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
     int rows = min(RW, N - n0);
     if (rows < 0) rows = 0;
 
-    int acc[RW][MB];
+    int acc[RW][MB][PLANES ? 4 : 1];
 #pragma unroll
     for (int r = 0; r < RW; ++r)
 #pragma unroll
-      for (int m = 0; m < MB; ++m) acc[r][m] = 0;
+      for (int m = 0; m < MB; ++m)
+#pragma unroll
+        for (int i = 0; i < (PLANES ? 4 : 1); ++i) acc[r][m][i] = 0;
 
-    if (rows > 0) {
-      const uint32_t* wrow = reinterpret_cast<const uint32_t*>(stage + static_cast<size_t>(r0) * KB);
-#pragma unroll 1
-      for (int t = lane; t < words; t += 32) {
-        uint4 Q[MB];
-#pragma unroll
-        for (int m = 0; m < MB; ++m)
-          if (m < Mc) Q[m] = *reinterpret_cast<const uint4*>(qs + static_cast<int64_t>(m) * K + 16 * t);
-#pragma unroll
-        for (int r = 0; r < RW; ++r) {
-          if (r < rows) {
-            const uint32_t w = wrow[r * (KB / 4) + t];
-            const uint32_t e0 = w & 0x03030303u;
-            const uint32_t e1 = (w >> 2) & 0x03030303u;
-            const uint32_t e2 = (w >> 4) & 0x03030303u;
-            const uint32_t e3 = (w >> 6) & 0x03030303u;
-#pragma unroll
-            for (int m = 0; m < MB; ++m) {
-              if (m < Mc) {
-                int a = acc[r][m];
-                a = dp4a_s32(e0, Q[m].x, a);
-                a = dp4a_s32(e1, Q[m].y, a);
-                a = dp4a_s32(e2, Q[m].z, a);
-                a = dp4a_s32(e3, Q[m].w, a);
-                acc[r][m] = a;
-              }
-            }
-          }
-        }
-      }
-    }
+    const uint32_t* wrow = reinterpret_cast<const uint32_t*>(stage + static_cast<size_t>(r0) * KB);
+    if (rows == RW)
+      gemv_rows<MB, RW, PLANES, true>(acc, wrow, words, qs, K, Mc, rows, lane);
+    else if (rows > 0)
+      gemv_rows<MB, RW, PLANES, false>(acc, wrow, words, qs, K, Mc, rows, lane);
     // the stage's shared memory may be refilled once every warp is done
     __syncwarp();
     if (lane == 0) mbar_arrive(empty(s));
@@ -284,7 +355,11 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
     for (int r = 0; r < RW; ++r) {
 #pragma unroll
       for (int m = 0; m < MB; ++m) {
-        int v = acc[r][m];
+        int v;
+        if constexpr (PLANES)
+          v = acc[r][m][0] + (acc[r][m][1] >> 2) + (acc[r][m][2] >> 4) + (acc[r][m][3] >> 6);
+        else
+          v = acc[r][m][0];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
         if (((r * MB + m) & 31) == lane && r < rows && m < Mc) {

@@ -103,9 +103,9 @@ bitnet_status bitnet_gemm(uint16_t* out, const int8_t* x_q,
  *   x         in,  [M, K] of dtype `dt` (only BITNET_BF16)
  *   w_packed, scale_wt, scale_wt_len as for bitnet_gemm.
  * Needs 1 <= M <= 15 (the page dispatches M < 16 here), and the quantised
- * rows plus two stages of weights must fit on chip:
- * 1024 + c(M * K) + 2 * c(2 * K) <= 232448 with c(v) = v rounded up to a
- * multiple of 128 (about (M + 4) * K <= 231000); otherwise BITNET_ERR_SHAPE. */
+ * rows plus one stage of sixteen weight rows must fit on chip:
+ * 2048 + c(M * K) + c(4 * K) <= 232448 with c(v) = v rounded up to a
+ * multiple of 128 (about (M + 4) * K <= 230000); otherwise BITNET_ERR_SHAPE. */
 bitnet_status bitnet_gemv_fused(uint16_t* out, const void* x, bitnet_dtype dt,
                                 const uint8_t* w_packed, const float* scale_wt,
                                 int64_t scale_wt_len, int64_t M, int64_t N,
