@@ -212,12 +212,13 @@ bitnet_status run_gemv(GemvParams p, bool preq, cudaStream_t st) {
   const int64_t KB = K / 4;
   const int warps = kGemvConsumerWarps;
   int rw = pow2_floor(kGemvStageTarget / (warps * KB));
-  const int by_n = pow2_floor(p.N / (static_cast<int64_t>(warps) * dev->sms));
-  if (rw > by_n) rw = by_n;
   const int acc_per_row = mb * (mb <= 2 ? 4 : 1);
   while (rw > 1 && rw * acc_per_row > 32) rw /= 2;
   if (rw > 8) rw = 8;
   if (rw < 1) rw = 1;
+  // small layers: keep at least 16 row blocks so the weights stream from
+  // several SMs at once
+  while (rw > 1 && (p.N + warps * rw - 1) / (warps * rw) < 16) rw /= 2;
   while (rw > 1 && gemv_smem(qrows, K, rw, 1) > kSmemLimit) rw /= 2;
   const size_t stage = align128(static_cast<size_t>(warps * rw) * KB);
   // ring depth: no deeper than the row blocks one CTA will see

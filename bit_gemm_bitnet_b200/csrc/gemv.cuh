@@ -69,10 +69,6 @@ __device__ __forceinline__ int bytesum_s8(uint32_t w) {
   return __dp4a(static_cast<int>(w), 0x01010101, 0);
 }
 
-__device__ __forceinline__ uint32_t absmax_bits16(const uint4& a, const uint4& b) {
-  return max(absmax_bits8(a), absmax_bits8(b));
-}
-
 // Partial dot products of one warp's RW rows of a stage with the quantised
 // activation rows, for lane `lane` (words lane, lane + 32, ...).
 // PLANES: four plane accumulators per (row, activation row); else one.
@@ -153,7 +149,6 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
   uint8_t* ring = qs + p.q_bytes;
   static_assert(kGemvConsumerWarps * MB * 4 <= kGemvHeaderBytes - 512, "reduction scratch");
   constexpr bool PLANES = MB <= 2;
-  constexpr bool HOLD = MB <= 2;  // keep the activation row in registers
 
   const int K = p.K, N = p.N;
   const int KB = K / 4;
@@ -212,29 +207,21 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
   pdl_wait();  // the activations may come from the previous kernel
   const int groups16 = K / 16;
   if constexpr (!PREQ) {
-    // absmax of every activation row (each thread owns 16-element groups
-    // tid, tid + 512, ...; with HOLD the first two stay in registers)
-    uint4 hv[HOLD ? MB : 1][2][2];
+    // absmax of every activation row; each thread owns the 4-element quads
+    // tid, tid + 512, ... of a row (loops kept rolled: a small code footprint)
+    const int quads = K / 4;
     uint32_t mb[MB];
 #pragma unroll
     for (int m = 0; m < MB; ++m) {
       mb[m] = 0;
       if (MB == 1 || m < Mc) {
-        const uint4* row = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m) * K);
-        if constexpr (HOLD) {
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int g = tid + j * kGemvConsumers;
-            if (g < groups16) {
-              hv[m][j][0] = __ldg(row + 2 * g);
-              hv[m][j][1] = __ldg(row + 2 * g + 1);
-              mb[m] = max(mb[m], absmax_bits16(hv[m][j][0], hv[m][j][1]));
-            }
-          }
-        }
+        const uint2* row = reinterpret_cast<const uint2*>(p.x + static_cast<int64_t>(m) * K);
 #pragma unroll 1
-        for (int g = tid + (HOLD ? 2 : 0) * kGemvConsumers; g < groups16; g += kGemvConsumers)
-          mb[m] = max(mb[m], absmax_bits16(__ldg(row + 2 * g), __ldg(row + 2 * g + 1)));
+        for (int u = tid; u < quads; u += kGemvConsumers) {
+          const uint2 v = __ldg(row + u);
+          mb[m] = max(mb[m], max(max(v.x & 0x7FFFu, (v.x >> 16) & 0x7FFFu),
+                                 max(v.y & 0x7FFFu, (v.y >> 16) & 0x7FFFu)));
+        }
       }
       mb[m] = __reduce_max_sync(0xFFFFFFFFu, mb[m]);
       if (lane == 0) red[warp * MB + m] = mb[m];
@@ -251,6 +238,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
       if (p.dbg_sa != nullptr && blockIdx.x == 0 && tid < Mc) p.dbg_sa[tid] = sb;
     }
     named_barrier_sync(1, kGemvConsumers);
+    // quantise: element 4b + i of 16-group g goes to byte 16g + 4i + b
     int qs_part[MB];
 #pragma unroll
     for (int m = 0; m < MB; ++m) {
@@ -259,27 +247,26 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
         RowQuant rqm;
         rqm.s = rq_s[m];
         rqm.r = rq_r[m];
-        const uint4* row = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m) * K);
-        auto quant_group = [&](int g, const uint4& a, const uint4& b) {
-          const uint2 lo = quant8(a, rqm);
-          const uint2 hi = quant8(b, rqm);
-          const uint4 nat = make_uint4(lo.x, lo.y, hi.x, hi.y);
-          qs_part[m] += bytesum_s8(nat.x) + bytesum_s8(nat.y) + bytesum_s8(nat.z) +
-                        bytesum_s8(nat.w);
-          *reinterpret_cast<uint4*>(qs + m * K + 16 * g) = transpose16(nat);
-          if (p.dbg_q != nullptr && blockIdx.x == 0)
-            *reinterpret_cast<uint4*>(p.dbg_q + static_cast<int64_t>(m) * K + 16 * g) = nat;
-        };
-        if constexpr (HOLD) {
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int g = tid + j * kGemvConsumers;
-            if (g < groups16) quant_group(g, hv[m][j][0], hv[m][j][1]);
-          }
-        }
+        const uint2* row = reinterpret_cast<const uint2*>(p.x + static_cast<int64_t>(m) * K);
+        uint8_t* qrow = qs + m * K;
 #pragma unroll 1
-        for (int g = tid + (HOLD ? 2 : 0) * kGemvConsumers; g < groups16; g += kGemvConsumers)
-          quant_group(g, __ldg(row + 2 * g), __ldg(row + 2 * g + 1));
+        for (int u = tid; u < quads; u += kGemvConsumers) {
+          const uint2 v = __ldg(row + u);
+          const int q0 = quant_one(bf16_bits_to_f32(v.x & 0xFFFFu), rqm);
+          const int q1 = quant_one(bf16_bits_to_f32(v.x >> 16), rqm);
+          const int q2 = quant_one(bf16_bits_to_f32(v.y & 0xFFFFu), rqm);
+          const int q3 = quant_one(bf16_bits_to_f32(v.y >> 16), rqm);
+          qs_part[m] += q0 + q1 + q2 + q3;
+          uint8_t* d = qrow + 16 * (u >> 2) + (u & 3);
+          d[0] = static_cast<uint8_t>(q0);
+          d[4] = static_cast<uint8_t>(q1);
+          d[8] = static_cast<uint8_t>(q2);
+          d[12] = static_cast<uint8_t>(q3);
+          if (p.dbg_q != nullptr && blockIdx.x == 0)
+            reinterpret_cast<uint32_t*>(p.dbg_q + static_cast<int64_t>(m) * K)[u] =
+                (static_cast<uint32_t>(q0) & 0xFFu) | ((static_cast<uint32_t>(q1) & 0xFFu) << 8) |
+                ((static_cast<uint32_t>(q2) & 0xFFu) << 16) | (static_cast<uint32_t>(q3) << 24);
+        }
       }
     }
     named_barrier_sync(1, kGemvConsumers);  // red[] reuse
@@ -351,28 +338,51 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
     __syncwarp();
     if (lane == 0) mbar_arrive(empty(s));
 
+    // Reduce the RW x MB lane partials over the warp: a butterfly that halves
+    // the number of values at each of the first log2(RW * MB) exchanges
+    // (reduce-scatter), then plain exchanges for the remaining lane bits.
+    constexpr int V = RW * MB;
+    static_assert((V & (V - 1)) == 0 && V <= 32, "V must be a power of two <= 32");
+    int vals[V];
 #pragma unroll
-    for (int r = 0; r < RW; ++r) {
+    for (int r = 0; r < RW; ++r)
 #pragma unroll
       for (int m = 0; m < MB; ++m) {
-        int v;
         if constexpr (PLANES)
-          v = acc[r][m][0] + (acc[r][m][1] >> 2) + (acc[r][m][2] >> 4) + (acc[r][m][3] >> 6);
+          vals[r * MB + m] = acc[r][m][0] + (acc[r][m][1] >> 2) + (acc[r][m][2] >> 4) +
+                             (acc[r][m][3] >> 6);
         else
-          v = acc[r][m][0];
+          vals[r * MB + m] = acc[r][m][0];
+      }
+    int idx = 0;  // which of the V values this lane ends up holding
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-        if (((r * MB + m) & 31) == lane && r < rows && m < Mc) {
-          const int n = n0 + r;
-          const int a = v - 2 * qsum[m];
-          const int64_t o = static_cast<int64_t>(m_base + m) * N + n;
-          if (p.acc_out != nullptr) {
-            p.acc_out[o] = a;
-          } else {
-            const float s_w = p.sw[p.sw_len == 1 ? 0 : n];
-            const float y = __fmul_rn(__fmul_rn(__int2float_rn(a), saf[m]), s_w);
-            p.out[o] = f32_to_bf16_bits(y);
-          }
+    for (int h = V / 2, o = 16; h >= 1; h /= 2, o /= 2) {
+      const bool hi = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < h; ++i) {
+        const int send = hi ? vals[i] : vals[i + h];
+        const int keep = hi ? vals[i + h] : vals[i];
+        vals[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+      }
+      idx += hi ? h : 0;
+    }
+    int v = vals[0];
+    constexpr int kDone = V >= 32 ? 32 : V;  // lane bits already summed: log2(V)
+#pragma unroll
+    for (int o = 32 / kDone / 2; o >= 1; o /= 2) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    // lanes that differ only in the low bits hold the same total; one stores
+    if ((lane & (32 / kDone - 1)) == 0) {
+      const int r = idx / MB, m = idx % MB;
+      if (r < rows && m < Mc) {
+        const int n = n0 + r;
+        const int a = v - 2 * qsum[m];
+        const int64_t o = static_cast<int64_t>(m_base + m) * N + n;
+        if (p.acc_out != nullptr) {
+          p.acc_out[o] = a;
+        } else {
+          const float s_w = p.sw[p.sw_len == 1 ? 0 : n];
+          const float y = __fmul_rn(__fmul_rn(__int2float_rn(a), saf[m]), s_w);
+          p.out[o] = f32_to_bf16_bits(y);
         }
       }
     }
