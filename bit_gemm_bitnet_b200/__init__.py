@@ -28,7 +28,7 @@ EXPORTS = (
     "bitnet_pack_weights", "bitnet_quantize_act", "bitnet_gemm",
     "bitnet_gemv_fused", "bitnet_linear_workspace_bytes", "bitnet_linear",
     "bitnet_device_status", "bitnet_status_string", "bitnet_gemm_acc_i32",
-    "bitnet_gemv_fused_debug",
+    "bitnet_gemv_fused_debug", "bitnet_linear_noalloc",
 )
 
 _lib = None
@@ -60,6 +60,7 @@ def lib():
             "bitnet_gemm": [P, P, P, P, P, I64, I64, I64, I64, P],
             "bitnet_gemv_fused": [P, P, I, P, P, I64, I64, I64, I64, P],
             "bitnet_linear": [P, P, I, P, P, I64, I64, I64, I64, P, SZ, P],
+            "bitnet_linear_noalloc": [P, P, I, P, P, I64, I64, I64, I64, P],
             "bitnet_device_status": [P],
             "bitnet_gemm_acc_i32": [P, P, P, I64, I64, I64, P],
             "bitnet_gemv_fused_debug": [P, P, P, P, I, P, I64, I64, I64, P],
@@ -210,6 +211,28 @@ def bitnet_linear(x, w_packed, scale_wt, out=None, workspace=None):
     _check(lib().bitnet_linear(_ptr(out), _ptr(x2), BF16, _ptr(w_packed), _ptr(sw),
                                sw.numel(), M, N, K, wsp, need, _stream(x.device)),
            "bitnet_linear")
+    return out.view(*orig[:-1], N)
+
+
+def bitnet_linear_noalloc(x, w_packed, scale_wt, out=None):
+    """bitnet_linear without a workspace argument: for M >= 16 the library
+    keeps the quantised activations in its built-in 16 MiB scratch (see
+    include/bitnet.h); calls that may overlap on the GPU must not share it."""
+    orig = x.shape
+    K = orig[-1]
+    x2 = x.reshape(-1, K)
+    _need(x2, torch.bfloat16, "x", 2)
+    _need(w_packed, torch.uint8, "w_packed", 2)
+    M = x2.shape[0]
+    N = w_packed.shape[0]
+    if w_packed.shape[1] * 4 != K:
+        raise ValueError(f"w_packed {tuple(w_packed.shape)} does not match K={K}")
+    sw = _scale_wt(scale_wt, N, x.device)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _check(lib().bitnet_linear_noalloc(_ptr(out), _ptr(x2), BF16, _ptr(w_packed), _ptr(sw),
+                                       sw.numel(), M, N, K, _stream(x.device)),
+           "bitnet_linear_noalloc")
     return out.view(*orig[:-1], N)
 
 

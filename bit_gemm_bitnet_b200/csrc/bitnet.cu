@@ -325,6 +325,38 @@ bool linear_uses_gemv(int64_t M, int64_t K) {
 
 using namespace bitnet;
 
+// ---------------------------------------------------------------------------
+// Allocation-free linear: built-in scratch.
+//
+// bitnet_linear needs a workspace for the quantised activations (int8 [M, K])
+// and their scales (bf16 [M]) when M >= 16. Callers that cannot allocate
+// device memory use bitnet_linear_noalloc instead, which places them in this
+// fixed array. It lives in the module's global memory of every GPU that loads
+// the library, for the life of the process; all calls on a device share it.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+// Device address of g_noalloc_scratch, looked up once per device. In host
+// code the array's name only stands in for the device symbol; kernels must
+// be given the address cudaGetSymbolAddress returns.
+void* g_noalloc_ptr[64] = {};
+
+bitnet_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BITNET_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return BITNET_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return BITNET_OK;
+}
+}  // namespace
+
 extern "C" {
 
 const char* bitnet_status_string(bitnet_status s) {
@@ -490,6 +522,28 @@ bitnet_status bitnet_linear(uint16_t* out, const void* x, bitnet_dtype dt,
   s = run_quantize(xq, sa, static_cast<const uint16_t*>(x), M, K, st);
   if (s != BITNET_OK) return s;
   return run_gemm(out, false, xq, w_packed, sa, scale_wt, scale_wt_len, M, N, K, st);
+}
+
+bitnet_status bitnet_linear_noalloc(uint16_t* out, const void* x, bitnet_dtype dt,
+                                    const uint8_t* w_packed, const float* scale_wt,
+                                    int64_t scale_wt_len, int64_t M, int64_t N, int64_t K,
+                                    void* stream) {
+  if (dt != BITNET_BF16) return BITNET_ERR_DTYPE;
+  bitnet_status s = check_compute_shape(M, N, K);
+  if (s != BITNET_OK) return s;
+  if (M == 0 || N == 0) return BITNET_OK;
+  if (out == nullptr || x == nullptr || w_packed == nullptr) return BITNET_ERR_NULL;
+  if (linear_uses_gemv(M, K))  // the fused GEMV needs no scratch
+    return bitnet_gemv_fused(out, x, dt, w_packed, scale_wt, scale_wt_len, M, N, K, stream);
+  const size_t need = bitnet_linear_workspace_bytes(M, K);
+  if (need > kNoAllocScratchBytes) return BITNET_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  s = noalloc_scratch(&scratch);
+  if (s != BITNET_OK) return s;
+  // x_q and the scales are written in full by the quantiser before the GEMM
+  // reads them, so nothing left from an earlier call is ever used.
+  return bitnet_linear(out, x, dt, w_packed, scale_wt, scale_wt_len, M, N, K, scratch,
+                       kNoAllocScratchBytes, stream);
 }
 
 bitnet_status bitnet_device_status(void* stream) {

@@ -128,6 +128,30 @@ bitnet_status bitnet_linear(uint16_t* out, const void* x, bitnet_dtype dt,
                             int64_t K, void* workspace, size_t workspace_bytes,
                             void* stream);
 
+/* bitnet_linear without a caller workspace, for callers that cannot allocate
+ * device memory: code running while a stream is being captured into a CUDA
+ * graph (cudaMalloc is not allowed there), code inside a framework that owns
+ * all device memory through its own pool, or latency-critical paths that
+ * cannot afford an allocation's implicit synchronisation. The paper has no
+ * counterpart; this is a convenience of this library's C ABI.
+ * Arguments and result are those of bitnet_linear. When M >= 16 (the split
+ * path), the int8 activations and their scales are placed in a scratch array
+ * built into the library: 16 MiB (16777216 bytes) per GPU, reserved by every
+ * GPU that loads the library until the process exits. Shapes whose
+ * bitnet_linear_workspace_bytes(M, K) exceeds it return BITNET_ERR_WORKSPACE
+ * and enqueue nothing. The call allocates nothing.
+ * The first call on a device looks up the scratch's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. Every call on a device shares the one scratch array: calls that
+ * may run at the same time on the GPU (different streams without ordering
+ * between them) race on it and must not overlap. Calls ordered on one stream
+ * are safe; each call overwrites whatever an earlier call left there. */
+bitnet_status bitnet_linear_noalloc(uint16_t* out, const void* x,
+                                    bitnet_dtype dt, const uint8_t* w_packed,
+                                    const float* scale_wt, int64_t scale_wt_len,
+                                    int64_t M, int64_t N, int64_t K,
+                                    void* stream);
+
 /* Synchronise `stream`, then read and clear the device-side error word the
  * kernels set when a bounded wait gives up. BITNET_ERR_TIMEOUT if it was
  * set (the outputs of the affected call are then unspecified), BITNET_OK
