@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--branches", type=int, default=16,
+                    help="graph branches for the independent calls of a step")
     return ap.parse_args()
 
 
@@ -409,9 +411,9 @@ def main():
               "calls_per_step": len(W.decode_2b_sweep()),
               "packed_weight_bytes_per_step": W.decode_2b_packed_bytes(),
               "l2": "inputs larger than L2 (603 MB of packed weights streamed per step)",
-              "issue_order": "independent calls (each has its own activation row) on 8 "
-                             "graph branches; 'issue_orders' reports the transformer-layer "
-                             "dependency order and a single stream",
+              "issue_order": f"independent calls (each has its own activation row) on "
+                             f"{args.branches} graph branches; 'issue_orders' reports the "
+                             "transformer-layer dependency order and a single stream",
               "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
     if args.impl == "reference":
@@ -455,7 +457,7 @@ def main():
     graphs = {}
     with torch.cuda.stream(stream):
         for order in ("independent", "layer", "stream"):
-            sweep = make_sweep(bn, d, order)
+            sweep = make_sweep(bn, d, order, branches=args.branches)
             sweep()
             torch.cuda.synchronize()
             bn.bitnet_device_status()

@@ -122,15 +122,16 @@ constexpr size_t kSmemLimit = 232448;  // per-CTA opt-in maximum on sm_100
 
 // Shared memory of the GEMV for `rows` activation rows of length K and a ring
 // of `stages` stages of `rw` rows per warp.
-size_t gemv_smem(int rows, int64_t K, int rw, int stages) {
+size_t gemv_smem(int rows, int64_t K, int cw, int rw, int stages) {
   return kGemvHeaderBytes + align128(static_cast<size_t>(rows) * K) +
-         static_cast<size_t>(stages) *
-             align128(static_cast<size_t>(kGemvConsumerWarps * rw) * (K / 4));
+         static_cast<size_t>(stages) * align128(static_cast<size_t>(cw * rw) * (K / 4));
 }
 
 // Does the GEMV fit `rows` activation rows of length K (one stage of one
-// row per warp at least)?
-bool gemv_fits(int rows, int64_t K) { return gemv_smem(rows, K, 1, 1) <= kSmemLimit; }
+// row per warp of the widest CTA at least)?
+bool gemv_fits(int rows, int64_t K) {
+  return gemv_smem(rows, K, kGemvMaxConsumerWarps, 1, 1) <= kSmemLimit;
+}
 
 int pow2_floor(int64_t v) {
   int r = 1;
@@ -138,10 +139,11 @@ int pow2_floor(int64_t v) {
   return r;
 }
 
-template <int MB, int RW, bool WIDE, bool PREQ>
+template <int CW, int MB, int RW, bool WIDE, bool PREQ>
 bitnet_status launch_gemv_t(const GemvParams& p, int grid_y, size_t smem, int sms,
                             cudaStream_t st) {
-  auto k = gemv_kernel<MB, RW, WIDE, PREQ>;
+  auto k = gemv_kernel<CW, MB, RW, WIDE, PREQ>;
+  constexpr int threads = (CW + 1) * 32;
   if (smem > 48 * 1024) {
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
@@ -149,40 +151,47 @@ bitnet_status launch_gemv_t(const GemvParams& p, int grid_y, size_t smem, int sm
   }
   // persistent: no more CTAs than row blocks, nor than can be resident
   int occ = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kGemvThreads, smem) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, threads, smem) != cudaSuccess)
     return BITNET_ERR_CUDA;
   if (occ < 1) occ = 1;
   const int nblocks = (p.N + p.rows_per_block - 1) / p.rows_per_block;
   int gx = nblocks < occ * sms ? nblocks : occ * sms;
   if (gx < 1) gx = 1;
-  return launch_pdl(k, dim3(gx, grid_y), dim3(kGemvThreads), smem, st, p);
+  return launch_pdl(k, dim3(gx, grid_y), dim3(threads), smem, st, p);
 }
 
-template <int MB, bool WIDE, bool PREQ>
+template <int CW, int MB, bool WIDE, bool PREQ>
 bitnet_status launch_gemv_rw(int rw, const GemvParams& p, int gy, size_t smem, int sms,
                              cudaStream_t st) {
   switch (rw) {
-    case 1: return launch_gemv_t<MB, 1, WIDE, PREQ>(p, gy, smem, sms, st);
-    case 2: return launch_gemv_t<MB, 2, WIDE, PREQ>(p, gy, smem, sms, st);
+    case 1: return launch_gemv_t<CW, MB, 1, WIDE, PREQ>(p, gy, smem, sms, st);
+    case 2: return launch_gemv_t<CW, MB, 2, WIDE, PREQ>(p, gy, smem, sms, st);
     case 4:
-      if constexpr (MB != 2 && MB <= 8) return launch_gemv_t<MB, 4, WIDE, PREQ>(p, gy, smem, sms, st);
+      if constexpr (MB != 2 && MB <= 8) return launch_gemv_t<CW, MB, 4, WIDE, PREQ>(p, gy, smem, sms, st);
       return BITNET_ERR_SHAPE;
     default:
-      if constexpr (MB == 1 || MB == 4) return launch_gemv_t<MB, 8, WIDE, PREQ>(p, gy, smem, sms, st);
+      if constexpr (MB == 1 || MB == 4) return launch_gemv_t<CW, MB, 8, WIDE, PREQ>(p, gy, smem, sms, st);
       return BITNET_ERR_SHAPE;
+  }
+}
+
+template <int CW, bool WIDE, bool PREQ>
+bitnet_status launch_gemv_mb(int mb, int rw, const GemvParams& p, int gy, size_t smem, int sms,
+                             cudaStream_t st) {
+  switch (mb) {
+    case 1: return launch_gemv_rw<CW, 1, WIDE, PREQ>(rw, p, gy, smem, sms, st);
+    case 2: return launch_gemv_rw<CW, 2, WIDE, PREQ>(rw, p, gy, smem, sms, st);
+    case 4: return launch_gemv_rw<CW, 4, WIDE, PREQ>(rw, p, gy, smem, sms, st);
+    case 8: return launch_gemv_rw<CW, 8, WIDE, PREQ>(rw, p, gy, smem, sms, st);
+    default: return launch_gemv_rw<CW, 16, WIDE, PREQ>(rw, p, gy, smem, sms, st);
   }
 }
 
 template <bool WIDE, bool PREQ>
-bitnet_status launch_gemv_mb(int mb, int rw, const GemvParams& p, int gy, size_t smem, int sms,
-                             cudaStream_t st) {
-  switch (mb) {
-    case 1: return launch_gemv_rw<1, WIDE, PREQ>(rw, p, gy, smem, sms, st);
-    case 2: return launch_gemv_rw<2, WIDE, PREQ>(rw, p, gy, smem, sms, st);
-    case 4: return launch_gemv_rw<4, WIDE, PREQ>(rw, p, gy, smem, sms, st);
-    case 8: return launch_gemv_rw<8, WIDE, PREQ>(rw, p, gy, smem, sms, st);
-    default: return launch_gemv_rw<16, WIDE, PREQ>(rw, p, gy, smem, sms, st);
-  }
+bitnet_status launch_gemv_cw(int cw, int mb, int rw, const GemvParams& p, int gy, size_t smem,
+                             int sms, cudaStream_t st) {
+  if (cw == 16) return launch_gemv_mb<16, WIDE, PREQ>(mb, rw, p, gy, smem, sms, st);
+  return launch_gemv_mb<4, WIDE, PREQ>(mb, rw, p, gy, smem, sms, st);
 }
 
 int bucket_of(int m) { return m <= 1 ? 1 : m <= 2 ? 2 : m <= 4 ? 4 : m <= 8 ? 8 : 16; }
@@ -207,39 +216,47 @@ bitnet_status run_gemv(GemvParams p, bool preq, cudaStream_t st) {
     if (gy > 65535) return BITNET_ERR_SHAPE;
   }
   if (!gemv_fits(qrows, K)) return BITNET_ERR_SHAPE;
-  // rows per warp per stage: a stage near 40 KB, enough row blocks to cover
-  // the SMs, and at most 32 accumulator registers per lane
+  // Consumer warps per CTA: 16 for large layers (many row blocks per SM),
+  // 4 for small ones, so that kernels of independent calls fit side by side.
   const int64_t KB = K / 4;
-  const int warps = kGemvConsumerWarps;
-  int rw = pow2_floor(kGemvStageTarget / (warps * KB));
-  const int acc_per_row = mb * (mb <= 2 ? 4 : 1);
-  while (rw > 1 && rw * acc_per_row > 32) rw /= 2;
-  if (rw > 8) rw = 8;
-  if (rw < 1) rw = 1;
-  // small layers: keep at least 16 row blocks so the weights stream from
-  // several SMs at once
-  while (rw > 1 && (p.N + warps * rw - 1) / (warps * rw) < 16) rw /= 2;
-  while (rw > 1 && gemv_smem(qrows, K, rw, 1) > kSmemLimit) rw /= 2;
-  const size_t stage = align128(static_cast<size_t>(warps * rw) * KB);
+  auto pick_rw = [&](int warps) {
+    // rows per warp per stage: a stage near 40 KB, at most 32 accumulator
+    // registers per lane, and at least 16 row blocks on small layers
+    int r = pow2_floor(kGemvStageTarget / (warps * KB));
+    const int acc_per_row = mb * (mb <= 2 ? 4 : 1);
+    while (r > 1 && r * acc_per_row > 32) r /= 2;
+    if (r > 8) r = 8;
+    if (r < 1) r = 1;
+    while (r > 1 && (p.N + warps * r - 1) / (warps * r) < 16) r /= 2;
+    while (r > 1 && gemv_smem(qrows, K, warps, r, 1) > kSmemLimit) r /= 2;
+    return r;
+  };
+  int cw = 16;
+  int rw = pick_rw(cw);
+  if ((p.N + cw * rw - 1) / (cw * rw) < 2 * static_cast<int64_t>(dev->sms)) {
+    cw = 4;
+    rw = pick_rw(cw);
+  }
+  const size_t stage = align128(static_cast<size_t>(cw * rw) * KB);
   // ring depth: no deeper than the row blocks one CTA will see
-  const int64_t nblocks = (p.N + warps * rw - 1) / (warps * rw);
+  const int64_t nblocks = (p.N + cw * rw - 1) / (cw * rw);
   const int64_t per_cta = (nblocks + dev->sms - 1) / dev->sms;
   int stages = static_cast<int>(kGemvRingTarget / stage);
   if (stages > per_cta) stages = static_cast<int>(per_cta);
   if (stages > kGemvMaxStages) stages = kGemvMaxStages;
   if (stages < 1) stages = 1;
-  while (stages > 1 && gemv_smem(qrows, K, rw, stages) > kSmemLimit) --stages;
-  p.rows_per_block = warps * rw;
+  while (stages > 1 && gemv_smem(qrows, K, cw, rw, stages) > kSmemLimit) --stages;
+  p.rows_per_block = cw * rw;
   p.stages = stages;
   p.q_bytes = static_cast<uint32_t>(align128(static_cast<size_t>(qrows) * K));
   p.stage_bytes = static_cast<uint32_t>(stage);
-  const size_t smem = gemv_smem(qrows, K, rw, stages);
+  const size_t smem = gemv_smem(qrows, K, cw, rw, stages);
   const bool wide = (K % 64) == 0;
   if (wide)
-    return preq ? launch_gemv_mb<true, true>(mb, rw, p, gy, smem, dev->sms, st)
-                : launch_gemv_mb<true, false>(mb, rw, p, gy, smem, dev->sms, st);
-  return preq ? launch_gemv_mb<false, true>(mb, rw, p, gy, smem, dev->sms, st)
-              : launch_gemv_mb<false, false>(mb, rw, p, gy, smem, dev->sms, st);
+    return preq ? launch_gemv_cw<true, true>(cw, mb, rw, p, gy, smem, dev->sms, st)
+                : launch_gemv_cw<true, false>(cw, mb, rw, p, gy, smem, dev->sms, st);
+  return preq ? launch_gemv_cw<false, true>(cw, mb, rw, p, gy, smem, dev->sms, st)
+              : launch_gemv_cw<false, false>(cw, mb, rw, p, gy, smem, dev->sms, st);
 }
 
 // ---------------------------------------------------------------- GEMM

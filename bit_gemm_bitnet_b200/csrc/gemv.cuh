@@ -29,9 +29,7 @@
 
 namespace bitnet {
 
-constexpr int kGemvConsumerWarps = 16;
-constexpr int kGemvConsumers = kGemvConsumerWarps * 32;
-constexpr int kGemvThreads = kGemvConsumers + 32;  // + producer warp
+constexpr int kGemvMaxConsumerWarps = 16;
 constexpr int kGemvMaxStages = 8;
 constexpr int kGemvHeaderBytes = 2048;
 constexpr int kGemvStageTarget = 40 * 1024;  // bytes per stage (aim)
@@ -47,7 +45,7 @@ struct GemvParams {
   const float* sw;
   int sw_len;
   int M, N, K;
-  int rows_per_block;     // 16 * RW
+  int rows_per_block;     // CW * RW
   int stages;             // ring depth (<= kGemvMaxStages)
   uint32_t q_bytes;       // shared bytes reserved for the quantised rows
   uint32_t stage_bytes;   // shared bytes per stage (>= rows_per_block * K/4)
@@ -131,12 +129,15 @@ __device__ __forceinline__ void gemv_rows(int (&acc)[RW][MB][PLANES ? 4 : 1],
   }
 }
 
+// CW: consumer warps per CTA (4 for small layers, 16 for large ones);
 // MB: rows of x per CTA (bucket); RW: weight rows per consumer warp per stage;
 // WIDE: K % 64 == 0 (rows 16-byte aligned: one bulk copy per stage),
 // otherwise the producer lanes copy the stage in 8-byte pieces;
 // PREQ: activations come pre-quantised (x_q + scale_act).
-template <int MB, int RW, bool WIDE, bool PREQ>
-__global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
+template <int CW, int MB, int RW, bool WIDE, bool PREQ>
+__global__ void __launch_bounds__((CW + 1) * 32) gemv_kernel(GemvParams p) {
+  constexpr int kGemvConsumerWarps = CW;
+  constexpr int kGemvConsumers = CW * 32;
   extern __shared__ __align__(128) uint8_t smem[];
   int* qsum = reinterpret_cast<int*>(smem);                  // [MB]
   float* saf = reinterpret_cast<float*>(smem + 64);          // [MB]
@@ -147,7 +148,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
   uint32_t* red = reinterpret_cast<uint32_t*>(smem + 512);   // [16 warps][MB]
   uint8_t* qs = smem + kGemvHeaderBytes;                     // [Mc][K]
   uint8_t* ring = qs + p.q_bytes;
-  static_assert(kGemvConsumerWarps * MB * 4 <= kGemvHeaderBytes - 512, "reduction scratch");
+  static_assert(kGemvMaxConsumerWarps * MB * 4 <= kGemvHeaderBytes - 512, "reduction scratch");
   constexpr bool PLANES = MB <= 2;
 
   const int K = p.K, N = p.N;
@@ -204,6 +205,15 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvParams p) {
   }
 
   // -------------------------------------------------------------- consumers
+  if constexpr (!PREQ) {
+    // Warm L2 with the activation rows before waiting for their producer.
+    // L2 is the point of coherence, so a line fetched early is updated by any
+    // later write; the loads that use the values come after the wait.
+    const char* xb = reinterpret_cast<const char*>(p.x);
+    const int64_t xbytes = static_cast<int64_t>(Mc) * K * 2;
+    for (int64_t off = static_cast<int64_t>(tid) * 128; off < xbytes; off += kGemvConsumers * 128)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(xb + off));
+  }
   pdl_wait();  // the activations may come from the previous kernel
   const int groups16 = K / 16;
   if constexpr (!PREQ) {
