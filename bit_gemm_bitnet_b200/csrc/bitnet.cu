@@ -190,8 +190,8 @@ bitnet_status launch_gemv_mb(int mb, int rw, const GemvParams& p, int gy, size_t
 template <bool WIDE, bool PREQ>
 bitnet_status launch_gemv_cw(int cw, int mb, int rw, const GemvParams& p, int gy, size_t smem,
                              int sms, cudaStream_t st) {
-  if (cw == 16) return launch_gemv_mb<16, WIDE, PREQ>(mb, rw, p, gy, smem, sms, st);
-  return launch_gemv_mb<4, WIDE, PREQ>(mb, rw, p, gy, smem, sms, st);
+  (void)cw;  // one CTA shape today: 16 consumer warps
+  return launch_gemv_mb<16, WIDE, PREQ>(mb, rw, p, gy, smem, sms, st);
 }
 
 int bucket_of(int m) { return m <= 1 ? 1 : m <= 2 ? 2 : m <= 4 ? 4 : m <= 8 ? 8 : 16; }
@@ -216,8 +216,6 @@ bitnet_status run_gemv(GemvParams p, bool preq, cudaStream_t st) {
     if (gy > 65535) return BITNET_ERR_SHAPE;
   }
   if (!gemv_fits(qrows, K)) return BITNET_ERR_SHAPE;
-  // Consumer warps per CTA: 16 for large layers (many row blocks per SM),
-  // 4 for small ones, so that kernels of independent calls fit side by side.
   const int64_t KB = K / 4;
   auto pick_rw = [&](int warps) {
     // rows per warp per stage: a stage near 40 KB, at most 32 accumulator
@@ -231,12 +229,10 @@ bitnet_status run_gemv(GemvParams p, bool preq, cudaStream_t st) {
     while (r > 1 && gemv_smem(qrows, K, warps, r, 1) > kSmemLimit) r /= 2;
     return r;
   };
-  int cw = 16;
-  int rw = pick_rw(cw);
-  if ((p.N + cw * rw - 1) / (cw * rw) < 2 * static_cast<int64_t>(dev->sms)) {
-    cw = 4;
-    rw = pick_rw(cw);
-  }
+  // 16 consumer warps: with fewer, the quantisation prologue of a small
+  // layer takes more dependent load rounds per thread and the layer slows.
+  const int cw = 16;
+  const int rw = pick_rw(cw);
   const size_t stage = align128(static_cast<size_t>(cw * rw) * KB);
   // ring depth: no deeper than the row blocks one CTA will see
   const int64_t nblocks = (p.N + cw * rw - 1) / (cw * rw);

@@ -129,7 +129,7 @@ __device__ __forceinline__ void gemv_rows(int (&acc)[RW][MB][PLANES ? 4 : 1],
   }
 }
 
-// CW: consumer warps per CTA (4 for small layers, 16 for large ones);
+// CW: consumer warps per CTA;
 // MB: rows of x per CTA (bucket); RW: weight rows per consumer warp per stage;
 // WIDE: K % 64 == 0 (rows 16-byte aligned: one bulk copy per stage),
 // otherwise the producer lanes copy the stage in 8-byte pieces;
@@ -226,11 +226,19 @@ __global__ void __launch_bounds__((CW + 1) * 32) gemv_kernel(GemvParams p) {
       mb[m] = 0;
       if (MB == 1 || m < Mc) {
         const uint2* row = reinterpret_cast<const uint2*>(p.x + static_cast<int64_t>(m) * K);
+        // four independent loads in flight per round
 #pragma unroll 1
-        for (int u = tid; u < quads; u += kGemvConsumers) {
-          const uint2 v = __ldg(row + u);
-          mb[m] = max(mb[m], max(max(v.x & 0x7FFFu, (v.x >> 16) & 0x7FFFu),
-                                 max(v.y & 0x7FFFu, (v.y >> 16) & 0x7FFFu)));
+        for (int u0 = tid; u0 < quads; u0 += 4 * kGemvConsumers) {
+          uint2 v[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int u = u0 + j * kGemvConsumers;
+            v[j] = u < quads ? __ldg(row + u) : make_uint2(0u, 0u);
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            mb[m] = max(mb[m], max(max(v[j].x & 0x7FFFu, (v[j].x >> 16) & 0x7FFFu),
+                                   max(v[j].y & 0x7FFFu, (v[j].y >> 16) & 0x7FFFu)));
         }
       }
       mb[m] = __reduce_max_sync(0xFFFFFFFFu, mb[m]);
