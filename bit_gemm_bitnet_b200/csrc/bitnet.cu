@@ -262,12 +262,15 @@ bool gemm_tcgen05_ok(const int8_t* xq, const uint8_t* wp, int64_t K) {
   return (K % 64) == 0 && aligned(xq, 16) && aligned(wp, 16);
 }
 
-bitnet_status run_gemm(void* out, bool acc_out, const int8_t* xq,
-                       const uint8_t* wp, const uint16_t* sa, const float* sw,
-                       int64_t sw_len, int64_t M, int64_t N, int64_t K,
-                       cudaStream_t st) {
+// perm: x_q has transposed 16-element groups and rowsum holds its per-row
+// code sums (the layout of bitnet_linear's workspace); tensor-core path only.
+bitnet_status run_gemm(void* out, bool acc_out, const int8_t* xq, const uint8_t* wp,
+                       const uint16_t* sa, const float* sw, int64_t sw_len, int64_t M,
+                       int64_t N, int64_t K, cudaStream_t st, bool perm = false,
+                       const int32_t* rowsum = nullptr) {
   if (M == 0 || N == 0) return BITNET_OK;
   if (!gemm_tcgen05_ok(xq, wp, K)) {
+    if (perm) return BITNET_ERR_SHAPE;  // callers only ask for perm when it applies
     GemvParams p = {};
     if (acc_out) p.acc_out = static_cast<int32_t*>(out);
     else p.out = static_cast<uint16_t*>(out);
@@ -292,22 +295,17 @@ bitnet_status run_gemm(void* out, bool acc_out, const int8_t* xq,
   const int64_t tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + gemm::BN - 1) / gemm::BN);
   if (tiles > INT32_MAX) return BITNET_ERR_SHAPE;
   const int grid = static_cast<int>(tiles < dev->sms ? tiles : dev->sms);
-  if (acc_out) {
-    auto k = gemm::gemm_i8_tcgen05_kernel<true>;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto go = [&](auto kernel) -> bitnet_status {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gemm::SMEM_BYTES) != cudaSuccess)
       return BITNET_ERR_CUDA;
-    return launch_pdl(k, dim3(grid), dim3(gemm::NUM_THREADS), gemm::SMEM_BYTES, st,
-                      mx, mw, out, sa, sw, static_cast<int>(sw_len), static_cast<int>(M),
+    return launch_pdl(kernel, dim3(grid), dim3(gemm::NUM_THREADS), gemm::SMEM_BYTES, st, mx,
+                      mw, out, sa, sw, static_cast<int>(sw_len), rowsum, static_cast<int>(M),
                       static_cast<int>(N), static_cast<int>(K));
-  }
-  auto k = gemm::gemm_i8_tcgen05_kernel<false>;
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           gemm::SMEM_BYTES) != cudaSuccess)
-    return BITNET_ERR_CUDA;
-  return launch_pdl(k, dim3(grid), dim3(gemm::NUM_THREADS), gemm::SMEM_BYTES, st, mx,
-                    mw, out, sa, sw, static_cast<int>(sw_len), static_cast<int>(M),
-                    static_cast<int>(N), static_cast<int>(K));
+  };
+  if (acc_out) return go(gemm::gemm_i8_tcgen05_kernel<true, false>);
+  if (perm) return go(gemm::gemm_i8_tcgen05_kernel<false, true>);
+  return go(gemm::gemm_i8_tcgen05_kernel<false, false>);
 }
 
 bitnet_status run_quantize(int8_t* xq, uint16_t* sa, const uint16_t* x, int64_t M,
@@ -325,6 +323,24 @@ bitnet_status run_quantize(int8_t* xq, uint16_t* sa, const uint16_t* x, int64_t 
   if (nvec <= 8 * kQuantThreads)
     return launch_pdl(quantize_rows_kernel<8>, grid, block, 0, st, xq, sa, x, static_cast<int>(K));
   return launch_pdl(quantize_rows_kernel<0>, grid, block, 0, st, xq, sa, x, static_cast<int>(K));
+}
+
+// The quantiser of bitnet_linear's tensor-core path: transposed 16-element
+// groups plus per-row code sums.
+bitnet_status run_quantize_perm(int8_t* xq, uint16_t* sa, int32_t* rowsum, const uint16_t* x,
+                                int64_t M, int64_t K, cudaStream_t st) {
+  if (M == 0) return BITNET_OK;
+  if (M > INT32_MAX) return BITNET_ERR_SHAPE;
+  const int64_t groups = K / 16;
+  const dim3 grid(static_cast<unsigned>(M)), block(kQuantThreads);
+  const int k = static_cast<int>(K);
+  if (groups <= 1 * kQuantThreads)
+    return launch_pdl(quantize_rows_perm_kernel<1>, grid, block, 0, st, xq, sa, rowsum, x, k);
+  if (groups <= 2 * kQuantThreads)
+    return launch_pdl(quantize_rows_perm_kernel<2>, grid, block, 0, st, xq, sa, rowsum, x, k);
+  if (groups <= 4 * kQuantThreads)
+    return launch_pdl(quantize_rows_perm_kernel<4>, grid, block, 0, st, xq, sa, rowsum, x, k);
+  return launch_pdl(quantize_rows_perm_kernel<0>, grid, block, 0, st, xq, sa, rowsum, x, k);
 }
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
@@ -507,8 +523,9 @@ bitnet_status bitnet_gemv_fused_debug(int32_t* acc, int8_t* x_q, uint16_t* scale
 size_t bitnet_linear_workspace_bytes(int64_t M, int64_t K) {
   if (M <= 0 || K <= 0) return 0;
   if (linear_uses_gemv(M, K)) return 0;
+  // int8 activations [M, K], bf16 scales [M], int32 per-row code sums [M]
   return align256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
-         align256(static_cast<size_t>(M) * 2);
+         align256(static_cast<size_t>(M) * 2) + align256(static_cast<size_t>(M) * 4);
 }
 
 bitnet_status bitnet_linear(uint16_t* out, const void* x, bitnet_dtype dt,
@@ -528,11 +545,21 @@ bitnet_status bitnet_linear(uint16_t* out, const void* x, bitnet_dtype dt,
   s = check_scale_wt(scale_wt, scale_wt_len, N);
   if (s != BITNET_OK) return s;
   if (!aligned(out, 16) || !aligned(x, 16) || !aligned(w_packed, 16)) return BITNET_ERR_ALIGN;
-  int8_t* xq = static_cast<int8_t*>(workspace);
-  uint16_t* sa = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) +
-                                             align256(static_cast<size_t>(M) * K));
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int8_t* xq = reinterpret_cast<int8_t*>(ws);
+  uint16_t* sa = reinterpret_cast<uint16_t*>(ws + align256(static_cast<size_t>(M) * K));
+  int32_t* rowsum = reinterpret_cast<int32_t*>(ws + align256(static_cast<size_t>(M) * K) +
+                                               align256(static_cast<size_t>(M) * 2));
   cudaStream_t st = as_stream(stream);
-  s = run_quantize(xq, sa, static_cast<const uint16_t*>(x), M, K, st);
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  if (gemm_tcgen05_ok(xq, w_packed, K)) {
+    // tensor-core path: transposed groups + row sums, weights as code planes
+    s = run_quantize_perm(xq, sa, rowsum, xb, M, K, st);
+    if (s != BITNET_OK) return s;
+    return run_gemm(out, false, xq, w_packed, sa, scale_wt, scale_wt_len, M, N, K, st, true,
+                    rowsum);
+  }
+  s = run_quantize(xq, sa, xb, M, K, st);
   if (s != BITNET_OK) return s;
   return run_gemm(out, false, xq, w_packed, sa, scale_wt, scale_wt_len, M, N, K, st);
 }

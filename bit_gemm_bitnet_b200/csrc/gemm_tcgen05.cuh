@@ -10,8 +10,10 @@
 //               stage into a double-buffered 128 x 256 int32 accumulator;
 //   warps 4-7   epilogue: tcgen05.ld of the accumulator, fp32 scaling,
 //               bf16 stores (or the raw int32 for the test hook);
-//   warps 8-11  unpack: 2-bit codes -> signed int8 weights written into the
-//               128-byte-swizzled K-major layout the MMA reads.
+//   warps 8-11  unpack: 2-bit codes -> int8 weights written into the
+//               128-byte-swizzled K-major layout the MMA reads (signed
+//               weights in natural order, or the unsigned code planes when
+//               the activations come with transposed 16-element groups).
 // Every wait is bounded (see mbar_wait); a role that gives up sets the device
 // error word and the CTA drains and exits.
 #pragma once
@@ -36,11 +38,13 @@ constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + BAR_BYT
 static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment");
 static_assert(SMEM_BYTES <= 232448, "too much shared memory");
 
-// Instruction descriptor: int32 D, signed int8 A and B, both K-major,
-// N = 256, M = 128.
-constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) |
-                            (static_cast<uint32_t>(BN >> 3) << 17) |
-                            (static_cast<uint32_t>(BM >> 4) << 24);
+// Instruction descriptors: int32 D, signed int8 A, B signed (weights
+// -1/0/+1) or unsigned (2-bit codes 0..3), both K-major, N = 256, M = 128.
+constexpr uint32_t kIdescShape = (2u << 4) | (1u << 7) |
+                                 (static_cast<uint32_t>(BN >> 3) << 17) |
+                                 (static_cast<uint32_t>(BM >> 4) << 24);
+constexpr uint32_t kIdescSignedB = kIdescShape | (1u << 10);
+constexpr uint32_t kIdescUnsignedB = kIdescShape;
 
 struct Smem {
   uint8_t* base;  // 1024-aligned
@@ -86,14 +90,29 @@ __device__ __forceinline__ uint4 unpack_word_s8(uint32_t w) {
                     prmt(t1, t3, 0x7632u) ^ 0x80808080u);
 }
 
-template <bool kAccOut>
+// One packed word -> its four 2-bit planes as unsigned codes, plane i in
+// word i: bytes (c(4t+i)) for t = 0..3. Matches activations whose 16-element
+// groups are stored transposed (element 4t + i at byte 4i + t).
+__device__ __forceinline__ uint4 unpack_word_planes(uint32_t w) {
+  return make_uint4(w & 0x03030303u, (w >> 2) & 0x03030303u, (w >> 4) & 0x03030303u,
+                    (w >> 6) & 0x03030303u);
+}
+
+// kPerm: activations come with transposed 16-element groups and per-row code
+// sums (from the quantiser of bitnet_linear); the weights then enter the MMA
+// as unsigned codes c = w + 2 and the epilogue subtracts 2 * rowsum[m].
+// Otherwise activations are in natural order and the weights are expanded to
+// signed int8 in natural order.
+template <bool kAccOut, bool kPerm>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_i8_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
                            const __grid_constant__ CUtensorMap tmap_w,
                            void* __restrict__ out,
                            const uint16_t* __restrict__ scale_act,
                            const float* __restrict__ scale_wt, int sw_len,
+                           const int32_t* __restrict__ rowsum,
                            int M, int N, int K) {
+  constexpr uint32_t kIdesc = kPerm ? kIdescUnsignedB : kIdescSignedB;
   extern __shared__ uint8_t smem_raw[];
   Smem sm;
   sm.base = reinterpret_cast<uint8_t*>(
@@ -206,6 +225,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int n_tile0 = (t % n_tiles) * BN;
       float sa = 0.0f;
       if (!kAccOut && m < M) sa = bf16_bits_to_f32(scale_act[m]);
+      const int corr = (kPerm && m < M) ? 2 * rowsum[m] : 0;
       const float sw0 = kAccOut ? 0.0f : scale_wt[0];
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
@@ -218,6 +238,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (m < M && n < N) {
           if constexpr (kAccOut) {
             int32_t* o = reinterpret_cast<int32_t*>(out) + static_cast<int64_t>(m) * N + n;
+            if constexpr (kPerm) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = static_cast<uint32_t>(static_cast<int>(v[j]) - corr);
+            }
             if (n + 32 <= N && (N & 3) == 0) {
 #pragma unroll
               for (int j = 0; j < 32; j += 4)
@@ -233,8 +257,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               const int nj = n + j;
               const float s0 = sw_len == 1 ? sw0 : (nj < N ? __ldg(scale_wt + nj) : 0.0f);
               const float s1 = sw_len == 1 ? sw0 : (nj + 1 < N ? __ldg(scale_wt + nj + 1) : 0.0f);
-              const float y0 = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j])), sa), s0);
-              const float y1 = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j + 1])), sa), s1);
+              const float y0 = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j]) - corr), sa), s0);
+              const float y1 = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j + 1]) - corr), sa), s1);
               h[j / 2] = static_cast<uint32_t>(f32_to_bf16_bits(y0)) |
                          (static_cast<uint32_t>(f32_to_bf16_bits(y1)) << 16);
             }
@@ -276,7 +300,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             // 16-byte chunk j of the row sits at chunk position j ^ (row % 8)
-            *reinterpret_cast<uint4*>(dst + ((j ^ sw) << 4)) = unpack_word_s8(pw[j]);
+            *reinterpret_cast<uint4*>(dst + ((j ^ sw) << 4)) =
+                kPerm ? unpack_word_planes(pw[j]) : unpack_word_s8(pw[j]);
           }
         }
         fence_proxy_async_smem();

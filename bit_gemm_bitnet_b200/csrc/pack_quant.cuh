@@ -114,4 +114,86 @@ __global__ void __launch_bounds__(kQuantThreads)
   if (tid == 0) sa[m] = f32_to_bf16_bits(rq.s);
 }
 
+// The same quantiser writing, for the tensor-core GEMM of bitnet_linear, each
+// 16-element group of a row transposed 4x4 (element 4t + i at byte 4i + t of
+// the group, the order in which the 2-bit planes of a packed weight word come
+// out) and the row's sum of codes. GPT > 0: the row is held in registers (GPT
+// groups per thread, K <= 16 * 256 * GPT); GPT == 0: two passes.
+template <int GPT>
+__global__ void __launch_bounds__(kQuantThreads)
+    quantize_rows_perm_kernel(int8_t* __restrict__ xq, uint16_t* __restrict__ sa,
+                              int32_t* __restrict__ rowsum, const uint16_t* __restrict__ x,
+                              int K) {
+  __shared__ uint32_t red[kQuantThreads / 32];
+  __shared__ int reds[kQuantThreads / 32];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int64_t m = blockIdx.x;
+  const uint4* row = reinterpret_cast<const uint4*>(x + m * K);
+  uint4* qrow = reinterpret_cast<uint4*>(xq + m * K);
+  const int ngroups = K / 16;
+  const int tid = threadIdx.x;
+
+  uint4 v[GPT > 0 ? GPT : 1][2];
+  uint32_t mb = 0;
+  if constexpr (GPT > 0) {
+#pragma unroll
+    for (int i = 0; i < GPT; ++i) {
+      const int g = tid + i * kQuantThreads;
+      if (g < ngroups) {
+        v[i][0] = ldg_stream_v4(row + 2 * g);
+        v[i][1] = ldg_stream_v4(row + 2 * g + 1);
+        mb = max(mb, max(absmax_bits8(v[i][0]), absmax_bits8(v[i][1])));
+      }
+    }
+  } else {
+    for (int g = tid; g < ngroups; g += kQuantThreads)
+      mb = max(mb, max(absmax_bits8(__ldg(row + 2 * g)), absmax_bits8(__ldg(row + 2 * g + 1))));
+  }
+  mb = __reduce_max_sync(0xFFFFFFFFu, mb);
+  if ((tid & 31) == 0) red[tid >> 5] = mb;
+  __syncthreads();
+  if (tid < 32) {
+    uint32_t t = tid < kQuantThreads / 32 ? red[tid] : 0u;
+    t = __reduce_max_sync(0xFFFFFFFFu, t);
+    if (tid == 0) red[0] = t;
+  }
+  __syncthreads();
+  const RowQuant rq = row_quant(bf16_bits_to_f32(red[0]));
+  int sum = 0;
+  auto emit = [&](int g, const uint4& a, const uint4& b) {
+    const uint2 lo = quant8(a, rq);
+    const uint2 hi = quant8(b, rq);
+    const uint32_t w0 = lo.x, w1 = lo.y, w2 = hi.x, w3 = hi.y;
+    sum += __dp4a(static_cast<int>(w0), 0x01010101, 0) + __dp4a(static_cast<int>(w1), 0x01010101, 0) +
+           __dp4a(static_cast<int>(w2), 0x01010101, 0) + __dp4a(static_cast<int>(w3), 0x01010101, 0);
+    // 4x4 byte transpose: out word i byte t = in word t byte i
+    const uint32_t t0 = __byte_perm(w0, w1, 0x5140u);
+    const uint32_t t1 = __byte_perm(w0, w1, 0x7362u);
+    const uint32_t t2 = __byte_perm(w2, w3, 0x5140u);
+    const uint32_t t3 = __byte_perm(w2, w3, 0x7362u);
+    qrow[g] = make_uint4(__byte_perm(t0, t2, 0x5410u), __byte_perm(t0, t2, 0x7632u),
+                         __byte_perm(t1, t3, 0x5410u), __byte_perm(t1, t3, 0x7632u));
+  };
+  if constexpr (GPT > 0) {
+#pragma unroll
+    for (int i = 0; i < GPT; ++i) {
+      const int g = tid + i * kQuantThreads;
+      if (g < ngroups) emit(g, v[i][0], v[i][1]);
+    }
+  } else {
+    for (int g = tid; g < ngroups; g += kQuantThreads)
+      emit(g, __ldg(row + 2 * g), __ldg(row + 2 * g + 1));
+  }
+  sum = __reduce_add_sync(0xFFFFFFFFu, sum);
+  if ((tid & 31) == 0) reds[tid >> 5] = sum;
+  __syncthreads();
+  if (tid == 0) {
+    int t = 0;
+    for (int w = 0; w < kQuantThreads / 32; ++w) t += reds[w];
+    rowsum[m] = t;
+    sa[m] = f32_to_bf16_bits(rq.s);
+  }
+}
+
 }  // namespace bitnet

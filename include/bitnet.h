@@ -112,8 +112,9 @@ bitnet_status bitnet_gemv_fused(uint16_t* out, const void* x, bitnet_dtype dt,
                                 int64_t K, void* stream);
 
 /* Workspace bitnet_linear needs for (M, K): 0 when it takes the fused GEMV
- * path, otherwise room for the int8 [M, K] activations and the bf16 [M]
- * scales, each 256-byte aligned. */
+ * path, otherwise room for the int8 [M, K] activations, the bf16 [M] scales
+ * and int32 [M] per-row sums of the codes, each 256-byte aligned. The layout
+ * inside the workspace is private to the library. */
 size_t bitnet_linear_workspace_bytes(int64_t M, int64_t K);
 
 /* One-shot BitLinear forward (bitnet_linear() on the bitnet-cpu page):

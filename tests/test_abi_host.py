@@ -42,8 +42,8 @@ def test_status_strings():
 def test_workspace_bytes():
     assert bn.bitnet_linear_workspace_bytes(1, 4096) == 0
     assert bn.bitnet_linear_workspace_bytes(15, 4096) == 0
-    assert bn.bitnet_linear_workspace_bytes(16, 4096) == 16 * 4096 + 256
-    assert bn.bitnet_linear_workspace_bytes(8192, 11008) == 8192 * 11008 + 16384
+    assert bn.bitnet_linear_workspace_bytes(16, 4096) == 16 * 4096 + 256 + 256
+    assert bn.bitnet_linear_workspace_bytes(8192, 11008) == 8192 * 11008 + 16384 + 32768
     # M * K over the fused GEMV's on-chip limit takes the split path
     assert bn.bitnet_linear_workspace_bytes(15, 16384) > 0
     assert bn.bitnet_linear_workspace_bytes(0, 4096) == 0

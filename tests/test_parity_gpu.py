@@ -252,3 +252,16 @@ def test_linear_workspace_errors():
                          ctypes.c_void_p(p.data_ptr()), ctypes.c_void_p(sw.data_ptr()), 1,
                          32, 64, 512, None, 0, None)
     assert st == bn.ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("M,K,N", [(130, 384, 300), (257, 2560, 520), (16, 11008, 256),
+                                   (200, 160, 64), (129, 4096, 4099)])
+def test_linear_split_path_ragged(M, K, N):
+    """M >= 16: quantise into the workspace, then the GEMM (tensor-core path
+    with transposed groups and row sums when K % 64 == 0, SIMT otherwise)."""
+    x = acts(98, M + K, M, K)
+    w = weights(98, N + K, N, K)
+    p = oracle.pack(w)
+    sw = synth.uniform_f32(synth.key(98, N, 3), N, 0.01, 0.1)
+    got = bn.bitnet_linear(to_dev(x, torch.bfloat16), to_dev(p), to_dev(sw))
+    assert_bf16_close(bf16_bits(got), oracle.linear(x, p, sw))
