@@ -4,13 +4,14 @@
 Default workload (one "step"): the BitNet-b1.58-2B decode sweep at M = 1 --
 30 layers x 7 BitLinears (Q, K, V, O, gate, up, down) plus the LM head, 211
 calls of the fused quantise + GEMV with fresh seeded weights per layer and a
-fresh activation row per call. The step is issued as the 211 C-ABI calls in
-order on one stream and replayed as a CUDA graph (programmatic dependent
-launch edges between the kernels). Metric: GB/s of algorithmic bytes
+fresh activation row per call. The calls are independent problems, so the
+step issues them round-robin on graph branches (programmatic dependent launch
+edges between consecutive kernels of a branch) and replays the CUDA graph. Metric: GB/s of algorithmic bytes
 (packed weights + bf16 activations + bf16 outputs + weight scales).
 
-Also reported: the prefill GEMM (M = 8192, K = 4096 -> N = 11008) in INT8
-TOPS against the dense INT8 tensor peak, and the LM-head GEMV alone.
+Also reported: the prefill workload (M in {2048, 8192} x four FFN shapes
+through bitnet_linear) in INT8 TOPS against the dense INT8 tensor peak, the
+LM-head GEMV alone, and the decode sweep in two dependent issue orders.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -55,6 +56,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--branches", type=int, default=16,
                     help="graph branches for the independent calls of a step")
+    ap.add_argument("--case", choices=("lm_head", "prefill", "decode_once"),
+                    help="profiling aid: run one small case a few times and exit "
+                         "(no JSON line); see profiles/ for the ncu commands")
     return ap.parse_args()
 
 
@@ -325,46 +329,69 @@ def lm_head_alone(bn, d, dev, reps=20):
 
 # ---------------------------------------------------------------- prefill
 
-def prefill(bn, dev, pk, reps=10):
-    M, K, N = 8192, 4096, 11008
-    x = synth.act_bf16(synth.key(W.W_PREFILL, 0, synth.T_ACT, 0), M, K)
-    w = synth.ternary(synth.key(W.W_PREFILL, 0, synth.T_WEIGHT, 0), N, K)
-    sw = synth.scale_wt(synth.key(W.W_PREFILL, 0, synth.T_SCALE_WT, 0))
-    xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
-    wp = bn.bitnet_pack_weights(torch.from_numpy(w).to(dev))
-    swd = torch.from_numpy(sw).to(dev)
-    xq, sa = bn.bitnet_quantize_act(xd)
-    out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    ws = torch.empty((bn.bitnet_linear_workspace_bytes(M, K),), dtype=torch.uint8, device=dev)
+def prefill(bn, dev, pk, reps=5):
+    """The prefill workload: M in {2048, 8192} x four FFN shapes through
+    bitnet_linear (per-token quantisation + tensor-core GEMM, bf16 out), each
+    timed with CUDA events with L2 flushed between repetitions. Also the public
+    bitnet_gemm on pre-quantised activations for the first shape."""
     flush = torch.empty((2 * L2_BYTES,), dtype=torch.uint8, device=dev)
-    tg, tl = [], []
-    for r in range(reps + 3):
-        flush.fill_(r & 0xFF)
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        e[0].record()
-        bn.bitnet_gemm(xq, wp, sa, swd, out=out)
-        e[1].record()
-        torch.cuda.synchronize()
-        flush.fill_((r + 1) & 0xFF)
-        f = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        f[0].record()
-        bn.bitnet_linear(xd, wp, swd, out=out, workspace=ws)
-        f[1].record()
-        torch.cuda.synchronize()
-        if r >= 3:
-            tg.append(e[0].elapsed_time(e[1]))
-            tl.append(f[0].elapsed_time(f[1]))
-    bn.bitnet_device_status()
-    ops = 2.0 * M * N * K
-    g_ms, l_ms = statistics.median(tg), statistics.median(tl)
-    tops = ops / g_ms / 1e9
     peak = pk["bf16_tflops"] * INT8_OVER_BF16
-    return {"M": M, "K": K, "N": N, "gemm_ms": g_ms, "gemm_tops": tops,
-            "linear_ms": l_ms, "linear_tops": ops / l_ms / 1e9,
+
+    def timed(fn):
+        ts = []
+        for r in range(reps + 2):
+            flush.fill_(r & 0xFF)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if r >= 2:
+                ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    Mmax = max(W.PREFILL_M)
+    cases, tot_ops, tot_ms = [], 0.0, 0.0
+    gemm_pub = None
+    for K, N in W.PREFILL_SHAPES:
+        x = synth.act_bf16(synth.key(W.W_PREFILL, Mmax, synth.T_ACT, K), Mmax, K)
+        w = synth.ternary(synth.key(W.W_PREFILL, Mmax, synth.T_WEIGHT, K), N, K)
+        sw = synth.scale_wt(synth.key(W.W_PREFILL, Mmax, synth.T_SCALE_WT, K))
+        xd_all = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+        del x
+        wp = bn.bitnet_pack_weights(torch.from_numpy(w).to(dev))
+        swd = torch.from_numpy(sw).to(dev)
+        for M in W.PREFILL_M:
+            xd = xd_all[:M]
+            out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty((bn.bitnet_linear_workspace_bytes(M, K),), dtype=torch.uint8,
+                             device=dev)
+            ms = timed(lambda: bn.bitnet_linear(xd, wp, swd, out=out, workspace=ws))
+            ops = 2.0 * M * N * K
+            cases.append({"M": M, "K": K, "N": N, "ms": ms, "tops": ops / ms / 1e9})
+            tot_ops += ops
+            tot_ms += ms
+            if gemm_pub is None and M == Mmax:
+                xq, sa = bn.bitnet_quantize_act(xd)
+                g_ms = timed(lambda: bn.bitnet_gemm(xq, wp, sa, swd, out=out))
+                gemm_pub = {"M": M, "K": K, "N": N, "ms": g_ms, "tops": ops / g_ms / 1e9,
+                            "frac": ops / g_ms / 1e9 / peak}
+                del xq, sa
+            del out, ws
+        del xd_all, wp
+    bn.bitnet_device_status()
+    tops = tot_ops / tot_ms / 1e9
+    return {"workload": "M in {2048, 8192} x (4096->11008, 11008->4096, 2560->6912, "
+                        "6912->2560) through bitnet_linear (quantise + GEMM)",
+            "tops": tops, "ms_total": tot_ms, "cases": cases,
             "roofline": {"bound": "tensor", "achieved": tops, "peak": peak, "unit": "TOPS",
                          "frac": tops / peak,
-                         "peak_source": f"{pk['source']} bf16 burst x {INT8_OVER_BF16:g} (int8/bf16 nominal)",
-                         "traffic": recorded_traffic("gemm_i8_tcgen05_kernel")}}
+                         "peak_source": f"{pk['source']} bf16 burst x {INT8_OVER_BF16:g} "
+                                        "(int8/bf16 nominal)",
+                         "kernel": "quantize_rows_perm_kernel + gemm_i8_tcgen05_kernel "
+                                   "(timed together)",
+                         "traffic": recorded_traffic("gemm_i8_tcgen05_kernel")},
+            "bitnet_gemm_natural_layout": gemm_pub}
 
 
 # ----------------------------------------------------------- CPU oracle
@@ -396,6 +423,36 @@ def cpu_baseline(seconds):
     return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"decode layer 0 (7 BitLinears, {nbytes // reps / 1e6:.1f} MB packed) x {reps}, "
                       f"M=1, columns split over {threads} threads, {dt:.1f} s"}
+
+
+# --------------------------------------------------------- profiling aid
+
+def run_case(bn, dev, case, reps=3):
+    """Small, self-contained invocations for ncu captures (one kernel kind,
+    a few launches, inputs larger than L2, well under a few GB)."""
+    if case == "decode_once":
+        d = build_decode(bn, dev, 0)
+        make_sweep(bn, d, "stream")()
+    elif case == "lm_head":
+        _, K, N = W.DECODE_2B_LM_HEAD
+        w = synth.ternary(synth.key(W.W_DECODE_2B, W.DECODE_2B_LAYERS, synth.T_WEIGHT, 7), N, K)
+        wp = bn.bitnet_pack_weights(torch.from_numpy(w).to(dev))
+        x = synth.act_bf16(synth.key(W.W_DECODE_2B, W.DECODE_2B_LAYERS, synth.T_ACT, 7), 1, K)
+        xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+        sw = torch.tensor([0.05], dtype=torch.float32, device=dev)
+        for _ in range(reps):
+            bn.bitnet_gemv_fused(xd, wp, sw)
+    else:
+        M, (K, N) = max(W.PREFILL_M), W.PREFILL_SHAPES[0]
+        x = synth.act_bf16(synth.key(W.W_PREFILL, M, synth.T_ACT, K), M, K)
+        w = synth.ternary(synth.key(W.W_PREFILL, M, synth.T_WEIGHT, K), N, K)
+        xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+        wp = bn.bitnet_pack_weights(torch.from_numpy(w).to(dev))
+        sw = torch.tensor([0.05], dtype=torch.float32, device=dev)
+        for _ in range(reps):
+            bn.bitnet_linear(xd, wp, sw)
+    torch.cuda.synchronize()
+    bn.bitnet_device_status()
 
 
 # ----------------------------------------------------------------- main
@@ -438,6 +495,9 @@ def main():
         raise SystemExit("bench.py needs a CUDA device")
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    if args.case:
+        run_case(bn, dev, args.case)
+        return 0
 
     pg = None
     if world > 1:
@@ -518,7 +578,7 @@ def main():
                 "gbs": d["bytes"] * world * args.steps / (other[o] / 1e3) / 1e9}
             for o in ("layer", "stream")},
         "lm_head_alone": {**lm, "frac": lm["gbs"] / pk["hbm_gbs"]},
-        "prefill_gemm": pre,
+        "prefill": pre,
     }
     print(json.dumps(line))
     if pg is not None:
