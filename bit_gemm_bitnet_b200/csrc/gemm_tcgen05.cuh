@@ -3,14 +3,14 @@
 // fused. Persistent: one CTA per SM walks the output tiles.
 //
 // Tile: 128 rows of x_q (MMA M) x 256 weight rows (MMA N) x 128 K per stage.
-// Warp roles (384 threads):
+// Warp roles (512 threads):
 //   warp 0      TMA producer: x_q tile (128-byte swizzle) and the packed
 //               weight tile (32 bytes per row) for each stage;
 //   warp 1      TMEM owner and MMA issuer (one thread): 4 MMAs of K = 32 per
 //               stage into a double-buffered 128 x 256 int32 accumulator;
 //   warps 4-7   epilogue: tcgen05.ld of the accumulator, fp32 scaling,
 //               bf16 stores (or the raw int32 for the test hook);
-//   warps 8-11  unpack: 2-bit codes -> int8 weights written into the
+//   warps 8-15  unpack: 2-bit codes -> int8 weights written into the
 //               128-byte-swizzled K-major layout the MMA reads (signed
 //               weights in natural order, or the unsigned code planes when
 //               the activations come with transposed 16-element groups).
@@ -31,7 +31,8 @@ constexpr int WU_BYTES = BN * BK;       // 32 KB, unpacked int8 weights
 constexpr int WP_BYTES = BN * BK / 4;   //  8 KB, packed weights
 constexpr int STAGE_BYTES = X_BYTES + WU_BYTES + WP_BYTES;
 constexpr int TX_BYTES = X_BYTES + WP_BYTES;
-constexpr int NUM_THREADS = 384;
+constexpr int NUM_THREADS = 512;
+constexpr int UNPACK_WARPS = 8;     // warps 8-15
 constexpr int TMEM_COLS = 512;          // 2 accumulators x 256 columns
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + BAR_BYTES;
@@ -129,7 +130,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(sm.full(s), 1);
-      mbar_init(sm.unpacked(s), 4);
+      mbar_init(sm.unpacked(s), UNPACK_WARPS);
       mbar_init(sm.empty(s), 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -279,7 +280,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp >= 8) {
     // -------------------------------------------------------------- unpack
-    const int u = threadIdx.x - 256;  // 0..127: weight rows u and u + 128
+    // 256 threads, each unpacking two half rows per stage: half row hr
+    // (row hr / 2, 16 packed bytes) is read with one conflict-free 16-byte
+    // load (consecutive lanes read consecutive 16-byte pieces).
+    const int u = threadIdx.x - 256;  // 0..255
     uint32_t it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
@@ -290,18 +294,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint8_t* wp = sm.wp(s);
         uint8_t* wu = sm.wu(s);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int r = u + 128 * h;
-          const uint4 p0 = *reinterpret_cast<const uint4*>(wp + r * 32);
-          const uint4 p1 = *reinterpret_cast<const uint4*>(wp + r * 32 + 16);
-          const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+        for (int i = 0; i < 2; ++i) {
+          const int hr = u + 256 * i;
+          const int r = hr >> 1, h = hr & 1;
+          const uint4 p = *reinterpret_cast<const uint4*>(wp + hr * 16);
+          const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
           uint8_t* dst = wu + r * 128;
           const int sw = r & 7;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
+          for (int jj = 0; jj < 4; ++jj) {
             // 16-byte chunk j of the row sits at chunk position j ^ (row % 8)
+            const int j = 4 * h + jj;
             *reinterpret_cast<uint4*>(dst + ((j ^ sw) << 4)) =
-                kPerm ? unpack_word_planes(pw[j]) : unpack_word_s8(pw[j]);
+                kPerm ? unpack_word_planes(pw[jj]) : unpack_word_s8(pw[jj]);
           }
         }
         fence_proxy_async_smem();
