@@ -137,10 +137,17 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def source_hash():
+KERNEL_SOURCES = {
+    "gemv_kernel": ("common.cuh", "pack_quant.cuh", "gemv.cuh"),
+    "gemm_i8_tcgen05_kernel": ("common.cuh", "pack_quant.cuh", "gemm_tcgen05.cuh"),
+}
+
+
+def source_hash(kernel):
+    """Hash of the device sources a kernel is built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_gemm_bitnet_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -148,17 +155,17 @@ def source_hash():
 
 
 def recorded_traffic(kernel):
-    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if
-    the kernel sources are unchanged since it was taken; else None."""
+    """DRAM bytes (read + write) of `kernel` from the committed ncu summary
+    (profiles/ncu_traffic.json), if the kernel's sources are unchanged since
+    the counters were taken; else None."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        rec = json.load(f)
-    if rec.get("source_hash") != source_hash():
+        rec = json.load(f).get(kernel)
+    if rec is None or rec.get("source_hash") != source_hash(kernel):
         return None
-    k = rec.get("kernels", {}).get(kernel)
-    return None if k is None else k.get("bytes_per_launch")
+    return rec.get("bytes")
 
 
 # ---------------------------------------------------------- decode sweep
@@ -565,7 +572,8 @@ def main():
                      "unit": "GB/s", "frac": per_rank_gbs / pk["hbm_gbs"],
                      "peak_source": f"{pk['source']} hbm_gbs",
                      "kernel": "gemv_kernel (all 211 launches of the step)",
-                     "traffic": recorded_traffic("gemv_kernel")},
+                     "traffic": recorded_traffic("gemv_kernel"),
+                     "traffic_per": "one step (211 launches), as achieved"},
         "cpu_baseline": cb,
         "e2e": {"value": e2e_val, "unit": UNIT,
                 "h2d_bytes_per_step": int(d["x_host"].numel() * 2),
