@@ -168,6 +168,26 @@ def recorded_traffic(kernel):
     return rec.get("bytes")
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank device times over all ranks (the job is
+    as slow as its slowest rank)."""
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def whole_job_gbs(bytes_per_step, world, steps, max_ms):
+    """Weak scaling: every rank moves bytes_per_step per step."""
+    return bytes_per_step * world * steps / (max_ms / 1e3) / 1e9
+
+
+def activation_variant(variant, rank):
+    """Generator variant of a call's activation row on `rank`: each rank
+    decodes its own tokens over the same weights."""
+    return variant + 16 * rank
+
+
 # ---------------------------------------------------------- decode sweep
 
 def sweep_calls():
@@ -200,7 +220,8 @@ def build_decode(bn, dev, rank):
     off = 0
     for layer, variant, K, N in calls:
         xv[off:off + K] = synth.act_bf16(
-            synth.key(W.W_DECODE_2B, layer, synth.T_ACT, variant + 16 * rank), 1, K)[0]
+            synth.key(W.W_DECODE_2B, layer, synth.T_ACT, activation_variant(variant, rank)),
+            1, K)[0]
         off += K
     x_dev = x_host.to(dev)
     out_dev = torch.empty((outs_total,), dtype=torch.bfloat16, device=dev)
@@ -543,15 +564,13 @@ def main():
     bn.bitnet_device_status()
 
     if pg is not None:
-        t = torch.tensor([total_ms, e2e_ms, other["layer"], other["stream"]],
-                         dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
-        other = {"layer": float(t[2]), "stream": float(t[3])}
+        total_ms, e2e_ms, lay, strm = max_over_ranks(
+            [total_ms, e2e_ms, other["layer"], other["stream"]], dev)
+        other = {"layer": lay, "stream": strm}
 
     ms_step = total_ms / args.steps
-    value = d["bytes"] * world * args.steps / (total_ms / 1e3) / 1e9
-    e2e_val = d["bytes"] * world * args.steps / (e2e_ms / 1e3) / 1e9
+    value = whole_job_gbs(d["bytes"], world, args.steps, total_ms)
+    e2e_val = whole_job_gbs(d["bytes"], world, args.steps, e2e_ms)
     per_rank_gbs = d["bytes"] / (ms_step / 1e3) / 1e9
     clocks = clk.summary()
     lm = lm_head_alone(bn, d, dev)
@@ -583,7 +602,7 @@ def main():
         "step_ms_min_median": [min(per), statistics.median(per)],
         "issue_orders": {
             o: {"ms_per_step": other[o] / args.steps,
-                "gbs": d["bytes"] * world * args.steps / (other[o] / 1e3) / 1e9}
+                "gbs": whole_job_gbs(d["bytes"], world, args.steps, other[o])}
             for o in ("layer", "stream")},
         "lm_head_alone": {**lm, "frac": lm["gbs"] / pk["hbm_gbs"]},
         "prefill": pre,
