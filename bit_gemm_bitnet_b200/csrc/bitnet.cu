@@ -190,8 +190,8 @@ bitnet_status launch_gemv_mb(int mb, int rw, const GemvParams& p, int gy, size_t
 template <bool WIDE, bool PREQ>
 bitnet_status launch_gemv_cw(int cw, int mb, int rw, const GemvParams& p, int gy, size_t smem,
                              int sms, cudaStream_t st) {
-  (void)cw;  // one CTA shape today: 16 consumer warps
-  return launch_gemv_mb<16, WIDE, PREQ>(mb, rw, p, gy, smem, sms, st);
+  if (cw == 16) return launch_gemv_mb<16, WIDE, PREQ>(mb, rw, p, gy, smem, sms, st);
+  return launch_gemv_mb<8, WIDE, PREQ>(mb, rw, p, gy, smem, sms, st);
 }
 
 int bucket_of(int m) { return m <= 1 ? 1 : m <= 2 ? 2 : m <= 4 ? 4 : m <= 8 ? 8 : 16; }
@@ -229,10 +229,15 @@ bitnet_status run_gemv(GemvParams p, bool preq, cudaStream_t st) {
     while (r > 1 && gemv_smem(qrows, K, warps, r, 1) > kSmemLimit) r /= 2;
     return r;
   };
-  // 16 consumer warps: with fewer, the quantisation prologue of a small
-  // layer takes more dependent load rounds per thread and the layer slows.
-  const int cw = 16;
-  const int rw = pick_rw(cw);
+  // 16 consumer warps for large layers (latency hiding in the steady state);
+  // 8 for small ones, whose CTAs are short-lived: smaller CTAs let the
+  // kernels of independent calls share the SMs.
+  int cw = 16;
+  int rw = pick_rw(cw);
+  if ((p.N + cw * rw - 1) / (cw * rw) < 2 * static_cast<int64_t>(dev->sms)) {
+    cw = 8;
+    rw = pick_rw(cw);
+  }
   const size_t stage = align128(static_cast<size_t>(cw * rw) * KB);
   // ring depth: no deeper than the row blocks one CTA will see
   const int64_t nblocks = (p.N + cw * rw - 1) / (cw * rw);
