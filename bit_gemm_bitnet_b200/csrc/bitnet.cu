@@ -234,7 +234,10 @@ bitnet_status run_gemv(GemvParams p, bool preq, cudaStream_t st) {
   // kernels of independent calls share the SMs.
   int cw = 16;
   int rw = pick_rw(cw);
-  if ((p.N + cw * rw - 1) / (cw * rw) < 2 * static_cast<int64_t>(dev->sms)) {
+  // (only while the prologue stays short: at most ~3 activation quads per
+  // consumer thread and activation row)
+  if ((p.N + cw * rw - 1) / (cw * rw) < 2 * static_cast<int64_t>(dev->sms) &&
+      K / 4 <= 3 * 8 * 32) {
     cw = 8;
     rw = pick_rw(cw);
   }
