@@ -6,7 +6,7 @@
 
 #include "../../include/bitnet.h"
 #include "common.cuh"
-#include "gemm_tcgen05.cuh"
+#include "gemm_ts.cuh"
 #include "gemv.cuh"
 #include "pack_quant.cuh"
 
@@ -296,24 +296,23 @@ bitnet_status run_gemm(void* out, bool acc_out, const int8_t* xq, const uint8_t*
   bitnet_status s = device_info(&dev);
   if (s != BITNET_OK) return s;
   CUtensorMap mx, mw;
-  if (!make_map_u8(&mx, xq, M, K, K, gemm::BM, gemm::BK, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_u8(&mw, wp, N, K / 4, K / 4, gemm::BN, gemm::BK / 4,
-                   CU_TENSOR_MAP_SWIZZLE_NONE))
+  if (!make_map_u8(&mx, xq, M, K, K, ts::BX, ts::BK, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_u8(&mw, wp, N, K / 4, K / 4, ts::BW, ts::BK / 4, CU_TENSOR_MAP_SWIZZLE_NONE))
     return BITNET_ERR_CUDA;
-  const int64_t tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + gemm::BN - 1) / gemm::BN);
+  const int64_t tiles = ((M + ts::BX - 1) / ts::BX) * ((N + ts::BW - 1) / ts::BW);
   if (tiles > INT32_MAX) return BITNET_ERR_SHAPE;
   const int grid = static_cast<int>(tiles < dev->sms ? tiles : dev->sms);
   auto go = [&](auto kernel) -> bitnet_status {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             gemm::SMEM_BYTES) != cudaSuccess)
+                             ts::SMEM_BYTES) != cudaSuccess)
       return BITNET_ERR_CUDA;
-    return launch_pdl(kernel, dim3(grid), dim3(gemm::NUM_THREADS), gemm::SMEM_BYTES, st, mx,
-                      mw, out, sa, sw, static_cast<int>(sw_len), rowsum, static_cast<int>(M),
+    return launch_pdl(kernel, dim3(grid), dim3(ts::NUM_THREADS), ts::SMEM_BYTES, st, mx, mw,
+                      out, sa, sw, static_cast<int>(sw_len), rowsum, static_cast<int>(M),
                       static_cast<int>(N), static_cast<int>(K));
   };
-  if (acc_out) return go(gemm::gemm_i8_tcgen05_kernel<true, false>);
-  if (perm) return go(gemm::gemm_i8_tcgen05_kernel<false, true>);
-  return go(gemm::gemm_i8_tcgen05_kernel<false, false>);
+  if (acc_out) return go(ts::gemm_i8_ts_kernel<true, false>);
+  if (perm) return go(ts::gemm_i8_ts_kernel<false, true>);
+  return go(ts::gemm_i8_ts_kernel<false, false>);
 }
 
 bitnet_status run_quantize(int8_t* xq, uint16_t* sa, const uint16_t* x, int64_t M,

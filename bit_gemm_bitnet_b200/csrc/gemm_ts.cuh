@@ -1,0 +1,298 @@
+// Batched ternary x INT8 GEMM on the 5th-generation tensor cores with the
+// weights as the tensor-memory operand (tcgen05.mma kind::i8, A from TMEM,
+// B from shared memory), int32 accumulators in TMEM, scale epilogue fused.
+//
+// D[n, m] = sum_k W[n, k] * x_q[m, k]: the MMA's M dimension is 128 weight
+// rows (TMEM lanes), its N dimension BX = 192 activation rows. Unpacked
+// weights go registers -> TMEM (tcgen05.st) and never touch shared memory, so
+// per 128-K stage the shared-memory traffic is the activation tile (written
+// by TMA, read by the MMA) and the small packed weight tile.
+//
+// TMEM (512 columns): two 192-column accumulators + four 32-column A stages.
+// Warp roles (512 threads), persistent (one CTA per SM):
+//   warp 0      TMA producer (x tile, 128-byte swizzle; packed weight tile)
+//   warp 1      TMEM owner, MMA issuer (one thread)
+//   warps 4-7   epilogue: tcgen05.ld, fp32 scales, bf16 (or int32) stores
+//   warps 8-15  unpack: packed codes -> int8 -> tcgen05.st into the A stage
+//               (two warps per TMEM sub-partition, 16 columns each)
+// Waits are bounded like the other kernels of this library.
+#pragma once
+#include "common.cuh"
+
+namespace bitnet {
+namespace ts {
+
+constexpr int BW = 128;                 // weight rows per tile (MMA M)
+constexpr int BX = 192;                 // activation rows per tile (MMA N)
+constexpr int BK = 128;                 // K per stage
+constexpr int STAGES = 4;
+constexpr int X_BYTES = BX * BK;        // 24 KB
+constexpr int WP_BYTES = BW * BK / 4;   //  4 KB
+constexpr int STAGE_BYTES = X_BYTES + WP_BYTES;
+constexpr int NUM_THREADS = 512;
+constexpr int TMEM_COLS = 512;
+constexpr int A_COL0 = 2 * BX;          // first A-stage column
+constexpr int A_COLS = BK / 4;          // 32 columns per A stage
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment");
+static_assert(A_COL0 + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
+static_assert(SMEM_BYTES <= 232448, "too much shared memory");
+
+// int32 D, A (weights) unsigned code planes or signed int8, B signed int8,
+// both K-major, N = BX, M = BW.
+constexpr uint32_t kIdescShape = (2u << 4) | (1u << 10) |
+                                 (static_cast<uint32_t>(BX >> 3) << 17) |
+                                 (static_cast<uint32_t>(BW >> 4) << 24);
+constexpr uint32_t kIdescUnsignedA = kIdescShape;
+constexpr uint32_t kIdescSignedA = kIdescShape | (1u << 7);
+
+struct Smem {
+  uint8_t* base;  // 1024-aligned
+  __device__ uint8_t* x(int s) const { return base + s * STAGE_BYTES; }
+  __device__ uint8_t* wp(int s) const { return base + s * STAGE_BYTES + X_BYTES; }
+  __device__ uint64_t* bars() const {
+    return reinterpret_cast<uint64_t*>(base + STAGES * STAGE_BYTES);
+  }
+  __device__ uint32_t full(int s) const { return smem_u32(bars() + s); }
+  __device__ uint32_t unpacked(int s) const { return smem_u32(bars() + STAGES + s); }
+  __device__ uint32_t empty(int s) const { return smem_u32(bars() + 2 * STAGES + s); }
+  __device__ uint32_t tfull(int a) const { return smem_u32(bars() + 3 * STAGES + a); }
+  __device__ uint32_t tempty(int a) const { return smem_u32(bars() + 3 * STAGES + 2 + a); }
+  __device__ uint32_t drain() const { return smem_u32(bars() + 3 * STAGES + 4); }
+  __device__ uint32_t* tmem_slot() const {
+    return reinterpret_cast<uint32_t*>(bars() + 3 * STAGES + 5);
+  }
+  __device__ int* abort_flag() const {
+    return reinterpret_cast<int*>(bars() + 3 * STAGES + 6);
+  }
+};
+
+// Packed word -> its four unsigned 2-bit code planes (plane i in word i).
+__device__ __forceinline__ void planes_of(uint32_t w, uint32_t* o) {
+  o[0] = w & 0x03030303u;
+  o[1] = (w >> 2) & 0x03030303u;
+  o[2] = (w >> 4) & 0x03030303u;
+  o[3] = (w >> 6) & 0x03030303u;
+}
+
+// Packed word -> 16 signed int8 weights in element order (4 words).
+__device__ __forceinline__ void signed_of(uint32_t w, uint32_t* o) {
+  const uint32_t e0 = ((w & 0x03030303u) | 0x80808080u) - 0x02020202u;
+  const uint32_t e1 = (((w >> 2) & 0x03030303u) | 0x80808080u) - 0x02020202u;
+  const uint32_t e2 = (((w >> 4) & 0x03030303u) | 0x80808080u) - 0x02020202u;
+  const uint32_t e3 = (((w >> 6) & 0x03030303u) | 0x80808080u) - 0x02020202u;
+  const uint32_t t0 = prmt(e0, e1, 0x5140u);
+  const uint32_t t1 = prmt(e0, e1, 0x7362u);
+  const uint32_t t2 = prmt(e2, e3, 0x5140u);
+  const uint32_t t3 = prmt(e2, e3, 0x7362u);
+  o[0] = prmt(t0, t2, 0x5410u) ^ 0x80808080u;
+  o[1] = prmt(t0, t2, 0x7632u) ^ 0x80808080u;
+  o[2] = prmt(t1, t3, 0x5410u) ^ 0x80808080u;
+  o[3] = prmt(t1, t3, 0x7632u) ^ 0x80808080u;
+}
+
+// kPerm: activations with transposed 16-element groups plus per-row code
+// sums; weights enter as unsigned code planes and the epilogue subtracts
+// 2 * rowsum[m]. Otherwise natural order and signed weights.
+template <bool kAccOut, bool kPerm>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_i8_ts_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                      const __grid_constant__ CUtensorMap tmap_w, void* __restrict__ out,
+                      const uint16_t* __restrict__ scale_act,
+                      const float* __restrict__ scale_wt, int sw_len,
+                      const int32_t* __restrict__ rowsum, int M, int N, int K) {
+  constexpr uint32_t kIdesc = kPerm ? kIdescUnsignedA : kIdescSignedA;
+  extern __shared__ uint8_t smem_raw[];
+  Smem sm;
+  sm.base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int x_tiles = (M + BX - 1) / BX;
+  const int w_tiles = (N + BW - 1) / BW;
+  const int num_tiles = x_tiles * w_tiles;
+  const int kblocks = (K + BK - 1) / BK;
+  volatile int* abort = sm.abort_flag();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(sm.full(s), 1);
+      mbar_init(sm.unpacked(s), 8);
+      mbar_init(sm.empty(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(sm.tfull(a), 1);
+      mbar_init(sm.tempty(a), 4);
+    }
+    mbar_init(sm.drain(), 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmap_x);
+    tma_prefetch_desc(&tmap_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(sm.tmem_slot()), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *sm.tmem_slot();
+
+  pdl_launch_dependents();
+  pdl_wait();  // x_q, scales and row sums may come from the previous kernel
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int m0 = (t / w_tiles) * BX;
+        const int n0 = (t % w_tiles) * BW;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait(sm.empty(s), ph ^ 1u, abort)) { ok = false; break; }
+          mbar_arrive_expect_tx(sm.full(s), STAGE_BYTES);
+          tma_load_2d(smem_u32(sm.x(s)), &tmap_x, sm.full(s), kb * BK, m0);
+          tma_load_2d(smem_u32(sm.wp(s)), &tmap_w, sm.full(s), kb * (BK / 4), n0);
+        }
+      }
+      const uint32_t first = it > STAGES ? it - STAGES : 0u;
+      for (uint32_t j = first; j < it; ++j)
+        mbar_wait_drain(sm.full(j % STAGES), (j / STAGES) & 1u);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, local = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
+        const int a = local & 1;
+        const uint32_t aph = (local >> 1) & 1u;
+        if (!mbar_wait(sm.tempty(a), aph ^ 1u, abort)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * BX);
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait(sm.full(s), ph, abort) ||
+              !mbar_wait(sm.unpacked(s), ph, abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + s * A_COLS);
+          const uint64_t bdesc = smem_desc_sw128(smem_u32(sm.x(s)));
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k) {
+            // 32 K bytes: 8 TMEM columns of A, +32 bytes inside B's swizzle atom
+            mma_i8_tmem_a(d_tmem, a_tmem + 8u * k, bdesc + 2u * k, kIdesc,
+                          (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(sm.empty(s));
+        }
+        if (ok) mma_commit(sm.tfull(a));
+      }
+      mma_commit(sm.drain());
+      mbar_wait_drain(sm.drain(), 0u);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    uint32_t local = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
+      const int a = local & 1;
+      const uint32_t aph = (local >> 1) & 1u;
+      const int m0 = (t / w_tiles) * BX;
+      const int n = (t % w_tiles) * BW + quarter * 32 + lane;
+      float swn = 0.0f;
+      if (!kAccOut && n < N) swn = scale_wt[sw_len == 1 ? 0 : n];
+      if (!mbar_wait(sm.tfull(a), aph, abort)) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < BX / 32; ++c) {
+        // lane j fetches the scalars of activation row m0 + 32c + j; they
+        // reach the other lanes by shuffles
+        const int ml = m0 + c * 32 + lane;
+        const float sa_l = (!kAccOut && ml < M) ? bf16_bits_to_f32(scale_act[ml]) : 0.0f;
+        const int corr_l = (kPerm && ml < M) ? 2 * rowsum[ml] : 0;
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                               static_cast<uint32_t>(a * BX + c * 32),
+                           v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float sa_j = __shfl_sync(0xFFFFFFFFu, sa_l, j);
+          const int corr_j = __shfl_sync(0xFFFFFFFFu, corr_l, j);
+          const int m = m0 + c * 32 + j;
+          if (m < M && n < N) {
+            const int acc = static_cast<int>(v[j]) - corr_j;
+            if constexpr (kAccOut) {
+              reinterpret_cast<int32_t*>(out)[static_cast<int64_t>(m) * N + n] = acc;
+            } else {
+              const float y = __fmul_rn(__fmul_rn(__int2float_rn(acc), sa_j), swn);
+              reinterpret_cast<uint16_t*>(out)[static_cast<int64_t>(m) * N + n] =
+                  f32_to_bf16_bits(y);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.tempty(a));
+    }
+  } else if (warp >= 8) {
+    // -------------------------------------------------------------- unpack
+    // warp -> TMEM sub-partition warp % 4 (weight rows 32 * (warp % 4) ...)
+    // and half (warp - 8) / 4 of the stage's 32 columns (64 K elements)
+    const int sub = warp & 3;
+    const int half = (warp - 8) >> 2;
+    const int r = sub * 32 + lane;  // weight row within the tile
+    const uint32_t lane_base = static_cast<uint32_t>(sub * 32) << 16;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1u;
+        if (!mbar_wait(sm.full(s), ph, abort)) { ok = false; break; }
+        const uint4 p = *reinterpret_cast<const uint4*>(sm.wp(s) + r * 32 + half * 16);
+        uint32_t o[16];
+        if constexpr (kPerm) {
+          planes_of(p.x, o + 0);
+          planes_of(p.y, o + 4);
+          planes_of(p.z, o + 8);
+          planes_of(p.w, o + 12);
+        } else {
+          signed_of(p.x, o + 0);
+          signed_of(p.y, o + 4);
+          signed_of(p.z, o + 8);
+          signed_of(p.w, o + 12);
+        }
+        tmem_st_32x32b_x16(tmem_base + lane_base +
+                               static_cast<uint32_t>(A_COL0 + s * A_COLS + half * 16),
+                           o);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sm.unpacked(s));
+      }
+    }
+  }
+
+  // ------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace ts
+}  // namespace bitnet
