@@ -34,7 +34,8 @@ constexpr int TMEM_COLS = 512;
 constexpr int A_COL0 = 2 * BX;          // first A-stage column
 constexpr int A_COLS = BK / 4;          // 32 columns per A stage
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+constexpr int EPI_BYTES = 4 * 32 * 32 * 4;  // per epilogue warp: one 32 x 32 chunk
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + EPI_BYTES;
 static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment");
 static_assert(A_COL0 + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
 static_assert(SMEM_BYTES <= 232448, "too much shared memory");
@@ -65,6 +66,11 @@ struct Smem {
   }
   __device__ int* abort_flag() const {
     return reinterpret_cast<int*>(bars() + 3 * STAGES + 6);
+  }
+  // warp-private staging of one 32 (activation rows) x 32 (weight rows)
+  // output chunk, 4 bytes per element (bf16 outputs use the first half)
+  __device__ uint8_t* epi(int quarter) const {
+    return base + STAGES * STAGE_BYTES + BAR_BYTES + quarter * (32 * 32 * 4);
   }
 };
 
@@ -224,19 +230,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                static_cast<uint32_t>(a * BX + c * 32),
                            v);
         tmem_ld_wait();
+        // the chunk goes through this warp's staging patch: lane = weight
+        // row n writes column `lane` of 32 activation rows, then the warp
+        // writes each activation row's 32 outputs with 16-byte stores
+        uint8_t* stg = sm.epi(quarter);
+        __syncwarp();  // the previous chunk's reads of the patch are done
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const float sa_j = __shfl_sync(0xFFFFFFFFu, sa_l, j);
           const int corr_j = __shfl_sync(0xFFFFFFFFu, corr_l, j);
+          const int acc = static_cast<int>(v[j]) - corr_j;
+          if constexpr (kAccOut) {
+            reinterpret_cast<int32_t*>(stg)[j * 32 + lane] = acc;
+          } else {
+            const float y = __fmul_rn(__fmul_rn(__int2float_rn(acc), sa_j), swn);
+            reinterpret_cast<uint16_t*>(stg)[j * 32 + lane] = f32_to_bf16_bits(y);
+          }
+        }
+        __syncwarp();
+        const int nb = (t % w_tiles) * BW + quarter * 32;  // first weight row of the chunk
+        constexpr int ebytes = kAccOut ? 4 : 2;
+        constexpr int per_row = 32 * ebytes / 16;          // 16-byte pieces per row
+#pragma unroll
+        for (int i = 0; i < per_row; ++i) {
+          const int piece = lane + 32 * i;  // 32 rows x per_row pieces
+          const int j = piece / per_row;
+          const int col = (piece % per_row) * (16 / ebytes);  // first n within the chunk
           const int m = m0 + c * 32 + j;
-          if (m < M && n < N) {
-            const int acc = static_cast<int>(v[j]) - corr_j;
-            if constexpr (kAccOut) {
-              reinterpret_cast<int32_t*>(out)[static_cast<int64_t>(m) * N + n] = acc;
+          const int n0 = nb + col;
+          if (m < M) {
+            uint8_t* dst = reinterpret_cast<uint8_t*>(out) + (static_cast<int64_t>(m) * N + n0) * ebytes;
+            const uint8_t* src = stg + (j * 32 + col) * ebytes;
+            if (n0 + 16 / ebytes <= N && ((N * ebytes) & 15) == 0) {
+              *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
             } else {
-              const float y = __fmul_rn(__fmul_rn(__int2float_rn(acc), sa_j), swn);
-              reinterpret_cast<uint16_t*>(out)[static_cast<int64_t>(m) * N + n] =
-                  f32_to_bf16_bits(y);
+              for (int e = 0; e < 16 / ebytes && n0 + e < N; ++e)
+                for (int b = 0; b < ebytes; ++b) dst[e * ebytes + b] = src[e * ebytes + b];
             }
           }
         }
