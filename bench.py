@@ -139,7 +139,7 @@ class ClockSampler:
 
 KERNEL_SOURCES = {
     "gemv_kernel": ("common.cuh", "pack_quant.cuh", "gemv.cuh"),
-    "gemm_i8_tcgen05_kernel": ("common.cuh", "pack_quant.cuh", "gemm_tcgen05.cuh"),
+    "gemm_i8_ts_kernel": ("common.cuh", "pack_quant.cuh", "gemm_ts.cuh"),
 }
 
 
@@ -416,9 +416,9 @@ def prefill(bn, dev, pk, reps=5):
                          "frac": tops / peak,
                          "peak_source": f"{pk['source']} bf16 burst x {INT8_OVER_BF16:g} "
                                         "(int8/bf16 nominal)",
-                         "kernel": "quantize_rows_perm_kernel + gemm_i8_tcgen05_kernel "
+                         "kernel": "quantize_rows_perm_kernel + gemm_i8_ts_kernel "
                                    "(timed together)",
-                         "traffic": recorded_traffic("gemm_i8_tcgen05_kernel")},
+                         "traffic": recorded_traffic("gemm_i8_ts_kernel")},
             "bitnet_gemm_natural_layout": gemm_pub}
 
 

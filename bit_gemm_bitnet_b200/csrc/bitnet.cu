@@ -264,7 +264,7 @@ bitnet_status run_gemv(GemvParams p, bool preq, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------- GEMM
-bool gemm_tcgen05_ok(const int8_t* xq, const uint8_t* wp, int64_t K) {
+bool gemm_tc_ok(const int8_t* xq, const uint8_t* wp, int64_t K) {
   // TMA: row pitches must be multiples of 16 bytes (K/4 for the packed
   // weights) and base addresses 16-byte aligned.
   return (K % 64) == 0 && aligned(xq, 16) && aligned(wp, 16);
@@ -277,7 +277,7 @@ bitnet_status run_gemm(void* out, bool acc_out, const int8_t* xq, const uint8_t*
                        int64_t N, int64_t K, cudaStream_t st, bool perm = false,
                        const int32_t* rowsum = nullptr) {
   if (M == 0 || N == 0) return BITNET_OK;
-  if (!gemm_tcgen05_ok(xq, wp, K)) {
+  if (!gemm_tc_ok(xq, wp, K)) {
     if (perm) return BITNET_ERR_SHAPE;  // callers only ask for perm when it applies
     GemvParams p = {};
     if (acc_out) p.acc_out = static_cast<int32_t*>(out);
@@ -559,7 +559,7 @@ bitnet_status bitnet_linear(uint16_t* out, const void* x, bitnet_dtype dt,
                                                align256(static_cast<size_t>(M) * 2));
   cudaStream_t st = as_stream(stream);
   const uint16_t* xb = static_cast<const uint16_t*>(x);
-  if (gemm_tcgen05_ok(xq, w_packed, K)) {
+  if (gemm_tc_ok(xq, w_packed, K)) {
     // tensor-core path: transposed groups + row sums, weights as code planes
     s = run_quantize_perm(xq, sa, rowsum, xb, M, K, st);
     if (s != BITNET_OK) return s;
