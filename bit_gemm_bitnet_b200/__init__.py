@@ -28,8 +28,16 @@ EXPORTS = (
     "bitnet_pack_weights", "bitnet_quantize_act", "bitnet_gemm",
     "bitnet_gemv_fused", "bitnet_linear_workspace_bytes", "bitnet_linear",
     "bitnet_device_status", "bitnet_status_string", "bitnet_gemm_acc_i32",
-    "bitnet_gemv_fused_debug", "bitnet_linear_noalloc",
+    "bitnet_gemv_fused_debug", "bitnet_linear_noalloc", "bitnet_gemv_fused_grouped",
 )
+
+
+class GemvProblem(ctypes.Structure):
+    """bitnet_gemv_problem of include/bitnet.h."""
+    _fields_ = [("out", ctypes.c_void_p), ("x", ctypes.c_void_p),
+                ("w_packed", ctypes.c_void_p), ("scale_wt", ctypes.c_void_p),
+                ("scale_wt_len", ctypes.c_int64), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int64)]
 
 _lib = None
 
@@ -61,6 +69,7 @@ def lib():
             "bitnet_gemv_fused": [P, P, I, P, P, I64, I64, I64, I64, P],
             "bitnet_linear": [P, P, I, P, P, I64, I64, I64, I64, P, SZ, P],
             "bitnet_linear_noalloc": [P, P, I, P, P, I64, I64, I64, I64, P],
+            "bitnet_gemv_fused_grouped": [P, I64, I64, I, P],
             "bitnet_device_status": [P],
             "bitnet_gemm_acc_i32": [P, P, P, I64, I64, I64, P],
             "bitnet_gemv_fused_debug": [P, P, P, P, I, P, I64, I64, I64, P],
@@ -183,6 +192,42 @@ def bitnet_gemv_fused(x, w_packed, scale_wt, out=None):
                                    sw.numel(), M, N, K, _stream(x.device)),
            "bitnet_gemv_fused")
     return out
+
+
+def gemv_problems(xs, w_packeds, scale_wts, outs):
+    """ctypes array of problem descriptors (the tensors must stay alive)."""
+    arr = (GemvProblem * len(xs))()
+    for i, (x, wp, sw, o) in enumerate(zip(xs, w_packeds, scale_wts, outs)):
+        arr[i] = GemvProblem(o.data_ptr(), x.data_ptr(), wp.data_ptr(), sw.data_ptr(),
+                             sw.numel(), wp.shape[0], x.shape[1])
+    return arr
+
+
+def bitnet_gemv_fused_grouped(xs, w_packeds, scale_wts, outs=None):
+    """Independent fused GEMV problems with the same M in one call:
+    xs[i] bf16 [M, K_i], w_packeds[i] uint8 [N_i, K_i/4] -> bf16 [M, N_i]."""
+    if not (len(xs) == len(w_packeds) == len(scale_wts)):
+        raise ValueError("xs, w_packeds and scale_wts must have the same length")
+    if len(xs) == 0:
+        return []
+    M = xs[0].shape[0]
+    sws, new_outs = [], []
+    for i, (x, wp, sw) in enumerate(zip(xs, w_packeds, scale_wts)):
+        _need(x, torch.bfloat16, f"xs[{i}]", 2)
+        _need(wp, torch.uint8, f"w_packeds[{i}]", 2)
+        if x.shape[0] != M:
+            raise ValueError("every problem of a group has the same M")
+        if wp.shape[1] * 4 != x.shape[1]:
+            raise ValueError(f"w_packeds[{i}] {tuple(wp.shape)} does not match K={x.shape[1]}")
+        sws.append(_scale_wt(sw, wp.shape[0], x.device))
+        if outs is None:
+            new_outs.append(torch.empty((M, wp.shape[0]), dtype=torch.bfloat16, device=x.device))
+    outs = outs if outs is not None else new_outs
+    arr = gemv_problems(xs, w_packeds, sws, outs)
+    _check(lib().bitnet_gemv_fused_grouped(ctypes.cast(arr, ctypes.c_void_p), len(xs), M, BF16,
+                                           _stream(xs[0].device)),
+           "bitnet_gemv_fused_grouped")
+    return outs
 
 
 def bitnet_linear_workspace_bytes(M, K):

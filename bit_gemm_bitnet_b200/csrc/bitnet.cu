@@ -8,6 +8,7 @@
 #include "common.cuh"
 #include "gemm_ts.cuh"
 #include "gemv.cuh"
+#include "gemv_grouped.cuh"
 #include "pack_quant.cuh"
 
 namespace bitnet {
@@ -263,6 +264,83 @@ bitnet_status run_gemv(GemvParams p, bool preq, cudaStream_t st) {
               : launch_gemv_cw<false, false>(cw, mb, rw, p, gy, smem, dev->sms, st);
 }
 
+// ------------------------------------------------------------ grouped GEMV
+template <int MB, int RW_MAX>
+bitnet_status launch_grouped_t(const GroupedParams& gp, size_t smem, int sms, cudaStream_t st) {
+  auto k = gemv_grouped_kernel<16, MB, RW_MAX>;
+  constexpr int threads = 17 * 32;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, threads, smem) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  if (occ < 1) occ = 1;
+  int grid = occ * sms;
+  if (grid > gp.units) grid = gp.units;
+  if (grid < 1) grid = 1;
+  return launch_pdl(k, dim3(grid), dim3(threads), smem, st, gp);
+}
+
+// The most weight rows a consumer warp takes per unit, by activation-row
+// bucket (at most 16 accumulator registers per lane).
+constexpr int grouped_rw_max(int mb) { return mb == 1 ? 4 : mb == 2 ? 2 : mb == 4 ? 4 : mb == 8 ? 2 : 1; }
+
+// Launch up to kGroupMax problems (all K % 64 == 0, validated) in one kernel.
+bitnet_status run_gemv_grouped(const bitnet_gemv_problem* pr, int count, int M, cudaStream_t st) {
+  DeviceInfo* dev = nullptr;
+  bitnet_status s = device_info(&dev);
+  if (s != BITNET_OK) return s;
+  static_assert(sizeof(GroupedParams) <= 32000, "kernel parameter space");
+  GroupedParams gp;
+  gp.count = count;
+  gp.M = M;
+  const int mb = bucket_of(M);
+  const int rw_max = grouped_rw_max(mb);
+  constexpr int cw = 16;
+  int units = 0;
+  int64_t kmax = 0;
+  size_t stage = 0;
+  for (int i = 0; i < count; ++i) {
+    const int64_t K = pr[i].K, N = pr[i].N, KB = K / 4;
+    int rw = pow2_floor(kGemvStageTarget / (cw * KB));
+    if (rw > rw_max) rw = rw_max;
+    if (rw < 1) rw = 1;
+    gp.unit0[i] = units;
+    gp.rw[i] = static_cast<int8_t>(rw);
+    gp.K[i] = static_cast<int>(K);
+    gp.N[i] = static_cast<int>(N);
+    gp.sw_len[i] = static_cast<int>(pr[i].scale_wt_len);
+    gp.x[i] = static_cast<const uint16_t*>(pr[i].x);
+    gp.wp[i] = pr[i].w_packed;
+    gp.sw[i] = pr[i].scale_wt;
+    gp.out[i] = pr[i].out;
+    units += static_cast<int>((N + cw * rw - 1) / (cw * rw));
+    if (K > kmax) kmax = K;
+    const size_t sb = align128(static_cast<size_t>(cw * rw) * KB);
+    if (sb > stage) stage = sb;
+  }
+  gp.unit0[count] = units;
+  gp.units = units;
+  if (units == 0) return BITNET_OK;
+  gp.q_bytes = static_cast<uint32_t>(align128(static_cast<size_t>(M) * kmax));
+  gp.stage_bytes = static_cast<uint32_t>(stage);
+  int stages = static_cast<int>(kGemvRingTarget / stage);
+  if (stages > kGemvMaxStages) stages = kGemvMaxStages;
+  if (stages < 1) stages = 1;
+  while (stages > 1 && kGemvHeaderBytes + gp.q_bytes + stages * stage > kSmemLimit) --stages;
+  gp.stages = stages;
+  const size_t smem = kGemvHeaderBytes + gp.q_bytes + static_cast<size_t>(stages) * stage;
+  if (smem > kSmemLimit) return BITNET_ERR_SHAPE;
+  switch (mb) {
+    case 1: return launch_grouped_t<1, grouped_rw_max(1)>(gp, smem, dev->sms, st);
+    case 2: return launch_grouped_t<2, grouped_rw_max(2)>(gp, smem, dev->sms, st);
+    case 4: return launch_grouped_t<4, grouped_rw_max(4)>(gp, smem, dev->sms, st);
+    case 8: return launch_grouped_t<8, grouped_rw_max(8)>(gp, smem, dev->sms, st);
+    default: return launch_grouped_t<16, grouped_rw_max(16)>(gp, smem, dev->sms, st);
+  }
+}
+
 // ---------------------------------------------------------------- GEMM
 bool gemm_tc_ok(const int8_t* xq, const uint8_t* wp, int64_t K) {
   // TMA: row pitches must be multiples of 16 bytes (K/4 for the packed
@@ -508,6 +586,47 @@ bitnet_status bitnet_gemv_fused(uint16_t* out, const void* x, bitnet_dtype dt,
   p.sw = scale_wt;
   p.sw_len = static_cast<int>(scale_wt_len);
   return run_gemv(p, false, as_stream(stream));
+}
+
+bitnet_status bitnet_gemv_fused_grouped(const bitnet_gemv_problem* problems, int64_t count,
+                                        int64_t M, bitnet_dtype dt, void* stream) {
+  if (dt != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (count < 0) return BITNET_ERR_SHAPE;
+  if (count == 0) return BITNET_OK;
+  if (problems == nullptr) return BITNET_ERR_NULL;
+  // validate everything before anything is enqueued
+  for (int64_t i = 0; i < count; ++i) {
+    const bitnet_gemv_problem& q = problems[i];
+    GemvParams p = {};
+    bitnet_status s = gemv_common(p, q.x, dt, q.w_packed, M, q.N, q.K);
+    if (s != BITNET_OK) return s;
+    if (q.N == 0) continue;
+    if (q.out == nullptr) return BITNET_ERR_NULL;
+    if (!aligned(q.out, 16)) return BITNET_ERR_ALIGN;
+    s = check_scale_wt(q.scale_wt, q.scale_wt_len, q.N);
+    if (s != BITNET_OK) return s;
+  }
+  cudaStream_t st = as_stream(stream);
+  bitnet_gemv_problem batch[kGroupMax];
+  int n = 0;
+  for (int64_t i = 0; i < count; ++i) {
+    const bitnet_gemv_problem& q = problems[i];
+    if (q.N == 0) continue;
+    if (q.K % 64 != 0) {  // rows not 16-byte aligned: its own launch
+      bitnet_status s = bitnet_gemv_fused(q.out, q.x, dt, q.w_packed, q.scale_wt,
+                                          q.scale_wt_len, M, q.N, q.K, stream);
+      if (s != BITNET_OK) return s;
+      continue;
+    }
+    batch[n++] = q;
+    if (n == kGroupMax) {
+      bitnet_status s = run_gemv_grouped(batch, n, static_cast<int>(M), st);
+      if (s != BITNET_OK) return s;
+      n = 0;
+    }
+  }
+  if (n > 0) return run_gemv_grouped(batch, n, static_cast<int>(M), st);
+  return BITNET_OK;
 }
 
 bitnet_status bitnet_gemv_fused_debug(int32_t* acc, int8_t* x_q, uint16_t* scale_act,

@@ -129,6 +129,177 @@ __device__ __forceinline__ void gemv_rows(int (&acc)[RW][MB][PLANES ? 4 : 1],
   }
 }
 
+// Quantise the Mc activation rows x [Mc, K] (bf16) into shared memory: codes
+// with 16-element groups transposed 4x4 (qs), per-row code sums (qsum), the
+// bf16-rounded scales as fp32 (saf). All CW consumer warps take part; the
+// caller synchronises the consumers (named barrier 1) afterwards. dbg_q /
+// dbg_sa, if not null, receive the natural-order codes and the scale bits.
+struct GemvSmem {
+  int* qsum;
+  float* saf;
+  float* rq_s;
+  float* rq_r;
+  uint32_t* red;
+  uint8_t* qs;
+};
+
+template <int CW, int MB>
+__device__ __forceinline__ void gemv_stage_activations(const GemvSmem& sh, const uint16_t* __restrict__ x,
+                                                       int K, int Mc, int8_t* dbg_q, uint16_t* dbg_sa) {
+  constexpr int kGemvConsumerWarps = CW;
+  constexpr int kGemvConsumers = CW * 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int* qsum = sh.qsum;
+  float* saf = sh.saf;
+  float* rq_s = sh.rq_s;
+  float* rq_r = sh.rq_r;
+  uint32_t* red = sh.red;
+  uint8_t* qs = sh.qs;
+    // absmax of every activation row; each thread owns the 4-element quads
+    // tid, tid + 512, ... of a row (loops kept rolled: a small code footprint)
+    const int quads = K / 4;
+    uint32_t mb[MB];
+#pragma unroll
+    for (int m = 0; m < MB; ++m) {
+      mb[m] = 0;
+      if (MB == 1 || m < Mc) {
+        const uint2* row = reinterpret_cast<const uint2*>(x + static_cast<int64_t>(m) * K);
+        // four independent loads in flight per round
+#pragma unroll 1
+        for (int u0 = tid; u0 < quads; u0 += 4 * kGemvConsumers) {
+          uint2 v[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int u = u0 + j * kGemvConsumers;
+            v[j] = u < quads ? __ldg(row + u) : make_uint2(0u, 0u);
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            mb[m] = max(mb[m], max(max(v[j].x & 0x7FFFu, (v[j].x >> 16) & 0x7FFFu),
+                                   max(v[j].y & 0x7FFFu, (v[j].y >> 16) & 0x7FFFu)));
+        }
+      }
+      mb[m] = __reduce_max_sync(0xFFFFFFFFu, mb[m]);
+      if (lane == 0) red[warp * MB + m] = mb[m];
+    }
+    named_barrier_sync(1, kGemvConsumers);
+    if (tid < MB) {  // one thread per activation row: its quantiser and scale
+      uint32_t t = 0;
+      for (int w = 0; w < kGemvConsumerWarps; ++w) t = max(t, red[w * MB + tid]);
+      const RowQuant q = row_quant(bf16_bits_to_f32(t));
+      rq_s[tid] = q.s;
+      rq_r[tid] = q.r;
+      const uint16_t sb = f32_to_bf16_bits(q.s);
+      saf[tid] = bf16_bits_to_f32(sb);
+      if (dbg_sa != nullptr && tid < Mc) dbg_sa[tid] = sb;
+    }
+    named_barrier_sync(1, kGemvConsumers);
+    // quantise: element 4b + i of 16-group g goes to byte 16g + 4i + b
+    int qs_part[MB];
+#pragma unroll
+    for (int m = 0; m < MB; ++m) {
+      qs_part[m] = 0;
+      if (MB == 1 || m < Mc) {
+        RowQuant rqm;
+        rqm.s = rq_s[m];
+        rqm.r = rq_r[m];
+        const uint2* row = reinterpret_cast<const uint2*>(x + static_cast<int64_t>(m) * K);
+        uint8_t* qrow = qs + m * K;
+#pragma unroll 1
+        for (int u = tid; u < quads; u += kGemvConsumers) {
+          const uint2 v = __ldg(row + u);
+          const int q0 = quant_one(bf16_bits_to_f32(v.x & 0xFFFFu), rqm);
+          const int q1 = quant_one(bf16_bits_to_f32(v.x >> 16), rqm);
+          const int q2 = quant_one(bf16_bits_to_f32(v.y & 0xFFFFu), rqm);
+          const int q3 = quant_one(bf16_bits_to_f32(v.y >> 16), rqm);
+          qs_part[m] += q0 + q1 + q2 + q3;
+          uint8_t* d = qrow + 16 * (u >> 2) + (u & 3);
+          d[0] = static_cast<uint8_t>(q0);
+          d[4] = static_cast<uint8_t>(q1);
+          d[8] = static_cast<uint8_t>(q2);
+          d[12] = static_cast<uint8_t>(q3);
+          if (dbg_q != nullptr)
+            reinterpret_cast<uint32_t*>(dbg_q + static_cast<int64_t>(m) * K)[u] =
+                (static_cast<uint32_t>(q0) & 0xFFu) | ((static_cast<uint32_t>(q1) & 0xFFu) << 8) |
+                ((static_cast<uint32_t>(q2) & 0xFFu) << 16) | (static_cast<uint32_t>(q3) << 24);
+        }
+      }
+    }
+    named_barrier_sync(1, kGemvConsumers);  // red[] reuse
+#pragma unroll
+    for (int m = 0; m < MB; ++m) {
+      const int s = __reduce_add_sync(0xFFFFFFFFu, qs_part[m]);
+      if (lane == 0) red[warp * MB + m] = static_cast<uint32_t>(s);
+    }
+    named_barrier_sync(1, kGemvConsumers);
+    if (tid < MB) {
+      int s = 0;
+      for (int w = 0; w < kGemvConsumerWarps; ++w) s += static_cast<int>(red[w * MB + tid]);
+      qsum[tid] = s;
+    }
+}
+
+// Reduce one warp's RW x MB lane partials and write the outputs of rows
+// n0 .. n0 + rows - 1: int32 to acc_out if given, else bf16 to out with the
+// fp32 epilogue (acc - 2 * qsum[m]) * saf[m] * sw[n or 0].
+template <int MB, int RW, bool PLANES>
+__device__ __forceinline__ void gemv_reduce_store(const int (&acc)[RW][MB][PLANES ? 4 : 1], int rows,
+                                                  int n0, int Mc, int m_base, int N,
+                                                  const int* qsum, const float* saf,
+                                                  uint16_t* __restrict__ out,
+                                                  int32_t* __restrict__ acc_out,
+                                                  const float* __restrict__ sw, int sw_len) {
+  const int lane = threadIdx.x & 31;
+  // Reduce the RW x MB lane partials over the warp: a butterfly that halves
+  // the number of values at each of the first log2(RW * MB) exchanges
+  // (reduce-scatter), then plain exchanges for the remaining lane bits.
+  constexpr int V = RW * MB;
+  static_assert((V & (V - 1)) == 0 && V <= 32, "V must be a power of two <= 32");
+  int vals[V];
+#pragma unroll
+  for (int r = 0; r < RW; ++r)
+#pragma unroll
+    for (int m = 0; m < MB; ++m) {
+      if constexpr (PLANES)
+        vals[r * MB + m] = acc[r][m][0] + (acc[r][m][1] >> 2) + (acc[r][m][2] >> 4) +
+                           (acc[r][m][3] >> 6);
+      else
+        vals[r * MB + m] = acc[r][m][0];
+    }
+  int idx = 0;  // which of the V values this lane ends up holding
+#pragma unroll
+  for (int h = V / 2, o = 16; h >= 1; h /= 2, o /= 2) {
+    const bool hi = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const int send = hi ? vals[i] : vals[i + h];
+      const int keep = hi ? vals[i + h] : vals[i];
+      vals[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+    }
+    idx += hi ? h : 0;
+  }
+  int v = vals[0];
+  constexpr int kDone = V >= 32 ? 32 : V;  // lane bits already summed: log2(V)
+#pragma unroll
+  for (int o = 32 / kDone / 2; o >= 1; o /= 2) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  // lanes that differ only in the low bits hold the same total; one stores
+  if ((lane & (32 / kDone - 1)) == 0) {
+    const int r = idx / MB, m = idx % MB;
+    if (r < rows && m < Mc) {
+      const int n = n0 + r;
+      const int a = v - 2 * qsum[m];
+      const int64_t o = static_cast<int64_t>(m_base + m) * N + n;
+      if (acc_out != nullptr) {
+        acc_out[o] = a;
+      } else {
+        const float s_w = sw[sw_len == 1 ? 0 : n];
+        const float y = __fmul_rn(__fmul_rn(__int2float_rn(a), saf[m]), s_w);
+        out[o] = f32_to_bf16_bits(y);
+      }
+    }
+  }
+}
+
 // CW: consumer warps per CTA;
 // MB: rows of x per CTA (bucket); RW: weight rows per consumer warp per stage;
 // WIDE: K % 64 == 0 (rows 16-byte aligned: one bulk copy per stage),
@@ -217,88 +388,9 @@ __global__ void __launch_bounds__((CW + 1) * 32) gemv_kernel(GemvParams p) {
   pdl_wait();  // the activations may come from the previous kernel
   const int groups16 = K / 16;
   if constexpr (!PREQ) {
-    // absmax of every activation row; each thread owns the 4-element quads
-    // tid, tid + 512, ... of a row (loops kept rolled: a small code footprint)
-    const int quads = K / 4;
-    uint32_t mb[MB];
-#pragma unroll
-    for (int m = 0; m < MB; ++m) {
-      mb[m] = 0;
-      if (MB == 1 || m < Mc) {
-        const uint2* row = reinterpret_cast<const uint2*>(p.x + static_cast<int64_t>(m) * K);
-        // four independent loads in flight per round
-#pragma unroll 1
-        for (int u0 = tid; u0 < quads; u0 += 4 * kGemvConsumers) {
-          uint2 v[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int u = u0 + j * kGemvConsumers;
-            v[j] = u < quads ? __ldg(row + u) : make_uint2(0u, 0u);
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            mb[m] = max(mb[m], max(max(v[j].x & 0x7FFFu, (v[j].x >> 16) & 0x7FFFu),
-                                   max(v[j].y & 0x7FFFu, (v[j].y >> 16) & 0x7FFFu)));
-        }
-      }
-      mb[m] = __reduce_max_sync(0xFFFFFFFFu, mb[m]);
-      if (lane == 0) red[warp * MB + m] = mb[m];
-    }
-    named_barrier_sync(1, kGemvConsumers);
-    if (tid < MB) {  // one thread per activation row: its quantiser and scale
-      uint32_t t = 0;
-      for (int w = 0; w < kGemvConsumerWarps; ++w) t = max(t, red[w * MB + tid]);
-      const RowQuant q = row_quant(bf16_bits_to_f32(t));
-      rq_s[tid] = q.s;
-      rq_r[tid] = q.r;
-      const uint16_t sb = f32_to_bf16_bits(q.s);
-      saf[tid] = bf16_bits_to_f32(sb);
-      if (p.dbg_sa != nullptr && blockIdx.x == 0 && tid < Mc) p.dbg_sa[tid] = sb;
-    }
-    named_barrier_sync(1, kGemvConsumers);
-    // quantise: element 4b + i of 16-group g goes to byte 16g + 4i + b
-    int qs_part[MB];
-#pragma unroll
-    for (int m = 0; m < MB; ++m) {
-      qs_part[m] = 0;
-      if (MB == 1 || m < Mc) {
-        RowQuant rqm;
-        rqm.s = rq_s[m];
-        rqm.r = rq_r[m];
-        const uint2* row = reinterpret_cast<const uint2*>(p.x + static_cast<int64_t>(m) * K);
-        uint8_t* qrow = qs + m * K;
-#pragma unroll 1
-        for (int u = tid; u < quads; u += kGemvConsumers) {
-          const uint2 v = __ldg(row + u);
-          const int q0 = quant_one(bf16_bits_to_f32(v.x & 0xFFFFu), rqm);
-          const int q1 = quant_one(bf16_bits_to_f32(v.x >> 16), rqm);
-          const int q2 = quant_one(bf16_bits_to_f32(v.y & 0xFFFFu), rqm);
-          const int q3 = quant_one(bf16_bits_to_f32(v.y >> 16), rqm);
-          qs_part[m] += q0 + q1 + q2 + q3;
-          uint8_t* d = qrow + 16 * (u >> 2) + (u & 3);
-          d[0] = static_cast<uint8_t>(q0);
-          d[4] = static_cast<uint8_t>(q1);
-          d[8] = static_cast<uint8_t>(q2);
-          d[12] = static_cast<uint8_t>(q3);
-          if (p.dbg_q != nullptr && blockIdx.x == 0)
-            reinterpret_cast<uint32_t*>(p.dbg_q + static_cast<int64_t>(m) * K)[u] =
-                (static_cast<uint32_t>(q0) & 0xFFu) | ((static_cast<uint32_t>(q1) & 0xFFu) << 8) |
-                ((static_cast<uint32_t>(q2) & 0xFFu) << 16) | (static_cast<uint32_t>(q3) << 24);
-        }
-      }
-    }
-    named_barrier_sync(1, kGemvConsumers);  // red[] reuse
-#pragma unroll
-    for (int m = 0; m < MB; ++m) {
-      const int s = __reduce_add_sync(0xFFFFFFFFu, qs_part[m]);
-      if (lane == 0) red[warp * MB + m] = static_cast<uint32_t>(s);
-    }
-    named_barrier_sync(1, kGemvConsumers);
-    if (tid < MB) {
-      int s = 0;
-      for (int w = 0; w < kGemvConsumerWarps; ++w) s += static_cast<int>(red[w * MB + tid]);
-      qsum[tid] = s;
-    }
+    gemv_stage_activations<CW, MB>(GemvSmem{qsum, saf, rq_s, rq_r, red, qs}, p.x, K, Mc,
+                                   blockIdx.x == 0 ? p.dbg_q : nullptr,
+                                   blockIdx.x == 0 ? p.dbg_sa : nullptr);
   } else {
     int qs_part[MB];
 #pragma unroll
@@ -356,54 +448,8 @@ __global__ void __launch_bounds__((CW + 1) * 32) gemv_kernel(GemvParams p) {
     __syncwarp();
     if (lane == 0) mbar_arrive(empty(s));
 
-    // Reduce the RW x MB lane partials over the warp: a butterfly that halves
-    // the number of values at each of the first log2(RW * MB) exchanges
-    // (reduce-scatter), then plain exchanges for the remaining lane bits.
-    constexpr int V = RW * MB;
-    static_assert((V & (V - 1)) == 0 && V <= 32, "V must be a power of two <= 32");
-    int vals[V];
-#pragma unroll
-    for (int r = 0; r < RW; ++r)
-#pragma unroll
-      for (int m = 0; m < MB; ++m) {
-        if constexpr (PLANES)
-          vals[r * MB + m] = acc[r][m][0] + (acc[r][m][1] >> 2) + (acc[r][m][2] >> 4) +
-                             (acc[r][m][3] >> 6);
-        else
-          vals[r * MB + m] = acc[r][m][0];
-      }
-    int idx = 0;  // which of the V values this lane ends up holding
-#pragma unroll
-    for (int h = V / 2, o = 16; h >= 1; h /= 2, o /= 2) {
-      const bool hi = (lane & o) != 0;
-#pragma unroll
-      for (int i = 0; i < h; ++i) {
-        const int send = hi ? vals[i] : vals[i + h];
-        const int keep = hi ? vals[i + h] : vals[i];
-        vals[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
-      }
-      idx += hi ? h : 0;
-    }
-    int v = vals[0];
-    constexpr int kDone = V >= 32 ? 32 : V;  // lane bits already summed: log2(V)
-#pragma unroll
-    for (int o = 32 / kDone / 2; o >= 1; o /= 2) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-    // lanes that differ only in the low bits hold the same total; one stores
-    if ((lane & (32 / kDone - 1)) == 0) {
-      const int r = idx / MB, m = idx % MB;
-      if (r < rows && m < Mc) {
-        const int n = n0 + r;
-        const int a = v - 2 * qsum[m];
-        const int64_t o = static_cast<int64_t>(m_base + m) * N + n;
-        if (p.acc_out != nullptr) {
-          p.acc_out[o] = a;
-        } else {
-          const float s_w = p.sw[p.sw_len == 1 ? 0 : n];
-          const float y = __fmul_rn(__fmul_rn(__int2float_rn(a), saf[m]), s_w);
-          p.out[o] = f32_to_bf16_bits(y);
-        }
-      }
-    }
+    gemv_reduce_store<MB, RW, PLANES>(acc, rows, n0, Mc, m_base, N, qsum, saf, p.out, p.acc_out,
+                                      p.sw, p.sw_len);
   }
 }
 

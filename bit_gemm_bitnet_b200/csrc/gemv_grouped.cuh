@@ -1,0 +1,150 @@
+// Grouped decode GEMV: many independent fused quantise + GEMV problems (same
+// M, any K and N) in one persistent launch.
+//
+// The row blocks ("units") of all problems form one list, in problem order.
+// Each CTA owns a contiguous range of it. Its producer warp streams the units'
+// packed weights (contiguous rows) through the shared-memory ring with bulk
+// async copies, crossing problem boundaries without a pause, while the
+// consumer warps quantise a problem's activation rows when they first reach
+// one of its units and then reduce its rows exactly as the single-problem
+// kernel does. One launch replaces one launch per problem, so the fixed cost
+// of a launch and of a CTA's start is paid once for the whole group.
+#pragma once
+#include "gemv.cuh"
+
+namespace bitnet {
+
+constexpr int kGroupMax = 256;  // problems per launch (kernel parameter space)
+
+struct GroupedParams {
+  int count;               // problems in this launch
+  int M;                   // activation rows of every problem (1..15)
+  int units;               // total units
+  int stages;
+  uint32_t q_bytes;        // shared bytes for the quantised rows (M * max K)
+  uint32_t stage_bytes;    // shared bytes per stage (the largest unit)
+  int unit0[kGroupMax + 1];  // first unit of each problem; unit0[count] = units
+  int8_t rw[kGroupMax];      // weight rows per consumer warp per unit
+  int K[kGroupMax];
+  int N[kGroupMax];
+  int sw_len[kGroupMax];
+  const uint16_t* x[kGroupMax];
+  const uint8_t* wp[kGroupMax];
+  const float* sw[kGroupMax];
+  uint16_t* out[kGroupMax];
+};
+
+// CW consumer warps; MB activation-row bucket; RW_MAX the most rows a warp
+// takes per unit. Every K is a multiple of 64 (16-byte aligned rows).
+template <int CW, int MB, int RW_MAX>
+__global__ void __launch_bounds__((CW + 1) * 32)
+    gemv_grouped_kernel(const __grid_constant__ GroupedParams p) {
+  constexpr int kConsumers = CW * 32;
+  constexpr bool PLANES = MB <= 2;
+  extern __shared__ __align__(128) uint8_t smem[];
+  int* qsum = reinterpret_cast<int*>(smem);
+  float* saf = reinterpret_cast<float*>(smem + 64);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 128);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + 256);
+  float* rq_s = reinterpret_cast<float*>(smem + 320);
+  float* rq_r = reinterpret_cast<float*>(smem + 384);
+  uint32_t* red = reinterpret_cast<uint32_t*>(smem + 512);
+  uint8_t* qs = smem + kGemvHeaderBytes;
+  uint8_t* ring = qs + p.q_bytes;
+  static_assert(kGemvMaxConsumerWarps * MB * 4 <= kGemvHeaderBytes - 512, "reduction scratch");
+
+  const int S = p.stages;
+  const int Mc = MB == 1 ? 1 : p.M;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int u_begin = static_cast<int>(static_cast<int64_t>(p.units) * blockIdx.x / gridDim.x);
+  const int u_end = static_cast<int>(static_cast<int64_t>(p.units) * (blockIdx.x + 1) / gridDim.x);
+  auto full = [&](int s) { return smem_u32(bars + s); };
+  auto empty = [&](int s) { return smem_u32(bars + kGemvMaxStages + s); };
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), CW);
+    }
+    *abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_launch_dependents();
+
+  // problem of the first unit of this CTA
+  int pr = 0;
+  while (pr < p.count - 1 && u_begin >= p.unit0[pr + 1]) ++pr;
+
+  if (warp == CW) {
+    // ------------------------------------------------------------ producer
+    uint32_t it = 0;
+    for (int u = u_begin; u < u_end; ++u, ++it) {
+      while (u >= p.unit0[pr + 1]) ++pr;
+      const int s = it % S;
+      const uint32_t ph = (it / S) & 1u;
+      if (!mbar_wait(empty(s), ph ^ 1u, abort)) break;
+      const int KB = p.K[pr] / 4;
+      const int rpu = CW * p.rw[pr];
+      const int row0 = (u - p.unit0[pr]) * rpu;
+      const int rows = min(rpu, p.N[pr] - row0);
+      if (lane == 0) {
+        const uint32_t bytes = static_cast<uint32_t>(rows) * KB;
+        mbar_arrive_expect_tx(full(s), bytes);
+        bulk_load(smem_u32(ring + static_cast<size_t>(s) * p.stage_bytes),
+                  p.wp[pr] + static_cast<int64_t>(row0) * KB, bytes, full(s));
+      }
+    }
+    const uint32_t first = it > static_cast<uint32_t>(S) ? it - S : 0u;
+    for (uint32_t j = first; j < it; ++j) mbar_wait_drain(full(j % S), (j / S) & 1u);
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  pdl_wait();  // activations may come from the previous kernel
+  const GemvSmem sh{qsum, saf, rq_s, rq_r, red, qs};
+  int staged = -1;     // problem whose activations are in shared memory
+  bool dead = false;   // a wait gave up: keep the barrier sequence, skip work
+  uint32_t it = 0;
+  for (int u = u_begin; u < u_end; ++u, ++it) {
+    while (u >= p.unit0[pr + 1]) ++pr;
+    const int K = p.K[pr];
+    if (pr != staged) {
+      // every consumer warp reaches each problem switch at the same unit
+      // (the staging only reads the activations, so it also runs after a
+      // wait gave up: every consumer warp keeps the same barrier sequence)
+      if (staged >= 0) named_barrier_sync(1, kConsumers);
+      gemv_stage_activations<CW, MB>(sh, p.x[pr], K, Mc, nullptr, nullptr);
+      named_barrier_sync(1, kConsumers);
+      staged = pr;
+    }
+    const int s = it % S;
+    const uint32_t ph = (it / S) & 1u;
+    if (!dead && !mbar_wait(full(s), ph, abort)) dead = true;
+    const int KB = K / 4;
+    const int rw = p.rw[pr];
+    const int r0 = warp * rw;
+    const int n0 = (u - p.unit0[pr]) * (CW * rw) + r0;
+    int rows = min(rw, p.N[pr] - n0);
+    if (rows < 0 || dead) rows = 0;
+
+    int acc[RW_MAX][MB][PLANES ? 4 : 1];
+#pragma unroll
+    for (int r = 0; r < RW_MAX; ++r)
+#pragma unroll
+      for (int m = 0; m < MB; ++m)
+#pragma unroll
+        for (int i = 0; i < (PLANES ? 4 : 1); ++i) acc[r][m][i] = 0;
+    if (rows > 0) {
+      const uint8_t* stage = ring + static_cast<size_t>(s) * p.stage_bytes;
+      const uint32_t* wrow = reinterpret_cast<const uint32_t*>(stage + static_cast<size_t>(r0) * KB);
+      gemv_rows<MB, RW_MAX, PLANES, false>(acc, wrow, K / 16, qs, K, Mc, rows, lane);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty(s));
+    gemv_reduce_store<MB, RW_MAX, PLANES>(acc, rows, n0, Mc, 0, p.N[pr], qsum, saf, p.out[pr],
+                                          nullptr, p.sw[pr], p.sw_len[pr]);
+  }
+}
+
+}  // namespace bitnet

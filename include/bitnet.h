@@ -111,6 +111,34 @@ bitnet_status bitnet_gemv_fused(uint16_t* out, const void* x, bitnet_dtype dt,
                                 int64_t scale_wt_len, int64_t M, int64_t N,
                                 int64_t K, void* stream);
 
+/* One problem of a grouped decode call (see bitnet_gemv_fused_grouped):
+ * the arguments of one bitnet_gemv_fused call, M excepted. */
+typedef struct {
+  uint16_t* out;            /* bf16 [M, N] */
+  const void* x;            /* [M, K] of the group's dtype */
+  const uint8_t* w_packed;  /* uint8 [N, K/4] */
+  const float* scale_wt;    /* fp32, scale_wt_len elements: 1 or N */
+  int64_t scale_wt_len;
+  int64_t N;
+  int64_t K;
+} bitnet_gemv_problem;
+
+/* Many independent bitnet_gemv_fused problems with the same M, in as few
+ * launches as possible (one per 256 problems). Each problem's result is the
+ * one bitnet_gemv_fused gives, bit for bit. Independent means: no problem
+ * reads what another one of the same call writes. Use it for the decode
+ * projections that share no data dependency (e.g. Q, K, V of a layer, or the
+ * independent calls of a sweep); one persistent launch streams all their
+ * weights back to back instead of paying a launch and a prologue per call.
+ *   problems  in, HOST array of `count` problem descriptors (read during
+ *             the call, not kept)
+ * Each problem obeys bitnet_gemv_fused's rules. Problems whose K is not a
+ * multiple of 64 are computed by their own bitnet_gemv_fused launch. The
+ * whole call is validated before anything is enqueued. */
+bitnet_status bitnet_gemv_fused_grouped(const bitnet_gemv_problem* problems,
+                                        int64_t count, int64_t M,
+                                        bitnet_dtype dt, void* stream);
+
 /* Workspace bitnet_linear needs for (M, K): 0 when it takes the fused GEMV
  * path, otherwise room for the int8 [M, K] activations, the bf16 [M] scales
  * and int32 [M] per-row sums of the codes, each 256-byte aligned. The layout

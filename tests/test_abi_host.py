@@ -93,3 +93,22 @@ def test_noop_sizes_return_ok_without_work():
     assert L.bitnet_pack_weights(None, None, 0, 8, None) == bn.OK
     assert L.bitnet_quantize_act(None, None, None, 0, 0, 64, None) == bn.OK
     assert L.bitnet_linear(None, None, 0, None, None, 1, 0, 4, 64, None, 0, None) == bn.OK
+
+
+def test_grouped_validation_before_launch():
+    L = bn.lib()
+    arr = (bn.GemvProblem * 2)()
+    for i in range(2):
+        arr[i] = bn.GemvProblem(0x10000, 0x10000, 0x10000, 0x10000, 1, 64, 128)
+    p = ctypes.cast(arr, ctypes.c_void_p)
+    assert L.bitnet_gemv_fused_grouped(p, 0, 1, 0, None) == bn.OK
+    assert L.bitnet_gemv_fused_grouped(None, 2, 1, 0, None) == bn.ERR_NULL
+    assert L.bitnet_gemv_fused_grouped(p, -1, 1, 0, None) == bn.ERR_SHAPE
+    assert L.bitnet_gemv_fused_grouped(p, 2, 16, 0, None) == bn.ERR_SHAPE
+    assert L.bitnet_gemv_fused_grouped(p, 2, 1, 1, None) == bn.ERR_DTYPE
+    arr[1] = bn.GemvProblem(0x10000, 0x10000, 0x10000, 0x10000, 1, 64, 48)   # K % 32
+    assert L.bitnet_gemv_fused_grouped(p, 2, 1, 0, None) == bn.ERR_SHAPE
+    arr[1] = bn.GemvProblem(0x10008, 0x10000, 0x10000, 0x10000, 1, 64, 128)  # out align
+    assert L.bitnet_gemv_fused_grouped(p, 2, 1, 0, None) == bn.ERR_ALIGN
+    arr[1] = bn.GemvProblem(0x10000, 0x10000, 0x10000, 0x10000, 3, 64, 128)  # scale len
+    assert L.bitnet_gemv_fused_grouped(p, 2, 1, 0, None) == bn.ERR_SHAPE

@@ -109,3 +109,35 @@ def test_prefill_linear_sampled_rows(M, KN):
     assert np.array_equal(bf16_bits(sa)[rows], s_ref)
     ref = oracle.linear(x[rows], p, sw, threads=THREADS)
     close(bf16_bits(y)[rows], ref)
+
+
+def test_decode_sweep_grouped_graph_matches_oracle():
+    """All 211 calls of the 2B decode sweep as one grouped call, captured in a
+    CUDA graph as the bench does; layers 0, 15, 29 and the LM head checked."""
+    names = [n for n, _, _ in W.DECODE_2B_LAYER]
+    calls = [(layer, names.index(n), K, N) for layer in range(W.DECODE_2B_LAYERS)
+             for n, K, N in W.DECODE_2B_LAYER]
+    calls.append((30, len(names), W.DECODE_2B_LM_HEAD[1], W.DECODE_2B_LM_HEAD[2]))
+    xs, wps, sws, outs, checks = [], [], [], [], {}
+    for i, (layer, v, K, N) in enumerate(calls):
+        w = synth.ternary(synth.key(W.W_DECODE_2B, layer, synth.T_WEIGHT, v), N, K)
+        sw = synth.scale_wt(synth.key(W.W_DECODE_2B, layer, synth.T_SCALE_WT, v))
+        x = synth.act_bf16(synth.key(W.W_DECODE_2B, layer, synth.T_ACT, v), 1, K)
+        xs.append(to_dev(x, torch.bfloat16))
+        wps.append(bn.bitnet_pack_weights(to_dev(w)))
+        sws.append(to_dev(sw))
+        outs.append(torch.zeros((1, N), dtype=torch.bfloat16, device="cuda"))
+        if layer in (0, 15, 30):
+            checks[i] = (x, oracle.pack(w), sw)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        bn.bitnet_gemv_fused_grouped(xs, wps, sws, outs)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            bn.bitnet_gemv_fused_grouped(xs, wps, sws, outs)
+        for o in outs:
+            o.fill_(0)
+        g.replay()
+    torch.cuda.synchronize()
+    for i, (x, p, sw) in checks.items():
+        close(bf16_bits(outs[i]), oracle.linear_cols_threads(x, p, sw, THREADS))

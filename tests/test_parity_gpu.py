@@ -265,3 +265,44 @@ def test_linear_split_path_ragged(M, K, N):
     sw = synth.uniform_f32(synth.key(98, N, 3), N, 0.01, 0.1)
     got = bn.bitnet_linear(to_dev(x, torch.bfloat16), to_dev(p), to_dev(sw))
     assert_bf16_close(bf16_bits(got), oracle.linear(x, p, sw))
+
+
+# -------------------------------------------------------------- grouped GEMV
+
+@pytest.mark.parametrize("M", [1, 2, 4, 15])
+def test_gemv_fused_grouped_matches_oracle_and_single_calls(M):
+    shapes = [(2560, 2560), (2560, 640), (6912, 300), (96, 40), (512, 1), (4096, 1000),
+              (128, 77)]
+    xs, wps, sws, host = [], [], [], []
+    for i, (K, N) in enumerate(shapes):
+        x = acts(99, 10 * M + i, M, K)
+        w = weights(99, 10 * M + i, N, K)
+        sw = synth.uniform_f32(synth.key(99, 10 * M + i, 3), N if i % 2 else 1, 0.01, 0.1)
+        p = oracle.pack(w)
+        host.append((x, p, sw))
+        xs.append(to_dev(x, torch.bfloat16))
+        wps.append(to_dev(p))
+        sws.append(to_dev(sw))
+    outs = bn.bitnet_gemv_fused_grouped(xs, wps, sws)
+    for (x, p, sw), o, xd, wd, sd in zip(host, outs, xs, wps, sws):
+        single = bn.bitnet_gemv_fused(xd, wd, sd)
+        assert np.array_equal(bf16_bits(o), bf16_bits(single))
+        assert_bf16_close(bf16_bits(o), oracle.linear(x, p, sw))
+
+
+def test_gemv_fused_grouped_more_than_one_launch():
+    # 300 problems: two launches of the grouped kernel
+    xs, wps, sws, refs = [], [], [], []
+    for i in range(300):
+        K, N = (128, 16 + i % 50) if i % 3 else (256, 33)
+        x = acts(100, i, 1, K)
+        w = weights(100, i, N, K)
+        p = oracle.pack(w)
+        sw = sw_of(100, i)
+        refs.append(oracle.linear(x, p, sw))
+        xs.append(to_dev(x, torch.bfloat16))
+        wps.append(to_dev(p))
+        sws.append(to_dev(sw))
+    outs = bn.bitnet_gemv_fused_grouped(xs, wps, sws)
+    for o, r in zip(outs, refs):
+        assert_bf16_close(bf16_bits(o), r)
