@@ -167,8 +167,10 @@ bitnet_status launch_gemv_rw(int rw, const GemvParams& p, int gy, size_t smem, i
   switch (rw) {
     case 1: return launch_gemv_t<CW, MB, 1, WIDE, PREQ>(p, gy, smem, sms, st);
     case 2: return launch_gemv_t<CW, MB, 2, WIDE, PREQ>(p, gy, smem, sms, st);
+    // instantiated exactly where rw * MB * (MB <= 2 ? 4 : 1) <= 32, the
+    // accumulator limit the caller applies
     case 4:
-      if constexpr (MB != 2 && MB <= 8) return launch_gemv_t<CW, MB, 4, WIDE, PREQ>(p, gy, smem, sms, st);
+      if constexpr (MB <= 8) return launch_gemv_t<CW, MB, 4, WIDE, PREQ>(p, gy, smem, sms, st);
       return BITNET_ERR_SHAPE;
     default:
       if constexpr (MB == 1 || MB == 4) return launch_gemv_t<CW, MB, 8, WIDE, PREQ>(p, gy, smem, sms, st);
