@@ -75,32 +75,53 @@ __device__ __forceinline__ void gemv_rows(int (&acc)[RW][MB][PLANES ? 4 : 1],
                                           const uint32_t* __restrict__ wrow, int words,
                                           const uint8_t* __restrict__ qs, int K, int Mc,
                                           int rows, int lane) {
+  if constexpr (PLANES) {
+    // One or two activation rows: two words per lane per iteration (t0 and
+    // t0 + 32), every shared-memory load of an iteration issued before its
+    // first use, so a warp waits for one round of loads per two words.
 #pragma unroll 1
-  for (int t = lane; t < words; t += 32) {
-    if constexpr (PLANES) {
-      uint4 Q[MB];
+    for (int t0 = lane; t0 < words; t0 += 64) {
+      const int t1 = t0 + 32;
+      const bool has1 = t1 < words;
+      uint4 Q0[MB], Q1[MB];
+      uint32_t w0[RW], w1[RW];
 #pragma unroll
-      for (int m = 0; m < MB; ++m)
-        if (MB == 1 || m < Mc) Q[m] = *reinterpret_cast<const uint4*>(qs + m * K + 16 * t);
+      for (int m = 0; m < MB; ++m) {
+        const bool mv = MB == 1 || m < Mc;
+        Q0[m] = mv ? *reinterpret_cast<const uint4*>(qs + m * K + 16 * t0) : make_uint4(0, 0, 0, 0);
+        Q1[m] = (mv && has1) ? *reinterpret_cast<const uint4*>(qs + m * K + 16 * t1)
+                             : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
       for (int r = 0; r < RW; ++r) {
-        if (FULL || r < rows) {
-          const uint32_t w = wrow[r * words + t];
+        const bool rv = FULL || r < rows;
+        w0[r] = rv ? wrow[r * words + t0] : 0u;
+        w1[r] = (rv && has1) ? wrow[r * words + t1] : 0u;  // zero weights add nothing
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint4* Q = h == 0 ? Q0 : Q1;
+        const uint32_t* wv = h == 0 ? w0 : w1;
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+          const uint32_t w = wv[r];
           const uint32_t p0 = w & 0x03030303u, p1 = w & 0x0C0C0C0Cu;
           const uint32_t p2 = w & 0x30303030u, p3 = w & 0xC0C0C0C0u;
 #pragma unroll
           for (int m = 0; m < MB; ++m) {
-            if (MB == 1 || m < Mc) {
-              acc[r][m][0] = dp4a_s32(p0, Q[m].x, acc[r][m][0]);
-              acc[r][m][1] = dp4a_s32(p1, Q[m].y, acc[r][m][1]);
-              acc[r][m][2] = dp4a_s32(p2, Q[m].z, acc[r][m][2]);
-              acc[r][m][3] = dp4a_us(p3, Q[m].w, acc[r][m][3]);
-            }
+            acc[r][m][0] = dp4a_s32(p0, Q[m].x, acc[r][m][0]);
+            acc[r][m][1] = dp4a_s32(p1, Q[m].y, acc[r][m][1]);
+            acc[r][m][2] = dp4a_s32(p2, Q[m].z, acc[r][m][2]);
+            acc[r][m][3] = dp4a_us(p3, Q[m].w, acc[r][m][3]);
           }
         }
       }
-    } else {
-      // planes of the warp's rows first, then one activation word at a time
+    }
+  } else {
+    // Many activation rows: planes of the warp's rows first, then one
+    // activation word at a time (keeps the registers bounded).
+#pragma unroll 1
+    for (int t = lane; t < words; t += 32) {
       uint32_t e[RW][4];
 #pragma unroll
       for (int r = 0; r < RW; ++r) {
