@@ -267,8 +267,43 @@ bitnet_status run_gemv(GemvParams p, bool preq, cudaStream_t st) {
 }
 
 // ------------------------------------------------------------ grouped GEMV
+// Split the units of a group over `grid` CTAs so that every CTA streams about
+// the same weight bytes (units differ in size from problem to problem). A
+// unit costs its bytes plus a fixed share for its epilogue.
+void partition_units(GroupedParams& gp, int grid, int cw) {
+  constexpr int64_t kUnitCost = 8192;
+  int64_t total = 0;
+  for (int i = 0; i < gp.count; ++i) {
+    const int64_t n = gp.unit0[i + 1] - gp.unit0[i];
+    if (n == 0) continue;
+    const int64_t KB = gp.K[i] / 4, rpu = static_cast<int64_t>(cw) * gp.rw[i];
+    total += (n - 1) * (rpu * KB + kUnitCost) + (gp.N[i] - (n - 1) * rpu) * KB + kUnitCost;
+  }
+  int c = 1;
+  int64_t cum = 0;  // cost of the units before problem i
+  gp.cta_u0[0] = 0;
+  for (int i = 0; i < gp.count && c < grid; ++i) {
+    const int64_t n = gp.unit0[i + 1] - gp.unit0[i];
+    if (n == 0) continue;
+    const int64_t KB = gp.K[i] / 4, rpu = static_cast<int64_t>(cw) * gp.rw[i];
+    const int64_t cf = rpu * KB + kUnitCost;
+    while (c < grid) {
+      const int64_t T = total * c / grid;
+      if (T <= cum) {
+        gp.cta_u0[c++] = gp.unit0[i];
+        continue;
+      }
+      const int64_t k = (T - cum + cf - 1) / cf;  // units of problem i before the boundary
+      if (k > n - 1) break;
+      gp.cta_u0[c++] = gp.unit0[i] + static_cast<int>(k);
+    }
+    cum += (n - 1) * cf + (gp.N[i] - (n - 1) * rpu) * KB + kUnitCost;
+  }
+  while (c <= grid) gp.cta_u0[c++] = gp.units;
+}
+
 template <int MB, int RW_MAX>
-bitnet_status launch_grouped_t(const GroupedParams& gp, size_t smem, int sms, cudaStream_t st) {
+bitnet_status launch_grouped_t(GroupedParams& gp, size_t smem, int sms, cudaStream_t st) {
   auto k = gemv_grouped_kernel<16, MB, RW_MAX>;
   constexpr int threads = 17 * 32;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -280,7 +315,9 @@ bitnet_status launch_grouped_t(const GroupedParams& gp, size_t smem, int sms, cu
   if (occ < 1) occ = 1;
   int grid = occ * sms;
   if (grid > gp.units) grid = gp.units;
+  if (grid > kGroupGridMax) grid = kGroupGridMax;
   if (grid < 1) grid = 1;
+  partition_units(gp, grid, 16);
   return launch_pdl(k, dim3(grid), dim3(threads), smem, st, gp);
 }
 

@@ -14,7 +14,8 @@
 
 namespace bitnet {
 
-constexpr int kGroupMax = 256;  // problems per launch (kernel parameter space)
+constexpr int kGroupMax = 256;       // problems per launch (kernel parameter space)
+constexpr int kGroupGridMax = 512;   // CTAs per launch
 
 struct GroupedParams {
   int count;               // problems in this launch
@@ -24,6 +25,7 @@ struct GroupedParams {
   uint32_t q_bytes;        // shared bytes for the quantised rows (M * max K)
   uint32_t stage_bytes;    // shared bytes per stage (the largest unit)
   int unit0[kGroupMax + 1];  // first unit of each problem; unit0[count] = units
+  int cta_u0[kGroupGridMax + 1];  // first unit of each CTA; cta_u0[grid] = units
   int8_t rw[kGroupMax];      // weight rows per consumer warp per unit
   int K[kGroupMax];
   int N[kGroupMax];
@@ -34,8 +36,34 @@ struct GroupedParams {
   uint16_t* out[kGroupMax];
 };
 
+// One consumer warp's share of a unit: rw == RW rows of a stage (fewer at a
+// problem's ragged end), then the release of the stage and the epilogue.
+template <int MB, int RW, bool PLANES>
+__device__ __forceinline__ void grouped_unit(const uint32_t* wrow, int K, const uint8_t* qs, int Mc,
+                                             int rows, int lane, int n0, int N, const int* qsum,
+                                             const float* saf, uint16_t* out, const float* sw,
+                                             int sw_len, uint32_t empty_bar) {
+  int acc[RW][MB][PLANES ? 4 : 1];
+#pragma unroll
+  for (int r = 0; r < RW; ++r)
+#pragma unroll
+    for (int m = 0; m < MB; ++m)
+#pragma unroll
+      for (int i = 0; i < (PLANES ? 4 : 1); ++i) acc[r][m][i] = 0;
+  if (rows == RW)
+    gemv_rows<MB, RW, PLANES, true>(acc, wrow, K / 16, qs, K, Mc, rows, lane);
+  else if (rows > 0)
+    gemv_rows<MB, RW, PLANES, false>(acc, wrow, K / 16, qs, K, Mc, rows, lane);
+  __syncwarp();
+  if (lane == 0) mbar_arrive(empty_bar);
+  gemv_reduce_store<MB, RW, PLANES>(acc, rows, n0, Mc, 0, N, qsum, saf, out, nullptr, sw, sw_len);
+}
+
 // CW consumer warps; MB activation-row bucket; RW_MAX the most rows a warp
-// takes per unit. Every K is a multiple of 64 (16-byte aligned rows).
+// takes per unit (a problem's own count, RW_MAX, RW_MAX / 2 or RW_MAX / 4,
+// picks the instantiation, so no work is spent on absent rows). Every K is a
+// multiple of 64 (16-byte aligned rows). CTA c takes the units
+// cta_u0[c] .. cta_u0[c + 1] - 1 (ranges balanced by bytes on the host).
 template <int CW, int MB, int RW_MAX>
 __global__ void __launch_bounds__((CW + 1) * 32)
     gemv_grouped_kernel(const __grid_constant__ GroupedParams p) {
@@ -56,8 +84,8 @@ __global__ void __launch_bounds__((CW + 1) * 32)
   const int S = p.stages;
   const int Mc = MB == 1 ? 1 : p.M;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int u_begin = static_cast<int>(static_cast<int64_t>(p.units) * blockIdx.x / gridDim.x);
-  const int u_end = static_cast<int>(static_cast<int64_t>(p.units) * (blockIdx.x + 1) / gridDim.x);
+  const int u_begin = p.cta_u0[blockIdx.x];
+  const int u_end = p.cta_u0[blockIdx.x + 1];
   auto full = [&](int s) { return smem_u32(bars + s); };
   auto empty = [&](int s) { return smem_u32(bars + kGemvMaxStages + s); };
 
@@ -128,22 +156,19 @@ __global__ void __launch_bounds__((CW + 1) * 32)
     int rows = min(rw, p.N[pr] - n0);
     if (rows < 0 || dead) rows = 0;
 
-    int acc[RW_MAX][MB][PLANES ? 4 : 1];
-#pragma unroll
-    for (int r = 0; r < RW_MAX; ++r)
-#pragma unroll
-      for (int m = 0; m < MB; ++m)
-#pragma unroll
-        for (int i = 0; i < (PLANES ? 4 : 1); ++i) acc[r][m][i] = 0;
-    if (rows > 0) {
-      const uint8_t* stage = ring + static_cast<size_t>(s) * p.stage_bytes;
-      const uint32_t* wrow = reinterpret_cast<const uint32_t*>(stage + static_cast<size_t>(r0) * KB);
-      gemv_rows<MB, RW_MAX, PLANES, false>(acc, wrow, K / 16, qs, K, Mc, rows, lane);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty(s));
-    gemv_reduce_store<MB, RW_MAX, PLANES>(acc, rows, n0, Mc, 0, p.N[pr], qsum, saf, p.out[pr],
-                                          nullptr, p.sw[pr], p.sw_len[pr]);
+    const uint32_t* wrow = reinterpret_cast<const uint32_t*>(
+        ring + static_cast<size_t>(s) * p.stage_bytes + static_cast<size_t>(r0) * KB);
+    if (rw == RW_MAX || RW_MAX == 1)
+      grouped_unit<MB, RW_MAX, PLANES>(wrow, K, qs, Mc, rows, lane, n0, p.N[pr], qsum, saf,
+                                       p.out[pr], p.sw[pr], p.sw_len[pr], empty(s));
+    else if (rw == RW_MAX / 2 || RW_MAX == 2)
+      grouped_unit<MB, (RW_MAX >= 2 ? RW_MAX / 2 : 1), PLANES>(
+          wrow, K, qs, Mc, rows, lane, n0, p.N[pr], qsum, saf, p.out[pr], p.sw[pr], p.sw_len[pr],
+          empty(s));
+    else
+      grouped_unit<MB, (RW_MAX >= 4 ? RW_MAX / 4 : 1), PLANES>(
+          wrow, K, qs, Mc, rows, lane, n0, p.N[pr], qsum, saf, p.out[pr], p.sw[pr], p.sw_len[pr],
+          empty(s));
   }
 }
 
