@@ -304,8 +304,8 @@ void partition_units(GroupedParams& gp, int grid, int cw) {
 
 template <int MB, int RW_MAX>
 bitnet_status launch_grouped_t(GroupedParams& gp, size_t smem, int sms, cudaStream_t st) {
-  auto k = gemv_grouped_kernel<16, MB, RW_MAX>;
-  constexpr int threads = 17 * 32;
+  auto k = gemv_grouped_kernel<kGroupedCW, MB, RW_MAX>;
+  constexpr int threads = (kGroupedCW + 1) * 32;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return BITNET_ERR_CUDA;
@@ -317,13 +317,13 @@ bitnet_status launch_grouped_t(GroupedParams& gp, size_t smem, int sms, cudaStre
   if (grid > gp.units) grid = gp.units;
   if (grid > kGroupGridMax) grid = kGroupGridMax;
   if (grid < 1) grid = 1;
-  partition_units(gp, grid, 16);
+  partition_units(gp, grid, kGroupedCW);
   return launch_pdl(k, dim3(grid), dim3(threads), smem, st, gp);
 }
 
 // The most weight rows a consumer warp takes per unit, by activation-row
-// bucket (at most 16 accumulator registers per lane).
-constexpr int grouped_rw_max(int mb) { return mb == 1 ? 4 : mb == 2 ? 2 : mb == 4 ? 4 : mb == 8 ? 2 : 1; }
+// bucket (at most 32 accumulator registers per lane).
+constexpr int grouped_rw_max(int mb) { return mb == 1 ? 8 : mb == 2 ? 4 : mb == 4 ? 8 : mb == 8 ? 4 : 1; }
 
 // Launch up to kGroupMax problems (all K % 64 == 0, validated) in one kernel.
 bitnet_status run_gemv_grouped(const bitnet_gemv_problem* pr, int count, int M, cudaStream_t st) {
@@ -336,13 +336,13 @@ bitnet_status run_gemv_grouped(const bitnet_gemv_problem* pr, int count, int M, 
   gp.M = M;
   const int mb = bucket_of(M);
   const int rw_max = grouped_rw_max(mb);
-  constexpr int cw = 16;
+  constexpr int cw = kGroupedCW;
   int units = 0;
   int64_t kmax = 0;
   size_t stage = 0;
   for (int i = 0; i < count; ++i) {
     const int64_t K = pr[i].K, N = pr[i].N, KB = K / 4;
-    int rw = pow2_floor(kGemvStageTarget / (cw * KB));
+    int rw = pow2_floor(kGroupedStageTarget / (cw * KB));
     if (rw > rw_max) rw = rw_max;
     if (rw < 1) rw = 1;
     gp.unit0[i] = units;

@@ -67,6 +67,44 @@ __device__ __forceinline__ int bytesum_s8(uint32_t w) {
   return __dp4a(static_cast<int>(w), 0x01010101, 0);
 }
 
+// NW words per lane (t0, t0 + 32, ...) of one warp's RW rows against one or
+// two activation rows, on four plane accumulators: every shared-memory load is
+// issued before the first use, so the warp waits for one round of loads.
+// `valid` false (a ragged tail) makes the lane add nothing.
+template <int MB, int RW, int NW, bool FULL>
+__device__ __forceinline__ void planes_block(int (&acc)[RW][MB][4], const uint32_t* __restrict__ wrow,
+                                             int words, const uint8_t* __restrict__ qs, int K,
+                                             int Mc, int rows, int t0, bool valid) {
+  uint4 Q[NW][MB];
+  uint32_t w[NW][RW];
+#pragma unroll
+  for (int j = 0; j < NW; ++j) {
+    const int t = t0 + 32 * j;
+#pragma unroll
+    for (int m = 0; m < MB; ++m)
+      Q[j][m] = (valid && (MB == 1 || m < Mc)) ? *reinterpret_cast<const uint4*>(qs + m * K + 16 * t)
+                                               : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+      w[j][r] = (valid && (FULL || r < rows)) ? wrow[r * words + t] : 0u;  // zero adds nothing
+  }
+#pragma unroll
+  for (int j = 0; j < NW; ++j)
+#pragma unroll
+    for (int r = 0; r < RW; ++r) {
+      const uint32_t v = w[j][r];
+      const uint32_t p0 = v & 0x03030303u, p1 = v & 0x0C0C0C0Cu;
+      const uint32_t p2 = v & 0x30303030u, p3 = v & 0xC0C0C0C0u;
+#pragma unroll
+      for (int m = 0; m < MB; ++m) {
+        acc[r][m][0] = dp4a_s32(p0, Q[j][m].x, acc[r][m][0]);
+        acc[r][m][1] = dp4a_s32(p1, Q[j][m].y, acc[r][m][1]);
+        acc[r][m][2] = dp4a_s32(p2, Q[j][m].z, acc[r][m][2]);
+        acc[r][m][3] = dp4a_us(p3, Q[j][m].w, acc[r][m][3]);
+      }
+    }
+}
+
 // Partial dot products of one warp's RW rows of a stage with the quantised
 // activation rows, for lane `lane` (words lane, lane + 32, ...).
 // PLANES: four plane accumulators per (row, activation row); else one.
@@ -76,47 +114,19 @@ __device__ __forceinline__ void gemv_rows(int (&acc)[RW][MB][PLANES ? 4 : 1],
                                           const uint8_t* __restrict__ qs, int K, int Mc,
                                           int rows, int lane) {
   if constexpr (PLANES) {
-    // One or two activation rows: two words per lane per iteration (t0 and
-    // t0 + 32), every shared-memory load of an iteration issued before its
-    // first use, so a warp waits for one round of loads per two words.
+    // Two words per lane per iteration while 64 remain, then one word; the
+    // loop bounds are warp-uniform.
+    int base = 0;
 #pragma unroll 1
-    for (int t0 = lane; t0 < words; t0 += 64) {
-      const int t1 = t0 + 32;
-      const bool has1 = t1 < words;
-      uint4 Q0[MB], Q1[MB];
-      uint32_t w0[RW], w1[RW];
-#pragma unroll
-      for (int m = 0; m < MB; ++m) {
-        const bool mv = MB == 1 || m < Mc;
-        Q0[m] = mv ? *reinterpret_cast<const uint4*>(qs + m * K + 16 * t0) : make_uint4(0, 0, 0, 0);
-        Q1[m] = (mv && has1) ? *reinterpret_cast<const uint4*>(qs + m * K + 16 * t1)
-                             : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int r = 0; r < RW; ++r) {
-        const bool rv = FULL || r < rows;
-        w0[r] = rv ? wrow[r * words + t0] : 0u;
-        w1[r] = (rv && has1) ? wrow[r * words + t1] : 0u;  // zero weights add nothing
-      }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint4* Q = h == 0 ? Q0 : Q1;
-        const uint32_t* wv = h == 0 ? w0 : w1;
-#pragma unroll
-        for (int r = 0; r < RW; ++r) {
-          const uint32_t w = wv[r];
-          const uint32_t p0 = w & 0x03030303u, p1 = w & 0x0C0C0C0Cu;
-          const uint32_t p2 = w & 0x30303030u, p3 = w & 0xC0C0C0C0u;
-#pragma unroll
-          for (int m = 0; m < MB; ++m) {
-            acc[r][m][0] = dp4a_s32(p0, Q[m].x, acc[r][m][0]);
-            acc[r][m][1] = dp4a_s32(p1, Q[m].y, acc[r][m][1]);
-            acc[r][m][2] = dp4a_s32(p2, Q[m].z, acc[r][m][2]);
-            acc[r][m][3] = dp4a_us(p3, Q[m].w, acc[r][m][3]);
-          }
-        }
-      }
+    for (; base + 64 <= words; base += 64)
+      planes_block<MB, RW, 2, FULL>(acc, wrow, words, qs, K, Mc, rows, base + lane, true);
+    if (base + 32 <= words) {
+      planes_block<MB, RW, 1, FULL>(acc, wrow, words, qs, K, Mc, rows, base + lane, true);
+      base += 32;
     }
+    if (base < words)
+      planes_block<MB, RW, 1, FULL>(acc, wrow, words, qs, K, Mc, rows, base + lane,
+                                    base + lane < words);
   } else {
     // Many activation rows: planes of the warp's rows first, then one
     // activation word at a time (keeps the registers bounded).

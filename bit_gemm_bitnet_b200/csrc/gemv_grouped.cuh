@@ -16,6 +16,11 @@ namespace bitnet {
 
 constexpr int kGroupMax = 256;       // problems per launch (kernel parameter space)
 constexpr int kGroupGridMax = 512;   // CTAs per launch
+constexpr int kGroupedCW = 16;       // consumer warps per CTA
+// Bytes per unit (aim): large units spread a unit's fixed cost (the wait, the
+// warp reduction, the stores) over more rows; two or three stages of the
+// ring still cover the memory latency.
+constexpr int kGroupedStageTarget = 80 * 1024;
 
 struct GroupedParams {
   int count;               // problems in this launch
@@ -59,9 +64,28 @@ __device__ __forceinline__ void grouped_unit(const uint32_t* wrow, int K, const 
   gemv_reduce_store<MB, RW, PLANES>(acc, rows, n0, Mc, 0, N, qsum, saf, out, nullptr, sw, sw_len);
 }
 
+// grouped_unit for the power of two rw <= RW: the instantiation with RW = rw.
+template <int MB, int RW, bool PLANES>
+__device__ __forceinline__ void grouped_unit_rw(int rw, const uint32_t* wrow, int K, const uint8_t* qs,
+                                                int Mc, int rows, int lane, int n0, int N,
+                                                const int* qsum, const float* saf, uint16_t* out,
+                                                const float* sw, int sw_len, uint32_t empty_bar) {
+  if constexpr (RW == 1) {
+    grouped_unit<MB, 1, PLANES>(wrow, K, qs, Mc, rows, lane, n0, N, qsum, saf, out, sw, sw_len,
+                                empty_bar);
+  } else {
+    if (rw >= RW)
+      grouped_unit<MB, RW, PLANES>(wrow, K, qs, Mc, rows, lane, n0, N, qsum, saf, out, sw, sw_len,
+                                   empty_bar);
+    else
+      grouped_unit_rw<MB, RW / 2, PLANES>(rw, wrow, K, qs, Mc, rows, lane, n0, N, qsum, saf, out,
+                                          sw, sw_len, empty_bar);
+  }
+}
+
 // CW consumer warps; MB activation-row bucket; RW_MAX the most rows a warp
-// takes per unit (a problem's own count, RW_MAX, RW_MAX / 2 or RW_MAX / 4,
-// picks the instantiation, so no work is spent on absent rows). Every K is a
+// takes per unit (a problem's own count, a power of two, picks the
+// instantiation, so no work is spent on absent rows). Every K is a
 // multiple of 64 (16-byte aligned rows). CTA c takes the units
 // cta_u0[c] .. cta_u0[c + 1] - 1 (ranges balanced by bytes on the host).
 template <int CW, int MB, int RW_MAX>
@@ -79,7 +103,7 @@ __global__ void __launch_bounds__((CW + 1) * 32)
   uint32_t* red = reinterpret_cast<uint32_t*>(smem + 512);
   uint8_t* qs = smem + kGemvHeaderBytes;
   uint8_t* ring = qs + p.q_bytes;
-  static_assert(kGemvMaxConsumerWarps * MB * 4 <= kGemvHeaderBytes - 512, "reduction scratch");
+  static_assert(CW * MB * 4 <= kGemvHeaderBytes - 512, "reduction scratch");
 
   const int S = p.stages;
   const int Mc = MB == 1 ? 1 : p.M;
@@ -158,17 +182,8 @@ __global__ void __launch_bounds__((CW + 1) * 32)
 
     const uint32_t* wrow = reinterpret_cast<const uint32_t*>(
         ring + static_cast<size_t>(s) * p.stage_bytes + static_cast<size_t>(r0) * KB);
-    if (rw == RW_MAX || RW_MAX == 1)
-      grouped_unit<MB, RW_MAX, PLANES>(wrow, K, qs, Mc, rows, lane, n0, p.N[pr], qsum, saf,
-                                       p.out[pr], p.sw[pr], p.sw_len[pr], empty(s));
-    else if (rw == RW_MAX / 2 || RW_MAX == 2)
-      grouped_unit<MB, (RW_MAX >= 2 ? RW_MAX / 2 : 1), PLANES>(
-          wrow, K, qs, Mc, rows, lane, n0, p.N[pr], qsum, saf, p.out[pr], p.sw[pr], p.sw_len[pr],
-          empty(s));
-    else
-      grouped_unit<MB, (RW_MAX >= 4 ? RW_MAX / 4 : 1), PLANES>(
-          wrow, K, qs, Mc, rows, lane, n0, p.N[pr], qsum, saf, p.out[pr], p.sw[pr], p.sw_len[pr],
-          empty(s));
+    grouped_unit_rw<MB, RW_MAX, PLANES>(rw, wrow, K, qs, Mc, rows, lane, n0, p.N[pr], qsum, saf,
+                                        p.out[pr], p.sw[pr], p.sw_len[pr], empty(s));
   }
 }
 
