@@ -124,27 +124,46 @@ __global__ void __launch_bounds__((CW + 1) * 32)
   __syncthreads();
   pdl_launch_dependents();
 
-  // problem of the first unit of this CTA
+  // problem of the first unit of this CTA: the last i with unit0[i] <= u_begin
   int pr = 0;
-  while (pr < p.count - 1 && u_begin >= p.unit0[pr + 1]) ++pr;
+  for (int lo = 0, hi = p.count - 1; lo <= hi;) {
+    const int mid = (lo + hi) >> 1;
+    if (p.unit0[mid] <= u_begin) {
+      pr = mid;
+      lo = mid + 1;
+    } else {
+      hi = mid - 1;
+    }
+  }
+  // the current problem's fields, held in registers: kernel parameters read
+  // with a run-time index are fetched again on every use
+  int u0 = p.unit0[pr], u1 = p.unit0[pr + 1];
 
   if (warp == CW) {
     // ------------------------------------------------------------ producer
+    int KB = p.K[pr] / 4, rpu = CW * p.rw[pr], N = p.N[pr];
+    const uint8_t* wp = p.wp[pr];
     uint32_t it = 0;
     for (int u = u_begin; u < u_end; ++u, ++it) {
-      while (u >= p.unit0[pr + 1]) ++pr;
+      while (u >= u1) {
+        ++pr;
+        u0 = u1;
+        u1 = p.unit0[pr + 1];
+        KB = p.K[pr] / 4;
+        rpu = CW * p.rw[pr];
+        N = p.N[pr];
+        wp = p.wp[pr];
+      }
       const int s = it % S;
       const uint32_t ph = (it / S) & 1u;
       if (!mbar_wait(empty(s), ph ^ 1u, abort)) break;
-      const int KB = p.K[pr] / 4;
-      const int rpu = CW * p.rw[pr];
-      const int row0 = (u - p.unit0[pr]) * rpu;
-      const int rows = min(rpu, p.N[pr] - row0);
+      const int row0 = (u - u0) * rpu;
+      const int rows = min(rpu, N - row0);
       if (lane == 0) {
         const uint32_t bytes = static_cast<uint32_t>(rows) * KB;
         mbar_arrive_expect_tx(full(s), bytes);
         bulk_load(smem_u32(ring + static_cast<size_t>(s) * p.stage_bytes),
-                  p.wp[pr] + static_cast<int64_t>(row0) * KB, bytes, full(s));
+                  wp + static_cast<int64_t>(row0) * KB, bytes, full(s));
       }
     }
     const uint32_t first = it > static_cast<uint32_t>(S) ? it - S : 0u;
@@ -157,11 +176,23 @@ __global__ void __launch_bounds__((CW + 1) * 32)
   const GemvSmem sh{qsum, saf, rq_s, rq_r, red, qs};
   int staged = -1;     // problem whose activations are in shared memory
   bool dead = false;   // a wait gave up: keep the barrier sequence, skip work
+  int K = 0, N = 0, rw = 1, sw_len = 1;
+  const float* sw = nullptr;
+  uint16_t* out = nullptr;
   uint32_t it = 0;
   for (int u = u_begin; u < u_end; ++u, ++it) {
-    while (u >= p.unit0[pr + 1]) ++pr;
-    const int K = p.K[pr];
+    while (u >= u1) {
+      ++pr;
+      u0 = u1;
+      u1 = p.unit0[pr + 1];
+    }
     if (pr != staged) {
+      K = p.K[pr];
+      N = p.N[pr];
+      rw = p.rw[pr];
+      sw_len = p.sw_len[pr];
+      sw = p.sw[pr];
+      out = p.out[pr];
       // every consumer warp reaches each problem switch at the same unit
       // (the staging only reads the activations, so it also runs after a
       // wait gave up: every consumer warp keeps the same barrier sequence)
@@ -174,16 +205,15 @@ __global__ void __launch_bounds__((CW + 1) * 32)
     const uint32_t ph = (it / S) & 1u;
     if (!dead && !mbar_wait(full(s), ph, abort)) dead = true;
     const int KB = K / 4;
-    const int rw = p.rw[pr];
     const int r0 = warp * rw;
-    const int n0 = (u - p.unit0[pr]) * (CW * rw) + r0;
-    int rows = min(rw, p.N[pr] - n0);
+    const int n0 = (u - u0) * (CW * rw) + r0;
+    int rows = min(rw, N - n0);
     if (rows < 0 || dead) rows = 0;
 
     const uint32_t* wrow = reinterpret_cast<const uint32_t*>(
         ring + static_cast<size_t>(s) * p.stage_bytes + static_cast<size_t>(r0) * KB);
-    grouped_unit_rw<MB, RW_MAX, PLANES>(rw, wrow, K, qs, Mc, rows, lane, n0, p.N[pr], qsum, saf,
-                                        p.out[pr], p.sw[pr], p.sw_len[pr], empty(s));
+    grouped_unit_rw<MB, RW_MAX, PLANES>(rw, wrow, K, qs, Mc, rows, lane, n0, N, qsum, saf, out, sw,
+                                        sw_len, empty(s));
   }
 }
 
