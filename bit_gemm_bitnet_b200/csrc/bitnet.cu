@@ -267,37 +267,47 @@ bitnet_status run_gemv(GemvParams p, bool preq, cudaStream_t st) {
 }
 
 // ------------------------------------------------------------ grouped GEMV
-// Split the units of a group over `grid` CTAs so that every CTA streams about
-// the same weight bytes (units differ in size from problem to problem). A
-// unit costs its bytes plus a fixed share for its epilogue.
+// Split the units of a group over `grid` CTAs so that every CTA does about the
+// same work. Units differ in bytes from problem to problem, and a byte costs
+// more when a warp takes fewer rows (each activation load serves fewer rows):
+// a unit's cost is its bytes x (rw + 0.72) / rw, and starting a problem (its
+// activations quantised into shared memory) costs as much as 110 KB of
+// weights. Both figures were fitted to per-CTA cycle counts of the decode
+// sweep of a 2B-parameter model.
 void partition_units(GroupedParams& gp, int grid, int cw) {
-  constexpr int64_t kUnitCost = 8192;
+  constexpr int64_t kProblemCost = 110 * 1024;
+  auto unit_cost = [&](int i, int64_t rows) {
+    const int64_t rw = gp.rw[i];
+    return rows * (gp.K[i] / 4) * (100 * rw + 72) / (100 * rw);
+  };
   int64_t total = 0;
   for (int i = 0; i < gp.count; ++i) {
     const int64_t n = gp.unit0[i + 1] - gp.unit0[i];
     if (n == 0) continue;
-    const int64_t KB = gp.K[i] / 4, rpu = static_cast<int64_t>(cw) * gp.rw[i];
-    total += (n - 1) * (rpu * KB + kUnitCost) + (gp.N[i] - (n - 1) * rpu) * KB + kUnitCost;
+    const int64_t rpu = static_cast<int64_t>(cw) * gp.rw[i];
+    total += kProblemCost + (n - 1) * unit_cost(i, rpu) + unit_cost(i, gp.N[i] - (n - 1) * rpu);
   }
   int c = 1;
-  int64_t cum = 0;  // cost of the units before problem i
+  int64_t cum = 0;  // cost of the problems before problem i
   gp.cta_u0[0] = 0;
   for (int i = 0; i < gp.count && c < grid; ++i) {
     const int64_t n = gp.unit0[i + 1] - gp.unit0[i];
     if (n == 0) continue;
-    const int64_t KB = gp.K[i] / 4, rpu = static_cast<int64_t>(cw) * gp.rw[i];
-    const int64_t cf = rpu * KB + kUnitCost;
+    const int64_t rpu = static_cast<int64_t>(cw) * gp.rw[i];
+    const int64_t cf = unit_cost(i, rpu);
+    // cost before unit k of problem i: cum for k = 0, cum + P + k * cf after
     while (c < grid) {
       const int64_t T = total * c / grid;
       if (T <= cum) {
         gp.cta_u0[c++] = gp.unit0[i];
         continue;
       }
-      const int64_t k = (T - cum + cf - 1) / cf;  // units of problem i before the boundary
+      int64_t k = (T - cum - kProblemCost + cf - 1) / cf;
+      if (k < 1) k = 1;
       if (k > n - 1) break;
       gp.cta_u0[c++] = gp.unit0[i] + static_cast<int>(k);
     }
-    cum += (n - 1) * cf + (gp.N[i] - (n - 1) * rpu) * KB + kUnitCost;
+    cum += kProblemCost + (n - 1) * cf + unit_cost(i, gp.N[i] - (n - 1) * rpu);
   }
   while (c <= grid) gp.cta_u0[c++] = gp.units;
 }
