@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the LLaMA GEMV (M <= 15) and mid-batch GEMM sections")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--branches", type=int, default=16,
@@ -371,8 +373,8 @@ def lm_head_alone(bn, d, dev, reps=20):
 def prefill(bn, dev, pk, reps=5):
     """The prefill workload: M in {2048, 8192} x four FFN shapes through
     bitnet_linear (per-token quantisation + tensor-core GEMM, bf16 out), each
-    timed with CUDA events with L2 flushed between repetitions. Also the public
-    bitnet_gemm on pre-quantised activations for the first shape."""
+    timed with CUDA events with L2 flushed between repetitions; and the GEMM
+    alone (bitnet_gemm on activations quantised beforehand) for every case."""
     flush = torch.empty((2 * L2_BYTES,), dtype=torch.uint8, device=dev)
     peak = pk["bf16_tflops"] * INT8_OVER_BF16
 
@@ -390,7 +392,7 @@ def prefill(bn, dev, pk, reps=5):
         return statistics.median(ts)
 
     Mmax = max(W.PREFILL_M)
-    cases, tot_ops, tot_ms = [], 0.0, 0.0
+    cases, tot_ops, tot_ms, tot_gemm_ms = [], 0.0, 0.0, 0.0
     gemm_pub = None
     for K, N in W.PREFILL_SHAPES:
         x = synth.act_bf16(synth.key(W.W_PREFILL, Mmax, synth.T_ACT, K), Mmax, K)
@@ -407,22 +409,29 @@ def prefill(bn, dev, pk, reps=5):
                              device=dev)
             ms = timed(lambda: bn.bitnet_linear(xd, wp, swd, out=out, workspace=ws))
             ops = 2.0 * M * N * K
-            cases.append({"M": M, "K": K, "N": N, "ms": ms, "tops": ops / ms / 1e9})
+            # the GEMM alone: bitnet_gemm on activations quantised beforehand
+            xq, sa = bn.bitnet_quantize_act(xd)
+            g_ms = timed(lambda: bn.bitnet_gemm(xq, wp, sa, swd, out=out))
+            del xq, sa
+            cases.append({"M": M, "K": K, "N": N, "ms": ms, "tops": ops / ms / 1e9,
+                          "gemm_ms": g_ms, "gemm_tops": ops / g_ms / 1e9})
             tot_ops += ops
             tot_ms += ms
+            tot_gemm_ms += g_ms
             if gemm_pub is None and M == Mmax:
-                xq, sa = bn.bitnet_quantize_act(xd)
-                g_ms = timed(lambda: bn.bitnet_gemm(xq, wp, sa, swd, out=out))
                 gemm_pub = {"M": M, "K": K, "N": N, "ms": g_ms, "tops": ops / g_ms / 1e9,
                             "frac": ops / g_ms / 1e9 / peak}
-                del xq, sa
             del out, ws
         del xd_all, wp
     bn.bitnet_device_status()
     tops = tot_ops / tot_ms / 1e9
+    gemm_tops = tot_ops / tot_gemm_ms / 1e9
     return {"workload": "M in {2048, 8192} x (4096->11008, 11008->4096, 2560->6912, "
                         "6912->2560) through bitnet_linear (quantise + GEMM)",
             "tops": tops, "ms_total": tot_ms, "cases": cases,
+            "gemm_only": {"tops": gemm_tops, "ms_total": tot_gemm_ms, "peak": peak,
+                          "frac": gemm_tops / peak,
+                          "kernel": "gemm_i8_ts_kernel via bitnet_gemm (pre-quantised)"},
             "roofline": {"bound": "tensor", "achieved": tops, "peak": peak, "unit": "TOPS",
                          "frac": tops / peak,
                          "peak_source": f"{pk['source']} bf16 burst x {INT8_OVER_BF16:g} "
@@ -431,6 +440,100 @@ def prefill(bn, dev, pk, reps=5):
                                    "(timed together)",
                          "traffic": recorded_traffic("gemm_i8_ts_kernel")},
             "bitnet_gemm_natural_layout": gemm_pub}
+
+
+# ------------------------------------------------- decode and mid-batch
+
+def weight_rotation(wp):
+    """Independent device copies of a packed weight tensor, together more than
+    twice the L2 size, so that a loop over them reads the weights from HBM."""
+    n = max(2, -(-2 * L2_BYTES // wp.numel()) + 1)
+    return [wp.clone() for _ in range(n)]
+
+
+def time_rotation(fns, reps=20, warmup=3):
+    """Median ms per call of one CUDA graph that issues every call in `fns`
+    (one call per weight copy), over `reps` replays."""
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for fn in fns:
+            fn()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for fn in fns:
+                fn()
+        for _ in range(warmup):
+            g.replay()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        ev[0].record(s)
+        for i in range(reps):
+            g.replay()
+            ev[i + 1].record(s)
+    torch.cuda.synchronize()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(reps)]
+    del g
+    return statistics.median(per) / len(fns)
+
+
+def llama_gemv(bn, dev, pk):
+    """LLaMA-7B projections at M in {1, 4, 8, 15} through bitnet_gemv_fused
+    (quantisation fused), weights rotated over copies larger than 2x L2."""
+    hbm = pk["hbm_gbs"]
+    cases = []
+    for v, (name, K, N) in enumerate(W.LLAMA_GEMV_SHAPES):
+        w = synth.ternary(synth.key(W.W_LLAMA_GEMV, 1, synth.T_WEIGHT, v), N, K)
+        copies = weight_rotation(bn.bitnet_pack_weights(torch.from_numpy(w).to(dev)))
+        del w
+        swd = torch.from_numpy(synth.scale_wt(synth.key(W.W_LLAMA_GEMV, 1, synth.T_SCALE_WT, v))).to(dev)
+        for M in W.LLAMA_GEMV_M:
+            x = synth.act_bf16(synth.key(W.W_LLAMA_GEMV, M, synth.T_ACT, v), M, K)
+            xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+            out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ms = time_rotation([lambda c=c: bn.bitnet_gemv_fused(xd, c, swd, out=out)
+                                for c in copies])
+            gbs = call_bytes(M, K, N) / ms / 1e6
+            cases.append({"M": M, "K": K, "N": N, "ms": ms, "gbs": gbs, "frac_hbm": gbs / hbm,
+                          "tops": 2.0 * M * N * K / ms / 1e9})
+        del copies
+    bn.bitnet_device_status()
+    return {"workload": "LLaMA-7B projections 4096->4096, 4096->11008, 11008->4096 at "
+                        "M in {1, 4, 8, 15} through bitnet_gemv_fused",
+            "l2": "weights rotated over copies totalling more than 2x L2",
+            "peak_hbm_gbs": hbm, "cases": cases}
+
+
+def midbatch(bn, dev, pk):
+    """M in {32, 64, 128, 256}, K=4096, N in {4096, 11008} through bitnet_gemm
+    on pre-quantised activations; each case against the roof that applies
+    (HBM bytes or tensor ops, whichever takes longer)."""
+    hbm = pk["hbm_gbs"]
+    tops_peak = pk["bf16_tflops"] * INT8_OVER_BF16
+    cases = []
+    for K, N in W.MIDBATCH_SHAPES:
+        w = synth.ternary(synth.key(W.W_MIDBATCH, 0, synth.T_WEIGHT, N), N, K)
+        copies = weight_rotation(bn.bitnet_pack_weights(torch.from_numpy(w).to(dev)))
+        del w
+        swd = torch.from_numpy(synth.scale_wt(synth.key(W.W_MIDBATCH, 0, synth.T_SCALE_WT, N))).to(dev)
+        for M in W.MIDBATCH_M:
+            x = synth.act_bf16(synth.key(W.W_MIDBATCH, M, synth.T_ACT, N), M, K, outliers=False)
+            xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+            xq, sa = bn.bitnet_quantize_act(xd)
+            out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ms = time_rotation([lambda c=c: bn.bitnet_gemm(xq, c, sa, swd, out=out)
+                                for c in copies])
+            ops = 2.0 * M * N * K
+            byts = N * K // 4 + M * K + 2 * M + 2 * M * N + 4
+            t_hbm, t_tc = byts / hbm / 1e6, ops / tops_peak / 1e9
+            cases.append({"M": M, "K": K, "N": N, "ms": ms, "tops": ops / ms / 1e9,
+                          "gbs": byts / ms / 1e6,
+                          "bound": "hbm" if t_hbm >= t_tc else "tensor",
+                          "frac": max(t_hbm, t_tc) / ms})
+        del copies
+    bn.bitnet_device_status()
+    return {"workload": "M in {32, 64, 128, 256} x K=4096 x N in {4096, 11008} through "
+                        "bitnet_gemm (pre-quantised int8 + bf16 scales)",
+            "l2": "weights rotated over copies totalling more than 2x L2",
+            "peak_hbm_gbs": hbm, "peak_tops": tops_peak, "cases": cases}
 
 
 # ----------------------------------------------------------- CPU oracle
@@ -588,6 +691,8 @@ def main():
     clocks = clk.summary()
     lm = lm_head_alone(bn, d, dev)
     pre = None if args.no_prefill else prefill(bn, dev, pk)
+    gemv_mb = None if args.no_secondary else llama_gemv(bn, dev, pk)
+    mid = None if args.no_secondary else midbatch(bn, dev, pk)
 
     if rank != 0:
         if pg is not None:
@@ -619,6 +724,8 @@ def main():
             for o in ("independent", "layer", "stream")},
         "lm_head_alone": {**lm, "frac": lm["gbs"] / pk["hbm_gbs"]},
         "prefill": pre,
+        "llama_gemv": gemv_mb,
+        "midbatch": mid,
     }
     print(json.dumps(line))
     if pg is not None:

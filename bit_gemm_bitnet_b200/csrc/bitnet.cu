@@ -347,14 +347,31 @@ bitnet_status run_gemv_grouped(const bitnet_gemv_problem* pr, int count, int M, 
   const int mb = bucket_of(M);
   const int rw_max = grouped_rw_max(mb);
   constexpr int cw = kGroupedCW;
+  auto rw_of = [&](int i, int shift) {
+    int rw = pow2_floor(kGroupedStageTarget / (cw * (pr[i].K / 4)));
+    if (rw > rw_max) rw = rw_max;
+    rw >>= shift;
+    return rw < 1 ? 1 : rw;
+  };
+  // Smaller units while the group has fewer than two per SM (a small group,
+  // or one problem alone), so that every SM streams.
+  int shift = 0;
+  for (;; ++shift) {
+    int64_t u = 0;
+    bool all_one = true;
+    for (int i = 0; i < count; ++i) {
+      const int rw = rw_of(i, shift);
+      all_one = all_one && rw == 1;
+      u += (pr[i].N + cw * rw - 1) / (cw * rw);
+    }
+    if (u >= 2 * dev->sms || all_one) break;
+  }
   int units = 0;
   int64_t kmax = 0;
   size_t stage = 0;
   for (int i = 0; i < count; ++i) {
     const int64_t K = pr[i].K, N = pr[i].N, KB = K / 4;
-    int rw = pow2_floor(kGroupedStageTarget / (cw * KB));
-    if (rw > rw_max) rw = rw_max;
-    if (rw < 1) rw = 1;
+    const int rw = rw_of(i, shift);
     gp.unit0[i] = units;
     gp.rw[i] = static_cast<int8_t>(rw);
     gp.K[i] = static_cast<int>(K);
