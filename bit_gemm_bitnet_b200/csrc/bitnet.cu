@@ -2,10 +2,13 @@
 //
 // Host code only validates arguments, picks a kernel variant and launches it
 // on the caller's stream; all arithmetic runs in the kernels included below.
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "../../include/bitnet.h"
 #include "common.cuh"
+#include "gemm_sk.cuh"
 #include "gemm_ts.cuh"
 #include "gemv.cuh"
 #include "gemv_grouped.cuh"
@@ -37,6 +40,28 @@ bitnet_status launch_pdl(Kernel k, dim3 grid, dim3 block, size_t smem,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, args...);
+  return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+}
+
+// PDL launch of clusters of `cluster_x` consecutive CTAs.
+template <typename Kernel, typename... Args>
+bitnet_status launch_pdl_cluster(Kernel k, dim3 grid, dim3 block, size_t smem, int cluster_x,
+                                 cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, k, args...);
   return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
 }
@@ -414,6 +439,99 @@ bool gemm_tc_ok(const int8_t* xq, const uint8_t* wp, int64_t K) {
   return (K % 64) == 0 && aligned(xq, 16) && aligned(wp, 16);
 }
 
+// ------------------------------------------------- few-row GEMM (M <= 256)
+
+constexpr int64_t kSkMaxRows = 256;  // activation rows the split-K kernel takes
+
+// Clusters of `split` CTAs of `kernel` that fit on the GPU at once (cached).
+int sk_clusters(const void* kernel, int split, int smem) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_pair(kernel, split);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(split * 64));
+  cfg.blockDim = dim3(sk::NUM_THREADS);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(split);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) n = 0;
+  cache[key] = n;
+  return n;
+}
+
+// Split of the K loop: the S (1..8, at most the number of K blocks) that
+// minimises waves x (K blocks per CTA + a fixed cost of about four K blocks
+// per CTA: its start, the reduction and the epilogue).
+template <typename Kernel>
+int sk_split(Kernel kernel, int smem, int64_t w_tiles, int64_t kblocks) {
+  int best = 1;
+  int64_t best_cost = INT64_MAX;
+  for (int S = 1; S <= sk::MAX_SPLIT && S <= kblocks; ++S) {
+    const int fit = sk_clusters(reinterpret_cast<const void*>(kernel), S, smem);
+    if (fit < 1) continue;
+    const int64_t waves = (w_tiles + fit - 1) / fit;
+    const int64_t cost = waves * ((kblocks + S - 1) / S + 4);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = S;
+    }
+  }
+  return best;
+}
+
+template <int BX, bool kAccOut, bool kPerm>
+bitnet_status launch_sk(const CUtensorMap& mx, const CUtensorMap& mw, void* out,
+                        const uint16_t* sa, const float* sw, int64_t sw_len,
+                        const int32_t* rowsum, int64_t M, int64_t N, int64_t K, cudaStream_t st) {
+  auto kernel = sk::gemm_i8_sk_kernel<BX, kAccOut, kPerm>;
+  constexpr int smem = sk::Cfg<BX>::SMEM_BYTES;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return BITNET_ERR_CUDA;
+  const int64_t w_tiles = (N + sk::BW - 1) / sk::BW;
+  const int64_t kblocks = (K + sk::BK - 1) / sk::BK;
+  const int S = sk_split(kernel, smem, w_tiles, kblocks);
+  if (w_tiles * S > INT32_MAX) return BITNET_ERR_SHAPE;
+  return launch_pdl_cluster(kernel, dim3(static_cast<unsigned>(w_tiles * S)),
+                            dim3(sk::NUM_THREADS), smem, S, st, mx, mw, out, sa, sw,
+                            static_cast<int>(sw_len), rowsum, static_cast<int>(M),
+                            static_cast<int>(N), static_cast<int>(K), S);
+}
+
+template <int BX>
+bitnet_status run_sk_bx(void* out, bool acc_out, const int8_t* xq, const uint8_t* wp,
+                        const uint16_t* sa, const float* sw, int64_t sw_len, int64_t M,
+                        int64_t N, int64_t K, cudaStream_t st, bool perm,
+                        const int32_t* rowsum) {
+  CUtensorMap mx, mw;
+  if (!make_map_u8(&mx, xq, M, K, K, BX, sk::BK, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_u8(&mw, wp, N, K / 4, K / 4, sk::BW, sk::BK / 4, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return BITNET_ERR_CUDA;
+  if (acc_out) return launch_sk<BX, true, false>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st);
+  if (perm) return launch_sk<BX, false, true>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st);
+  return launch_sk<BX, false, false>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st);
+}
+
+bitnet_status run_gemm_sk(void* out, bool acc_out, const int8_t* xq, const uint8_t* wp,
+                          const uint16_t* sa, const float* sw, int64_t sw_len, int64_t M,
+                          int64_t N, int64_t K, cudaStream_t st, bool perm,
+                          const int32_t* rowsum) {
+  if (M <= 16) return run_sk_bx<16>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum);
+  if (M <= 32) return run_sk_bx<32>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum);
+  if (M <= 64) return run_sk_bx<64>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum);
+  if (M <= 128) return run_sk_bx<128>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum);
+  return run_sk_bx<256>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum);
+}
+
 // perm: x_q has transposed 16-element groups and rowsum holds its per-row
 // code sums (the layout of bitnet_linear's workspace); tensor-core path only.
 bitnet_status run_gemm(void* out, bool acc_out, const int8_t* xq, const uint8_t* wp,
@@ -436,6 +554,7 @@ bitnet_status run_gemm(void* out, bool acc_out, const int8_t* xq, const uint8_t*
     p.K = static_cast<int>(K);
     return run_gemv(p, true, st);
   }
+  if (M <= kSkMaxRows) return run_gemm_sk(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum);
   DeviceInfo* dev = nullptr;
   bitnet_status s = device_info(&dev);
   if (s != BITNET_OK) return s;

@@ -14,7 +14,7 @@
 //   warp 1      TMEM owner, MMA issuer (one thread)
 //   warps 4-7   epilogue: tcgen05.ld, fp32 scales, bf16 (or int32) stores
 //   warps 8-15  unpack: packed codes -> int8 -> tcgen05.st into the A stage
-//               (two warps per TMEM sub-partition, 16 columns each)
+//               (two groups of four warps on alternate stages)
 // Waits are bounded like the other kernels of this library.
 #pragma once
 #include "common.cuh"
@@ -31,7 +31,8 @@ constexpr int WP_BYTES = BW * BK / 4;   //  4 KB
 constexpr int STAGE_BYTES = X_BYTES + WP_BYTES;
 constexpr int NUM_THREADS = 512;
 constexpr int TMEM_COLS = 512;
-constexpr int A_COL0 = 2 * BX;          // first A-stage column
+constexpr int NACC = 2;                 // accumulator buffers (epilogue overlaps the next tile)
+constexpr int A_COL0 = NACC * BX;       // first A-stage column
 constexpr int A_COLS = BK / 4;          // 32 columns per A stage
 constexpr int BAR_BYTES = 256;
 constexpr int EPI_BYTES = 4 * 32 * 32 * 4;  // per epilogue warp: one 32 x 32 chunk
@@ -125,10 +126,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(sm.full(s), 1);
-      mbar_init(sm.unpacked(s), 8);
+      mbar_init(sm.unpacked(s), 4);
       mbar_init(sm.empty(s), 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < NACC; ++a) {
       mbar_init(sm.tfull(a), 1);
       mbar_init(sm.tempty(a), 4);
     }
@@ -179,8 +180,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t it = 0, local = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
-        const int a = local & 1;
-        const uint32_t aph = (local >> 1) & 1u;
+        const int a = static_cast<int>(local % NACC);
+        const uint32_t aph = (local / NACC) & 1u;
         if (!mbar_wait(sm.tempty(a), aph ^ 1u, abort)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * BX);
@@ -210,13 +211,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int quarter = warp & 3;
     uint32_t local = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
-      const int a = local & 1;
-      const uint32_t aph = (local >> 1) & 1u;
+      const int a = static_cast<int>(local % NACC);
+      const uint32_t aph = (local / NACC) & 1u;
       const int m0 = (t / w_tiles) * BX;
       const int n = (t % w_tiles) * BW + quarter * 32 + lane;
       float swn = 0.0f;
       if (!kAccOut && n < N) swn = scale_wt[sw_len == 1 ? 0 : n];
-      if (!mbar_wait(sm.tfull(a), aph, abort)) break;
+      if (!mbar_wait_warp(sm.tfull(a), aph, abort)) break;
       tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < BX / 32; ++c) {
@@ -276,35 +277,48 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp >= 8) {
     // -------------------------------------------------------------- unpack
-    // warp -> TMEM sub-partition warp % 4 (weight rows 32 * (warp % 4) ...)
-    // and half (warp - 8) / 4 of the stage's 32 columns (64 K elements)
+    // Two groups of four warps take alternate stages, so two stages are
+    // unpacked at once (a stage's unpack is a chain of dependent steps: wait,
+    // load, unpack, tensor-memory store, wait for the store, arrive). Warp ->
+    // TMEM sub-partition warp % 4 (weight rows 32 * (warp % 4) ...), all 32
+    // columns (128 K elements) of its group's stages.
     const int sub = warp & 3;
-    const int half = (warp - 8) >> 2;
+    const uint32_t group = static_cast<uint32_t>((warp - 8) >> 2);
     const int r = sub * 32 + lane;  // weight row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(sub * 32) << 16;
     uint32_t it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
       for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        if ((it & 1u) != group) continue;
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1u;
-        if (!mbar_wait(sm.full(s), ph, abort)) { ok = false; break; }
-        const uint4 p = *reinterpret_cast<const uint4*>(sm.wp(s) + r * 32 + half * 16);
-        uint32_t o[16];
+        if (!mbar_wait_warp(sm.full(s), ph, abort)) { ok = false; break; }
+        const uint4 p0 = *reinterpret_cast<const uint4*>(sm.wp(s) + r * 32);
+        const uint4 p1 = *reinterpret_cast<const uint4*>(sm.wp(s) + r * 32 + 16);
+        uint32_t o[16], o2[16];
         if constexpr (kPerm) {
-          planes_of(p.x, o + 0);
-          planes_of(p.y, o + 4);
-          planes_of(p.z, o + 8);
-          planes_of(p.w, o + 12);
+          planes_of(p0.x, o + 0);
+          planes_of(p0.y, o + 4);
+          planes_of(p0.z, o + 8);
+          planes_of(p0.w, o + 12);
+          planes_of(p1.x, o2 + 0);
+          planes_of(p1.y, o2 + 4);
+          planes_of(p1.z, o2 + 8);
+          planes_of(p1.w, o2 + 12);
         } else {
-          signed_of(p.x, o + 0);
-          signed_of(p.y, o + 4);
-          signed_of(p.z, o + 8);
-          signed_of(p.w, o + 12);
+          signed_of(p0.x, o + 0);
+          signed_of(p0.y, o + 4);
+          signed_of(p0.z, o + 8);
+          signed_of(p0.w, o + 12);
+          signed_of(p1.x, o2 + 0);
+          signed_of(p1.y, o2 + 4);
+          signed_of(p1.z, o2 + 8);
+          signed_of(p1.w, o2 + 12);
         }
-        tmem_st_32x32b_x16(tmem_base + lane_base +
-                               static_cast<uint32_t>(A_COL0 + s * A_COLS + half * 16),
-                           o);
+        const uint32_t col = tmem_base + lane_base + static_cast<uint32_t>(A_COL0 + s * A_COLS);
+        tmem_st_32x32b_x16(col, o);
+        tmem_st_32x32b_x16(col + 16u, o2);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();

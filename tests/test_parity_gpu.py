@@ -181,6 +181,29 @@ def test_gemm_matches_oracle(M, K, N):
     assert_bf16_close(bf16_bits(got), ref)
 
 
+# M <= 256 takes the split-K tensor-core kernel: one N tile (the K loop split
+# over a cluster of up to 8 CTAs), a ragged last K block (K % 128 == 64), a
+# ragged N, every activation-row width (16 ... 256) and a few splits.
+SK_CASES = [(33, 4096, 128), (2, 192, 130), (17, 640, 1000), (64, 8256, 200),
+            (256, 1024, 4096), (100, 2560, 131), (1, 11008, 4099), (129, 64, 256),
+            (16, 4096, 11008)]
+
+
+@pytest.mark.parametrize("M,K,N", SK_CASES)
+def test_gemm_split_k_bitexact_and_oracle(M, K, N):
+    rng = np.random.default_rng(M * 31 + K + N)
+    q = rng.integers(-127, 128, size=(M, K)).astype(np.int8)
+    w = weights(99, N, N, K)
+    p = oracle.pack(w)
+    pd = to_dev(p)
+    acc = bn.bitnet_gemm_acc_i32(to_dev(q), pd)
+    assert np.array_equal(acc.cpu().numpy(), oracle.acc(q, p))
+    sa = f32_to_bf16_bits(rng.uniform(0.001, 0.05, size=M).astype(np.float32))
+    sw = synth.uniform_f32(synth.key(99, N, 3), N, 0.01, 0.1)
+    got = bn.bitnet_gemm(to_dev(q), pd, to_dev(sa, torch.bfloat16), to_dev(sw))
+    assert_bf16_close(bf16_bits(got), oracle.gemm(q, p, sa, sw))
+
+
 def test_gemm_extreme_accumulators():
     # |acc| = 127 * K at the largest K of the workloads
     K, M, N = 11008, 3, 256
@@ -255,7 +278,8 @@ def test_linear_workspace_errors():
 
 
 @pytest.mark.parametrize("M,K,N", [(130, 384, 300), (257, 2560, 520), (16, 11008, 256),
-                                   (200, 160, 64), (129, 4096, 4099)])
+                                   (200, 160, 64), (129, 4096, 4099), (256, 2560, 640),
+                                   (31, 6912, 2560), (64, 4160, 96)])
 def test_linear_split_path_ragged(M, K, N):
     """M >= 16: quantise into the workspace, then the GEMM (tensor-core path
     with transposed groups and row sums when K % 64 == 0, SIMT otherwise)."""
