@@ -329,21 +329,67 @@ def time_graph(g, steps, warmup, barrier):
     return ev[0].elapsed_time(ev[-1]), per
 
 
-def time_e2e(g, d, steps, warmup, barrier):
-    def step():
-        d["x_dev"].copy_(d["x_host"], non_blocking=True)
-        g.replay()
-        d["out_host"].copy_(d["out_dev"], non_blocking=True)
-    for _ in range(warmup):
-        step()
+def second_buffers(d, dev):
+    """A copy of the decode set-up with its own device activation and output
+    buffers (same weights), for double-buffered end-to-end steps."""
+    d2 = dict(d)
+    d2["x_dev"] = torch.empty_like(d["x_dev"])
+    d2["out_dev"] = torch.empty_like(d["out_dev"])
+    d2["out_host"] = torch.empty_like(d["out_host"]).pin_memory()
+    xs, outs = [], []
+    xo = oo = 0
+    for _, _, K, N in d["calls"]:
+        xs.append(d2["x_dev"][xo:xo + K].view(1, K))
+        outs.append(d2["out_dev"][oo:oo + N].view(1, N))
+        xo += K
+        oo += N
+    d2["xs"], d2["outs"] = xs, outs
+    return d2
+
+
+def time_e2e(graphs, ds, steps, warmup, barrier):
+    """End to end through the C ABI, every step copying its activations from
+    pinned host memory and its outputs back. Two buffer sets alternate, so
+    the upload of step i+1 and the download of step i-1 run on their own
+    streams while step i computes (a serving loop's double buffering)."""
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_up = [torch.cuda.Event() for _ in ds]
+    ev_comp = [torch.cuda.Event() for _ in ds]
+    ev_down = [torch.cuda.Event() for _ in ds]
+
+    def step(i):
+        b = i % len(ds)
+        d = ds[b]
+        up.wait_event(ev_comp[b])        # step i-2 has finished reading x_dev[b]
+        with torch.cuda.stream(up):
+            d["x_dev"].copy_(d["x_host"], non_blocking=True)
+        ev_up[b].record(up)
+        comp.wait_event(ev_up[b])
+        comp.wait_event(ev_down[b])      # step i-2's outputs have been read back
+        graphs[b].replay()
+        ev_comp[b].record(comp)
+        down.wait_event(ev_comp[b])
+        with torch.cuda.stream(down):
+            d["out_host"].copy_(d["out_dev"], non_blocking=True)
+        ev_down[b].record(down)
+
+    def drain():
+        for b in range(len(ds)):
+            comp.wait_event(ev_down[b])
+
+    for i in range(warmup):
+        step(i)
+    drain()
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        step()
-    e1.record()
+    e0.record(comp)
+    for i in range(steps):
+        step(i)
+    drain()
+    e1.record(comp)
     torch.cuda.synchronize()
     barrier()
     return e0.elapsed_time(e1)
@@ -657,9 +703,16 @@ def main():
 
     pk = peaks()
     d = build_decode(bn, dev, rank)
+    d2 = second_buffers(d, dev)
     stream = torch.cuda.Stream(device=dev)
     graphs = {}
     with torch.cuda.stream(stream):
+        sweep2 = make_sweep(bn, d2, "grouped")
+        sweep2()
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2, stream=stream):
+            sweep2()
+        torch.cuda.synchronize()
         for order in ("grouped", "independent", "layer", "stream"):
             sweep = make_sweep(bn, d, order, branches=args.branches)
             sweep()
@@ -672,7 +725,7 @@ def main():
             graphs[order] = g
         with ClockSampler(local) as clk:
             total_ms, per = time_graph(graphs["grouped"], args.steps, args.warmup, barrier)
-        e2e_ms = time_e2e(graphs["grouped"], d, args.steps, args.warmup, barrier)
+        e2e_ms = time_e2e([graphs["grouped"], g2], [d, d2], args.steps, args.warmup, barrier)
         other = {}
         for order in ("independent", "layer", "stream"):
             t_ms, _ = time_graph(graphs[order], args.steps, args.warmup, barrier)

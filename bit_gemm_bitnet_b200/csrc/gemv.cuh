@@ -105,18 +105,61 @@ __device__ __forceinline__ void planes_block(int (&acc)[RW][MB][4], const uint32
     }
 }
 
+// Four consecutive words per lane (t = base + 4 lane ... + 3) of one warp's RW
+// rows: one 128-bit load per row, four 128-bit activation loads (the QUAD
+// layout of q_pos), every load issued before the first use.
+template <int MB, int RW, bool FULL>
+__device__ __forceinline__ void planes_quad(int (&acc)[RW][MB][4], const uint32_t* __restrict__ wrow,
+                                            int words, const uint8_t* __restrict__ qs, int K,
+                                            int Mc, int rows, int base, int lane) {
+  uint4 Q[4][MB];
+  uint4 w[RW];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int m = 0; m < MB; ++m)
+      Q[j][m] = (MB == 1 || m < Mc)
+                    ? *reinterpret_cast<const uint4*>(qs + m * K + 16 * (base + 32 * j + lane))
+                    : make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int r = 0; r < RW; ++r)
+    w[r] = (FULL || r < rows) ? *reinterpret_cast<const uint4*>(wrow + r * words + base + 4 * lane)
+                              : make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int r = 0; r < RW; ++r) {
+      const uint32_t v = j == 0 ? w[r].x : j == 1 ? w[r].y : j == 2 ? w[r].z : w[r].w;
+      const uint32_t p0 = v & 0x03030303u, p1 = v & 0x0C0C0C0Cu;
+      const uint32_t p2 = v & 0x30303030u, p3 = v & 0xC0C0C0C0u;
+#pragma unroll
+      for (int m = 0; m < MB; ++m) {
+        acc[r][m][0] = dp4a_s32(p0, Q[j][m].x, acc[r][m][0]);
+        acc[r][m][1] = dp4a_s32(p1, Q[j][m].y, acc[r][m][1]);
+        acc[r][m][2] = dp4a_s32(p2, Q[j][m].z, acc[r][m][2]);
+        acc[r][m][3] = dp4a_us(p3, Q[j][m].w, acc[r][m][3]);
+      }
+    }
+}
+
 // Partial dot products of one warp's RW rows of a stage with the quantised
 // activation rows, for lane `lane` (words lane, lane + 32, ...).
 // PLANES: four plane accumulators per (row, activation row); else one.
-template <int MB, int RW, bool PLANES, bool FULL>
+template <int MB, int RW, bool PLANES, bool FULL, bool QUAD = false>
 __device__ __forceinline__ void gemv_rows(int (&acc)[RW][MB][PLANES ? 4 : 1],
                                           const uint32_t* __restrict__ wrow, int words,
                                           const uint8_t* __restrict__ qs, int K, int Mc,
                                           int rows, int lane) {
   if constexpr (PLANES) {
-    // Two words per lane per iteration while 64 remain, then one word; the
-    // loop bounds are warp-uniform.
+    // (QUAD) four consecutive words per lane over every whole block of 128
+    // words; then two words per lane per iteration while 64 remain, then one
+    // word. The loop bounds are warp-uniform.
     int base = 0;
+    if constexpr (QUAD) {
+#pragma unroll 1
+      for (; base + 128 <= words; base += 128)
+        planes_quad<MB, RW, FULL>(acc, wrow, words, qs, K, Mc, rows, base, lane);
+    }
 #pragma unroll 1
     for (; base + 64 <= words; base += 64)
       planes_block<MB, RW, 2, FULL>(acc, wrow, words, qs, K, Mc, rows, base + lane, true);
@@ -174,7 +217,20 @@ struct GemvSmem {
   uint8_t* qs;
 };
 
-template <int CW, int MB>
+// Position of 16-byte activation group g in shared memory. With QUAD, the
+// groups of every whole block of 128 are permuted so that group 128b + 4l + j
+// sits at 128b + 32j + l: lane l's four consecutive groups of a block are then
+// read by four conflict-free 128-bit loads (one per j, lanes consecutive).
+// Groups after the last whole block keep their place.
+template <bool QUAD>
+__device__ __forceinline__ int q_pos(int g, int full_end) {
+  if constexpr (QUAD) {
+    if (g < full_end) return (g & ~127) | ((g & 3) << 5) | ((g >> 2) & 31);
+  }
+  return g;
+}
+
+template <int CW, int MB, bool QUAD = false>
 __device__ __forceinline__ void gemv_stage_activations(const GemvSmem& sh, const uint16_t* __restrict__ x,
                                                        int K, int Mc, int8_t* dbg_q, uint16_t* dbg_sa) {
   constexpr int kGemvConsumerWarps = CW;
@@ -244,7 +300,7 @@ __device__ __forceinline__ void gemv_stage_activations(const GemvSmem& sh, const
           const int q2 = quant_one(bf16_bits_to_f32(v.y & 0xFFFFu), rqm);
           const int q3 = quant_one(bf16_bits_to_f32(v.y >> 16), rqm);
           qs_part[m] += q0 + q1 + q2 + q3;
-          uint8_t* d = qrow + 16 * (u >> 2) + (u & 3);
+          uint8_t* d = qrow + 16 * q_pos<QUAD>(u >> 2, (K / 16) & ~127) + (u & 3);
           d[0] = static_cast<uint8_t>(q0);
           d[4] = static_cast<uint8_t>(q1);
           d[8] = static_cast<uint8_t>(q2);

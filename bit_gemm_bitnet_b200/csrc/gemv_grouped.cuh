@@ -56,9 +56,9 @@ __device__ __forceinline__ void grouped_unit(const uint32_t* wrow, int K, const 
 #pragma unroll
       for (int i = 0; i < (PLANES ? 4 : 1); ++i) acc[r][m][i] = 0;
   if (rows == RW)
-    gemv_rows<MB, RW, PLANES, true>(acc, wrow, K / 16, qs, K, Mc, rows, lane);
+    gemv_rows<MB, RW, PLANES, true, PLANES>(acc, wrow, K / 16, qs, K, Mc, rows, lane);
   else if (rows > 0)
-    gemv_rows<MB, RW, PLANES, false>(acc, wrow, K / 16, qs, K, Mc, rows, lane);
+    gemv_rows<MB, RW, PLANES, false, PLANES>(acc, wrow, K / 16, qs, K, Mc, rows, lane);
   __syncwarp();
   if (lane == 0) mbar_arrive(empty_bar);
   gemv_reduce_store<MB, RW, PLANES>(acc, rows, n0, Mc, 0, N, qsum, saf, out, nullptr, sw, sw_len);
@@ -89,7 +89,7 @@ __device__ __forceinline__ void grouped_unit_rw(int rw, const uint32_t* wrow, in
 // multiple of 64 (16-byte aligned rows). CTA c takes the units
 // cta_u0[c] .. cta_u0[c + 1] - 1 (ranges balanced by bytes on the host).
 template <int CW, int MB, int RW_MAX>
-__global__ void __launch_bounds__((CW + 1) * 32)
+__global__ void __launch_bounds__((CW + 1) * 32, 1)
     gemv_grouped_kernel(const __grid_constant__ GroupedParams p) {
   constexpr int kConsumers = CW * 32;
   constexpr bool PLANES = MB <= 2;
@@ -197,7 +197,7 @@ __global__ void __launch_bounds__((CW + 1) * 32)
       // (the staging only reads the activations, so it also runs after a
       // wait gave up: every consumer warp keeps the same barrier sequence)
       if (staged >= 0) named_barrier_sync(1, kConsumers);
-      gemv_stage_activations<CW, MB>(sh, p.x[pr], K, Mc, nullptr, nullptr);
+      gemv_stage_activations<CW, MB, PLANES>(sh, p.x[pr], K, Mc, nullptr, nullptr);
       named_barrier_sync(1, kConsumers);
       staged = pr;
     }

@@ -296,7 +296,7 @@ def test_linear_split_path_ragged(M, K, N):
 @pytest.mark.parametrize("M", [1, 2, 4, 15])
 def test_gemv_fused_grouped_matches_oracle_and_single_calls(M):
     shapes = [(2560, 2560), (2560, 640), (6912, 300), (96, 40), (512, 1), (4096, 1000),
-              (128, 77)]
+              (128, 77), (2112, 130), (8192, 64)]
     xs, wps, sws, host = [], [], [], []
     for i, (K, N) in enumerate(shapes):
         x = acts(99, 10 * M + i, M, K)
