@@ -9,6 +9,7 @@
 #include "../../include/bitnet.h"
 #include "common.cuh"
 #include "gemm_sk.cuh"
+#include "gemm_skq.cuh"
 #include "gemm_ts.cuh"
 #include "gemv.cuh"
 #include "gemv_grouped.cuh"
@@ -532,6 +533,52 @@ bitnet_status run_gemm_sk(void* out, bool acc_out, const int8_t* xq, const uint8
   return run_sk_bx<256>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum);
 }
 
+// ------------------------------ fused quantise + tensor-core GEMV (4 <= M)
+
+constexpr int64_t kSkqMinRows = 8;  // fewer rows: the dp4a GEMV (measured faster there)
+
+bool skq_ok(const void* x, const uint8_t* wp, int64_t M, int64_t K) {
+  return M >= kSkqMinRows && M <= skq::BX && K % 64 == 0 && aligned(x, 16) && aligned(wp, 16);
+}
+
+bitnet_status run_gemv_skq(uint16_t* out, const uint16_t* x, const uint8_t* wp,
+                           const float* sw, int64_t sw_len, int64_t M, int64_t N, int64_t K,
+                           cudaStream_t st) {
+  auto kernel = skq::gemv_i8_skq_kernel;
+  constexpr int smem = skq::SMEM_BYTES;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return BITNET_ERR_CUDA;
+  CUtensorMap mw;
+  if (!make_map_u8(&mw, wp, N, K / 4, K / 4, skq::BW, skq::BK / 4, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return BITNET_ERR_CUDA;
+  const int64_t w_tiles = (N + skq::BW - 1) / skq::BW;
+  const int64_t kblocks = (K + skq::BK - 1) / skq::BK;
+  // the split as for the few-row GEMM, with at most MAX_KB K blocks per CTA
+  // (the resident activations) and at most QMAX activation items per thread
+  int best = 0;
+  int64_t best_cost = INT64_MAX;
+  for (int S = 1; S <= sk::MAX_SPLIT && S <= kblocks; ++S) {
+    const int64_t per_cta = (kblocks + S - 1) / S;
+    if (per_cta > skq::MAX_KB || per_cta * (skq::BK / 4) * M > skq::NUM_THREADS * skq::QMAX)
+      continue;
+    const int fit = sk_clusters(reinterpret_cast<const void*>(kernel), S, smem);
+    if (fit < 1) continue;
+    const int64_t waves = (w_tiles + fit - 1) / fit;
+    const int64_t cost = waves * ((kblocks + S - 1) / S + 4);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = S;
+    }
+  }
+  if (best == 0) return BITNET_ERR_SHAPE;
+  if (w_tiles * best > INT32_MAX) return BITNET_ERR_SHAPE;
+  return launch_pdl_cluster(kernel, dim3(static_cast<unsigned>(w_tiles * best)),
+                            dim3(skq::NUM_THREADS), smem, best, st, mw, out, x, sw,
+                            static_cast<int>(sw_len), static_cast<int>(M), static_cast<int>(N),
+                            static_cast<int>(K), best);
+}
+
 // perm: x_q has transposed 16-element groups and rowsum holds its per-row
 // code sums (the layout of bitnet_linear's workspace); tensor-core path only.
 bitnet_status run_gemm(void* out, bool acc_out, const int8_t* xq, const uint8_t* wp,
@@ -770,6 +817,11 @@ bitnet_status bitnet_gemv_fused(uint16_t* out, const void* x, bitnet_dtype dt,
   p.out = out;
   p.sw = scale_wt;
   p.sw_len = static_cast<int>(scale_wt_len);
+  if (skq_ok(x, w_packed, M, K) && K / 128 <= sk::MAX_SPLIT * skq::MAX_KB) {
+    const bitnet_status r = run_gemv_skq(out, static_cast<const uint16_t*>(x), w_packed,
+                                         scale_wt, scale_wt_len, M, N, K, as_stream(stream));
+    if (r != BITNET_ERR_SHAPE) return r;
+  }
   return run_gemv(p, false, as_stream(stream));
 }
 

@@ -58,11 +58,30 @@ __device__ __forceinline__ RowQuant row_quant(float absmax) {
 // |x/s| * 3 * 2^-24 <= 2.3e-5 (|x/s| <= ~127), so whenever y is at least
 // 1e-4 away from a half-integer both round to the same integer. Only inputs
 // within 1e-4 of a tie take the true IEEE division.
+// rint is the magic-number method: for |y| < 2^22, y + 1.5 * 2^23 lies in
+// [2^23, 2^24), where the spacing of floats is 1, so the IEEE addition itself
+// rounds y to the nearest integer, halves to even; that integer is the sum's
+// bit pattern minus the pattern of 1.5 * 2^23, and subtracting 1.5 * 2^23
+// back is exact. (Two adds on the FMA pipe instead of the conversion pipe.)
+__device__ __forceinline__ int rint_small(float y, float* r) {
+  const float t = __fadd_rn(y, 12582912.0f);
+  *r = __fsub_rn(t, 12582912.0f);
+  return __float_as_int(t) - 0x4B400000;
+}
+
+// The exact quotient of a near-tie, out of line: ties are rare, and kept out
+// of the callers' code the IEEE division is neither executed for every
+// element nor repeated in every unrolled copy of a quantisation loop.
+__device__ __noinline__ int quant_tie(float x, float s) {
+  float r;
+  return rint_small(__fdiv_rn(x, s), &r);
+}
+
 __device__ __forceinline__ int quant_one(float x, const RowQuant& q) {
   float y = __fmul_rn(x, q.r);
-  const float d = y - floorf(y);
-  if (fabsf(d - 0.5f) < 1e-4f) y = __fdiv_rn(x, q.s);
-  int v = __float2int_rn(y);
+  float ry;
+  int v = rint_small(y, &ry);
+  if (fabsf(fabsf(__fsub_rn(y, ry)) - 0.5f) < 1e-4f) v = quant_tie(x, q.s);
   v = v < -127 ? -127 : v;
   v = v > 127 ? 127 : v;
   return v;
@@ -373,6 +392,15 @@ __device__ __forceinline__ uint4 dsmem_ld_v4(uint32_t saddr, uint32_t rank) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "r"(remote)
                : "memory");
+  return v;
+}
+
+// 4 bytes of CTA `rank`'s shared memory at the address that `saddr` has in
+// this CTA's shared window.
+__device__ __forceinline__ uint32_t dsmem_ld_u32(uint32_t saddr, uint32_t rank) {
+  uint32_t remote, v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(saddr), "r"(rank));
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
   return v;
 }
 
