@@ -112,7 +112,7 @@ def test_quantize_rejects_bad_shape():
 
 GEMV_CASES = [(1, 512, 512), (4, 512, 512), (1, 2560, 640), (2, 96, 40), (3, 160, 33),
               (15, 4096, 300), (8, 11008, 130), (1, 2560, 128256 // 16), (5, 6912, 2560),
-              (1, 32, 1), (9, 1024, 4099)]
+              (1, 32, 1), (9, 1024, 4099), (12, 2112, 77), (10, 64, 5), (14, 8256, 260)]
 
 
 @pytest.mark.parametrize("M,K,N", GEMV_CASES)
