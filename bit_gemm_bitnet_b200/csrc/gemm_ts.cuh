@@ -8,7 +8,9 @@
 // per 128-K stage the shared-memory traffic is the activation tile (written
 // by TMA, read by the MMA) and the small packed weight tile.
 //
-// TMEM (512 columns): two 192-column accumulators + four 32-column A stages.
+// TMEM (512 columns): two 192-column accumulators + four 32-column A stages;
+// shared memory holds six stages of activation and packed tiles (the two
+// rings are separate, so TMA runs further ahead than tensor memory allows).
 // Warp roles (512 threads), persistent (one CTA per SM):
 //   warp 0      TMA producer (x tile, 128-byte swizzle; packed weight tile)
 //   warp 1      TMEM owner, MMA issuer (one thread)
@@ -25,7 +27,8 @@ namespace ts {
 constexpr int BW = 128;                 // weight rows per tile (MMA M)
 constexpr int BX = 192;                 // activation rows per tile (MMA N)
 constexpr int BK = 128;                 // K per stage
-constexpr int STAGES = 4;
+constexpr int STAGES = 6;                // shared-memory stages (activation + packed tiles)
+constexpr int ASTAGES = 4;               // tensor-memory A stages (unpacked weights)
 constexpr int X_BYTES = BX * BK;        // 24 KB
 constexpr int WP_BYTES = BW * BK / 4;   //  4 KB
 constexpr int STAGE_BYTES = X_BYTES + WP_BYTES;
@@ -38,7 +41,7 @@ constexpr int BAR_BYTES = 256;
 constexpr int EPI_BYTES = 4 * 32 * 32 * 4;  // per epilogue warp: one 32 x 32 chunk
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + EPI_BYTES;
 static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment");
-static_assert(A_COL0 + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
+static_assert(A_COL0 + ASTAGES * A_COLS <= TMEM_COLS, "TMEM budget");
 static_assert(SMEM_BYTES <= 232448, "too much shared memory");
 
 // int32 D, A (weights) unsigned code planes or signed int8, B signed int8,
@@ -57,16 +60,19 @@ struct Smem {
     return reinterpret_cast<uint64_t*>(base + STAGES * STAGE_BYTES);
   }
   __device__ uint32_t full(int s) const { return smem_u32(bars() + s); }
-  __device__ uint32_t unpacked(int s) const { return smem_u32(bars() + STAGES + s); }
-  __device__ uint32_t empty(int s) const { return smem_u32(bars() + 2 * STAGES + s); }
-  __device__ uint32_t tfull(int a) const { return smem_u32(bars() + 3 * STAGES + a); }
-  __device__ uint32_t tempty(int a) const { return smem_u32(bars() + 3 * STAGES + 2 + a); }
-  __device__ uint32_t drain() const { return smem_u32(bars() + 3 * STAGES + 4); }
+  __device__ uint32_t empty(int s) const { return smem_u32(bars() + STAGES + s); }
+  // tensor-memory A stage a: unpacked (4 unpack warps arrive) / free again
+  // (the MMAs that read it have completed)
+  __device__ uint32_t unpacked(int a) const { return smem_u32(bars() + 2 * STAGES + a); }
+  __device__ uint32_t afree(int a) const { return smem_u32(bars() + 2 * STAGES + ASTAGES + a); }
+  __device__ uint32_t tfull(int a) const { return smem_u32(bars() + 2 * STAGES + 2 * ASTAGES + a); }
+  __device__ uint32_t tempty(int a) const { return smem_u32(bars() + 2 * STAGES + 2 * ASTAGES + 2 + a); }
+  __device__ uint32_t drain() const { return smem_u32(bars() + 2 * STAGES + 2 * ASTAGES + 4); }
   __device__ uint32_t* tmem_slot() const {
-    return reinterpret_cast<uint32_t*>(bars() + 3 * STAGES + 5);
+    return reinterpret_cast<uint32_t*>(bars() + 2 * STAGES + 2 * ASTAGES + 5);
   }
   __device__ int* abort_flag() const {
-    return reinterpret_cast<int*>(bars() + 3 * STAGES + 6);
+    return reinterpret_cast<int*>(bars() + 2 * STAGES + 2 * ASTAGES + 6);
   }
   // warp-private staging of one 32 (activation rows) x 32 (weight rows)
   // output chunk, 4 bytes per element (bf16 outputs use the first half)
@@ -126,8 +132,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(sm.full(s), 1);
-      mbar_init(sm.unpacked(s), 4);
       mbar_init(sm.empty(s), 1);
+    }
+    for (int a = 0; a < ASTAGES; ++a) {
+      mbar_init(sm.unpacked(a), 4);
+      mbar_init(sm.afree(a), 1);
     }
     for (int a = 0; a < NACC; ++a) {
       mbar_init(sm.tfull(a), 1);
@@ -187,11 +196,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * BX);
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1u;
-          if (!mbar_wait(sm.full(s), ph, abort) ||
-              !mbar_wait(sm.unpacked(s), ph, abort)) { ok = false; break; }
+          const int as = static_cast<int>(it % ASTAGES);
+          // the unpack warps arrive only after they saw the stage's tiles land
+          // (full), so this one wait also orders the activation tile's reads
+          if (!mbar_wait(sm.unpacked(as), (it / ASTAGES) & 1u, abort)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + s * A_COLS);
+          const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + as * A_COLS);
           const uint64_t bdesc = smem_desc_sw128(smem_u32(sm.x(s)));
 #pragma unroll
           for (int k = 0; k < BK / 32; ++k) {
@@ -200,6 +210,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                           (kb > 0 || k > 0) ? 1u : 0u);
           }
           mma_commit(sm.empty(s));
+          mma_commit(sm.afree(as));
         }
         if (ok) mma_commit(sm.tfull(a));
       }
@@ -292,8 +303,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int kb = 0; kb < kblocks; ++kb, ++it) {
         if ((it & 1u) != group) continue;
         const int s = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1u;
-        if (!mbar_wait_warp(sm.full(s), ph, abort)) { ok = false; break; }
+        const int as = static_cast<int>(it % ASTAGES);
+        if (!mbar_wait_warp(sm.full(s), (it / STAGES) & 1u, abort) ||
+            !mbar_wait_warp(sm.afree(as), ((it / ASTAGES) & 1u) ^ 1u, abort)) { ok = false; break; }
         const uint4 p0 = *reinterpret_cast<const uint4*>(sm.wp(s) + r * 32);
         const uint4 p1 = *reinterpret_cast<const uint4*>(sm.wp(s) + r * 32 + 16);
         uint32_t o[16], o2[16];
@@ -316,13 +328,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           signed_of(p1.z, o2 + 8);
           signed_of(p1.w, o2 + 12);
         }
-        const uint32_t col = tmem_base + lane_base + static_cast<uint32_t>(A_COL0 + s * A_COLS);
+        const uint32_t col = tmem_base + lane_base + static_cast<uint32_t>(A_COL0 + as * A_COLS);
         tmem_st_32x32b_x16(col, o);
         tmem_st_32x32b_x16(col + 16u, o2);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(sm.unpacked(s));
+        if (lane == 0) mbar_arrive(sm.unpacked(as));
       }
     }
   }
