@@ -230,7 +230,97 @@ __device__ __forceinline__ int q_pos(int g, int full_end) {
   return g;
 }
 
-template <int CW, int MB, bool QUAD = false>
+// The staging of one or two activation rows with at most NQ quads per thread
+// (single-problem kernel): every quad is loaded once and kept in registers
+// for the quantise pass, and the code sums go to their own slots (no barrier
+// to reuse red[]).
+template <int CW, int MB, int NQ, bool QUAD>
+__device__ __forceinline__ void gemv_stage_cached(const GemvSmem& sh, const uint16_t* __restrict__ x,
+                                                  int K, int Mc, uint16_t* dbg_sa) {
+  constexpr int kGemvConsumerWarps = CW;
+  constexpr int kGemvConsumers = CW * 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int* qsum = sh.qsum;
+  float* saf = sh.saf;
+  float* rq_s = sh.rq_s;
+  float* rq_r = sh.rq_r;
+  uint32_t* red = sh.red;
+  uint8_t* qs = sh.qs;
+  const int quads = K / 4;
+  uint2 v[MB][NQ];
+  uint32_t mb[MB];
+#pragma unroll
+  for (int m = 0; m < MB; ++m) {
+    const bool live = MB == 1 || m < Mc;
+    const uint2* row = reinterpret_cast<const uint2*>(x + static_cast<int64_t>(m) * K);
+#pragma unroll
+    for (int j = 0; j < NQ; ++j) {
+      const int u = tid + j * kGemvConsumers;
+      v[m][j] = (live && u < quads) ? __ldg(row + u) : make_uint2(0u, 0u);
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < MB; ++m) {
+    mb[m] = 0;
+#pragma unroll
+    for (int j = 0; j < NQ; ++j)
+      mb[m] = max(mb[m], max(max(v[m][j].x & 0x7FFFu, (v[m][j].x >> 16) & 0x7FFFu),
+                             max(v[m][j].y & 0x7FFFu, (v[m][j].y >> 16) & 0x7FFFu)));
+    mb[m] = __reduce_max_sync(0xFFFFFFFFu, mb[m]);
+    if (lane == 0) red[warp * MB + m] = mb[m];
+  }
+  named_barrier_sync(1, kGemvConsumers);
+  if (tid < MB) {
+    uint32_t t = 0;
+    for (int w = 0; w < kGemvConsumerWarps; ++w) t = max(t, red[w * MB + tid]);
+    const RowQuant q = row_quant(bf16_bits_to_f32(t));
+    rq_s[tid] = q.s;
+    rq_r[tid] = q.r;
+    const uint16_t sb = f32_to_bf16_bits(q.s);
+    saf[tid] = bf16_bits_to_f32(sb);
+    if (dbg_sa != nullptr && tid < Mc) dbg_sa[tid] = sb;
+  }
+  named_barrier_sync(1, kGemvConsumers);
+  uint32_t* red2 = red + kGemvMaxConsumerWarps * MB;  // code sums per warp
+#pragma unroll
+  for (int m = 0; m < MB; ++m) {
+    int part = 0;
+    if (MB == 1 || m < Mc) {
+      RowQuant rqm;
+      rqm.s = rq_s[m];
+      rqm.r = rq_r[m];
+      uint8_t* qrow = qs + m * K;
+#pragma unroll
+      for (int j = 0; j < NQ; ++j) {
+        const int u = tid + j * kGemvConsumers;
+        if (u < quads) {
+          const int q0 = quant_one(bf16_bits_to_f32(v[m][j].x & 0xFFFFu), rqm);
+          const int q1 = quant_one(bf16_bits_to_f32(v[m][j].x >> 16), rqm);
+          const int q2 = quant_one(bf16_bits_to_f32(v[m][j].y & 0xFFFFu), rqm);
+          const int q3 = quant_one(bf16_bits_to_f32(v[m][j].y >> 16), rqm);
+          part += q0 + q1 + q2 + q3;
+          uint8_t* d = qrow + 16 * q_pos<QUAD>(u >> 2, (K / 16) & ~127) + (u & 3);
+          d[0] = static_cast<uint8_t>(q0);
+          d[4] = static_cast<uint8_t>(q1);
+          d[8] = static_cast<uint8_t>(q2);
+          d[12] = static_cast<uint8_t>(q3);
+        }
+      }
+    }
+    part = __reduce_add_sync(0xFFFFFFFFu, part);
+    if (lane == 0) red2[warp * MB + m] = static_cast<uint32_t>(part);
+  }
+  named_barrier_sync(1, kGemvConsumers);
+  if (tid < MB) {
+    int t = 0;
+    for (int w = 0; w < kGemvConsumerWarps; ++w) t += static_cast<int>(red2[w * MB + tid]);
+    qsum[tid] = t;
+  }
+}
+
+// CACHE: the single-problem kernel keeps one or two rows' quads in
+// registers between the passes (4 or 8 per thread, by K).
+template <int CW, int MB, bool QUAD = false, bool CACHE = false>
 __device__ __forceinline__ void gemv_stage_activations(const GemvSmem& sh, const uint16_t* __restrict__ x,
                                                        int K, int Mc, int8_t* dbg_q, uint16_t* dbg_sa) {
   constexpr int kGemvConsumerWarps = CW;
@@ -242,9 +332,19 @@ __device__ __forceinline__ void gemv_stage_activations(const GemvSmem& sh, const
   float* rq_r = sh.rq_r;
   uint32_t* red = sh.red;
   uint8_t* qs = sh.qs;
+  const int quads = K / 4;
+  if constexpr (CACHE && MB <= 2) {
+    if (dbg_q == nullptr && quads <= 4 * kGemvConsumers) {
+      gemv_stage_cached<CW, MB, 4, QUAD>(sh, x, K, Mc, dbg_sa);
+      return;
+    }
+    if (dbg_q == nullptr && quads <= 8 * kGemvConsumers) {
+      gemv_stage_cached<CW, MB, 8, QUAD>(sh, x, K, Mc, dbg_sa);
+      return;
+    }
+  }
     // absmax of every activation row; each thread owns the 4-element quads
     // tid, tid + 512, ... of a row (loops kept rolled: a small code footprint)
-    const int quads = K / 4;
     uint32_t mb[MB];
 #pragma unroll
     for (int m = 0; m < MB; ++m) {
@@ -475,7 +575,7 @@ __global__ void __launch_bounds__((CW + 1) * 32) gemv_kernel(GemvParams p) {
   pdl_wait();  // the activations may come from the previous kernel
   const int groups16 = K / 16;
   if constexpr (!PREQ) {
-    gemv_stage_activations<CW, MB>(GemvSmem{qsum, saf, rq_s, rq_r, red, qs}, p.x, K, Mc,
+    gemv_stage_activations<CW, MB, false, true>(GemvSmem{qsum, saf, rq_s, rq_r, red, qs}, p.x, K, Mc,
                                    blockIdx.x == 0 ? p.dbg_q : nullptr,
                                    blockIdx.x == 0 ? p.dbg_sa : nullptr);
   } else {
