@@ -59,7 +59,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--branches", type=int, default=16,
                     help="graph branches for the independent calls of a step")
-    ap.add_argument("--case", choices=("lm_head", "prefill", "decode_once"),
+    ap.add_argument("--case", choices=("lm_head", "prefill", "decode_once", "midbatch", "gemv_m15"),
                     help="profiling aid: run one small case a few times and exit "
                          "(no JSON line); see profiles/ for the ncu commands")
     return ap.parse_args()
@@ -538,12 +538,22 @@ def llama_gemv(bn, dev, pk):
             ms = time_rotation([lambda c=c: bn.bitnet_gemv_fused(xd, c, swd, out=out)
                                 for c in copies])
             gbs = call_bytes(M, K, N) / ms / 1e6
+            # the same problems as one grouped call (independent projections
+            # of a layer, such as Q, K and V, can be issued this way)
+            gouts = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in copies]
+            g_ms = time_rotation([lambda: bn.bitnet_gemv_fused_grouped(
+                [xd] * len(copies), copies, [swd] * len(copies), gouts)]) / len(copies)
+            del gouts
+            g_gbs = call_bytes(M, K, N) / g_ms / 1e6
             cases.append({"M": M, "K": K, "N": N, "ms": ms, "gbs": gbs, "frac_hbm": gbs / hbm,
-                          "tops": 2.0 * M * N * K / ms / 1e9})
+                          "tops": 2.0 * M * N * K / ms / 1e9,
+                          "grouped": {"problems": len(copies), "ms_per_problem": g_ms,
+                                      "gbs": g_gbs, "frac_hbm": g_gbs / hbm}})
         del copies
     bn.bitnet_device_status()
     return {"workload": "LLaMA-7B projections 4096->4096, 4096->11008, 11008->4096 at "
-                        "M in {1, 4, 8, 15} through bitnet_gemv_fused",
+                        "M in {1, 4, 8, 15} through bitnet_gemv_fused, one call at a time, "
+                        "and the same problems as one bitnet_gemv_fused_grouped call",
             "l2": "weights rotated over copies totalling more than 2x L2",
             "peak_hbm_gbs": hbm, "cases": cases}
 
@@ -621,6 +631,25 @@ def run_case(bn, dev, case, reps=3):
     if case == "decode_once":
         d = build_decode(bn, dev, 0)
         make_sweep(bn, d, "grouped")()
+    elif case in ("midbatch", "gemv_m15"):
+        # one few-row GEMM (M = 64, 4096 -> 11008, pre-quantised) or one fused
+        # tensor-core GEMV (M = 15, 11008 -> 4096), weights larger than L2
+        # across the repetitions' copies
+        M, K, N = (64, 4096, 11008) if case == "midbatch" else (15, 11008, 4096)
+        w = synth.ternary(synth.key(W.W_MIDBATCH, M, synth.T_WEIGHT, N), N, K)
+        wp = bn.bitnet_pack_weights(torch.from_numpy(w).to(dev))
+        copies = weight_rotation(wp)
+        x = synth.act_bf16(synth.key(W.W_MIDBATCH, M, synth.T_ACT, N), M, K)
+        xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+        sw = torch.tensor([0.05], dtype=torch.float32, device=dev)
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        if case == "midbatch":
+            xq, sa = bn.bitnet_quantize_act(xd)
+            for r in range(reps):
+                bn.bitnet_gemm(xq, copies[r % len(copies)], sa, sw, out=out)
+        else:
+            for r in range(reps):
+                bn.bitnet_gemv_fused(xd, copies[r % len(copies)], sw, out=out)
     elif case == "lm_head":
         _, K, N = W.DECODE_2B_LM_HEAD
         w = synth.ternary(synth.key(W.W_DECODE_2B, W.DECODE_2B_LAYERS, synth.T_WEIGHT, 7), N, K)
