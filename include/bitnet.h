@@ -90,7 +90,10 @@ bitnet_status bitnet_quantize_act(int8_t* x_q, uint16_t* scale_act,
  *   w_packed   in,  uint8 [N, K/4]
  *   scale_act  in,  bf16 [M]
  *   scale_wt   in,  fp32, scale_wt_len elements: 1 (per tensor) or N
- * Any M >= 0. */
+ * Any M >= 0. Kernels: with K % 64 == 0 and 16-byte aligned x_q and
+ * w_packed, M <= 256 runs a tensor-core kernel whose K loop is split over a
+ * thread-block cluster, and larger M a persistent tensor-core kernel;
+ * otherwise a SIMT kernel. All give the same result. */
 bitnet_status bitnet_gemm(uint16_t* out, const int8_t* x_q,
                           const uint8_t* w_packed, const uint16_t* scale_act,
                           const float* scale_wt, int64_t scale_wt_len,
@@ -105,7 +108,11 @@ bitnet_status bitnet_gemm(uint16_t* out, const int8_t* x_q,
  * Needs 1 <= M <= 15 (the page dispatches M < 16 here), and the quantised
  * rows plus one stage of sixteen weight rows must fit on chip:
  * 2048 + c(M * K) + c(4 * K) <= 232448 with c(v) = v rounded up to a
- * multiple of 128 (about (M + 4) * K <= 230000); otherwise BITNET_ERR_SHAPE. */
+ * multiple of 128 (about (M + 4) * K <= 230000); otherwise BITNET_ERR_SHAPE.
+ * Kernels: with 8 <= M, K % 64 == 0, 16-byte aligned x and w_packed and
+ * K <= 128 * 8 * min(48, floor(384 / M)), a tensor-core kernel with the
+ * quantisation inside (its K loop split over a thread-block cluster);
+ * otherwise a dp4a GEMV. Both give the same result. */
 bitnet_status bitnet_gemv_fused(uint16_t* out, const void* x, bitnet_dtype dt,
                                 const uint8_t* w_packed, const float* scale_wt,
                                 int64_t scale_wt_len, int64_t M, int64_t N,
@@ -161,8 +168,8 @@ bitnet_status bitnet_linear(uint16_t* out, const void* x, bitnet_dtype dt,
  * device memory: code running while a stream is being captured into a CUDA
  * graph (cudaMalloc is not allowed there), code inside a framework that owns
  * all device memory through its own pool, or latency-critical paths that
- * cannot afford an allocation's implicit synchronisation. The paper has no
- * counterpart; this is a convenience of this library's C ABI.
+ * cannot afford an allocation's implicit synchronisation. The bitnet-cpu page
+ * has no counterpart; this is a convenience of this library's C ABI.
  * Arguments and result are those of bitnet_linear. When M >= 16 (the split
  * path), the int8 activations and their scales are placed in a scratch array
  * built into the library: 16 MiB (16777216 bytes) per GPU, reserved by every
