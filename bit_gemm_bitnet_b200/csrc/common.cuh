@@ -316,6 +316,35 @@ __device__ __forceinline__ void tmem_st_wait() {
 }
 
 // Arrive once on the mbarrier when all prior tcgen05.mma of this thread end.
+// The four kind::i8 MMAs of one 128-wide K block (A from tensor memory,
+// columns a + 8k; B descriptor b + 2k), with a non-blocking test of the
+// mbarrier phase the next K block needs issued ahead of them: its answer is
+// read only after the four MMAs are issued, so the barrier's round trip
+// overlaps them instead of preceding the next block. Returns whether that
+// phase has completed (false: the caller waits for it).
+__device__ __forceinline__ bool mma4_i8_tmem_a_test(uint32_t d_tmem, uint32_t a_tmem,
+                                                    uint64_t bdesc, uint32_t idesc,
+                                                    uint32_t accumulate, uint32_t next_bar,
+                                                    uint32_t next_parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p, t, q;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 q, [%5], %6;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.u32 t, 0, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%1], [%2], %3, %7, p;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%1], [%8], %9, %7, t;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%1], [%10], %11, %7, t;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%1], [%12], %13, %7, t;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(ok)
+      : "r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(accumulate), "r"(next_bar), "r"(next_parity),
+        "r"(idesc), "r"(a_tmem + 8u), "l"(bdesc + 2u), "r"(a_tmem + 16u), "l"(bdesc + 4u),
+        "r"(a_tmem + 24u), "l"(bdesc + 6u)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 "

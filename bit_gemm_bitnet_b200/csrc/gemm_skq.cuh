@@ -258,20 +258,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
+      bool ready = false;  // the next block's unpack barrier already completed
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
         const int s = it % ST;
-        const uint32_t ph = (it / ST) & 1u;
-        if (!mbar_wait(sm.full(s), ph, abort) || !mbar_wait(sm.unpacked(s), ph, abort)) {
+        // the unpack warps arrive only after they saw the stage land (full),
+        // so this wait also orders the MMA's reads of the stage
+        if (!ready && !mbar_wait(sm.unpacked(s), (it / ST) & 1u, abort)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + s * A_COLS);
         const uint64_t bdesc = smem_desc_sw128(smem_u32(sm.xt(kb - kb0)));
-#pragma unroll
-        for (int k = 0; k < BK / 32; ++k)
-          mma_i8_tmem_a(tmem_base, a_tmem + 8u * k, bdesc + 2u * k, kIdesc,
-                        (kb > kb0 || k > 0) ? 1u : 0u);
+        const uint32_t nx = it + 1;
+        ready = mma4_i8_tmem_a_test(tmem_base, a_tmem, bdesc, kIdesc, kb > kb0 ? 1u : 0u,
+                                    sm.unpacked(static_cast<int>(nx % ST)), (nx / ST) & 1u);
         mma_commit(sm.empty(s));
       }
       if (ok) mma_commit(sm.tfull());

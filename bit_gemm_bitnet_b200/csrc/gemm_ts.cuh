@@ -26,7 +26,7 @@ namespace ts {
 
 constexpr int BW = 128;                 // weight rows per tile (MMA M)
 constexpr int BX = 192;                 // activation rows per tile (MMA N)
-constexpr int BK = 128;                 // K per stage
+constexpr int BK = 128;                 // K per stage (four K = 32 MMAs)
 constexpr int STAGES = 6;                // shared-memory stages (activation + packed tiles)
 constexpr int ASTAGES = 4;               // tensor-memory A stages (unpacked weights)
 constexpr int X_BYTES = BX * BK;        // 24 KB
@@ -188,6 +188,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       uint32_t it = 0, local = 0;
       bool ok = true;
+      bool ready = false;  // the next block's unpack barrier already completed
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
         const int a = static_cast<int>(local % NACC);
         const uint32_t aph = (local / NACC) & 1u;
@@ -198,17 +199,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int s = it % STAGES;
           const int as = static_cast<int>(it % ASTAGES);
           // the unpack warps arrive only after they saw the stage's tiles land
-          // (full), so this one wait also orders the activation tile's reads
-          if (!mbar_wait(sm.unpacked(as), (it / ASTAGES) & 1u, abort)) { ok = false; break; }
+          // (full), so this one wait also orders the activation tile's reads;
+          // `ready` is the look-ahead test made with the previous block's MMAs
+          if (!ready && !mbar_wait(sm.unpacked(as), (it / ASTAGES) & 1u, abort)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + as * A_COLS);
           const uint64_t bdesc = smem_desc_sw128(smem_u32(sm.x(s)));
-#pragma unroll
-          for (int k = 0; k < BK / 32; ++k) {
-            // 32 K bytes: 8 TMEM columns of A, +32 bytes inside B's swizzle atom
-            mma_i8_tmem_a(d_tmem, a_tmem + 8u * k, bdesc + 2u * k, kIdesc,
-                          (kb > 0 || k > 0) ? 1u : 0u);
-          }
+          // 4 x 32 K bytes: 8 TMEM columns of A each, +32 bytes inside B's
+          // swizzle atom; the next block's unpack barrier is tested meanwhile
+          const uint32_t nx = it + 1;
+          ready = mma4_i8_tmem_a_test(d_tmem, a_tmem, bdesc, kIdesc, kb > 0 ? 1u : 0u,
+                                      sm.unpacked(static_cast<int>(nx % ASTAGES)),
+                                      (nx / ASTAGES) & 1u);
           mma_commit(sm.empty(s));
           mma_commit(sm.afree(as));
         }
