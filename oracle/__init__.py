@@ -30,6 +30,8 @@ def lib():
         L.oracle_pack.argtypes = [_P, _I64, _I64, _P]
         L.oracle_unpack.argtypes = [_P, _I64, _I64, _P]
         L.oracle_quantize.argtypes = [_P, _I64, _I64, _P, _P]
+        L.oracle_quantize_f32.argtypes = [_P, _I64, _I64, _P, _P]
+        L.oracle_linear_f32.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P]
         L.oracle_acc.argtypes = [_P, _P, _I64, _I64, _I64, _P]
         L.oracle_epilogue.argtypes = [_P, _P, _P, _I64, _I64, _I64, _P]
         L.oracle_gemm.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]
@@ -42,7 +44,8 @@ def lib():
                                                  _I64, _P, ctypes.c_int]
         L.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
         L.oracle_f32_to_bf16.restype = ctypes.c_uint16
-        for name in ("oracle_pack", "oracle_unpack", "oracle_quantize",
+        for name in ("oracle_pack", "oracle_unpack", "oracle_quantize", "oracle_quantize_f32",
+                     "oracle_linear_f32",
                      "oracle_acc", "oracle_epilogue", "oracle_gemm",
                      "oracle_linear", "oracle_linear_threads",
                      "oracle_gemm_threads", "oracle_linear_threads_cols"):
@@ -94,6 +97,29 @@ def quantize(x_bf16_bits):
     s = np.empty((M,), np.uint16)
     _check(lib().oracle_quantize(_ptr(x), M, K, _ptr(q), _ptr(s)), "quantize")
     return q, s
+
+
+def quantize_f32(x):
+    """float32 [M, K] -> (int8 [M, K], bf16 bits [M])."""
+    x = _c(x, np.float32)
+    M, K = x.shape
+    q = np.empty((M, K), np.int8)
+    s = np.empty((M,), np.uint16)
+    _check(lib().oracle_quantize_f32(_ptr(x), M, K, _ptr(q), _ptr(s)), "quantize_f32")
+    return q, s
+
+
+def linear_f32(x, packed, scale_wt):
+    """float32 [M, K] -> bf16 bits [M, N]: quantize_f32, then gemm."""
+    x = _c(x, np.float32)
+    packed = _c(packed, np.uint8)
+    sw = _c(scale_wt, np.float32)
+    M, K = x.shape
+    N = packed.shape[0]
+    out = np.empty((M, N), np.uint16)
+    _check(lib().oracle_linear_f32(_ptr(x), _ptr(packed), _ptr(sw), sw.size, M, N, K,
+                                   _ptr(out)), "linear_f32")
+    return out
 
 
 def acc(q, packed, N=None):

@@ -106,30 +106,49 @@ int oracle_unpack(const uint8_t* packed, int64_t N, int64_t K, int8_t* w) {
   return OK;
 }
 
-// quantize_activation for bf16 rows x [M, K] (given as raw bf16 bits).
-// q int8 [M, K]; scale bf16 [M] (raw bits).
+// quantize_activation for one row of K fp32 values: absmax clamped at
+// eps = 1e-5, s = absmax / 127 (IEEE fp32 division), q = clamp(round-half-
+// even(x / s), -127, 127), scale = bf16(s).
+static void quantize_row(const float* row, int64_t K, int8_t* q, uint16_t* scale) {
+  float absmax = 0.0f;
+  for (int64_t k = 0; k < K; ++k) {
+    const float a = std::fabs(row[k]);
+    if (a > absmax) absmax = a;
+  }
+  if (absmax < 1e-5f) absmax = 1e-5f;  // clamp(min=eps)
+  const float s = absmax / 127.0f;
+  for (int64_t k = 0; k < K; ++k) {
+    const float v = row[k] / s;
+    float r = std::nearbyint(v);  // half-to-even under FE_TONEAREST
+    if (r < -127.0f) r = -127.0f;
+    if (r > 127.0f) r = 127.0f;
+    q[k] = static_cast<int8_t>(r);
+  }
+  *scale = float_to_bf16_bits_rne(s);
+}
+
+// quantize_activation for bf16 rows x [M, K] (given as raw bf16 bits; each
+// value is widened to fp32 exactly first). q int8 [M, K]; scale bf16 [M]
+// (raw bits).
 int oracle_quantize(const uint16_t* x, int64_t M, int64_t K, int8_t* q,
                     uint16_t* scale) {
   if (M < 0 || K <= 0) return ERR_SHAPE;
   std::fesetround(FE_TONEAREST);
+  std::vector<float> row(static_cast<size_t>(K));
   for (int64_t m = 0; m < M; ++m) {
-    const uint16_t* row = x + m * K;
-    float absmax = 0.0f;
-    for (int64_t k = 0; k < K; ++k) {
-      const float a = std::fabs(bf16_bits_to_float(row[k]));
-      if (a > absmax) absmax = a;
-    }
-    if (absmax < 1e-5f) absmax = 1e-5f;  // clamp(min=eps)
-    const float s = absmax / 127.0f;
-    for (int64_t k = 0; k < K; ++k) {
-      const float v = bf16_bits_to_float(row[k]) / s;
-      float r = std::nearbyint(v);  // half-to-even under FE_TONEAREST
-      if (r < -127.0f) r = -127.0f;
-      if (r > 127.0f) r = 127.0f;
-      q[m * K + k] = static_cast<int8_t>(r);
-    }
-    scale[m] = float_to_bf16_bits_rne(s);
+    for (int64_t k = 0; k < K; ++k) row[k] = bf16_bits_to_float(x[m * K + k]);
+    quantize_row(row.data(), K, q + m * K, scale + m);
   }
+  return OK;
+}
+
+// quantize_activation for fp32 rows x [M, K] (the bitnet-cpu page accepts
+// float32 activations as well as bf16).
+int oracle_quantize_f32(const float* x, int64_t M, int64_t K, int8_t* q,
+                        uint16_t* scale) {
+  if (M < 0 || K <= 0) return ERR_SHAPE;
+  std::fesetround(FE_TONEAREST);
+  for (int64_t m = 0; m < M; ++m) quantize_row(x + m * K, K, q + m * K, scale + m);
   return OK;
 }
 
@@ -193,6 +212,18 @@ int oracle_linear(const uint16_t* x, const uint8_t* packed,
   std::vector<int8_t> q(static_cast<size_t>(M) * static_cast<size_t>(K));
   std::vector<uint16_t> sa(static_cast<size_t>(M));
   int st = oracle_quantize(x, M, K, q.data(), sa.data());
+  if (st != OK) return st;
+  return oracle_gemm(q.data(), packed, sa.data(), scale_wt, scale_wt_len, M, N,
+                     K, out);
+}
+
+// bitnet_linear for fp32 rows: quantize_f32, then gemm.
+int oracle_linear_f32(const float* x, const uint8_t* packed, const float* scale_wt,
+                      int64_t scale_wt_len, int64_t M, int64_t N, int64_t K,
+                      uint16_t* out) {
+  std::vector<int8_t> q(static_cast<size_t>(M) * static_cast<size_t>(K));
+  std::vector<uint16_t> sa(static_cast<size_t>(M));
+  int st = oracle_quantize_f32(x, M, K, q.data(), sa.data());
   if (st != OK) return st;
   return oracle_gemm(q.data(), packed, sa.data(), scale_wt, scale_wt_len, M, N,
                      K, out);

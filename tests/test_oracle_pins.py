@@ -158,6 +158,45 @@ def test_quantize_matches_torch_fp32_evaluation():
     assert np.array_equal(st, s)
 
 
+def test_quantize_f32_golden_examples():
+    """fp32 rows (the bitnet-cpu page also takes float32 activations), worked
+    by hand from the page's quantize_activation: s = absmax / 127."""
+    x = np.array([[254.0, 3.0, -5.0, 1.0],            # s = 2: 1.5 -> 2, -2.5 -> -2, 0.5 -> 0
+                  [127.0, 0.3, -63.5, 1.0000001],     # s = 1: -63.5 -> -64 (even), 0.3 -> 0
+                  [0.0, 0.0, 0.0, 0.0]], np.float32)  # clamped absmax: q = 0
+    q, s = oracle.quantize_f32(x)
+    assert q.tolist() == [[127, 2, -2, 0], [127, 0, -64, 1], [0, 0, 0, 0]]
+    assert s[0] == 0x4000 and s[1] == 0x3F80
+    assert s[2] == f32_to_bf16_bits_np(np.float32(1e-5) / np.float32(127.0))
+
+
+def test_quantize_f32_matches_torch_fp32_evaluation():
+    """Library special case: the page's expression on float32 tensors."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((129, 1536)).astype(np.float32)
+    x[:, ::97] *= 20.0
+    x[0, :8] = np.array([127, 0.5, 1.5, 2.5, -0.5, -1.5, 3.5, -2.5], np.float32)  # exact ties
+    q, s = oracle.quantize_f32(x)
+    xt = torch.from_numpy(x.copy())
+    absmax = xt.abs().amax(dim=-1, keepdim=True).clamp(min=1e-5)
+    scale = absmax / 127.0
+    qt = (xt / scale).round().clamp(-127, 127).to(torch.int8)
+    st = scale.squeeze(-1).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(qt.numpy(), q)
+    assert np.array_equal(st, s)
+
+
+def test_quantize_f32_agrees_with_bf16_path_on_bf16_values():
+    """Rows whose values are bf16 give the same codes and scales either way."""
+    x = synth.act_bf16(synth.key(97, 3, synth.T_ACT), 33, 640)
+    xf = (x.astype(np.uint32) << 16).view(np.float32)
+    assert [a.tolist() for a in oracle.quantize(x)] == [a.tolist() for a in oracle.quantize_f32(xf)]
+    p = oracle.pack(synth.ternary(synth.key(97, 3, synth.T_WEIGHT), 40, 640))
+    sw = np.array([0.05], np.float32)
+    assert np.array_equal(oracle.linear(x, p, sw), oracle.linear_f32(xf, p, sw))
+
+
 def test_f32_to_bf16_matches_torch_rounding():
     torch = pytest.importorskip("torch")
     rng = np.random.default_rng(5)
