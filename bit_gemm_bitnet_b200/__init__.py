@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libbitnet_b200.so")
 OK, ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_VALUE, ERR_WORKSPACE, \
     ERR_CUDA, ERR_TIMEOUT = range(9)
 BF16 = 0
+F32 = 1
 
 # every symbol include/bitnet.h declares
 EXPORTS = (
@@ -106,6 +107,15 @@ def _stream(device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
+def _act_dt(t, name, ndim=None):
+    """Activations: bf16 or float32; returns the C dtype code."""
+    if isinstance(t, torch.Tensor) and t.dtype == torch.float32:
+        _need(t, torch.float32, name, ndim)
+        return F32
+    _need(t, torch.bfloat16, name, ndim)
+    return BF16
+
+
 def _need(t, dtype, name, ndim=None):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
@@ -146,15 +156,15 @@ def bitnet_pack_weights(w, out=None):
 
 
 def bitnet_quantize_act(x, x_q=None, scale_act=None):
-    """bf16 [..., K] -> (int8 [M, K], bf16 [M])."""
+    """bf16 or float32 [..., K] -> (int8 [M, K], bf16 [M])."""
     x2 = x.reshape(-1, x.shape[-1])
-    _need(x2, torch.bfloat16, "x", 2)
+    dt = _act_dt(x2, "x", 2)
     M, K = x2.shape
     if x_q is None:
         x_q = torch.empty((M, K), dtype=torch.int8, device=x.device)
     if scale_act is None:
         scale_act = torch.empty((M,), dtype=torch.bfloat16, device=x.device)
-    _check(lib().bitnet_quantize_act(_ptr(x_q), _ptr(scale_act), _ptr(x2), BF16, M, K,
+    _check(lib().bitnet_quantize_act(_ptr(x_q), _ptr(scale_act), _ptr(x2), dt, M, K,
                                      _stream(x.device)), "bitnet_quantize_act")
     return x_q, scale_act
 
@@ -178,8 +188,8 @@ def bitnet_gemm(x_q, w_packed, scale_act, scale_wt, out=None):
 
 
 def bitnet_gemv_fused(x, w_packed, scale_wt, out=None):
-    """bf16 [M, K] (M < 16) -> bf16 [M, N], quantisation fused."""
-    _need(x, torch.bfloat16, "x", 2)
+    """bf16 or float32 [M, K] (M < 16) -> bf16 [M, N], quantisation fused."""
+    dt = _act_dt(x, "x", 2)
     _need(w_packed, torch.uint8, "w_packed", 2)
     M, K = x.shape
     N = w_packed.shape[0]
@@ -188,7 +198,7 @@ def bitnet_gemv_fused(x, w_packed, scale_wt, out=None):
     sw = _scale_wt(scale_wt, N, x.device)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    _check(lib().bitnet_gemv_fused(_ptr(out), _ptr(x), BF16, _ptr(w_packed), _ptr(sw),
+    _check(lib().bitnet_gemv_fused(_ptr(out), _ptr(x), dt, _ptr(w_packed), _ptr(sw),
                                    sw.numel(), M, N, K, _stream(x.device)),
            "bitnet_gemv_fused")
     return out
@@ -235,12 +245,12 @@ def bitnet_linear_workspace_bytes(M, K):
 
 
 def bitnet_linear(x, w_packed, scale_wt, out=None, workspace=None):
-    """bf16 [..., K] -> bf16 [..., N]; dispatches by M like the page's
-    bitnet_linear (fused GEMV for M < 16, else quantise + GEMM)."""
+    """bf16 or float32 [..., K] -> bf16 [..., N]; dispatches by M like the
+    page's bitnet_linear (fused GEMV for M < 16, else quantise + GEMM)."""
     orig = x.shape
     K = orig[-1]
     x2 = x.reshape(-1, K)
-    _need(x2, torch.bfloat16, "x", 2)
+    dt = _act_dt(x2, "x", 2)
     _need(w_packed, torch.uint8, "w_packed", 2)
     M = x2.shape[0]
     N = w_packed.shape[0]
@@ -253,7 +263,7 @@ def bitnet_linear(x, w_packed, scale_wt, out=None, workspace=None):
     if need and (workspace is None or workspace.numel() < need):
         workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
     wsp = _ptr(workspace) if need else None
-    _check(lib().bitnet_linear(_ptr(out), _ptr(x2), BF16, _ptr(w_packed), _ptr(sw),
+    _check(lib().bitnet_linear(_ptr(out), _ptr(x2), dt, _ptr(w_packed), _ptr(sw),
                                sw.numel(), M, N, K, wsp, need, _stream(x.device)),
            "bitnet_linear")
     return out.view(*orig[:-1], N)
@@ -266,7 +276,7 @@ def bitnet_linear_noalloc(x, w_packed, scale_wt, out=None):
     orig = x.shape
     K = orig[-1]
     x2 = x.reshape(-1, K)
-    _need(x2, torch.bfloat16, "x", 2)
+    dt = _act_dt(x2, "x", 2)
     _need(w_packed, torch.uint8, "w_packed", 2)
     M = x2.shape[0]
     N = w_packed.shape[0]
@@ -275,7 +285,7 @@ def bitnet_linear_noalloc(x, w_packed, scale_wt, out=None):
     sw = _scale_wt(scale_wt, N, x.device)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    _check(lib().bitnet_linear_noalloc(_ptr(out), _ptr(x2), BF16, _ptr(w_packed), _ptr(sw),
+    _check(lib().bitnet_linear_noalloc(_ptr(out), _ptr(x2), dt, _ptr(w_packed), _ptr(sw),
                                        sw.numel(), M, N, K, _stream(x.device)),
            "bitnet_linear_noalloc")
     return out.view(*orig[:-1], N)

@@ -642,6 +642,24 @@ bitnet_status run_quantize(int8_t* xq, uint16_t* sa, const uint16_t* x, int64_t 
   return launch_pdl(quantize_rows_kernel<0>, grid, block, 0, st, xq, sa, x, static_cast<int>(K));
 }
 
+// float32 activations: the natural-layout quantiser, one CTA per row.
+bitnet_status run_quantize_f32(int8_t* xq, uint16_t* sa, const float* x, int64_t M, int64_t K,
+                               cudaStream_t st) {
+  if (M == 0) return BITNET_OK;
+  if (M > INT32_MAX) return BITNET_ERR_SHAPE;
+  return launch_pdl(quantize_rows_f32_kernel, dim3(static_cast<unsigned>(M)),
+                    dim3(kQuantThreads), 0, st, xq, sa, x, static_cast<int>(K));
+}
+
+// float32 activations: the quantiser of bitnet_linear's tensor-core path.
+bitnet_status run_quantize_perm_f32(int8_t* xq, uint16_t* sa, int32_t* rowsum, const float* x,
+                                    int64_t M, int64_t K, cudaStream_t st) {
+  if (M == 0) return BITNET_OK;
+  if (M > INT32_MAX) return BITNET_ERR_SHAPE;
+  return launch_pdl(quantize_rows_perm_f32_kernel, dim3(static_cast<unsigned>(M)),
+                    dim3(kQuantThreads), 0, st, xq, sa, rowsum, x, static_cast<int>(K));
+}
+
 // The quantiser of bitnet_linear's tensor-core path: transposed 16-element
 // groups plus per-row code sums.
 bitnet_status run_quantize_perm(int8_t* xq, uint16_t* sa, int32_t* rowsum, const uint16_t* x,
@@ -749,11 +767,13 @@ bitnet_status bitnet_pack_weights(uint8_t* w_packed, const int8_t* w, int64_t N,
 
 bitnet_status bitnet_quantize_act(int8_t* x_q, uint16_t* scale_act, const void* x,
                                   bitnet_dtype dt, int64_t M, int64_t K, void* stream) {
-  if (dt != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (dt != BITNET_BF16 && dt != BITNET_F32) return BITNET_ERR_DTYPE;
   if (M < 0 || K <= 0 || K % 32 != 0 || K > INT32_MAX) return BITNET_ERR_SHAPE;
   if (M == 0) return BITNET_OK;
   if (x_q == nullptr || scale_act == nullptr || x == nullptr) return BITNET_ERR_NULL;
   if (!aligned(x, 16) || !aligned(x_q, 16) || !aligned(scale_act, 2)) return BITNET_ERR_ALIGN;
+  if (dt == BITNET_F32)
+    return run_quantize_f32(x_q, scale_act, static_cast<const float*>(x), M, K, as_stream(stream));
   return run_quantize(x_q, scale_act, static_cast<const uint16_t*>(x), M, K,
                       as_stream(stream));
 }
@@ -788,13 +808,14 @@ bitnet_status bitnet_gemm_acc_i32(int32_t* acc, const int8_t* x_q, const uint8_t
 
 static bitnet_status gemv_common(GemvParams& p, const void* x, bitnet_dtype dt,
                                  const uint8_t* w_packed, int64_t M, int64_t N, int64_t K) {
-  if (dt != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (dt != BITNET_BF16 && dt != BITNET_F32) return BITNET_ERR_DTYPE;
   bitnet_status s = check_compute_shape(M, N, K);
   if (s != BITNET_OK) return s;
   if (M < 1 || M > kGemvMaxM || !gemv_fits(static_cast<int>(M), K)) return BITNET_ERR_SHAPE;
   if (x == nullptr || w_packed == nullptr) return BITNET_ERR_NULL;
   if (!aligned(x, 16) || !aligned(w_packed, 16)) return BITNET_ERR_ALIGN;
-  p.x = static_cast<const uint16_t*>(x);
+  p.x = x;
+  p.x_f32 = dt == BITNET_F32 ? 1 : 0;
   p.wp = w_packed;
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
@@ -817,7 +838,7 @@ bitnet_status bitnet_gemv_fused(uint16_t* out, const void* x, bitnet_dtype dt,
   p.out = out;
   p.sw = scale_wt;
   p.sw_len = static_cast<int>(scale_wt_len);
-  if (skq_ok(x, w_packed, M, K) && K / 128 <= sk::MAX_SPLIT * skq::MAX_KB) {
+  if (dt == BITNET_BF16 && skq_ok(x, w_packed, M, K) && K / 128 <= sk::MAX_SPLIT * skq::MAX_KB) {
     const bitnet_status r = run_gemv_skq(out, static_cast<const uint16_t*>(x), w_packed,
                                          scale_wt, scale_wt_len, M, N, K, as_stream(stream));
     if (r != BITNET_ERR_SHAPE) return r;
@@ -827,7 +848,7 @@ bitnet_status bitnet_gemv_fused(uint16_t* out, const void* x, bitnet_dtype dt,
 
 bitnet_status bitnet_gemv_fused_grouped(const bitnet_gemv_problem* problems, int64_t count,
                                         int64_t M, bitnet_dtype dt, void* stream) {
-  if (dt != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (dt != BITNET_BF16 && dt != BITNET_F32) return BITNET_ERR_DTYPE;
   if (count < 0) return BITNET_ERR_SHAPE;
   if (count == 0) return BITNET_OK;
   if (problems == nullptr) return BITNET_ERR_NULL;
@@ -849,7 +870,7 @@ bitnet_status bitnet_gemv_fused_grouped(const bitnet_gemv_problem* problems, int
   for (int64_t i = 0; i < count; ++i) {
     const bitnet_gemv_problem& q = problems[i];
     if (q.N == 0) continue;
-    if (q.K % 64 != 0) {  // rows not 16-byte aligned: its own launch
+    if (q.K % 64 != 0 || dt == BITNET_F32) {  // its own launch (the grouped kernel reads bf16)
       bitnet_status s = bitnet_gemv_fused(q.out, q.x, dt, q.w_packed, q.scale_wt,
                                           q.scale_wt_len, M, q.N, q.K, stream);
       if (s != BITNET_OK) return s;
@@ -895,7 +916,7 @@ bitnet_status bitnet_linear(uint16_t* out, const void* x, bitnet_dtype dt,
                             const uint8_t* w_packed, const float* scale_wt,
                             int64_t scale_wt_len, int64_t M, int64_t N, int64_t K,
                             void* workspace, size_t workspace_bytes, void* stream) {
-  if (dt != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (dt != BITNET_BF16 && dt != BITNET_F32) return BITNET_ERR_DTYPE;
   bitnet_status s = check_compute_shape(M, N, K);
   if (s != BITNET_OK) return s;
   if (M == 0 || N == 0) return BITNET_OK;
@@ -915,14 +936,16 @@ bitnet_status bitnet_linear(uint16_t* out, const void* x, bitnet_dtype dt,
                                                align256(static_cast<size_t>(M) * 2));
   cudaStream_t st = as_stream(stream);
   const uint16_t* xb = static_cast<const uint16_t*>(x);
+  const float* xf = static_cast<const float*>(x);
   if (gemm_tc_ok(xq, w_packed, K)) {
     // tensor-core path: transposed groups + row sums, weights as code planes
-    s = run_quantize_perm(xq, sa, rowsum, xb, M, K, st);
+    s = dt == BITNET_F32 ? run_quantize_perm_f32(xq, sa, rowsum, xf, M, K, st)
+                         : run_quantize_perm(xq, sa, rowsum, xb, M, K, st);
     if (s != BITNET_OK) return s;
     return run_gemm(out, false, xq, w_packed, sa, scale_wt, scale_wt_len, M, N, K, st, true,
                     rowsum);
   }
-  s = run_quantize(xq, sa, xb, M, K, st);
+  s = dt == BITNET_F32 ? run_quantize_f32(xq, sa, xf, M, K, st) : run_quantize(xq, sa, xb, M, K, st);
   if (s != BITNET_OK) return s;
   return run_gemm(out, false, xq, w_packed, sa, scale_wt, scale_wt_len, M, N, K, st);
 }
@@ -931,7 +954,7 @@ bitnet_status bitnet_linear_noalloc(uint16_t* out, const void* x, bitnet_dtype d
                                     const uint8_t* w_packed, const float* scale_wt,
                                     int64_t scale_wt_len, int64_t M, int64_t N, int64_t K,
                                     void* stream) {
-  if (dt != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (dt != BITNET_BF16 && dt != BITNET_F32) return BITNET_ERR_DTYPE;
   bitnet_status s = check_compute_shape(M, N, K);
   if (s != BITNET_OK) return s;
   if (M == 0 || N == 0) return BITNET_OK;

@@ -38,7 +38,7 @@ constexpr int kGemvRingTarget = 160 * 1024;  // bytes of stages per CTA (aim)
 struct GemvParams {
   uint16_t* out;          // bf16 [M, N], or
   int32_t* acc_out;       // int32 [M, N] (test hook)
-  const uint16_t* x;      // bf16 [M, K] (fused quantisation)
+  const void* x;          // [M, K] bf16, or float32 if x_f32 (fused quantisation)
   const int8_t* xq;       // int8 [M, K] (pre-quantised path)
   const uint16_t* sa_in;  // bf16 [M]    (pre-quantised path)
   const uint8_t* wp;      // uint8 [N, K/4]
@@ -51,6 +51,7 @@ struct GemvParams {
   uint32_t stage_bytes;   // shared bytes per stage (>= rows_per_block * K/4)
   int8_t* dbg_q;          // optional: codes quantised on chip (block 0)
   uint16_t* dbg_sa;       // optional: their scales (block 0)
+  int x_f32;              // x holds float32 values
 };
 
 // 4x4 byte transpose of a 16-byte group: out word i byte b = in word b byte i.
@@ -208,6 +209,22 @@ __device__ __forceinline__ void gemv_rows(int (&acc)[RW][MB][PLANES ? 4 : 1],
 // bf16-rounded scales as fp32 (saf). All CW consumer warps take part; the
 // caller synchronises the consumers (named barrier 1) afterwards. dbg_q /
 // dbg_sa, if not null, receive the natural-order codes and the scale bits.
+// Four consecutive activations of a row as fp32: bf16 rows are widened
+// exactly, float32 rows are read as they are.
+__device__ __forceinline__ float4 load_quad(const void* x, bool f32, int64_t row_off, int u) {
+  if (f32) return __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(x) + row_off) + u);
+  const uint2 v = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(x) + row_off) + u);
+  return make_float4(bf16_bits_to_f32(v.x & 0xFFFFu), bf16_bits_to_f32(v.x >> 16),
+                     bf16_bits_to_f32(v.y & 0xFFFFu), bf16_bits_to_f32(v.y >> 16));
+}
+
+// Largest magnitude of four fp32 values, as magnitude bits (the order of
+// the bits of non-negative floats is the order of their values).
+__device__ __forceinline__ uint32_t mag_max4(const float4& v) {
+  return max(max(__float_as_uint(v.x) & 0x7FFFFFFFu, __float_as_uint(v.y) & 0x7FFFFFFFu),
+             max(__float_as_uint(v.z) & 0x7FFFFFFFu, __float_as_uint(v.w) & 0x7FFFFFFFu));
+}
+
 struct GemvSmem {
   int* qsum;
   float* saf;
@@ -321,8 +338,9 @@ __device__ __forceinline__ void gemv_stage_cached(const GemvSmem& sh, const uint
 // CACHE: the single-problem kernel keeps one or two rows' quads in
 // registers between the passes (4 or 8 per thread, by K).
 template <int CW, int MB, bool QUAD = false, bool CACHE = false>
-__device__ __forceinline__ void gemv_stage_activations(const GemvSmem& sh, const uint16_t* __restrict__ x,
-                                                       int K, int Mc, int8_t* dbg_q, uint16_t* dbg_sa) {
+__device__ __forceinline__ void gemv_stage_activations(const GemvSmem& sh, const void* __restrict__ x,
+                                                       int K, int Mc, int8_t* dbg_q, uint16_t* dbg_sa,
+                                                       bool f32 = false) {
   constexpr int kGemvConsumerWarps = CW;
   constexpr int kGemvConsumers = CW * 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -334,36 +352,36 @@ __device__ __forceinline__ void gemv_stage_activations(const GemvSmem& sh, const
   uint8_t* qs = sh.qs;
   const int quads = K / 4;
   if constexpr (CACHE && MB <= 2) {
-    if (dbg_q == nullptr && quads <= 4 * kGemvConsumers) {
-      gemv_stage_cached<CW, MB, 4, QUAD>(sh, x, K, Mc, dbg_sa);
+    const uint16_t* xb = static_cast<const uint16_t*>(x);
+    if (!f32 && dbg_q == nullptr && quads <= 4 * kGemvConsumers) {
+      gemv_stage_cached<CW, MB, 4, QUAD>(sh, xb, K, Mc, dbg_sa);
       return;
     }
-    if (dbg_q == nullptr && quads <= 8 * kGemvConsumers) {
-      gemv_stage_cached<CW, MB, 8, QUAD>(sh, x, K, Mc, dbg_sa);
+    if (!f32 && dbg_q == nullptr && quads <= 8 * kGemvConsumers) {
+      gemv_stage_cached<CW, MB, 8, QUAD>(sh, xb, K, Mc, dbg_sa);
       return;
     }
   }
-    // absmax of every activation row; each thread owns the 4-element quads
-    // tid, tid + 512, ... of a row (loops kept rolled: a small code footprint)
+    // absmax of every activation row (as fp32 magnitude bits); each thread
+    // owns the 4-element quads tid, tid + 512, ... of a row (loops kept
+    // rolled: a small code footprint)
     uint32_t mb[MB];
 #pragma unroll
     for (int m = 0; m < MB; ++m) {
       mb[m] = 0;
       if (MB == 1 || m < Mc) {
-        const uint2* row = reinterpret_cast<const uint2*>(x + static_cast<int64_t>(m) * K);
+        const int64_t off = static_cast<int64_t>(m) * K;
         // four independent loads in flight per round
 #pragma unroll 1
         for (int u0 = tid; u0 < quads; u0 += 4 * kGemvConsumers) {
-          uint2 v[4];
+          float4 v[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int u = u0 + j * kGemvConsumers;
-            v[j] = u < quads ? __ldg(row + u) : make_uint2(0u, 0u);
+            v[j] = u < quads ? load_quad(x, f32, off, u) : make_float4(0.f, 0.f, 0.f, 0.f);
           }
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            mb[m] = max(mb[m], max(max(v[j].x & 0x7FFFu, (v[j].x >> 16) & 0x7FFFu),
-                                   max(v[j].y & 0x7FFFu, (v[j].y >> 16) & 0x7FFFu)));
+          for (int j = 0; j < 4; ++j) mb[m] = max(mb[m], mag_max4(v[j]));
         }
       }
       mb[m] = __reduce_max_sync(0xFFFFFFFFu, mb[m]);
@@ -373,7 +391,7 @@ __device__ __forceinline__ void gemv_stage_activations(const GemvSmem& sh, const
     if (tid < MB) {  // one thread per activation row: its quantiser and scale
       uint32_t t = 0;
       for (int w = 0; w < kGemvConsumerWarps; ++w) t = max(t, red[w * MB + tid]);
-      const RowQuant q = row_quant(bf16_bits_to_f32(t));
+      const RowQuant q = row_quant(__uint_as_float(t));
       rq_s[tid] = q.s;
       rq_r[tid] = q.r;
       const uint16_t sb = f32_to_bf16_bits(q.s);
@@ -390,15 +408,15 @@ __device__ __forceinline__ void gemv_stage_activations(const GemvSmem& sh, const
         RowQuant rqm;
         rqm.s = rq_s[m];
         rqm.r = rq_r[m];
-        const uint2* row = reinterpret_cast<const uint2*>(x + static_cast<int64_t>(m) * K);
+        const int64_t off = static_cast<int64_t>(m) * K;
         uint8_t* qrow = qs + m * K;
 #pragma unroll 1
         for (int u = tid; u < quads; u += kGemvConsumers) {
-          const uint2 v = __ldg(row + u);
-          const int q0 = quant_one(bf16_bits_to_f32(v.x & 0xFFFFu), rqm);
-          const int q1 = quant_one(bf16_bits_to_f32(v.x >> 16), rqm);
-          const int q2 = quant_one(bf16_bits_to_f32(v.y & 0xFFFFu), rqm);
-          const int q3 = quant_one(bf16_bits_to_f32(v.y >> 16), rqm);
+          const float4 v = load_quad(x, f32, off, u);
+          const int q0 = quant_one(v.x, rqm);
+          const int q1 = quant_one(v.y, rqm);
+          const int q2 = quant_one(v.z, rqm);
+          const int q3 = quant_one(v.w, rqm);
           qs_part[m] += q0 + q1 + q2 + q3;
           uint8_t* d = qrow + 16 * q_pos<QUAD>(u >> 2, (K / 16) & ~127) + (u & 3);
           d[0] = static_cast<uint8_t>(q0);
@@ -568,7 +586,7 @@ __global__ void __launch_bounds__((CW + 1) * 32) gemv_kernel(GemvParams p) {
     // L2 is the point of coherence, so a line fetched early is updated by any
     // later write; the loads that use the values come after the wait.
     const char* xb = reinterpret_cast<const char*>(p.x);
-    const int64_t xbytes = static_cast<int64_t>(Mc) * K * 2;
+    const int64_t xbytes = static_cast<int64_t>(Mc) * K * (p.x_f32 ? 4 : 2);
     for (int64_t off = static_cast<int64_t>(tid) * 128; off < xbytes; off += kGemvConsumers * 128)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(xb + off));
   }
@@ -577,7 +595,7 @@ __global__ void __launch_bounds__((CW + 1) * 32) gemv_kernel(GemvParams p) {
   if constexpr (!PREQ) {
     gemv_stage_activations<CW, MB, false, true>(GemvSmem{qsum, saf, rq_s, rq_r, red, qs}, p.x, K, Mc,
                                    blockIdx.x == 0 ? p.dbg_q : nullptr,
-                                   blockIdx.x == 0 ? p.dbg_sa : nullptr);
+                                   blockIdx.x == 0 ? p.dbg_sa : nullptr, p.x_f32 != 0);
   } else {
     int qs_part[MB];
 #pragma unroll

@@ -196,4 +196,94 @@ __global__ void __launch_bounds__(kQuantThreads)
   }
 }
 
+// ------------------------------------------------ float32 activations
+
+// Row absmax (as fp32 magnitude bits) and the row quantiser of one fp32 row,
+// over the CTA; two passes over global memory (K % 4 == 0, 16-byte rows).
+__device__ __forceinline__ RowQuant row_quant_f32(const float4* row, int nvec, uint32_t* red) {
+  const int tid = threadIdx.x;
+  uint32_t mb = 0;
+  for (int i = tid; i < nvec; i += kQuantThreads) {
+    const float4 v = __ldg(row + i);
+    mb = max(mb, max(max(__float_as_uint(v.x) & 0x7FFFFFFFu, __float_as_uint(v.y) & 0x7FFFFFFFu),
+                     max(__float_as_uint(v.z) & 0x7FFFFFFFu, __float_as_uint(v.w) & 0x7FFFFFFFu)));
+  }
+  mb = __reduce_max_sync(0xFFFFFFFFu, mb);
+  if ((tid & 31) == 0) red[tid >> 5] = mb;
+  __syncthreads();
+  if (tid < 32) {
+    uint32_t t = tid < kQuantThreads / 32 ? red[tid] : 0u;
+    t = __reduce_max_sync(0xFFFFFFFFu, t);
+    if (tid == 0) red[0] = t;
+  }
+  __syncthreads();
+  return row_quant(__uint_as_float(red[0]));
+}
+
+// Four fp32 values -> four int8 codes (natural order, one word).
+__device__ __forceinline__ uint32_t quant4_f32(const float4& v, const RowQuant& rq) {
+  return (static_cast<uint32_t>(quant_one(v.x, rq)) & 0xFFu) |
+         ((static_cast<uint32_t>(quant_one(v.y, rq)) & 0xFFu) << 8) |
+         ((static_cast<uint32_t>(quant_one(v.z, rq)) & 0xFFu) << 16) |
+         (static_cast<uint32_t>(quant_one(v.w, rq)) << 24);
+}
+
+// quantize_activation for float32 rows (natural layout), one CTA per row.
+__global__ void __launch_bounds__(kQuantThreads)
+    quantize_rows_f32_kernel(int8_t* __restrict__ xq, uint16_t* __restrict__ sa,
+                             const float* __restrict__ x, int K) {
+  __shared__ uint32_t red[kQuantThreads / 32];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int64_t m = blockIdx.x;
+  const float4* row = reinterpret_cast<const float4*>(x + m * K);
+  uint32_t* qrow = reinterpret_cast<uint32_t*>(xq + m * K);
+  const int nvec = K / 4;
+  const RowQuant rq = row_quant_f32(row, nvec, red);
+  for (int i = threadIdx.x; i < nvec; i += kQuantThreads) qrow[i] = quant4_f32(__ldg(row + i), rq);
+  if (threadIdx.x == 0) sa[m] = f32_to_bf16_bits(rq.s);
+}
+
+// The same with the layout of bitnet_linear's workspace (16-element groups
+// transposed 4x4) and the row's code sum, for float32 rows (K % 16 == 0).
+__global__ void __launch_bounds__(kQuantThreads)
+    quantize_rows_perm_f32_kernel(int8_t* __restrict__ xq, uint16_t* __restrict__ sa,
+                                  int32_t* __restrict__ rowsum, const float* __restrict__ x,
+                                  int K) {
+  __shared__ uint32_t red[kQuantThreads / 32];
+  __shared__ int reds[kQuantThreads / 32];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int64_t m = blockIdx.x;
+  const float4* row = reinterpret_cast<const float4*>(x + m * K);
+  uint4* qrow = reinterpret_cast<uint4*>(xq + m * K);
+  const int tid = threadIdx.x;
+  const RowQuant rq = row_quant_f32(row, K / 4, red);
+  int sum = 0;
+  for (int g = tid; g < K / 16; g += kQuantThreads) {
+    const uint32_t w0 = quant4_f32(__ldg(row + 4 * g), rq);
+    const uint32_t w1 = quant4_f32(__ldg(row + 4 * g + 1), rq);
+    const uint32_t w2 = quant4_f32(__ldg(row + 4 * g + 2), rq);
+    const uint32_t w3 = quant4_f32(__ldg(row + 4 * g + 3), rq);
+    sum += __dp4a(static_cast<int>(w0), 0x01010101, 0) + __dp4a(static_cast<int>(w1), 0x01010101, 0) +
+           __dp4a(static_cast<int>(w2), 0x01010101, 0) + __dp4a(static_cast<int>(w3), 0x01010101, 0);
+    // 4x4 byte transpose: out word i byte t = in word t byte i
+    const uint32_t t0 = __byte_perm(w0, w1, 0x5140u);
+    const uint32_t t1 = __byte_perm(w0, w1, 0x7362u);
+    const uint32_t t2 = __byte_perm(w2, w3, 0x5140u);
+    const uint32_t t3 = __byte_perm(w2, w3, 0x7362u);
+    qrow[g] = make_uint4(__byte_perm(t0, t2, 0x5410u), __byte_perm(t0, t2, 0x7632u),
+                         __byte_perm(t1, t3, 0x5410u), __byte_perm(t1, t3, 0x7632u));
+  }
+  sum = __reduce_add_sync(0xFFFFFFFFu, sum);
+  if ((tid & 31) == 0) reds[tid >> 5] = sum;
+  __syncthreads();
+  if (tid == 0) {
+    int t = 0;
+    for (int w = 0; w < kQuantThreads / 32; ++w) t += reds[w];
+    rowsum[m] = t;
+    sa[m] = f32_to_bf16_bits(rq.s);
+  }
+}
+
 }  // namespace bitnet

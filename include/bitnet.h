@@ -53,7 +53,9 @@ typedef enum {
 } bitnet_status;
 
 typedef enum {
-  BITNET_BF16 = 0 /* activations in bf16; other values are rejected */
+  BITNET_BF16 = 0, /* activations in bf16 */
+  BITNET_F32 = 1   /* activations in float32 (the bitnet-cpu page accepts
+                      both); other values are rejected */
 } bitnet_dtype;
 
 /* Pack ternary weights into 2-bit codes, four per byte.
@@ -76,7 +78,7 @@ bitnet_status bitnet_pack_weights(uint8_t* w_packed, const int8_t* w,
  * fp32 before any arithmetic.
  *   x_q        out, int8 [M, K]
  *   scale_act  out, bf16 [M]
- *   x          in,  [M, K] of dtype `dt` (only BITNET_BF16) */
+ *   x          in,  [M, K] of dtype `dt` (BITNET_BF16 or BITNET_F32) */
 bitnet_status bitnet_quantize_act(int8_t* x_q, uint16_t* scale_act,
                                   const void* x, bitnet_dtype dt, int64_t M,
                                   int64_t K, void* stream);
@@ -103,7 +105,7 @@ bitnet_status bitnet_gemm(uint16_t* out, const int8_t* x_q,
  * bitnet-cpu page; the fused dp4a GEMV of the bitnet-tc announcement).
  * Same result, bit for bit, as bitnet_quantize_act followed by bitnet_gemm.
  *   out       out, bf16 [M, N]
- *   x         in,  [M, K] of dtype `dt` (only BITNET_BF16)
+ *   x         in,  [M, K] of dtype `dt` (BITNET_BF16 or BITNET_F32)
  *   w_packed, scale_wt, scale_wt_len as for bitnet_gemm.
  * Needs 1 <= M <= 15 (the page dispatches M < 16 here), and the quantised
  * rows plus one stage of sixteen weight rows must fit on chip:
@@ -112,7 +114,7 @@ bitnet_status bitnet_gemm(uint16_t* out, const int8_t* x_q,
  * Kernels: with 8 <= M, K % 64 == 0, 16-byte aligned x and w_packed and
  * K <= 128 * 8 * min(48, floor(384 / M)), a tensor-core kernel with the
  * quantisation inside (its K loop split over a thread-block cluster);
- * otherwise a dp4a GEMV. Both give the same result. */
+ * otherwise a dp4a GEMV (always for BITNET_F32). Both give the same result. */
 bitnet_status bitnet_gemv_fused(uint16_t* out, const void* x, bitnet_dtype dt,
                                 const uint8_t* w_packed, const float* scale_wt,
                                 int64_t scale_wt_len, int64_t M, int64_t N,
@@ -140,8 +142,9 @@ typedef struct {
  *   problems  in, HOST array of `count` problem descriptors (read during
  *             the call, not kept)
  * Each problem obeys bitnet_gemv_fused's rules. Problems whose K is not a
- * multiple of 64 are computed by their own bitnet_gemv_fused launch. The
- * whole call is validated before anything is enqueued. */
+ * multiple of 64, and every problem of a BITNET_F32 call, are computed by
+ * their own bitnet_gemv_fused launch. The whole call is validated before
+ * anything is enqueued. */
 bitnet_status bitnet_gemv_fused_grouped(const bitnet_gemv_problem* problems,
                                         int64_t count, int64_t M,
                                         bitnet_dtype dt, void* stream);

@@ -64,7 +64,12 @@ ODD = P(0x10008)
     (lambda L: L.bitnet_gemm(FAKE, FAKE, ODD, FAKE, FAKE, 1, 4, 4, 64, None), bn.ERR_ALIGN),
     (lambda L: L.bitnet_gemv_fused(FAKE, FAKE, 0, FAKE, FAKE, 1, 16, 4, 64, None), bn.ERR_SHAPE),
     (lambda L: L.bitnet_gemv_fused(FAKE, FAKE, 0, FAKE, FAKE, 1, 0, 4, 64, None), bn.ERR_SHAPE),
-    (lambda L: L.bitnet_gemv_fused(FAKE, FAKE, 1, FAKE, FAKE, 1, 1, 4, 64, None), bn.ERR_DTYPE),
+    (lambda L: L.bitnet_gemv_fused(FAKE, FAKE, 2, FAKE, FAKE, 1, 1, 4, 64, None), bn.ERR_DTYPE),
+    # float32 activations (dtype 1) are validated like bf16 ones
+    (lambda L: L.bitnet_gemv_fused(FAKE, ODD, 1, FAKE, FAKE, 1, 1, 4, 64, None), bn.ERR_ALIGN),
+    (lambda L: L.bitnet_quantize_act(FAKE, FAKE, FAKE, 1, 2, 40, None), bn.ERR_SHAPE),
+    (lambda L: L.bitnet_linear(FAKE, FAKE, 1, FAKE, FAKE, 1, 32, 4, 64, None, 0, None),
+     bn.ERR_WORKSPACE),
     (lambda L: L.bitnet_gemv_fused(FAKE, ODD, 0, FAKE, FAKE, 1, 1, 4, 64, None), bn.ERR_ALIGN),
     (lambda L: L.bitnet_gemv_fused(FAKE, FAKE, 0, FAKE, FAKE, 1, 15, 4, 16384, None), bn.ERR_SHAPE),
     (lambda L: L.bitnet_quantize_act(FAKE, FAKE, FAKE, 0, 2, 40, None), bn.ERR_SHAPE),

@@ -330,3 +330,39 @@ def test_gemv_fused_grouped_more_than_one_launch():
     outs = bn.bitnet_gemv_fused_grouped(xs, wps, sws)
     for o, r in zip(outs, refs):
         assert_bf16_close(bf16_bits(o), r)
+
+
+# ---------------------------------------------------------- float32 input
+
+F32_CASES = [(1, 512, 512), (4, 2560, 640), (15, 4096, 300), (9, 1024, 131), (3, 96, 40),
+             (16, 1024, 384), (64, 2560, 520), (300, 4096, 256), (37, 160, 77)]
+
+
+def acts_f32(layer, M, K):
+    rng = np.random.default_rng(layer * 7919 + M * 31 + K)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[:, ::101] *= 20.0
+    if M > 1:
+        x[1, :6] = np.array([127.0, 0.5, 1.5, -2.5, 3.5, -0.5], np.float32)  # exact ties
+    return x
+
+
+@pytest.mark.parametrize("M,K,N", F32_CASES)
+def test_float32_activations_match_oracle(M, K, N):
+    """float32 activations (the dtype the bitnet-cpu page accepts besides
+    bf16) through the quantiser, the fused GEMV and bitnet_linear."""
+    x = acts_f32(M, M, K)
+    w = weights(93, M + K, N, K)
+    p = oracle.pack(w)
+    sw = sw_of(93, M)
+    xd = to_dev(x)
+    q_ref, s_ref = oracle.quantize_f32(x)
+    xq, sa = bn.bitnet_quantize_act(xd)
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+    assert np.array_equal(bf16_bits(sa), s_ref)
+    ref = oracle.linear_f32(x, p, sw)
+    pd = to_dev(p)
+    assert_bf16_close(bf16_bits(bn.bitnet_linear(xd, pd, to_dev(sw))), ref)
+    assert_bf16_close(bf16_bits(bn.bitnet_linear_noalloc(xd, pd, to_dev(sw))), ref)
+    if M < 16:
+        assert_bf16_close(bf16_bits(bn.bitnet_gemv_fused(xd, pd, to_dev(sw))), ref)
