@@ -110,7 +110,7 @@ def test_grouped_validation_before_launch():
     assert L.bitnet_gemv_fused_grouped(None, 2, 1, 0, None) == bn.ERR_NULL
     assert L.bitnet_gemv_fused_grouped(p, -1, 1, 0, None) == bn.ERR_SHAPE
     assert L.bitnet_gemv_fused_grouped(p, 2, 16, 0, None) == bn.ERR_SHAPE
-    assert L.bitnet_gemv_fused_grouped(p, 2, 1, 1, None) == bn.ERR_DTYPE
+    assert L.bitnet_gemv_fused_grouped(p, 2, 1, 2, None) == bn.ERR_DTYPE
     arr[1] = bn.GemvProblem(0x10000, 0x10000, 0x10000, 0x10000, 1, 64, 48)   # K % 32
     assert L.bitnet_gemv_fused_grouped(p, 2, 1, 0, None) == bn.ERR_SHAPE
     arr[1] = bn.GemvProblem(0x10008, 0x10000, 0x10000, 0x10000, 1, 64, 128)  # out align
