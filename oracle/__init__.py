@@ -31,6 +31,7 @@ def lib():
         L.oracle_unpack.argtypes = [_P, _I64, _I64, _P]
         L.oracle_quantize.argtypes = [_P, _I64, _I64, _P, _P]
         L.oracle_quantize_f32.argtypes = [_P, _I64, _I64, _P, _P]
+        L.oracle_ternarize_absmean.argtypes = [_P, _I64, _I64, ctypes.c_int, _P, _P]
         L.oracle_linear_f32.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P]
         L.oracle_acc.argtypes = [_P, _P, _I64, _I64, _I64, _P]
         L.oracle_epilogue.argtypes = [_P, _P, _P, _I64, _I64, _I64, _P]
@@ -45,6 +46,7 @@ def lib():
         L.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
         L.oracle_f32_to_bf16.restype = ctypes.c_uint16
         for name in ("oracle_pack", "oracle_unpack", "oracle_quantize", "oracle_quantize_f32",
+                     "oracle_ternarize_absmean",
                      "oracle_linear_f32",
                      "oracle_acc", "oracle_epilogue", "oracle_gemm",
                      "oracle_linear", "oracle_linear_threads",
@@ -120,6 +122,17 @@ def linear_f32(x, packed, scale_wt):
     _check(lib().oracle_linear_f32(_ptr(x), _ptr(packed), _ptr(sw), sw.size, M, N, K,
                                    _ptr(out)), "linear_f32")
     return out
+
+
+def ternarize_absmean(w, per_row=True):
+    """float32 [N, K] -> (int8 ternary [N, K], float32 scale [N] or [1])."""
+    w = _c(w, np.float32)
+    N, K = w.shape
+    wt = np.empty((N, K), np.int8)
+    sc = np.empty((N if per_row else 1,), np.float32)
+    _check(lib().oracle_ternarize_absmean(_ptr(w), N, K, 1 if per_row else 0, _ptr(wt), _ptr(sc)),
+           "ternarize_absmean")
+    return wt, sc
 
 
 def acc(q, packed, N=None):

@@ -332,4 +332,85 @@ int oracle_linear_threads_cols(const uint16_t* x, const uint8_t* packed,
 // library conversion on its own.
 uint16_t oracle_f32_to_bf16(float f) { return float_to_bf16_bits_rne(f); }
 
+// ------------------------------------------------------------------------
+// Absmean ternarisation (bitnet-cpu page: BitLinear.from_dense per output
+// row, gamma clamped at 1e-8; BitLinearKernel per tensor, clamped at 1e-5):
+//   gamma = max(mean |w|, eps), code = clamp(round-half-even(w / gamma), -1, 1),
+//   scale = bf16(gamma).
+// Reading of the mean (the page computes it with a float32 reduction, whose
+// result depends on the summation order): the sum of |w| is exact, as an
+// integer in units of 2^-64 (|w| * 2^64 truncated toward zero: exact for
+// |w| >= 2^-40, and |w| < 2^47 is required), then
+// mean = float(double(sum) / count * 2^-64) with each operation rounded to
+// nearest even. Integer addition does not depend on the order.
+
+typedef unsigned __int128 u128;
+
+static bool abs_fixed(float w, u128* out) {
+  if (!std::isfinite(w)) return false;
+  const float a = std::fabs(w);
+  if (a >= 140737488355328.0f) return false;  // 2^47
+  if (a == 0.0f) {
+    *out = 0;
+    return true;
+  }
+  int e = 0;
+  const float fr = std::frexp(a, &e);  // a = fr * 2^e, fr in [0.5, 1)
+  const uint64_t m = static_cast<uint64_t>(std::ldexp(fr, 24));  // 24-bit integer
+  const int sh = e - 24 + 64;  // a * 2^64 = m * 2^sh
+  if (sh >= 0) *out = static_cast<u128>(m) << sh;
+  else if (sh > -64) *out = static_cast<u128>(m >> (-sh));
+  else *out = 0;
+  return true;
+}
+
+static float mean_of(u128 sum, int64_t count) {
+  const double d = static_cast<double>(sum) / static_cast<double>(count);
+  return static_cast<float>(std::ldexp(d, -64));
+}
+
+static void ternarize_row(const float* w, int64_t K, float gamma, int8_t* wt) {
+  for (int64_t k = 0; k < K; ++k) {
+    float r = std::nearbyint(w[k] / gamma);  // half-to-even under FE_TONEAREST
+    if (r < -1.0f) r = -1.0f;
+    if (r > 1.0f) r = 1.0f;
+    wt[k] = static_cast<int8_t>(r);
+  }
+}
+
+// per_row != 0: scale [N]; per_row == 0: one gamma for the tensor, scale [1].
+// scale holds bf16(gamma) widened to fp32. ERR_VALUE for non-finite or huge
+// weights.
+int oracle_ternarize_absmean(const float* w, int64_t N, int64_t K, int per_row, int8_t* wt,
+                             float* scale) {
+  if (N < 0 || K <= 0) return ERR_SHAPE;
+  std::fesetround(FE_TONEAREST);
+  if (per_row) {
+    for (int64_t n = 0; n < N; ++n) {
+      u128 s = 0;
+      for (int64_t k = 0; k < K; ++k) {
+        u128 a;
+        if (!abs_fixed(w[n * K + k], &a)) return ERR_VALUE;
+        s += a;
+      }
+      float gamma = mean_of(s, K);
+      if (gamma < 1e-8f) gamma = 1e-8f;
+      ternarize_row(w + n * K, K, gamma, wt + n * K);
+      scale[n] = bf16_bits_to_float(float_to_bf16_bits_rne(gamma));
+    }
+    return OK;
+  }
+  u128 s = 0;
+  for (int64_t i = 0; i < N * K; ++i) {
+    u128 a;
+    if (!abs_fixed(w[i], &a)) return ERR_VALUE;
+    s += a;
+  }
+  float gamma = N > 0 ? mean_of(s, N * K) : 1e-5f;
+  if (gamma < 1e-5f) gamma = 1e-5f;
+  for (int64_t n = 0; n < N; ++n) ternarize_row(w + n * K, K, gamma, wt + n * K);
+  scale[0] = bf16_bits_to_float(float_to_bf16_bits_rne(gamma));
+  return OK;
+}
+
 }  // extern "C"

@@ -332,3 +332,57 @@ def test_linear_close_to_float64_dequantised_product():
     y = bf16_to_f32(oracle.linear(x, p, sw)).astype(np.float64)
     ref = (q.astype(np.float64) @ w.astype(np.float64).T) * bf16_to_f32(sa)[:, None] * 0.05
     assert np.allclose(y, ref, rtol=2 ** -7, atol=1e-6)
+
+
+# --------------------------------------------------- absmean ternarisation
+
+def test_ternarize_golden_example():
+    """Worked by hand from BitLinear.from_dense on the bitnet-cpu page:
+    mean|w| = 4.1 / 4 = 1.025; w / gamma = 0.49, -1.46, 0.098, 1.95."""
+    w = np.array([[0.5, -1.5, 0.1, 2.0], [0.0, 0.0, 0.0, 0.0]], np.float32)
+    wt, sc = oracle.ternarize_absmean(w)
+    assert wt.tolist() == [[0, -1, 0, 1], [0, 0, 0, 0]]
+    assert sc[0] == np.float32(1.0234375)                        # bf16(1.025)
+    bits = f32_to_bf16_bits_np(np.float32(1e-8))                 # zero row: gamma = eps
+    assert sc[1] == (np.uint32(bits) << 16).view(np.float32)
+    wt, sc = oracle.ternarize_absmean(w, per_row=False)          # mean over 8 = 0.5125
+    assert wt.tolist() == [[1, -1, 0, 1], [0, 0, 0, 0]]          # 0.5 / 0.5125 = 0.976 -> 1
+    assert sc[0] == np.float32(0.51171875)                       # bf16(0.5125)
+
+
+def test_ternarize_recovers_scaled_ternary_matrices():
+    """w = gamma_n * t with t ternary: mean|w| = gamma_n * nnz / K <= gamma_n,
+    so w / mean is 0 or at least 1 in magnitude and the codes are t."""
+    rng = np.random.default_rng(3)
+    t = rng.choice(np.array([-1, 0, 1], np.int8), size=(64, 320), p=[0.3, 0.4, 0.3])
+    t[:, 0] = 1
+    g = rng.uniform(0.01, 0.5, size=(64, 1)).astype(np.float32)
+    wt, _ = oracle.ternarize_absmean(t.astype(np.float32) * g)
+    assert np.array_equal(wt, t)
+    wt, _ = oracle.ternarize_absmean(t.astype(np.float32) * np.float32(0.07), per_row=False)
+    assert np.array_equal(wt, t)
+
+
+def test_ternarize_matches_float64_definition():
+    """Library special case: for ordinary weights the float64 sum of |w| is
+    exact, so gamma = max(float32(sum / K), eps) and the codes follow with a
+    float32 division and round-half-even."""
+    rng = np.random.default_rng(9)
+    w = (rng.standard_normal((96, 2560)) * 0.02).astype(np.float32)
+    w[0, :4] = [0.0, 0.0, 0.0, 0.0]
+    for per_row, eps in ((True, 1e-8), (False, 1e-5)):
+        wt, sc = oracle.ternarize_absmean(w, per_row=per_row)
+        a = np.abs(w).astype(np.float64)
+        mean = a.sum(axis=1) / w.shape[1] if per_row else np.array([a.sum() / w.size])
+        gamma = np.maximum(mean.astype(np.float32), np.float32(eps))
+        gb = (f32_to_bf16_bits_np(gamma).astype(np.uint32) << 16).view(np.float32)
+        assert np.array_equal(sc, gb)
+        ref = np.clip(np.rint(w / gamma.reshape(-1, 1)), -1, 1).astype(np.int8)
+        assert np.array_equal(wt, ref)
+
+
+def test_ternarize_rejects_non_finite():
+    w = np.zeros((2, 8), np.float32)
+    w[1, 3] = np.inf
+    with pytest.raises(Exception):
+        oracle.ternarize_absmean(w)
