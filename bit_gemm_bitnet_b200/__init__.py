@@ -26,7 +26,7 @@ F32 = 1
 
 # every symbol include/bitnet.h declares
 EXPORTS = (
-    "bitnet_pack_weights", "bitnet_quantize_act", "bitnet_gemm",
+    "bitnet_ternarize_absmean", "bitnet_pack_weights", "bitnet_quantize_act", "bitnet_gemm",
     "bitnet_gemv_fused", "bitnet_linear_workspace_bytes", "bitnet_linear",
     "bitnet_device_status", "bitnet_status_string", "bitnet_gemm_acc_i32",
     "bitnet_gemv_fused_debug", "bitnet_linear_noalloc", "bitnet_gemv_fused_grouped",
@@ -65,6 +65,7 @@ def lib():
         P, I64, SZ, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
         sig = {
             "bitnet_pack_weights": [P, P, I64, I64, P],
+            "bitnet_ternarize_absmean": [P, P, P, I64, I64, I, P],
             "bitnet_quantize_act": [P, P, P, I, I64, I64, P],
             "bitnet_gemm": [P, P, P, P, P, I64, I64, I64, I64, P],
             "bitnet_gemv_fused": [P, P, I, P, P, I64, I64, I64, I64, P],
@@ -153,6 +154,22 @@ def bitnet_pack_weights(w, out=None):
     _check(lib().bitnet_pack_weights(_ptr(out), _ptr(w), N, K, _stream(w.device)),
            "bitnet_pack_weights")
     return out
+
+
+def bitnet_ternarize_absmean(w, per_row=True, w_t=None, scale_wt=None):
+    """float32 [N, K] weights -> (int8 ternary [N, K], float32 scale [N] or
+    [1]): absmean ternarisation (BitLinear.from_dense per row; BitLinearKernel
+    per tensor), ready for bitnet_pack_weights."""
+    _need(w, torch.float32, "w", 2)
+    N, K = w.shape
+    if w_t is None:
+        w_t = torch.empty((N, K), dtype=torch.int8, device=w.device)
+    if scale_wt is None:
+        scale_wt = torch.empty((N if per_row else 1,), dtype=torch.float32, device=w.device)
+    _check(lib().bitnet_ternarize_absmean(_ptr(w_t), _ptr(scale_wt), _ptr(w), N, K,
+                                          1 if per_row else 0, _stream(w.device)),
+           "bitnet_ternarize_absmean")
+    return w_t, scale_wt
 
 
 def bitnet_quantize_act(x, x_q=None, scale_act=None):

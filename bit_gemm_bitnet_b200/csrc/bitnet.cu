@@ -11,6 +11,7 @@
 #include "gemm_sk.cuh"
 #include "gemm_skq.cuh"
 #include "gemm_ts.cuh"
+#include "ternarize.cuh"
 #include "gemv.cuh"
 #include "gemv_grouped.cuh"
 #include "pack_quant.cuh"
@@ -760,6 +761,37 @@ bitnet_status bitnet_pack_weights(uint8_t* w_packed, const int8_t* w, int64_t N,
   unsigned bad = 0;
   if (cudaMemcpyFromSymbolAsync(&bad, g_pack_bad_value, sizeof bad, 0,
                                 cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return BITNET_ERR_CUDA;
+  return bad ? BITNET_ERR_VALUE : BITNET_OK;
+}
+
+bitnet_status bitnet_ternarize_absmean(int8_t* w_t, float* scale_wt, const float* w, int64_t N,
+                                       int64_t K, int per_row, void* stream) {
+  if (N < 0 || K <= 0 || K > INT32_MAX || K % (per_row ? 4 : 16) != 0 || N > INT32_MAX)
+    return BITNET_ERR_SHAPE;
+  if (N == 0) return BITNET_OK;
+  if (w_t == nullptr || scale_wt == nullptr || w == nullptr) return BITNET_ERR_NULL;
+  if (!aligned(w, 16) || !aligned(w_t, 16) || !aligned(scale_wt, 4)) return BITNET_ERR_ALIGN;
+  cudaStream_t st = as_stream(stream);
+  const unsigned zero = 0;
+  if (cudaMemcpyToSymbolAsync(g_ternarize_bad, &zero, sizeof zero, 0, cudaMemcpyHostToDevice,
+                              st) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  const dim3 rows(static_cast<unsigned>(N)), block(kTernThreads);
+  const int k = static_cast<int>(K);
+  if (per_row) {
+    ternarize_rows_kernel<<<rows, block, 0, st>>>(w_t, scale_wt, w, k);
+  } else {
+    ternarize_rowsum_kernel<<<rows, block, 0, st>>>(w_t, w, k);
+    ternarize_total_kernel<<<1, block, 0, st>>>(scale_wt, w_t, N, k);
+    ternarize_apply_kernel<<<rows, block, 0, st>>>(w_t, scale_wt, w, k);
+    ternarize_round_scale_kernel<<<1, 32, 0, st>>>(scale_wt);
+  }
+  if (cudaGetLastError() != cudaSuccess) return BITNET_ERR_CUDA;
+  unsigned bad = 0;
+  if (cudaMemcpyFromSymbolAsync(&bad, g_ternarize_bad, sizeof bad, 0, cudaMemcpyDeviceToHost,
+                                st) != cudaSuccess)
     return BITNET_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return BITNET_ERR_CUDA;
   return bad ? BITNET_ERR_VALUE : BITNET_OK;

@@ -1,0 +1,173 @@
+// Absmean ternarisation of float32 weights (the load-time step before
+// packing): BitLinear.from_dense on the bitnet-cpu page (one gamma per output
+// row, clamped at 1e-8) and BitLinearKernel (one gamma for the tensor,
+// clamped at 1e-5):
+//   gamma = max(mean |w|, eps), code = clamp(round-half-even(w / gamma), -1, 1),
+//   scale = bf16(gamma).
+// The mean's sum is exact: |w| * 2^64 truncated toward zero is an integer
+// (exact for |w| >= 2^-40; |w| < 2^47 is required), summed in 128 bits, so
+// the result does not depend on the order of the additions. Then
+// mean = float(double(sum) / count * 2^-64), each operation rounded to
+// nearest even.
+#pragma once
+#include "common.cuh"
+
+namespace bitnet {
+
+typedef unsigned __int128 u128;
+
+__device__ unsigned g_ternarize_bad;  // set when a weight is non-finite or >= 2^47
+
+// |w| * 2^64, truncated toward zero; false for non-finite or |w| >= 2^47.
+__device__ __forceinline__ bool abs_fixed(float w, u128* out) {
+  const uint32_t bits = __float_as_uint(w) & 0x7FFFFFFFu;
+  *out = 0;
+  if (bits >= 0x57000000u) return false;  // 2^47 and above, Inf, NaN
+  const int e = static_cast<int>(bits >> 23);
+  if (e == 0) {  // zero and subnormals: below 2^-126, nothing above 2^-64
+    *out = 0;
+    return true;
+  }
+  const uint64_t m = (bits & 0x7FFFFFu) | 0x800000u;  // |w| = m * 2^(e - 150)
+  const int sh = e - 86;                                // |w| * 2^64 = m * 2^sh
+  if (sh >= 0) *out = static_cast<u128>(m) << sh;
+  else if (sh > -64) *out = static_cast<u128>(m >> (-sh));
+  else *out = 0;
+  return true;
+}
+
+// The 128-bit integer rounded to the nearest double, halves to even.
+__device__ __forceinline__ double u128_to_double_rn(u128 v) {
+  const uint64_t hi = static_cast<uint64_t>(v >> 64), lo = static_cast<uint64_t>(v);
+  if (hi == 0) return __ull2double_rn(lo);
+  const int top = 127 - __clzll(static_cast<long long>(hi));  // highest set bit
+  const int drop = top - 52;                                   // bits below the 53 kept
+  const u128 kept = v >> drop;
+  const u128 rest = v - (kept << drop);
+  const u128 half = static_cast<u128>(1) << (drop - 1);
+  uint64_t mant = static_cast<uint64_t>(kept);
+  if (rest > half || (rest == half && (mant & 1u))) ++mant;  // may carry to 2^53: still exact
+  return ldexp(static_cast<double>(mant), drop);
+}
+
+__device__ __forceinline__ float mean_of(u128 sum, double count) {
+  return static_cast<float>(ldexp(__ddiv_rn(u128_to_double_rn(sum), count), -64));
+}
+
+// Sum of the |w| of the CTA's items, exact; the per-thread partial sums are
+// combined by thread 0 in a fixed order. `part` holds 2 words per thread.
+__device__ __forceinline__ u128 cta_sum(u128 mine, uint64_t* part) {
+  const int tid = threadIdx.x;
+  part[2 * tid] = static_cast<uint64_t>(mine);
+  part[2 * tid + 1] = static_cast<uint64_t>(mine >> 64);
+  __syncthreads();
+  u128 total = 0;
+  if (tid == 0)
+    for (int t = 0; t < static_cast<int>(blockDim.x); ++t)
+      total += (static_cast<u128>(part[2 * t + 1]) << 64) | part[2 * t];
+  return total;  // valid in thread 0
+}
+
+constexpr int kTernThreads = 256;
+
+// Four codes of w[0..3] / gamma, packed little-endian.
+__device__ __forceinline__ uint32_t ternary4(const float4& v, float gamma) {
+  auto one = [&](float x) {
+    int r = __float2int_rn(__fdiv_rn(x, gamma));
+    r = r < -1 ? -1 : (r > 1 ? 1 : r);
+    return static_cast<uint32_t>(r) & 0xFFu;
+  };
+  return one(v.x) | (one(v.y) << 8) | (one(v.z) << 16) | (one(v.w) << 24);
+}
+
+__device__ __forceinline__ u128 row_abs_sum(const float4* row, int nvec, bool* ok) {
+  u128 s = 0;
+  for (int i = threadIdx.x; i < nvec; i += kTernThreads) {
+    const float4 v = __ldg(row + i);
+    u128 a = 0;
+    *ok &= abs_fixed(v.x, &a);
+    s += a;
+    *ok &= abs_fixed(v.y, &a);
+    s += a;
+    *ok &= abs_fixed(v.z, &a);
+    s += a;
+    *ok &= abs_fixed(v.w, &a);
+    s += a;
+  }
+  return s;
+}
+
+// One gamma per output row: one CTA per row (K % 4 == 0).
+__global__ void __launch_bounds__(kTernThreads)
+    ternarize_rows_kernel(int8_t* __restrict__ wt, float* __restrict__ scale,
+                          const float* __restrict__ w, int K) {
+  __shared__ uint64_t part[2 * kTernThreads];
+  __shared__ float gamma_s;
+  const int64_t n = blockIdx.x;
+  const float4* row = reinterpret_cast<const float4*>(w + n * K);
+  const int nvec = K / 4;
+  bool ok = true;
+  const u128 total = cta_sum(row_abs_sum(row, nvec, &ok), part);
+  if (!ok) atomicOr(&g_ternarize_bad, 1u);
+  if (threadIdx.x == 0) {
+    float g = mean_of(total, static_cast<double>(K));
+    gamma_s = g < 1e-8f ? 1e-8f : g;
+  }
+  __syncthreads();
+  const float gamma = gamma_s;
+  uint32_t* out = reinterpret_cast<uint32_t*>(wt + n * K);
+  for (int i = threadIdx.x; i < nvec; i += kTernThreads) out[i] = ternary4(__ldg(row + i), gamma);
+  if (threadIdx.x == 0) scale[n] = bf16_bits_to_f32(f32_to_bf16_bits(gamma));
+}
+
+// One gamma for the tensor, step 1: each row's exact sum, kept in the first
+// 16 bytes of the row's output (K % 16 == 0).
+__global__ void __launch_bounds__(kTernThreads)
+    ternarize_rowsum_kernel(int8_t* __restrict__ wt, const float* __restrict__ w, int K) {
+  __shared__ uint64_t part[2 * kTernThreads];
+  const int64_t n = blockIdx.x;
+  bool ok = true;
+  const u128 total = cta_sum(row_abs_sum(reinterpret_cast<const float4*>(w + n * K), K / 4, &ok),
+                             part);
+  if (!ok) atomicOr(&g_ternarize_bad, 1u);
+  if (threadIdx.x == 0) {
+    uint64_t* dst = reinterpret_cast<uint64_t*>(wt + n * K);
+    dst[0] = static_cast<uint64_t>(total);
+    dst[1] = static_cast<uint64_t>(total >> 64);
+  }
+}
+
+// Step 2 (one CTA): the tensor's sum, gamma (fp32) into scale[0].
+__global__ void __launch_bounds__(kTernThreads)
+    ternarize_total_kernel(float* __restrict__ scale, const int8_t* __restrict__ wt, int64_t N,
+                           int K) {
+  __shared__ uint64_t part[2 * kTernThreads];
+  u128 s = 0;
+  for (int64_t n = threadIdx.x; n < N; n += kTernThreads) {
+    const uint64_t* src = reinterpret_cast<const uint64_t*>(wt + n * K);
+    s += (static_cast<u128>(src[1]) << 64) | src[0];
+  }
+  const u128 total = cta_sum(s, part);
+  if (threadIdx.x == 0) {
+    const float g = mean_of(total, static_cast<double>(N) * static_cast<double>(K));
+    scale[0] = g < 1e-5f ? 1e-5f : g;
+  }
+}
+
+// Step 3: the codes, with gamma from scale[0]; one CTA per row.
+__global__ void __launch_bounds__(kTernThreads)
+    ternarize_apply_kernel(int8_t* __restrict__ wt, const float* __restrict__ scale,
+                           const float* __restrict__ w, int K) {
+  const int64_t n = blockIdx.x;
+  const float gamma = scale[0];
+  const float4* row = reinterpret_cast<const float4*>(w + n * K);
+  uint32_t* out = reinterpret_cast<uint32_t*>(wt + n * K);
+  for (int i = threadIdx.x; i < K / 4; i += kTernThreads) out[i] = ternary4(__ldg(row + i), gamma);
+}
+
+// Step 4: scale[0] = bf16(gamma), once every row has its codes.
+__global__ void ternarize_round_scale_kernel(float* scale) {
+  if (threadIdx.x == 0) scale[0] = bf16_bits_to_f32(f32_to_bf16_bits(scale[0]));
+}
+
+}  // namespace bitnet

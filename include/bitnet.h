@@ -70,6 +70,24 @@ typedef enum {
 bitnet_status bitnet_pack_weights(uint8_t* w_packed, const int8_t* w,
                                   int64_t N, int64_t K, void* stream);
 
+/* Absmean ternarisation of float32 weights, the step before packing:
+ * BitLinear.from_dense on the bitnet-cpu page (per_row != 0: one gamma per
+ * output row, clamped at 1e-8) or BitLinearKernel (per_row == 0: one gamma
+ * for the tensor, clamped at 1e-5):
+ *   gamma = max(mean |w|, eps), w_t = clamp(round-half-even(w / gamma), -1, 1),
+ *   scale_wt = bf16(gamma), returned widened to fp32.
+ * The mean's sum is exact (|w| * 2^64 truncated toward zero, summed as an
+ * integer), then mean = float(double(sum) / count * 2^-64): the result does
+ * not depend on any summation order.
+ *   w_t       out, int8 [N, K] ternary (then bitnet_pack_weights)
+ *   scale_wt  out, fp32 [N] (per_row) or [1]
+ *   w         in,  fp32 [N, K], finite, |w| < 2^47
+ * K % 4 == 0 (per row) or K % 16 == 0 (per tensor; the row sums pass through
+ * w_t). Synchronises the stream to report BITNET_ERR_VALUE for a weight that
+ * is not finite or too large. */
+bitnet_status bitnet_ternarize_absmean(int8_t* w_t, float* scale_wt, const float* w,
+                                       int64_t N, int64_t K, int per_row, void* stream);
+
 /* Per-token absmax INT8 activation quantisation.
  * Defined by quantize_activation() on the bitnet-cpu page: for each row m,
  * absmax = max_k |x[m,k]| clamped below at 1e-5, s = absmax / 127 (fp32,

@@ -76,6 +76,10 @@ ODD = P(0x10008)
     (lambda L: L.bitnet_quantize_act(FAKE, FAKE, None, 0, 2, 64, None), bn.ERR_NULL),
     (lambda L: L.bitnet_quantize_act(FAKE, FAKE, FAKE, 2, 2, 64, None), bn.ERR_DTYPE),
     (lambda L: L.bitnet_pack_weights(FAKE, FAKE, 4, 6, None), bn.ERR_SHAPE),
+    (lambda L: L.bitnet_ternarize_absmean(FAKE, FAKE, FAKE, 4, 6, 1, None), bn.ERR_SHAPE),
+    (lambda L: L.bitnet_ternarize_absmean(FAKE, FAKE, FAKE, 4, 8, 0, None), bn.ERR_SHAPE),
+    (lambda L: L.bitnet_ternarize_absmean(None, FAKE, FAKE, 4, 16, 1, None), bn.ERR_NULL),
+    (lambda L: L.bitnet_ternarize_absmean(FAKE, FAKE, ODD, 4, 16, 1, None), bn.ERR_ALIGN),
     (lambda L: L.bitnet_pack_weights(None, FAKE, 4, 8, None), bn.ERR_NULL),
     (lambda L: L.bitnet_linear(FAKE, FAKE, 0, FAKE, FAKE, 1, 32, 4, 64, None, 0, None),
      bn.ERR_WORKSPACE),

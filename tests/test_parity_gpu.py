@@ -366,3 +366,50 @@ def test_float32_activations_match_oracle(M, K, N):
     assert_bf16_close(bf16_bits(bn.bitnet_linear_noalloc(xd, pd, to_dev(sw))), ref)
     if M < 16:
         assert_bf16_close(bf16_bits(bn.bitnet_gemv_fused(xd, pd, to_dev(sw))), ref)
+
+
+# --------------------------------------------------- absmean ternarisation
+
+TERN_CASES = [(64, 320), (300, 4096), (4096, 2560), (7, 96), (1, 16)]
+
+
+def dense_weights(N, K, seed):
+    rng = np.random.default_rng(seed)
+    w = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    w[0, : min(K, 8)] = 0.0
+    if N > 2:
+        w[2] = 0.0                        # an all-zero row: gamma = eps
+    return w
+
+
+@pytest.mark.parametrize("per_row", [True, False])
+@pytest.mark.parametrize("N,K", TERN_CASES)
+def test_ternarize_absmean_bitexact(N, K, per_row):
+    w = dense_weights(N, K, N * 17 + K)
+    wt_ref, sc_ref = oracle.ternarize_absmean(w, per_row=per_row)
+    wt, sc = bn.bitnet_ternarize_absmean(to_dev(w), per_row=per_row)
+    assert np.array_equal(wt.cpu().numpy(), wt_ref)
+    assert np.array_equal(sc.cpu().numpy(), sc_ref)
+
+
+def test_ternarize_then_pack_and_linear_match_oracle():
+    """The load-time chain the page's BitLinear.from_dense runs: ternarise,
+    pack, then the layer, against the oracle's chain."""
+    N, K, M = 384, 1024, 20
+    w = dense_weights(N, K, 5)
+    wt, sc = bn.bitnet_ternarize_absmean(to_dev(w))
+    p = bn.bitnet_pack_weights(wt)
+    x = acts(92, 0, M, K)
+    wt_ref, sc_ref = oracle.ternarize_absmean(w)
+    ref = oracle.linear(x, oracle.pack(wt_ref), sc_ref)
+    assert_bf16_close(bf16_bits(bn.bitnet_linear(to_dev(x, torch.bfloat16), p, sc)), ref)
+
+
+def test_ternarize_rejects_non_finite():
+    w = torch.zeros((4, 64), dtype=torch.float32, device="cuda")
+    w[1, 5] = float("nan")
+    with pytest.raises(bn.BitnetValueError):
+        bn.bitnet_ternarize_absmean(w)
+    w[1, 5] = 2.0 ** 48
+    with pytest.raises(bn.BitnetValueError):
+        bn.bitnet_ternarize_absmean(w, per_row=False)
