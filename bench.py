@@ -592,6 +592,64 @@ def midbatch(bn, dev, pk):
             "peak_hbm_gbs": hbm, "peak_tops": tops_peak, "cases": cases}
 
 
+def extra_rows(bn, dev, pk):
+    """The rows beyond the layer itself: absmean ternarisation of a dense
+    float32 matrix (11008 x 4096, per row and per tensor; 180 MB read, 45 MB
+    written, plus the per-tensor form's second read), and the layer on float32
+    activations (decode GEMV at M = 1, bitnet_linear at M = 2048)."""
+    hbm = pk["hbm_gbs"]
+    tops_peak = pk["bf16_tflops"] * INT8_OVER_BF16
+    flush = torch.empty((2 * L2_BYTES,), dtype=torch.uint8, device=dev)
+
+    def timed(fn, reps=5):
+        ts = []
+        for r in range(reps + 2):
+            flush.fill_(r & 0xFF)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if r >= 2:
+                ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    out = {}
+    N, K = 11008, 4096
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    w = torch.randn((N, K), device=dev, generator=g) * 0.02
+    wt = torch.empty((N, K), dtype=torch.int8, device=dev)
+    for per_row, name in ((True, "ternarize_per_row"), (False, "ternarize_per_tensor")):
+        sc = torch.empty((N if per_row else 1,), dtype=torch.float32, device=dev)
+        ms = timed(lambda: bn.bitnet_ternarize_absmean(w, per_row=per_row, w_t=wt, scale_wt=sc))
+        byts = N * K * 4 * (1 if per_row else 2) + N * K + 4 * sc.numel()
+        out[name] = {"N": N, "K": K, "ms": ms, "gbs": byts / ms / 1e6,
+                     "frac_hbm": byts / ms / 1e6 / hbm,
+                     "note": "includes the call's synchronisation for the value check"}
+    del w, wt
+    wp = bn.bitnet_pack_weights(torch.ones((N, K), dtype=torch.int8, device=dev))
+    copies = weight_rotation(wp)
+    sw = torch.tensor([0.05], dtype=torch.float32, device=dev)
+    x1 = torch.randn((1, K), device=dev, generator=g)
+    o1 = torch.empty((1, N), dtype=torch.bfloat16, device=dev)
+    ms = time_rotation([lambda c=c: bn.bitnet_gemv_fused(x1, c, sw, out=o1) for c in copies])
+    byts = N * K // 4 + 4 * K + 2 * N + 4
+    out["gemv_f32_m1"] = {"M": 1, "K": K, "N": N, "ms": ms, "gbs": byts / ms / 1e6,
+                          "frac_hbm": byts / ms / 1e6 / hbm}
+    del copies
+    M = 2048
+    xl = torch.randn((M, K), device=dev, generator=g)
+    ol = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty((bn.bitnet_linear_workspace_bytes(M, K),), dtype=torch.uint8, device=dev)
+    ms = timed(lambda: bn.bitnet_linear(xl, wp, sw, out=ol, workspace=ws))
+    ops = 2.0 * M * N * K
+    out["linear_f32_m2048"] = {"M": M, "K": K, "N": N, "ms": ms, "tops": ops / ms / 1e9,
+                               "frac": ops / ms / 1e9 / tops_peak}
+    bn.bitnet_device_status()
+    return out
+
+
 # ----------------------------------------------------------- CPU oracle
 
 def cpu_baseline(seconds):
@@ -775,6 +833,7 @@ def main():
     pre = None if args.no_prefill else prefill(bn, dev, pk)
     gemv_mb = None if args.no_secondary else llama_gemv(bn, dev, pk)
     mid = None if args.no_secondary else midbatch(bn, dev, pk)
+    extra = None if args.no_secondary else extra_rows(bn, dev, pk)
 
     if rank != 0:
         if pg is not None:
@@ -808,6 +867,7 @@ def main():
         "prefill": pre,
         "llama_gemv": gemv_mb,
         "midbatch": mid,
+        "extra_rows": extra,
     }
     print(json.dumps(line))
     if pg is not None:

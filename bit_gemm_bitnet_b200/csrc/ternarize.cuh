@@ -54,30 +54,52 @@ __device__ __forceinline__ float mean_of(u128 sum, double count) {
   return static_cast<float>(ldexp(__ddiv_rn(u128_to_double_rn(sum), count), -64));
 }
 
-// Sum of the |w| of the CTA's items, exact; the per-thread partial sums are
-// combined by thread 0 in a fixed order. `part` holds 2 words per thread.
+// Sum of the |w| of the CTA's items, exact (integer additions in any order):
+// a butterfly over each warp's 128-bit partial sums (two 64-bit halves with
+// the carry), then thread 0 adds the warps' sums. `part` holds 2 words per
+// warp.
 __device__ __forceinline__ u128 cta_sum(u128 mine, uint64_t* part) {
-  const int tid = threadIdx.x;
-  part[2 * tid] = static_cast<uint64_t>(mine);
-  part[2 * tid + 1] = static_cast<uint64_t>(mine >> 64);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint64_t lo = static_cast<uint64_t>(mine), hi = static_cast<uint64_t>(mine >> 64);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const uint64_t olo = __shfl_xor_sync(0xFFFFFFFFu, lo, o);
+    const uint64_t ohi = __shfl_xor_sync(0xFFFFFFFFu, hi, o);
+    const uint64_t nlo = lo + olo;
+    hi = hi + ohi + (nlo < lo ? 1u : 0u);
+    lo = nlo;
+  }
+  if (lane == 0) {
+    part[2 * warp] = lo;
+    part[2 * warp + 1] = hi;
+  }
   __syncthreads();
   u128 total = 0;
   if (tid == 0)
-    for (int t = 0; t < static_cast<int>(blockDim.x); ++t)
-      total += (static_cast<u128>(part[2 * t + 1]) << 64) | part[2 * t];
+    for (int w = 0; w < static_cast<int>(blockDim.x) / 32; ++w)
+      total += (static_cast<u128>(part[2 * w + 1]) << 64) | part[2 * w];
   return total;  // valid in thread 0
 }
 
 constexpr int kTernThreads = 256;
 
+// The code of one weight: clamp(round-half-even(fl(w / gamma)), -1, 1), which
+// only depends on whether |fl(w / gamma)| is below, at or above 1/2. The
+// product w * fl(1 / gamma) is within 2^-22 |w / gamma| of the quotient, so it
+// decides alone unless it lies within 1e-6 of 1/2; there the exact quotient
+// decides.
+__device__ __forceinline__ uint32_t ternary1(float x, float gamma, float rgamma) {
+  float y = __fmul_rn(x, rgamma);
+  if (fabsf(fabsf(y) - 0.5f) < 1e-6f) y = __fdiv_rn(x, gamma);
+  const float a = fabsf(y);
+  const int r = a > 0.5f ? (y > 0.0f ? 1 : -1) : 0;  // a == 0.5 rounds to 0 (even)
+  return static_cast<uint32_t>(r) & 0xFFu;
+}
+
 // Four codes of w[0..3] / gamma, packed little-endian.
-__device__ __forceinline__ uint32_t ternary4(const float4& v, float gamma) {
-  auto one = [&](float x) {
-    int r = __float2int_rn(__fdiv_rn(x, gamma));
-    r = r < -1 ? -1 : (r > 1 ? 1 : r);
-    return static_cast<uint32_t>(r) & 0xFFu;
-  };
-  return one(v.x) | (one(v.y) << 8) | (one(v.z) << 16) | (one(v.w) << 24);
+__device__ __forceinline__ uint32_t ternary4(const float4& v, float gamma, float rgamma) {
+  return ternary1(v.x, gamma, rgamma) | (ternary1(v.y, gamma, rgamma) << 8) |
+         (ternary1(v.z, gamma, rgamma) << 16) | (ternary1(v.w, gamma, rgamma) << 24);
 }
 
 __device__ __forceinline__ u128 row_abs_sum(const float4* row, int nvec, bool* ok) {
@@ -101,7 +123,7 @@ __device__ __forceinline__ u128 row_abs_sum(const float4* row, int nvec, bool* o
 __global__ void __launch_bounds__(kTernThreads)
     ternarize_rows_kernel(int8_t* __restrict__ wt, float* __restrict__ scale,
                           const float* __restrict__ w, int K) {
-  __shared__ uint64_t part[2 * kTernThreads];
+  __shared__ uint64_t part[2 * (kTernThreads / 32)];
   __shared__ float gamma_s;
   const int64_t n = blockIdx.x;
   const float4* row = reinterpret_cast<const float4*>(w + n * K);
@@ -115,8 +137,10 @@ __global__ void __launch_bounds__(kTernThreads)
   }
   __syncthreads();
   const float gamma = gamma_s;
+  const float rgamma = __fdiv_rn(1.0f, gamma);
   uint32_t* out = reinterpret_cast<uint32_t*>(wt + n * K);
-  for (int i = threadIdx.x; i < nvec; i += kTernThreads) out[i] = ternary4(__ldg(row + i), gamma);
+  for (int i = threadIdx.x; i < nvec; i += kTernThreads)
+    out[i] = ternary4(__ldg(row + i), gamma, rgamma);
   if (threadIdx.x == 0) scale[n] = bf16_bits_to_f32(f32_to_bf16_bits(gamma));
 }
 
@@ -124,7 +148,7 @@ __global__ void __launch_bounds__(kTernThreads)
 // 16 bytes of the row's output (K % 16 == 0).
 __global__ void __launch_bounds__(kTernThreads)
     ternarize_rowsum_kernel(int8_t* __restrict__ wt, const float* __restrict__ w, int K) {
-  __shared__ uint64_t part[2 * kTernThreads];
+  __shared__ uint64_t part[2 * (kTernThreads / 32)];
   const int64_t n = blockIdx.x;
   bool ok = true;
   const u128 total = cta_sum(row_abs_sum(reinterpret_cast<const float4*>(w + n * K), K / 4, &ok),
@@ -141,7 +165,7 @@ __global__ void __launch_bounds__(kTernThreads)
 __global__ void __launch_bounds__(kTernThreads)
     ternarize_total_kernel(float* __restrict__ scale, const int8_t* __restrict__ wt, int64_t N,
                            int K) {
-  __shared__ uint64_t part[2 * kTernThreads];
+  __shared__ uint64_t part[2 * (kTernThreads / 32)];
   u128 s = 0;
   for (int64_t n = threadIdx.x; n < N; n += kTernThreads) {
     const uint64_t* src = reinterpret_cast<const uint64_t*>(wt + n * K);
@@ -160,9 +184,11 @@ __global__ void __launch_bounds__(kTernThreads)
                            const float* __restrict__ w, int K) {
   const int64_t n = blockIdx.x;
   const float gamma = scale[0];
+  const float rgamma = __fdiv_rn(1.0f, gamma);
   const float4* row = reinterpret_cast<const float4*>(w + n * K);
   uint32_t* out = reinterpret_cast<uint32_t*>(wt + n * K);
-  for (int i = threadIdx.x; i < K / 4; i += kTernThreads) out[i] = ternary4(__ldg(row + i), gamma);
+  for (int i = threadIdx.x; i < K / 4; i += kTernThreads)
+    out[i] = ternary4(__ldg(row + i), gamma, rgamma);
 }
 
 // Step 4: scale[0] = bf16(gamma), once every row has its codes.
