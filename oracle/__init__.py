@@ -31,6 +31,7 @@ def lib():
         L.oracle_unpack.argtypes = [_P, _I64, _I64, _P]
         L.oracle_quantize.argtypes = [_P, _I64, _I64, _P, _P]
         L.oracle_quantize_f32.argtypes = [_P, _I64, _I64, _P, _P]
+        L.oracle_linear_bias.argtypes = [_P, _P, _P, _I64, _P, _I64, _I64, _I64, _P]
         L.oracle_ternarize_absmean.argtypes = [_P, _I64, _I64, ctypes.c_int, _P, _P]
         L.oracle_linear_f32.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P]
         L.oracle_acc.argtypes = [_P, _P, _I64, _I64, _I64, _P]
@@ -46,7 +47,7 @@ def lib():
         L.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
         L.oracle_f32_to_bf16.restype = ctypes.c_uint16
         for name in ("oracle_pack", "oracle_unpack", "oracle_quantize", "oracle_quantize_f32",
-                     "oracle_ternarize_absmean",
+                     "oracle_ternarize_absmean", "oracle_linear_bias",
                      "oracle_linear_f32",
                      "oracle_acc", "oracle_epilogue", "oracle_gemm",
                      "oracle_linear", "oracle_linear_threads",
@@ -133,6 +134,20 @@ def ternarize_absmean(w, per_row=True):
     _check(lib().oracle_ternarize_absmean(_ptr(w), N, K, 1 if per_row else 0, _ptr(wt), _ptr(sc)),
            "ternarize_absmean")
     return wt, sc
+
+
+def linear_bias(x_bf16_bits, packed, scale_wt, bias_bf16_bits):
+    """bitnet_linear, then + bias (bf16 [N]) as the page's BitLinear.forward."""
+    x = _c(x_bf16_bits, np.uint16)
+    packed = _c(packed, np.uint8)
+    sw = _c(scale_wt, np.float32)
+    b = _c(bias_bf16_bits, np.uint16)
+    M, K = x.shape
+    N = packed.shape[0]
+    out = np.empty((M, N), np.uint16)
+    _check(lib().oracle_linear_bias(_ptr(x), _ptr(packed), _ptr(sw), sw.size, _ptr(b), M, N, K,
+                                    _ptr(out)), "linear_bias")
+    return out
 
 
 def acc(q, packed, N=None):

@@ -332,6 +332,23 @@ int oracle_linear_threads_cols(const uint16_t* x, const uint8_t* packed,
 // library conversion on its own.
 uint16_t oracle_f32_to_bf16(float f) { return float_to_bf16_bits_rne(f); }
 
+// bitnet_linear followed by the layer's bias (BitLinear.forward on the
+// bitnet-cpu page: y = bitnet_linear(...); y = y + bias, both bf16): the
+// bf16 output of the layer plus the bf16 bias, added in fp32 and rounded to
+// bf16 again. bias is bf16 [N] (raw bits).
+int oracle_linear_bias(const uint16_t* x, const uint8_t* packed, const float* scale_wt,
+                       int64_t scale_wt_len, const uint16_t* bias, int64_t M, int64_t N,
+                       int64_t K, uint16_t* out) {
+  int st = oracle_linear(x, packed, scale_wt, scale_wt_len, M, N, K, out);
+  if (st != OK) return st;
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t n = 0; n < N; ++n) {
+      const float y = bf16_bits_to_float(out[m * N + n]) + bf16_bits_to_float(bias[n]);
+      out[m * N + n] = float_to_bf16_bits_rne(y);
+    }
+  return OK;
+}
+
 // ------------------------------------------------------------------------
 // Absmean ternarisation (bitnet-cpu page: BitLinear.from_dense per output
 // row, gamma clamped at 1e-8; BitLinearKernel per tensor, clamped at 1e-5):

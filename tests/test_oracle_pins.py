@@ -386,3 +386,41 @@ def test_ternarize_rejects_non_finite():
     w[1, 3] = np.inf
     with pytest.raises(Exception):
         oracle.ternarize_absmean(w)
+
+
+# --------------------------------------------------------------- bias
+
+
+def test_linear_bias_rounding_worked_examples():
+    """y + bias in bf16 (BitLinear.forward on the bitnet-cpu page). The layer
+    outputs exactly +1.0 or -1.0 (one input 127 -> q = 127 at scale 1.0, one
+    weight +1 or -1, scale_wt = 1/127: 127 * fl(1/127) rounds to bf16 1.0).
+    bf16 has 8 significant bits, so an ulp at 1.0 is 2^-7 and:
+    bias 2^-9 (a quarter ulp) -> 1.0; 2^-8 (half an ulp, a tie) -> 1.0, the
+    even neighbour; 2^-7 -> 1.0078125; 0.5 -> 1.5; -1.0 + 0 -> -1.0."""
+    K = 32
+    x = np.zeros((1, K), np.uint16)
+    x[0, 0] = f32_to_bf16_bits_np(np.float32(127.0))
+    w = np.zeros((5, K), np.int8)
+    w[:4, 0] = 1
+    w[4, 0] = -1
+    p = oracle.pack(w)
+    sw = np.array([np.float32(1.0) / np.float32(127.0)], np.float32)
+    bias = f32_to_bf16_bits_np(np.array([2 ** -9, 2 ** -8, 2 ** -7, 0.5, 0.0], np.float32))
+    yb = (oracle.linear(x, p, sw).astype(np.uint32) << 16).view(np.float32)[0]
+    assert yb.tolist() == [1.0, 1.0, 1.0, 1.0, -1.0]
+    y = (oracle.linear_bias(x, p, sw, bias).astype(np.uint32) << 16).view(np.float32)[0]
+    assert y.tolist() == [1.0, 1.0, 1.0078125, 1.5, -1.0]
+
+
+def test_linear_bias_matches_torch_bf16_addition():
+    torch = pytest.importorskip("torch")
+    x = synth.act_bf16(synth.key(91, 0, synth.T_ACT), 9, 256)
+    p = oracle.pack(synth.ternary(synth.key(91, 0, synth.T_WEIGHT), 70, 256))
+    sw = synth.uniform_f32(synth.key(91, 0, 3), 70, 0.01, 0.1)
+    bias = f32_to_bf16_bits_np(np.random.default_rng(4).standard_normal(70).astype(np.float32))
+    bias[:3] = [0x0000, 0x8000, 0x3F80]
+    y = torch.from_numpy(oracle.linear(x, p, sw).view(np.int16).copy()).view(torch.bfloat16)
+    b = torch.from_numpy(bias.view(np.int16).copy()).view(torch.bfloat16)
+    ref = (y + b).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.linear_bias(x, p, sw, bias), ref)
