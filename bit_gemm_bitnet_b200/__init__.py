@@ -30,6 +30,7 @@ EXPORTS = (
     "bitnet_gemv_fused", "bitnet_linear_workspace_bytes", "bitnet_linear",
     "bitnet_device_status", "bitnet_status_string", "bitnet_gemm_acc_i32",
     "bitnet_gemv_fused_debug", "bitnet_linear_noalloc", "bitnet_gemv_fused_grouped",
+    "bitnet_linear_bias",
 )
 
 
@@ -70,6 +71,7 @@ def lib():
             "bitnet_gemm": [P, P, P, P, P, I64, I64, I64, I64, P],
             "bitnet_gemv_fused": [P, P, I, P, P, I64, I64, I64, I64, P],
             "bitnet_linear": [P, P, I, P, P, I64, I64, I64, I64, P, SZ, P],
+            "bitnet_linear_bias": [P, P, I, P, P, I64, P, I64, I64, I64, P, SZ, P],
             "bitnet_linear_noalloc": [P, P, I, P, P, I64, I64, I64, I64, P],
             "bitnet_gemv_fused_grouped": [P, I64, I64, I, P],
             "bitnet_device_status": [P],
@@ -261,9 +263,11 @@ def bitnet_linear_workspace_bytes(M, K):
     return int(lib().bitnet_linear_workspace_bytes(M, K))
 
 
-def bitnet_linear(x, w_packed, scale_wt, out=None, workspace=None):
+def bitnet_linear(x, w_packed, scale_wt, out=None, workspace=None, bias=None):
     """bf16 or float32 [..., K] -> bf16 [..., N]; dispatches by M like the
-    page's bitnet_linear (fused GEMV for M < 16, else quantise + GEMM)."""
+    page's bitnet_linear (fused GEMV for M < 16, else quantise + GEMM).
+    bias (bf16 [N]), if given, is added in the epilogue as the page's
+    BitLinear.forward adds it to the bf16 output."""
     orig = x.shape
     K = orig[-1]
     x2 = x.reshape(-1, K)
@@ -280,9 +284,18 @@ def bitnet_linear(x, w_packed, scale_wt, out=None, workspace=None):
     if need and (workspace is None or workspace.numel() < need):
         workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
     wsp = _ptr(workspace) if need else None
-    _check(lib().bitnet_linear(_ptr(out), _ptr(x2), dt, _ptr(w_packed), _ptr(sw),
-                               sw.numel(), M, N, K, wsp, need, _stream(x.device)),
-           "bitnet_linear")
+    if bias is None:
+        _check(lib().bitnet_linear(_ptr(out), _ptr(x2), dt, _ptr(w_packed), _ptr(sw),
+                                   sw.numel(), M, N, K, wsp, need, _stream(x.device)),
+               "bitnet_linear")
+    else:
+        _need(bias, torch.bfloat16, "bias", 1)
+        if bias.numel() != N:
+            raise ValueError(f"bias has {bias.numel()} elements, expected N={N}")
+        _check(lib().bitnet_linear_bias(_ptr(out), _ptr(x2), dt, _ptr(w_packed), _ptr(sw),
+                                        sw.numel(), _ptr(bias), M, N, K, wsp, need,
+                                        _stream(x.device)),
+               "bitnet_linear_bias")
     return out.view(*orig[:-1], N)
 
 

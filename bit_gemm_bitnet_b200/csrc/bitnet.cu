@@ -493,7 +493,8 @@ int sk_split(Kernel kernel, int smem, int64_t w_tiles, int64_t kblocks) {
 template <int BX, bool kAccOut, bool kPerm>
 bitnet_status launch_sk(const CUtensorMap& mx, const CUtensorMap& mw, void* out,
                         const uint16_t* sa, const float* sw, int64_t sw_len,
-                        const int32_t* rowsum, int64_t M, int64_t N, int64_t K, cudaStream_t st) {
+                        const int32_t* rowsum, int64_t M, int64_t N, int64_t K, cudaStream_t st,
+                        const uint16_t* bias) {
   auto kernel = sk::gemm_i8_sk_kernel<BX, kAccOut, kPerm>;
   constexpr int smem = sk::Cfg<BX>::SMEM_BYTES;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
@@ -506,32 +507,32 @@ bitnet_status launch_sk(const CUtensorMap& mx, const CUtensorMap& mw, void* out,
   return launch_pdl_cluster(kernel, dim3(static_cast<unsigned>(w_tiles * S)),
                             dim3(sk::NUM_THREADS), smem, S, st, mx, mw, out, sa, sw,
                             static_cast<int>(sw_len), rowsum, static_cast<int>(M),
-                            static_cast<int>(N), static_cast<int>(K), S);
+                            static_cast<int>(N), static_cast<int>(K), S, bias);
 }
 
 template <int BX>
 bitnet_status run_sk_bx(void* out, bool acc_out, const int8_t* xq, const uint8_t* wp,
                         const uint16_t* sa, const float* sw, int64_t sw_len, int64_t M,
                         int64_t N, int64_t K, cudaStream_t st, bool perm,
-                        const int32_t* rowsum) {
+                        const int32_t* rowsum, const uint16_t* bias) {
   CUtensorMap mx, mw;
   if (!make_map_u8(&mx, xq, M, K, K, BX, sk::BK, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_u8(&mw, wp, N, K / 4, K / 4, sk::BW, sk::BK / 4, CU_TENSOR_MAP_SWIZZLE_NONE))
     return BITNET_ERR_CUDA;
-  if (acc_out) return launch_sk<BX, true, false>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st);
-  if (perm) return launch_sk<BX, false, true>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st);
-  return launch_sk<BX, false, false>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st);
+  if (acc_out) return launch_sk<BX, true, false>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st, nullptr);
+  if (perm) return launch_sk<BX, false, true>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st, bias);
+  return launch_sk<BX, false, false>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st, bias);
 }
 
 bitnet_status run_gemm_sk(void* out, bool acc_out, const int8_t* xq, const uint8_t* wp,
                           const uint16_t* sa, const float* sw, int64_t sw_len, int64_t M,
                           int64_t N, int64_t K, cudaStream_t st, bool perm,
-                          const int32_t* rowsum) {
-  if (M <= 16) return run_sk_bx<16>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum);
-  if (M <= 32) return run_sk_bx<32>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum);
-  if (M <= 64) return run_sk_bx<64>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum);
-  if (M <= 128) return run_sk_bx<128>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum);
-  return run_sk_bx<256>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum);
+                          const int32_t* rowsum, const uint16_t* bias) {
+  if (M <= 16) return run_sk_bx<16>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
+  if (M <= 32) return run_sk_bx<32>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
+  if (M <= 64) return run_sk_bx<64>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
+  if (M <= 128) return run_sk_bx<128>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
+  return run_sk_bx<256>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
 }
 
 // ------------------------------ fused quantise + tensor-core GEMV (4 <= M)
@@ -544,7 +545,7 @@ bool skq_ok(const void* x, const uint8_t* wp, int64_t M, int64_t K) {
 
 bitnet_status run_gemv_skq(uint16_t* out, const uint16_t* x, const uint8_t* wp,
                            const float* sw, int64_t sw_len, int64_t M, int64_t N, int64_t K,
-                           cudaStream_t st) {
+                           cudaStream_t st, const uint16_t* bias) {
   auto kernel = skq::gemv_i8_skq_kernel;
   constexpr int smem = skq::SMEM_BYTES;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
@@ -577,7 +578,7 @@ bitnet_status run_gemv_skq(uint16_t* out, const uint16_t* x, const uint8_t* wp,
   return launch_pdl_cluster(kernel, dim3(static_cast<unsigned>(w_tiles * best)),
                             dim3(skq::NUM_THREADS), smem, best, st, mw, out, x, sw,
                             static_cast<int>(sw_len), static_cast<int>(M), static_cast<int>(N),
-                            static_cast<int>(K), best);
+                            static_cast<int>(K), best, bias);
 }
 
 // perm: x_q has transposed 16-element groups and rowsum holds its per-row
@@ -585,7 +586,7 @@ bitnet_status run_gemv_skq(uint16_t* out, const uint16_t* x, const uint8_t* wp,
 bitnet_status run_gemm(void* out, bool acc_out, const int8_t* xq, const uint8_t* wp,
                        const uint16_t* sa, const float* sw, int64_t sw_len, int64_t M,
                        int64_t N, int64_t K, cudaStream_t st, bool perm = false,
-                       const int32_t* rowsum = nullptr) {
+                       const int32_t* rowsum = nullptr, const uint16_t* bias = nullptr) {
   if (M == 0 || N == 0) return BITNET_OK;
   if (!gemm_tc_ok(xq, wp, K)) {
     if (perm) return BITNET_ERR_SHAPE;  // callers only ask for perm when it applies
@@ -600,9 +601,11 @@ bitnet_status run_gemm(void* out, bool acc_out, const int8_t* xq, const uint8_t*
     p.M = static_cast<int>(M);
     p.N = static_cast<int>(N);
     p.K = static_cast<int>(K);
+    p.bias = bias;
     return run_gemv(p, true, st);
   }
-  if (M <= kSkMaxRows) return run_gemm_sk(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum);
+  if (M <= kSkMaxRows)
+    return run_gemm_sk(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
   DeviceInfo* dev = nullptr;
   bitnet_status s = device_info(&dev);
   if (s != BITNET_OK) return s;
@@ -619,7 +622,7 @@ bitnet_status run_gemm(void* out, bool acc_out, const int8_t* xq, const uint8_t*
       return BITNET_ERR_CUDA;
     return launch_pdl(kernel, dim3(grid), dim3(ts::NUM_THREADS), ts::SMEM_BYTES, st, mx, mw,
                       out, sa, sw, static_cast<int>(sw_len), rowsum, static_cast<int>(M),
-                      static_cast<int>(N), static_cast<int>(K));
+                      static_cast<int>(N), static_cast<int>(K), acc_out ? nullptr : bias);
   };
   if (acc_out) return go(ts::gemm_i8_ts_kernel<true, false>);
   if (perm) return go(ts::gemm_i8_ts_kernel<false, true>);
@@ -855,10 +858,10 @@ static bitnet_status gemv_common(GemvParams& p, const void* x, bitnet_dtype dt,
   return BITNET_OK;
 }
 
-bitnet_status bitnet_gemv_fused(uint16_t* out, const void* x, bitnet_dtype dt,
-                                const uint8_t* w_packed, const float* scale_wt,
-                                int64_t scale_wt_len, int64_t M, int64_t N, int64_t K,
-                                void* stream) {
+static bitnet_status gemv_fused_impl(uint16_t* out, const void* x, bitnet_dtype dt,
+                                     const uint8_t* w_packed, const float* scale_wt,
+                                     int64_t scale_wt_len, const uint16_t* bias, int64_t M,
+                                     int64_t N, int64_t K, void* stream) {
   GemvParams p = {};
   bitnet_status s = gemv_common(p, x, dt, w_packed, M, N, K);
   if (s != BITNET_OK) return s;
@@ -867,15 +870,24 @@ bitnet_status bitnet_gemv_fused(uint16_t* out, const void* x, bitnet_dtype dt,
   if (!aligned(out, 16)) return BITNET_ERR_ALIGN;
   s = check_scale_wt(scale_wt, scale_wt_len, N);
   if (s != BITNET_OK) return s;
+  if (bias != nullptr && !aligned(bias, 2)) return BITNET_ERR_ALIGN;
   p.out = out;
   p.sw = scale_wt;
   p.sw_len = static_cast<int>(scale_wt_len);
+  p.bias = bias;
   if (dt == BITNET_BF16 && skq_ok(x, w_packed, M, K) && K / 128 <= sk::MAX_SPLIT * skq::MAX_KB) {
     const bitnet_status r = run_gemv_skq(out, static_cast<const uint16_t*>(x), w_packed,
-                                         scale_wt, scale_wt_len, M, N, K, as_stream(stream));
+                                         scale_wt, scale_wt_len, M, N, K, as_stream(stream), bias);
     if (r != BITNET_ERR_SHAPE) return r;
   }
   return run_gemv(p, false, as_stream(stream));
+}
+
+bitnet_status bitnet_gemv_fused(uint16_t* out, const void* x, bitnet_dtype dt,
+                                const uint8_t* w_packed, const float* scale_wt,
+                                int64_t scale_wt_len, int64_t M, int64_t N, int64_t K,
+                                void* stream) {
+  return gemv_fused_impl(out, x, dt, w_packed, scale_wt, scale_wt_len, nullptr, M, N, K, stream);
 }
 
 bitnet_status bitnet_gemv_fused_grouped(const bitnet_gemv_problem* problems, int64_t count,
@@ -944,16 +956,18 @@ size_t bitnet_linear_workspace_bytes(int64_t M, int64_t K) {
          align256(static_cast<size_t>(M) * 2) + align256(static_cast<size_t>(M) * 4);
 }
 
-bitnet_status bitnet_linear(uint16_t* out, const void* x, bitnet_dtype dt,
-                            const uint8_t* w_packed, const float* scale_wt,
-                            int64_t scale_wt_len, int64_t M, int64_t N, int64_t K,
-                            void* workspace, size_t workspace_bytes, void* stream) {
+static bitnet_status linear_impl(uint16_t* out, const void* x, bitnet_dtype dt,
+                                 const uint8_t* w_packed, const float* scale_wt,
+                                 int64_t scale_wt_len, const uint16_t* bias, int64_t M, int64_t N,
+                                 int64_t K, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
   if (dt != BITNET_BF16 && dt != BITNET_F32) return BITNET_ERR_DTYPE;
   bitnet_status s = check_compute_shape(M, N, K);
   if (s != BITNET_OK) return s;
   if (M == 0 || N == 0) return BITNET_OK;
   if (linear_uses_gemv(M, K))
-    return bitnet_gemv_fused(out, x, dt, w_packed, scale_wt, scale_wt_len, M, N, K, stream);
+    return gemv_fused_impl(out, x, dt, w_packed, scale_wt, scale_wt_len, bias, M, N, K, stream);
+  if (bias != nullptr && !aligned(bias, 2)) return BITNET_ERR_ALIGN;
   const size_t need = bitnet_linear_workspace_bytes(M, K);
   if (workspace == nullptr || workspace_bytes < need) return BITNET_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return BITNET_ERR_ALIGN;
@@ -975,11 +989,30 @@ bitnet_status bitnet_linear(uint16_t* out, const void* x, bitnet_dtype dt,
                          : run_quantize_perm(xq, sa, rowsum, xb, M, K, st);
     if (s != BITNET_OK) return s;
     return run_gemm(out, false, xq, w_packed, sa, scale_wt, scale_wt_len, M, N, K, st, true,
-                    rowsum);
+                    rowsum, bias);
   }
   s = dt == BITNET_F32 ? run_quantize_f32(xq, sa, xf, M, K, st) : run_quantize(xq, sa, xb, M, K, st);
   if (s != BITNET_OK) return s;
-  return run_gemm(out, false, xq, w_packed, sa, scale_wt, scale_wt_len, M, N, K, st);
+  return run_gemm(out, false, xq, w_packed, sa, scale_wt, scale_wt_len, M, N, K, st, false,
+                  nullptr, bias);
+}
+
+bitnet_status bitnet_linear(uint16_t* out, const void* x, bitnet_dtype dt,
+                            const uint8_t* w_packed, const float* scale_wt,
+                            int64_t scale_wt_len, int64_t M, int64_t N, int64_t K,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  return linear_impl(out, x, dt, w_packed, scale_wt, scale_wt_len, nullptr, M, N, K, workspace,
+                     workspace_bytes, stream);
+}
+
+bitnet_status bitnet_linear_bias(uint16_t* out, const void* x, bitnet_dtype dt,
+                                 const uint8_t* w_packed, const float* scale_wt,
+                                 int64_t scale_wt_len, const uint16_t* bias, int64_t M,
+                                 int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  if (bias == nullptr) return BITNET_ERR_NULL;
+  return linear_impl(out, x, dt, w_packed, scale_wt, scale_wt_len, bias, M, N, K, workspace,
+                     workspace_bytes, stream);
 }
 
 bitnet_status bitnet_linear_noalloc(uint16_t* out, const void* x, bitnet_dtype dt,

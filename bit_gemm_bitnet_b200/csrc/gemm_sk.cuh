@@ -102,7 +102,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                       const __grid_constant__ CUtensorMap tmap_w, void* __restrict__ out,
                       const uint16_t* __restrict__ scale_act,
                       const float* __restrict__ scale_wt, int sw_len,
-                      const int32_t* __restrict__ rowsum, int M, int N, int K, int S) {
+                      const int32_t* __restrict__ rowsum, int M, int N, int K, int S,
+                      const uint16_t* __restrict__ bias) {
   using C = Cfg<BX>;
   constexpr int ST = C::STAGES;
   constexpr uint32_t kIdesc = kPerm ? C::kIdescShape : (C::kIdescShape | (1u << 7));
@@ -323,6 +324,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int j = 0; j < 4; ++j) {
           const float swj = (n + j < N) ? scale_wt[sw_len == 1 ? 0 : n + j] : 0.0f;
           y[j] = f32_to_bf16_bits(__fmul_rn(__fmul_rn(__int2float_rn(a[j]), sa), swj));
+          if (bias != nullptr && n + j < N) y[j] = add_bias_bf16(y[j], bias, n + j);
         }
         uint16_t* o = static_cast<uint16_t*>(out) + static_cast<int64_t>(m) * N + n;
         if (whole) {

@@ -99,7 +99,8 @@ __device__ __forceinline__ int sw128_off(int m, int kk) {
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemv_i8_skq_kernel(const __grid_constant__ CUtensorMap tmap_w, uint16_t* __restrict__ out,
                        const uint16_t* __restrict__ x, const float* __restrict__ scale_wt,
-                       int sw_len, int M, int N, int K, int S) {
+                       int sw_len, int M, int N, int K, int S,
+                       const uint16_t* __restrict__ bias) {
   extern __shared__ uint8_t smem_raw[];
   Smem sm;
   sm.base = reinterpret_cast<uint8_t*>(
@@ -361,6 +362,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int j = 0; j < 4; ++j) {
         const float swj = (n + j < N) ? scale_wt[sw_len == 1 ? 0 : n + j] : 0.0f;
         y[j] = f32_to_bf16_bits(__fmul_rn(__fmul_rn(__int2float_rn(a[j]), sa), swj));
+        if (bias != nullptr && n + j < N) y[j] = add_bias_bf16(y[j], bias, n + j);
       }
       uint16_t* o = out + static_cast<int64_t>(m) * N + n;
       if (n + 3 < N && (N & 3) == 0) {

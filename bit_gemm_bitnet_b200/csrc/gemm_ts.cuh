@@ -114,7 +114,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                       const __grid_constant__ CUtensorMap tmap_w, void* __restrict__ out,
                       const uint16_t* __restrict__ scale_act,
                       const float* __restrict__ scale_wt, int sw_len,
-                      const int32_t* __restrict__ rowsum, int M, int N, int K) {
+                      const int32_t* __restrict__ rowsum, int M, int N, int K,
+                      const uint16_t* __restrict__ bias) {
   constexpr uint32_t kIdesc = kPerm ? kIdescUnsignedA : kIdescSignedA;
   extern __shared__ uint8_t smem_raw[];
   Smem sm;
@@ -233,6 +234,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int n = (t % w_tiles) * BW + quarter * 32 + lane;
       float swn = 0.0f;
       if (!kAccOut && n < N) swn = scale_wt[sw_len == 1 ? 0 : n];
+      const uint16_t* bias_n = (bias != nullptr && n < N) ? bias : nullptr;  // lane's weight row
       if (!mbar_wait_warp(sm.tfull(a), aph, abort)) break;
       tc_fence_after();
 #pragma unroll 1
@@ -261,7 +263,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             reinterpret_cast<int32_t*>(stg)[j * 32 + lane] = acc;
           } else {
             const float y = __fmul_rn(__fmul_rn(__int2float_rn(acc), sa_j), swn);
-            reinterpret_cast<uint16_t*>(stg)[j * 32 + lane] = f32_to_bf16_bits(y);
+            reinterpret_cast<uint16_t*>(stg)[j * 32 + lane] =
+                add_bias_bf16(f32_to_bf16_bits(y), bias_n, n);
           }
         }
         __syncwarp();

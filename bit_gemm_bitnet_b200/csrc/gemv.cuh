@@ -52,6 +52,7 @@ struct GemvParams {
   int8_t* dbg_q;          // optional: codes quantised on chip (block 0)
   uint16_t* dbg_sa;       // optional: their scales (block 0)
   int x_f32;              // x holds float32 values
+  const uint16_t* bias;   // optional bf16 [N], added to the bf16 output
 };
 
 // 4x4 byte transpose of a 16-byte group: out word i byte b = in word b byte i.
@@ -453,7 +454,8 @@ __device__ __forceinline__ void gemv_reduce_store(const int (&acc)[RW][MB][PLANE
                                                   const int* qsum, const float* saf,
                                                   uint16_t* __restrict__ out,
                                                   int32_t* __restrict__ acc_out,
-                                                  const float* __restrict__ sw, int sw_len) {
+                                                  const float* __restrict__ sw, int sw_len,
+                                                  const uint16_t* __restrict__ bias = nullptr) {
   const int lane = threadIdx.x & 31;
   // Reduce the RW x MB lane partials over the warp: a butterfly that halves
   // the number of values at each of the first log2(RW * MB) exchanges
@@ -499,7 +501,7 @@ __device__ __forceinline__ void gemv_reduce_store(const int (&acc)[RW][MB][PLANE
       } else {
         const float s_w = sw[sw_len == 1 ? 0 : n];
         const float y = __fmul_rn(__fmul_rn(__int2float_rn(a), saf[m]), s_w);
-        out[o] = f32_to_bf16_bits(y);
+        out[o] = add_bias_bf16(f32_to_bf16_bits(y), bias, n);
       }
     }
   }
@@ -654,7 +656,7 @@ __global__ void __launch_bounds__((CW + 1) * 32) gemv_kernel(GemvParams p) {
     if (lane == 0) mbar_arrive(empty(s));
 
     gemv_reduce_store<MB, RW, PLANES>(acc, rows, n0, Mc, m_base, N, qsum, saf, p.out, p.acc_out,
-                                      p.sw, p.sw_len);
+                                      p.sw, p.sw_len, p.bias);
   }
 }
 

@@ -185,6 +185,19 @@ bitnet_status bitnet_linear(uint16_t* out, const void* x, bitnet_dtype dt,
                             int64_t K, void* workspace, size_t workspace_bytes,
                             void* stream);
 
+/* bitnet_linear followed by the layer's bias, fused into the epilogue
+ * (BitLinear.forward on the bitnet-cpu page: y = bitnet_linear(...) + bias,
+ * a bf16 addition):
+ *   out[m,n] = bf16( fp32(y[m,n]) + fp32(bias[n]) ), y the bf16 result of
+ *   bitnet_linear.
+ *   bias  in, bf16 [N] (2-byte aligned, not NULL)
+ * The other arguments, the workspace and the result are bitnet_linear's. */
+bitnet_status bitnet_linear_bias(uint16_t* out, const void* x, bitnet_dtype dt,
+                                 const uint8_t* w_packed, const float* scale_wt,
+                                 int64_t scale_wt_len, const uint16_t* bias, int64_t M,
+                                 int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
 /* bitnet_linear without a caller workspace, for callers that cannot allocate
  * device memory: code running while a stream is being captured into a CUDA
  * graph (cudaMalloc is not allowed there), code inside a framework that owns

@@ -88,6 +88,11 @@ ODD = P(0x10008)
     (lambda L: L.bitnet_linear(FAKE, FAKE, 0, FAKE, FAKE, 1, 32, 4, 65, FAKE, 1 << 20, None),
      bn.ERR_SHAPE),
     (lambda L: L.bitnet_gemm_acc_i32(FAKE, None, FAKE, 4, 4, 64, None), bn.ERR_NULL),
+    (lambda L: L.bitnet_linear_bias(FAKE, FAKE, 0, FAKE, FAKE, 1, None, 4, 4, 64, None, 0, None),
+     bn.ERR_NULL),
+    (lambda L: L.bitnet_linear_bias(FAKE, FAKE, 0, FAKE, FAKE, 1, P(0x10001), 4, 4, 64, None, 0,
+                                    None),
+     bn.ERR_ALIGN),
     (lambda L: L.bitnet_gemv_fused_debug(FAKE, FAKE, None, FAKE, 0, FAKE, 1, 4, 64, None),
      bn.ERR_NULL),
 ])

@@ -413,3 +413,28 @@ def test_ternarize_rejects_non_finite():
     w[1, 5] = 2.0 ** 48
     with pytest.raises(bn.BitnetValueError):
         bn.bitnet_ternarize_absmean(w, per_row=False)
+
+
+# ----------------------------------------------------------- fused bias
+
+@pytest.mark.parametrize("M,K,N", [(1, 2560, 640), (3, 96, 40), (8, 4096, 300), (12, 2112, 77),
+                                   (20, 1024, 384), (300, 4096, 256), (37, 160, 77),
+                                   (2048, 2560, 1000)])
+def test_linear_bias_matches_oracle(M, K, N):
+    """The layer with its bf16 bias fused into every kernel's epilogue: the
+    fused dp4a and tensor-core GEMVs, the split-K and persistent GEMMs and
+    the SIMT path, against the oracle's y + bias."""
+    x = acts(90, M + K, M, K)
+    w = weights(90, N + K, N, K)
+    p = oracle.pack(w)
+    sw = synth.uniform_f32(synth.key(90, N, 3), N, 0.01, 0.1)
+    bias = f32_to_bf16_bits(np.random.default_rng(M + N).standard_normal(N).astype(np.float32))
+    bias[:2] = [0x0000, 0x8000]
+    got = bn.bitnet_linear(to_dev(x, torch.bfloat16), to_dev(p), to_dev(sw),
+                           bias=to_dev(bias, torch.bfloat16))
+    rows = np.arange(M) if M <= 64 else np.unique(np.r_[np.random.default_rng(M).choice(M, 40, replace=False), 0, M - 1])
+    ref = oracle.linear_bias(x[rows], p, sw, bias)
+    assert_bf16_close(bf16_bits(got)[rows], ref)
+    # without the bias the result is bitnet_linear's
+    plain = bn.bitnet_linear(to_dev(x, torch.bfloat16), to_dev(p), to_dev(sw))
+    assert_bf16_close(bf16_bits(plain)[rows], oracle.linear(x[rows], p, sw))
