@@ -595,8 +595,9 @@ def midbatch(bn, dev, pk):
 def extra_rows(bn, dev, pk):
     """The rows beyond the layer itself: absmean ternarisation of a dense
     float32 matrix (11008 x 4096, per row and per tensor; 180 MB read, 45 MB
-    written, plus the per-tensor form's second read), and the layer on float32
-    activations (decode GEMV at M = 1, bitnet_linear at M = 2048)."""
+    written, plus the per-tensor form's second read), the layer on float32
+    activations (decode GEMV at M = 1, bitnet_linear at M = 2048), and the
+    fused bias epilogue (bitnet_linear with and without bias at M = 2048)."""
     hbm = pk["hbm_gbs"]
     tops_peak = pk["bf16_tflops"] * INT8_OVER_BF16
     flush = torch.empty((2 * L2_BYTES,), dtype=torch.uint8, device=dev)
@@ -646,6 +647,13 @@ def extra_rows(bn, dev, pk):
     ops = 2.0 * M * N * K
     out["linear_f32_m2048"] = {"M": M, "K": K, "N": N, "ms": ms, "tops": ops / ms / 1e9,
                                "frac": ops / ms / 1e9 / tops_peak}
+    # the fused bias epilogue, against the same bf16 call without it
+    bias = (torch.randn((N,), device=dev, generator=g) * 0.1).to(torch.bfloat16)
+    xb = xl.to(torch.bfloat16)
+    ms_plain = timed(lambda: bn.bitnet_linear(xb, wp, sw, out=ol, workspace=ws))
+    ms_bias = timed(lambda: bn.bitnet_linear(xb, wp, sw, out=ol, workspace=ws, bias=bias))
+    out["linear_bias_m2048"] = {"M": M, "K": K, "N": N, "ms": ms_bias, "ms_without_bias": ms_plain,
+                                "tops": ops / ms_bias / 1e9, "frac": ops / ms_bias / 1e9 / tops_peak}
     bn.bitnet_device_status()
     return out
 
