@@ -31,6 +31,10 @@ def lib():
         L.oracle_unpack.argtypes = [_P, _I64, _I64, _P]
         L.oracle_quantize.argtypes = [_P, _I64, _I64, _P, _P]
         L.oracle_quantize_f32.argtypes = [_P, _I64, _I64, _P, _P]
+        L.oracle_rmsnorm.argtypes = [_P, _P, ctypes.c_float, _I64, _I64, _P]
+        L.oracle_rmsnorm_quantize.argtypes = [_P, _P, ctypes.c_float, _I64, _I64, _P, _P]
+        L.oracle_linear_rmsnorm.argtypes = [_P, _P, ctypes.c_float, _P, _P, _I64, _I64, _I64,
+                                            _I64, _P]
         L.oracle_linear_bias.argtypes = [_P, _P, _P, _I64, _P, _I64, _I64, _I64, _P]
         L.oracle_ternarize_absmean.argtypes = [_P, _I64, _I64, ctypes.c_int, _P, _P]
         L.oracle_linear_f32.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P]
@@ -47,7 +51,8 @@ def lib():
         L.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
         L.oracle_f32_to_bf16.restype = ctypes.c_uint16
         for name in ("oracle_pack", "oracle_unpack", "oracle_quantize", "oracle_quantize_f32",
-                     "oracle_ternarize_absmean", "oracle_linear_bias",
+                     "oracle_ternarize_absmean", "oracle_linear_bias", "oracle_rmsnorm",
+                     "oracle_rmsnorm_quantize", "oracle_linear_rmsnorm",
                      "oracle_linear_f32",
                      "oracle_acc", "oracle_epilogue", "oracle_gemm",
                      "oracle_linear", "oracle_linear_threads",
@@ -147,6 +152,40 @@ def linear_bias(x_bf16_bits, packed, scale_wt, bias_bf16_bits):
     out = np.empty((M, N), np.uint16)
     _check(lib().oracle_linear_bias(_ptr(x), _ptr(packed), _ptr(sw), sw.size, _ptr(b), M, N, K,
                                     _ptr(out)), "linear_bias")
+    return out
+
+
+def rmsnorm(x_bf16_bits, g_bf16_bits, eps):
+    """bf16 bits [M, K], norm weight bf16 bits [K] -> z bf16 bits [M, K]."""
+    x = _c(x_bf16_bits, np.uint16)
+    g = _c(g_bf16_bits, np.uint16)
+    M, K = x.shape
+    z = np.empty((M, K), np.uint16)
+    _check(lib().oracle_rmsnorm(_ptr(x), _ptr(g), float(eps), M, K, _ptr(z)), "rmsnorm")
+    return z
+
+
+def rmsnorm_quantize(x_bf16_bits, g_bf16_bits, eps):
+    x = _c(x_bf16_bits, np.uint16)
+    g = _c(g_bf16_bits, np.uint16)
+    M, K = x.shape
+    q = np.empty((M, K), np.int8)
+    s = np.empty((M,), np.uint16)
+    _check(lib().oracle_rmsnorm_quantize(_ptr(x), _ptr(g), float(eps), M, K, _ptr(q), _ptr(s)),
+           "rmsnorm_quantize")
+    return q, s
+
+
+def linear_rmsnorm(x_bf16_bits, g_bf16_bits, eps, packed, scale_wt):
+    x = _c(x_bf16_bits, np.uint16)
+    g = _c(g_bf16_bits, np.uint16)
+    packed = _c(packed, np.uint8)
+    sw = _c(scale_wt, np.float32)
+    M, K = x.shape
+    N = packed.shape[0]
+    out = np.empty((M, N), np.uint16)
+    _check(lib().oracle_linear_rmsnorm(_ptr(x), _ptr(g), float(eps), _ptr(packed), _ptr(sw),
+                                       sw.size, M, N, K, _ptr(out)), "linear_rmsnorm")
     return out
 
 

@@ -430,4 +430,56 @@ int oracle_ternarize_absmean(const float* w, int64_t N, int64_t K, int per_row, 
   return OK;
 }
 
+// ------------------------------------------------------------------------
+// RMSNorm before the quantiser (BitLinearKernel on the bitnet-cpu page runs
+// the module's rms_norm on its input first). The page does not spell the norm
+// out; the reading is the usual RMSNorm in fp32 with its weight g applied to
+// the result cast back to bf16:
+//   var = mean(x^2), r = 1 / sqrt(var + eps), y = bf16(x * r), z = bf16(g * y),
+// then quantize_activation(z). The sum of squares is exact (each x^2 of a bf16
+// x is exact in fp32, summed as an integer in units of 2^-64, as for the
+// absmean), var = float(double(sum) / K * 2^-64), sqrt and 1/. are IEEE.
+// ERR_VALUE when some |x| >= 2^23 (x^2 would leave the exact range).
+
+int oracle_rmsnorm(const uint16_t* x, const uint16_t* g, float eps, int64_t M, int64_t K,
+                   uint16_t* z) {
+  if (M < 0 || K <= 0) return ERR_SHAPE;
+  std::fesetround(FE_TONEAREST);
+  for (int64_t m = 0; m < M; ++m) {
+    const uint16_t* row = x + m * K;
+    u128 s = 0;
+    for (int64_t k = 0; k < K; ++k) {
+      const float v = bf16_bits_to_float(row[k]);
+      if (!(std::fabs(v) < 8388608.0f)) return ERR_VALUE;  // 2^23, also NaN
+      u128 a;
+      if (!abs_fixed(v * v, &a)) return ERR_VALUE;
+      s += a;
+    }
+    const float var = mean_of(s, K);
+    const float r = 1.0f / std::sqrt(var + eps);
+    for (int64_t k = 0; k < K; ++k) {
+      const float y = bf16_bits_to_float(float_to_bf16_bits_rne(bf16_bits_to_float(row[k]) * r));
+      z[m * K + k] = float_to_bf16_bits_rne(bf16_bits_to_float(g[k]) * y);
+    }
+  }
+  return OK;
+}
+
+int oracle_rmsnorm_quantize(const uint16_t* x, const uint16_t* g, float eps, int64_t M,
+                            int64_t K, int8_t* q, uint16_t* scale) {
+  std::vector<uint16_t> z(static_cast<size_t>(M) * static_cast<size_t>(K));
+  int st = oracle_rmsnorm(x, g, eps, M, K, z.data());
+  if (st != OK) return st;
+  return oracle_quantize(z.data(), M, K, q, scale);
+}
+
+int oracle_linear_rmsnorm(const uint16_t* x, const uint16_t* g, float eps,
+                          const uint8_t* packed, const float* scale_wt, int64_t scale_wt_len,
+                          int64_t M, int64_t N, int64_t K, uint16_t* out) {
+  std::vector<uint16_t> z(static_cast<size_t>(M) * static_cast<size_t>(K));
+  int st = oracle_rmsnorm(x, g, eps, M, K, z.data());
+  if (st != OK) return st;
+  return oracle_linear(z.data(), packed, scale_wt, scale_wt_len, M, N, K, out);
+}
+
 }  // extern "C"

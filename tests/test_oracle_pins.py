@@ -424,3 +424,58 @@ def test_linear_bias_matches_torch_bf16_addition():
     b = torch.from_numpy(bias.view(np.int16).copy()).view(torch.bfloat16)
     ref = (y + b).view(torch.int16).numpy().view(np.uint16)
     assert np.array_equal(oracle.linear_bias(x, p, sw, bias), ref)
+
+
+# ------------------------------------------------------ RMSNorm -> quantise
+
+def test_rmsnorm_worked_example():
+    """x = [3, 4], g = 1, eps = 0: mean(x^2) = 12.5, r = 1/sqrt(12.5) =
+    0.28284271; x * r = 0.84852814, 1.13137085 -> bf16 0.84765625, 1.1328125;
+    the quantiser's s = 1.1328125 / 127, so q = [round(95.03), 127]."""
+    x = f32_to_bf16_bits_np(np.array([[3.0, 4.0]], np.float32))
+    g = f32_to_bf16_bits_np(np.array([1.0, 1.0], np.float32))
+    z = (oracle.rmsnorm(x, g, 0.0).astype(np.uint32) << 16).view(np.float32)
+    assert z.tolist() == [[0.84765625, 1.1328125]]
+    q, s = oracle.rmsnorm_quantize(x, g, 0.0)
+    assert q.tolist() == [[95, 127]]
+    assert s[0] == f32_to_bf16_bits_np(np.float32(1.1328125) / np.float32(127.0))
+
+
+def test_rmsnorm_invariant_under_power_of_two_scaling():
+    """With eps = 0 every step scales exactly by powers of two, so x * 2^k
+    gives the same normalised row, bit for bit."""
+    x = synth.act_bf16(synth.key(89, 0, synth.T_ACT), 6, 512)
+    g = f32_to_bf16_bits_np(np.random.default_rng(2).uniform(0.5, 1.5, 512).astype(np.float32))
+    xf = (x.astype(np.uint32) << 16).view(np.float32)
+    z0 = oracle.rmsnorm(x, g, 0.0)
+    for k in (-3, 5):
+        xs = f32_to_bf16_bits_np(xf * np.float32(2.0 ** k))
+        assert np.array_equal(oracle.rmsnorm(xs, g, 0.0), z0)
+
+
+def test_rmsnorm_matches_torch_fp32_evaluation():
+    """The usual RMSNorm in fp32 (as the transformers BitNet module writes
+    it), on rows where torch's fp32 mean of squares is exact (small integer
+    values, K a power of two)."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(8)
+    xf = rng.integers(-8, 9, size=(17, 64)).astype(np.float32)
+    xf[3] = 0.0
+    gf = rng.uniform(0.25, 2.0, 64).astype(np.float32)
+    x = f32_to_bf16_bits_np(xf)
+    g = f32_to_bf16_bits_np(gf)
+    eps = 1e-5
+    xt = torch.from_numpy(x.view(np.int16).copy()).view(torch.bfloat16)
+    gt = torch.from_numpy(g.view(np.int16).copy()).view(torch.bfloat16)
+    h = xt.float()
+    var = h.pow(2).mean(-1, keepdim=True)
+    y = (h * torch.rsqrt(var + eps)).to(torch.bfloat16)
+    ref = (gt * y).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.rmsnorm(x, g, eps), ref)
+
+
+def test_rmsnorm_zero_weight_gives_zero_codes():
+    x = synth.act_bf16(synth.key(89, 1, synth.T_ACT), 3, 256)
+    g = np.zeros(256, np.uint16)
+    q, _ = oracle.rmsnorm_quantize(x, g, 1e-5)
+    assert not q.any()
