@@ -596,8 +596,10 @@ def extra_rows(bn, dev, pk):
     """The rows beyond the layer itself: absmean ternarisation of a dense
     float32 matrix (11008 x 4096, per row and per tensor; 180 MB read, 45 MB
     written, plus the per-tensor form's second read), the layer on float32
-    activations (decode GEMV at M = 1, bitnet_linear at M = 2048), and the
-    fused bias epilogue (bitnet_linear with and without bias at M = 2048)."""
+    activations (decode GEMV at M = 1, bitnet_linear at M = 2048), the
+    fused bias epilogue (bitnet_linear with and without bias at M = 2048),
+    and RMSNorm before the quantiser (alone at M = 2048; bitnet_linear_rmsnorm
+    at M = 2048 and M = 1, each beside the same call without the norm)."""
     hbm = pk["hbm_gbs"]
     tops_peak = pk["bf16_tflops"] * INT8_OVER_BF16
     flush = torch.empty((2 * L2_BYTES,), dtype=torch.uint8, device=dev)
@@ -654,6 +656,32 @@ def extra_rows(bn, dev, pk):
     ms_bias = timed(lambda: bn.bitnet_linear(xb, wp, sw, out=ol, workspace=ws, bias=bias))
     out["linear_bias_m2048"] = {"M": M, "K": K, "N": N, "ms": ms_bias, "ms_without_bias": ms_plain,
                                 "tops": ops / ms_bias / 1e9, "frac": ops / ms_bias / 1e9 / tops_peak}
+    # RMSNorm before the quantiser: alone (x read, codes written), in front
+    # of the prefill GEMM, and in front of the decode GEMV
+    gn = (1.0 + 0.1 * torch.randn((K,), device=dev, generator=g)).to(torch.bfloat16)
+    xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    sa = torch.empty((M,), dtype=torch.bfloat16, device=dev)
+    ms = timed(lambda: bn.bitnet_rmsnorm_quantize_act(xb, gn, 1e-6, x_q=xq, scale_act=sa))
+    byts = 2 * M * K + 2 * K + M * K + 2 * M
+    out["rmsnorm_quant_m2048"] = {"M": M, "K": K, "ms": ms, "gbs": byts / ms / 1e6,
+                                  "frac_hbm": byts / ms / 1e6 / hbm}
+    wsn = torch.empty((bn.bitnet_linear_rmsnorm_workspace_bytes(M, K),), dtype=torch.uint8,
+                      device=dev)
+    ms = timed(lambda: bn.bitnet_linear_rmsnorm(xb, gn, 1e-6, wp, sw, out=ol, workspace=wsn))
+    out["linear_rmsnorm_m2048"] = {"M": M, "K": K, "N": N, "ms": ms, "ms_without_norm": ms_plain,
+                                   "tops": ops / ms / 1e9, "frac": ops / ms / 1e9 / tops_peak}
+    del xl, ol, xq
+    copies = weight_rotation(wp)
+    xd = torch.randn((1, K), device=dev, generator=g).to(torch.bfloat16)
+    ws1 = torch.empty((bn.bitnet_linear_rmsnorm_workspace_bytes(1, K),), dtype=torch.uint8,
+                      device=dev)
+    ms_norm = time_rotation([lambda c=c: bn.bitnet_linear_rmsnorm(xd, gn, 1e-6, c, sw, out=o1,
+                                                                  workspace=ws1) for c in copies])
+    ms_plain1 = time_rotation([lambda c=c: bn.bitnet_gemv_fused(xd, c, sw, out=o1) for c in copies])
+    byts = N * K // 4 + 2 * K + 2 * N + 4
+    out["linear_rmsnorm_m1"] = {"M": 1, "K": K, "N": N, "ms": ms_norm, "ms_without_norm": ms_plain1,
+                                "gbs": byts / ms_norm / 1e6, "frac_hbm": byts / ms_norm / 1e6 / hbm}
+    del copies
     bn.bitnet_device_status()
     return out
 

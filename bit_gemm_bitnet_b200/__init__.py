@@ -30,7 +30,8 @@ EXPORTS = (
     "bitnet_gemv_fused", "bitnet_linear_workspace_bytes", "bitnet_linear",
     "bitnet_device_status", "bitnet_status_string", "bitnet_gemm_acc_i32",
     "bitnet_gemv_fused_debug", "bitnet_linear_noalloc", "bitnet_gemv_fused_grouped",
-    "bitnet_linear_bias",
+    "bitnet_linear_bias", "bitnet_rmsnorm_quantize_act", "bitnet_linear_rmsnorm_workspace_bytes",
+    "bitnet_linear_rmsnorm",
 )
 
 
@@ -64,6 +65,7 @@ def lib():
                 "`python -m bit_gemm_bitnet_b200.build` (nvcc, sm_100a)")
         L = ctypes.CDLL(LIB_PATH)
         P, I64, SZ, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+        F = ctypes.c_float
         sig = {
             "bitnet_pack_weights": [P, P, I64, I64, P],
             "bitnet_ternarize_absmean": [P, P, P, I64, I64, I, P],
@@ -73,6 +75,8 @@ def lib():
             "bitnet_linear": [P, P, I, P, P, I64, I64, I64, I64, P, SZ, P],
             "bitnet_linear_bias": [P, P, I, P, P, I64, P, I64, I64, I64, P, SZ, P],
             "bitnet_linear_noalloc": [P, P, I, P, P, I64, I64, I64, I64, P],
+            "bitnet_rmsnorm_quantize_act": [P, P, P, P, F, I64, I64, P],
+            "bitnet_linear_rmsnorm": [P, P, P, F, P, P, I64, I64, I64, I64, P, SZ, P],
             "bitnet_gemv_fused_grouped": [P, I64, I64, I, P],
             "bitnet_device_status": [P],
             "bitnet_gemm_acc_i32": [P, P, P, I64, I64, I64, P],
@@ -84,6 +88,8 @@ def lib():
             f.restype = ctypes.c_int
         L.bitnet_linear_workspace_bytes.argtypes = [I64, I64]
         L.bitnet_linear_workspace_bytes.restype = SZ
+        L.bitnet_linear_rmsnorm_workspace_bytes.argtypes = [I64, I64]
+        L.bitnet_linear_rmsnorm_workspace_bytes.restype = SZ
         L.bitnet_status_string.argtypes = [ctypes.c_int]
         L.bitnet_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -318,6 +324,57 @@ def bitnet_linear_noalloc(x, w_packed, scale_wt, out=None):
     _check(lib().bitnet_linear_noalloc(_ptr(out), _ptr(x2), dt, _ptr(w_packed), _ptr(sw),
                                        sw.numel(), M, N, K, _stream(x.device)),
            "bitnet_linear_noalloc")
+    return out.view(*orig[:-1], N)
+
+
+def bitnet_rmsnorm_quantize_act(x, g, eps, x_q=None, scale_act=None):
+    """bf16 [M, K] -> RMSNorm with weight g (bf16 [K]) and epsilon eps, then
+    the per-token quantiser: int8 [M, K] codes, bf16 [M] scales."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(g, torch.bfloat16, "g", 1)
+    M, K = x.shape
+    if g.numel() != K:
+        raise ValueError(f"g has {g.numel()} elements, expected K={K}")
+    if x_q is None:
+        x_q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if scale_act is None:
+        scale_act = torch.empty((M,), dtype=torch.bfloat16, device=x.device)
+    _check(lib().bitnet_rmsnorm_quantize_act(_ptr(x_q), _ptr(scale_act), _ptr(x), _ptr(g),
+                                             float(eps), M, K, _stream(x.device)),
+           "bitnet_rmsnorm_quantize_act")
+    return x_q, scale_act
+
+
+def bitnet_linear_rmsnorm_workspace_bytes(M, K):
+    return int(lib().bitnet_linear_rmsnorm_workspace_bytes(M, K))
+
+
+def bitnet_linear_rmsnorm(x, g, eps, w_packed, scale_wt, out=None, workspace=None):
+    """RMSNorm (weight g, epsilon eps), the quantiser and the ternary GEMM:
+    bf16 [..., K] -> bf16 [..., N]."""
+    orig = x.shape
+    K = orig[-1]
+    x2 = x.reshape(-1, K)
+    _need(x2, torch.bfloat16, "x", 2)
+    _need(g, torch.bfloat16, "g", 1)
+    _need(w_packed, torch.uint8, "w_packed", 2)
+    M = x2.shape[0]
+    N = w_packed.shape[0]
+    if w_packed.shape[1] * 4 != K:
+        raise ValueError(f"w_packed {tuple(w_packed.shape)} does not match K={K}")
+    if g.numel() != K:
+        raise ValueError(f"g has {g.numel()} elements, expected K={K}")
+    sw = _scale_wt(scale_wt, N, x.device)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    need = bitnet_linear_rmsnorm_workspace_bytes(M, K)
+    if need and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
+    _check(lib().bitnet_linear_rmsnorm(_ptr(out), _ptr(x2), _ptr(g), float(eps), _ptr(w_packed),
+                                       _ptr(sw), sw.numel(), M, N, K,
+                                       _ptr(workspace) if need else None, need,
+                                       _stream(x.device)),
+           "bitnet_linear_rmsnorm")
     return out.view(*orig[:-1], N)
 
 

@@ -2,6 +2,7 @@
 //
 // Host code only validates arguments, picks a kernel variant and launches it
 // on the caller's stream; all arithmetic runs in the kernels included below.
+#include <cmath>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -12,6 +13,7 @@
 #include "gemm_skq.cuh"
 #include "gemm_ts.cuh"
 #include "ternarize.cuh"
+#include "rmsnorm.cuh"
 #include "gemv.cuh"
 #include "gemv_grouped.cuh"
 #include "pack_quant.cuh"
@@ -1037,6 +1039,86 @@ bitnet_status bitnet_linear_noalloc(uint16_t* out, const void* x, bitnet_dtype d
                        kNoAllocScratchBytes, stream);
 }
 
+// ------------------------------------------------ RMSNorm -> quantise
+
+static bitnet_status run_rmsnorm_quant(int8_t* xq, uint16_t* sa, int32_t* rowsum,
+                                       const uint16_t* x, const uint16_t* g, float eps,
+                                       int64_t M, int64_t K, int mode, cudaStream_t st) {
+  if (M == 0) return BITNET_OK;
+  if (M > INT32_MAX) return BITNET_ERR_SHAPE;
+  const dim3 grid(static_cast<unsigned>(M)), block(kTernThreads);
+  const int k = static_cast<int>(K);
+  if (mode == kRmsPerm)
+    return launch_pdl(rmsnorm_quant_kernel<kRmsPerm>, grid, block, 0, st, xq, sa, rowsum, x, g,
+                      eps, k);
+  if (mode == kRmsZ)
+    return launch_pdl(rmsnorm_quant_kernel<kRmsZ>, grid, block, 0, st, xq, sa, rowsum, x, g, eps,
+                      k);
+  return launch_pdl(rmsnorm_quant_kernel<kRmsCodes>, grid, block, 0, st, xq, sa, rowsum, x, g,
+                    eps, k);
+}
+
+bitnet_status bitnet_rmsnorm_quantize_act(int8_t* x_q, uint16_t* scale_act, const uint16_t* x,
+                                          const uint16_t* g, float eps, int64_t M, int64_t K,
+                                          void* stream) {
+  if (M < 0 || K <= 0 || K % 32 != 0 || K > INT32_MAX) return BITNET_ERR_SHAPE;
+  if (!(eps > 0.0f) || !std::isfinite(eps)) return BITNET_ERR_VALUE;
+  if (M == 0) return BITNET_OK;
+  if (x_q == nullptr || scale_act == nullptr || x == nullptr || g == nullptr)
+    return BITNET_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(g, 16) || !aligned(x_q, 16) || !aligned(scale_act, 2))
+    return BITNET_ERR_ALIGN;
+  return run_rmsnorm_quant(x_q, scale_act, nullptr, x, g, eps, M, K, kRmsCodes,
+                           as_stream(stream));
+}
+
+size_t bitnet_linear_rmsnorm_workspace_bytes(int64_t M, int64_t K) {
+  if (M <= 0 || K <= 0) return 0;
+  if (linear_uses_gemv(M, K)) return align256(static_cast<size_t>(M) * static_cast<size_t>(K) * 2);
+  return align256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
+         align256(static_cast<size_t>(M) * 2) + align256(static_cast<size_t>(M) * 4);
+}
+
+bitnet_status bitnet_linear_rmsnorm(uint16_t* out, const uint16_t* x, const uint16_t* g,
+                                    float eps, const uint8_t* w_packed, const float* scale_wt,
+                                    int64_t scale_wt_len, int64_t M, int64_t N, int64_t K,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  bitnet_status s = check_compute_shape(M, N, K);
+  if (s != BITNET_OK) return s;
+  if (!(eps > 0.0f) || !std::isfinite(eps)) return BITNET_ERR_VALUE;
+  if (M == 0 || N == 0) return BITNET_OK;
+  const size_t need = bitnet_linear_rmsnorm_workspace_bytes(M, K);
+  if (workspace == nullptr || workspace_bytes < need) return BITNET_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return BITNET_ERR_ALIGN;
+  if (out == nullptr || x == nullptr || g == nullptr || w_packed == nullptr)
+    return BITNET_ERR_NULL;
+  s = check_scale_wt(scale_wt, scale_wt_len, N);
+  if (s != BITNET_OK) return s;
+  if (!aligned(out, 16) || !aligned(x, 16) || !aligned(g, 16) || !aligned(w_packed, 16))
+    return BITNET_ERR_ALIGN;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = as_stream(stream);
+  if (linear_uses_gemv(M, K)) {
+    // few rows: the normalised bf16 rows, then the fused GEMV quantises them
+    int8_t* z = reinterpret_cast<int8_t*>(ws);
+    s = run_rmsnorm_quant(z, nullptr, nullptr, x, g, eps, M, K, kRmsZ, st);
+    if (s != BITNET_OK) return s;
+    return gemv_fused_impl(out, z, BITNET_BF16, w_packed, scale_wt, scale_wt_len, nullptr, M, N,
+                           K, stream);
+  }
+  int8_t* xq = reinterpret_cast<int8_t*>(ws);
+  uint16_t* sa = reinterpret_cast<uint16_t*>(ws + align256(static_cast<size_t>(M) * K));
+  int32_t* rowsum = reinterpret_cast<int32_t*>(ws + align256(static_cast<size_t>(M) * K) +
+                                               align256(static_cast<size_t>(M) * 2));
+  const bool tc = gemm_tc_ok(xq, w_packed, K);
+  s = run_rmsnorm_quant(xq, sa, rowsum, x, g, eps, M, K, tc ? kRmsPerm : kRmsCodes, st);
+  if (s != BITNET_OK) return s;
+  if (tc)
+    return run_gemm(out, false, xq, w_packed, sa, scale_wt, scale_wt_len, M, N, K, st, true,
+                    rowsum);
+  return run_gemm(out, false, xq, w_packed, sa, scale_wt, scale_wt_len, M, N, K, st);
+}
+
 bitnet_status bitnet_device_status(void* stream) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return BITNET_ERR_CUDA;
   unsigned v = 0;
@@ -1045,7 +1127,7 @@ bitnet_status bitnet_device_status(void* stream) {
     const unsigned zero = 0;
     if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero) != cudaSuccess)
       return BITNET_ERR_CUDA;
-    return BITNET_ERR_TIMEOUT;
+    return (v & kDevErrTimeout) ? BITNET_ERR_TIMEOUT : BITNET_ERR_VALUE;
   }
   return BITNET_OK;
 }

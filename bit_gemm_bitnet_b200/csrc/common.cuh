@@ -14,6 +14,7 @@ namespace bitnet {
 
 // Error bits of the device status word (read by bitnet_device_status).
 constexpr unsigned kDevErrTimeout = 1u;
+constexpr unsigned kDevErrValue = 2u;  // an input outside a kernel's exact range
 
 // Bounded waits give up after this many nanoseconds of global time.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s

@@ -198,6 +198,42 @@ bitnet_status bitnet_linear_bias(uint16_t* out, const void* x, bitnet_dtype dt,
                                  int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
                                  void* stream);
 
+/* RMSNorm fused with the per-token quantiser (BitLinearKernel on the
+ * bitnet-cpu page applies the module's rms_norm to its input first). The norm
+ * is the usual fp32 RMSNorm with its weight applied after the cast back to
+ * bf16, per row:
+ *   r = 1 / sqrt(mean(x^2) + eps)   (the sum of squares exact, sqrt and /
+ *                                    IEEE fp32)
+ *   z = bf16(g * bf16(x * r)),  then quantize_activation(z)
+ *   x_q, scale_act  out, as bitnet_quantize_act
+ *   x               in,  bf16 [M, K], |x| < 2^23 (else bitnet_device_status
+ *                        reports BITNET_ERR_VALUE)
+ *   g               in,  bf16 [K], the norm's weight
+ *   eps             the norm's epsilon: finite and > 0 (else BITNET_ERR_VALUE;
+ *                   a zero row would otherwise divide by zero)
+ * K % 32 == 0; x, g and x_q 16-byte aligned. */
+bitnet_status bitnet_rmsnorm_quantize_act(int8_t* x_q, uint16_t* scale_act, const uint16_t* x,
+                                          const uint16_t* g, float eps, int64_t M, int64_t K,
+                                          void* stream);
+
+/* Workspace of bitnet_linear_rmsnorm for (M, K). Where bitnet_linear takes
+ * the fused GEMV (M < 16 and the GEMV's fit rule): the normalised bf16 [M, K]
+ * rows, which the GEMV then quantises. Otherwise the int8 [M, K] codes, bf16
+ * [M] scales and int32 [M] code sums. Each part 256-byte aligned; 0 for
+ * M == 0. */
+size_t bitnet_linear_rmsnorm_workspace_bytes(int64_t M, int64_t K);
+
+/* RMSNorm, quantiser and the layer in one call, on the caller's stream:
+ * the norm's kernel writes its result into `workspace` (the quantised rows,
+ * or for few rows the bf16 normalised rows), then the kernels of
+ * bitnet_linear run on it; the result equals bitnet_linear applied to
+ * bf16(g * bf16(x * r)). Arguments as bitnet_rmsnorm_quantize_act and
+ * bitnet_linear; x is bf16, workspace 256-byte aligned. */
+bitnet_status bitnet_linear_rmsnorm(uint16_t* out, const uint16_t* x, const uint16_t* g,
+                                    float eps, const uint8_t* w_packed, const float* scale_wt,
+                                    int64_t scale_wt_len, int64_t M, int64_t N, int64_t K,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* bitnet_linear without a caller workspace, for callers that cannot allocate
  * device memory: code running while a stream is being captured into a CUDA
  * graph (cudaMalloc is not allowed there), code inside a framework that owns

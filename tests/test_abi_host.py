@@ -95,9 +95,41 @@ ODD = P(0x10008)
      bn.ERR_ALIGN),
     (lambda L: L.bitnet_gemv_fused_debug(FAKE, FAKE, None, FAKE, 0, FAKE, 1, 4, 64, None),
      bn.ERR_NULL),
+    (lambda L: L.bitnet_rmsnorm_quantize_act(FAKE, FAKE, FAKE, FAKE, 1e-5, 4, 48, None),
+     bn.ERR_SHAPE),
+    (lambda L: L.bitnet_rmsnorm_quantize_act(FAKE, FAKE, FAKE, FAKE, 0.0, 4, 64, None),
+     bn.ERR_VALUE),
+    (lambda L: L.bitnet_rmsnorm_quantize_act(FAKE, FAKE, FAKE, FAKE, float("nan"), 4, 64, None),
+     bn.ERR_VALUE),
+    (lambda L: L.bitnet_rmsnorm_quantize_act(FAKE, FAKE, FAKE, FAKE, float("inf"), 4, 64, None),
+     bn.ERR_VALUE),
+    (lambda L: L.bitnet_rmsnorm_quantize_act(FAKE, FAKE, FAKE, None, 1e-5, 4, 64, None),
+     bn.ERR_NULL),
+    (lambda L: L.bitnet_rmsnorm_quantize_act(FAKE, FAKE, P(0x10008), FAKE, 1e-5, 4, 64, None),
+     bn.ERR_ALIGN),
+    (lambda L: L.bitnet_linear_rmsnorm(FAKE, FAKE, FAKE, -1.0, FAKE, FAKE, 1, 4, 4, 64, FAKE,
+                                       1 << 20, None), bn.ERR_VALUE),
+    (lambda L: L.bitnet_linear_rmsnorm(FAKE, FAKE, FAKE, 1e-5, FAKE, FAKE, 1, 4, 4, 64, FAKE, 500,
+                                       None), bn.ERR_WORKSPACE),
+    (lambda L: L.bitnet_linear_rmsnorm(FAKE, FAKE, FAKE, 1e-5, FAKE, FAKE, 1, 32, 4, 64, FAKE,
+                                       2559, None), bn.ERR_WORKSPACE),
+    (lambda L: L.bitnet_linear_rmsnorm(FAKE, FAKE, None, 1e-5, FAKE, FAKE, 1, 4, 4, 64, FAKE,
+                                       1 << 20, None), bn.ERR_NULL),
+    (lambda L: L.bitnet_linear_rmsnorm(FAKE, FAKE, FAKE, 1e-5, FAKE, FAKE, 1, 4, 4, 96,
+                                       P(0x10080), 1 << 20, None), bn.ERR_ALIGN),
 ])
 def test_validation_rejects_before_launch(call, expect):
     assert call(bn.lib()) == expect
+
+
+def test_rmsnorm_workspace_size():
+    """Rows the fused GEMV takes: the bf16 normalised rows. Otherwise int8
+    codes, bf16 scales and int32 code sums. Each part rounded up to 256 bytes."""
+    L = bn.lib()
+    assert L.bitnet_linear_rmsnorm_workspace_bytes(3, 64) == 512
+    assert L.bitnet_linear_rmsnorm_workspace_bytes(32, 64) == 2048 + 256 + 256
+    assert L.bitnet_linear_rmsnorm_workspace_bytes(300, 2560) == 768000 + 768 + 1280
+    assert L.bitnet_linear_rmsnorm_workspace_bytes(0, 64) == 0
 
 
 def test_noop_sizes_return_ok_without_work():

@@ -438,3 +438,78 @@ def test_linear_bias_matches_oracle(M, K, N):
     # without the bias the result is bitnet_linear's
     plain = bn.bitnet_linear(to_dev(x, torch.bfloat16), to_dev(p), to_dev(sw))
     assert_bf16_close(bf16_bits(plain)[rows], oracle.linear(x[rows], p, sw))
+
+
+# ------------------------------------------------------ RMSNorm -> quantise
+
+RMS_CASES = [(1, 64), (2, 96), (7, 2560), (64, 4096), (300, 2560), (5, 11008), (1, 27648)]
+
+
+def norm_weight(K, seed):
+    """bf16 norm weights around 1 with a zero, a negative and a 2 in front."""
+    g = (1.0 + 0.25 * np.random.default_rng(seed).standard_normal(K)).astype(np.float32)
+    g[:3] = [0.0, -1.0, 2.0]
+    return f32_to_bf16_bits(g)
+
+
+def norm_inputs(M, K, seed):
+    """Activations with a zero row (r = 1/sqrt(eps)), a row scaled by 2^12
+    (large squares) and a row scaled by 2^-70 (squares below 2^-64)."""
+    x = acts(95, seed, M, K)
+    xf = (x.astype(np.uint32) << 16).view(np.float32)
+    if M > 2:
+        x[2] = 0
+    if M > 3:
+        x[3] = f32_to_bf16_bits(xf[3] * np.float32(2.0 ** 12))
+    if M > 4:
+        x[4] = f32_to_bf16_bits(xf[4] * np.float32(2.0 ** -70))
+    return x
+
+
+@pytest.mark.parametrize("eps", [1e-5, 1e-6])
+@pytest.mark.parametrize("M,K", RMS_CASES)
+def test_rmsnorm_quantize_bitexact(M, K, eps):
+    x = norm_inputs(M, K, M + K)
+    g = norm_weight(K, M * 3 + K)
+    q_ref, s_ref = oracle.rmsnorm_quantize(x, g, eps)
+    q, s = bn.bitnet_rmsnorm_quantize_act(to_dev(x, torch.bfloat16), to_dev(g, torch.bfloat16),
+                                          eps)
+    bn.bitnet_device_status()
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(bf16_bits(s), s_ref)
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 2560, 640), (2, 96, 40), (12, 2112, 77), (64, 4096, 300),
+                                   (16, 11008, 256), (300, 2560, 520), (2048, 2560, 256)])
+def test_linear_rmsnorm_matches_oracle(M, K, N):
+    """Norm, quantiser and GEMM in one call: the tensor-core GEMMs (permuted
+    workspace plus code sums) and the SIMT path (K % 64 != 0)."""
+    x = norm_inputs(M, K, M * 5 + K)
+    g = norm_weight(K, N + K)
+    w = weights(96, N + K, N, K)
+    p = oracle.pack(w)
+    sw = synth.uniform_f32(synth.key(96, N, 3), N, 0.01, 0.1)
+    got = bn.bitnet_linear_rmsnorm(to_dev(x, torch.bfloat16), to_dev(g, torch.bfloat16), 1e-6,
+                                   to_dev(p), to_dev(sw))
+    bn.bitnet_device_status()
+    rows = np.arange(M) if M <= 64 else np.unique(np.r_[np.random.default_rng(M).choice(M, 40, replace=False), 0, 2, 3, 4, M - 1])
+    ref = oracle.linear_rmsnorm(x[rows], g, 1e-6, p, sw)
+    assert_bf16_close(bf16_bits(got)[rows], ref)
+
+
+def test_rmsnorm_flags_out_of_range_input():
+    """|x| >= 2^23 (whose square the exact sum does not take) and NaN are
+    reported by bitnet_device_status; the flag is cleared after it is read."""
+    K = 256
+    g = to_dev(norm_weight(K, 1), torch.bfloat16)
+    for bad in (2.0 ** 24, float("nan")):
+        x = torch.ones((3, K), dtype=torch.bfloat16, device="cuda")
+        x[1, 7] = bad
+        bn.bitnet_rmsnorm_quantize_act(x, g, 1e-5)
+        with pytest.raises(bn.BitnetValueError):
+            bn.bitnet_device_status()
+        bn.bitnet_device_status()
+    with pytest.raises(bn.BitnetValueError):
+        bn.bitnet_rmsnorm_quantize_act(x, g, 0.0)
+    with pytest.raises(ValueError):
+        bn.bitnet_rmsnorm_quantize_act(x, g[:128], 1e-5)
