@@ -59,7 +59,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--branches", type=int, default=16,
                     help="graph branches for the independent calls of a step")
-    ap.add_argument("--case", choices=("lm_head", "prefill", "decode_once", "midbatch", "gemv_m15"),
+    ap.add_argument("--case", choices=("lm_head", "prefill", "decode_once", "midbatch", "gemv_m15",
+                                       "rmsnorm"),
                     help="profiling aid: run one small case a few times and exit "
                          "(no JSON line); see profiles/ for the ncu commands")
     return ap.parse_args()
@@ -416,6 +417,32 @@ def lm_head_alone(bn, d, dev, reps=20):
 
 # ---------------------------------------------------------------- prefill
 
+def time_flushed(fn, flush, reps=5, graph=True):
+    """Median device ms of one fn() call with L2 flushed before each
+    repetition. With graph=True the call is captured once in a CUDA graph and
+    replayed, so the host's own cost of issuing it (which can outlast the
+    flush) does not fall between the events."""
+    run = fn
+    if graph:
+        fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        run = g.replay
+    ts = []
+    for r in range(reps + 2):
+        flush.fill_(r & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run()
+        e1.record()
+        torch.cuda.synchronize()
+        if r >= 2:
+            ts.append(e0.elapsed_time(e1))
+    return statistics.median(ts)
+
+
 def prefill(bn, dev, pk, reps=5):
     """The prefill workload: M in {2048, 8192} x four FFN shapes through
     bitnet_linear (per-token quantisation + tensor-core GEMM, bf16 out), each
@@ -425,17 +452,7 @@ def prefill(bn, dev, pk, reps=5):
     peak = pk["bf16_tflops"] * INT8_OVER_BF16
 
     def timed(fn):
-        ts = []
-        for r in range(reps + 2):
-            flush.fill_(r & 0xFF)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            fn()
-            e1.record()
-            torch.cuda.synchronize()
-            if r >= 2:
-                ts.append(e0.elapsed_time(e1))
-        return statistics.median(ts)
+        return time_flushed(fn, flush, reps)
 
     Mmax = max(W.PREFILL_M)
     cases, tot_ops, tot_ms, tot_gemm_ms = [], 0.0, 0.0, 0.0
@@ -604,18 +621,8 @@ def extra_rows(bn, dev, pk):
     tops_peak = pk["bf16_tflops"] * INT8_OVER_BF16
     flush = torch.empty((2 * L2_BYTES,), dtype=torch.uint8, device=dev)
 
-    def timed(fn, reps=5):
-        ts = []
-        for r in range(reps + 2):
-            flush.fill_(r & 0xFF)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            fn()
-            e1.record()
-            torch.cuda.synchronize()
-            if r >= 2:
-                ts.append(e0.elapsed_time(e1))
-        return statistics.median(ts)
+    def timed(fn, graph=True):
+        return time_flushed(fn, flush, 5, graph)
 
     out = {}
     N, K = 11008, 4096
@@ -625,7 +632,8 @@ def extra_rows(bn, dev, pk):
     wt = torch.empty((N, K), dtype=torch.int8, device=dev)
     for per_row, name in ((True, "ternarize_per_row"), (False, "ternarize_per_tensor")):
         sc = torch.empty((N if per_row else 1,), dtype=torch.float32, device=dev)
-        ms = timed(lambda: bn.bitnet_ternarize_absmean(w, per_row=per_row, w_t=wt, scale_wt=sc))
+        ms = timed(lambda: bn.bitnet_ternarize_absmean(w, per_row=per_row, w_t=wt, scale_wt=sc),
+                   graph=False)  # the call synchronises for its value check
         byts = N * K * 4 * (1 if per_row else 2) + N * K + 4 * sc.numel()
         out[name] = {"N": N, "K": K, "ms": ms, "gbs": byts / ms / 1e6,
                      "frac_hbm": byts / ms / 1e6 / hbm,
@@ -744,6 +752,16 @@ def run_case(bn, dev, case, reps=3):
         else:
             for r in range(reps):
                 bn.bitnet_gemv_fused(xd, copies[r % len(copies)], sw, out=out)
+    elif case == "rmsnorm":
+        # RMSNorm + quantiser over M = 2048 rows of K = 4096 (16.8 MB in)
+        M, K = 2048, 4096
+        x = synth.act_bf16(synth.key(W.W_PREFILL, M, synth.T_ACT, K), M, K)
+        xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+        g = torch.ones((K,), dtype=torch.bfloat16, device=dev)
+        xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+        sa = torch.empty((M,), dtype=torch.bfloat16, device=dev)
+        for _ in range(reps):
+            bn.bitnet_rmsnorm_quantize_act(xd, g, 1e-6, x_q=xq, scale_act=sa)
     elif case == "lm_head":
         _, K, N = W.DECODE_2B_LM_HEAD
         w = synth.ternary(synth.key(W.W_DECODE_2B, W.DECODE_2B_LAYERS, synth.T_WEIGHT, 7), N, K)

@@ -1048,6 +1048,21 @@ static bitnet_status run_rmsnorm_quant(int8_t* xq, uint16_t* sa, int32_t* rowsum
   if (M > INT32_MAX) return BITNET_ERR_SHAPE;
   const dim3 grid(static_cast<unsigned>(M)), block(kTernThreads);
   const int k = static_cast<int>(K);
+  const int64_t per_thread = (K / 16 + kTernThreads - 1) / kTernThreads;  // 16-element groups
+  if (per_thread <= 4) {
+#define BITNET_RMS_REG(MODE, NG)                                                                  \
+  return launch_pdl(rmsnorm_quant_reg_kernel<MODE, NG>, grid, block, 0, st, xq, sa, rowsum, x, g, \
+                    eps, k)
+#define BITNET_RMS_REG_NG(MODE)       \
+  if (per_thread <= 1) BITNET_RMS_REG(MODE, 1); \
+  if (per_thread <= 2) BITNET_RMS_REG(MODE, 2); \
+  BITNET_RMS_REG(MODE, 4)
+    if (mode == kRmsPerm) { BITNET_RMS_REG_NG(kRmsPerm); }
+    if (mode == kRmsZ) { BITNET_RMS_REG_NG(kRmsZ); }
+    BITNET_RMS_REG_NG(kRmsCodes);
+#undef BITNET_RMS_REG_NG
+#undef BITNET_RMS_REG
+  }
   if (mode == kRmsPerm)
     return launch_pdl(rmsnorm_quant_kernel<kRmsPerm>, grid, block, 0, st, xq, sa, rowsum, x, g,
                       eps, k);

@@ -18,6 +18,54 @@ __device__ __forceinline__ float rms_z(uint32_t xbits16, uint32_t gbits16, float
   return bf16_bits_to_f32(f32_to_bf16_bits(__fmul_rn(bf16_bits_to_f32(gbits16), y)));
 }
 
+// Sum over the 2*NW bf16 values packed in `w` of trunc(x^2 * 2^64), exact
+// (the definition the slow path below spells out). A bf16 x with exponent
+// field b >= 1 is m * 2^(b - 134), m in [128, 255], so trunc(x^2 * 2^64) is
+// the integer m^2 * 2^(2b - 204) when b >= 102, and 0 when b < 95. When
+// every value is in one of those two classes and the first spans at most 21
+// binades below the largest exponent bmax, the terms are summed in 64 bits
+// in units of 2^(2 bmax - 246) (each below 2^58) and the sum shifted into
+// place once. Otherwise each term goes through abs_fixed. `ok` is cleared
+// for |x| >= 2^23 and non-finite x.
+template <int NW>
+__device__ __forceinline__ u128 sumsq_fixed(const uint32_t (&w)[NW], bool* ok) {
+  static_assert(NW <= 32, "64 terms below 2^58 each fit in 64 bits");
+  uint32_t bmax = 0;
+#pragma unroll
+  for (int i = 0; i < NW; ++i) bmax = max(bmax, max((w[i] >> 7) & 0xFFu, (w[i] >> 23) & 0xFFu));
+  if (bmax >= 150u) {  // 2^23 and above, Inf, NaN
+    *ok = false;
+    return 0;
+  }
+  bool fast = true;
+  uint64_t acc = 0;
+#pragma unroll
+  for (int i = 0; i < 2 * NW; ++i) {
+    const uint32_t h = (w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
+    const uint32_t b = (h >> 7) & 0xFFu;
+    if (b >= 95u) {
+      fast &= b >= 102u && b + 21u >= bmax;
+      const uint32_t m = (h & 0x7Fu) | 0x80u;
+      const int sh = max(2 * (static_cast<int>(b) - static_cast<int>(bmax)) + 42, 0);
+      acc += static_cast<uint64_t>(m * m) << sh;
+    }
+  }
+  if (fast) {
+    if (acc == 0) return 0;
+    const int e = 2 * static_cast<int>(bmax) - 246;  // bmax >= 102 here
+    return e >= 0 ? static_cast<u128>(acc) << e : static_cast<u128>(acc >> -e);  // exact: an integer
+  }
+  u128 s = 0;
+#pragma unroll
+  for (int i = 0; i < 2 * NW; ++i) {
+    const float f = bf16_bits_to_f32((w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
+    u128 a = 0;
+    abs_fixed(__fmul_rn(f, f), &a);
+    s += a;
+  }
+  return s;
+}
+
 enum RmsOut : int {
   kRmsCodes = 0,  // int8 codes in natural order + bf16 scale
   kRmsPerm = 1,   // codes with 16-element groups transposed 4x4 (the tensor-core
@@ -49,15 +97,8 @@ __global__ void __launch_bounds__(kTernThreads)
   bool ok = true;
   for (int i = tid; i < nq; i += kTernThreads) {
     const uint2 v = __ldg(row + i);
-    const uint32_t h[4] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float f = bf16_bits_to_f32(h[j]);
-      ok &= fabsf(f) < 8388608.0f;  // 2^23 (false for NaN)
-      u128 a = 0;
-      ok &= abs_fixed(__fmul_rn(f, f), &a);
-      s += a;
-    }
+    const uint32_t w2[2] = {v.x, v.y};
+    s += sumsq_fixed(w2, &ok);
   }
   if (!ok) atomicOr(&g_device_error, kDevErrValue);
   const u128 total = cta_sum(s, part);
@@ -134,6 +175,142 @@ __global__ void __launch_bounds__(kTernThreads)
   } else {
     uint32_t* qrow = reinterpret_cast<uint32_t*>(xq + m * K);
     for (int i = tid; i < nq; i += kTernThreads) qrow[i] = codes4(i);
+  }
+  if (tid == 0) sa[m] = f32_to_bf16_bits(rq.s);
+}
+
+// The same with the row held in registers: one read of x from HBM. Each
+// thread owns the 16-element groups tid, tid + 256, ... (NG of them, K <=
+// 4096 * NG); g, a load-time constant like the packed weights, is read
+// before the previous kernel on the stream has finished.
+template <int MODE, int NG>
+__global__ void __launch_bounds__(kTernThreads)
+    rmsnorm_quant_reg_kernel(int8_t* __restrict__ xq, uint16_t* __restrict__ sa,
+                             int32_t* __restrict__ rowsum, const uint16_t* __restrict__ x,
+                             const uint16_t* __restrict__ g, float eps, int K) {
+  __shared__ uint64_t part[2 * (kTernThreads / 32)];
+  __shared__ uint32_t red[kTernThreads / 32];
+  __shared__ float r_s;
+  pdl_launch_dependents();
+  const int64_t m = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int ng = K / 16;
+  const uint4* row = reinterpret_cast<const uint4*>(x + m * K);
+  const uint4* gw = reinterpret_cast<const uint4*>(g);
+  uint4 xv[NG][2], gv[NG][2];
+#pragma unroll
+  for (int j = 0; j < NG; ++j) {
+    const int gi = tid + j * kTernThreads;
+    gv[j][0] = gi < ng ? __ldg(gw + 2 * gi) : make_uint4(0u, 0u, 0u, 0u);
+    gv[j][1] = gi < ng ? __ldg(gw + 2 * gi + 1) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  pdl_wait();
+#pragma unroll
+  for (int j = 0; j < NG; ++j) {
+    const int gi = tid + j * kTernThreads;
+    xv[j][0] = gi < ng ? __ldg(row + 2 * gi) : make_uint4(0u, 0u, 0u, 0u);
+    xv[j][1] = gi < ng ? __ldg(row + 2 * gi + 1) : make_uint4(0u, 0u, 0u, 0u);
+  }
+
+  // exact sum of squares (padding groups hold zeros)
+  u128 s = 0;
+  bool ok = true;
+#pragma unroll
+  for (int j = 0; j < NG; ++j) {
+    const uint32_t w8[8] = {xv[j][0].x, xv[j][0].y, xv[j][0].z, xv[j][0].w,
+                            xv[j][1].x, xv[j][1].y, xv[j][1].z, xv[j][1].w};
+    s += sumsq_fixed(w8, &ok);
+  }
+  if (!ok) atomicOr(&g_device_error, kDevErrValue);
+  const u128 total = cta_sum(s, part);
+  if (tid == 0)
+    r_s = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(mean_of(total, static_cast<double>(K)), eps)));
+  __syncthreads();
+  const float r = r_s;
+
+  // z = bf16(g * bf16(x * r)) in place of x; its absmax as bf16 magnitude bits
+  uint32_t mb = 0;
+#pragma unroll
+  for (int j = 0; j < NG; ++j)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t* xw = reinterpret_cast<uint32_t*>(&xv[j][h]);
+      const uint32_t* gww = reinterpret_cast<const uint32_t*>(&gv[j][h]);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const uint32_t z0 = f32_to_bf16_bits(rms_z(xw[t] & 0xFFFFu, gww[t] & 0xFFFFu, r));
+        const uint32_t z1 = f32_to_bf16_bits(rms_z(xw[t] >> 16, gww[t] >> 16, r));
+        xw[t] = z0 | (z1 << 16);
+        mb = max(mb, max(z0 & 0x7FFFu, z1 & 0x7FFFu));
+      }
+    }
+
+  if constexpr (MODE == kRmsZ) {
+    uint4* zrow = reinterpret_cast<uint4*>(xq) + m * (K / 8);
+#pragma unroll
+    for (int j = 0; j < NG; ++j) {
+      const int gi = tid + j * kTernThreads;
+      if (gi < ng) {
+        zrow[2 * gi] = xv[j][0];
+        zrow[2 * gi + 1] = xv[j][1];
+      }
+    }
+    return;
+  }
+
+  mb = __reduce_max_sync(0xFFFFFFFFu, mb);
+  if (lane == 0) red[warp] = mb;
+  __syncthreads();
+  if (tid < 32) {
+    uint32_t t = tid < kTernThreads / 32 ? red[tid] : 0u;
+    t = __reduce_max_sync(0xFFFFFFFFu, t);
+    if (tid == 0) red[0] = t;
+  }
+  __syncthreads();
+  const RowQuant rq = row_quant(bf16_bits_to_f32(red[0]));
+
+  uint4* qrow = reinterpret_cast<uint4*>(xq + m * K);
+  int sum = 0;
+#pragma unroll
+  for (int j = 0; j < NG; ++j) {
+    const int gi = tid + j * kTernThreads;
+    if (gi < ng) {
+      uint32_t w[4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t* zw = reinterpret_cast<const uint32_t*>(&xv[j][h]);
+        w[2 * h] = quant4_f32(make_float4(bf16_bits_to_f32(zw[0] & 0xFFFFu), bf16_bits_to_f32(zw[0] >> 16),
+                                          bf16_bits_to_f32(zw[1] & 0xFFFFu), bf16_bits_to_f32(zw[1] >> 16)),
+                              rq);
+        w[2 * h + 1] = quant4_f32(make_float4(bf16_bits_to_f32(zw[2] & 0xFFFFu), bf16_bits_to_f32(zw[2] >> 16),
+                                              bf16_bits_to_f32(zw[3] & 0xFFFFu), bf16_bits_to_f32(zw[3] >> 16)),
+                                  rq);
+      }
+      if constexpr (MODE == kRmsPerm) {
+        sum += __dp4a(static_cast<int>(w[0]), 0x01010101, 0) + __dp4a(static_cast<int>(w[1]), 0x01010101, 0) +
+               __dp4a(static_cast<int>(w[2]), 0x01010101, 0) + __dp4a(static_cast<int>(w[3]), 0x01010101, 0);
+        // 4x4 byte transpose: out word i byte t = in word t byte i
+        const uint32_t t0 = __byte_perm(w[0], w[1], 0x5140u);
+        const uint32_t t1 = __byte_perm(w[0], w[1], 0x7362u);
+        const uint32_t t2 = __byte_perm(w[2], w[3], 0x5140u);
+        const uint32_t t3 = __byte_perm(w[2], w[3], 0x7362u);
+        qrow[gi] = make_uint4(__byte_perm(t0, t2, 0x5410u), __byte_perm(t0, t2, 0x7632u),
+                              __byte_perm(t1, t3, 0x5410u), __byte_perm(t1, t3, 0x7632u));
+      } else {
+        qrow[gi] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  }
+  if constexpr (MODE == kRmsPerm) {
+    sum = __reduce_add_sync(0xFFFFFFFFu, sum);
+    __syncthreads();  // red[0] has been read by every thread
+    if (lane == 0) red[warp] = static_cast<uint32_t>(sum);
+    __syncthreads();
+    if (tid == 0) {
+      int t = 0;
+      for (int w = 0; w < kTernThreads / 32; ++w) t += static_cast<int>(red[w]);
+      rowsum[m] = t;
+    }
   }
   if (tid == 0) sa[m] = f32_to_bf16_bits(rq.s);
 }

@@ -442,7 +442,8 @@ def test_linear_bias_matches_oracle(M, K, N):
 
 # ------------------------------------------------------ RMSNorm -> quantise
 
-RMS_CASES = [(1, 64), (2, 96), (7, 2560), (64, 4096), (300, 2560), (5, 11008), (1, 27648)]
+RMS_CASES = [(1, 64), (2, 96), (7, 2560), (64, 4096), (300, 2560), (3, 8192), (5, 11008),
+             (2, 16384), (2, 16416), (1, 27648)]
 
 
 def norm_weight(K, seed):
@@ -454,7 +455,8 @@ def norm_weight(K, seed):
 
 def norm_inputs(M, K, seed):
     """Activations with a zero row (r = 1/sqrt(eps)), a row scaled by 2^12
-    (large squares) and a row scaled by 2^-70 (squares below 2^-64)."""
+    (large squares), a row scaled by 2^-70 (squares below 2^-64), and rows
+    mixing magnitudes far apart (the exact sum's general case)."""
     x = acts(95, seed, M, K)
     xf = (x.astype(np.uint32) << 16).view(np.float32)
     if M > 2:
@@ -463,6 +465,11 @@ def norm_inputs(M, K, seed):
         x[3] = f32_to_bf16_bits(xf[3] * np.float32(2.0 ** 12))
     if M > 4:
         x[4] = f32_to_bf16_bits(xf[4] * np.float32(2.0 ** -70))
+    if M > 5:  # squares in [2^-64, 2^-50): truncated at 2^-64
+        x[5, ::3] = f32_to_bf16_bits(xf[5, ::3] * np.float32(2.0 ** -28))
+    if M > 6:  # exponents spread over more than 21 binades
+        x[6, ::5] = f32_to_bf16_bits(xf[6, ::5] * np.float32(2.0 ** -24))
+        x[6, 1::7] = f32_to_bf16_bits(xf[6, 1::7] * np.float32(2.0 ** 16))
     return x
 
 
