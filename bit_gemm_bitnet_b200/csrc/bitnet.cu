@@ -343,8 +343,9 @@ void partition_units(GroupedParams& gp, int grid, int cw) {
 
 template <int MB, int RW_MAX>
 bitnet_status launch_grouped_t(GroupedParams& gp, size_t smem, int sms, cudaStream_t st) {
-  auto k = gemv_grouped_kernel<kGroupedCW, MB, RW_MAX>;
-  constexpr int threads = (kGroupedCW + 1) * 32;
+  constexpr int cw = grouped_cw(MB);
+  auto k = gemv_grouped_kernel<cw, MB, RW_MAX>;
+  constexpr int threads = (cw + 1) * 32;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return BITNET_ERR_CUDA;
@@ -356,7 +357,7 @@ bitnet_status launch_grouped_t(GroupedParams& gp, size_t smem, int sms, cudaStre
   if (grid > gp.units) grid = gp.units;
   if (grid > kGroupGridMax) grid = kGroupGridMax;
   if (grid < 1) grid = 1;
-  partition_units(gp, grid, kGroupedCW);
+  partition_units(gp, grid, cw);
   return launch_pdl(k, dim3(grid), dim3(threads), smem, st, gp);
 }
 
@@ -375,7 +376,7 @@ bitnet_status run_gemv_grouped(const bitnet_gemv_problem* pr, int count, int M, 
   gp.M = M;
   const int mb = bucket_of(M);
   const int rw_max = grouped_rw_max(mb);
-  constexpr int cw = kGroupedCW;
+  const int cw = mb == 1 ? grouped_cw(1) : kGroupedMaxCW;
   auto rw_of = [&](int i, int shift) {
     int rw = pow2_floor(kGroupedStageTarget / (cw * (pr[i].K / 4)));
     if (rw > rw_max) rw = rw_max;

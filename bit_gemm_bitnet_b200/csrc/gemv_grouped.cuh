@@ -16,7 +16,12 @@ namespace bitnet {
 
 constexpr int kGroupMax = 256;       // problems per launch (kernel parameter space)
 constexpr int kGroupGridMax = 512;   // CTAs per launch
-constexpr int kGroupedCW = 16;       // consumer warps per CTA
+// Consumer warps per CTA, by activation-row bucket. One row: 15 (with the
+// producer 16 warps, four per scheduler, so each thread may hold 128
+// registers: more rows in flight per warp). More rows: 16 (the dp4a work per
+// weight grows with the rows and wants every warp).
+constexpr int grouped_cw(int mb) { return mb == 1 ? 15 : 16; }
+constexpr int kGroupedMaxCW = 16;
 // Bytes per unit (aim): large units spread a unit's fixed cost (the wait, the
 // warp reduction, the stores) over more rows; two or three stages of the
 // ring still cover the memory latency.
