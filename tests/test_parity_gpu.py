@@ -520,3 +520,27 @@ def test_rmsnorm_flags_out_of_range_input():
         bn.bitnet_rmsnorm_quantize_act(x, g, 0.0)
     with pytest.raises(ValueError):
         bn.bitnet_rmsnorm_quantize_act(x, g[:128], 1e-5)
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8])
+def test_gemv_grouped_wide_rows(M):
+    """Grouped problems with ragged N, K from 128 to 7680 (units of one or two
+    rows per warp), per-row and per-tensor weight scales, against the oracle
+    and the single-problem kernel."""
+    shapes = [(2560, 2560), (2560, 640), (6912, 300), (128, 77), (4096, 1000), (256, 1),
+              (7680, 130), (1152, 200)]
+    xs, wps, sws, host = [], [], [], []
+    for i, (K, N) in enumerate(shapes):
+        x = acts(101, 10 * M + i, M, K)
+        w = weights(101, 10 * M + i, N, K)
+        sw = synth.uniform_f32(synth.key(101, 10 * M + i, 3), N if i % 2 else 1, 0.01, 0.1)
+        p = oracle.pack(w)
+        host.append((x, p, sw))
+        xs.append(to_dev(x, torch.bfloat16))
+        wps.append(to_dev(p))
+        sws.append(to_dev(sw))
+    outs = bn.bitnet_gemv_fused_grouped(xs, wps, sws)
+    bn.bitnet_device_status()
+    for (x, p, sw), o, xd, wd, sd in zip(host, outs, xs, wps, sws):
+        assert_bf16_close(bf16_bits(o), oracle.linear(x, p, sw))
+        assert np.array_equal(bf16_bits(o), bf16_bits(bn.bitnet_gemv_fused(xd, wd, sd)))
