@@ -313,6 +313,13 @@ def make_sweep(bn, d, order="independent", branches=8):
     return sweep
 
 
+# A few milliseconds of device spin before the first timed event: the host
+# then enqueues every timed step while the device is still busy, so a stall
+# of the host (a context switch, the clock sampler starting) cannot leave
+# the device idle between timed steps. The spin itself is outside the events.
+HOST_LEAD_CYCLES = 6_000_000
+
+
 def time_graph(g, steps, warmup, barrier):
     for _ in range(warmup):
         g.replay()
@@ -320,6 +327,7 @@ def time_graph(g, steps, warmup, barrier):
     barrier()
     torch.cuda.synchronize()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    torch.cuda._sleep(HOST_LEAD_CYCLES)
     ev[0].record()
     for i in range(steps):
         g.replay()
@@ -528,6 +536,7 @@ def time_rotation(fns, reps=20, warmup=3):
         for _ in range(warmup):
             g.replay()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        torch.cuda._sleep(HOST_LEAD_CYCLES)
         ev[0].record(s)
         for i in range(reps):
             g.replay()

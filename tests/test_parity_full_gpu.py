@@ -12,7 +12,7 @@ import oracle
 import synth
 from synth import workloads as W
 import bit_gemm_bitnet_b200 as bn
-from helpers import bf16_bits, bf16_ulp_diff, to_dev
+from helpers import bf16_bits, bf16_ulp_diff, f32_to_bf16_bits, to_dev
 
 pytestmark = pytest.mark.gpu
 THREADS = max(1, min(32, os.cpu_count() or 1))
@@ -141,3 +141,68 @@ def test_decode_sweep_grouped_graph_matches_oracle():
     torch.cuda.synchronize()
     for i, (x, p, sw) in checks.items():
         close(bf16_bits(outs[i]), oracle.linear_cols_threads(x, p, sw, THREADS))
+
+
+# ------------------------------------- the widened rows at the bench's sizes
+
+def _ffn_weights(N=11008, K=4096):
+    w = synth.ternary(synth.key(W.W_PREFILL, 1, synth.T_WEIGHT, N), N, K)
+    return w, oracle.pack(w), bn.bitnet_pack_weights(to_dev(w))
+
+
+def _sample(M, seed):
+    return np.unique(np.r_[np.random.default_rng(seed).choice(M, 40, replace=False), 0, M - 1])
+
+
+@pytest.mark.parametrize("per_row", [True, False])
+def test_ternarize_bench_size(per_row):
+    """11008 x 4096 float32 weights, as the bench ternarises them."""
+    w = (np.random.default_rng(7).standard_normal((11008, 4096)) * 0.02).astype(np.float32)
+    wt_ref, sc_ref = oracle.ternarize_absmean(w, per_row=per_row)
+    wt, sc = bn.bitnet_ternarize_absmean(to_dev(w), per_row=per_row)
+    assert np.array_equal(wt.cpu().numpy(), wt_ref)
+    assert np.array_equal(sc.cpu().numpy(), sc_ref)
+
+
+def test_float32_gemv_and_linear_bench_size():
+    """float32 activations: the decode GEMV at M = 1 (every output) and
+    bitnet_linear at M = 2048 (sampled rows), 4096 -> 11008."""
+    w, p, pd = _ffn_weights()
+    sw = np.array([0.05], np.float32)
+    x1 = np.random.default_rng(11).standard_normal((1, 4096)).astype(np.float32)
+    close(bf16_bits(bn.bitnet_gemv_fused(to_dev(x1), pd, to_dev(sw))), oracle.linear_f32(x1, p, sw))
+    x = np.random.default_rng(12).standard_normal((2048, 4096)).astype(np.float32)
+    y = bn.bitnet_linear(to_dev(x), pd, to_dev(sw))
+    rows = _sample(2048, 12)
+    close(bf16_bits(y)[rows], oracle.linear_f32(x[rows], p, sw))
+
+
+def test_linear_bias_bench_size():
+    w, p, pd = _ffn_weights()
+    sw = synth.uniform_f32(synth.key(W.W_PREFILL, 2, 3), 11008, 0.01, 0.1)
+    x = synth.act_bf16(synth.key(W.W_PREFILL, 2048, synth.T_ACT, 11008), 2048, 4096)
+    bias = f32_to_bf16_bits((np.random.default_rng(13).standard_normal(11008) * 0.1).astype(np.float32))
+    y = bn.bitnet_linear(to_dev(x, torch.bfloat16), pd, to_dev(sw), bias=to_dev(bias, torch.bfloat16))
+    rows = _sample(2048, 13)
+    close(bf16_bits(y)[rows], oracle.linear_bias(x[rows], p, sw, bias))
+
+
+def test_rmsnorm_bench_size():
+    """RMSNorm + quantiser over 2048 rows of 4096 (every code and scale), and
+    bitnet_linear_rmsnorm at M = 2048 (sampled rows) and M = 1."""
+    K = 4096
+    x = synth.act_bf16(synth.key(W.W_PREFILL, 2048, synth.T_ACT, K), 2048, K)
+    g = f32_to_bf16_bits((1.0 + 0.1 * np.random.default_rng(14).standard_normal(K)).astype(np.float32))
+    xd, gd = to_dev(x, torch.bfloat16), to_dev(g, torch.bfloat16)
+    q_ref, s_ref = oracle.rmsnorm_quantize(x, g, 1e-6)
+    q, s = bn.bitnet_rmsnorm_quantize_act(xd, gd, 1e-6)
+    bn.bitnet_device_status()
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(bf16_bits(s), s_ref)
+    w, p, pd = _ffn_weights()
+    sw = np.array([0.05], np.float32)
+    y = bn.bitnet_linear_rmsnorm(xd, gd, 1e-6, pd, to_dev(sw))
+    rows = _sample(2048, 14)
+    close(bf16_bits(y)[rows], oracle.linear_rmsnorm(x[rows], g, 1e-6, p, sw))
+    y1 = bn.bitnet_linear_rmsnorm(xd[:1], gd, 1e-6, pd, to_dev(sw))
+    close(bf16_bits(y1), oracle.linear_rmsnorm(x[:1], g, 1e-6, p, sw))
