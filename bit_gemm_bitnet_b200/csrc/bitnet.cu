@@ -864,7 +864,8 @@ static bitnet_status gemv_common(GemvParams& p, const void* x, bitnet_dtype dt,
 static bitnet_status gemv_fused_impl(uint16_t* out, const void* x, bitnet_dtype dt,
                                      const uint8_t* w_packed, const float* scale_wt,
                                      int64_t scale_wt_len, const uint16_t* bias, int64_t M,
-                                     int64_t N, int64_t K, void* stream) {
+                                     int64_t N, int64_t K, void* stream,
+                                     const uint16_t* norm_g = nullptr, float norm_eps = 0.0f) {
   GemvParams p = {};
   bitnet_status s = gemv_common(p, x, dt, w_packed, M, N, K);
   if (s != BITNET_OK) return s;
@@ -878,7 +879,10 @@ static bitnet_status gemv_fused_impl(uint16_t* out, const void* x, bitnet_dtype 
   p.sw = scale_wt;
   p.sw_len = static_cast<int>(scale_wt_len);
   p.bias = bias;
-  if (dt == BITNET_BF16 && skq_ok(x, w_packed, M, K) && K / 128 <= sk::MAX_SPLIT * skq::MAX_KB) {
+  p.norm_g = norm_g;
+  p.norm_eps = norm_eps;
+  if (norm_g == nullptr && dt == BITNET_BF16 && skq_ok(x, w_packed, M, K) &&
+      K / 128 <= sk::MAX_SPLIT * skq::MAX_KB) {
     const bitnet_status r = run_gemv_skq(out, static_cast<const uint16_t*>(x), w_packed,
                                          scale_wt, scale_wt_len, M, N, K, as_stream(stream), bias);
     if (r != BITNET_ERR_SHAPE) return r;
@@ -1088,8 +1092,13 @@ bitnet_status bitnet_rmsnorm_quantize_act(int8_t* x_q, uint16_t* scale_act, cons
                            as_stream(stream));
 }
 
+// One or two rows of up to 16384 that the fused GEMV takes: the GEMV's
+// register-cached staging normalises them itself (one launch, no scratch).
+bool rmsnorm_in_gemv(int64_t M, int64_t K) { return M <= 2 && K <= 16384 && linear_uses_gemv(M, K); }
+
 size_t bitnet_linear_rmsnorm_workspace_bytes(int64_t M, int64_t K) {
   if (M <= 0 || K <= 0) return 0;
+  if (rmsnorm_in_gemv(M, K)) return 0;
   if (linear_uses_gemv(M, K)) return align256(static_cast<size_t>(M) * static_cast<size_t>(K) * 2);
   return align256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
          align256(static_cast<size_t>(M) * 2) + align256(static_cast<size_t>(M) * 4);
@@ -1104,14 +1113,17 @@ bitnet_status bitnet_linear_rmsnorm(uint16_t* out, const uint16_t* x, const uint
   if (!(eps > 0.0f) || !std::isfinite(eps)) return BITNET_ERR_VALUE;
   if (M == 0 || N == 0) return BITNET_OK;
   const size_t need = bitnet_linear_rmsnorm_workspace_bytes(M, K);
-  if (workspace == nullptr || workspace_bytes < need) return BITNET_ERR_WORKSPACE;
-  if (!aligned(workspace, 256)) return BITNET_ERR_ALIGN;
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return BITNET_ERR_WORKSPACE;
+  if (need > 0 && !aligned(workspace, 256)) return BITNET_ERR_ALIGN;
   if (out == nullptr || x == nullptr || g == nullptr || w_packed == nullptr)
     return BITNET_ERR_NULL;
   s = check_scale_wt(scale_wt, scale_wt_len, N);
   if (s != BITNET_OK) return s;
   if (!aligned(out, 16) || !aligned(x, 16) || !aligned(g, 16) || !aligned(w_packed, 16))
     return BITNET_ERR_ALIGN;
+  if (rmsnorm_in_gemv(M, K))
+    return gemv_fused_impl(out, x, BITNET_BF16, w_packed, scale_wt, scale_wt_len, nullptr, M, N, K,
+                           stream, g, eps);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaStream_t st = as_stream(stream);
   if (linear_uses_gemv(M, K)) {

@@ -26,6 +26,7 @@
 #pragma once
 #include "common.cuh"
 #include "pack_quant.cuh"
+#include "rmsnorm.cuh"
 
 namespace bitnet {
 
@@ -53,6 +54,8 @@ struct GemvParams {
   uint16_t* dbg_sa;       // optional: their scales (block 0)
   int x_f32;              // x holds float32 values
   const uint16_t* bias;   // optional bf16 [N], added to the bf16 output
+  const uint16_t* norm_g; // optional bf16 [K]: RMSNorm the rows (weight g) before quantising
+  float norm_eps;         // its epsilon
 };
 
 // 4x4 byte transpose of a 16-byte group: out word i byte b = in word b byte i.
@@ -252,9 +255,14 @@ __device__ __forceinline__ int q_pos(int g, int full_end) {
 // (single-problem kernel): every quad is loaded once and kept in registers
 // for the quantise pass, and the code sums go to their own slots (no barrier
 // to reuse red[]).
+// With norm_g, the rows are first RMS-normalised exactly as the norm kernel
+// does (rmsnorm.cuh): every CTA derives the same r = 1 / sqrt(mean(x^2) +
+// eps) from the exact sum of squares and quantises z = bf16(g * bf16(x * r)).
 template <int CW, int MB, int NQ, bool QUAD>
 __device__ __forceinline__ void gemv_stage_cached(const GemvSmem& sh, const uint16_t* __restrict__ x,
-                                                  int K, int Mc, uint16_t* dbg_sa) {
+                                                  int K, int Mc, uint16_t* dbg_sa,
+                                                  const uint16_t* __restrict__ norm_g,
+                                                  float norm_eps) {
   constexpr int kGemvConsumerWarps = CW;
   constexpr int kGemvConsumers = CW * 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -276,6 +284,66 @@ __device__ __forceinline__ void gemv_stage_cached(const GemvSmem& sh, const uint
       const int u = tid + j * kGemvConsumers;
       v[m][j] = (live && u < quads) ? __ldg(row + u) : make_uint2(0u, 0u);
     }
+  }
+  if (norm_g != nullptr) {
+    // the norm's weights, requested before the sums need the barrier
+    const uint2* gw = reinterpret_cast<const uint2*>(norm_g);
+    uint2 gv[NQ];
+#pragma unroll
+    for (int j = 0; j < NQ; ++j) {
+      const int u = tid + j * kGemvConsumers;
+      gv[j] = u < quads ? __ldg(gw + u) : make_uint2(0u, 0u);
+    }
+    // exact sums of squares: each warp's by butterflies on the two 64-bit
+    // halves, one slot pair per warp and row past the reduction scratch
+    uint64_t* part = reinterpret_cast<uint64_t*>(red + 256);
+    bool ok = true;
+#pragma unroll
+    for (int m = 0; m < MB; ++m) {
+      u128 ss = 0;
+#pragma unroll
+      for (int j = 0; j < NQ; ++j) {
+        const uint32_t w2[2] = {v[m][j].x, v[m][j].y};
+        ss += sumsq_fixed(w2, &ok);
+      }
+      uint64_t lo = static_cast<uint64_t>(ss), hi = static_cast<uint64_t>(ss >> 64);
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) {
+        const uint64_t olo = __shfl_xor_sync(0xFFFFFFFFu, lo, o);
+        const uint64_t ohi = __shfl_xor_sync(0xFFFFFFFFu, hi, o);
+        const uint64_t nlo = lo + olo;
+        hi = hi + ohi + (nlo < lo ? 1u : 0u);
+        lo = nlo;
+      }
+      if (lane == 0) {
+        part[2 * (warp * MB + m)] = lo;
+        part[2 * (warp * MB + m) + 1] = hi;
+      }
+    }
+    if (!ok) atomicOr(&g_device_error, kDevErrValue);
+    named_barrier_sync(1, kGemvConsumers);
+    if (tid < MB) {
+      u128 total = 0;
+      for (int w = 0; w < kGemvConsumerWarps; ++w)
+        total += (static_cast<u128>(part[2 * (w * MB + tid) + 1]) << 64) | part[2 * (w * MB + tid)];
+      rq_s[tid] = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(mean_of(total, static_cast<double>(K)), norm_eps)));
+    }
+    named_barrier_sync(1, kGemvConsumers);
+    // z in place of x (padding quads hold zeros in x and g: z = 0)
+#pragma unroll
+    for (int m = 0; m < MB; ++m) {
+      const float r = rq_s[m];
+#pragma unroll
+      for (int j = 0; j < NQ; ++j) {
+        const uint32_t z0 = f32_to_bf16_bits(rms_z(v[m][j].x & 0xFFFFu, gv[j].x & 0xFFFFu, r));
+        const uint32_t z1 = f32_to_bf16_bits(rms_z(v[m][j].x >> 16, gv[j].x >> 16, r));
+        const uint32_t z2 = f32_to_bf16_bits(rms_z(v[m][j].y & 0xFFFFu, gv[j].y & 0xFFFFu, r));
+        const uint32_t z3 = f32_to_bf16_bits(rms_z(v[m][j].y >> 16, gv[j].y >> 16, r));
+        v[m][j] = make_uint2(z0 | (z1 << 16), z2 | (z3 << 16));
+      }
+    }
+    // every thread has read r before thread m writes the row's quantiser
+    // into rq_s (after the next barrier)
   }
 #pragma unroll
   for (int m = 0; m < MB; ++m) {
@@ -341,7 +409,9 @@ __device__ __forceinline__ void gemv_stage_cached(const GemvSmem& sh, const uint
 template <int CW, int MB, bool QUAD = false, bool CACHE = false>
 __device__ __forceinline__ void gemv_stage_activations(const GemvSmem& sh, const void* __restrict__ x,
                                                        int K, int Mc, int8_t* dbg_q, uint16_t* dbg_sa,
-                                                       bool f32 = false) {
+                                                       bool f32 = false,
+                                                       const uint16_t* norm_g = nullptr,
+                                                       float norm_eps = 0.0f) {
   constexpr int kGemvConsumerWarps = CW;
   constexpr int kGemvConsumers = CW * 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -355,14 +425,17 @@ __device__ __forceinline__ void gemv_stage_activations(const GemvSmem& sh, const
   if constexpr (CACHE && MB <= 2) {
     const uint16_t* xb = static_cast<const uint16_t*>(x);
     if (!f32 && dbg_q == nullptr && quads <= 4 * kGemvConsumers) {
-      gemv_stage_cached<CW, MB, 4, QUAD>(sh, xb, K, Mc, dbg_sa);
+      gemv_stage_cached<CW, MB, 4, QUAD>(sh, xb, K, Mc, dbg_sa, norm_g, norm_eps);
       return;
     }
     if (!f32 && dbg_q == nullptr && quads <= 8 * kGemvConsumers) {
-      gemv_stage_cached<CW, MB, 8, QUAD>(sh, xb, K, Mc, dbg_sa);
+      gemv_stage_cached<CW, MB, 8, QUAD>(sh, xb, K, Mc, dbg_sa, norm_g, norm_eps);
       return;
     }
   }
+  // the norm is only fused where the rows stay in registers (the host
+  // checks): anything else is reported rather than quantised unnormalised
+  if (norm_g != nullptr && tid == 0) atomicOr(&g_device_error, kDevErrValue);
     // absmax of every activation row (as fp32 magnitude bits); each thread
     // owns the 4-element quads tid, tid + 512, ... of a row (loops kept
     // rolled: a small code footprint)
@@ -597,7 +670,8 @@ __global__ void __launch_bounds__((CW + 1) * 32) gemv_kernel(GemvParams p) {
   if constexpr (!PREQ) {
     gemv_stage_activations<CW, MB, false, true>(GemvSmem{qsum, saf, rq_s, rq_r, red, qs}, p.x, K, Mc,
                                    blockIdx.x == 0 ? p.dbg_q : nullptr,
-                                   blockIdx.x == 0 ? p.dbg_sa : nullptr, p.x_f32 != 0);
+                                   blockIdx.x == 0 ? p.dbg_sa : nullptr, p.x_f32 != 0,
+                                   p.norm_g, p.norm_eps);
   } else {
     int qs_part[MB];
 #pragma unroll

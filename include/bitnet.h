@@ -216,19 +216,27 @@ bitnet_status bitnet_rmsnorm_quantize_act(int8_t* x_q, uint16_t* scale_act, cons
                                           const uint16_t* g, float eps, int64_t M, int64_t K,
                                           void* stream);
 
-/* Workspace of bitnet_linear_rmsnorm for (M, K). Where bitnet_linear takes
- * the fused GEMV (M < 16 and the GEMV's fit rule): the normalised bf16 [M, K]
- * rows, which the GEMV then quantises. Otherwise the int8 [M, K] codes, bf16
- * [M] scales and int32 [M] code sums. Each part 256-byte aligned; 0 for
- * M == 0. */
+/* Workspace of bitnet_linear_rmsnorm for (M, K), in bytes. There are three
+ * cases:
+ *   - M <= 2 and K <= 16384, where bitnet_linear takes the fused GEMV: 0.
+ *     The GEMV normalises the rows itself, in one launch.
+ *   - Otherwise, where bitnet_linear takes the fused GEMV (M < 16 and the
+ *     GEMV's fit rule): the normalised bf16 [M, K] rows, which the GEMV then
+ *     quantises.
+ *   - Otherwise: the int8 [M, K] codes, the bf16 [M] scales and the int32 [M]
+ *     code sums.
+ * Each part is 256-byte aligned. The size is 0 for M == 0. */
 size_t bitnet_linear_rmsnorm_workspace_bytes(int64_t M, int64_t K);
 
-/* RMSNorm, quantiser and the layer in one call, on the caller's stream:
- * the norm's kernel writes its result into `workspace` (the quantised rows,
- * or for few rows the bf16 normalised rows), then the kernels of
- * bitnet_linear run on it; the result equals bitnet_linear applied to
- * bf16(g * bf16(x * r)). Arguments as bitnet_rmsnorm_quantize_act and
- * bitnet_linear; x is bf16, workspace 256-byte aligned. */
+/* RMSNorm, quantiser and the layer in one call, on the caller's stream. The
+ * result equals bitnet_linear applied to bf16(g * bf16(x * r)).
+ *   - M <= 2, K <= 16384: the fused GEMV normalises the rows in its own
+ *     staging (one launch; workspace unused, may be NULL).
+ *   - Otherwise the norm's kernel writes into `workspace` (the quantised
+ *     rows, or for few rows the bf16 normalised rows), then the kernels of
+ *     bitnet_linear run on it.
+ * Arguments as bitnet_rmsnorm_quantize_act and bitnet_linear; x is bf16,
+ * workspace 256-byte aligned. */
 bitnet_status bitnet_linear_rmsnorm(uint16_t* out, const uint16_t* x, const uint16_t* g,
                                     float eps, const uint8_t* w_packed, const float* scale_wt,
                                     int64_t scale_wt_len, int64_t M, int64_t N, int64_t K,

@@ -130,6 +130,10 @@ def test_rmsnorm_workspace_size():
     assert L.bitnet_linear_rmsnorm_workspace_bytes(32, 64) == 2048 + 256 + 256
     assert L.bitnet_linear_rmsnorm_workspace_bytes(300, 2560) == 768000 + 768 + 1280
     assert L.bitnet_linear_rmsnorm_workspace_bytes(0, 64) == 0
+    # one or two rows the fused GEMV takes are normalised inside it: no scratch
+    assert L.bitnet_linear_rmsnorm_workspace_bytes(1, 4096) == 0
+    assert L.bitnet_linear_rmsnorm_workspace_bytes(2, 16384) == 0
+    assert L.bitnet_linear_rmsnorm_workspace_bytes(3, 4096) == 3 * 4096 * 2
 
 
 def test_noop_sizes_return_ok_without_work():

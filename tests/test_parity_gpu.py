@@ -486,11 +486,14 @@ def test_rmsnorm_quantize_bitexact(M, K, eps):
     assert np.array_equal(bf16_bits(s), s_ref)
 
 
-@pytest.mark.parametrize("M,K,N", [(1, 2560, 640), (2, 96, 40), (12, 2112, 77), (64, 4096, 300),
+@pytest.mark.parametrize("M,K,N", [(1, 2560, 640), (2, 96, 40), (2, 16384, 130), (1, 11008, 300),
+                                   (3, 4096, 200), (12, 2112, 77), (64, 4096, 300),
                                    (16, 11008, 256), (300, 2560, 520), (2048, 2560, 256)])
 def test_linear_rmsnorm_matches_oracle(M, K, N):
-    """Norm, quantiser and GEMM in one call: the tensor-core GEMMs (permuted
-    workspace plus code sums) and the SIMT path (K % 64 != 0)."""
+    """Norm, quantiser and the layer in one call: the norm inside the fused
+    GEMV's staging (M <= 2), the norm kernel in front of the fused GEMV
+    (3 <= M < 16), the tensor-core GEMMs (permuted workspace plus code sums)
+    and the SIMT path (K % 64 != 0)."""
     x = norm_inputs(M, K, M * 5 + K)
     g = norm_weight(K, N + K)
     w = weights(96, N + K, N, K)
@@ -516,6 +519,14 @@ def test_rmsnorm_flags_out_of_range_input():
         with pytest.raises(bn.BitnetValueError):
             bn.bitnet_device_status()
         bn.bitnet_device_status()
+    # the same check inside the fused GEMV's staging (one row)
+    w = to_dev(oracle.pack(weights(97, 1, 64, K)))
+    xb = torch.ones((1, K), dtype=torch.bfloat16, device="cuda")
+    xb[0, 3] = 2.0 ** 24
+    bn.bitnet_linear_rmsnorm(xb, g, 1e-5, w, torch.tensor([0.05], device="cuda"))
+    with pytest.raises(bn.BitnetValueError):
+        bn.bitnet_device_status()
+    bn.bitnet_device_status()
     with pytest.raises(bn.BitnetValueError):
         bn.bitnet_rmsnorm_quantize_act(x, g, 0.0)
     with pytest.raises(ValueError):
