@@ -141,9 +141,12 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# the headers each kernel's translation unit reads (gemv.cuh includes the norm
+# helpers of rmsnorm.cuh, which include ternarize.cuh)
+_GEMV_HEADERS = ("common.cuh", "pack_quant.cuh", "ternarize.cuh", "rmsnorm.cuh", "gemv.cuh")
 KERNEL_SOURCES = {
-    "gemv_kernel": ("common.cuh", "pack_quant.cuh", "gemv.cuh"),
-    "gemv_grouped_kernel": ("common.cuh", "pack_quant.cuh", "gemv.cuh", "gemv_grouped.cuh"),
+    "gemv_kernel": _GEMV_HEADERS,
+    "gemv_grouped_kernel": _GEMV_HEADERS + ("gemv_grouped.cuh",),
     "gemm_i8_ts_kernel": ("common.cuh", "pack_quant.cuh", "gemm_ts.cuh"),
 }
 

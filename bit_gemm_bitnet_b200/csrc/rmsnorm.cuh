@@ -23,37 +23,47 @@ __device__ __forceinline__ float rms_z(uint32_t xbits16, uint32_t gbits16, float
 // field b >= 1 is m * 2^(b - 134), m in [128, 255], so trunc(x^2 * 2^64) is
 // the integer m^2 * 2^(2b - 204) when b >= 102, and 0 when b < 95. When
 // every value is in one of those two classes and the first spans at most 21
-// binades below the largest exponent bmax, the terms are summed in 64 bits
-// in units of 2^(2 bmax - 246) (each below 2^58) and the sum shifted into
-// place once. Otherwise each term goes through abs_fixed. `ok` is cleared
-// for |x| >= 2^23 and non-finite x.
+// binades below the largest exponent bmax, each term is an integer below
+// 2^58 in units of 2^(2 bmax - 246): (x * 2^(155 - bmax))^2, exact in fp32
+// (an 8-bit significand squared), converted exactly to 64 bits and summed;
+// the sum is shifted into place once. Otherwise each term goes through
+// abs_fixed. `ok` is cleared for |x| >= 2^23 and non-finite x.
 template <int NW>
 __device__ __forceinline__ u128 sumsq_fixed(const uint32_t (&w)[NW], bool* ok) {
   static_assert(NW <= 32, "64 terms below 2^58 each fit in 64 bits");
-  uint32_t bmax = 0;
+  uint32_t e[NW];  // both exponent fields of each word
+  uint32_t em = 0;
 #pragma unroll
-  for (int i = 0; i < NW; ++i) bmax = max(bmax, max((w[i] >> 7) & 0xFFu, (w[i] >> 23) & 0xFFu));
+  for (int i = 0; i < NW; ++i) {
+    e[i] = (w[i] >> 7) & 0x00FF00FFu;
+    em = __vmaxu2(em, e[i]);
+  }
+  const uint32_t bmax = max(em & 0xFFFFu, em >> 16);
   if (bmax >= 150u) {  // 2^23 and above, Inf, NaN
     *ok = false;
     return 0;
   }
-  bool fast = true;
-  uint64_t acc = 0;
+  const uint32_t lo = bmax > 123u ? bmax - 21u : 102u;
+  uint32_t good = 0xFFFFFFFFu;
+  uint32_t keep[NW];  // the values, with those below 2^-32 (whose terms are 0) zeroed
 #pragma unroll
-  for (int i = 0; i < 2 * NW; ++i) {
-    const uint32_t h = (w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
-    const uint32_t b = (h >> 7) & 0xFFu;
-    if (b >= 95u) {
-      fast &= b >= 102u && b + 21u >= bmax;
-      const uint32_t m = (h & 0x7Fu) | 0x80u;
-      const int sh = max(2 * (static_cast<int>(b) - static_cast<int>(bmax)) + 42, 0);
-      acc += static_cast<uint64_t>(m * m) << sh;
-    }
+  for (int i = 0; i < NW; ++i) {
+    const uint32_t below = __vcmpltu2(e[i], 0x005F005Fu);  // b < 95
+    good &= below | __vcmpgeu2(e[i], lo * 0x00010001u);
+    keep[i] = w[i] & ~below;
   }
-  if (fast) {
-    if (acc == 0) return 0;
-    const int e = 2 * static_cast<int>(bmax) - 246;  // bmax >= 102 here
-    return e >= 0 ? static_cast<u128>(acc) << e : static_cast<u128>(acc >> -e);  // exact: an integer
+  if (good == 0xFFFFFFFFu) {
+    if (bmax < 102u) return 0;  // every value is below 2^-32
+    const float sc = __int_as_float(static_cast<int>(282u - bmax) << 23);  // 2^(155 - bmax)
+    uint64_t acc = 0;
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+      const float y0 = __fmul_rn(bf16_bits_to_f32(keep[i] & 0xFFFFu), sc);
+      const float y1 = __fmul_rn(bf16_bits_to_f32(keep[i] >> 16), sc);
+      acc += __float2ull_rz(__fmul_rn(y0, y0)) + __float2ull_rz(__fmul_rn(y1, y1));
+    }
+    const int e2 = 2 * static_cast<int>(bmax) - 246;
+    return e2 >= 0 ? static_cast<u128>(acc) << e2 : static_cast<u128>(acc >> -e2);  // exact: an integer
   }
   u128 s = 0;
 #pragma unroll
