@@ -102,20 +102,53 @@ __device__ __forceinline__ uint32_t ternary4(const float4& v, float gamma, float
          (ternary1(v.z, gamma, rgamma) << 16) | (ternary1(v.w, gamma, rgamma) << 24);
 }
 
+// Sum of trunc(|w| * 2^64) over four values (abs_fixed's terms), exact. With
+// e the exponent field of |w| = m * 2^(e - 150) (m < 2^24), a term is the
+// integer m * 2^(e - 86) when e >= 86 and 0 when e < 63. When every value is
+// in one of those two classes and the first spans at most 38 binades below
+// the largest exponent emax, each term is an integer below 2^62 in units of
+// 2^(emax - 124): |w| * 2^(188 - emax), exact in fp32. The terms are
+// converted exactly, summed in 64 bits and shifted into place once.
+// Otherwise each goes through abs_fixed.
+__device__ __forceinline__ u128 abs_sum4(const float4& v, bool* ok) {
+  const uint32_t a[4] = {__float_as_uint(v.x) & 0x7FFFFFFFu, __float_as_uint(v.y) & 0x7FFFFFFFu,
+                         __float_as_uint(v.z) & 0x7FFFFFFFu, __float_as_uint(v.w) & 0x7FFFFFFFu};
+  const uint32_t amax = max(max(a[0], a[1]), max(a[2], a[3]));
+  const uint32_t emax = amax >> 23;
+  if (amax < 0x57000000u) {  // below 2^47 and finite
+    const uint32_t lo = emax > 124u ? emax - 38u : 86u;
+    bool good = true;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t e = a[k] >> 23;
+      good &= e < 63u || e >= lo;
+    }
+    if (good) {
+      if (emax < 86u) return 0;  // every value below 2^-64
+      const float sc = __int_as_float(static_cast<int>(315u - emax) << 23);  // 2^(188 - emax)
+      uint64_t acc = 0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if ((a[k] >> 23) >= 63u) acc += __float2ull_rz(__fmul_rn(__uint_as_float(a[k]), sc));
+      const int e2 = static_cast<int>(emax) - 124;
+      return e2 >= 0 ? static_cast<u128>(acc) << e2 : static_cast<u128>(acc >> -e2);
+    }
+  }
+  u128 s = 0, t = 0;
+  *ok &= abs_fixed(v.x, &t);
+  s += t;
+  *ok &= abs_fixed(v.y, &t);
+  s += t;
+  *ok &= abs_fixed(v.z, &t);
+  s += t;
+  *ok &= abs_fixed(v.w, &t);
+  s += t;
+  return s;
+}
+
 __device__ __forceinline__ u128 row_abs_sum(const float4* row, int nvec, bool* ok) {
   u128 s = 0;
-  for (int i = threadIdx.x; i < nvec; i += kTernThreads) {
-    const float4 v = __ldg(row + i);
-    u128 a = 0;
-    *ok &= abs_fixed(v.x, &a);
-    s += a;
-    *ok &= abs_fixed(v.y, &a);
-    s += a;
-    *ok &= abs_fixed(v.z, &a);
-    s += a;
-    *ok &= abs_fixed(v.w, &a);
-    s += a;
-  }
+  for (int i = threadIdx.x; i < nvec; i += kTernThreads) s += abs_sum4(__ldg(row + i), ok);
   return s;
 }
 

@@ -379,6 +379,12 @@ def dense_weights(N, K, seed):
     w[0, : min(K, 8)] = 0.0
     if N > 2:
         w[2] = 0.0                        # an all-zero row: gamma = eps
+    if N > 4:
+        # magnitudes whose |w| * 2^64 is truncated (2^-60 .. 2^-45) or far
+        # below the rest of their group (the exact sum's general case)
+        w[3, ::7] *= np.float32(2.0 ** -40)
+        w[4, 1::5] *= np.float32(2.0 ** -110)
+        w[4, ::9] *= np.float32(2.0 ** 30)
     return w
 
 
