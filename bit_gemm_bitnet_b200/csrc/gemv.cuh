@@ -596,10 +596,14 @@ __global__ void __launch_bounds__((CW + 1) * 32) gemv_kernel(GemvParams p) {
   volatile int* abort = reinterpret_cast<volatile int*>(smem + 256);
   float* rq_s = reinterpret_cast<float*>(smem + 320);        // [MB]
   float* rq_r = reinterpret_cast<float*>(smem + 384);        // [MB]
-  uint32_t* red = reinterpret_cast<uint32_t*>(smem + 512);   // [16 warps][MB]
+  uint32_t* red = reinterpret_cast<uint32_t*>(smem + 512);   // [16 warps][MB], code sums after
+  // (the fused RMSNorm's 128-bit partial sums, [16 warps][MB] pairs of 64-bit
+  // words, start at red + 256 words: smem + 1536)
   uint8_t* qs = smem + kGemvHeaderBytes;                     // [Mc][K]
   uint8_t* ring = qs + p.q_bytes;
   static_assert(kGemvMaxConsumerWarps * MB * 4 <= kGemvHeaderBytes - 512, "reduction scratch");
+  static_assert(MB > 2 || 1536 + kGemvMaxConsumerWarps * MB * 16 <= kGemvHeaderBytes,
+                "the norm's partial sums fit in the header");
   constexpr bool PLANES = MB <= 2;
 
   const int K = p.K, N = p.N;
