@@ -801,8 +801,6 @@ def run_case(bn, dev, case, reps=3):
 def main():
     args = parse()
     rank, world, local = dist_env()
-    if world != args.gpus and args.gpus > 1:
-        pass
     config = {"workload": "bitnet-b1.58-2B decode sweep, M=1: 30 layers x 7 BitLinears "
                           "(2560->2560, 2560->640 x2, 2560->2560, 2560->6912 x2, 6912->2560) "
                           "+ LM head 2560->128256",
