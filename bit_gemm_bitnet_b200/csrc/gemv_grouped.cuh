@@ -150,6 +150,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1)
     const uint8_t* wp = p.wp[pr];
     uint32_t it = 0;
     for (int u = u_begin; u < u_end; ++u, ++it) {
+      bool next = false;
       while (u >= u1) {
         ++pr;
         u0 = u1;
@@ -158,6 +159,17 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1)
         rpu = CW * p.rw[pr];
         N = p.N[pr];
         wp = p.wp[pr];
+        next = true;
+      }
+      if (next) {
+        // warm L2 with the problem's activation rows, which the consumers
+        // stage when they reach this unit, up to two stages later (2 % on
+        // the decode step). L2 is the point of coherence: a line fetched
+        // before the previous kernel wrote it is updated by that write.
+        const char* xb = reinterpret_cast<const char*>(p.x[pr]);
+        const int xbytes = (MB == 1 ? 1 : p.M) * KB * 8;  // bf16 [M, K]
+        for (int off = lane * 128; off < xbytes; off += 32 * 128)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(xb + off));
       }
       const int s = it % S;
       const uint32_t ph = (it / S) & 1u;
