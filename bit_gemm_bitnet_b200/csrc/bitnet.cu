@@ -169,10 +169,10 @@ int pow2_floor(int64_t v) {
   return r;
 }
 
-template <int CW, int MB, int RW, bool WIDE, bool PREQ>
+template <int CW, int MB, int RW, bool WIDE, bool PREQ, bool NORM>
 bitnet_status launch_gemv_t(const GemvParams& p, int grid_y, size_t smem, int sms,
                             cudaStream_t st) {
-  auto k = gemv_kernel<CW, MB, RW, WIDE, PREQ>;
+  auto k = gemv_kernel<CW, MB, RW, WIDE, PREQ, NORM>;
   constexpr int threads = (CW + 1) * 32;
   if (smem > 48 * 1024) {
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -190,40 +190,48 @@ bitnet_status launch_gemv_t(const GemvParams& p, int grid_y, size_t smem, int sm
   return launch_pdl(k, dim3(gx, grid_y), dim3(threads), smem, st, p);
 }
 
-template <int CW, int MB, bool WIDE, bool PREQ>
+template <int CW, int MB, bool WIDE, bool PREQ, bool NORM>
 bitnet_status launch_gemv_rw(int rw, const GemvParams& p, int gy, size_t smem, int sms,
                              cudaStream_t st) {
   switch (rw) {
-    case 1: return launch_gemv_t<CW, MB, 1, WIDE, PREQ>(p, gy, smem, sms, st);
-    case 2: return launch_gemv_t<CW, MB, 2, WIDE, PREQ>(p, gy, smem, sms, st);
+    case 1: return launch_gemv_t<CW, MB, 1, WIDE, PREQ, NORM>(p, gy, smem, sms, st);
+    case 2: return launch_gemv_t<CW, MB, 2, WIDE, PREQ, NORM>(p, gy, smem, sms, st);
     // instantiated exactly where rw * MB * (MB <= 2 ? 4 : 1) <= 32, the
     // accumulator limit the caller applies
     case 4:
-      if constexpr (MB <= 8) return launch_gemv_t<CW, MB, 4, WIDE, PREQ>(p, gy, smem, sms, st);
+      if constexpr (MB <= 8) return launch_gemv_t<CW, MB, 4, WIDE, PREQ, NORM>(p, gy, smem, sms, st);
       return BITNET_ERR_SHAPE;
     default:
-      if constexpr (MB == 1 || MB == 4) return launch_gemv_t<CW, MB, 8, WIDE, PREQ>(p, gy, smem, sms, st);
+      if constexpr (MB == 1 || MB == 4) return launch_gemv_t<CW, MB, 8, WIDE, PREQ, NORM>(p, gy, smem, sms, st);
       return BITNET_ERR_SHAPE;
   }
 }
 
-template <int CW, bool WIDE, bool PREQ>
+// NORM (the fused RMSNorm): one or two fused rows only, its own
+// instantiations, so that the other kernels carry none of its registers.
+template <int CW, bool WIDE, bool PREQ, bool NORM = false>
 bitnet_status launch_gemv_mb(int mb, int rw, const GemvParams& p, int gy, size_t smem, int sms,
                              cudaStream_t st) {
-  switch (mb) {
-    case 1: return launch_gemv_rw<CW, 1, WIDE, PREQ>(rw, p, gy, smem, sms, st);
-    case 2: return launch_gemv_rw<CW, 2, WIDE, PREQ>(rw, p, gy, smem, sms, st);
-    case 4: return launch_gemv_rw<CW, 4, WIDE, PREQ>(rw, p, gy, smem, sms, st);
-    case 8: return launch_gemv_rw<CW, 8, WIDE, PREQ>(rw, p, gy, smem, sms, st);
-    default: return launch_gemv_rw<CW, 16, WIDE, PREQ>(rw, p, gy, smem, sms, st);
+  if constexpr (NORM) {
+    if (mb == 1) return launch_gemv_rw<CW, 1, WIDE, false, true>(rw, p, gy, smem, sms, st);
+    if (mb == 2) return launch_gemv_rw<CW, 2, WIDE, false, true>(rw, p, gy, smem, sms, st);
+    return BITNET_ERR_SHAPE;
+  } else {
+    switch (mb) {
+      case 1: return launch_gemv_rw<CW, 1, WIDE, PREQ, false>(rw, p, gy, smem, sms, st);
+      case 2: return launch_gemv_rw<CW, 2, WIDE, PREQ, false>(rw, p, gy, smem, sms, st);
+      case 4: return launch_gemv_rw<CW, 4, WIDE, PREQ, false>(rw, p, gy, smem, sms, st);
+      case 8: return launch_gemv_rw<CW, 8, WIDE, PREQ, false>(rw, p, gy, smem, sms, st);
+      default: return launch_gemv_rw<CW, 16, WIDE, PREQ, false>(rw, p, gy, smem, sms, st);
+    }
   }
 }
 
-template <bool WIDE, bool PREQ>
+template <bool WIDE, bool PREQ, bool NORM = false>
 bitnet_status launch_gemv_cw(int cw, int mb, int rw, const GemvParams& p, int gy, size_t smem,
                              int sms, cudaStream_t st) {
-  if (cw == 16) return launch_gemv_mb<16, WIDE, PREQ>(mb, rw, p, gy, smem, sms, st);
-  return launch_gemv_mb<8, WIDE, PREQ>(mb, rw, p, gy, smem, sms, st);
+  if (cw == 16) return launch_gemv_mb<16, WIDE, PREQ, NORM>(mb, rw, p, gy, smem, sms, st);
+  return launch_gemv_mb<8, WIDE, PREQ, NORM>(mb, rw, p, gy, smem, sms, st);
 }
 
 int bucket_of(int m) { return m <= 1 ? 1 : m <= 2 ? 2 : m <= 4 ? 4 : m <= 8 ? 8 : 16; }
@@ -288,6 +296,9 @@ bitnet_status run_gemv(GemvParams p, bool preq, cudaStream_t st) {
   p.stage_bytes = static_cast<uint32_t>(stage);
   const size_t smem = gemv_smem(qrows, K, cw, rw, stages);
   const bool wide = (K % 64) == 0;
+  if (p.norm_g != nullptr && !preq)
+    return wide ? launch_gemv_cw<true, false, true>(cw, mb, rw, p, gy, smem, dev->sms, st)
+                : launch_gemv_cw<false, false, true>(cw, mb, rw, p, gy, smem, dev->sms, st);
   if (wide)
     return preq ? launch_gemv_cw<true, true>(cw, mb, rw, p, gy, smem, dev->sms, st)
                 : launch_gemv_cw<true, false>(cw, mb, rw, p, gy, smem, dev->sms, st);

@@ -258,7 +258,7 @@ __device__ __forceinline__ int q_pos(int g, int full_end) {
 // With norm_g, the rows are first RMS-normalised exactly as the norm kernel
 // does (rmsnorm.cuh): every CTA derives the same r = 1 / sqrt(mean(x^2) +
 // eps) from the exact sum of squares and quantises z = bf16(g * bf16(x * r)).
-template <int CW, int MB, int NQ, bool QUAD>
+template <int CW, int MB, int NQ, bool QUAD, bool NORM>
 __device__ __forceinline__ void gemv_stage_cached(const GemvSmem& sh, const uint16_t* __restrict__ x,
                                                   int K, int Mc, uint16_t* dbg_sa,
                                                   const uint16_t* __restrict__ norm_g,
@@ -285,7 +285,7 @@ __device__ __forceinline__ void gemv_stage_cached(const GemvSmem& sh, const uint
       v[m][j] = (live && u < quads) ? __ldg(row + u) : make_uint2(0u, 0u);
     }
   }
-  if (norm_g != nullptr) {
+  if constexpr (NORM) {
     // the norm's weights, requested before the sums need the barrier
     const uint2* gw = reinterpret_cast<const uint2*>(norm_g);
     uint2 gv[NQ];
@@ -406,7 +406,7 @@ __device__ __forceinline__ void gemv_stage_cached(const GemvSmem& sh, const uint
 
 // CACHE: the single-problem kernel keeps one or two rows' quads in
 // registers between the passes (4 or 8 per thread, by K).
-template <int CW, int MB, bool QUAD = false, bool CACHE = false>
+template <int CW, int MB, bool QUAD = false, bool CACHE = false, bool NORM = false>
 __device__ __forceinline__ void gemv_stage_activations(const GemvSmem& sh, const void* __restrict__ x,
                                                        int K, int Mc, int8_t* dbg_q, uint16_t* dbg_sa,
                                                        bool f32 = false,
@@ -425,17 +425,17 @@ __device__ __forceinline__ void gemv_stage_activations(const GemvSmem& sh, const
   if constexpr (CACHE && MB <= 2) {
     const uint16_t* xb = static_cast<const uint16_t*>(x);
     if (!f32 && dbg_q == nullptr && quads <= 4 * kGemvConsumers) {
-      gemv_stage_cached<CW, MB, 4, QUAD>(sh, xb, K, Mc, dbg_sa, norm_g, norm_eps);
+      gemv_stage_cached<CW, MB, 4, QUAD, NORM>(sh, xb, K, Mc, dbg_sa, norm_g, norm_eps);
       return;
     }
     if (!f32 && dbg_q == nullptr && quads <= 8 * kGemvConsumers) {
-      gemv_stage_cached<CW, MB, 8, QUAD>(sh, xb, K, Mc, dbg_sa, norm_g, norm_eps);
+      gemv_stage_cached<CW, MB, 8, QUAD, NORM>(sh, xb, K, Mc, dbg_sa, norm_g, norm_eps);
       return;
     }
   }
   // the norm is only fused where the rows stay in registers (the host
   // checks): anything else is reported rather than quantised unnormalised
-  if (norm_g != nullptr && tid == 0) atomicOr(&g_device_error, kDevErrValue);
+  if (NORM && tid == 0) atomicOr(&g_device_error, kDevErrValue);
     // absmax of every activation row (as fp32 magnitude bits); each thread
     // owns the 4-element quads tid, tid + 512, ... of a row (loops kept
     // rolled: a small code footprint)
@@ -600,7 +600,8 @@ __device__ __forceinline__ void gemv_reduce_store(const int (&acc)[RW][MB][PLANE
 // WIDE: K % 64 == 0 (rows 16-byte aligned: one bulk copy per stage),
 // otherwise the producer lanes copy the stage in 8-byte pieces;
 // PREQ: activations come pre-quantised (x_q + scale_act).
-template <int CW, int MB, int RW, bool WIDE, bool PREQ>
+// NORM: the rows are RMS-normalised in the staging (p.norm_g, p.norm_eps).
+template <int CW, int MB, int RW, bool WIDE, bool PREQ, bool NORM = false>
 __global__ void __launch_bounds__((CW + 1) * 32) gemv_kernel(GemvParams p) {
   constexpr int kGemvConsumerWarps = CW;
   constexpr int kGemvConsumers = CW * 32;
@@ -687,8 +688,8 @@ __global__ void __launch_bounds__((CW + 1) * 32) gemv_kernel(GemvParams p) {
   pdl_wait();  // the activations may come from the previous kernel
   const int groups16 = K / 16;
   if constexpr (!PREQ) {
-    gemv_stage_activations<CW, MB, false, true>(GemvSmem{qsum, saf, rq_s, rq_r, red, qs}, p.x, K, Mc,
-                                   blockIdx.x == 0 ? p.dbg_q : nullptr,
+    gemv_stage_activations<CW, MB, false, true, NORM>(GemvSmem{qsum, saf, rq_s, rq_r, red, qs}, p.x,
+                                   K, Mc, blockIdx.x == 0 ? p.dbg_q : nullptr,
                                    blockIdx.x == 0 ? p.dbg_sa : nullptr, p.x_f32 != 0,
                                    p.norm_g, p.norm_eps);
   } else {
