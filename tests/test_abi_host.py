@@ -162,3 +162,24 @@ def test_grouped_validation_before_launch():
     assert L.bitnet_gemv_fused_grouped(p, 2, 1, 0, None) == bn.ERR_ALIGN
     arr[1] = bn.GemvProblem(0x10000, 0x10000, 0x10000, 0x10000, 3, 64, 128)  # scale len
     assert L.bitnet_gemv_fused_grouped(p, 2, 1, 0, None) == bn.ERR_SHAPE
+
+
+def test_bench_traffic_record_names_existing_sources():
+    """The bench reports the recorded DRAM traffic only while the kernel's
+    sources hash as they did at capture; every header it hashes must exist,
+    and the record must name a summary that is committed."""
+    import json
+    import os
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import bench
+    csrc = os.path.join(root, "bit_gemm_bitnet_b200", "csrc")
+    for kernel, files in bench.KERNEL_SOURCES.items():
+        for f in files:
+            assert os.path.exists(os.path.join(csrc, f)), (kernel, f)
+        assert len(bench.source_hash(kernel)) == 16
+    rec = json.load(open(os.path.join(root, "profiles", "ncu_traffic.json")))
+    for kernel, r in rec.items():
+        assert os.path.exists(os.path.join(root, r["summary"])), r["summary"]
+        assert r["bytes"] > 0
