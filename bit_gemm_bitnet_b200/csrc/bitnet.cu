@@ -387,7 +387,10 @@ bitnet_status run_gemv_grouped(const bitnet_gemv_problem* pr, int count, int M, 
   gp.M = M;
   const int mb = bucket_of(M);
   const int rw_max = grouped_rw_max(mb);
-  const int cw = mb == 1 ? grouped_cw(1) : kGroupedMaxCW;
+  const int cw = grouped_cw(mb);  // as launch_grouped_t instantiates it
+  static_assert(grouped_cw(1) <= kGroupedMaxCW && grouped_cw(16) <= kGroupedMaxCW &&
+                    kGroupedMaxCW <= kGemvMaxConsumerWarps,
+                "the staging's per-warp scratch covers every grouped CTA");
   auto rw_of = [&](int i, int shift) {
     int rw = pow2_floor(kGroupedStageTarget / (cw * (pr[i].K / 4)));
     if (rw > rw_max) rw = rw_max;
