@@ -143,6 +143,15 @@ def test_noop_sizes_return_ok_without_work():
     assert L.bitnet_pack_weights(None, None, 0, 8, None) == bn.OK
     assert L.bitnet_quantize_act(None, None, None, 0, 0, 64, None) == bn.OK
     assert L.bitnet_linear(None, None, 0, None, None, 1, 0, 4, 64, None, 0, None) == bn.OK
+    # the widened rows' entries: empty inputs are no-ops too
+    assert L.bitnet_ternarize_absmean(None, None, None, 0, 64, 1, None) == bn.OK
+    assert L.bitnet_ternarize_absmean(None, None, None, 0, 64, 0, None) == bn.OK
+    assert L.bitnet_linear_bias(None, None, 0, None, None, 1, FAKE, 0, 4, 64, None, 0, None) == bn.OK
+    assert L.bitnet_rmsnorm_quantize_act(None, None, None, None, 1e-5, 0, 64, None) == bn.OK
+    assert L.bitnet_linear_rmsnorm(None, None, None, 1e-5, None, None, 1, 0, 4, 64, None, 0,
+                                   None) == bn.OK
+    assert L.bitnet_linear_rmsnorm(None, None, None, 1e-5, None, None, 1, 4, 0, 64, None, 0,
+                                   None) == bn.OK
 
 
 def test_grouped_validation_before_launch():
