@@ -39,6 +39,7 @@ def lib():
         L.oracle_ternarize_absmean.argtypes = [_P, _I64, _I64, ctypes.c_int, _P, _P]
         L.oracle_linear_f32.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P]
         L.oracle_acc.argtypes = [_P, _P, _I64, _I64, _I64, _P]
+        L.oracle_acc_threads.argtypes = [_P, _P, _I64, _I64, _I64, _P, ctypes.c_int]
         L.oracle_epilogue.argtypes = [_P, _P, _P, _I64, _I64, _I64, _P]
         L.oracle_gemm.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]
         L.oracle_linear.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P]
@@ -54,7 +55,7 @@ def lib():
                      "oracle_ternarize_absmean", "oracle_linear_bias", "oracle_rmsnorm",
                      "oracle_rmsnorm_quantize", "oracle_linear_rmsnorm",
                      "oracle_linear_f32",
-                     "oracle_acc", "oracle_epilogue", "oracle_gemm",
+                     "oracle_acc", "oracle_acc_threads", "oracle_epilogue", "oracle_gemm",
                      "oracle_linear", "oracle_linear_threads",
                      "oracle_gemm_threads", "oracle_linear_threads_cols"):
             getattr(L, name).restype = ctypes.c_int
@@ -197,6 +198,18 @@ def acc(q, packed, N=None):
     N = packed.shape[0] if N is None else N
     out = np.empty((M, N), np.int32)
     _check(lib().oracle_acc(_ptr(q), _ptr(packed), M, N, K, _ptr(out)), "acc")
+    return out
+
+
+def acc_threads(q, packed, threads):
+    """acc() with the weight rows split over host threads (same result)."""
+    q = _c(q, np.int8)
+    packed = _c(packed, np.uint8)
+    M, K = q.shape
+    N = packed.shape[0]
+    out = np.empty((M, N), np.int32)
+    _check(lib().oracle_acc_threads(_ptr(q), _ptr(packed), M, N, K, _ptr(out), int(threads)),
+           "acc_threads")
     return out
 
 

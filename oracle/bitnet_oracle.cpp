@@ -328,6 +328,39 @@ int oracle_linear_threads_cols(const uint16_t* x, const uint8_t* packed,
   return OK;
 }
 
+// oracle_acc with the weight rows (output columns) split across host
+// threads: each thread runs the scalar definition above on its slice. Only
+// the order in which independent outputs are computed changes, so the
+// result is oracle_acc's; used where a full-size comparison needs it fast.
+int oracle_acc_threads(const int8_t* q, const uint8_t* packed, int64_t M, int64_t N, int64_t K,
+                       int32_t* acc, int nthreads) {
+  if (M < 0 || N < 0 || K < 0 || K % 4 != 0) return ERR_SHAPE;
+  if (nthreads < 1) nthreads = 1;
+  if (N < nthreads) nthreads = static_cast<int>(N > 0 ? N : 1);
+  std::vector<int> status(static_cast<size_t>(nthreads), OK);
+  std::vector<std::thread> pool;
+  const int64_t per = (N + nthreads - 1) / nthreads;
+  const int64_t KB = K / 4;
+  for (int t = 0; t < nthreads; ++t) {
+    const int64_t n0 = t * per;
+    const int64_t n1 = (n0 + per < N) ? n0 + per : N;
+    if (n0 >= n1) continue;
+    pool.emplace_back([=, &status] {
+      const int64_t nn = n1 - n0;
+      std::vector<int32_t> part(static_cast<size_t>(M) * static_cast<size_t>(nn));
+      const int s = oracle_acc(q, packed + n0 * KB, M, nn, K, part.data());
+      if (s == OK)
+        for (int64_t m = 0; m < M; ++m)
+          for (int64_t n = 0; n < nn; ++n) acc[m * N + n0 + n] = part[static_cast<size_t>(m * nn + n)];
+      status[static_cast<size_t>(t)] = s;
+    });
+  }
+  for (auto& th : pool) th.join();
+  for (int s : status)
+    if (s != OK) return s;
+  return OK;
+}
+
 // Narrowing used by the oracle, exposed so a test can pin it against a
 // library conversion on its own.
 uint16_t oracle_f32_to_bf16(float f) { return float_to_bf16_bits_rne(f); }

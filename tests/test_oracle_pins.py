@@ -479,3 +479,19 @@ def test_rmsnorm_zero_weight_gives_zero_codes():
     g = np.zeros(256, np.uint16)
     q, _ = oracle.rmsnorm_quantize(x, g, 1e-5)
     assert not q.any()
+
+
+@pytest.mark.parametrize("M,N,K,threads", [(1, 37, 64, 8), (5, 3, 128, 8), (16, 300, 256, 7),
+                                           (2, 1, 32, 4)])
+def test_acc_threads_is_the_brute_force_sum(M, N, K, threads):
+    """The threaded driver of the contraction (used by the full-size parity
+    tests) against an int64 brute-force sum of the unpacked weights: the
+    split over weight rows, including more threads than rows, changes no
+    output."""
+    rng = np.random.default_rng(M * 100 + N + K)
+    q = rng.integers(-127, 128, size=(M, K)).astype(np.int8)
+    w = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    ref = q.astype(np.int64) @ w.astype(np.int64).T
+    got = oracle.acc_threads(q, oracle.pack(w), threads)
+    assert got.dtype == np.int32
+    assert np.array_equal(got.astype(np.int64), ref)
