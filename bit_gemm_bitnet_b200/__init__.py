@@ -31,7 +31,7 @@ EXPORTS = (
     "bitnet_device_status", "bitnet_status_string", "bitnet_gemm_acc_i32",
     "bitnet_gemv_fused_debug", "bitnet_linear_noalloc", "bitnet_gemv_fused_grouped",
     "bitnet_linear_bias", "bitnet_rmsnorm_quantize_act", "bitnet_linear_rmsnorm_workspace_bytes",
-    "bitnet_linear_rmsnorm",
+    "bitnet_linear_rmsnorm", "bitnet_linear_acc_i32", "bitnet_gemv_fused_grouped_acc_i32",
 )
 
 
@@ -81,6 +81,8 @@ def lib():
             "bitnet_device_status": [P],
             "bitnet_gemm_acc_i32": [P, P, P, I64, I64, I64, P],
             "bitnet_gemv_fused_debug": [P, P, P, P, I, P, I64, I64, I64, P],
+            "bitnet_linear_acc_i32": [P, P, P, P, I, P, I64, I64, I64, P, SZ, P],
+            "bitnet_gemv_fused_grouped_acc_i32": [P, P, P, I64, I64, I, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -138,6 +140,30 @@ def _need(t, dtype, name, ndim=None):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _out(out, dtype, shape, device, name="out"):
+    """A caller-supplied output buffer, checked before anything is launched
+    (dtype, device, shape, contiguity), or a new one."""
+    if out is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    _need(out, dtype, name)
+    if tuple(out.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(out.shape)}")
+    if out.device != torch.device(device):
+        raise ValueError(f"{name} is on {out.device}, expected {device}")
+    return out
+
+
+def _out_rows(out, orig, M, N, device):
+    """bf16 output of the linear entries: shape (M, N) or the input's leading
+    dimensions followed by N; returned as an (M, N) view."""
+    if out is None:
+        return torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    if tuple(out.shape) == tuple(orig[:-1]) + (N,):
+        _need(out, torch.bfloat16, "out")
+        out = out.view(M, N)
+    return _out(out, torch.bfloat16, (M, N), device)
+
+
 def _scale_wt(scale_wt, N, device):
     """fp32 weight scale of length 1 or N (bf16 [N] is widened exactly)."""
     if not isinstance(scale_wt, torch.Tensor):
@@ -157,8 +183,7 @@ def bitnet_pack_weights(w, out=None):
     """int8 [N, K] in {-1, 0, +1} -> uint8 [N, K/4] (synchronises)."""
     _need(w, torch.int8, "w", 2)
     N, K = w.shape
-    if out is None:
-        out = torch.empty((N, K // 4), dtype=torch.uint8, device=w.device)
+    out = _out(out, torch.uint8, (N, K // 4), w.device)
     _check(lib().bitnet_pack_weights(_ptr(out), _ptr(w), N, K, _stream(w.device)),
            "bitnet_pack_weights")
     return out
@@ -170,10 +195,8 @@ def bitnet_ternarize_absmean(w, per_row=True, w_t=None, scale_wt=None):
     per tensor), ready for bitnet_pack_weights."""
     _need(w, torch.float32, "w", 2)
     N, K = w.shape
-    if w_t is None:
-        w_t = torch.empty((N, K), dtype=torch.int8, device=w.device)
-    if scale_wt is None:
-        scale_wt = torch.empty((N if per_row else 1,), dtype=torch.float32, device=w.device)
+    w_t = _out(w_t, torch.int8, (N, K), w.device, "w_t")
+    scale_wt = _out(scale_wt, torch.float32, (N if per_row else 1,), w.device, "scale_wt")
     _check(lib().bitnet_ternarize_absmean(_ptr(w_t), _ptr(scale_wt), _ptr(w), N, K,
                                           1 if per_row else 0, _stream(w.device)),
            "bitnet_ternarize_absmean")
@@ -185,10 +208,8 @@ def bitnet_quantize_act(x, x_q=None, scale_act=None):
     x2 = x.reshape(-1, x.shape[-1])
     dt = _act_dt(x2, "x", 2)
     M, K = x2.shape
-    if x_q is None:
-        x_q = torch.empty((M, K), dtype=torch.int8, device=x.device)
-    if scale_act is None:
-        scale_act = torch.empty((M,), dtype=torch.bfloat16, device=x.device)
+    x_q = _out(x_q, torch.int8, (M, K), x.device, "x_q")
+    scale_act = _out(scale_act, torch.bfloat16, (M,), x.device, "scale_act")
     _check(lib().bitnet_quantize_act(_ptr(x_q), _ptr(scale_act), _ptr(x2), dt, M, K,
                                      _stream(x.device)), "bitnet_quantize_act")
     return x_q, scale_act
@@ -203,9 +224,10 @@ def bitnet_gemm(x_q, w_packed, scale_act, scale_wt, out=None):
     N = w_packed.shape[0]
     if w_packed.shape[1] * 4 != K:
         raise ValueError(f"w_packed {tuple(w_packed.shape)} does not match K={K}")
+    if scale_act.numel() != M:
+        raise ValueError(f"scale_act has {scale_act.numel()} elements, expected M={M}")
     sw = _scale_wt(scale_wt, N, x_q.device)
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=x_q.device)
+    out = _out(out, torch.bfloat16, (M, N), x_q.device)
     _check(lib().bitnet_gemm(_ptr(out), _ptr(x_q), _ptr(w_packed), _ptr(scale_act),
                              _ptr(sw), sw.numel(), M, N, K, _stream(x_q.device)),
            "bitnet_gemm")
@@ -221,8 +243,7 @@ def bitnet_gemv_fused(x, w_packed, scale_wt, out=None):
     if w_packed.shape[1] * 4 != K:
         raise ValueError(f"w_packed {tuple(w_packed.shape)} does not match K={K}")
     sw = _scale_wt(scale_wt, N, x.device)
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    out = _out(out, torch.bfloat16, (M, N), x.device)
     _check(lib().bitnet_gemv_fused(_ptr(out), _ptr(x), dt, _ptr(w_packed), _ptr(sw),
                                    sw.numel(), M, N, K, _stream(x.device)),
            "bitnet_gemv_fused")
@@ -257,7 +278,13 @@ def bitnet_gemv_fused_grouped(xs, w_packeds, scale_wts, outs=None):
         sws.append(_scale_wt(sw, wp.shape[0], x.device))
         if outs is None:
             new_outs.append(torch.empty((M, wp.shape[0]), dtype=torch.bfloat16, device=x.device))
-    outs = outs if outs is not None else new_outs
+    if outs is None:
+        outs = new_outs
+    else:
+        if len(outs) != len(xs):
+            raise ValueError("outs must have one tensor per problem")
+        for i, (o, wp) in enumerate(zip(outs, w_packeds)):
+            _out(o, torch.bfloat16, (M, wp.shape[0]), xs[0].device, f"outs[{i}]")
     arr = gemv_problems(xs, w_packeds, sws, outs)
     _check(lib().bitnet_gemv_fused_grouped(ctypes.cast(arr, ctypes.c_void_p), len(xs), M, BF16,
                                            _stream(xs[0].device)),
@@ -284,8 +311,7 @@ def bitnet_linear(x, w_packed, scale_wt, out=None, workspace=None, bias=None):
     if w_packed.shape[1] * 4 != K:
         raise ValueError(f"w_packed {tuple(w_packed.shape)} does not match K={K}")
     sw = _scale_wt(scale_wt, N, x.device)
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    out = _out_rows(out, orig, M, N, x.device)
     need = bitnet_linear_workspace_bytes(M, K)
     if need and (workspace is None or workspace.numel() < need):
         workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
@@ -319,8 +345,7 @@ def bitnet_linear_noalloc(x, w_packed, scale_wt, out=None):
     if w_packed.shape[1] * 4 != K:
         raise ValueError(f"w_packed {tuple(w_packed.shape)} does not match K={K}")
     sw = _scale_wt(scale_wt, N, x.device)
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    out = _out_rows(out, orig, M, N, x.device)
     _check(lib().bitnet_linear_noalloc(_ptr(out), _ptr(x2), dt, _ptr(w_packed), _ptr(sw),
                                        sw.numel(), M, N, K, _stream(x.device)),
            "bitnet_linear_noalloc")
@@ -335,10 +360,8 @@ def bitnet_rmsnorm_quantize_act(x, g, eps, x_q=None, scale_act=None):
     M, K = x.shape
     if g.numel() != K:
         raise ValueError(f"g has {g.numel()} elements, expected K={K}")
-    if x_q is None:
-        x_q = torch.empty((M, K), dtype=torch.int8, device=x.device)
-    if scale_act is None:
-        scale_act = torch.empty((M,), dtype=torch.bfloat16, device=x.device)
+    x_q = _out(x_q, torch.int8, (M, K), x.device, "x_q")
+    scale_act = _out(scale_act, torch.bfloat16, (M,), x.device, "scale_act")
     _check(lib().bitnet_rmsnorm_quantize_act(_ptr(x_q), _ptr(scale_act), _ptr(x), _ptr(g),
                                              float(eps), M, K, _stream(x.device)),
            "bitnet_rmsnorm_quantize_act")
@@ -365,8 +388,7 @@ def bitnet_linear_rmsnorm(x, g, eps, w_packed, scale_wt, out=None, workspace=Non
     if g.numel() != K:
         raise ValueError(f"g has {g.numel()} elements, expected K={K}")
     sw = _scale_wt(scale_wt, N, x.device)
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    out = _out_rows(out, orig, M, N, x.device)
     need = bitnet_linear_rmsnorm_workspace_bytes(M, K)
     if need and (workspace is None or workspace.numel() < need):
         workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
@@ -391,8 +413,7 @@ def bitnet_gemm_acc_i32(x_q, w_packed, out=None):
     _need(w_packed, torch.uint8, "w_packed", 2)
     M, K = x_q.shape
     N = w_packed.shape[0]
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.int32, device=x_q.device)
+    out = _out(out, torch.int32, (M, N), x_q.device)
     _check(lib().bitnet_gemm_acc_i32(_ptr(out), _ptr(x_q), _ptr(w_packed), M, N, K,
                                      _stream(x_q.device)), "bitnet_gemm_acc_i32")
     return out
@@ -411,6 +432,59 @@ def bitnet_gemv_fused_debug(x, w_packed):
                                          _ptr(w_packed), M, N, K, _stream(x.device)),
            "bitnet_gemv_fused_debug")
     return acc, xq, sa
+
+
+def bitnet_linear_acc_i32(x, w_packed, workspace=None):
+    """bitnet_linear's dispatch and kernels with int32 sums stored instead of
+    the epilogue -> (int32 acc [M, N], int8 codes [M, K], bf16 scales [M],
+    the workspace used or None)."""
+    dt = _act_dt(x, "x", 2)
+    _need(w_packed, torch.uint8, "w_packed", 2)
+    M, K = x.shape
+    N = w_packed.shape[0]
+    if w_packed.shape[1] * 4 != K:
+        raise ValueError(f"w_packed {tuple(w_packed.shape)} does not match K={K}")
+    acc = torch.empty((M, N), dtype=torch.int32, device=x.device)
+    xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    sa = torch.empty((M,), dtype=torch.bfloat16, device=x.device)
+    need = bitnet_linear_workspace_bytes(M, K)
+    if need and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
+    _check(lib().bitnet_linear_acc_i32(_ptr(acc), _ptr(xq), _ptr(sa), _ptr(x), dt,
+                                       _ptr(w_packed), M, N, K,
+                                       _ptr(workspace) if need else None, need,
+                                       _stream(x.device)), "bitnet_linear_acc_i32")
+    return acc, xq, sa, (workspace if need else None)
+
+
+def bitnet_gemv_fused_grouped_acc_i32(xs, w_packeds):
+    """bitnet_gemv_fused_grouped's dispatch and kernel with int32 sums stored
+    -> a list of (int32 acc [M, N_i], int8 codes [M, K_i], bf16 scales [M])."""
+    if len(xs) != len(w_packeds):
+        raise ValueError("xs and w_packeds must have the same length")
+    if len(xs) == 0:
+        return []
+    M = xs[0].shape[0]
+    dev = xs[0].device
+    res, keep = [], []
+    for i, (x, wp) in enumerate(zip(xs, w_packeds)):
+        _need(x, torch.bfloat16, f"xs[{i}]", 2)
+        _need(wp, torch.uint8, f"w_packeds[{i}]", 2)
+        if x.shape[0] != M or wp.shape[1] * 4 != x.shape[1]:
+            raise ValueError(f"problem {i}: shapes {tuple(x.shape)}, {tuple(wp.shape)}")
+        res.append((torch.empty((M, wp.shape[0]), dtype=torch.int32, device=dev),
+                    torch.empty((M, x.shape[1]), dtype=torch.int8, device=dev),
+                    torch.empty((M,), dtype=torch.bfloat16, device=dev)))
+        keep.append(torch.ones(1, dtype=torch.float32, device=dev))
+    arr = gemv_problems(xs, w_packeds, keep, [r[0] for r in res])
+    qs = (ctypes.c_void_p * len(xs))(*[r[1].data_ptr() for r in res])
+    sas = (ctypes.c_void_p * len(xs))(*[r[2].data_ptr() for r in res])
+    _check(lib().bitnet_gemv_fused_grouped_acc_i32(ctypes.cast(arr, ctypes.c_void_p),
+                                                   ctypes.cast(qs, ctypes.c_void_p),
+                                                   ctypes.cast(sas, ctypes.c_void_p), len(xs), M,
+                                                   BF16, _stream(dev)),
+           "bitnet_gemv_fused_grouped_acc_i32")
+    return res
 
 
 # the page's Python names

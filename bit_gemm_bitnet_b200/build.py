@@ -14,6 +14,10 @@ OUT = os.path.join(HERE, "libbitnet_b200.so")
 SOURCES = [os.path.join(CSRC, "bitnet.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
     os.path.join(ROOT, "include", "bitnet.h")]
+# The failure-path test library (tests only): the decode GEMV with a 1 ms
+# wait limit and a stage its producer can be told to leave out.
+WAIT_TEST_OUT = os.path.join(HERE, "libbitnet_b200_waittest.so")
+WAIT_TEST_SOURCES = [os.path.join(CSRC, "wait_test.cu")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
@@ -24,14 +28,22 @@ def flags():
             "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and os.path.exists(OUT):
-        t = os.path.getmtime(OUT)
-        if all(os.path.getmtime(d) <= t for d in DEPS):
-            return OUT
-    cmd = [NVCC] + flags() + (["-Xptxas", "-v"] if verbose else []) + SOURCES + ["-o", OUT]
+def _build_one(sources, out, force, verbose):
+    deps = DEPS + sources
+    if not force and os.path.exists(out):
+        t = os.path.getmtime(out)
+        if all(os.path.getmtime(d) <= t for d in deps):
+            return out
+    cmd = [NVCC] + flags() + (["-Xptxas", "-v"] if verbose else []) + sources + ["-o", out]
     subprocess.check_call(cmd)
-    return OUT
+    return out
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Build the product library (and the failure-path test library);
+    returns the product library's path."""
+    _build_one(WAIT_TEST_SOURCES, WAIT_TEST_OUT, force, verbose)
+    return _build_one(SOURCES, OUT, force, verbose)
 
 
 if __name__ == "__main__":

@@ -77,6 +77,7 @@ struct DeviceInfo {
 
 DeviceInfo g_dev[64];
 std::mutex g_mu;
+std::mutex g_mu_hook;  // the grouped accumulator hook's parameter block
 
 bitnet_status device_info(DeviceInfo** out) {
   int dev = 0;
@@ -352,10 +353,10 @@ void partition_units(GroupedParams& gp, int grid, int cw) {
   while (c <= grid) gp.cta_u0[c++] = gp.units;
 }
 
-template <int MB, int RW_MAX>
-bitnet_status launch_grouped_t(GroupedParams& gp, size_t smem, int sms, cudaStream_t st) {
+template <int MB, int RW_MAX, bool ACC, typename P>
+bitnet_status launch_grouped_t(P& gp, size_t smem, int sms, cudaStream_t st) {
   constexpr int cw = grouped_cw(MB);
-  auto k = gemv_grouped_kernel<cw, MB, RW_MAX>;
+  auto k = gemv_grouped_kernel<cw, MB, RW_MAX, ACC, P>;
   constexpr int threads = (cw + 1) * 32;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
@@ -377,12 +378,15 @@ bitnet_status launch_grouped_t(GroupedParams& gp, size_t smem, int sms, cudaStre
 constexpr int grouped_rw_max(int mb) { return mb == 1 ? 8 : mb == 2 ? 4 : mb == 4 ? 8 : mb == 8 ? 4 : 1; }
 
 // Launch up to kGroupMax problems (all K % 64 == 0, validated) in one kernel.
-bitnet_status run_gemv_grouped(const bitnet_gemv_problem* pr, int count, int M, cudaStream_t st) {
+// ACC: the accumulator hook (P = GroupedDebugParams, its debug pointers set
+// by the caller); the partition and the launch are the product's.
+template <bool ACC, typename P>
+bitnet_status run_gemv_grouped_t(P& gp, const bitnet_gemv_problem* pr, int count, int M,
+                                 cudaStream_t st) {
   DeviceInfo* dev = nullptr;
   bitnet_status s = device_info(&dev);
   if (s != BITNET_OK) return s;
-  static_assert(sizeof(GroupedParams) <= 32000, "kernel parameter space");
-  GroupedParams gp;
+  static_assert(sizeof(P) <= 32000, "kernel parameter space");
   gp.count = count;
   gp.M = M;
   const int mb = bucket_of(M);
@@ -443,12 +447,30 @@ bitnet_status run_gemv_grouped(const bitnet_gemv_problem* pr, int count, int M, 
   const size_t smem = kGemvHeaderBytes + gp.q_bytes + static_cast<size_t>(stages) * stage;
   if (smem > kSmemLimit) return BITNET_ERR_SHAPE;
   switch (mb) {
-    case 1: return launch_grouped_t<1, grouped_rw_max(1)>(gp, smem, dev->sms, st);
-    case 2: return launch_grouped_t<2, grouped_rw_max(2)>(gp, smem, dev->sms, st);
-    case 4: return launch_grouped_t<4, grouped_rw_max(4)>(gp, smem, dev->sms, st);
-    case 8: return launch_grouped_t<8, grouped_rw_max(8)>(gp, smem, dev->sms, st);
-    default: return launch_grouped_t<16, grouped_rw_max(16)>(gp, smem, dev->sms, st);
+    case 1: return launch_grouped_t<1, grouped_rw_max(1), ACC>(gp, smem, dev->sms, st);
+    case 2: return launch_grouped_t<2, grouped_rw_max(2), ACC>(gp, smem, dev->sms, st);
+    case 4: return launch_grouped_t<4, grouped_rw_max(4), ACC>(gp, smem, dev->sms, st);
+    case 8: return launch_grouped_t<8, grouped_rw_max(8), ACC>(gp, smem, dev->sms, st);
+    default: return launch_grouped_t<16, grouped_rw_max(16), ACC>(gp, smem, dev->sms, st);
   }
+}
+
+bitnet_status run_gemv_grouped(const bitnet_gemv_problem* pr, int count, int M, cudaStream_t st) {
+  GroupedParams gp;
+  return run_gemv_grouped_t<false>(gp, pr, count, M, st);
+}
+
+// The accumulator hook of the grouped launch: problem i's `out` is its int32
+// [M, N] output; its codes and scales go to q[i] and sa[i].
+bitnet_status run_gemv_grouped_acc(const bitnet_gemv_problem* pr, int8_t* const* q,
+                                   uint16_t* const* sa, int count, int M, cudaStream_t st) {
+  static GroupedDebugParams gp;  // 18 KB: kept off the stack (the hook's calls are serialised)
+  std::lock_guard<std::mutex> lock(g_mu_hook);
+  for (int i = 0; i < count; ++i) {
+    gp.dbg_q[i] = q[i];
+    gp.dbg_sa[i] = sa[i];
+  }
+  return run_gemv_grouped_t<true>(gp, pr, count, M, st);
 }
 
 // ---------------------------------------------------------------- GEMM
@@ -536,6 +558,7 @@ bitnet_status run_sk_bx(void* out, bool acc_out, const int8_t* xq, const uint8_t
   if (!make_map_u8(&mx, xq, M, K, K, BX, sk::BK, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_u8(&mw, wp, N, K / 4, K / 4, sk::BW, sk::BK / 4, CU_TENSOR_MAP_SWIZZLE_NONE))
     return BITNET_ERR_CUDA;
+  if (acc_out && perm) return launch_sk<BX, true, true>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st, nullptr);
   if (acc_out) return launch_sk<BX, true, false>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st, nullptr);
   if (perm) return launch_sk<BX, false, true>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st, bias);
   return launch_sk<BX, false, false>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st, bias);
@@ -560,10 +583,13 @@ bool skq_ok(const void* x, const uint8_t* wp, int64_t M, int64_t K) {
   return M >= kSkqMinRows && M <= skq::BX && K % 64 == 0 && aligned(x, 16) && aligned(wp, 16);
 }
 
-bitnet_status run_gemv_skq(uint16_t* out, const uint16_t* x, const uint8_t* wp,
+// acc_out (the accumulator hook): int32 sums to `out`, codes to dbg_q and
+// scales to dbg_sa, from the same kernel with the epilogue replaced.
+bitnet_status run_gemv_skq(void* out, const uint16_t* x, const uint8_t* wp,
                            const float* sw, int64_t sw_len, int64_t M, int64_t N, int64_t K,
-                           cudaStream_t st, const uint16_t* bias) {
-  auto kernel = skq::gemv_i8_skq_kernel;
+                           cudaStream_t st, const uint16_t* bias, bool acc_out = false,
+                           int8_t* dbg_q = nullptr, uint16_t* dbg_sa = nullptr) {
+  auto kernel = acc_out ? skq::gemv_i8_skq_kernel<true> : skq::gemv_i8_skq_kernel<false>;
   constexpr int smem = skq::SMEM_BYTES;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
@@ -595,7 +621,7 @@ bitnet_status run_gemv_skq(uint16_t* out, const uint16_t* x, const uint8_t* wp,
   return launch_pdl_cluster(kernel, dim3(static_cast<unsigned>(w_tiles * best)),
                             dim3(skq::NUM_THREADS), smem, best, st, mw, out, x, sw,
                             static_cast<int>(sw_len), static_cast<int>(M), static_cast<int>(N),
-                            static_cast<int>(K), best, bias);
+                            static_cast<int>(K), best, bias, dbg_q, dbg_sa);
 }
 
 // perm: x_q has transposed 16-element groups and rowsum holds its per-row
@@ -641,6 +667,7 @@ bitnet_status run_gemm(void* out, bool acc_out, const int8_t* xq, const uint8_t*
                       out, sa, sw, static_cast<int>(sw_len), rowsum, static_cast<int>(M),
                       static_cast<int>(N), static_cast<int>(K), acc_out ? nullptr : bias);
   };
+  if (acc_out && perm) return go(ts::gemm_i8_ts_kernel<true, true>);
   if (acc_out) return go(ts::gemm_i8_ts_kernel<true, false>);
   if (perm) return go(ts::gemm_i8_ts_kernel<false, true>);
   return go(ts::gemm_i8_ts_kernel<false, false>);
@@ -700,6 +727,36 @@ bitnet_status run_quantize_perm(int8_t* xq, uint16_t* sa, int32_t* rowsum, const
 }
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+// Accumulator hook only: the workspace's codes back in natural order (the
+// tensor-core layout transposes every 16-element group 4 x 4, its own
+// inverse) and its scales, into the hook's outputs.
+__global__ void unpermute_codes_kernel(int8_t* __restrict__ dst, const int8_t* __restrict__ src,
+                                       int64_t groups) {
+  for (int64_t g = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; g < groups;
+       g += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    reinterpret_cast<uint4*>(dst)[g] = transpose16(reinterpret_cast<const uint4*>(src)[g]);
+}
+
+bitnet_status copy_workspace_codes(int8_t* q, uint16_t* sa, const int8_t* ws_q,
+                                   const uint16_t* ws_sa, int64_t M, int64_t K, bool permuted,
+                                   cudaStream_t st) {
+  const int64_t bytes = M * K;
+  if (permuted) {
+    const int64_t groups = bytes / 16;
+    int64_t blocks = (groups + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    unpermute_codes_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(q, ws_q, groups);
+    if (cudaGetLastError() != cudaSuccess) return BITNET_ERR_CUDA;
+  } else if (cudaMemcpyAsync(q, ws_q, static_cast<size_t>(bytes), cudaMemcpyDeviceToDevice, st) !=
+             cudaSuccess) {
+    return BITNET_ERR_CUDA;
+  }
+  if (cudaMemcpyAsync(sa, ws_sa, static_cast<size_t>(M) * 2, cudaMemcpyDeviceToDevice, st) !=
+      cudaSuccess)
+    return BITNET_ERR_CUDA;
+  return BITNET_OK;
+}
 
 bool linear_uses_gemv(int64_t M, int64_t K) {
   return M >= 1 && M <= kLinearGemvMaxM && K <= INT32_MAX && gemv_fits(static_cast<int>(M), K);
@@ -875,30 +932,54 @@ static bitnet_status gemv_common(GemvParams& p, const void* x, bitnet_dtype dt,
   return BITNET_OK;
 }
 
+// Where the accumulator hooks send their results: int32 sums instead of the
+// bf16 outputs, and the int8 codes [M, K] (natural order) and bf16 scales [M]
+// the path quantised. Null for every product call.
+struct AccHook {
+  int32_t* acc;
+  int8_t* q;
+  uint16_t* sa;
+};
+
+// The fused GEMV's dispatch (shared by bitnet_gemv_fused, bitnet_linear at
+// M < 16 and the accumulator hook): the tensor-core GEMV for 8 <= M < 16
+// where it applies, else the dp4a GEMV.
 static bitnet_status gemv_fused_impl(uint16_t* out, const void* x, bitnet_dtype dt,
                                      const uint8_t* w_packed, const float* scale_wt,
                                      int64_t scale_wt_len, const uint16_t* bias, int64_t M,
                                      int64_t N, int64_t K, void* stream,
-                                     const uint16_t* norm_g = nullptr, float norm_eps = 0.0f) {
+                                     const uint16_t* norm_g = nullptr, float norm_eps = 0.0f,
+                                     const AccHook* hook = nullptr) {
   GemvParams p = {};
   bitnet_status s = gemv_common(p, x, dt, w_packed, M, N, K);
   if (s != BITNET_OK) return s;
   if (N == 0) return BITNET_OK;
-  if (out == nullptr) return BITNET_ERR_NULL;
-  if (!aligned(out, 16)) return BITNET_ERR_ALIGN;
-  s = check_scale_wt(scale_wt, scale_wt_len, N);
-  if (s != BITNET_OK) return s;
-  if (bias != nullptr && !aligned(bias, 2)) return BITNET_ERR_ALIGN;
-  p.out = out;
-  p.sw = scale_wt;
-  p.sw_len = static_cast<int>(scale_wt_len);
-  p.bias = bias;
+  if (hook == nullptr) {
+    if (out == nullptr) return BITNET_ERR_NULL;
+    if (!aligned(out, 16)) return BITNET_ERR_ALIGN;
+    s = check_scale_wt(scale_wt, scale_wt_len, N);
+    if (s != BITNET_OK) return s;
+    if (bias != nullptr && !aligned(bias, 2)) return BITNET_ERR_ALIGN;
+    p.out = out;
+    p.sw = scale_wt;
+    p.sw_len = static_cast<int>(scale_wt_len);
+    p.bias = bias;
+  } else {
+    p.acc_out = hook->acc;
+    p.dbg_q = hook->q;
+    p.dbg_sa = hook->sa;
+    p.sw_len = 1;
+  }
   p.norm_g = norm_g;
   p.norm_eps = norm_eps;
   if (norm_g == nullptr && dt == BITNET_BF16 && skq_ok(x, w_packed, M, K) &&
       K / 128 <= sk::MAX_SPLIT * skq::MAX_KB) {
-    const bitnet_status r = run_gemv_skq(out, static_cast<const uint16_t*>(x), w_packed,
-                                         scale_wt, scale_wt_len, M, N, K, as_stream(stream), bias);
+    const bitnet_status r =
+        hook == nullptr
+            ? run_gemv_skq(out, static_cast<const uint16_t*>(x), w_packed, scale_wt,
+                           scale_wt_len, M, N, K, as_stream(stream), bias)
+            : run_gemv_skq(hook->acc, static_cast<const uint16_t*>(x), w_packed, nullptr, 1, M,
+                           N, K, as_stream(stream), nullptr, true, hook->q, hook->sa);
     if (r != BITNET_ERR_SHAPE) return r;
   }
   return run_gemv(p, false, as_stream(stream));
@@ -911,12 +992,18 @@ bitnet_status bitnet_gemv_fused(uint16_t* out, const void* x, bitnet_dtype dt,
   return gemv_fused_impl(out, x, dt, w_packed, scale_wt, scale_wt_len, nullptr, M, N, K, stream);
 }
 
-bitnet_status bitnet_gemv_fused_grouped(const bitnet_gemv_problem* problems, int64_t count,
-                                        int64_t M, bitnet_dtype dt, void* stream) {
+// The grouped GEMV's dispatch: problems with K % 64 == 0 and bf16 rows go
+// to the grouped kernel, up to kGroupMax per launch; the rest are single
+// calls. hq / hsa (the accumulator hook, else null): where each problem's
+// codes and scales go; each problem's `out` is then its int32 output.
+static bitnet_status grouped_impl(const bitnet_gemv_problem* problems, int64_t count, int64_t M,
+                                  bitnet_dtype dt, void* stream, int8_t* const* hq,
+                                  uint16_t* const* hsa) {
   if (dt != BITNET_BF16 && dt != BITNET_F32) return BITNET_ERR_DTYPE;
   if (count < 0) return BITNET_ERR_SHAPE;
   if (count == 0) return BITNET_OK;
   if (problems == nullptr) return BITNET_ERR_NULL;
+  const bool hook = hq != nullptr;
   // validate everything before anything is enqueued
   for (int64_t i = 0; i < count; ++i) {
     const bitnet_gemv_problem& q = problems[i];
@@ -926,30 +1013,66 @@ bitnet_status bitnet_gemv_fused_grouped(const bitnet_gemv_problem* problems, int
     if (q.N == 0) continue;
     if (q.out == nullptr) return BITNET_ERR_NULL;
     if (!aligned(q.out, 16)) return BITNET_ERR_ALIGN;
-    s = check_scale_wt(q.scale_wt, q.scale_wt_len, q.N);
-    if (s != BITNET_OK) return s;
+    if (hook) {
+      if (hq[i] == nullptr || hsa[i] == nullptr) return BITNET_ERR_NULL;
+      if (!aligned(hq[i], 16) || !aligned(hsa[i], 2)) return BITNET_ERR_ALIGN;
+    } else {
+      s = check_scale_wt(q.scale_wt, q.scale_wt_len, q.N);
+      if (s != BITNET_OK) return s;
+    }
   }
   cudaStream_t st = as_stream(stream);
   bitnet_gemv_problem batch[kGroupMax];
+  int8_t* bq[kGroupMax];
+  uint16_t* bsa[kGroupMax];
   int n = 0;
+  auto flush = [&]() -> bitnet_status {
+    const int k = n;
+    n = 0;
+    return hook ? run_gemv_grouped_acc(batch, bq, bsa, k, static_cast<int>(M), st)
+                : run_gemv_grouped(batch, k, static_cast<int>(M), st);
+  };
   for (int64_t i = 0; i < count; ++i) {
     const bitnet_gemv_problem& q = problems[i];
     if (q.N == 0) continue;
     if (q.K % 64 != 0 || dt == BITNET_F32) {  // its own launch (the grouped kernel reads bf16)
-      bitnet_status s = bitnet_gemv_fused(q.out, q.x, dt, q.w_packed, q.scale_wt,
-                                          q.scale_wt_len, M, q.N, q.K, stream);
+      bitnet_status s;
+      if (hook) {
+        const AccHook h{static_cast<int32_t*>(static_cast<void*>(q.out)), hq[i], hsa[i]};
+        s = gemv_fused_impl(nullptr, q.x, dt, q.w_packed, nullptr, 1, nullptr, M, q.N, q.K, stream,
+                            nullptr, 0.0f, &h);
+      } else {
+        s = bitnet_gemv_fused(q.out, q.x, dt, q.w_packed, q.scale_wt, q.scale_wt_len, M, q.N,
+                              q.K, stream);
+      }
       if (s != BITNET_OK) return s;
       continue;
     }
-    batch[n++] = q;
-    if (n == kGroupMax) {
-      bitnet_status s = run_gemv_grouped(batch, n, static_cast<int>(M), st);
+    batch[n] = q;
+    if (hook) {
+      bq[n] = hq[i];
+      bsa[n] = hsa[i];
+    }
+    if (++n == kGroupMax) {
+      bitnet_status s = flush();
       if (s != BITNET_OK) return s;
-      n = 0;
     }
   }
-  if (n > 0) return run_gemv_grouped(batch, n, static_cast<int>(M), st);
+  if (n > 0) return flush();
   return BITNET_OK;
+}
+
+bitnet_status bitnet_gemv_fused_grouped(const bitnet_gemv_problem* problems, int64_t count,
+                                        int64_t M, bitnet_dtype dt, void* stream) {
+  return grouped_impl(problems, count, M, dt, stream, nullptr, nullptr);
+}
+
+bitnet_status bitnet_gemv_fused_grouped_acc_i32(const bitnet_gemv_problem* problems,
+                                                int8_t* const* x_q, uint16_t* const* scale_act,
+                                                int64_t count, int64_t M, bitnet_dtype dt,
+                                                void* stream) {
+  if (count > 0 && (x_q == nullptr || scale_act == nullptr)) return BITNET_ERR_NULL;
+  return grouped_impl(problems, count, M, dt, stream, x_q, scale_act);
 }
 
 bitnet_status bitnet_gemv_fused_debug(int32_t* acc, int8_t* x_q, uint16_t* scale_act,
@@ -977,25 +1100,33 @@ size_t bitnet_linear_workspace_bytes(int64_t M, int64_t K) {
          align256(static_cast<size_t>(M) * 2) + align256(static_cast<size_t>(M) * 4);
 }
 
+// bitnet_linear's dispatch (shared with bitnet_linear_bias,
+// bitnet_linear_noalloc and the accumulator hook): M < 16 -> the fused GEMV;
+// else the quantiser into the workspace, then the GEMM.
 static bitnet_status linear_impl(uint16_t* out, const void* x, bitnet_dtype dt,
                                  const uint8_t* w_packed, const float* scale_wt,
                                  int64_t scale_wt_len, const uint16_t* bias, int64_t M, int64_t N,
                                  int64_t K, void* workspace, size_t workspace_bytes,
-                                 void* stream) {
+                                 void* stream, const AccHook* hook = nullptr) {
   if (dt != BITNET_BF16 && dt != BITNET_F32) return BITNET_ERR_DTYPE;
   bitnet_status s = check_compute_shape(M, N, K);
   if (s != BITNET_OK) return s;
   if (M == 0 || N == 0) return BITNET_OK;
   if (linear_uses_gemv(M, K))
-    return gemv_fused_impl(out, x, dt, w_packed, scale_wt, scale_wt_len, bias, M, N, K, stream);
+    return gemv_fused_impl(out, x, dt, w_packed, scale_wt, scale_wt_len, bias, M, N, K, stream,
+                           nullptr, 0.0f, hook);
   if (bias != nullptr && !aligned(bias, 2)) return BITNET_ERR_ALIGN;
   const size_t need = bitnet_linear_workspace_bytes(M, K);
   if (workspace == nullptr || workspace_bytes < need) return BITNET_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return BITNET_ERR_ALIGN;
-  if (out == nullptr || x == nullptr || w_packed == nullptr) return BITNET_ERR_NULL;
-  s = check_scale_wt(scale_wt, scale_wt_len, N);
-  if (s != BITNET_OK) return s;
-  if (!aligned(out, 16) || !aligned(x, 16) || !aligned(w_packed, 16)) return BITNET_ERR_ALIGN;
+  if (x == nullptr || w_packed == nullptr) return BITNET_ERR_NULL;
+  if (hook == nullptr) {
+    if (out == nullptr) return BITNET_ERR_NULL;
+    s = check_scale_wt(scale_wt, scale_wt_len, N);
+    if (s != BITNET_OK) return s;
+    if (!aligned(out, 16)) return BITNET_ERR_ALIGN;
+  }
+  if (!aligned(x, 16) || !aligned(w_packed, 16)) return BITNET_ERR_ALIGN;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int8_t* xq = reinterpret_cast<int8_t*>(ws);
   uint16_t* sa = reinterpret_cast<uint16_t*>(ws + align256(static_cast<size_t>(M) * K));
@@ -1004,18 +1135,23 @@ static bitnet_status linear_impl(uint16_t* out, const void* x, bitnet_dtype dt,
   cudaStream_t st = as_stream(stream);
   const uint16_t* xb = static_cast<const uint16_t*>(x);
   const float* xf = static_cast<const float*>(x);
-  if (gemm_tc_ok(xq, w_packed, K)) {
+  const bool tc = gemm_tc_ok(xq, w_packed, K);
+  if (tc) {
     // tensor-core path: transposed groups + row sums, weights as code planes
     s = dt == BITNET_F32 ? run_quantize_perm_f32(xq, sa, rowsum, xf, M, K, st)
                          : run_quantize_perm(xq, sa, rowsum, xb, M, K, st);
-    if (s != BITNET_OK) return s;
-    return run_gemm(out, false, xq, w_packed, sa, scale_wt, scale_wt_len, M, N, K, st, true,
-                    rowsum, bias);
+  } else {
+    s = dt == BITNET_F32 ? run_quantize_f32(xq, sa, xf, M, K, st)
+                         : run_quantize(xq, sa, xb, M, K, st);
   }
-  s = dt == BITNET_F32 ? run_quantize_f32(xq, sa, xf, M, K, st) : run_quantize(xq, sa, xb, M, K, st);
   if (s != BITNET_OK) return s;
-  return run_gemm(out, false, xq, w_packed, sa, scale_wt, scale_wt_len, M, N, K, st, false,
-                  nullptr, bias);
+  if (hook == nullptr)
+    return run_gemm(out, false, xq, w_packed, sa, scale_wt, scale_wt_len, M, N, K, st, tc,
+                    tc ? rowsum : nullptr, bias);
+  s = run_gemm(hook->acc, true, xq, w_packed, sa, nullptr, 1, M, N, K, st, tc,
+               tc ? rowsum : nullptr, nullptr);
+  if (s != BITNET_OK) return s;
+  return copy_workspace_codes(hook->q, hook->sa, xq, sa, M, K, tc, st);
 }
 
 bitnet_status bitnet_linear(uint16_t* out, const void* x, bitnet_dtype dt,
@@ -1034,6 +1170,21 @@ bitnet_status bitnet_linear_bias(uint16_t* out, const void* x, bitnet_dtype dt,
   if (bias == nullptr) return BITNET_ERR_NULL;
   return linear_impl(out, x, dt, w_packed, scale_wt, scale_wt_len, bias, M, N, K, workspace,
                      workspace_bytes, stream);
+}
+
+bitnet_status bitnet_linear_acc_i32(int32_t* acc, int8_t* x_q, uint16_t* scale_act,
+                                    const void* x, bitnet_dtype dt, const uint8_t* w_packed,
+                                    int64_t M, int64_t N, int64_t K, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  if (dt != BITNET_BF16 && dt != BITNET_F32) return BITNET_ERR_DTYPE;
+  bitnet_status s = check_compute_shape(M, N, K);
+  if (s != BITNET_OK) return s;
+  if (M == 0 || N == 0) return BITNET_OK;
+  if (acc == nullptr || x_q == nullptr || scale_act == nullptr) return BITNET_ERR_NULL;
+  if (!aligned(acc, 16) || !aligned(x_q, 16) || !aligned(scale_act, 2)) return BITNET_ERR_ALIGN;
+  const AccHook hook{acc, x_q, scale_act};
+  return linear_impl(nullptr, x, dt, w_packed, nullptr, 1, nullptr, M, N, K, workspace,
+                     workspace_bytes, stream, &hook);
 }
 
 bitnet_status bitnet_linear_noalloc(uint16_t* out, const void* x, bitnet_dtype dt,

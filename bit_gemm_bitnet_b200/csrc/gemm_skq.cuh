@@ -96,11 +96,17 @@ __device__ __forceinline__ int sw128_off(int m, int kk) {
 
 // Grid: (N / BW tiles) x S CTAs, clusters of S consecutive CTAs; 1 <= M <= 16;
 // K % 64 == 0; x 16-byte aligned. Outputs bf16 [M, N].
+// kAccOut (the accumulator hook): the same kernel storing the int32 sums to
+// `out` read as int32 [M, N]; every CTA also writes its slice's codes to
+// dbg_q (int8 [M, K], natural order) and the CTAs of the first tile the
+// scales to dbg_sa (bf16 [M]).
+template <bool kAccOut>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    gemv_i8_skq_kernel(const __grid_constant__ CUtensorMap tmap_w, uint16_t* __restrict__ out,
+    gemv_i8_skq_kernel(const __grid_constant__ CUtensorMap tmap_w, void* __restrict__ out,
                        const uint16_t* __restrict__ x, const float* __restrict__ scale_wt,
                        int sw_len, int M, int N, int K, int S,
-                       const uint16_t* __restrict__ bias) {
+                       const uint16_t* __restrict__ bias, int8_t* __restrict__ dbg_q,
+                       uint16_t* __restrict__ dbg_sa) {
   extern __shared__ uint8_t smem_raw[];
   Smem sm;
   sm.base = reinterpret_cast<uint8_t*>(
@@ -204,6 +210,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       qs = rq.s;
       qr = rq.r;
       sa = bf16_bits_to_f32(f32_to_bf16_bits(rq.s));
+      if (kAccOut && blockIdx.x < static_cast<unsigned>(S)) dbg_sa[tid] = f32_to_bf16_bits(rq.s);
     }
     sm.rq_s()[tid] = qs;
     sm.rq_r()[tid] = qr;
@@ -228,6 +235,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int kk = 4 * u;
       *reinterpret_cast<uint32_t*>(sm.xt(kk / BK) + sw128_off(m, kk % BK)) =
           q0 | (q1 << 8) | (q2 << 16) | (q3 << 24);
+      if constexpr (kAccOut)
+        *reinterpret_cast<uint32_t*>(dbg_q + static_cast<int64_t>(m) * K + k0 + kk) =
+            q0 | (q1 << 8) | (q2 << 16) | (q3 << 24);
     }
   }
   {
@@ -356,6 +366,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           a[2] += static_cast<int>(v[q].z);
           a[3] += static_cast<int>(v[q].w);
         }
+      if constexpr (kAccOut) {
+        int32_t* o = static_cast<int32_t*>(out) + static_cast<int64_t>(m) * N + n;
+        if (n + 3 < N && (N & 3) == 0) {
+          *reinterpret_cast<int4*>(o) = make_int4(a[0], a[1], a[2], a[3]);
+        } else {
+          for (int j = 0; j < 4 && n + j < N; ++j) o[j] = a[j];
+        }
+        continue;
+      }
       const float sa = sm.saf()[m];
       uint16_t y[4];
 #pragma unroll
@@ -364,7 +383,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         y[j] = f32_to_bf16_bits(__fmul_rn(__fmul_rn(__int2float_rn(a[j]), sa), swj));
         if (bias != nullptr && n + j < N) y[j] = add_bias_bf16(y[j], bias, n + j);
       }
-      uint16_t* o = out + static_cast<int64_t>(m) * N + n;
+      uint16_t* o = static_cast<uint16_t*>(out) + static_cast<int64_t>(m) * N + n;
       if (n + 3 < N && (N & 3) == 0) {
         *reinterpret_cast<uint2*>(o) =
             make_uint2(static_cast<uint32_t>(y[0]) | (static_cast<uint32_t>(y[1]) << 16),

@@ -36,6 +36,13 @@ constexpr int kGemvHeaderBytes = 2048;
 constexpr int kGemvStageTarget = 40 * 1024;  // bytes per stage (aim)
 constexpr int kGemvRingTarget = 160 * 1024;  // bytes of stages per CTA (aim)
 
+#ifdef BITNET_WAIT_TEST
+// Failure-path test library only (never in the product library): the ring
+// index whose copy CTA 0's producer leaves out, or -1. The consumers waiting
+// for that stage then give up their bounded wait.
+__device__ int g_wait_test_skip = -1;
+#endif
+
 struct GemvParams {
   uint16_t* out;          // bf16 [M, N], or
   int32_t* acc_out;       // int32 [M, N] (test hook)
@@ -260,7 +267,7 @@ __device__ __forceinline__ int q_pos(int g, int full_end) {
 // eps) from the exact sum of squares and quantises z = bf16(g * bf16(x * r)).
 template <int CW, int MB, int NQ, bool QUAD, bool NORM>
 __device__ __forceinline__ void gemv_stage_cached(const GemvSmem& sh, const uint16_t* __restrict__ x,
-                                                  int K, int Mc, uint16_t* dbg_sa,
+                                                  int K, int Mc, int8_t* dbg_q, uint16_t* dbg_sa,
                                                   const uint16_t* __restrict__ norm_g,
                                                   float norm_eps) {
   constexpr int kGemvConsumerWarps = CW;
@@ -390,6 +397,10 @@ __device__ __forceinline__ void gemv_stage_cached(const GemvSmem& sh, const uint
           d[4] = static_cast<uint8_t>(q1);
           d[8] = static_cast<uint8_t>(q2);
           d[12] = static_cast<uint8_t>(q3);
+          if (dbg_q != nullptr)
+            reinterpret_cast<uint32_t*>(dbg_q + static_cast<int64_t>(m) * K)[u] =
+                (static_cast<uint32_t>(q0) & 0xFFu) | ((static_cast<uint32_t>(q1) & 0xFFu) << 8) |
+                ((static_cast<uint32_t>(q2) & 0xFFu) << 16) | (static_cast<uint32_t>(q3) << 24);
         }
       }
     }
@@ -424,12 +435,12 @@ __device__ __forceinline__ void gemv_stage_activations(const GemvSmem& sh, const
   const int quads = K / 4;
   if constexpr (CACHE && MB <= 2) {
     const uint16_t* xb = static_cast<const uint16_t*>(x);
-    if (!f32 && dbg_q == nullptr && quads <= 4 * kGemvConsumers) {
-      gemv_stage_cached<CW, MB, 4, QUAD, NORM>(sh, xb, K, Mc, dbg_sa, norm_g, norm_eps);
+    if (!f32 && quads <= 4 * kGemvConsumers) {
+      gemv_stage_cached<CW, MB, 4, QUAD, NORM>(sh, xb, K, Mc, dbg_q, dbg_sa, norm_g, norm_eps);
       return;
     }
-    if (!f32 && dbg_q == nullptr && quads <= 8 * kGemvConsumers) {
-      gemv_stage_cached<CW, MB, 8, QUAD, NORM>(sh, xb, K, Mc, dbg_sa, norm_g, norm_eps);
+    if (!f32 && quads <= 8 * kGemvConsumers) {
+      gemv_stage_cached<CW, MB, 8, QUAD, NORM>(sh, xb, K, Mc, dbg_q, dbg_sa, norm_g, norm_eps);
       return;
     }
   }
@@ -648,11 +659,17 @@ __global__ void __launch_bounds__((CW + 1) * 32) gemv_kernel(GemvParams p) {
   if (warp == kGemvConsumerWarps) {
     // ------------------------------------------------------------ producer
     // Weights do not depend on the previous kernel: no griddepcontrol.wait.
+#ifdef BITNET_WAIT_TEST
+    const int skip = blockIdx.x == 0 ? g_wait_test_skip : -1;
+#endif
     uint32_t it = 0;
     for (int b = blockIdx.x; b < nblocks; b += gridDim.x, ++it) {
       const int s = it % S;
       const uint32_t ph = (it / S) & 1u;
       if (!mbar_wait(empty(s), ph ^ 1u, abort)) break;
+#ifdef BITNET_WAIT_TEST
+      if (static_cast<int>(it) == skip) continue;  // this stage is never filled
+#endif
       const int n0 = b * RPB;
       const int rows = min(RPB, N - n0);
       const uint8_t* src = p.wp + static_cast<int64_t>(n0) * KB;
@@ -671,7 +688,12 @@ __global__ void __launch_bounds__((CW + 1) * 32) gemv_kernel(GemvParams p) {
     }
     // drain: every copy issued has landed before the CTA may exit
     const uint32_t first = it > static_cast<uint32_t>(S) ? it - S : 0u;
-    for (uint32_t j = first; j < it; ++j) mbar_wait_drain(full(j % S), (j / S) & 1u);
+    for (uint32_t j = first; j < it; ++j) {
+#ifdef BITNET_WAIT_TEST
+      if (static_cast<int>(j) == skip) continue;  // nothing was requested there
+#endif
+      mbar_wait_drain(full(j % S), (j / S) & 1u);
+    }
     return;
   }
 

@@ -43,12 +43,20 @@ struct GroupedParams {
   const uint16_t* x[kGroupMax];
   const uint8_t* wp[kGroupMax];
   const float* sw[kGroupMax];
-  uint16_t* out[kGroupMax];
+  uint16_t* out[kGroupMax];   // bf16 [M, N]; int32 [M, N] in the accumulator hook
+};
+
+// The accumulator hook's parameters: the product's, plus where each problem's
+// int8 codes [M, K] (natural order) and bf16 scales [M] staged on chip go.
+struct GroupedDebugParams : GroupedParams {
+  int8_t* dbg_q[kGroupMax];
+  uint16_t* dbg_sa[kGroupMax];
 };
 
 // One consumer warp's share of a unit: rw == RW rows of a stage (fewer at a
-// problem's ragged end), then the release of the stage and the epilogue.
-template <int MB, int RW, bool PLANES>
+// problem's ragged end), then the release of the stage and the epilogue
+// (ACC: the int32 sums are stored instead, to `out` read as int32 [M, N]).
+template <int MB, int RW, bool PLANES, bool ACC>
 __device__ __forceinline__ void grouped_unit(const uint32_t* wrow, int K, const uint8_t* qs, int Mc,
                                              int rows, int lane, int n0, int N, const int* qsum,
                                              const float* saf, uint16_t* out, const float* sw,
@@ -66,25 +74,29 @@ __device__ __forceinline__ void grouped_unit(const uint32_t* wrow, int K, const 
     gemv_rows<MB, RW, PLANES, false, PLANES>(acc, wrow, K / 16, qs, K, Mc, rows, lane);
   __syncwarp();
   if (lane == 0) mbar_arrive(empty_bar);
-  gemv_reduce_store<MB, RW, PLANES>(acc, rows, n0, Mc, 0, N, qsum, saf, out, nullptr, sw, sw_len);
+  if constexpr (ACC)
+    gemv_reduce_store<MB, RW, PLANES>(acc, rows, n0, Mc, 0, N, qsum, saf, nullptr,
+                                      reinterpret_cast<int32_t*>(out), sw, sw_len);
+  else
+    gemv_reduce_store<MB, RW, PLANES>(acc, rows, n0, Mc, 0, N, qsum, saf, out, nullptr, sw, sw_len);
 }
 
 // grouped_unit for the power of two rw <= RW: the instantiation with RW = rw.
-template <int MB, int RW, bool PLANES>
+template <int MB, int RW, bool PLANES, bool ACC>
 __device__ __forceinline__ void grouped_unit_rw(int rw, const uint32_t* wrow, int K, const uint8_t* qs,
                                                 int Mc, int rows, int lane, int n0, int N,
                                                 const int* qsum, const float* saf, uint16_t* out,
                                                 const float* sw, int sw_len, uint32_t empty_bar) {
   if constexpr (RW == 1) {
-    grouped_unit<MB, 1, PLANES>(wrow, K, qs, Mc, rows, lane, n0, N, qsum, saf, out, sw, sw_len,
-                                empty_bar);
+    grouped_unit<MB, 1, PLANES, ACC>(wrow, K, qs, Mc, rows, lane, n0, N, qsum, saf, out, sw,
+                                     sw_len, empty_bar);
   } else {
     if (rw >= RW)
-      grouped_unit<MB, RW, PLANES>(wrow, K, qs, Mc, rows, lane, n0, N, qsum, saf, out, sw, sw_len,
-                                   empty_bar);
+      grouped_unit<MB, RW, PLANES, ACC>(wrow, K, qs, Mc, rows, lane, n0, N, qsum, saf, out, sw,
+                                        sw_len, empty_bar);
     else
-      grouped_unit_rw<MB, RW / 2, PLANES>(rw, wrow, K, qs, Mc, rows, lane, n0, N, qsum, saf, out,
-                                          sw, sw_len, empty_bar);
+      grouped_unit_rw<MB, RW / 2, PLANES, ACC>(rw, wrow, K, qs, Mc, rows, lane, n0, N, qsum, saf,
+                                               out, sw, sw_len, empty_bar);
   }
 }
 
@@ -93,9 +105,12 @@ __device__ __forceinline__ void grouped_unit_rw(int rw, const uint32_t* wrow, in
 // instantiation, so no work is spent on absent rows). Every K is a
 // multiple of 64 (16-byte aligned rows). CTA c takes the units
 // cta_u0[c] .. cta_u0[c + 1] - 1 (ranges balanced by bytes on the host).
-template <int CW, int MB, int RW_MAX>
+// ACC (the accumulator hook, P = GroupedDebugParams): the same kernel storing
+// int32 sums, and every CTA that stages a problem also writes its codes and
+// scales (identical values from every such CTA).
+template <int CW, int MB, int RW_MAX, bool ACC = false, typename P = GroupedParams>
 __global__ void __launch_bounds__((CW + 1) * 32, 1)
-    gemv_grouped_kernel(const __grid_constant__ GroupedParams p) {
+    gemv_grouped_kernel(const __grid_constant__ P p) {
   constexpr int kConsumers = CW * 32;
   constexpr bool PLANES = MB <= 2;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -214,7 +229,10 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1)
       // (the staging only reads the activations, so it also runs after a
       // wait gave up: every consumer warp keeps the same barrier sequence)
       if (staged >= 0) named_barrier_sync(1, kConsumers);
-      gemv_stage_activations<CW, MB, PLANES>(sh, p.x[pr], K, Mc, nullptr, nullptr);
+      if constexpr (ACC)
+        gemv_stage_activations<CW, MB, PLANES>(sh, p.x[pr], K, Mc, p.dbg_q[pr], p.dbg_sa[pr]);
+      else
+        gemv_stage_activations<CW, MB, PLANES>(sh, p.x[pr], K, Mc, nullptr, nullptr);
       named_barrier_sync(1, kConsumers);
       staged = pr;
     }
@@ -229,8 +247,8 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1)
 
     const uint32_t* wrow = reinterpret_cast<const uint32_t*>(
         ring + static_cast<size_t>(s) * p.stage_bytes + static_cast<size_t>(r0) * KB);
-    grouped_unit_rw<MB, RW_MAX, PLANES>(rw, wrow, K, qs, Mc, rows, lane, n0, N, qsum, saf, out, sw,
-                                        sw_len, empty(s));
+    grouped_unit_rw<MB, RW_MAX, PLANES, ACC>(rw, wrow, K, qs, Mc, rows, lane, n0, N, qsum, saf, out,
+                                             sw, sw_len, empty(s));
   }
 }
 

@@ -243,11 +243,11 @@ bitnet_status bitnet_linear_rmsnorm(uint16_t* out, const uint16_t* x, const uint
                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /* bitnet_linear without a caller workspace, for callers that cannot allocate
- * device memory: code running while a stream is being captured into a CUDA
- * graph (cudaMalloc is not allowed there), code inside a framework that owns
- * all device memory through its own pool, or latency-critical paths that
- * cannot afford an allocation's implicit synchronisation. The bitnet-cpu page
- * has no counterpart; this is a convenience of this library's C ABI.
+ * device memory themselves: code inside a framework that owns all device
+ * memory through its own pool and hands out none for a library's scratch, or
+ * a latency-critical path that cannot afford an allocation's implicit
+ * synchronisation. The bitnet-cpu page has no counterpart; this is a
+ * convenience of this library's C ABI.
  * Arguments and result are those of bitnet_linear. When M >= 16 (the split
  * path), the int8 activations and their scales are placed in a scratch array
  * built into the library: 16 MiB (16777216 bytes) per GPU, reserved by every
@@ -256,7 +256,9 @@ bitnet_status bitnet_linear_rmsnorm(uint16_t* out, const uint16_t* x, const uint
  * and enqueue nothing. The call allocates nothing.
  * The first call on a device looks up the scratch's device address (once per
  * device, with that device current); make that first call before any stream
- * capture. Every call on a device shares the one scratch array: calls that
+ * capture. The address is kept for the life of the process: it does not
+ * survive a reset of the device's context (cudaDeviceReset), after which this
+ * entry point must not be called again in the same process. Every call on a device shares the one scratch array: calls that
  * may run at the same time on the GPU (different streams without ordering
  * between them) race on it and must not overlap. Calls ordered on one stream
  * are safe; each call overwrites whatever an earlier call left there. */
@@ -292,6 +294,28 @@ bitnet_status bitnet_gemv_fused_debug(int32_t* acc, int8_t* x_q,
                                       bitnet_dtype dt, const uint8_t* w_packed,
                                       int64_t M, int64_t N, int64_t K,
                                       void* stream);
+
+/* bitnet_linear's own dispatch and kernels (the fused GEMVs for M < 16; the
+ * quantiser into `workspace`, then the split-K or persistent GEMM on the
+ * tensor-core layout, or the SIMT path, for M >= 16) with the epilogue
+ * replaced: acc (int32 [M, N], 16-byte aligned) receives the exact sums,
+ * x_q (int8 [M, K], natural order, 16-byte aligned) the codes and scale_act
+ * (bf16 [M]) the scales the path quantised. Arguments otherwise as
+ * bitnet_linear (no weight scale is read). */
+bitnet_status bitnet_linear_acc_i32(int32_t* acc, int8_t* x_q, uint16_t* scale_act,
+                                    const void* x, bitnet_dtype dt, const uint8_t* w_packed,
+                                    int64_t M, int64_t N, int64_t K, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/* bitnet_gemv_fused_grouped's own dispatch and kernel with the epilogue
+ * replaced: problems[i].out is problem i's int32 [M, N_i] output (16-byte
+ * aligned; scale_wt is not read); x_q[i] (int8 [M, K_i], 16-byte aligned) and
+ * scale_act[i] (bf16 [M]) receive the codes and scales it quantised. x_q and
+ * scale_act are host arrays of `count` device pointers. */
+bitnet_status bitnet_gemv_fused_grouped_acc_i32(const bitnet_gemv_problem* problems,
+                                                int8_t* const* x_q, uint16_t* const* scale_act,
+                                                int64_t count, int64_t M, bitnet_dtype dt,
+                                                void* stream);
 
 #ifdef __cplusplus
 }

@@ -117,9 +117,37 @@ ODD = P(0x10008)
                                        1 << 20, None), bn.ERR_NULL),
     (lambda L: L.bitnet_linear_rmsnorm(FAKE, FAKE, FAKE, 1e-5, FAKE, FAKE, 1, 4, 4, 96,
                                        P(0x10080), 1 << 20, None), bn.ERR_ALIGN),
+    # the accumulator hooks validate like the product entries
+    (lambda L: L.bitnet_linear_acc_i32(FAKE, None, FAKE, FAKE, 0, FAKE, 4, 4, 64, None, 0, None),
+     bn.ERR_NULL),
+    (lambda L: L.bitnet_linear_acc_i32(ODD, FAKE, FAKE, FAKE, 0, FAKE, 4, 4, 64, None, 0, None),
+     bn.ERR_ALIGN),
+    (lambda L: L.bitnet_linear_acc_i32(FAKE, FAKE, FAKE, FAKE, 0, FAKE, 32, 4, 64, None, 0, None),
+     bn.ERR_WORKSPACE),
+    (lambda L: L.bitnet_linear_acc_i32(FAKE, FAKE, FAKE, FAKE, 3, FAKE, 4, 4, 64, None, 0, None),
+     bn.ERR_DTYPE),
+    (lambda L: L.bitnet_gemv_fused_grouped_acc_i32(FAKE, None, FAKE, 1, 1, 0, None), bn.ERR_NULL),
+    # the allocation-free linear refuses a shape whose activations do not fit
+    # its built-in scratch before any CUDA call (M = 4096, K = 8192 needs 32 MiB)
+    (lambda L: L.bitnet_linear_noalloc(FAKE, FAKE, 0, FAKE, FAKE, 1, 4096, 256, 8192, None),
+     bn.ERR_WORKSPACE),
 ])
 def test_validation_rejects_before_launch(call, expect):
     assert call(bn.lib()) == expect
+
+
+def test_failure_path_switch_only_in_the_test_library():
+    """The stage-skipping switch and the 1 ms wait limit live in the test
+    library alone; the product library exports none of its entry points."""
+    assert not hasattr(bn.lib(), "bitnet_wait_test_gemv")
+    path = os.path.join(os.path.dirname(bn.LIB_PATH), "libbitnet_b200_waittest.so")
+    T = ctypes.CDLL(path)
+    assert hasattr(T, "bitnet_wait_test_gemv") and hasattr(T, "bitnet_wait_test_status")
+    T.bitnet_wait_test_gemv.argtypes = [P, P, P, P, ctypes.c_int64, ctypes.c_int64,
+                                        ctypes.c_int, P]
+    # validation happens before any CUDA call
+    assert T.bitnet_wait_test_gemv(FAKE, FAKE, FAKE, FAKE, 64, 96, -1, None) == bn.ERR_SHAPE
+    assert T.bitnet_wait_test_gemv(None, FAKE, FAKE, FAKE, 64, 128, -1, None) == bn.ERR_NULL
 
 
 def test_rmsnorm_workspace_size():

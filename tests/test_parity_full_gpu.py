@@ -25,8 +25,11 @@ def _gpu(cuda_ok):
 
 
 def close(got, ref):
+    """Exact bf16 equality with the oracle (the stated contract is 1 ulp;
+    every stage is a function of its inputs, so the outputs must agree)."""
     d = bf16_ulp_diff(got, ref)
     assert d.max() <= 1, f"max ulp {d.max()}"
+    assert np.array_equal(got, ref), f"{int((d > 0).sum())} outputs differ by one ulp"
 
 
 def test_decode_sweep_graph_matches_oracle():
@@ -68,9 +71,17 @@ def test_llama_gemv_full(M, shape):
     x = synth.act_bf16(synth.key(W.W_LLAMA_GEMV, M, synth.T_ACT, v), M, K)
     sw = synth.scale_wt(synth.key(W.W_LLAMA_GEMV, M, synth.T_SCALE_WT, v))
     p = oracle.pack(w)
-    got = bn.bitnet_gemv_fused(to_dev(x, torch.bfloat16), bn.bitnet_pack_weights(to_dev(w)),
-                               to_dev(sw))
-    close(bf16_bits(got), oracle.linear_cols_threads(x, p, sw, THREADS))
+    xd, pd = to_dev(x, torch.bfloat16), bn.bitnet_pack_weights(to_dev(w))
+    got = bn.bitnet_gemv_fused(xd, pd, to_dev(sw))
+    # the same dispatch with int32 sums: gemv_kernel for M < 8, the
+    # tensor-core gemv_i8_skq_kernel for M = 8 and 15
+    acc, xq, sa, _ = bn.bitnet_linear_acc_i32(xd, pd)
+    q_ref, s_ref = oracle.quantize(x)
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+    assert np.array_equal(bf16_bits(sa), s_ref)
+    acc_ref = oracle.acc_threads(q_ref, p, THREADS)
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    close(bf16_bits(got), oracle.epilogue(acc_ref, s_ref, sw))
 
 
 @pytest.mark.parametrize("M", W.MIDBATCH_M)
@@ -84,16 +95,23 @@ def test_midbatch_gemm(M, KN):
     p = oracle.pack(w)
     pd = bn.bitnet_pack_weights(to_dev(w))
     got = bn.bitnet_gemm(to_dev(q), pd, to_dev(sa, torch.bfloat16), to_dev(sw))
-    rows = np.arange(M) if M <= 64 else np.unique(np.r_[np.random.default_rng(M).choice(M, 24, replace=False), M - 1])
-    ref = oracle.gemm_threads(q[rows], p, sa[rows], sw, THREADS)
-    close(bf16_bits(got)[rows], ref)
+    # every row: gemm_i8_sk_kernel's int32 sums (its accumulator-hook
+    # instantiation) and bf16 outputs
+    acc_ref = oracle.acc_threads(q, p, THREADS)
     acc = bn.bitnet_gemm_acc_i32(to_dev(q), pd).cpu().numpy()
-    assert np.array_equal(acc[rows[:8]], oracle.acc(q[rows[:8]], p))
+    assert np.array_equal(acc, acc_ref)
+    close(bf16_bits(got), oracle.epilogue(acc_ref, sa, sw))
 
 
 @pytest.mark.parametrize("M", W.PREFILL_M)
 @pytest.mark.parametrize("KN", W.PREFILL_SHAPES)
-def test_prefill_linear_sampled_rows(M, KN):
+def test_prefill_linear(M, KN):
+    """bitnet_linear at prefill sizes: the permuted-layout quantiser and
+    gemm_i8_ts_kernel<perm>. Every row at M = 2048; at M = 8192 a seeded
+    sample of 512 rows plus the first and last (quantisation and the
+    contraction are row-local, so the oracle computes those rows alone).
+    Codes, scales and int32 sums come from the accumulator hook (the same
+    quantiser and GEMM kernel with an int32 store)."""
     K, N = KN
     x = synth.act_bf16(synth.key(W.W_PREFILL, M, synth.T_ACT, K), M, K)
     w = synth.ternary(synth.key(W.W_PREFILL, M, synth.T_WEIGHT, K), N, K)
@@ -101,24 +119,33 @@ def test_prefill_linear_sampled_rows(M, KN):
     p = oracle.pack(w)
     xd = to_dev(x, torch.bfloat16)
     pd = bn.bitnet_pack_weights(to_dev(w))
-    y = bn.bitnet_linear(xd, pd, to_dev(sw))
-    xq, sa = bn.bitnet_quantize_act(xd)
-    rows = np.unique(np.r_[np.random.default_rng(M + K).choice(M, 40, replace=False), 0, M - 1])
+    y = bf16_bits(bn.bitnet_linear(xd, pd, to_dev(sw)))
+    acc, xq, sa, _ = bn.bitnet_linear_acc_i32(xd, pd)
+    acc, xq, sa = acc.cpu().numpy(), xq.cpu().numpy(), bf16_bits(sa)
+    if M <= 2048:
+        rows = np.arange(M)
+    else:
+        rows = np.unique(np.r_[np.random.default_rng(M + K).choice(M, 512, replace=False), 0, M - 1])
     q_ref, s_ref = oracle.quantize(x[rows])
-    assert np.array_equal(xq.cpu().numpy()[rows], q_ref)
-    assert np.array_equal(bf16_bits(sa)[rows], s_ref)
-    ref = oracle.linear(x[rows], p, sw, threads=THREADS)
-    close(bf16_bits(y)[rows], ref)
+    assert np.array_equal(xq[rows], q_ref)
+    assert np.array_equal(sa[rows], s_ref)
+    acc_ref = oracle.acc_threads(q_ref, p, THREADS)
+    assert np.array_equal(acc[rows], acc_ref)
+    close(y[rows], oracle.epilogue(acc_ref, s_ref, sw))
 
 
 def test_decode_sweep_grouped_graph_matches_oracle():
     """All 211 calls of the 2B decode sweep as one grouped call, captured in a
-    CUDA graph as the bench does; layers 0 and 15 and the LM head checked."""
+    CUDA graph as the bench does. Every problem is checked against the
+    oracle: its bf16 outputs, and through the accumulator hook (the same
+    partition and gemv_grouped_kernel with an int32 store) its int32 sums,
+    codes and scale. The CTA ranges cut across problem boundaries, so every
+    unit boundary of every problem is covered."""
     names = [n for n, _, _ in W.DECODE_2B_LAYER]
     calls = [(layer, names.index(n), K, N) for layer in range(W.DECODE_2B_LAYERS)
              for n, K, N in W.DECODE_2B_LAYER]
     calls.append((30, len(names), W.DECODE_2B_LM_HEAD[1], W.DECODE_2B_LM_HEAD[2]))
-    xs, wps, sws, outs, checks = [], [], [], [], {}
+    xs, wps, sws, outs, host = [], [], [], [], []
     for i, (layer, v, K, N) in enumerate(calls):
         w = synth.ternary(synth.key(W.W_DECODE_2B, layer, synth.T_WEIGHT, v), N, K)
         sw = synth.scale_wt(synth.key(W.W_DECODE_2B, layer, synth.T_SCALE_WT, v))
@@ -127,8 +154,7 @@ def test_decode_sweep_grouped_graph_matches_oracle():
         wps.append(bn.bitnet_pack_weights(to_dev(w)))
         sws.append(to_dev(sw))
         outs.append(torch.zeros((1, N), dtype=torch.bfloat16, device="cuda"))
-        if layer in (0, 15, 30):
-            checks[i] = (x, oracle.pack(w), sw)
+        host.append((x, oracle.pack(w), sw))
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
         bn.bitnet_gemv_fused_grouped(xs, wps, sws, outs)
@@ -138,9 +164,16 @@ def test_decode_sweep_grouped_graph_matches_oracle():
         for o in outs:
             o.fill_(0)
         g.replay()
+        res = bn.bitnet_gemv_fused_grouped_acc_i32(xs, wps)
     torch.cuda.synchronize()
-    for i, (x, p, sw) in checks.items():
-        close(bf16_bits(outs[i]), oracle.linear_cols_threads(x, p, sw, THREADS))
+    bn.bitnet_device_status()
+    for i, ((x, p, sw), o, (acc, xq, sa)) in enumerate(zip(host, outs, res)):
+        q_ref, s_ref = oracle.quantize(x)
+        assert np.array_equal(xq.cpu().numpy(), q_ref), f"problem {i}"
+        assert np.array_equal(bf16_bits(sa), s_ref), f"problem {i}"
+        acc_ref = oracle.acc_threads(q_ref, p, THREADS)
+        assert np.array_equal(acc.cpu().numpy(), acc_ref), f"problem {i}"
+        close(bf16_bits(o), oracle.epilogue(acc_ref, s_ref, sw))
 
 
 # ------------------------------------- the widened rows at the bench's sizes
