@@ -257,7 +257,12 @@ def make_sweep(bn, d, order="independent", branches=8):
       layer        the dependency order of a transformer layer: Q, K, V
                    concurrently, then O, then gate and up concurrently, then
                    down; layers one after another, the LM head last;
-      stream       every call after the previous one on one stream.
+      stream       every call after the previous one on one stream;
+      layer_grouped  the dependency order of a transformer layer on one
+                   stream, with the stages a layer can group issued as one
+                   grouped call: Q|K|V, then O, then gate|up, then down;
+                   layers one after another, the LM head last (4 launches
+                   per layer, 121 per step).
     Within a stream, consecutive kernels overlap through programmatic
     dependent launch; across streams they are ordered by events only."""
     import ctypes
@@ -270,6 +275,21 @@ def make_sweep(bn, d, order="independent", branches=8):
                      ctypes.c_void_p(s.data_ptr()), K, N))
     side = [torch.cuda.Stream() for _ in range(max(branches, 3))]
     grouped = bn.gemv_problems(d["xs"], d["packed"], d["scales"], d["outs"])
+    # layer_grouped: per layer, the problem arrays of its Q|K|V and gate|up
+    # stages (kept alive with the closure)
+    stage_groups = []
+    by_layer_idx = {}
+    for i, (layer, variant, K, N) in enumerate(d["calls"]):
+        by_layer_idx.setdefault(layer, {})[variant] = i
+    for layer in sorted(by_layer_idx):
+        idx = by_layer_idx[layer]
+        if len(idx) == 1:
+            stage_groups.append([[next(iter(idx.values()))]])
+            continue
+        stage_groups.append([[idx[0], idx[1], idx[2]], [idx[3]], [idx[4], idx[5]], [idx[6]]])
+    stage_arrays = [[(bn.gemv_problems([d["xs"][i] for i in grp], [d["packed"][i] for i in grp],
+                                       [d["scales"][i] for i in grp], [d["outs"][i] for i in grp]),
+                      len(grp)) for grp in stages] for stages in stage_groups]
 
     def issue(a):
         _, _, o, x, p, s, K, N = a
@@ -288,7 +308,18 @@ def make_sweep(bn, d, order="independent", branches=8):
         for i in range(len(groups)):
             main.wait_stream(side[i])
 
+    def grouped_call(arr, n):
+        st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        r = L.bitnet_gemv_fused_grouped(ctypes.cast(arr, ctypes.c_void_p), n, 1, 0, st)
+        if r != 0:
+            raise RuntimeError(f"bitnet_gemv_fused_grouped: {bn.status_string(r)}")
+
     def sweep():
+        if order == "layer_grouped":
+            for stages in stage_arrays:
+                for arr, n in stages:
+                    grouped_call(arr, n)
+            return
         if order == "grouped":
             st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
             r = L.bitnet_gemv_fused_grouped(ctypes.cast(grouped, ctypes.c_void_p), len(args), 1,
@@ -321,6 +352,10 @@ def make_sweep(bn, d, order="independent", branches=8):
 # of the host (a context switch, the clock sampler starting) cannot leave
 # the device idle between timed steps. The spin itself is outside the events.
 HOST_LEAD_CYCLES = 6_000_000
+
+
+# the issue orders timed beside the headline's single grouped launch
+ORDERS = ("layer_grouped", "independent", "layer", "stream")
 
 
 def time_graph(g, steps, warmup, barrier):
@@ -585,6 +620,56 @@ def llama_gemv(bn, dev, pk):
                         "and the same problems as one bitnet_gemv_fused_grouped call",
             "l2": "weights rotated over copies totalling more than 2x L2",
             "peak_hbm_gbs": hbm, "cases": cases}
+
+
+def eager_calls(bn, dev, reps=200):
+    """Per-call cost of eager (not graph-captured) calls through the C ABI:
+    `issue_us` is the host time per call of `reps` back-to-back calls (the
+    library's own host work, plus a ctypes call from Python), and
+    `latency_us` the wall clock of one call followed by a stream
+    synchronisation (median)."""
+    import ctypes
+    L = bn.lib()
+    P = ctypes.c_void_p
+    st = P(torch.cuda.current_stream(dev).cuda_stream)
+    res = {}
+    K, N = 4096, 4096
+    w = synth.ternary(synth.key(W.W_LLAMA_GEMV, 1, synth.T_WEIGHT, 0), N, K)
+    wp = bn.bitnet_pack_weights(torch.from_numpy(w).to(dev))
+    sw = torch.full((1,), 0.05, dtype=torch.float32, device=dev)
+    cases = []
+    for M in (1, 15):
+        x = torch.randn((M, K), generator=torch.Generator().manual_seed(M)).to(dev, torch.bfloat16)
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        args = (P(out.data_ptr()), P(x.data_ptr()), 0, P(wp.data_ptr()), P(sw.data_ptr()), 1, M,
+                N, K, st)
+        cases.append((f"bitnet_gemv_fused M={M} {K}->{N}", L.bitnet_gemv_fused, args))
+    for M in (64,):
+        xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev)
+        sa = torch.full((M,), 0.01, dtype=torch.bfloat16, device=dev)
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        args = (P(out.data_ptr()), P(xq.data_ptr()), P(wp.data_ptr()), P(sa.data_ptr()),
+                P(sw.data_ptr()), 1, M, N, K, st)
+        cases.append((f"bitnet_gemm M={M} {K}->{N}", L.bitnet_gemm, args))
+    for name, fn, args in cases:
+        for _ in range(10):
+            assert fn(*args) == 0
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            fn(*args)
+        t1 = time.perf_counter()
+        torch.cuda.synchronize(dev)
+        lat = []
+        for _ in range(50):
+            t2 = time.perf_counter()
+            fn(*args)
+            torch.cuda.current_stream(dev).synchronize()
+            lat.append(time.perf_counter() - t2)
+        res[name] = {"issue_us": (t1 - t0) / reps * 1e6,
+                     "latency_us": statistics.median(lat) * 1e6}
+    bn.bitnet_device_status()
+    return res
 
 
 def midbatch(bn, dev, pk):
@@ -864,7 +949,7 @@ def main():
         with torch.cuda.graph(g2, stream=stream):
             sweep2()
         torch.cuda.synchronize()
-        for order in ("grouped", "independent", "layer", "stream"):
+        for order in ("grouped", "layer_grouped", "independent", "layer", "stream"):
             sweep = make_sweep(bn, d, order, branches=args.branches)
             sweep()
             torch.cuda.synchronize()
@@ -878,15 +963,15 @@ def main():
             total_ms, per = time_graph(graphs["grouped"], args.steps, args.warmup, barrier)
         e2e_ms = time_e2e([graphs["grouped"], g2], [d, d2], args.steps, args.warmup, barrier)
         other = {}
-        for order in ("independent", "layer", "stream"):
+        for order in ORDERS:
             t_ms, _ = time_graph(graphs[order], args.steps, args.warmup, barrier)
             other[order] = t_ms
     bn.bitnet_device_status()
 
     if pg is not None:
-        total_ms, e2e_ms, ind, lay, strm = max_over_ranks(
-            [total_ms, e2e_ms, other["independent"], other["layer"], other["stream"]], dev)
-        other = {"independent": ind, "layer": lay, "stream": strm}
+        vals = max_over_ranks([total_ms, e2e_ms] + [other[o] for o in ORDERS], dev)
+        total_ms, e2e_ms = vals[0], vals[1]
+        other = dict(zip(ORDERS, vals[2:]))
 
     ms_step = total_ms / args.steps
     value = whole_job_gbs(d["bytes"], world, args.steps, total_ms)
@@ -898,6 +983,7 @@ def main():
     gemv_mb = None if args.no_secondary else llama_gemv(bn, dev, pk)
     mid = None if args.no_secondary else midbatch(bn, dev, pk)
     extra = None if args.no_secondary else extra_rows(bn, dev, pk)
+    eager = None if args.no_secondary else eager_calls(bn, dev)
 
     if rank != 0:
         if pg is not None:
@@ -923,15 +1009,24 @@ def main():
         "gpu_launches": args.steps,  # one grouped launch per step
         "clocks": clocks,
         "step_ms_min_median": [min(per), statistics.median(per)],
+        "decode_layer_order": {
+            "what": "the same 211 problems in a transformer layer's dependency order on one "
+                    "stream: Q|K|V grouped, O, gate|up grouped, down; layers in sequence, LM "
+                    "head last (121 launches per step, chained by programmatic dependent launch)",
+            "ms_per_step": other["layer_grouped"] / args.steps,
+            "gbs": whole_job_gbs(d["bytes"], world, args.steps, other["layer_grouped"]),
+            "frac_hbm": whole_job_gbs(d["bytes"], 1, args.steps, other["layer_grouped"])
+            / pk["hbm_gbs"]},
         "issue_orders": {
             o: {"ms_per_step": other[o] / args.steps,
                 "gbs": whole_job_gbs(d["bytes"], world, args.steps, other[o])}
-            for o in ("independent", "layer", "stream")},
+            for o in ORDERS},
         "lm_head_alone": {**lm, "frac": lm["gbs"] / pk["hbm_gbs"]},
         "prefill": pre,
         "llama_gemv": gemv_mb,
         "midbatch": mid,
         "extra_rows": extra,
+        "eager_calls": eager,
     }
     print(json.dumps(line))
     if pg is not None:

@@ -5,6 +5,7 @@
 #include <cmath>
 #include <map>
 #include <mutex>
+#include <tuple>
 #include <utility>
 
 #include "../../include/bitnet.h"
@@ -93,6 +94,55 @@ bitnet_status device_info(DeviceInfo** out) {
   return BITNET_OK;
 }
 
+int current_device() {
+  int dev = 0;
+  return cudaGetDevice(&dev) == cudaSuccess ? dev : -1;
+}
+
+// The kernel attribute that opens dynamic shared memory beyond 48 KB is a
+// driver call: made once per (kernel, device) for the largest size asked
+// so far, not on every launch.
+bitnet_status ensure_smem(const void* kernel, size_t smem) {
+  if (smem <= 48 * 1024) return BITNET_OK;
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, size_t> done;
+  const int dev = current_device();
+  if (dev < 0) return BITNET_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  size_t& have = done[std::make_pair(kernel, dev)];
+  if (have >= smem) return BITNET_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  have = smem;
+  return BITNET_OK;
+}
+
+// Resident CTAs per SM of `kernel` at `threads` and `smem` (an occupancy
+// query is a driver call: cached per kernel, device and launch shape).
+bitnet_status occupancy(const void* kernel, int threads, size_t smem, int* occ) {
+  static std::mutex mu;
+  static std::map<std::tuple<const void*, int, int, size_t>, int> cache;
+  const int dev = current_device();
+  if (dev < 0) return BITNET_ERR_CUDA;
+  const auto key = std::make_tuple(kernel, dev, threads, smem);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      *occ = it->second;
+      return BITNET_OK;
+    }
+  }
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  cache[key] = n;
+  *occ = n;
+  return BITNET_OK;
+}
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point, so the
 // library does not link libcuda directly.
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
@@ -117,9 +167,9 @@ EncodeTiledFn encode_fn() {
 
 // 2-D uint8 tensor map: rows x cols bytes, row pitch `pitch` bytes,
 // box of box_rows x box_cols bytes.
-bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-                 uint64_t pitch, uint32_t box_rows, uint32_t box_cols,
-                 CUtensorMapSwizzle swz) {
+bool encode_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                   uint64_t pitch, uint32_t box_rows, uint32_t box_cols,
+                   CUtensorMapSwizzle swz) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {cols, rows};
@@ -130,6 +180,32 @@ bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// encode_map_u8 through a small cache keyed by every encoded field: a call
+// that repeats the operands of an earlier one (a layer's weights, a
+// workspace) reuses its map instead of encoding it again.
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                 uint64_t pitch, uint32_t box_rows, uint32_t box_cols,
+                 CUtensorMapSwizzle swz) {
+  using Key = std::tuple<const void*, uint64_t, uint64_t, uint64_t, uint32_t, uint32_t, int>;
+  static std::mutex mu;
+  static std::map<Key, CUtensorMap> cache;
+  constexpr size_t kMaxEntries = 4096;
+  const Key key{base, rows, cols, pitch, box_rows, box_cols, static_cast<int>(swz)};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      *m = it->second;
+      return true;
+    }
+  }
+  if (!encode_map_u8(m, base, rows, cols, pitch, box_rows, box_cols, swz)) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() >= kMaxEntries) cache.clear();
+  cache.emplace(key, *m);
+  return true;
 }
 
 bitnet_status check_compute_shape(int64_t M, int64_t N, int64_t K) {
@@ -175,14 +251,10 @@ bitnet_status launch_gemv_t(const GemvParams& p, int grid_y, size_t smem, int sm
                             cudaStream_t st) {
   auto k = gemv_kernel<CW, MB, RW, WIDE, PREQ, NORM>;
   constexpr int threads = (CW + 1) * 32;
-  if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return BITNET_ERR_CUDA;
-  }
+  if (ensure_smem(reinterpret_cast<const void*>(k), smem) != BITNET_OK) return BITNET_ERR_CUDA;
   // persistent: no more CTAs than row blocks, nor than can be resident
   int occ = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, threads, smem) != cudaSuccess)
+  if (occupancy(reinterpret_cast<const void*>(k), threads, smem, &occ) != BITNET_OK)
     return BITNET_ERR_CUDA;
   if (occ < 1) occ = 1;
   const int nblocks = (p.N + p.rows_per_block - 1) / p.rows_per_block;
@@ -358,11 +430,9 @@ bitnet_status launch_grouped_t(P& gp, size_t smem, int sms, cudaStream_t st) {
   constexpr int cw = grouped_cw(MB);
   auto k = gemv_grouped_kernel<cw, MB, RW_MAX, ACC, P>;
   constexpr int threads = (cw + 1) * 32;
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return BITNET_ERR_CUDA;
+  if (ensure_smem(reinterpret_cast<const void*>(k), smem) != BITNET_OK) return BITNET_ERR_CUDA;
   int occ = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, threads, smem) != cudaSuccess)
+  if (occupancy(reinterpret_cast<const void*>(k), threads, smem, &occ) != BITNET_OK)
     return BITNET_ERR_CUDA;
   if (occ < 1) occ = 1;
   int grid = occ * sms;
@@ -536,8 +606,7 @@ bitnet_status launch_sk(const CUtensorMap& mx, const CUtensorMap& mw, void* out,
                         const uint16_t* bias) {
   auto kernel = sk::gemm_i8_sk_kernel<BX, kAccOut, kPerm>;
   constexpr int smem = sk::Cfg<BX>::SMEM_BYTES;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-      cudaSuccess)
+  if (ensure_smem(reinterpret_cast<const void*>(kernel), smem) != BITNET_OK)
     return BITNET_ERR_CUDA;
   const int64_t w_tiles = (N + sk::BW - 1) / sk::BW;
   const int64_t kblocks = (K + sk::BK - 1) / sk::BK;
@@ -591,8 +660,7 @@ bitnet_status run_gemv_skq(void* out, const uint16_t* x, const uint8_t* wp,
                            int8_t* dbg_q = nullptr, uint16_t* dbg_sa = nullptr) {
   auto kernel = acc_out ? skq::gemv_i8_skq_kernel<true> : skq::gemv_i8_skq_kernel<false>;
   constexpr int smem = skq::SMEM_BYTES;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-      cudaSuccess)
+  if (ensure_smem(reinterpret_cast<const void*>(kernel), smem) != BITNET_OK)
     return BITNET_ERR_CUDA;
   CUtensorMap mw;
   if (!make_map_u8(&mw, wp, N, K / 4, K / 4, skq::BW, skq::BK / 4, CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -660,8 +728,7 @@ bitnet_status run_gemm(void* out, bool acc_out, const int8_t* xq, const uint8_t*
   if (tiles > INT32_MAX) return BITNET_ERR_SHAPE;
   const int grid = static_cast<int>(tiles < dev->sms ? tiles : dev->sms);
   auto go = [&](auto kernel) -> bitnet_status {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             ts::SMEM_BYTES) != cudaSuccess)
+    if (ensure_smem(reinterpret_cast<const void*>(kernel), ts::SMEM_BYTES) != BITNET_OK)
       return BITNET_ERR_CUDA;
     return launch_pdl(kernel, dim3(grid), dim3(ts::NUM_THREADS), ts::SMEM_BYTES, st, mx, mw,
                       out, sa, sw, static_cast<int>(sw_len), rowsum, static_cast<int>(M),
