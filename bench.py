@@ -442,23 +442,51 @@ def time_e2e(graphs, ds, steps, warmup, barrier):
     return e0.elapsed_time(e1)
 
 
+class L2Flush:
+    """Flush L2 between timed repetitions: write one buffer twice the size of
+    L2, then read another one of that size. The write evicts the timed
+    call's data; the read then evicts the written (dirty) lines, so their
+    write-back to HBM happens here rather than inside the timed call."""
+
+    def __init__(self, dev):
+        self.a = torch.empty((2 * L2_BYTES,), dtype=torch.uint8, device=dev)
+        self.b = torch.ones((2 * L2_BYTES // 4,), dtype=torch.int32, device=dev)
+
+    def __call__(self, r):
+        self.a.fill_(r & 0xFF)
+        self.b.amax()
+
+
 def lm_head_alone(bn, d, dev, reps=20):
-    """The LM-head GEMV (82 MB of packed weights) timed alone, L2 flushed."""
+    """The LM-head GEMV (82 MB of packed weights) timed alone, L2 flushed:
+    bitnet_gemv_fused as the product dispatches it, and for comparison the
+    single-problem GEMV kernel (reached through bitnet_linear_bias with a
+    zero bias, which that kernel alone takes)."""
     i = len(d["calls"]) - 1
     _, _, K, N = d["calls"][i]
-    flush = torch.empty((2 * L2_BYTES,), dtype=torch.uint8, device=dev)
-    times = []
-    for r in range(reps + 3):
-        flush.fill_(r & 0xFF)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        bn.bitnet_gemv_fused(d["xs"][i], d["packed"][i], d["scales"][i], out=d["outs"][i])
-        e1.record()
-        torch.cuda.synchronize()
-        if r >= 3:
-            times.append(e0.elapsed_time(e1))
-    ms = statistics.median(times)
-    return {"K": K, "N": N, "ms": ms, "gbs": call_bytes(1, K, N) / ms / 1e6}
+    flush = L2Flush(dev)
+    zero_bias = torch.zeros((N,), dtype=torch.bfloat16, device=dev)
+
+    def timed(fn):
+        times = []
+        for r in range(reps + 3):
+            flush(r)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if r >= 3:
+                times.append(e0.elapsed_time(e1))
+        return statistics.median(times)
+
+    ms = timed(lambda: bn.bitnet_gemv_fused(d["xs"][i], d["packed"][i], d["scales"][i],
+                                            out=d["outs"][i]))
+    ms_single = timed(lambda: bn.bitnet_linear(d["xs"][i], d["packed"][i], d["scales"][i],
+                                               out=d["outs"][i], bias=zero_bias))
+    return {"K": K, "N": N, "ms": ms, "gbs": call_bytes(1, K, N) / ms / 1e6,
+            "single_kernel_ms": ms_single,
+            "single_kernel_gbs": call_bytes(1, K, N) / ms_single / 1e6}
 
 
 # ---------------------------------------------------------------- prefill
@@ -478,7 +506,7 @@ def time_flushed(fn, flush, reps=5, graph=True):
         run = g.replay
     ts = []
     for r in range(reps + 2):
-        flush.fill_(r & 0xFF)
+        flush(r)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         run()
@@ -494,7 +522,7 @@ def prefill(bn, dev, pk, reps=5):
     bitnet_linear (per-token quantisation + tensor-core GEMM, bf16 out), each
     timed with CUDA events with L2 flushed between repetitions; and the GEMM
     alone (bitnet_gemm on activations quantised beforehand) for every case."""
-    flush = torch.empty((2 * L2_BYTES,), dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     peak = pk["bf16_tflops"] * INT8_OVER_BF16
 
     def timed(fn):
@@ -609,10 +637,17 @@ def llama_gemv(bn, dev, pk):
                 [xd] * len(copies), copies, [swd] * len(copies), gouts)]) / len(copies)
             del gouts
             g_gbs = call_bytes(M, K, N) / g_ms / 1e6
-            cases.append({"M": M, "K": K, "N": N, "ms": ms, "gbs": gbs, "frac_hbm": gbs / hbm,
-                          "tops": 2.0 * M * N * K / ms / 1e9,
-                          "grouped": {"problems": len(copies), "ms_per_problem": g_ms,
-                                      "gbs": g_gbs, "frac_hbm": g_gbs / hbm}})
+            case = {"M": M, "K": K, "N": N, "ms": ms, "gbs": gbs, "frac_hbm": gbs / hbm,
+                    "tops": 2.0 * M * N * K / ms / 1e9,
+                    "grouped": {"problems": len(copies), "ms_per_problem": g_ms,
+                                "gbs": g_gbs, "frac_hbm": g_gbs / hbm}}
+            if M <= 2:
+                # one problem per grouped call, the calls one after another
+                s_ms = time_rotation([lambda c=c: bn.bitnet_gemv_fused_grouped(
+                    [xd], [c], [swd], [out]) for c in copies])
+                s_gbs = call_bytes(M, K, N) / s_ms / 1e6
+                case["grouped_single"] = {"ms": s_ms, "gbs": s_gbs, "frac_hbm": s_gbs / hbm}
+            cases.append(case)
         del copies
     bn.bitnet_device_status()
     return {"workload": "LLaMA-7B projections 4096->4096, 4096->11008, 11008->4096 at "
@@ -716,7 +751,7 @@ def extra_rows(bn, dev, pk):
     at M = 2048 and M = 1, each beside the same call without the norm)."""
     hbm = pk["hbm_gbs"]
     tops_peak = pk["bf16_tflops"] * INT8_OVER_BF16
-    flush = torch.empty((2 * L2_BYTES,), dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
 
     def timed(fn, graph=True):
         return time_flushed(fn, flush, 5, graph)

@@ -447,26 +447,16 @@ bitnet_status launch_grouped_t(P& gp, size_t smem, int sms, cudaStream_t st) {
 // bucket (at most 32 accumulator registers per lane).
 constexpr int grouped_rw_max(int mb) { return mb == 1 ? 8 : mb == 2 ? 4 : mb == 4 ? 8 : mb == 8 ? 4 : 1; }
 
-// Launch up to kGroupMax problems (all K % 64 == 0, validated) in one kernel.
-// ACC: the accumulator hook (P = GroupedDebugParams, its debug pointers set
-// by the caller); the partition and the launch are the product's.
-template <bool ACC, typename P>
-bitnet_status run_gemv_grouped_t(P& gp, const bitnet_gemv_problem* pr, int count, int M,
-                                 cudaStream_t st) {
-  DeviceInfo* dev = nullptr;
-  bitnet_status s = device_info(&dev);
-  if (s != BITNET_OK) return s;
-  static_assert(sizeof(P) <= 32000, "kernel parameter space");
-  gp.count = count;
-  gp.M = M;
-  const int mb = bucket_of(M);
-  const int rw_max = grouped_rw_max(mb);
-  const int cw = grouped_cw(mb);  // as launch_grouped_t instantiates it
-  static_assert(grouped_cw(1) <= kGroupedMaxCW && grouped_cw(16) <= kGroupedMaxCW &&
-                    kGroupedMaxCW <= kGemvMaxConsumerWarps,
-                "the staging's per-warp scratch covers every grouped CTA");
+// Split a group into units for `cw` consumer warps (rows per warp aimed at
+// `stage_target` bytes per unit) and size the ring (aimed at `ring` bytes);
+// fills gp and returns the dynamic shared memory, or 0 if one stage does not
+// fit under `limit`.
+template <typename P>
+size_t plan_grouped(P& gp, const bitnet_gemv_problem* pr, int count, int M, int sms, int cw,
+                    int stage_target, int ring, size_t limit) {
+  const int rw_max = grouped_rw_max(bucket_of(M));
   auto rw_of = [&](int i, int shift) {
-    int rw = pow2_floor(kGroupedStageTarget / (cw * (pr[i].K / 4)));
+    int rw = pow2_floor(stage_target / (cw * (pr[i].K / 4)));
     if (rw > rw_max) rw = rw_max;
     rw >>= shift;
     return rw < 1 ? 1 : rw;
@@ -482,7 +472,7 @@ bitnet_status run_gemv_grouped_t(P& gp, const bitnet_gemv_problem* pr, int count
       all_one = all_one && rw == 1;
       u += (pr[i].N + cw * rw - 1) / (cw * rw);
     }
-    if (u >= 2 * dev->sms || all_one) break;
+    if (u >= 2 * sms || all_one) break;
   }
   int units = 0;
   int64_t kmax = 0;
@@ -506,16 +496,39 @@ bitnet_status run_gemv_grouped_t(P& gp, const bitnet_gemv_problem* pr, int count
   }
   gp.unit0[count] = units;
   gp.units = units;
-  if (units == 0) return BITNET_OK;
   gp.q_bytes = static_cast<uint32_t>(align128(static_cast<size_t>(M) * kmax));
   gp.stage_bytes = static_cast<uint32_t>(stage);
-  int stages = static_cast<int>(kGemvRingTarget / stage);
+  int stages = static_cast<int>(ring / stage);
   if (stages > kGemvMaxStages) stages = kGemvMaxStages;
   if (stages < 1) stages = 1;
-  while (stages > 1 && kGemvHeaderBytes + gp.q_bytes + stages * stage > kSmemLimit) --stages;
+  while (stages > 1 && kGemvHeaderBytes + gp.q_bytes + stages * stage > limit) --stages;
   gp.stages = stages;
   const size_t smem = kGemvHeaderBytes + gp.q_bytes + static_cast<size_t>(stages) * stage;
-  if (smem > kSmemLimit) return BITNET_ERR_SHAPE;
+  return smem <= limit ? smem : 0;
+}
+
+// Launch up to kGroupMax problems (all K % 64 == 0, validated) in one kernel.
+// ACC: the accumulator hook (P = GroupedDebugParams, its debug pointers set
+// by the caller); the partition and the launch are the product's.
+template <bool ACC, typename P>
+bitnet_status run_gemv_grouped_t(P& gp, const bitnet_gemv_problem* pr, int count, int M,
+                                 cudaStream_t st) {
+  DeviceInfo* dev = nullptr;
+  bitnet_status s = device_info(&dev);
+  if (s != BITNET_OK) return s;
+  static_assert(sizeof(P) <= 32000, "kernel parameter space");
+  static_assert(grouped_cw(1) <= kGroupedMaxCW && grouped_cw(16) <= kGroupedMaxCW &&
+                    kGroupedMaxCW <= kGemvMaxConsumerWarps,
+                "the staging's per-warp scratch covers every grouped CTA");
+  gp.count = count;
+  gp.M = M;
+  const int mb = bucket_of(M);
+  int64_t total_bytes = 0;
+  for (int i = 0; i < count; ++i) total_bytes += pr[i].N * (pr[i].K / 4);
+  if (total_bytes == 0) return BITNET_OK;
+  const size_t smem = plan_grouped(gp, pr, count, M, dev->sms, grouped_cw(mb),
+                                   kGroupedStageTarget, kGemvRingTarget, kSmemLimit);
+  if (smem == 0) return BITNET_ERR_SHAPE;
   switch (mb) {
     case 1: return launch_grouped_t<1, grouped_rw_max(1), ACC>(gp, smem, dev->sms, st);
     case 2: return launch_grouped_t<2, grouped_rw_max(2), ACC>(gp, smem, dev->sms, st);
@@ -999,6 +1012,10 @@ static bitnet_status gemv_common(GemvParams& p, const void* x, bitnet_dtype dt,
   return BITNET_OK;
 }
 
+// Packed bytes from which a single fused GEMV of one or two rows takes the
+// grouped kernel (the 2B model's LM head, 82 MB, does; its layers do not).
+constexpr int64_t kGemvViaGroupedBytes = int64_t(32) << 20;
+
 // Where the accumulator hooks send their results: int32 sums instead of the
 // bf16 outputs, and the int8 codes [M, K] (natural order) and bf16 scales [M]
 // the path quantised. Null for every product call.
@@ -1039,6 +1056,18 @@ static bitnet_status gemv_fused_impl(uint16_t* out, const void* x, bitnet_dtype 
   }
   p.norm_g = norm_g;
   p.norm_eps = norm_eps;
+  // One or two activation rows against a large weight matrix (an LM head):
+  // the grouped kernel's one-problem launch (units of up to 80 KB, one CTA
+  // per SM, one problem's activations staged once per CTA) streams the
+  // weights faster than the single-call kernel's tiling.
+  if (M <= 2 && norm_g == nullptr && bias == nullptr && dt == BITNET_BF16 && K % 64 == 0 &&
+      N * (K / 4) >= kGemvViaGroupedBytes && aligned(x, 16) && aligned(w_packed, 16)) {
+    bitnet_gemv_problem q{hook == nullptr ? out : static_cast<uint16_t*>(static_cast<void*>(hook->acc)),
+                          x, w_packed, scale_wt, scale_wt_len, N, K};
+    return hook == nullptr ? run_gemv_grouped(&q, 1, static_cast<int>(M), as_stream(stream))
+                           : run_gemv_grouped_acc(&q, &hook->q, &hook->sa, 1, static_cast<int>(M),
+                                                  as_stream(stream));
+  }
   if (norm_g == nullptr && dt == BITNET_BF16 && skq_ok(x, w_packed, M, K) &&
       K / 128 <= sk::MAX_SPLIT * skq::MAX_KB) {
     const bitnet_status r =

@@ -579,6 +579,8 @@ def test_gemv_grouped_wide_rows(M):
 # (M, K, N, the kernel instantiation the product reaches)
 LINEAR_PATHS = [
     (1, 2560, 640, "gemv_kernel MB=1 (register-cached staging)"),
+    (1, 4096, 32768, "gemv_grouped_kernel, one-problem launch (32 MB layer)"),
+    (2, 2560, 52432, "gemv_grouped_kernel MB=2, one-problem launch, ragged units"),
     (2, 4096, 300, "gemv_kernel MB=2"),
     (1, 96, 40, "gemv_kernel MB=1, K % 64 != 0 (8-byte copies)"),
     (3, 160, 33, "gemv_kernel MB=4, K % 64 != 0"),
