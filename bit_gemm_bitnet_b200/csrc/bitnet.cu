@@ -10,6 +10,7 @@
 
 #include "../../include/bitnet.h"
 #include "common.cuh"
+#include "gemm_fr.cuh"
 #include "gemm_sk.cuh"
 #include "gemm_skq.cuh"
 #include "gemm_ts.cuh"
@@ -646,14 +647,79 @@ bitnet_status run_sk_bx(void* out, bool acc_out, const int8_t* xq, const uint8_t
   return launch_sk<BX, false, false>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st, bias);
 }
 
+// ------------------------------------- few-row GEMM, 512-wide K stages
+
+// The split of the K loop for the few-row kernel: the S that minimises
+// waves x (512-wide K blocks per CTA + a CTA's fixed cost, about four blocks,
+// + the cluster reduction's, about four more, when S > 1).
+template <typename Kernel>
+int fr_split(Kernel kernel, int smem, int sms, int64_t w_tiles, int64_t kblocks) {
+  int best = 1;
+  int64_t best_cost = INT64_MAX;
+  for (int S = 1; S <= fr::MAX_SPLIT && S <= kblocks; ++S) {
+    const int fit = S == 1 ? sms : sk_clusters(reinterpret_cast<const void*>(kernel), S, smem);
+    if (fit < 1) continue;
+    const int64_t waves = (w_tiles + fit - 1) / fit;
+    const int64_t cost = waves * ((kblocks + S - 1) / S + 4 + (S > 1 ? 4 : 0));
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = S;
+    }
+  }
+  return best;
+}
+
+template <int BX, bool kAccOut, bool kPerm>
+bitnet_status launch_fr(const CUtensorMap& mx, const CUtensorMap& mw, void* out,
+                        const uint16_t* sa, const float* sw, int64_t sw_len,
+                        const int32_t* rowsum, int64_t M, int64_t N, int64_t K, cudaStream_t st,
+                        const uint16_t* bias) {
+  auto kernel = fr::gemm_i8_fr_kernel<BX, kAccOut, kPerm>;
+  constexpr int smem = fr::Cfg<BX>::SMEM_BYTES;
+  if (ensure_smem(reinterpret_cast<const void*>(kernel), smem) != BITNET_OK)
+    return BITNET_ERR_CUDA;
+  DeviceInfo* dev = nullptr;
+  bitnet_status s = device_info(&dev);
+  if (s != BITNET_OK) return s;
+  const int64_t w_tiles = (N + fr::BW - 1) / fr::BW;
+  const int64_t kblocks = (K + fr::BKS - 1) / fr::BKS;
+  const int S = fr_split(kernel, smem, dev->sms, w_tiles, kblocks);
+  if (w_tiles * S > INT32_MAX) return BITNET_ERR_SHAPE;
+  const dim3 grid(static_cast<unsigned>(w_tiles * S)), block(fr::NUM_THREADS);
+  if (S == 1)
+    return launch_pdl(kernel, grid, block, smem, st, mx, mw, out, sa, sw,
+                      static_cast<int>(sw_len), rowsum, static_cast<int>(M), static_cast<int>(N),
+                      static_cast<int>(K), 1, bias);
+  return launch_pdl_cluster(kernel, grid, block, smem, S, st, mx, mw, out, sa, sw,
+                            static_cast<int>(sw_len), rowsum, static_cast<int>(M),
+                            static_cast<int>(N), static_cast<int>(K), S, bias);
+}
+
+template <int BX>
+bitnet_status run_fr_bx(void* out, bool acc_out, const int8_t* xq, const uint8_t* wp,
+                        const uint16_t* sa, const float* sw, int64_t sw_len, int64_t M,
+                        int64_t N, int64_t K, cudaStream_t st, bool perm,
+                        const int32_t* rowsum, const uint16_t* bias) {
+  CUtensorMap mx, mw;
+  if (!make_map_u8(&mx, xq, M, K, K, BX, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_u8(&mw, wp, N, K / 4, K / 4, fr::BW, fr::BKS / 4, CU_TENSOR_MAP_SWIZZLE_128B))
+    return BITNET_ERR_CUDA;
+  if (acc_out && perm) return launch_fr<BX, true, true>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st, nullptr);
+  if (acc_out) return launch_fr<BX, true, false>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st, nullptr);
+  if (perm) return launch_fr<BX, false, true>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st, bias);
+  return launch_fr<BX, false, false>(mx, mw, out, sa, sw, sw_len, rowsum, M, N, K, st, bias);
+}
+
 bitnet_status run_gemm_sk(void* out, bool acc_out, const int8_t* xq, const uint8_t* wp,
                           const uint16_t* sa, const float* sw, int64_t sw_len, int64_t M,
                           int64_t N, int64_t K, cudaStream_t st, bool perm,
                           const int32_t* rowsum, const uint16_t* bias) {
-  if (M <= 16) return run_sk_bx<16>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
-  if (M <= 32) return run_sk_bx<32>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
-  if (M <= 64) return run_sk_bx<64>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
-  if (M <= 128) return run_sk_bx<128>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
+  // up to 128 rows: the few-row kernel with 512-wide K stages; more: the
+  // split-K kernel's 256-row tile
+  if (M <= 16) return run_fr_bx<16>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
+  if (M <= 32) return run_fr_bx<32>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
+  if (M <= 64) return run_fr_bx<64>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
+  if (M <= 128) return run_fr_bx<128>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
   return run_sk_bx<256>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
 }
 

@@ -19,8 +19,8 @@
 // Warp roles (512 threads, one CTA per SM):
 //   warp 0      TMA producer
 //   warp 1      tensor-memory owner, MMA issuer (one thread)
-//   warps 4-15  unpack: packed codes -> int8 -> tcgen05.st into an A stage
-//               (three groups of four warps, stages in turn); then warps 4-7
+//   warps 4-11  unpack: packed codes -> int8 -> tcgen05.st into an A stage
+//               (two groups of four warps, stages in turn); then warps 4-7
 //               move the accumulator to the shared-memory partial tile
 //   all         the cluster reduction and the epilogue
 // Waits on mbarriers are bounded like the other kernels of this library;
@@ -49,6 +49,7 @@ template <int BX>
 struct Cfg {
   static_assert(BX == 16 || BX == 32 || BX == 64 || BX == 128 || BX == 256, "MMA N");
   static constexpr int STAGES = BX == 256 ? 4 : 8;
+  static_assert(STAGES % 2 == 0, "stages a multiple of the two unpack groups");
   static constexpr int X_BYTES = BX * BK;
   static constexpr int STAGE_BYTES = X_BYTES + WP_BYTES;
   static constexpr int PART_BYTES = BX * BW * 4;   // int32 partial tile [BX][BW]
@@ -199,11 +200,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mma_commit(sm.drain());
       mbar_wait_drain(sm.drain(), 0u);
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 12) {
     // -------------------------------------------------------------- unpack
-    // Three groups of four warps take the stages in turn, so three stages
-    // are unpacked at once (a stage's unpack is a chain of dependent steps:
-    // wait, load, unpack, tensor-memory store, wait for the store, arrive).
+    // Two groups of four warps take the stages in turn, so two stages are
+    // unpacked at once (a stage's unpack is a chain of dependent steps: wait,
+    // load, unpack, tensor-memory store, wait for the store, arrive). The
+    // number of groups divides the number of stages, so a group that waits
+    // for a stage's k-th fill is never two fills ahead of the barrier (a
+    // parity wait cannot be satisfied by an earlier fill).
     // Warp -> TMEM sub-partition warp % 4 (weight rows 32 * (warp % 4) ...),
     // all 32 columns (128 K elements) of its group's stages.
     const int sub = warp & 3;
@@ -212,7 +216,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t lane_base = static_cast<uint32_t>(sub * 32) << 16;
     uint32_t it = 0;
     for (int kb = kb0; kb < kb1; ++kb, ++it) {
-      if (it % 3u != group) continue;
+      if (it % 2u != group) continue;
       const int s = it % ST;
       const uint32_t ph = (it / ST) & 1u;
       if (!mbar_wait_warp(sm.full(s), ph, abort)) break;

@@ -35,7 +35,11 @@ constexpr int NUM_THREADS = sk::NUM_THREADS;
 constexpr int TMEM_COLS = sk::TMEM_COLS;
 constexpr int A_COL0 = 32;                  // A stages right after the 16-column accumulator
 constexpr int A_COLS = sk::A_COLS;
-constexpr int ST = 14;                       // weight stages (56 KB in flight)
+// weight stages (60 KB in flight); a multiple of the three unpack groups, so
+// a group that waits for a stage's k-th fill is never two fills ahead of the
+// barrier (a parity wait cannot be satisfied by an earlier fill)
+constexpr int ST = 15;
+static_assert(ST % 3 == 0, "stages a multiple of the unpack groups");
 constexpr int WP_BYTES = sk::WP_BYTES;       // 4 KB per stage
 constexpr int XT_BYTES = BX * BK;            // one K block of activations, 2 KB
 constexpr int ACT_BUDGET = 96 * 1024;        // resident activations per CTA

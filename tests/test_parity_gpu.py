@@ -187,9 +187,10 @@ def test_gemm_matches_oracle(M, K, N):
     assert_bf16_close(bf16_bits(got), ref)
 
 
-# M <= 256 takes the split-K tensor-core kernel: one N tile (the K loop split
-# over a cluster of up to 8 CTAs), a ragged last K block (K % 128 == 64), a
-# ragged N, every activation-row width (16 ... 256) and a few splits.
+# M <= 128 takes the few-row kernel (512-wide K stages; the K loop split over
+# a cluster of up to 8 CTAs where the tiles do not fill the GPU), 128 < M <=
+# 256 the split-K kernel's 256-row tile: ragged last K stages, ragged N,
+# every activation-row width (16 ... 256) and a few splits.
 SK_CASES = [(33, 4096, 128), (2, 192, 130), (17, 640, 1000), (64, 8256, 200),
             (256, 1024, 4096), (100, 2560, 131), (1, 11008, 4099), (129, 64, 256),
             (16, 4096, 11008)]
@@ -590,9 +591,11 @@ LINEAR_PATHS = [
     (12, 2112, 77, "gemv_i8_skq_kernel, ragged N"),
     (15, 11008, 130, "gemv_i8_skq_kernel, M = 15"),
     (9, 1024, 4099, "gemv_i8_skq_kernel, N % 4 != 0"),
-    (16, 4096, 256, "gemm_i8_sk_kernel<16, perm>"),
-    (33, 4096, 130, "gemm_i8_sk_kernel<64, perm>, ragged N"),
-    (100, 2560, 131, "gemm_i8_sk_kernel<128, perm>"),
+    (16, 4096, 256, "gemm_i8_fr_kernel<16, perm>"),
+    (33, 4096, 130, "gemm_i8_fr_kernel<64, perm>, ragged N"),
+    (100, 2560, 131, "gemm_i8_fr_kernel<128, perm>, ragged last K stage"),
+    (64, 11008, 4096, "gemm_i8_fr_kernel<64, perm>, one CTA per tile"),
+    (20, 64, 300, "gemm_i8_fr_kernel<32, perm>, K below one stage"),
     (256, 1024, 4096, "gemm_i8_sk_kernel<256, perm>"),
     (129, 64, 256, "gemm_i8_sk_kernel<256, perm>, one K block of 64"),
     (257, 2560, 520, "gemm_i8_ts_kernel<perm>, ragged M and N tiles"),
