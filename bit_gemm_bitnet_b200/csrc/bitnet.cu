@@ -742,22 +742,24 @@ bitnet_status run_gemv_skq(void* out, const uint16_t* x, const uint8_t* wp,
   if (ensure_smem(reinterpret_cast<const void*>(kernel), smem) != BITNET_OK)
     return BITNET_ERR_CUDA;
   CUtensorMap mw;
-  if (!make_map_u8(&mw, wp, N, K / 4, K / 4, skq::BW, skq::BK / 4, CU_TENSOR_MAP_SWIZZLE_NONE))
+  if (!make_map_u8(&mw, wp, N, K / 4, K / 4, skq::BW, skq::BKS / 4, CU_TENSOR_MAP_SWIZZLE_128B))
     return BITNET_ERR_CUDA;
   const int64_t w_tiles = (N + skq::BW - 1) / skq::BW;
-  const int64_t kblocks = (K + skq::BK - 1) / skq::BK;
-  // the split as for the few-row GEMM, with at most MAX_KB K blocks per CTA
-  // (the resident activations) and at most QMAX activation items per thread
+  const int64_t kstages = (K + skq::BKS - 1) / skq::BKS;
+  // the split: at most MAX_KB / 4 stages per CTA (the resident activations)
+  // and at most QMAX activation items per thread; the cost as for the
+  // few-row GEMM, in 512-wide stages (a CTA's fixed cost about four, the
+  // cluster's activation scales and reduction about four more)
   int best = 0;
   int64_t best_cost = INT64_MAX;
-  for (int S = 1; S <= sk::MAX_SPLIT && S <= kblocks; ++S) {
-    const int64_t per_cta = (kblocks + S - 1) / S;
-    if (per_cta > skq::MAX_KB || per_cta * (skq::BK / 4) * M > skq::NUM_THREADS * skq::QMAX)
+  for (int S = 1; S <= sk::MAX_SPLIT && S <= kstages; ++S) {
+    const int64_t per_cta = (kstages + S - 1) / S;
+    if (per_cta * 4 > skq::MAX_KB || per_cta * (skq::BKS / 4) * M > skq::NUM_THREADS * skq::QMAX)
       continue;
     const int fit = sk_clusters(reinterpret_cast<const void*>(kernel), S, smem);
     if (fit < 1) continue;
     const int64_t waves = (w_tiles + fit - 1) / fit;
-    const int64_t cost = waves * ((kblocks + S - 1) / S + 4);
+    const int64_t cost = waves * (per_cta + 4 + (S > 1 ? 4 : 0));
     if (cost < best_cost) {
       best_cost = cost;
       best = S;
@@ -1135,7 +1137,7 @@ static bitnet_status gemv_fused_impl(uint16_t* out, const void* x, bitnet_dtype 
                                                   as_stream(stream));
   }
   if (norm_g == nullptr && dt == BITNET_BF16 && skq_ok(x, w_packed, M, K) &&
-      K / 128 <= sk::MAX_SPLIT * skq::MAX_KB) {
+      (K + skq::BKS - 1) / skq::BKS <= sk::MAX_SPLIT * (skq::MAX_KB / 4)) {
     const bitnet_status r =
         hook == nullptr
             ? run_gemv_skq(out, static_cast<const uint16_t*>(x), w_packed, scale_wt,

@@ -41,13 +41,17 @@ constexpr int NUM_THREADS = 512;
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = 128;            // accumulator columns reserved (BX <= 128)
 constexpr int A_COLS = BKS / 4;          // 128 columns per A stage
-// Two unpack groups take the stages in turn, each always into its own A
-// stage. The number of groups divides the number of shared-memory stages, so
-// a group that waits for a stage's k-th fill is never two fills ahead of the
-// barrier: a parity wait cannot be satisfied by an earlier fill.
-constexpr int GROUPS = 2;
-constexpr int A_STAGES = GROUPS;
+// Two groups of four unpack warps take the stages in turn. The number of
+// groups divides the number of shared-memory stages, so a group that waits
+// for a stage's k-th fill is never two fills ahead of the barrier (a parity
+// wait cannot be satisfied by an earlier fill). Three A stages in tensor
+// memory (stage it in it % 3) let the next stages be unpacked while the MMAs
+// of stage it run; their barriers stay within one phase because the MMAs
+// complete in order. (Three unpack groups, where the stages allow, measured
+// no faster: the unpack's instruction issue, not its parallelism, limits.)
+constexpr int A_STAGES = 3;
 constexpr int BAR_BYTES = 256;
+constexpr int SCAL_BYTES = 2 * 128 * 4;  // per activation row: fp32 scale, 2 * code sum
 constexpr int MAX_SPLIT = 8;
 constexpr int SMEM_CAP = 225 * 1024;
 // Shared memory is padded to more than half an SM's, so that two CTAs (which
@@ -61,11 +65,13 @@ struct Cfg {
   static constexpr int X_BYTES = 4 * X_SUB;         // BX rows x 512 K
   static constexpr int STAGE_BYTES = WP_BYTES + X_BYTES;
   static constexpr int PART_BYTES = BX * BW * 4;    // int32 partial tile [BX][BW]
-  static constexpr int ST0 = (SMEM_CAP - 1024 - BAR_BYTES) / STAGE_BYTES;
+  static constexpr int ST0 = (SMEM_CAP - 1024 - BAR_BYTES - SCAL_BYTES) / STAGE_BYTES;
+  static constexpr int GROUPS = 2;
   static constexpr int STAGES = ST0 >= 4 ? 4 : 2;
-  static constexpr int RAW = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr int RAW = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + SCAL_BYTES;
   static constexpr int SMEM_BYTES = RAW > MIN_SMEM ? RAW : MIN_SMEM;
   static_assert(STAGES >= 2 && STAGES % GROUPS == 0, "stages a multiple of the unpack groups");
+  static_assert(4 + 4 * GROUPS <= NUM_THREADS / 32, "unpack warps");
   static_assert(PART_BYTES <= STAGES * STAGE_BYTES, "the partial tile reuses the stages");
   static_assert(STAGE_BYTES % 1024 == 0 && X_SUB % 1024 == 0, "1024-byte alignment");
   static_assert(ACC_COLS + A_STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
@@ -98,6 +104,11 @@ struct Smem {
   __device__ int* abort_flag() const {
     return reinterpret_cast<int*>(bars() + 2 * ST + 2 * A_STAGES + 3);
   }
+  // the epilogue's per-activation-row scalars, staged once per CTA
+  __device__ float* row_sa() const {
+    return reinterpret_cast<float*>(base + ST * Cfg<BX>::STAGE_BYTES + BAR_BYTES);
+  }
+  __device__ int* row_corr() const { return reinterpret_cast<int*>(row_sa() + 128); }
 };
 
 // First weight row (within the tile) of CTA `rank`'s share of the reduction:
@@ -149,6 +160,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int n0 = tile * BW;
   const int kblocks = (K + BKS - 1) / BKS;
   const int kb0 = kblocks * rank / S, kb1 = kblocks * (rank + 1) / S;
+  // Each tile walks its K-slice starting at its own stage (the int32 sum is
+  // exact in any order): every tile's CTA reads the same activation tile, and
+  // staggered starts spread those reads over the L2 instead of sending every
+  // CTA to the same lines at once.
+  const int nkb = kb1 - kb0;
+  const int rot = nkb > 0 ? tile % nkb : 0;
+  auto kb_of = [&](uint32_t it) { return kb0 + static_cast<int>((it + rot) % nkb); };
   volatile int* abort = sm.abort_flag();
 
   if (threadIdx.x == 0) {
@@ -186,20 +204,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // the packed weights are load-time constants: the first stages' weight
       // tiles are requested before waiting for the previous kernel, whose
       // output the activations may be; each stage's barrier expects both
-      const int pre = min(ST, kb1 - kb0);
+      const int pre = min(ST, nkb);
       for (int i = 0; i < pre; ++i) {
         mbar_arrive_expect_tx(sm.full(i), C::STAGE_BYTES);
-        tma_load_2d(smem_u32(sm.wp(i)), &tmap_w, sm.full(i), (kb0 + i) * (BKS / 4), n0);
+        tma_load_2d(smem_u32(sm.wp(i)), &tmap_w, sm.full(i), kb_of(i) * (BKS / 4), n0);
       }
       pdl_wait();
       for (int i = 0; i < pre; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           tma_load_2d(smem_u32(sm.x(i) + j * C::X_SUB), &tmap_x, sm.full(i),
-                      (kb0 + i) * BKS + 128 * j, 0);
+                      kb_of(i) * BKS + 128 * j, 0);
       uint32_t it = static_cast<uint32_t>(pre);
-      for (int kb = kb0 + pre; kb < kb1; ++kb, ++it) {
+      for (; it < static_cast<uint32_t>(nkb); ++it) {
         const int s = it % ST;
+        const int kb = kb_of(it);
         const uint32_t ph = (it / ST) & 1u;
         if (!mbar_wait(sm.empty(s), ph ^ 1u, abort)) break;
         mbar_arrive_expect_tx(sm.full(s), C::STAGE_BYTES);
@@ -214,9 +233,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      uint32_t it = 0;
       bool ok = true;
-      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+      for (uint32_t it = 0; it < static_cast<uint32_t>(nkb); ++it) {
         const int s = it % ST;
         const int a = static_cast<int>(it % A_STAGES);
         // the unpack warps arrive only after they saw the stage land (full),
@@ -227,7 +245,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_after();
         mma_stage<BX>(tmem_base, tmem_base + static_cast<uint32_t>(ACC_COLS + a * A_COLS),
-                      smem_u32(sm.x(s)), kIdesc, kb == kb0);
+                      smem_u32(sm.x(s)), kIdesc, it == 0);
         mma_commit(sm.afree(a));
         mma_commit(sm.empty(s));  // the activation tile may be refilled
       }
@@ -235,9 +253,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mma_commit(sm.drain());
       mbar_wait_drain(sm.drain(), 0u);
     }
-  } else if (warp >= 4 && warp < 4 + 4 * GROUPS) {
+  } else if (warp >= 4 && warp < 4 + 4 * C::GROUPS) {
     // -------------------------------------------------------------- unpack
-    // Group g takes stages it = g, g + 2, ... into A stage g. A warp's
+    // Group g takes stages it = g, g + GROUPS, ... into A stage it % 3. A warp's
     // lane r owns weight row 32 * (warp % 4) + r: eight 16-byte pieces of
     // the row's 128 packed bytes (64 weights each) per stage, each expanded
     // to 16 tensor-memory columns.
@@ -245,10 +263,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t group = static_cast<uint32_t>((warp - 4) >> 2);
     const int r = sub * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(sub * 32) << 16;
-    uint32_t it = 0;
     bool ok = true;
-    for (int kb = kb0; kb < kb1; ++kb, ++it) {
-      if (it % GROUPS != group) continue;
+    for (uint32_t it = group; it < static_cast<uint32_t>(nkb); it += C::GROUPS) {
       const int s = it % ST;
       const int a = static_cast<int>(it % A_STAGES);
       if (!mbar_wait_warp(sm.full(s), (it / ST) & 1u, abort) ||
@@ -285,6 +301,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (warp < 8) {
       // ------------------------ accumulator -> registers -> (partial tile)
       const int quarter = warp & 3;
+      if (S == 1) {
+        // the epilogue's per-row scalars, staged while the last MMAs run
+        pdl_wait();  // scales and row sums may come from the previous kernel
+        for (int m = threadIdx.x - 128; m < BX; m += 128) {
+          sm.row_sa()[m] = (!kAccOut && m < M) ? bf16_bits_to_f32(scale_act[m]) : 0.0f;
+          sm.row_corr()[m] = (kPerm && m < M) ? 2 * rowsum[m] : 0;
+        }
+        named_barrier_sync(2, 128);  // warps 4-7
+      }
       if (mbar_wait_warp(sm.tfull(), 0u, abort)) {
         tc_fence_after();
         const int n = n0 + quarter * 32 + lane;
@@ -294,7 +319,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // column = activation row m (rows of a warp are consecutive n)
           float swn = 0.0f;
           if (!kAccOut && n < N) swn = scale_wt[sw_len == 1 ? 0 : n];
-          pdl_wait();  // scales and row sums may come from the previous kernel
 #pragma unroll 1
           for (int c = 0; c < BX; c += 16) {
             uint32_t v[16];
@@ -305,13 +329,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               for (int j = 0; j < 16; ++j) {
                 const int m = c + j;
                 if (m < M) {
-                  int acc = static_cast<int>(v[j]);
-                  if constexpr (kPerm) acc -= 2 * rowsum[m];
+                  const int acc = static_cast<int>(v[j]) - sm.row_corr()[m];
                   if constexpr (kAccOut) {
                     static_cast<int32_t*>(out)[static_cast<int64_t>(m) * N + n] = acc;
                   } else {
-                    const float sa = bf16_bits_to_f32(scale_act[m]);
-                    const float y = __fmul_rn(__fmul_rn(__int2float_rn(acc), sa), swn);
+                    const float y = __fmul_rn(__fmul_rn(__int2float_rn(acc), sm.row_sa()[m]), swn);
                     static_cast<uint16_t*>(out)[static_cast<int64_t>(m) * N + n] =
                         add_bias_bf16(f32_to_bf16_bits(y), bias, n);
                   }
@@ -338,6 +360,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (S > 1) {
     // ------------------------------------- cluster reduction and epilogue
     pdl_wait();  // scales and row sums may come from the previous kernel
+    for (int m = threadIdx.x; m < BX; m += NUM_THREADS) {
+      sm.row_sa()[m] = (!kAccOut && m < M) ? bf16_bits_to_f32(scale_act[m]) : 0.0f;
+      sm.row_corr()[m] = (kPerm && m < M) ? 2 * rowsum[m] : 0;
+    }
     tc_fence_before();
     __syncwarp();
     cluster_sync();  // every CTA's partial tile is in its shared memory
@@ -365,8 +391,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           a4[2] += static_cast<int>(v[q].z);
           a4[3] += static_cast<int>(v[q].w);
         }
-      if constexpr (kPerm) {
-        const int corr = 2 * rowsum[m];
+      {
+        const int corr = sm.row_corr()[m];
 #pragma unroll
         for (int j = 0; j < 4; ++j) a4[j] -= corr;
       }
@@ -379,7 +405,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int j = 0; j < 4 && n + j < N; ++j) o[j] = a4[j];
         }
       } else {
-        const float sa = bf16_bits_to_f32(scale_act[m]);
+        const float sa = sm.row_sa()[m];
         uint16_t y[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {

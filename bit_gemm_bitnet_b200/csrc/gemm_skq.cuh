@@ -13,14 +13,17 @@
 //      shared memory, directly in the 128-byte-swizzled K-major layout of the
 //      MMA's B operand (16 rows; zeros past K; rows past M are computed but
 //      never read back), where it stays for the whole K loop;
-//   3. only the packed weights stream through TMA, requested before the wait
-//      for the previous kernel (they are load-time constants); unpack warps
-//      expand them into tensor memory (the A operand) and one thread issues
-//      tcgen05.mma kind::i8;
+//   3. only the packed weights stream through TMA, 512 K per stage (one full
+//      128-byte line of each of the tile's 128 rows, 128-byte swizzled),
+//      requested before the wait for the previous kernel (they are load-time
+//      constants); unpack warps expand them into tensor memory (the A
+//      operand, 128 columns per stage) and one thread issues the stage's
+//      sixteen tcgen05.mma kind::i8;
 //   4. the int32 partials are reduced over the cluster and the epilogue
 //      bf16((acc * bf16(scale)) * scale_wt) is applied, as in gemm_sk.cuh.
-// Shared memory for the resident activations is 16 x 128 bytes per K block of
-// the slice, so the host picks S with at most MAX_KB K blocks per CTA.
+// Shared memory for the resident activations is 16 x 128 bytes per 128-wide
+// K block of the slice, so the host picks S with at most MAX_KB such blocks
+// (MAX_KB / 4 stages) per CTA.
 #pragma once
 #include "common.cuh"
 #include "gemm_sk.cuh"
@@ -30,28 +33,31 @@ namespace skq {
 
 constexpr int BX = 16;                       // MMA N: activation rows (padded)
 constexpr int BW = sk::BW;
-constexpr int BK = sk::BK;
+constexpr int BK = 128;                      // K per resident activation tile
+constexpr int BKS = 512;                     // K per weight stage
 constexpr int NUM_THREADS = sk::NUM_THREADS;
 constexpr int TMEM_COLS = sk::TMEM_COLS;
-constexpr int A_COL0 = 32;                  // A stages right after the 16-column accumulator
-constexpr int A_COLS = sk::A_COLS;
-// weight stages (60 KB in flight); a multiple of the three unpack groups, so
-// a group that waits for a stage's k-th fill is never two fills ahead of the
+constexpr int A_COL0 = 32;                   // A stages right after the 16-column accumulator
+constexpr int A_COLS = BKS / 4;              // 128 columns per A stage
+constexpr int GROUPS = 3;                    // unpack groups, each with its own A stage
+// weight stages (96 KB in flight); a multiple of the unpack groups, so a
+// group that waits for a stage's k-th fill is never two fills ahead of the
 // barrier (a parity wait cannot be satisfied by an earlier fill)
-constexpr int ST = 15;
-static_assert(ST % 3 == 0, "stages a multiple of the unpack groups");
-constexpr int WP_BYTES = sk::WP_BYTES;       // 4 KB per stage
+constexpr int ST = 6;
+static_assert(ST % GROUPS == 0, "stages a multiple of the unpack groups");
+constexpr int WP_BYTES = BW * BKS / 4;       // 16 KB per stage
 constexpr int XT_BYTES = BX * BK;            // one K block of activations, 2 KB
 constexpr int ACT_BUDGET = 96 * 1024;        // resident activations per CTA
 constexpr int MAX_KB = ACT_BUDGET / XT_BYTES;  // K blocks per CTA (48)
 constexpr int QMAX = 24;                     // activation items per thread (registers)
 constexpr int PART_BYTES = BX * BW * 4;      // int32 partial tile, 8 KB
 constexpr int HDR_BYTES = 2048;              // barriers, per-row scalars, per-warp maxima
-static_assert(3 * ST + 4 <= 64, "barriers fit below the per-row scalars");
+static_assert(2 * ST + 2 * GROUPS + 4 <= 64, "barriers fit below the per-row scalars");
 constexpr int SMEM_BYTES = 1024 + HDR_BYTES + ST * WP_BYTES + ACT_BUDGET + PART_BYTES;
 static_assert(SMEM_BYTES > 116 * 1024, "one CTA per SM (each holds all TMEM columns)");
 static_assert(SMEM_BYTES <= 232448, "too much shared memory");
-static_assert(A_COL0 + ST * A_COLS <= TMEM_COLS, "TMEM budget");
+static_assert(A_COL0 + GROUPS * A_COLS <= TMEM_COLS, "TMEM budget");
+static_assert(MAX_KB % 4 == 0, "whole stages of resident activations");
 
 // int32 D; A (weights) and B (activations) signed int8; K-major; N = 16.
 constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) |
@@ -62,14 +68,17 @@ struct Smem {
   uint8_t* base;  // 1024-aligned
   __device__ uint64_t* bars() const { return reinterpret_cast<uint64_t*>(base); }
   __device__ uint32_t full(int s) const { return smem_u32(bars() + s); }
-  __device__ uint32_t unpacked(int s) const { return smem_u32(bars() + ST + s); }
-  __device__ uint32_t empty(int s) const { return smem_u32(bars() + 2 * ST + s); }
-  __device__ uint32_t tfull() const { return smem_u32(bars() + 3 * ST); }
-  __device__ uint32_t drain() const { return smem_u32(bars() + 3 * ST + 1); }
+  __device__ uint32_t empty(int s) const { return smem_u32(bars() + ST + s); }
+  __device__ uint32_t unpacked(int a) const { return smem_u32(bars() + 2 * ST + a); }
+  __device__ uint32_t afree(int a) const { return smem_u32(bars() + 2 * ST + GROUPS + a); }
+  __device__ uint32_t tfull() const { return smem_u32(bars() + 2 * ST + 2 * GROUPS); }
+  __device__ uint32_t drain() const { return smem_u32(bars() + 2 * ST + 2 * GROUPS + 1); }
   __device__ uint32_t* tmem_slot() const {
-    return reinterpret_cast<uint32_t*>(bars() + 3 * ST + 2);
+    return reinterpret_cast<uint32_t*>(bars() + 2 * ST + 2 * GROUPS + 2);
   }
-  __device__ int* abort_flag() const { return reinterpret_cast<int*>(bars() + 3 * ST + 3); }
+  __device__ int* abort_flag() const {
+    return reinterpret_cast<int*>(bars() + 2 * ST + 2 * GROUPS + 3);
+  }
   // per activation row: this CTA's partial absmax (bf16 magnitude bits),
   // the row's quantiser (s, 1/s) and its bf16-rounded scale as fp32
   __device__ uint32_t* amax() const { return reinterpret_cast<uint32_t*>(base + 512); }
@@ -121,16 +130,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int lane = tid & 31;
   const int rank = static_cast<int>(cluster_ctarank());
   const int n0 = (blockIdx.x / S) * BW;
-  const int kblocks = (K + BK - 1) / BK;
-  const int kb0 = kblocks * rank / S, kb1 = kblocks * (rank + 1) / S;
-  const int k0 = kb0 * BK;
+  const int kstages = (K + BKS - 1) / BKS;
+  const int ks0 = kstages * rank / S, ks1 = kstages * (rank + 1) / S;
+  const int k0 = ks0 * BKS;
   volatile int* abort = sm.abort_flag();
 
   if (tid == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(sm.full(s), 1);
-      mbar_init(sm.unpacked(s), 4);
       mbar_init(sm.empty(s), 1);
+    }
+    for (int a = 0; a < GROUPS; ++a) {
+      mbar_init(sm.unpacked(a), 4);
+      mbar_init(sm.afree(a), 1);
     }
     mbar_init(sm.tfull(), 1);
     mbar_init(sm.drain(), 1);
@@ -150,11 +162,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   pdl_launch_dependents();
 
   // the first weight stages: load-time constants, requested before the wait
-  const int pre = min(ST, kb1 - kb0);
+  const int pre = min(ST, ks1 - ks0);
   if (tid == 0) {
     for (int i = 0; i < pre; ++i) {
       mbar_arrive_expect_tx(sm.full(i), WP_BYTES);
-      tma_load_2d(smem_u32(sm.wp(i)), &tmap_w, sm.full(i), (kb0 + i) * (BK / 4), n0);
+      tma_load_2d(smem_u32(sm.wp(i)), &tmap_w, sm.full(i), (ks0 + i) * (BKS / 4), n0);
     }
   }
   pdl_wait();  // x may come from the previous kernel
@@ -164,7 +176,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // the whole slice) and keeps them in registers for step 2. A warp's 32
   // consecutive items span at most two rows (a slice has a multiple of 16
   // groups), reduced separately into the warp's own slots.
-  const int k1 = min(kb1 * BK, K);
+  const int k1 = min(ks1 * BKS, K);
   const int nq = (k1 - k0) / 4;  // 4-element groups of the slice (K % 64 == 0)
   const int items = M * nq;      // <= NUM_THREADS * QMAX (host)
   const uint32_t magic = static_cast<uint32_t>((0x100000000ull + nq - 1) / nq);
@@ -223,7 +235,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
 
   // ---- 2. quantise the registers' items into the resident B tiles; the
-  // groups past K of a last, half-filled K block are zeros
+  // groups past K of a last, partly filled stage are zeros
 #pragma unroll
   for (int j = 0; j < QMAX; ++j) {
     const int i = tid + j * NUM_THREADS;
@@ -245,8 +257,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
   {
-    const int span = (kb1 - kb0) * (BK / 4);  // groups incl. the padding
-    const int pad = span - nq;                 // 0 or 16
+    const int span = (ks1 - ks0) * (BKS / 4);  // groups incl. the padding
+    const int pad = span - nq;                  // a multiple of 16, below 128
     for (int i = tid; i < M * pad; i += NUM_THREADS) {
       const int m = i / pad, kk = 4 * (nq + i - m * pad);
       *reinterpret_cast<uint32_t*>(sm.xt(kk / BK) + sw128_off(m, kk % BK)) = 0u;
@@ -259,12 +271,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       uint32_t it = static_cast<uint32_t>(pre);
-      for (int kb = kb0 + pre; kb < kb1; ++kb, ++it) {
+      for (int ks = ks0 + pre; ks < ks1; ++ks, ++it) {
         const int s = it % ST;
         const uint32_t ph = (it / ST) & 1u;
         if (!mbar_wait(sm.empty(s), ph ^ 1u, abort)) break;
         mbar_arrive_expect_tx(sm.full(s), WP_BYTES);
-        tma_load_2d(smem_u32(sm.wp(s)), &tmap_w, sm.full(s), kb * (BK / 4), n0);
+        tma_load_2d(smem_u32(sm.wp(s)), &tmap_w, sm.full(s), ks * (BKS / 4), n0);
       }
       const uint32_t first = it > ST ? it - ST : 0u;
       for (uint32_t j = first; j < it; ++j) mbar_wait_drain(sm.full(j % ST), (j / ST) & 1u);
@@ -273,21 +285,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      bool ready = false;  // the next block's unpack barrier already completed
-      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+      for (int ks = ks0; ks < ks1; ++ks, ++it) {
         const int s = it % ST;
-        // the unpack warps arrive only after they saw the stage land (full),
-        // so this wait also orders the MMA's reads of the stage
-        if (!ready && !mbar_wait(sm.unpacked(s), (it / ST) & 1u, abort)) {
+        const int a = static_cast<int>(it % GROUPS);
+        if (!mbar_wait(sm.unpacked(a), (it / GROUPS) & 1u, abort)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + s * A_COLS);
-        const uint64_t bdesc = smem_desc_sw128(smem_u32(sm.xt(kb - kb0)));
-        const uint32_t nx = it + 1;
-        ready = mma4_i8_tmem_a_test(tmem_base, a_tmem, bdesc, kIdesc, kb > kb0 ? 1u : 0u,
-                                    sm.unpacked(static_cast<int>(nx % ST)), (nx / ST) & 1u);
+        // sixteen K = 32 MMAs: A columns a0 + 8i, B the stage's four
+        // resident 128-wide activation tiles (+32 bytes per step)
+        const uint32_t a0 = tmem_base + static_cast<uint32_t>(A_COL0 + a * A_COLS);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint64_t bdesc = smem_desc_sw128(smem_u32(sm.xt(4 * (ks - ks0) + j)));
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            mma_i8_tmem_a(tmem_base, a0 + static_cast<uint32_t>(32 * j + 8 * q),
+                          bdesc + 2u * static_cast<uint32_t>(q), kIdesc,
+                          (ks > ks0 || j > 0 || q > 0) ? 1u : 0u);
+        }
+        mma_commit(sm.afree(a));
         mma_commit(sm.empty(s));
       }
       if (ok) mma_commit(sm.tfull());
@@ -295,36 +313,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait_drain(sm.drain(), 0u);
     }
   } else if (warp >= 4) {
-    // unpack: three groups of four warps take the stages in turn; warp ->
-    // TMEM sub-partition warp % 4, all 32 columns of its group's stages
+    // unpack: three groups of four warps take the stages in turn, group g
+    // always into A stage g; warp -> TMEM sub-partition warp % 4, lane r ->
+    // weight row 32 (warp % 4) + r: eight 16-byte pieces of the row's 128
+    // packed bytes (the 128-byte swizzle puts piece c at c ^ (r % 8)), each
+    // expanded to 16 tensor-memory columns
     const int sub = warp & 3;
     const uint32_t group = static_cast<uint32_t>((warp - 4) >> 2);
     const int r = sub * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(sub * 32) << 16;
     uint32_t it = 0;
-    for (int kb = kb0; kb < kb1; ++kb, ++it) {
-      if (it % 3u != group) continue;
+    for (int ks = ks0; ks < ks1; ++ks, ++it) {
+      if (it % GROUPS != group) continue;
       const int s = it % ST;
-      const uint32_t ph = (it / ST) & 1u;
-      if (!mbar_wait_warp(sm.full(s), ph, abort)) break;
-      const uint4 p0 = *reinterpret_cast<const uint4*>(sm.wp(s) + r * 32);
-      const uint4 p1 = *reinterpret_cast<const uint4*>(sm.wp(s) + r * 32 + 16);
-      uint32_t o[16], o2[16];
-      ts::signed_of(p0.x, o + 0);
-      ts::signed_of(p0.y, o + 4);
-      ts::signed_of(p0.z, o + 8);
-      ts::signed_of(p0.w, o + 12);
-      ts::signed_of(p1.x, o2 + 0);
-      ts::signed_of(p1.y, o2 + 4);
-      ts::signed_of(p1.z, o2 + 8);
-      ts::signed_of(p1.w, o2 + 12);
-      const uint32_t col = tmem_base + lane_base + static_cast<uint32_t>(A_COL0 + s * A_COLS);
-      tmem_st_32x32b_x16(col, o);
-      tmem_st_32x32b_x16(col + 16u, o2);
+      const int a = static_cast<int>(group);
+      if (!mbar_wait_warp(sm.full(s), (it / ST) & 1u, abort) ||
+          !mbar_wait_warp(sm.afree(a), ((it / GROUPS) & 1u) ^ 1u, abort))
+        break;
+      const uint8_t* row = sm.wp(s) + r * 128;
+      const uint32_t col0 = tmem_base + lane_base + static_cast<uint32_t>(A_COL0 + a * A_COLS);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 p = *reinterpret_cast<const uint4*>(row + (((c ^ r) & 7) << 4));
+        uint32_t o[16];
+        ts::signed_of(p.x, o + 0);
+        ts::signed_of(p.y, o + 4);
+        ts::signed_of(p.z, o + 8);
+        ts::signed_of(p.w, o + 12);
+        tmem_st_32x32b_x16(col0 + static_cast<uint32_t>(16 * c), o);
+      }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(sm.unpacked(s));
+      if (lane == 0) mbar_arrive(sm.unpacked(a));
     }
     if (warp < 8) {
       // accumulator -> shared partial tile [16 activation rows][128 weight rows]

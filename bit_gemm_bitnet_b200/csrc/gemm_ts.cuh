@@ -171,13 +171,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         const int m0 = (t / w_tiles) * BX;
         const int n0 = (t % w_tiles) * BW;
+        // The CTAs working on one activation tile (different weight tiles)
+        // start their K loops at different blocks (the int32 sum is exact in
+        // any order), so they do not all read the same lines at once.
+        const int rot = (t % w_tiles) % kblocks;
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!mbar_wait(sm.empty(s), ph ^ 1u, abort)) { ok = false; break; }
+          const int kr = kb + rot < kblocks ? kb + rot : kb + rot - kblocks;
           mbar_arrive_expect_tx(sm.full(s), STAGE_BYTES);
-          tma_load_2d(smem_u32(sm.x(s)), &tmap_x, sm.full(s), kb * BK, m0);
-          tma_load_2d(smem_u32(sm.wp(s)), &tmap_w, sm.full(s), kb * (BK / 4), n0);
+          tma_load_2d(smem_u32(sm.x(s)), &tmap_x, sm.full(s), kr * BK, m0);
+          tma_load_2d(smem_u32(sm.wp(s)), &tmap_w, sm.full(s), kr * (BK / 4), n0);
         }
       }
       const uint32_t first = it > STAGES ? it - STAGES : 0u;
