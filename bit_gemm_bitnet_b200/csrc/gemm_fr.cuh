@@ -22,9 +22,9 @@
 // Warp roles (512 threads, one CTA per SM):
 //   warp 0      TMA producer
 //   warp 1      tensor-memory owner, MMA issuer (one thread)
-//   warps 4-11  unpack: two groups of four warps take the stages in turn
-//               (warp -> tensor-memory lanes 32 * (warp % 4) ..); warps 4-7
-//               then move the accumulator out
+//   warps 4-11  unpack: every stage, each warp half the columns of its
+//               tensor-memory lanes 32 * (warp % 4) ..; warps 4-7 then move
+//               the accumulator out
 //   all         the reduction (S > 1) and the epilogue
 // Every wait is bounded; every thread reaches both cluster barriers.
 #pragma once
@@ -41,14 +41,14 @@ constexpr int NUM_THREADS = 512;
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = 128;            // accumulator columns reserved (BX <= 128)
 constexpr int A_COLS = BKS / 4;          // 128 columns per A stage
-// Two groups of four unpack warps take the stages in turn. The number of
-// groups divides the number of shared-memory stages, so a group that waits
-// for a stage's k-th fill is never two fills ahead of the barrier (a parity
-// wait cannot be satisfied by an earlier fill). Three A stages in tensor
+// Eight unpack warps share every stage: warp w expands columns
+// [64 (w / 4), 64 (w / 4) + 64) of tensor-memory lanes 32 (w % 4) .., half of
+// each row's 128 packed bytes, so a stage is unpacked in half the time one
+// warp per row would take. Every warp sees every stage in order, so no
+// barrier is ever waited on two phases ahead. Three A stages in tensor
 // memory (stage it in it % 3) let the next stages be unpacked while the MMAs
-// of stage it run; their barriers stay within one phase because the MMAs
-// complete in order. (Three unpack groups, where the stages allow, measured
-// no faster: the unpack's instruction issue, not its parallelism, limits.)
+// of stage it run.
+constexpr int UNPACK_WARPS = 8;
 constexpr int A_STAGES = 3;
 constexpr int BAR_BYTES = 256;
 constexpr int SCAL_BYTES = 2 * 128 * 4;  // per activation row: fp32 scale, 2 * code sum
@@ -66,12 +66,10 @@ struct Cfg {
   static constexpr int STAGE_BYTES = WP_BYTES + X_BYTES;
   static constexpr int PART_BYTES = BX * BW * 4;    // int32 partial tile [BX][BW]
   static constexpr int ST0 = (SMEM_CAP - 1024 - BAR_BYTES - SCAL_BYTES) / STAGE_BYTES;
-  static constexpr int GROUPS = 2;
   static constexpr int STAGES = ST0 >= 4 ? 4 : 2;
   static constexpr int RAW = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + SCAL_BYTES;
   static constexpr int SMEM_BYTES = RAW > MIN_SMEM ? RAW : MIN_SMEM;
-  static_assert(STAGES >= 2 && STAGES % GROUPS == 0, "stages a multiple of the unpack groups");
-  static_assert(4 + 4 * GROUPS <= NUM_THREADS / 32, "unpack warps");
+  static_assert(STAGES >= 2, "at least two stages");
   static_assert(PART_BYTES <= STAGES * STAGE_BYTES, "the partial tile reuses the stages");
   static_assert(STAGE_BYTES % 1024 == 0 && X_SUB % 1024 == 0, "1024-byte alignment");
   static_assert(ACC_COLS + A_STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
@@ -175,7 +173,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(sm.empty(s), 1);  // the stage's MMAs have completed
     }
     for (int a = 0; a < A_STAGES; ++a) {
-      mbar_init(sm.unpacked(a), 4);
+      mbar_init(sm.unpacked(a), UNPACK_WARPS);
       mbar_init(sm.afree(a), 1);
     }
     mbar_init(sm.tfull(), 1);
@@ -253,18 +251,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mma_commit(sm.drain());
       mbar_wait_drain(sm.drain(), 0u);
     }
-  } else if (warp >= 4 && warp < 4 + 4 * C::GROUPS) {
+  } else if (warp >= 4 && warp < 4 + UNPACK_WARPS) {
     // -------------------------------------------------------------- unpack
-    // Group g takes stages it = g, g + GROUPS, ... into A stage it % 3. A warp's
-    // lane r owns weight row 32 * (warp % 4) + r: eight 16-byte pieces of
-    // the row's 128 packed bytes (64 weights each) per stage, each expanded
-    // to 16 tensor-memory columns.
+    // Lane r of warp w owns weight row 32 * (w % 4) + r and the half
+    // h = (w - 4) / 4 of its 128 packed bytes: four 16-byte pieces (64
+    // weights each; the 128-byte swizzle puts piece c at c ^ (r % 8)), each
+    // expanded to 16 tensor-memory columns of the stage's A stage it % 3.
     const int sub = warp & 3;
-    const uint32_t group = static_cast<uint32_t>((warp - 4) >> 2);
+    const int half = (warp - 4) >> 2;
     const int r = sub * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(sub * 32) << 16;
     bool ok = true;
-    for (uint32_t it = group; it < static_cast<uint32_t>(nkb); it += C::GROUPS) {
+    for (uint32_t it = 0; it < static_cast<uint32_t>(nkb); ++it) {
       const int s = it % ST;
       const int a = static_cast<int>(it % A_STAGES);
       if (!mbar_wait_warp(sm.full(s), (it / ST) & 1u, abort) ||
@@ -272,11 +270,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ok = false;
         break;
       }
-      // the 128-byte swizzle puts 16-byte piece c of row r at c ^ (r % 8)
       const uint8_t* row = sm.wp(s) + r * 128;
       const uint32_t col0 = tmem_base + lane_base + static_cast<uint32_t>(ACC_COLS + a * A_COLS);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c = 4 * half + cc;
         const uint4 p = *reinterpret_cast<const uint4*>(row + (((c ^ r) & 7) << 4));
         uint32_t o[16];
         if constexpr (kPerm) {

@@ -39,12 +39,13 @@ constexpr int NUM_THREADS = sk::NUM_THREADS;
 constexpr int TMEM_COLS = sk::TMEM_COLS;
 constexpr int A_COL0 = 32;                   // A stages right after the 16-column accumulator
 constexpr int A_COLS = BKS / 4;              // 128 columns per A stage
-constexpr int GROUPS = 3;                    // unpack groups, each with its own A stage
-// weight stages (96 KB in flight); a multiple of the unpack groups, so a
-// group that waits for a stage's k-th fill is never two fills ahead of the
-// barrier (a parity wait cannot be satisfied by an earlier fill)
-constexpr int ST = 6;
-static_assert(ST % GROUPS == 0, "stages a multiple of the unpack groups");
+// Eight unpack warps share every stage (each half the columns of its 32
+// tensor-memory lanes); every warp sees every stage in order, so no barrier
+// is ever waited on two phases ahead. Three A stages in tensor memory (stage
+// it in it % 3) let the next stages be unpacked while the MMAs run.
+constexpr int UNPACK_WARPS = 8;
+constexpr int GROUPS = 3;                    // A stages
+constexpr int ST = 6;                        // weight stages (96 KB in flight)
 constexpr int WP_BYTES = BW * BKS / 4;       // 16 KB per stage
 constexpr int XT_BYTES = BX * BK;            // one K block of activations, 2 KB
 constexpr int ACT_BUDGET = 96 * 1024;        // resident activations per CTA
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(sm.empty(s), 1);
     }
     for (int a = 0; a < GROUPS; ++a) {
-      mbar_init(sm.unpacked(a), 4);
+      mbar_init(sm.unpacked(a), UNPACK_WARPS);
       mbar_init(sm.afree(a), 1);
     }
     mbar_init(sm.tfull(), 1);
@@ -312,28 +313,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mma_commit(sm.drain());
       mbar_wait_drain(sm.drain(), 0u);
     }
-  } else if (warp >= 4) {
-    // unpack: three groups of four warps take the stages in turn, group g
-    // always into A stage g; warp -> TMEM sub-partition warp % 4, lane r ->
-    // weight row 32 (warp % 4) + r: eight 16-byte pieces of the row's 128
-    // packed bytes (the 128-byte swizzle puts piece c at c ^ (r % 8)), each
-    // expanded to 16 tensor-memory columns
+  } else if (warp >= 4 && warp < 4 + UNPACK_WARPS) {
+    // unpack: every stage, lane r of warp w -> weight row 32 (w % 4) + r and
+    // the half h = (w - 4) / 4 of its 128 packed bytes: four 16-byte pieces
+    // (the 128-byte swizzle puts piece c at c ^ (r % 8)), each expanded to 16
+    // tensor-memory columns of the stage's A stage it % 3
     const int sub = warp & 3;
-    const uint32_t group = static_cast<uint32_t>((warp - 4) >> 2);
+    const int half = (warp - 4) >> 2;
     const int r = sub * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(sub * 32) << 16;
     uint32_t it = 0;
     for (int ks = ks0; ks < ks1; ++ks, ++it) {
-      if (it % GROUPS != group) continue;
       const int s = it % ST;
-      const int a = static_cast<int>(group);
+      const int a = static_cast<int>(it % GROUPS);
       if (!mbar_wait_warp(sm.full(s), (it / ST) & 1u, abort) ||
           !mbar_wait_warp(sm.afree(a), ((it / GROUPS) & 1u) ^ 1u, abort))
         break;
       const uint8_t* row = sm.wp(s) + r * 128;
       const uint32_t col0 = tmem_base + lane_base + static_cast<uint32_t>(A_COL0 + a * A_COLS);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c = 4 * half + cc;
         const uint4 p = *reinterpret_cast<const uint4*>(row + (((c ^ r) & 7) << 4));
         uint32_t o[16];
         ts::signed_of(p.x, o + 0);
