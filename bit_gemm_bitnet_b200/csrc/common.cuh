@@ -94,9 +94,12 @@ __device__ __forceinline__ int quant_one(float x, const RowQuant& q) {
 
 // The layer's bias (BitLinear.forward on the bitnet-cpu page adds it to the
 // bf16 output): bf16(float(y) + float(bias[n])); no bias when bias is null.
+__device__ __forceinline__ uint16_t add_bias_bf16_v(uint16_t y, uint16_t b) {
+  return f32_to_bf16_bits(__fadd_rn(bf16_bits_to_f32(y), bf16_bits_to_f32(b)));
+}
 __device__ __forceinline__ uint16_t add_bias_bf16(uint16_t y, const uint16_t* bias, int64_t n) {
   if (bias == nullptr) return y;
-  return f32_to_bf16_bits(__fadd_rn(bf16_bits_to_f32(y), bf16_bits_to_f32(bias[n])));
+  return add_bias_bf16_v(y, bias[n]);
 }
 
 // --------------------------------------------------------- PDL (griddep)

@@ -51,7 +51,9 @@ constexpr int A_COLS = BKS / 4;          // 128 columns per A stage
 constexpr int UNPACK_WARPS = 8;
 constexpr int A_STAGES = 3;
 constexpr int BAR_BYTES = 256;
-constexpr int SCAL_BYTES = 2 * 128 * 4;  // per activation row: fp32 scale, 2 * code sum
+// per activation row: fp32 scale, 2 * code sum; per weight row: fp32 scale,
+// bf16 bias
+constexpr int SCAL_BYTES = 3 * 128 * 4 + 128 * 2;
 constexpr int MAX_SPLIT = 8;
 constexpr int SMEM_CAP = 225 * 1024;
 // Shared memory is padded to more than half an SM's, so that two CTAs (which
@@ -107,6 +109,9 @@ struct Smem {
     return reinterpret_cast<float*>(base + ST * Cfg<BX>::STAGE_BYTES + BAR_BYTES);
   }
   __device__ int* row_corr() const { return reinterpret_cast<int*>(row_sa() + 128); }
+  // the reduction's per-weight-row scalars (S > 1), staged once per CTA
+  __device__ float* col_sw() const { return row_sa() + 256; }
+  __device__ uint16_t* col_bias() const { return reinterpret_cast<uint16_t*>(row_sa() + 384); }
 };
 
 // First weight row (within the tile) of CTA `rank`'s share of the reduction:
@@ -308,33 +313,68 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         named_barrier_sync(2, 128);  // warps 4-7
       }
+      // lane = weight row n of this warp's quarter of the tile
+      const int nq = n0 + quarter * 32;
+      const int n = nq + lane;
+      float swn = 0.0f;
+      uint16_t bn = 0;
+      if (S == 1 && !kAccOut && n < N) {
+        swn = scale_wt[sw_len == 1 ? 0 : n];
+        if (bias != nullptr) bn = bias[n];
+      }
       if (mbar_wait_warp(sm.tfull(), 0u, abort)) {
         tc_fence_after();
-        const int n = n0 + quarter * 32 + lane;
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
         if (S == 1) {
-          // the epilogue straight from the accumulator: lane = weight row n,
-          // column = activation row m (rows of a warp are consecutive n)
-          float swn = 0.0f;
-          if (!kAccOut && n < N) swn = scale_wt[sw_len == 1 ? 0 : n];
+          // The epilogue straight from the accumulator (column = activation
+          // row m), CH rows at a time. Lane j holds row j's scalars and the
+          // shuffles hand them out; the chunk goes through a shared-memory
+          // patch (the stage buffers are idle once tfull has fired) and
+          // leaves as 16-byte pieces of output rows.
+          constexpr int CH = BX < 32 ? BX : 32;
+          constexpr int EB = kAccOut ? 4 : 2;        // output element bytes
+          constexpr int PER_ROW = 32 * EB / 16;      // 16-byte pieces per patch row
+          uint8_t* stg = sm.wp(0) + quarter * (32 * 32 * 4);
 #pragma unroll 1
-          for (int c = 0; c < BX; c += 16) {
-            uint32_t v[16];
-            tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(c), v);
+          for (int c = 0; c < BX; c += CH) {
+            const float sa_l = sm.row_sa()[c + (lane & (CH - 1))];
+            const int corr_l = sm.row_corr()[c + (lane & (CH - 1))];
+            uint32_t v[CH];
+            if constexpr (CH == 32) {
+              tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c), v);
+            } else {
+              tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(c), v);
+            }
             tmem_ld_wait();
-            if (n < N) {
+            __syncwarp();  // the previous chunk's reads of the patch are done
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const int m = c + j;
-                if (m < M) {
-                  const int acc = static_cast<int>(v[j]) - sm.row_corr()[m];
-                  if constexpr (kAccOut) {
-                    static_cast<int32_t*>(out)[static_cast<int64_t>(m) * N + n] = acc;
-                  } else {
-                    const float y = __fmul_rn(__fmul_rn(__int2float_rn(acc), sm.row_sa()[m]), swn);
-                    static_cast<uint16_t*>(out)[static_cast<int64_t>(m) * N + n] =
-                        add_bias_bf16(f32_to_bf16_bits(y), bias, n);
-                  }
+            for (int j = 0; j < CH; ++j) {
+              const int acc = static_cast<int>(v[j]) - __shfl_sync(0xFFFFFFFFu, corr_l, j);
+              if constexpr (kAccOut) {
+                reinterpret_cast<int32_t*>(stg)[j * 32 + lane] = acc;
+              } else {
+                const float sa_j = __shfl_sync(0xFFFFFFFFu, sa_l, j);
+                const uint16_t y = f32_to_bf16_bits(__fmul_rn(__fmul_rn(__int2float_rn(acc), sa_j), swn));
+                reinterpret_cast<uint16_t*>(stg)[j * 32 + lane] =
+                    bias != nullptr ? add_bias_bf16_v(y, bn) : y;
+              }
+            }
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < CH * PER_ROW / 32; ++i) {
+              const int piece = lane + 32 * i;
+              const int j = piece / PER_ROW;
+              const int col = (piece % PER_ROW) * (16 / EB);
+              const int m = c + j;
+              const int nc = nq + col;
+              if (m < M && nc < N) {
+                uint8_t* dst = static_cast<uint8_t*>(out) + (static_cast<int64_t>(m) * N + nc) * EB;
+                const uint8_t* src = stg + (j * 32 + col) * EB;
+                if (nc + 16 / EB <= N && ((N * EB) & 15) == 0) {
+                  *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+                } else {
+                  for (int e = 0; e < 16 / EB && nc + e < N; ++e)
+                    for (int b = 0; b < EB; ++b) dst[e * EB + b] = src[e * EB + b];
                 }
               }
             }
@@ -361,6 +401,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int m = threadIdx.x; m < BX; m += NUM_THREADS) {
       sm.row_sa()[m] = (!kAccOut && m < M) ? bf16_bits_to_f32(scale_act[m]) : 0.0f;
       sm.row_corr()[m] = (kPerm && m < M) ? 2 * rowsum[m] : 0;
+    }
+    for (int i = threadIdx.x; i < BW; i += NUM_THREADS) {
+      const int n = n0 + i;
+      sm.col_sw()[i] = (!kAccOut && n < N) ? scale_wt[sw_len == 1 ? 0 : n] : 0.0f;
+      sm.col_bias()[i] = (bias != nullptr && n < N) ? bias[n] : static_cast<uint16_t>(0);
     }
     tc_fence_before();
     __syncwarp();
@@ -407,9 +452,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint16_t y[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float swj = (n + j < N) ? scale_wt[sw_len == 1 ? 0 : n + j] : 0.0f;
-          y[j] = f32_to_bf16_bits(__fmul_rn(__fmul_rn(__int2float_rn(a4[j]), sa), swj));
-          if (bias != nullptr && n + j < N) y[j] = add_bias_bf16(y[j], bias, n + j);
+          y[j] = f32_to_bf16_bits(__fmul_rn(__fmul_rn(__int2float_rn(a4[j]), sa), sm.col_sw()[rl + j]));
+          if (bias != nullptr) y[j] = add_bias_bf16_v(y[j], sm.col_bias()[rl + j]);
         }
         uint16_t* o = static_cast<uint16_t*>(out) + static_cast<int64_t>(m) * N + n;
         if (whole) {

@@ -53,7 +53,10 @@ struct Cfg {
   static constexpr int X_BYTES = BX * BK;
   static constexpr int STAGE_BYTES = X_BYTES + WP_BYTES;
   static constexpr int PART_BYTES = BX * BW * 4;   // int32 partial tile [BX][BW]
-  static constexpr int RAW = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  // the reduction's scalars: per activation row fp32 scale and 2 * code sum,
+  // per weight row fp32 scale and bf16 bias
+  static constexpr int SCAL_BYTES = 2 * BX * 4 + BW * 4 + BW * 2;
+  static constexpr int RAW = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + SCAL_BYTES;
   static constexpr int SMEM_BYTES = RAW > MIN_SMEM ? RAW : MIN_SMEM;
   static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(PART_BYTES <= STAGES * STAGE_BYTES, "the partial tile reuses the stages");
@@ -87,6 +90,13 @@ struct Smem {
     return reinterpret_cast<uint32_t*>(bars() + 3 * ST + 2);
   }
   __device__ int* abort_flag() const { return reinterpret_cast<int*>(bars() + 3 * ST + 3); }
+  // the reduction's scalars, staged once per CTA before it
+  __device__ float* row_sa() const {
+    return reinterpret_cast<float*>(base + ST * Cfg<BX>::STAGE_BYTES + BAR_BYTES);
+  }
+  __device__ int* row_corr() const { return reinterpret_cast<int*>(row_sa() + BX); }
+  __device__ float* col_sw() const { return row_sa() + 2 * BX; }
+  __device__ uint16_t* col_bias() const { return reinterpret_cast<uint16_t*>(col_sw() + BW); }
 };
 
 // First weight row (within the tile) of CTA `rank`'s share of the reduction:
@@ -280,9 +290,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   // --------------------------------------- cluster reduction and epilogue
   pdl_wait();  // scales and row sums may come from the previous kernel
+  for (int m = threadIdx.x; m < BX; m += NUM_THREADS) {
+    sm.row_sa()[m] = (!kAccOut && m < M) ? bf16_bits_to_f32(scale_act[m]) : 0.0f;
+    sm.row_corr()[m] = (kPerm && m < M) ? 2 * rowsum[m] : 0;
+  }
+  for (int i = threadIdx.x; i < BW; i += NUM_THREADS) {
+    const int n = n0 + i;
+    sm.col_sw()[i] = (!kAccOut && n < N) ? scale_wt[sw_len == 1 ? 0 : n] : 0.0f;
+    sm.col_bias()[i] = (bias != nullptr && n < N) ? bias[n] : static_cast<uint16_t>(0);
+  }
   tc_fence_before();
   __syncwarp();
-  cluster_sync();  // every CTA's partial tile is in its shared memory
+  cluster_sync();  // every CTA's partial tile (and the scalars) are in shared memory
   {
     const int r_lo = share_row(rank, S), r_hi = share_row(rank + 1, S);
     const int G = (r_hi - r_lo) / 4;  // 16-byte groups per activation row
@@ -309,7 +328,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           a[3] += static_cast<int>(v[q].w);
         }
       if constexpr (kPerm) {
-        const int corr = 2 * rowsum[m];
+        const int corr = sm.row_corr()[m];
 #pragma unroll
         for (int j = 0; j < 4; ++j) a[j] -= corr;
       }
@@ -322,13 +341,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int j = 0; j < 4 && n + j < N; ++j) o[j] = a[j];
         }
       } else {
-        const float sa = bf16_bits_to_f32(scale_act[m]);
+        const float sa = sm.row_sa()[m];
         uint16_t y[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float swj = (n + j < N) ? scale_wt[sw_len == 1 ? 0 : n + j] : 0.0f;
-          y[j] = f32_to_bf16_bits(__fmul_rn(__fmul_rn(__int2float_rn(a[j]), sa), swj));
-          if (bias != nullptr && n + j < N) y[j] = add_bias_bf16(y[j], bias, n + j);
+          y[j] = f32_to_bf16_bits(__fmul_rn(__fmul_rn(__int2float_rn(a[j]), sa), sm.col_sw()[rl + j]));
+          if (bias != nullptr) y[j] = add_bias_bf16_v(y[j], sm.col_bias()[rl + j]);
         }
         uint16_t* o = static_cast<uint16_t*>(out) + static_cast<int64_t>(m) * N + n;
         if (whole) {

@@ -52,7 +52,7 @@ constexpr int ACT_BUDGET = 96 * 1024;        // resident activations per CTA
 constexpr int MAX_KB = ACT_BUDGET / XT_BYTES;  // K blocks per CTA (48)
 constexpr int QMAX = 24;                     // activation items per thread (registers)
 constexpr int PART_BYTES = BX * BW * 4;      // int32 partial tile, 8 KB
-constexpr int HDR_BYTES = 2048;              // barriers, per-row scalars, per-warp maxima
+constexpr int HDR_BYTES = 3072;              // barriers, per-row and per-column scalars, per-warp maxima
 static_assert(2 * ST + 2 * GROUPS + 4 <= 64, "barriers fit below the per-row scalars");
 constexpr int SMEM_BYTES = 1024 + HDR_BYTES + ST * WP_BYTES + ACT_BUDGET + PART_BYTES;
 static_assert(SMEM_BYTES > 116 * 1024, "one CTA per SM (each holds all TMEM columns)");
@@ -88,6 +88,9 @@ struct Smem {
   __device__ float* rq_s() const { return reinterpret_cast<float*>(base + 576); }
   __device__ float* rq_r() const { return reinterpret_cast<float*>(base + 640); }
   __device__ float* saf() const { return reinterpret_cast<float*>(base + 704); }
+  // per weight row of the tile: fp32 scale and bf16 bias, for the reduction
+  __device__ float* col_sw() const { return reinterpret_cast<float*>(base + 2048); }
+  __device__ uint16_t* col_bias() const { return reinterpret_cast<uint16_t*>(base + 2560); }
   __device__ uint8_t* wp(int s) const { return base + HDR_BYTES + s * WP_BYTES; }
   // K block j of the CTA's slice: 16 rows x 128 bytes, 128-byte swizzle
   __device__ uint8_t* xt(int j) const { return base + HDR_BYTES + ST * WP_BYTES + j * XT_BYTES; }
@@ -363,9 +366,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 
   // ---- 4. cluster reduction and epilogue
+  for (int i = tid; i < BW; i += NUM_THREADS) {
+    const int n = n0 + i;
+    sm.col_sw()[i] = (!kAccOut && n < N) ? scale_wt[sw_len == 1 ? 0 : n] : 0.0f;
+    sm.col_bias()[i] = (bias != nullptr && n < N) ? bias[n] : static_cast<uint16_t>(0);
+  }
   tc_fence_before();
   __syncwarp();
-  cluster_sync();  // every CTA's partial tile is in its shared memory
+  cluster_sync();  // every CTA's partial tile (and the scalars) are in shared memory
   {
     const int r_lo = sk::share_row(rank, S), r_hi = sk::share_row(rank + 1, S);
     const int G = (r_hi - r_lo) / 4;
@@ -404,9 +412,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint16_t y[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float swj = (n + j < N) ? scale_wt[sw_len == 1 ? 0 : n + j] : 0.0f;
-        y[j] = f32_to_bf16_bits(__fmul_rn(__fmul_rn(__int2float_rn(a[j]), sa), swj));
-        if (bias != nullptr && n + j < N) y[j] = add_bias_bf16(y[j], bias, n + j);
+        y[j] = f32_to_bf16_bits(__fmul_rn(__fmul_rn(__int2float_rn(a[j]), sa), sm.col_sw()[rl + j]));
+        if (bias != nullptr) y[j] = add_bias_bf16_v(y[j], sm.col_bias()[rl + j]);
       }
       uint16_t* o = static_cast<uint16_t*>(out) + static_cast<int64_t>(m) * N + n;
       if (n + 3 < N && (N & 3) == 0) {
