@@ -137,8 +137,9 @@ __device__ __forceinline__ void mma_stage(uint32_t d_tmem, uint32_t a_tmem, uint
 
 // kPerm: activations with transposed 16-element groups plus per-row code
 // sums (bitnet_linear's workspace); weights enter as unsigned code planes and
-// the epilogue subtracts 2 * rowsum[m]. Otherwise natural order and signed
-// weights. kAccOut: int32 sums to `out` instead of the bf16 epilogue.
+// the epilogue subtracts 2 * rowsum[m]. Otherwise natural order: the weights
+// enter as 64 * w (signed), and the sums leave the accumulator shifted right
+// by 6. kAccOut: int32 sums to `out` instead of the bf16 epilogue.
 // Grid: (N / BW tiles) x S CTAs, clusters of S consecutive CTAs; M <= BX.
 template <int BX, bool kAccOut, bool kPerm>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -151,6 +152,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   using C = Cfg<BX>;
   constexpr int ST = C::STAGES;
   constexpr uint32_t kIdesc = kPerm ? C::kIdescShape : (C::kIdescShape | (1u << 7));
+  constexpr int kShift = kPerm ? 0 : ts::kScaledShift;
   extern __shared__ uint8_t smem_raw[];
   Smem<BX> sm;
   sm.base = reinterpret_cast<uint8_t*>(
@@ -288,10 +290,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ts::planes_of(p.z, o + 8);
           ts::planes_of(p.w, o + 12);
         } else {
-          ts::signed_of(p.x, o + 0);
-          ts::signed_of(p.y, o + 4);
-          ts::signed_of(p.z, o + 8);
-          ts::signed_of(p.w, o + 12);
+          ts::scaled_of(p.x, o + 0);
+          ts::scaled_of(p.y, o + 4);
+          ts::scaled_of(p.z, o + 8);
+          ts::scaled_of(p.w, o + 12);
         }
         tmem_st_32x32b_x16(col0 + static_cast<uint32_t>(16 * c), o);
       }
@@ -349,7 +351,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             __syncwarp();  // the previous chunk's reads of the patch are done
 #pragma unroll
             for (int j = 0; j < CH; ++j) {
-              const int acc = static_cast<int>(v[j]) - __shfl_sync(0xFFFFFFFFu, corr_l, j);
+              const int acc = (static_cast<int>(v[j]) >> kShift) - __shfl_sync(0xFFFFFFFFu, corr_l, j);
               if constexpr (kAccOut) {
                 reinterpret_cast<int32_t*>(stg)[j * 32 + lane] = acc;
               } else {
@@ -388,7 +390,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(c), v);
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) part[(c + j) * BW + rr] = static_cast<int32_t>(v[j]);
+            for (int j = 0; j < 16; ++j) part[(c + j) * BW + rr] = static_cast<int32_t>(v[j]) >> kShift;
           }
         }
       }

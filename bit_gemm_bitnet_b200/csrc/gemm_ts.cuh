@@ -89,6 +89,30 @@ __device__ __forceinline__ void planes_of(uint32_t w, uint32_t* o) {
   o[3] = (w >> 6) & 0x03030303u;
 }
 
+// Packed word -> its 16 weights times 64, as int8 in element order (4
+// words). Field i of every byte, XOR 2 (the code minus 2, modulo 4), is
+// moved to the top two bits of its byte, where it reads as (code - 2) * 64;
+// a 4 x 4 byte transpose then puts the fields in element order (field i of
+// byte j is element 4j + i). Sums over these weights are 64 times the true
+// sums: exact in int32 while 64 * |sum| < 2^31, and shifted back right by 6.
+// Twelve integer-pipe operations per word; the three shifts may go to the
+// multiply-add pipe.
+constexpr int kScaledShift = 6;
+__device__ __forceinline__ void scaled_of(uint32_t w, uint32_t* o) {
+  const uint32_t e0 = ((w & 0x03030303u) ^ 0x02020202u) * 64u;
+  const uint32_t e1 = ((w & 0x0C0C0C0Cu) ^ 0x08080808u) * 16u;
+  const uint32_t e2 = ((w & 0x30303030u) ^ 0x20202020u) * 4u;
+  const uint32_t e3 = (w & 0xC0C0C0C0u) ^ 0x80808080u;
+  const uint32_t t0 = prmt(e0, e1, 0x5140u);
+  const uint32_t t1 = prmt(e0, e1, 0x7362u);
+  const uint32_t t2 = prmt(e2, e3, 0x5140u);
+  const uint32_t t3 = prmt(e2, e3, 0x7362u);
+  o[0] = prmt(t0, t2, 0x5410u);
+  o[1] = prmt(t0, t2, 0x7632u);
+  o[2] = prmt(t1, t3, 0x5410u);
+  o[3] = prmt(t1, t3, 0x7632u);
+}
+
 // Packed word -> 16 signed int8 weights in element order (4 words).
 __device__ __forceinline__ void signed_of(uint32_t w, uint32_t* o) {
   const uint32_t e0 = ((w & 0x03030303u) | 0x80808080u) - 0x02020202u;

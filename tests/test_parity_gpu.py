@@ -223,6 +223,22 @@ def test_gemm_extreme_accumulators():
     assert np.array_equal(acc, oracle.acc(q, p))
 
 
+@pytest.mark.parametrize("K", [131008, 131072])
+def test_gemm_scaled_weight_limit(K):
+    # The natural-order few-row kernel sums 64 * w in int32. At its largest K,
+    # x = -128 against code 0 (w = -2) gives 64 * 256 * K just below 2^31; one
+    # step beyond, the call takes the 256-row split-K kernel. Both are exact.
+    M, N = 2, 128
+    q = np.full((M, K), -128, np.int8)
+    q[1] = 127
+    p = np.random.default_rng(K).integers(0, 256, (N, K // 4), dtype=np.uint8)
+    p[0] = 0x00  # code 0 everywhere: w = -2
+    p[1] = 0xFF  # code 3 everywhere: w = +1
+    acc = bn.bitnet_gemm_acc_i32(to_dev(q), to_dev(p)).cpu().numpy()
+    assert np.array_equal(acc, oracle.acc(q, p))
+    assert acc[0, 0] == 256 * K and acc[1, 1] == 127 * K
+
+
 def test_gemm_empty_and_sentinel():
     # M = 0 is a no-op; outputs outside [M, N] are never written
     p = torch.zeros((64, 128), dtype=torch.uint8, device="cuda")
