@@ -23,8 +23,8 @@
 //   warp 0      TMA producer
 //   warp 1      tensor-memory owner, MMA issuer (one thread)
 //   warps 4-11  unpack: every stage, each warp half the columns of its
-//               tensor-memory lanes 32 * (warp % 4) ..; warps 4-7 then move
-//               the accumulator out
+//               tensor-memory lanes 32 * (warp % 4) ..; then each moves half
+//               the accumulator columns of those lanes out
 //   all         the reduction (S > 1) and the epilogue
 // Every wait is bounded; every thread reaches both cluster barriers.
 #pragma once
@@ -73,6 +73,7 @@ struct Cfg {
   static constexpr int SMEM_BYTES = RAW > MIN_SMEM ? RAW : MIN_SMEM;
   static_assert(STAGES >= 2, "at least two stages");
   static_assert(PART_BYTES <= STAGES * STAGE_BYTES, "the partial tile reuses the stages");
+  static_assert(8 * 32 * 32 * 4 <= STAGES * STAGE_BYTES, "the epilogue patches reuse the stages");
   static_assert(STAGE_BYTES % 1024 == 0 && X_SUB % 1024 == 0, "1024-byte alignment");
   static_assert(ACC_COLS + A_STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "too much shared memory");
@@ -303,17 +304,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (lane == 0) mbar_arrive(sm.unpacked(a));
     }
     (void)ok;
-    if (warp < 8) {
+    {
       // ------------------------ accumulator -> registers -> (partial tile)
+      // Warp w reads the tensor-memory lanes of quarter w % 4 and takes every
+      // other chunk of activation rows, from chunk (w - 4) / 4 on.
       const int quarter = warp & 3;
+      const int ehalf = (warp - 4) >> 2;
       if (S == 1) {
         // the epilogue's per-row scalars, staged while the last MMAs run
         pdl_wait();  // scales and row sums may come from the previous kernel
-        for (int m = threadIdx.x - 128; m < BX; m += 128) {
+        for (int m = threadIdx.x - 128; m < BX; m += 256) {
           sm.row_sa()[m] = (!kAccOut && m < M) ? bf16_bits_to_f32(scale_act[m]) : 0.0f;
           sm.row_corr()[m] = (kPerm && m < M) ? 2 * rowsum[m] : 0;
         }
-        named_barrier_sync(2, 128);  // warps 4-7
+        named_barrier_sync(2, 256);  // warps 4-11
       }
       // lane = weight row n of this warp's quarter of the tile
       const int nq = n0 + quarter * 32;
@@ -336,9 +340,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           constexpr int CH = BX < 32 ? BX : 32;
           constexpr int EB = kAccOut ? 4 : 2;        // output element bytes
           constexpr int PER_ROW = 32 * EB / 16;      // 16-byte pieces per patch row
-          uint8_t* stg = sm.wp(0) + quarter * (32 * 32 * 4);
+          uint8_t* stg = sm.wp(0) + (warp - 4) * (32 * 32 * 4);
 #pragma unroll 1
-          for (int c = 0; c < BX; c += CH) {
+          for (int c = ehalf * CH; c < BX; c += 2 * CH) {
             const float sa_l = sm.row_sa()[c + (lane & (CH - 1))];
             const int corr_l = sm.row_corr()[c + (lane & (CH - 1))];
             uint32_t v[CH];
@@ -385,7 +389,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           int32_t* part = sm.part();
           const int rr = quarter * 32 + lane;
 #pragma unroll 1
-          for (int c = 0; c < BX; c += 16) {
+          for (int c = ehalf * 16; c < BX; c += 32) {
             uint32_t v[16];
             tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(c), v);
             tmem_ld_wait();
