@@ -567,8 +567,9 @@ bool gemm_tc_ok(const int8_t* xq, const uint8_t* wp, int64_t K) {
   return (K % 64) == 0 && aligned(xq, 16) && aligned(wp, 16);
 }
 
-// The natural-order few-row kernel takes the weights as 64 * w: its int32
-// sums stay exact while 64 * 256 * K < 2^31 (|x| <= 128, |w| <= 2).
+// The natural-order few-row and split-K kernels take the weights as 64 * w:
+// their int32 sums stay exact while 64 * 256 * K < 2^31 (|x| <= 128,
+// |w| <= 2). Longer K goes to the persistent kernel (signed weights).
 constexpr int64_t kScaledMaxK = INT32_MAX / (64 * 256) / 64 * 64;
 
 // ------------------------------------------------- few-row GEMM (M <= 256)
@@ -721,11 +722,8 @@ bitnet_status run_gemm_sk(void* out, bool acc_out, const int8_t* xq, const uint8
                           const uint16_t* sa, const float* sw, int64_t sw_len, int64_t M,
                           int64_t N, int64_t K, cudaStream_t st, bool perm,
                           const int32_t* rowsum, const uint16_t* bias) {
-  // up to 128 rows: the few-row kernel with 512-wide K stages; more (or a K
-  // too long for its scaled natural-order weights): the split-K kernel's
-  // 256-row tile
-  if (!perm && K > kScaledMaxK)
-    return run_sk_bx<256>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
+  // up to 128 rows: the few-row kernel with 512-wide K stages; more: the
+  // split-K kernel's 256-row tile
   if (M <= 16) return run_fr_bx<16>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
   if (M <= 32) return run_fr_bx<32>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
   if (M <= 64) return run_fr_bx<64>(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
@@ -806,7 +804,7 @@ bitnet_status run_gemm(void* out, bool acc_out, const int8_t* xq, const uint8_t*
     p.bias = bias;
     return run_gemv(p, true, st);
   }
-  if (M <= kSkMaxRows)
+  if (M <= kSkMaxRows && (perm || K <= kScaledMaxK))
     return run_gemm_sk(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
   DeviceInfo* dev = nullptr;
   bitnet_status s = device_info(&dev);

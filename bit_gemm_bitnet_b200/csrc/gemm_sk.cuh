@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   using C = Cfg<BX>;
   constexpr int ST = C::STAGES;
   constexpr uint32_t kIdesc = kPerm ? C::kIdescShape : (C::kIdescShape | (1u << 7));
+  constexpr int kShift = kPerm ? 0 : ts::kScaledShift;  // natural order: 64 * w
   extern __shared__ uint8_t smem_raw[];
   Smem<BX> sm;
   sm.base = reinterpret_cast<uint8_t*>(
@@ -243,14 +244,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ts::planes_of(p1.z, o2 + 8);
         ts::planes_of(p1.w, o2 + 12);
       } else {
-        ts::signed_of(p0.x, o + 0);
-        ts::signed_of(p0.y, o + 4);
-        ts::signed_of(p0.z, o + 8);
-        ts::signed_of(p0.w, o + 12);
-        ts::signed_of(p1.x, o2 + 0);
-        ts::signed_of(p1.y, o2 + 4);
-        ts::signed_of(p1.z, o2 + 8);
-        ts::signed_of(p1.w, o2 + 12);
+        ts::scaled_of(p0.x, o + 0);
+        ts::scaled_of(p0.y, o + 4);
+        ts::scaled_of(p0.z, o + 8);
+        ts::scaled_of(p0.w, o + 12);
+        ts::scaled_of(p1.x, o2 + 0);
+        ts::scaled_of(p1.y, o2 + 4);
+        ts::scaled_of(p1.z, o2 + 8);
+        ts::scaled_of(p1.w, o2 + 12);
       }
       const uint32_t col = tmem_base + lane_base + static_cast<uint32_t>(A_COL0 + s * A_COLS);
       tmem_st_32x32b_x16(col, o);
@@ -275,13 +276,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tmem_ld_32x32b_x16(taddr, v);
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) part[(c + j) * BW + r] = static_cast<int32_t>(v[j]);
+            for (int j = 0; j < 16; ++j) part[(c + j) * BW + r] = static_cast<int32_t>(v[j]) >> kShift;
           } else {
             uint32_t v[32];
             tmem_ld_32x32b_x32(taddr, v);
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) part[(c + j) * BW + r] = static_cast<int32_t>(v[j]);
+            for (int j = 0; j < 32; ++j) part[(c + j) * BW + r] = static_cast<int32_t>(v[j]) >> kShift;
           }
         }
       }

@@ -339,10 +339,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int c = 4 * half + cc;
         const uint4 p = *reinterpret_cast<const uint4*>(row + (((c ^ r) & 7) << 4));
         uint32_t o[16];
-        ts::signed_of(p.x, o + 0);
-        ts::signed_of(p.y, o + 4);
-        ts::signed_of(p.z, o + 8);
-        ts::signed_of(p.w, o + 12);
+        ts::scaled_of(p.x, o + 0);
+        ts::scaled_of(p.y, o + 4);
+        ts::scaled_of(p.z, o + 8);
+        ts::scaled_of(p.w, o + 12);
         tmem_st_32x32b_x16(col0 + static_cast<uint32_t>(16 * c), o);
       }
       tmem_st_wait();
@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld_wait();
         int32_t* part = sm.part();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) part[j * BW + r] = static_cast<int32_t>(v[j]);
+        for (int j = 0; j < 16; ++j) part[j * BW + r] = static_cast<int32_t>(v[j]) >> ts::kScaledShift;
       }
     }
   }

@@ -223,12 +223,14 @@ def test_gemm_extreme_accumulators():
     assert np.array_equal(acc, oracle.acc(q, p))
 
 
+@pytest.mark.parametrize("M", [2, 130])
 @pytest.mark.parametrize("K", [131008, 131072])
-def test_gemm_scaled_weight_limit(K):
-    # The natural-order few-row kernel sums 64 * w in int32. At its largest K,
-    # x = -128 against code 0 (w = -2) gives 64 * 256 * K just below 2^31; one
-    # step beyond, the call takes the 256-row split-K kernel. Both are exact.
-    M, N = 2, 128
+def test_gemm_scaled_weight_limit(M, K):
+    # The natural-order few-row and split-K kernels sum 64 * w in int32. At
+    # their largest K, x = -128 against code 0 (w = -2) gives 64 * 256 * K just
+    # below 2^31; one step beyond, the call takes the persistent kernel. Both
+    # are exact.
+    N = 128 if M <= 2 else 64
     q = np.full((M, K), -128, np.int8)
     q[1] = 127
     p = np.random.default_rng(K).integers(0, 256, (N, K // 4), dtype=np.uint8)
