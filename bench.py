@@ -484,9 +484,16 @@ def lm_head_alone(bn, d, dev, reps=20):
                                             out=d["outs"][i]))
     ms_single = timed(lambda: bn.bitnet_linear(d["xs"][i], d["packed"][i], d["scales"][i],
                                                out=d["outs"][i], bias=zero_bias))
+    # the pages' comparison: the same layer as a dense bf16 cuBLAS GEMV (the
+    # time does not depend on the weight values)
+    wb = torch.full((N, K), 0.5, dtype=torch.bfloat16, device=dev)
+    ob = torch.empty((1, N), dtype=torch.bfloat16, device=dev)
+    c_ms = timed(lambda: torch.mm(d["xs"][i], wb.t(), out=ob))
+    del wb
     return {"K": K, "N": N, "ms": ms, "gbs": call_bytes(1, K, N) / ms / 1e6,
             "single_kernel_ms": ms_single,
-            "single_kernel_gbs": call_bytes(1, K, N) / ms_single / 1e6}
+            "single_kernel_gbs": call_bytes(1, K, N) / ms_single / 1e6,
+            "cublas_bf16": {"ms": c_ms, "speedup": c_ms / ms}}
 
 
 # ---------------------------------------------------------------- prefill
@@ -537,7 +544,10 @@ def prefill(bn, dev, pk, reps=5):
         sw = synth.scale_wt(synth.key(W.W_PREFILL, Mmax, synth.T_SCALE_WT, K))
         xd_all = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
         del x
-        wp = bn.bitnet_pack_weights(torch.from_numpy(w).to(dev))
+        wd = torch.from_numpy(w).to(dev)
+        wp = bn.bitnet_pack_weights(wd)
+        wb = wd.to(torch.bfloat16)
+        del wd
         swd = torch.from_numpy(sw).to(dev)
         for M in W.PREFILL_M:
             xd = xd_all[:M]
@@ -550,8 +560,11 @@ def prefill(bn, dev, pk, reps=5):
             xq, sa = bn.bitnet_quantize_act(xd)
             g_ms = timed(lambda: bn.bitnet_gemm(xq, wp, sa, swd, out=out))
             del xq, sa
+            # the pages' comparison: the same layer as a dense bf16 cuBLAS GEMM
+            c_ms = timed(lambda: torch.mm(xd, wb.t(), out=out))
             cases.append({"M": M, "K": K, "N": N, "ms": ms, "tops": ops / ms / 1e9,
-                          "gemm_ms": g_ms, "gemm_tops": ops / g_ms / 1e9})
+                          "gemm_ms": g_ms, "gemm_tops": ops / g_ms / 1e9,
+                          "cublas_bf16": {"ms": c_ms, "speedup": c_ms / ms}})
             tot_ops += ops
             tot_ms += ms
             tot_gemm_ms += g_ms
@@ -559,7 +572,7 @@ def prefill(bn, dev, pk, reps=5):
                 gemm_pub = {"M": M, "K": K, "N": N, "ms": g_ms, "tops": ops / g_ms / 1e9,
                             "frac": ops / g_ms / 1e9 / peak}
             del out, ws
-        del xd_all, wp
+        del xd_all, wp, wb
     bn.bitnet_device_status()
     tops = tot_ops / tot_ms / 1e9
     gemm_tops = tot_ops / tot_gemm_ms / 1e9
@@ -613,6 +626,24 @@ def time_rotation(fns, reps=20, warmup=3):
     return statistics.median(per) / len(fns)
 
 
+def bf16_rotation(w_int8):
+    """Independent bf16 copies of a weight matrix (the dense layer cuBLAS
+    would run), together more than twice the L2 size."""
+    wb = w_int8.to(torch.bfloat16)
+    n = max(2, -(-2 * L2_BYTES // (wb.numel() * 2)) + 1)
+    return [wb.clone() for _ in range(n)]
+
+
+def cublas_bf16(ms_ours, x_bf16, wb_copies, N):
+    """The pages' kernel-level comparison: the same layer as a dense bf16
+    GEMM through cuBLAS (torch.mm, y = x W^T), weights rotated like ours.
+    A library reference point beside our kernel, not part of the path."""
+    M = x_bf16.shape[0]
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=x_bf16.device)
+    ms = time_rotation([lambda c=c: torch.mm(x_bf16, c.t(), out=out) for c in wb_copies])
+    return {"ms": ms, "speedup": ms / ms_ours}
+
+
 def llama_gemv(bn, dev, pk):
     """LLaMA-7B projections at M in {1, 4, 8, 15} through bitnet_gemv_fused
     (quantisation fused), weights rotated over copies larger than 2x L2."""
@@ -620,8 +651,10 @@ def llama_gemv(bn, dev, pk):
     cases = []
     for v, (name, K, N) in enumerate(W.LLAMA_GEMV_SHAPES):
         w = synth.ternary(synth.key(W.W_LLAMA_GEMV, 1, synth.T_WEIGHT, v), N, K)
-        copies = weight_rotation(bn.bitnet_pack_weights(torch.from_numpy(w).to(dev)))
-        del w
+        wd = torch.from_numpy(w).to(dev)
+        copies = weight_rotation(bn.bitnet_pack_weights(wd))
+        wb_copies = bf16_rotation(wd)
+        del w, wd
         swd = torch.from_numpy(synth.scale_wt(synth.key(W.W_LLAMA_GEMV, 1, synth.T_SCALE_WT, v))).to(dev)
         for M in W.LLAMA_GEMV_M:
             x = synth.act_bf16(synth.key(W.W_LLAMA_GEMV, M, synth.T_ACT, v), M, K)
@@ -647,12 +680,14 @@ def llama_gemv(bn, dev, pk):
                     [xd], [c], [swd], [out]) for c in copies])
                 s_gbs = call_bytes(M, K, N) / s_ms / 1e6
                 case["grouped_single"] = {"ms": s_ms, "gbs": s_gbs, "frac_hbm": s_gbs / hbm}
+            case["cublas_bf16"] = cublas_bf16(ms, xd, wb_copies, N)
             cases.append(case)
-        del copies
+        del copies, wb_copies
     bn.bitnet_device_status()
     return {"workload": "LLaMA-7B projections 4096->4096, 4096->11008, 11008->4096 at "
                         "M in {1, 4, 8, 15} through bitnet_gemv_fused, one call at a time, "
-                        "and the same problems as one bitnet_gemv_fused_grouped call",
+                        "and the same problems as one bitnet_gemv_fused_grouped call; cublas_bf16 is "
+                        "the same layer as a dense bf16 torch.mm (speedup = its time / ours)",
             "l2": "weights rotated over copies totalling more than 2x L2",
             "peak_hbm_gbs": hbm, "cases": cases}
 
@@ -716,8 +751,10 @@ def midbatch(bn, dev, pk):
     cases = []
     for K, N in W.MIDBATCH_SHAPES:
         w = synth.ternary(synth.key(W.W_MIDBATCH, 0, synth.T_WEIGHT, N), N, K)
-        copies = weight_rotation(bn.bitnet_pack_weights(torch.from_numpy(w).to(dev)))
-        del w
+        wd = torch.from_numpy(w).to(dev)
+        copies = weight_rotation(bn.bitnet_pack_weights(wd))
+        wb_copies = bf16_rotation(wd)
+        del w, wd
         swd = torch.from_numpy(synth.scale_wt(synth.key(W.W_MIDBATCH, 0, synth.T_SCALE_WT, N))).to(dev)
         for M in W.MIDBATCH_M:
             x = synth.act_bf16(synth.key(W.W_MIDBATCH, M, synth.T_ACT, N), M, K, outliers=False)
@@ -732,11 +769,13 @@ def midbatch(bn, dev, pk):
             cases.append({"M": M, "K": K, "N": N, "ms": ms, "tops": ops / ms / 1e9,
                           "gbs": byts / ms / 1e6,
                           "bound": "hbm" if t_hbm >= t_tc else "tensor",
-                          "frac": max(t_hbm, t_tc) / ms})
-        del copies
+                          "frac": max(t_hbm, t_tc) / ms,
+                          "cublas_bf16": cublas_bf16(ms, xd, wb_copies, N)})
+        del copies, wb_copies
     bn.bitnet_device_status()
     return {"workload": "M in {32, 64, 128, 256} x K=4096 x N in {4096, 11008} through "
-                        "bitnet_gemm (pre-quantised int8 + bf16 scales)",
+                        "bitnet_gemm (pre-quantised int8 + bf16 scales); cublas_bf16 is the "
+                        "same layer as a dense bf16 torch.mm (speedup = its time / ours)",
             "l2": "weights rotated over copies totalling more than 2x L2",
             "peak_hbm_gbs": hbm, "peak_tops": tops_peak, "cases": cases}
 
