@@ -804,11 +804,15 @@ bitnet_status run_gemm(void* out, bool acc_out, const int8_t* xq, const uint8_t*
     p.bias = bias;
     return run_gemv(p, true, st);
   }
-  if (M <= kSkMaxRows && (perm || K <= kScaledMaxK))
-    return run_gemm_sk(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
   DeviceInfo* dev = nullptr;
   bitnet_status s = device_info(&dev);
   if (s != BITNET_OK) return s;
+  // 129..192 rows are one tile of the persistent kernel; where the weight
+  // tiles fill at least half the SMs, that beats the split-K kernel's
+  // 256-row tile (measured: 21 against 25 us at M = 160..192, N = 11008)
+  const bool ts_one_wave = M > 128 && M <= ts::BX && (N + ts::BW - 1) / ts::BW >= dev->sms / 2;
+  if (M <= kSkMaxRows && (perm || K <= kScaledMaxK) && !ts_one_wave)
+    return run_gemm_sk(out, acc_out, xq, wp, sa, sw, sw_len, M, N, K, st, perm, rowsum, bias);
   CUtensorMap mx, mw;
   if (!make_map_u8(&mx, xq, M, K, K, ts::BX, ts::BK, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_u8(&mw, wp, N, K / 4, K / 4, ts::BW, ts::BK / 4, CU_TENSOR_MAP_SWIZZLE_NONE))

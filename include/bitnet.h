@@ -113,9 +113,10 @@ bitnet_status bitnet_quantize_act(int8_t* x_q, uint16_t* scale_act,
  * Any M >= 0. Kernels: with K % 64 == 0 and 16-byte aligned x_q and
  * w_packed, M <= 256 runs a tensor-core kernel whose K loop is split over a
  * thread-block cluster, and larger M a persistent tensor-core kernel;
- * otherwise a SIMT kernel. (With K > 131008, M <= 256 takes the persistent
- * kernel too: the others' int32 sums of 64 * w could overflow.) All give the
- * same result. */
+ * otherwise a SIMT kernel. The persistent kernel also takes 129..192 rows
+ * when the N / 128 weight tiles fill at least half the SMs (one wave of
+ * 192-row tiles), and M <= 256 with K > 131008 (the others' int32 sums of
+ * 64 * w could overflow). All give the same result. */
 bitnet_status bitnet_gemm(uint16_t* out, const int8_t* x_q,
                           const uint8_t* w_packed, const uint16_t* scale_act,
                           const float* scale_wt, int64_t scale_wt_len,

@@ -223,6 +223,24 @@ def test_gemm_extreme_accumulators():
     assert np.array_equal(acc, oracle.acc(q, p))
 
 
+@pytest.mark.parametrize("M,N", [(150, 9600), (192, 11008)])
+def test_gemm_one_wave_rows_bitexact(M, N):
+    # 129..192 rows with at least 74 weight tiles take the persistent kernel
+    # (one 192-row tile per weight tile); its int32 sums and bf16 outputs,
+    # natural order (bitnet_gemm) and permuted (bitnet_linear), match the
+    # oracle exactly
+    K = 1024
+    x = acts(131, M, M, K)
+    w = weights(131, M, N, K)
+    p = oracle.pack(w)
+    q, sa = oracle.quantize(x)
+    acc = bn.bitnet_gemm_acc_i32(to_dev(q), to_dev(p)).cpu().numpy()
+    assert np.array_equal(acc, oracle.acc(q, p))
+    sw = sw_of(131, M)
+    got = bn.bitnet_linear(to_dev(x, torch.bfloat16), to_dev(p), to_dev(sw))
+    assert_bf16_close(bf16_bits(got), oracle.linear(x, p, sw))
+
+
 @pytest.mark.parametrize("M", [2, 130])
 @pytest.mark.parametrize("K", [131008, 131072])
 def test_gemm_scaled_weight_limit(M, K):
