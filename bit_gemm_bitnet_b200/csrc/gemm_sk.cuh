@@ -48,7 +48,7 @@ constexpr int MIN_SMEM = 120 * 1024;
 template <int BX>
 struct Cfg {
   static_assert(BX == 16 || BX == 32 || BX == 64 || BX == 128 || BX == 256, "MMA N");
-  static constexpr int STAGES = BX == 256 ? 4 : 8;
+  static constexpr int STAGES = BX == 256 ? 6 : 8;
   static_assert(STAGES % 2 == 0, "stages a multiple of the two unpack groups");
   static constexpr int X_BYTES = BX * BK;
   static constexpr int STAGE_BYTES = X_BYTES + WP_BYTES;
