@@ -22,6 +22,7 @@
 // Warp roles (512 threads, one CTA per SM):
 //   warp 0      TMA producer
 //   warp 1      tensor-memory owner, MMA issuer (one thread)
+//   warps 2-3   stage the epilogue's per-row and per-column scalars
 //   warps 4-11  unpack: every stage, each warp half the columns of its
 //               tensor-memory lanes 32 * (warp % 4) ..; then each moves half
 //               the accumulator columns of those lanes out
@@ -259,6 +260,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mma_commit(sm.drain());
       mbar_wait_drain(sm.drain(), 0u);
     }
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------- epilogue scalars
+    // staged while the K loop runs: per activation row the fp32 scale and
+    // 2 * code sum, per weight row of the tile the fp32 scale and bf16 bias
+    pdl_wait();  // scales and row sums may come from the previous kernel
+    for (int m = threadIdx.x - 64; m < BX; m += 64) {
+      sm.row_sa()[m] = (!kAccOut && m < M) ? bf16_bits_to_f32(scale_act[m]) : 0.0f;
+      sm.row_corr()[m] = (kPerm && m < M) ? 2 * rowsum[m] : 0;
+    }
+    for (int i = threadIdx.x - 64; i < BW; i += 64) {
+      const int n = n0 + i;
+      sm.col_sw()[i] = (!kAccOut && n < N) ? scale_wt[sw_len == 1 ? 0 : n] : 0.0f;
+      sm.col_bias()[i] = (bias != nullptr && n < N) ? bias[n] : static_cast<uint16_t>(0);
+    }
+    if (S == 1) named_barrier_sync(2, 320);  // warps 2-11
   } else if (warp >= 4 && warp < 4 + UNPACK_WARPS) {
     // -------------------------------------------------------------- unpack
     // Lane r of warp w owns weight row 32 * (w % 4) + r and the half
@@ -311,23 +327,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int quarter = warp & 3;
       const int ehalf = (warp - 4) >> 2;
       if (S == 1) {
-        // the epilogue's per-row scalars, staged while the last MMAs run
-        pdl_wait();  // scales and row sums may come from the previous kernel
-        for (int m = threadIdx.x - 128; m < BX; m += 256) {
-          sm.row_sa()[m] = (!kAccOut && m < M) ? bf16_bits_to_f32(scale_act[m]) : 0.0f;
-          sm.row_corr()[m] = (kPerm && m < M) ? 2 * rowsum[m] : 0;
-        }
-        named_barrier_sync(2, 256);  // warps 4-11
+        pdl_wait();  // the output may still be read by the previous kernel
+        named_barrier_sync(2, 320);  // warps 2-11: the scalars are staged
       }
       // lane = weight row n of this warp's quarter of the tile
       const int nq = n0 + quarter * 32;
-      const int n = nq + lane;
-      float swn = 0.0f;
-      uint16_t bn = 0;
-      if (S == 1 && !kAccOut && n < N) {
-        swn = scale_wt[sw_len == 1 ? 0 : n];
-        if (bias != nullptr) bn = bias[n];
-      }
+      const float swn = sm.col_sw()[quarter * 32 + lane];
+      const uint16_t bn = sm.col_bias()[quarter * 32 + lane];
       if (mbar_wait_warp(sm.tfull(), 0u, abort)) {
         tc_fence_after();
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -403,19 +409,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (S > 1) {
     // ------------------------------------- cluster reduction and epilogue
-    pdl_wait();  // scales and row sums may come from the previous kernel
-    for (int m = threadIdx.x; m < BX; m += NUM_THREADS) {
-      sm.row_sa()[m] = (!kAccOut && m < M) ? bf16_bits_to_f32(scale_act[m]) : 0.0f;
-      sm.row_corr()[m] = (kPerm && m < M) ? 2 * rowsum[m] : 0;
-    }
-    for (int i = threadIdx.x; i < BW; i += NUM_THREADS) {
-      const int n = n0 + i;
-      sm.col_sw()[i] = (!kAccOut && n < N) ? scale_wt[sw_len == 1 ? 0 : n] : 0.0f;
-      sm.col_bias()[i] = (bias != nullptr && n < N) ? bias[n] : static_cast<uint16_t>(0);
-    }
+    pdl_wait();  // the output may still be read by the previous kernel
     tc_fence_before();
     __syncwarp();
-    cluster_sync();  // every CTA's partial tile is in its shared memory
+    cluster_sync();  // every CTA's partial tile (and its staged scalars) is in shared memory
     const int r_lo = share_row(rank, S), r_hi = share_row(rank + 1, S);
     const int G = (r_hi - r_lo) / 4;  // 16-byte groups per activation row
     const int total = M * G;

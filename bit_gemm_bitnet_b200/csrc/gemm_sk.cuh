@@ -19,6 +19,7 @@
 // Warp roles (512 threads, one CTA per SM):
 //   warp 0      TMA producer
 //   warp 1      tensor-memory owner, MMA issuer (one thread)
+//   warps 2-3   stage the epilogue's per-row and per-column scalars
 //   warps 4-11  unpack: packed codes -> int8 -> tcgen05.st into an A stage
 //               (two groups of four warps, stages in turn); then warps 4-7
 //               move the accumulator to the shared-memory partial tile
@@ -211,6 +212,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mma_commit(sm.drain());
       mbar_wait_drain(sm.drain(), 0u);
     }
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------- epilogue scalars
+    // staged while the K loop runs: per activation row the fp32 scale and
+    // 2 * code sum, per weight row of the tile the fp32 scale and bf16 bias
+    pdl_wait();  // scales and row sums may come from the previous kernel
+    for (int m = threadIdx.x - 64; m < BX; m += 64) {
+      sm.row_sa()[m] = (!kAccOut && m < M) ? bf16_bits_to_f32(scale_act[m]) : 0.0f;
+      sm.row_corr()[m] = (kPerm && m < M) ? 2 * rowsum[m] : 0;
+    }
+    for (int i = threadIdx.x - 64; i < BW; i += 64) {
+      const int n = n0 + i;
+      sm.col_sw()[i] = (!kAccOut && n < N) ? scale_wt[sw_len == 1 ? 0 : n] : 0.0f;
+      sm.col_bias()[i] = (bias != nullptr && n < N) ? bias[n] : static_cast<uint16_t>(0);
+    }
   } else if (warp >= 4 && warp < 12) {
     // -------------------------------------------------------------- unpack
     // Two groups of four warps take the stages in turn, so two stages are
@@ -290,19 +305,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 
   // --------------------------------------- cluster reduction and epilogue
-  pdl_wait();  // scales and row sums may come from the previous kernel
-  for (int m = threadIdx.x; m < BX; m += NUM_THREADS) {
-    sm.row_sa()[m] = (!kAccOut && m < M) ? bf16_bits_to_f32(scale_act[m]) : 0.0f;
-    sm.row_corr()[m] = (kPerm && m < M) ? 2 * rowsum[m] : 0;
-  }
-  for (int i = threadIdx.x; i < BW; i += NUM_THREADS) {
-    const int n = n0 + i;
-    sm.col_sw()[i] = (!kAccOut && n < N) ? scale_wt[sw_len == 1 ? 0 : n] : 0.0f;
-    sm.col_bias()[i] = (bias != nullptr && n < N) ? bias[n] : static_cast<uint16_t>(0);
-  }
+  pdl_wait();  // the output may still be read by the previous kernel
   tc_fence_before();
   __syncwarp();
-  cluster_sync();  // every CTA's partial tile (and the scalars) are in shared memory
+  cluster_sync();  // every CTA's partial tile (and the staged scalars) are in shared memory
   {
     const int r_lo = share_row(rank, S), r_hi = share_row(rank + 1, S);
     const int G = (r_hi - r_lo) / 4;  // 16-byte groups per activation row

@@ -316,6 +316,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mma_commit(sm.drain());
       mbar_wait_drain(sm.drain(), 0u);
     }
+  } else if (warp == 2 || warp == 3) {
+    // the reduction's per-weight-row scalars, staged while the K loop runs
+    for (int i = tid - 64; i < BW; i += 64) {
+      const int n = n0 + i;
+      sm.col_sw()[i] = (!kAccOut && n < N) ? scale_wt[sw_len == 1 ? 0 : n] : 0.0f;
+      sm.col_bias()[i] = (bias != nullptr && n < N) ? bias[n] : static_cast<uint16_t>(0);
+    }
   } else if (warp >= 4 && warp < 4 + UNPACK_WARPS) {
     // unpack: every stage, lane r of warp w -> weight row 32 (w % 4) + r and
     // the half h = (w - 4) / 4 of its 128 packed bytes: four 16-byte pieces
@@ -366,11 +373,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 
   // ---- 4. cluster reduction and epilogue
-  for (int i = tid; i < BW; i += NUM_THREADS) {
-    const int n = n0 + i;
-    sm.col_sw()[i] = (!kAccOut && n < N) ? scale_wt[sw_len == 1 ? 0 : n] : 0.0f;
-    sm.col_bias()[i] = (bias != nullptr && n < N) ? bias[n] : static_cast<uint16_t>(0);
-  }
   tc_fence_before();
   __syncwarp();
   cluster_sync();  // every CTA's partial tile (and the scalars) are in shared memory
