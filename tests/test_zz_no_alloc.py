@@ -16,6 +16,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 import bit_gemm_bitnet_b200 as bn
 from helpers import bf16_bits, to_dev
@@ -35,10 +36,15 @@ def call_noalloc(x, wp, sw, out, M, N, K):
                                           M, N, K, st)
 
 
-def inputs(seed, M, K, N):
+def host_inputs(seed, M, K, N):
     x = synth.act_bf16(synth.key(77, seed, synth.T_ACT), M, K)
     w = synth.ternary(synth.key(77, seed, synth.T_WEIGHT), N, K)
     sw = synth.uniform_f32(synth.key(77, seed, synth.T_SCALE_WT), N, 0.01, 0.1)
+    return x, w, sw
+
+
+def inputs(seed, M, K, N):
+    x, w, sw = host_inputs(seed, M, K, N)
     xd = to_dev(x, torch.bfloat16)
     wp = bn.bitnet_pack_weights(to_dev(w))
     return xd, wp, to_dev(sw)
@@ -55,6 +61,18 @@ def test_noalloc_matches_linear_with_workspace_on_two_calls(cuda_ok):
         assert call_noalloc(xd, wp, sw, out, M, N, K) == bn.OK
         torch.cuda.synchronize()
         assert np.array_equal(bf16_bits(out), bf16_bits(ref)), f"call {seed}"
+    bn.bitnet_device_status()
+
+
+def test_noalloc_matches_oracle(cuda_ok):
+    # the allocation-free call against the scalar CPU oracle directly
+    M, K, N = 40, 1024, 384
+    x, w, sw = host_inputs(20, M, K, N)
+    xd, wp, swd = inputs(20, M, K, N)
+    out = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    assert call_noalloc(xd, wp, swd, out, M, N, K) == bn.OK
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_bits(out), oracle.linear(x, oracle.pack(w), sw))
     bn.bitnet_device_status()
 
 
